@@ -1,0 +1,340 @@
+"""Plain CPU oracle for the quantized gated Delta-rule decode step (test infrastructure).
+
+This package is TEST INFRASTRUCTURE. Only the test suite, the package's ``smoke()`` check and
+the benchmark's CPU-baseline leg may import it. It wraps ``stepq_oracle.c`` (plain C, compiled
+here with gcc at -O2 -ffp-contract=off) through ctypes and shares no code with the CUDA
+library. See the header of ``stepq_oracle.c`` for what each function follows in
+"STEPQuant: When and Where Errors Matter in Delta-Rule Recurrent State Quantization".
+
+Array conventions (NumPy, C-contiguous):
+  state S          float32 [B][H][dk][dv]   (row = key channel i, column = value channel j)
+  q, k             uint16 bf16 bits [B][H][dk];  v: uint16 [B][H][dv]
+  beta             float32 [B][H];  gate: float32 [B][H] or [B][H][dk]
+  bits             uint8 [H][dk];  w: float32 [H][dk]
+  r, c             uint16 binary16 bits [B][H][dk], [B][H][dv]
+  packed           uint8 [B * bytes_per_seq]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+_HERE = Path(__file__).resolve().parent
+_SRC = _HERE / "stepq_oracle.c"
+_BUILD = _HERE / "_build"
+_LIB_PATH = _BUILD / "libstepq_oracle.so"
+_lib = None
+
+ORC_OK, ORC_EINVAL, ORC_EUNSUPPORTED, ORC_EBUDGET = 0, 1, 2, 4
+
+
+def build(force: bool = False) -> Path:
+    """Compile the oracle library with gcc (plain C99, no fused multiply-add)."""
+    _BUILD.mkdir(exist_ok=True)
+    if force or not _LIB_PATH.exists() or _LIB_PATH.stat().st_mtime < _SRC.stat().st_mtime:
+        tmp = _LIB_PATH.with_suffix(f".{os.getpid()}.tmp")
+        cmd = ["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+               "-fPIC", "-shared", "-o", str(tmp), str(_SRC), "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(str(build()))
+        _lib.orc_scale_to_half.restype = ctypes.c_uint16
+        _lib.orc_scale_to_half.argtypes = [ctypes.c_double]
+        _lib.orc_half_to_float.restype = ctypes.c_float
+        _lib.orc_half_to_float.argtypes = [ctypes.c_uint16]
+        _lib.orc_layout.restype = ctypes.c_int64
+        _lib.orc_tile_bytes.restype = ctypes.c_int64
+    return _lib
+
+
+def _p(a):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else ctypes.c_void_p(0)
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a
+
+
+def _check(rc, what):
+    if rc != ORC_OK:
+        raise RuntimeError(f"oracle {what} failed with status {rc}")
+
+
+# ---------------------------------------------------------------------------------------------
+# scalars and layout
+# ---------------------------------------------------------------------------------------------
+
+def scale_to_half(x: float) -> int:
+    return int(lib().orc_scale_to_half(float(x)))
+
+
+def half_to_float(h) -> np.ndarray:
+    return np.asarray(h, dtype=np.uint16).view(np.float16).astype(np.float32)
+
+
+def layout(bits: np.ndarray, dv: int):
+    """(head_off int64 [H], bytes_per_seq) for a bit map [H][dk]."""
+    bits = _c(bits, np.uint8)
+    H, dk = bits.shape
+    head_off = np.zeros(H, dtype=np.int64)
+    n = lib().orc_layout(H, dk, dv, _p(bits), _p(head_off))
+    return head_off, int(n)
+
+
+def tile_bytes(bits_row: np.ndarray, dv: int) -> int:
+    bits_row = _c(bits_row, np.uint8)
+    return int(lib().orc_tile_bytes(len(bits_row), dv, _p(bits_row)))
+
+
+# ---------------------------------------------------------------------------------------------
+# tile-level
+# ---------------------------------------------------------------------------------------------
+
+def quantise_tile(X, bits, r, c):
+    X = _c(X, np.float32); bits = _c(bits, np.uint8); r = _c(r, np.uint16); c = _c(c, np.uint16)
+    dk, dv = X.shape
+    codes = np.zeros((dk, dv), dtype=np.int32)
+    lib().orc_quantise_tile(dk, dv, _p(X), _p(bits), _p(r), _p(c), _p(codes))
+    return codes
+
+
+def pack_codes(codes, bits):
+    codes = _c(codes, np.int32); bits = _c(bits, np.uint8)
+    dk, dv = codes.shape
+    out = np.zeros(tile_bytes(bits, dv), dtype=np.uint8)
+    lib().orc_pack_codes(dk, dv, _p(bits), _p(codes), _p(out))
+    return out
+
+
+def unpack_codes(packed, bits, dv):
+    packed = _c(packed, np.uint8); bits = _c(bits, np.uint8)
+    dk = len(bits)
+    codes = np.zeros((dk, dv), dtype=np.int32)
+    lib().orc_unpack_codes(dk, dv, _p(bits), _p(packed), _p(codes))
+    return codes
+
+
+def fit_tile(X, w, bits, detail=False):
+    X = _c(X, np.float32); w = _c(w, np.float32); bits = _c(bits, np.uint8)
+    dk, dv = X.shape
+    r = np.zeros(dk, dtype=np.uint16); c = np.zeros(dv, dtype=np.uint16)
+    if not detail:
+        lib().orc_fit_tile(dk, dv, _p(X), _p(w), _p(bits), _p(r), _p(c))
+        return r, c
+    c0 = np.zeros(dv, dtype=np.float32); z0 = np.zeros((dk, dv), dtype=np.int32)
+    c1 = np.zeros(dv, dtype=np.float64)
+    lib().orc_fit_tile_detail(dk, dv, _p(X), _p(w), _p(bits), _p(r), _p(c), _p(c0), _p(z0), _p(c1))
+    return r, c, dict(c0=c0, z0=z0, c1=c1)
+
+
+def pack_tile(X, bits, r, c):
+    X = _c(X, np.float32); bits = _c(bits, np.uint8); r = _c(r, np.uint16); c = _c(c, np.uint16)
+    dk, dv = X.shape
+    out = np.zeros(tile_bytes(bits, dv), dtype=np.uint8)
+    lib().orc_pack_tile(dk, dv, _p(X), _p(bits), _p(r), _p(c), _p(out))
+    return out
+
+
+def unpack_tile(packed, bits, r, c, dv):
+    packed = _c(packed, np.uint8); bits = _c(bits, np.uint8); r = _c(r, np.uint16); c = _c(c, np.uint16)
+    dk = len(bits)
+    X = np.zeros((dk, dv), dtype=np.float32)
+    lib().orc_unpack_tile(dk, dv, _p(packed), _p(bits), _p(r), _p(c), _p(X))
+    return X
+
+
+def delta_update(S, q, k, v, beta, gate):
+    """One gated Delta-rule update in float64. gate: scalar or [dk]. Returns (X, o)."""
+    S = _c(S, np.float64)
+    dk, dv = S.shape
+    g = np.broadcast_to(np.asarray(gate, dtype=np.float64), (dk,)).copy()
+    q = _c(q, np.float64); k = _c(k, np.float64); v = _c(v, np.float64)
+    X = np.zeros((dk, dv)); o = np.zeros(dv)
+    lib().orc_delta_update(dk, dv, _p(S), _p(q), _p(k), _p(v), ctypes.c_double(float(beta)), _p(g),
+                           _p(X), _p(o))
+    return X, o
+
+
+def int8_quantise_tile(X):
+    X = _c(X, np.float32)
+    dk, dv = X.shape
+    codes = np.zeros((dk, dv), dtype=np.int8); s = np.zeros(dk, dtype=np.uint16)
+    lib().orc_int8_quantise_tile(dk, dv, _p(X), _p(codes), _p(s))
+    return codes, s
+
+
+# ---------------------------------------------------------------------------------------------
+# batch-level (the same calls as the CUDA library's C-ABI)
+# ---------------------------------------------------------------------------------------------
+
+def _dims(S_or_shape):
+    return S_or_shape.shape if hasattr(S_or_shape, "shape") else S_or_shape
+
+
+def fit_scales(S, w, bits, nthreads=0):
+    S = _c(S, np.float32); w = _c(w, np.float32); bits = _c(bits, np.uint8)
+    B, H, dk, dv = S.shape
+    r = np.zeros((B, H, dk), dtype=np.uint16); c = np.zeros((B, H, dv), dtype=np.uint16)
+    _check(lib().orc_fit_scales(B, H, dk, dv, _p(S), _p(w), _p(bits), _p(r), _p(c), nthreads), "fit_scales")
+    return r, c
+
+
+def pack_state(S, bits, r, c, nthreads=0):
+    S = _c(S, np.float32); bits = _c(bits, np.uint8); r = _c(r, np.uint16); c = _c(c, np.uint16)
+    B, H, dk, dv = S.shape
+    head_off, bps = layout(bits, dv)
+    packed = np.zeros(B * bps, dtype=np.uint8)
+    _check(lib().orc_pack_state(B, H, dk, dv, _p(S), _p(bits), _p(head_off), ctypes.c_int64(bps),
+                                _p(r), _p(c), _p(packed), nthreads), "pack_state")
+    return packed
+
+
+def unpack_state(packed, bits, r, c, nthreads=0):
+    packed = _c(packed, np.uint8); bits = _c(bits, np.uint8); r = _c(r, np.uint16); c = _c(c, np.uint16)
+    B, H, dk = r.shape
+    dv = c.shape[2]
+    head_off, bps = layout(bits, dv)
+    S = np.zeros((B, H, dk, dv), dtype=np.float32)
+    _check(lib().orc_unpack_state(B, H, dk, dv, _p(packed), _p(bits), _p(head_off), ctypes.c_int64(bps),
+                                  _p(r), _p(c), _p(S), nthreads), "unpack_state")
+    return S
+
+
+def decode_step(tok, bits, w, packed, r, c, nthreads=0):
+    """One quantized decode step over all tiles. tok: dict(q, k, v, beta, gate).
+    Returns (packed_out, r_out, c_out, o)."""
+    q = _c(tok["q"], np.uint16); k = _c(tok["k"], np.uint16); v = _c(tok["v"], np.uint16)
+    beta = _c(tok["beta"], np.float32); gate = _c(tok["gate"], np.float32)
+    bits = _c(bits, np.uint8); w = _c(w, np.float32)
+    packed = _c(packed, np.uint8); r = _c(r, np.uint16); c = _c(c, np.uint16)
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    gpc = int(gate.ndim == 3)
+    head_off, bps = layout(bits, dv)
+    p_out = np.zeros_like(packed); r_out = np.zeros_like(r); c_out = np.zeros_like(c)
+    o = np.zeros((B, H, dv), dtype=np.float32)
+    _check(lib().orc_decode_step(B, H, dk, dv, gpc, _p(q), _p(k), _p(v), _p(beta), _p(gate), _p(bits),
+                                 _p(w), _p(head_off), ctypes.c_int64(bps), _p(packed), _p(r), _p(c),
+                                 _p(p_out), _p(r_out), _p(c_out), _p(o), nthreads), "decode_step")
+    return p_out, r_out, c_out, o
+
+
+def decode_step_fp32(tok, S, nthreads=0):
+    q = _c(tok["q"], np.uint16); k = _c(tok["k"], np.uint16); v = _c(tok["v"], np.uint16)
+    beta = _c(tok["beta"], np.float32); gate = _c(tok["gate"], np.float32)
+    S = _c(S, np.float32)
+    B, H, dk, dv = S.shape
+    S_out = np.zeros_like(S); o = np.zeros((B, H, dv), dtype=np.float32)
+    _check(lib().orc_decode_step_fp32(B, H, dk, dv, int(gate.ndim == 3), _p(q), _p(k), _p(v), _p(beta),
+                                      _p(gate), _p(S), _p(S_out), _p(o), nthreads), "decode_step_fp32")
+    return S_out, o
+
+
+def int8_quantise_state(S):
+    S = _c(S, np.float32)
+    B, H, dk, dv = S.shape
+    codes = np.zeros((B, H, dk, dv), dtype=np.int8); s = np.zeros((B, H, dk), dtype=np.uint16)
+    lib().orc_int8_quantise_state(B, H, dk, dv, _p(S), _p(codes), _p(s))
+    return codes, s
+
+
+def decode_step_int8(tok, codes, s, nthreads=0):
+    q = _c(tok["q"], np.uint16); k = _c(tok["k"], np.uint16); v = _c(tok["v"], np.uint16)
+    beta = _c(tok["beta"], np.float32); gate = _c(tok["gate"], np.float32)
+    codes = _c(codes, np.int8); s = _c(s, np.uint16)
+    B, H, dk, dv = codes.shape
+    c_out = np.zeros_like(codes); s_out = np.zeros_like(s); o = np.zeros((B, H, dv), dtype=np.float32)
+    _check(lib().orc_decode_step_int8(B, H, dk, dv, int(gate.ndim == 3), _p(q), _p(k), _p(v), _p(beta),
+                                      _p(gate), _p(codes), _p(s), _p(c_out), _p(s_out), _p(o), nthreads),
+           "decode_step_int8")
+    return c_out, s_out, o
+
+
+# ---------------------------------------------------------------------------------------------
+# offline calibration
+# ---------------------------------------------------------------------------------------------
+
+def row_impact(calib):
+    """w [H][dk] from a calibration stream dict(q, k, beta, gate) with a leading step axis."""
+    q = _c(calib["q"], np.uint16); k = _c(calib["k"], np.uint16)
+    beta = _c(calib["beta"], np.float32); gate = _c(calib["gate"], np.float32)
+    T, B, H, dk = q.shape
+    w = np.zeros((H, dk), dtype=np.float32)
+    _check(lib().orc_row_impact(T, B, H, dk, int(gate.ndim == 4), _p(q), _p(k), _p(beta), _p(gate), _p(w)),
+           "row_impact")
+    return w
+
+
+def calib_distortion(S, w, b, nthreads=0):
+    """(d_row [H][dk], d_head [H]) at uniform width b over the sample states S [B][H][dk][dv]."""
+    S = _c(S, np.float32); w = _c(w, np.float32)
+    B, H, dk, dv = S.shape
+    d_row = np.zeros((H, dk)); d_head = np.zeros(H)
+    _check(lib().orc_calib_distortion(B, H, dk, dv, _p(S), _p(w), int(b), _p(d_row), _p(d_head), nthreads),
+           "calib_distortion")
+    return d_row, d_head
+
+
+def allocate_bits(J, cand, budget, mode):
+    """Bit widths (uint8 [n_units]) minimising sum J[u][k] with exactly ``budget`` bits.
+    mode 1: multiple-choice DP; mode 0: Lagrangian allocation with repair."""
+    J = _c(J, np.float64)
+    cand = _c(cand, np.int32)
+    n, nc = J.shape
+    out = np.zeros(n, dtype=np.uint8)
+    rc = lib().orc_allocate_bits(n, nc, _p(cand), _p(J), ctypes.c_int64(int(budget)), int(mode), _p(out))
+    if rc != ORC_OK:
+        raise ValueError(f"oracle allocate_bits failed with status {rc}")
+    return out
+
+
+def lifetime(gate):
+    """Unit lifetime L_u = 1 / (1 - g_u): the sum over j >= 0 of the retention product g_u^j."""
+    g = np.asarray(gate, dtype=np.float64)
+    return 1.0 / (1.0 - g)
+
+
+def objective(d, gate):
+    """J_u(b) = L_u d_u(b): lifetime-weighted distortion, d [n_units][n_cand]."""
+    return lifetime(gate)[:, None] * np.asarray(d, dtype=np.float64)
+
+
+def calibrate(alloc, candidates, nominal_bits, gates, S0, calib):
+    """The offline calibration done by the oracle (App. A.3, B.3, C.2): returns
+    (bits uint8 [H][dk] or None, w float32 [H][dk]).
+
+    alloc: "dp_head" (head units, multiple-choice DP, Eq. 17 distortion) or "lagrange_row"
+    (key-row units, Lagrangian allocation with repair, Eq. 18 distortion); any other value
+    returns bits=None (the caller supplies a fixed map). gates: unit gates [H] or [H][dk];
+    S0: the sample states [B][H][dk][dv]; calib: the calibration stream."""
+    w = row_impact(calib)
+    H, dk = w.shape
+    if alloc not in ("dp_head", "lagrange_row"):
+        return None, w
+    cand = [int(b) for b in candidates]
+    gates = np.asarray(gates, dtype=np.float32)
+    drows, dheads = [], []
+    for b in cand:
+        dr, dh = calib_distortion(S0, w, b)
+        drows.append(dr)
+        dheads.append(dh)
+    if alloc == "dp_head":
+        dist = np.stack(dheads, axis=1)                          # [H][n_cand]
+        g = gates if gates.ndim == 1 else gates.mean(axis=1)
+        bh = allocate_bits(objective(dist, g), cand, nominal_bits * H, mode=1)
+        return np.repeat(bh[:, None], dk, axis=1).astype(np.uint8), w
+    dist = np.stack([dr.reshape(-1) for dr in drows], axis=1)   # [H*dk][n_cand]
+    g = gates.reshape(-1) if gates.ndim == 2 else np.repeat(gates, dk)
+    br = allocate_bits(objective(dist, g), cand, nominal_bits * H * dk, mode=0)
+    return br.reshape(H, dk).astype(np.uint8), w

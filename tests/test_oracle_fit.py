@@ -1,0 +1,97 @@
+"""Pins of the oracle's key-row-aware dual-axis fit (STEPQuant §4.3, App. C.1): the row
+factor definition, the no-clip column initialisation, the least-squares optimality of the
+fixed-code column update, and the decode step as the composition the workflow table lists."""
+import numpy as np
+import pytest
+
+import oracle
+from recurrent_state_quantization_gated_b200 import synth
+
+
+def _tile(d=128, seed=0):
+    S = synth.random_tile_state(1, 1, d, seed=seed)[0, 0]
+    bits = synth.random_bits(1, d, seed=seed + 1)[0]
+    w = synth.random_weights(1, d, seed=seed + 2)[0]
+    return S, bits, w
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_row_factor_is_mean_abs_over_impact(d):
+    S, bits, w = _tile(d, 3)
+    r, _ = oracle.fit_tile(S, w, bits)
+    m = np.abs(S.astype(np.float64)).mean(axis=1)
+    expect = np.clip(np.maximum(m, 2.0 ** -14) / w.astype(np.float64), 2.0 ** -14, 65504).astype(np.float16)
+    np.testing.assert_array_equal(r, expect.view(np.uint16))
+
+
+def test_column_init_clips_nothing_and_is_tight():
+    S, bits, w = _tile(128, 5)
+    r, c, det = oracle.fit_tile(S, w, bits, detail=True)
+    rf = oracle.half_to_float(r).astype(np.float64)
+    bound = rf * 2.0 ** (8 - bits.astype(np.float64)) * (2.0 ** (bits.astype(np.float64) - 1) - 1)
+    ratio = np.abs(S) / (bound[:, None] * det["c0"][None, :].astype(np.float64))
+    assert ratio.max() <= 1 + 1e-6
+    np.testing.assert_allclose(ratio.max(axis=0), 1.0, rtol=1e-6)   # some entry of each column reaches the edge
+    qb = (2 ** (bits.astype(np.int64) - 1) - 1)
+    assert np.all(np.abs(det["z0"]) <= qb[:, None])
+
+
+@pytest.mark.parametrize("seed", [5, 6, 7])
+def test_column_update_is_the_weighted_least_squares_optimum(seed):
+    """For the fixed codes z0 the weighted objective sum_i w_i^2 (X_ij - r_i c_j z_ij)^2 has zero
+    derivative in c_j at c1, and c1 does no worse than the initial scale c0."""
+    S, bits, w = _tile(128, seed)
+    r, c, det = oracle.fit_tile(S, w, bits, detail=True)
+    rf = oracle.half_to_float(r).astype(np.float64)
+    V = rf[:, None] * (2.0 ** (8 - bits.astype(np.float64)))[:, None] * det["z0"]
+    W2 = (w.astype(np.float64) ** 2)[:, None]
+    X = S.astype(np.float64)
+
+    def objective(cvec):
+        return np.sum(W2 * (X - V * cvec[None, :]) ** 2, axis=0)
+
+    c1 = det["c1"]
+    grad = -2 * np.sum(W2 * V * (X - V * c1[None, :]), axis=0)
+    scale = 2 * np.sum(W2 * np.abs(V * X), axis=0) + 1e-300
+    assert np.max(np.abs(grad) / scale) < 1e-12
+    assert np.all(objective(c1) <= objective(det["c0"].astype(np.float64)) * (1 + 1e-12))
+    for eps in (1e-3, -1e-3):                        # a local minimum along each column
+        assert np.all(objective(c1 * (1 + eps)) >= objective(c1))
+    np.testing.assert_array_equal(c, np.clip(c1, 2.0 ** -14, 65504).astype(np.float16).view(np.uint16))
+
+
+def test_zero_column_keeps_initial_scale():
+    S, bits, w = _tile(64, 9)
+    S[:, 5] = 0.0
+    r, c, det = oracle.fit_tile(S, w, bits, detail=True)
+    assert det["c0"][5] == np.float32(2.0 ** -14)
+    assert det["c1"][5] == det["c0"][5]
+    assert c[5] == np.float16(2.0 ** -14).view(np.uint16)
+
+
+@pytest.mark.parametrize("gpc", [False, True])
+def test_decode_tile_is_unpack_update_fit_pack(gpc):
+    """Table C2: reconstruct, update, emit the readout before requantisation, refit, repack."""
+    d = 64
+    wl = synth.workload(0)
+    S = synth.random_tile_state(1, 1, d, seed=12)
+    bits = synth.half_bits(wl)[:1]
+    w = synth.random_weights(1, d, seed=13)
+    r, c = oracle.fit_scales(S, w, bits)
+    packed = oracle.pack_state(S, bits, r, c)
+    tok = synth.tokens(wl, 0, seqs=[0])
+    tok = {k: v[:, :1] for k, v in tok.items()}
+    if gpc:
+        tok["gate"] = np.ascontiguousarray(np.linspace(0.9, 1.0, d, dtype=np.float32)[None, None, :])
+    p1, r1, c1, o = oracle.decode_step(tok, bits, w, packed, r, c)
+    Shat = oracle.unpack_state(packed, bits, r, c)[0, 0].astype(np.float64)
+    qf = synth.bf16_bits_to_f32(tok["q"][0, 0]); kf = synth.bf16_bits_to_f32(tok["k"][0, 0])
+    vf = synth.bf16_bits_to_f32(tok["v"][0, 0])
+    g = tok["gate"][0, 0]
+    X, o_ref = oracle.delta_update(Shat, qf, kf, vf, float(tok["beta"][0, 0]), g)
+    np.testing.assert_allclose(o[0, 0], o_ref.astype(np.float32), rtol=0, atol=0)
+    X32 = X.astype(np.float32)
+    rr, cc = oracle.fit_tile(X32, w[0], bits[0])
+    np.testing.assert_array_equal(r1[0, 0], rr)
+    np.testing.assert_array_equal(c1[0, 0], cc)
+    np.testing.assert_array_equal(p1, oracle.pack_tile(X32, bits[0], rr, cc))
