@@ -1,0 +1,378 @@
+#!/usr/bin/env python3
+"""Throughput of the fused quantized gated Delta-rule decode step on B200.
+
+One step = one decode token for every (sequence, head) tile of the workload: unpack and
+dequantise the packed recurrent state, gated Delta update, readout, refit of the dual-axis
+scales and repack -- one launch of the fused kernel. The default workload is the Qwen-style
+Gated DeltaNet layer decode (B=64 sequences, H=32 heads, d_k=d_v=128, 6-bit nominal budget,
+head-level bits from the lifetime-aware DP allocation), on seeded synthetic data.
+
+Timing: R state replicas (independent layers of the same shape) are stepped round-robin so
+that more than the 126 MB L2 is touched between two uses of a replica; one round of R
+launches is captured in a CUDA graph and replayed; CUDA events on the launching stream bracket
+the K timed steps, after W untimed warm-up steps, with a barrier + synchronize on both sides.
+Under torchrun every rank runs its own replicas (weak scaling, no collective on the data path)
+and the time is the maximum over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "quantized delta-rule decode: state updates/s and HBM GB/s vs ~8 TB/s peak"
+UNIT = "state-updates/s"
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=1, help="synthetic workload index (1 = Qwen-style GDN)")
+    ap.add_argument("--replicas", type=int, default=0, help="state replicas cycled (0 = enough to exceed L2)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--kernel", choices=["quant", "fp32", "int8"], default="quant")
+    ap.add_argument("--e2e-steps", type=int, default=400)
+    return ap.parse_args()
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = None
+
+    def __enter__(self):
+        if shutil.which("nvidia-smi") is None:
+            return self
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits", "-lms", "20"],
+                                     stdout=self.tmp, stderr=subprocess.DEVNULL)
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.tmp is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in Path(self.tmp.name).read_text().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smmax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwth=parts[6], swth=parts[7], swpc=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.tmp.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwth", "hw_thermal_slowdown"),
+                              ("swth", "sw_thermal_slowdown"), ("swpc", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smmax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+def algorithmic_bytes(layout_bps: int, B: int, H: int, d: int, gate_per_channel: bool, kernel: str) -> int:
+    """Bytes a launch must move: state read + write, scales read + write, q/k/v, beta, gate, o.
+    The per-head bit map, row-impact vector and head offsets (L2-resident) are not counted."""
+    tiles = B * H
+    qkv = 3 * 2 * d
+    gate = 4 * d if gate_per_channel else 4
+    small = tiles * (qkv + 4 + gate + 4 * d)
+    if kernel == "quant":
+        return 2 * B * layout_bps + tiles * 2 * (2 * d + 2 * d) + small
+    if kernel == "int8":
+        return tiles * 2 * (d * d + 2 * d) + small
+    return tiles * 2 * (4 * d * d) + small
+
+
+def run_reference(args, wl):
+    """The oracle (plain C, host cores) on a bounded sample of the same workload."""
+    import oracle
+    from recurrent_state_quantization_gated_b200 import synth
+    cores = len(os.sched_getaffinity(0))
+    seqs = list(range(min(wl.B, 8)))
+    S0 = synth.initial_state(wl, seqs)
+    bits = synth.half_bits(wl) if wl.alloc == "half48" else np.full((wl.H, wl.d), wl.nominal_bits, np.uint8)
+    w = np.ones((wl.H, wl.d), dtype=np.float32)
+    r, c = oracle.fit_scales(S0, w, bits, nthreads=cores)
+    packed = oracle.pack_state(S0, bits, r, c, nthreads=cores)
+    tiles = len(seqs) * wl.H
+    times = []
+    for step in range(args.warmup + args.steps):
+        tok = synth.tokens(wl, step % wl.T, seqs=seqs)
+        t0 = time.perf_counter()
+        packed, r, c, _ = oracle.decode_step(tok, bits, w, packed, r, c, nthreads=cores)
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = tiles * len(times) / total
+    sample = f"{len(seqs)} of {wl.B} sequences x {wl.H} heads ({tiles} tiles) per step, {len(times)} timed steps"
+    return dict(value=value, ms_per_step=1e3 * total / len(times), cores=cores, sample=sample)
+
+
+def cpu_baseline(wl, bits, seconds):
+    import oracle
+    from recurrent_state_quantization_gated_b200 import synth
+    cores = len(os.sched_getaffinity(0))
+    seqs = list(range(min(wl.B, 16)))
+    S0 = synth.initial_state(wl, seqs)
+    w = np.ones((wl.H, wl.d), dtype=np.float32)
+    r, c = oracle.fit_scales(S0, w, bits, nthreads=cores)
+    packed = oracle.pack_state(S0, bits, r, c, nthreads=cores)
+    tiles = len(seqs) * wl.H
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        tok = synth.tokens(wl, steps % wl.T, seqs=seqs)
+        packed, r, c, _ = oracle.decode_step(tok, bits, w, packed, r, c, nthreads=cores)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": tiles * steps / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{steps} decode steps of {len(seqs)} sequences x {wl.H} heads ({tiles} tiles), "
+                      f"OpenMP over tiles, {el:.1f} s"}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from recurrent_state_quantization_gated_b200 import synth
+    wl = synth.workload(args.workload)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        ref = run_reference(args, wl)
+        line = {"metric": METRIC, "value": ref["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ref["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "d": wl.d},
+                "cpu_baseline": {"value": ref["value"], "unit": UNIT, "cores": ref["cores"], "kind": "oracle",
+                                 "sample": ref["sample"]},
+                "e2e": {"value": ref["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    from recurrent_state_quantization_gated_b200 import api, runtime
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- offline calibration and initial quantisation (untimed) -------------------------
+    S0_host = synth.initial_state(wl)
+    S0 = torch.from_numpy(S0_host).cuda()
+    del S0_host
+    cal = synth.calib_tokens(wl)
+    cal_dev = {k: (torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).cuda().view(torch.bfloat16)
+                   if v.dtype == np.uint16 else torch.from_numpy(np.ascontiguousarray(v)).cuda())
+               for k, v in cal.items()}
+    if wl.alloc == "half48":
+        bits = synth.half_bits(wl)
+        w = api.stepq_row_impact(cal_dev["q"], cal_dev["k"], cal_dev["beta"], cal_dev["gate"])
+    else:
+        bits, w = runtime.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), S0, cal_dev)
+    layout = runtime.Layout.build(bits, wl.d)
+    base = runtime.QuantizedState.from_fp32(S0, layout, w)
+    tiles = wl.B * wl.H
+    bytes_launch = algorithmic_bytes(layout.bytes_per_seq, wl.B, wl.H, wl.d, wl.gate_per_channel, args.kernel)
+
+    # Replicas: enough independent states that > 2x L2 is touched between reuses.
+    per_rep = bytes_launch
+    R = args.replicas or max(2, int(np.ceil(2 * L2_BYTES / per_rep)))
+    R = min(R, 64)
+    reps, toks, outs = [], [], []
+    for i in range(R):
+        if args.kernel == "quant":
+            reps.append(dict(packed=base.packed.clone(), r=base.r.clone(), c=base.c.clone()))
+        elif args.kernel == "fp32":
+            reps.append(dict(S=S0.clone()))
+        else:
+            cds, s = api.stepq_int8_quantize_state(S0)
+            reps.append(dict(codes=cds, s=s))
+        toks.append(runtime.to_device_tokens(synth.tokens(wl, i % wl.T)))
+        outs.append(torch.empty((wl.B, wl.H, wl.d), dtype=torch.float32, device="cuda"))
+    del S0
+    torch.cuda.synchronize()
+
+    def launch(i):
+        st, tk, o = reps[i], toks[i], outs[i]
+        if args.kernel == "quant":
+            api.stepq_decode_step(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
+                                  layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
+                                  st["packed"], st["r"], st["c"], o)
+        elif args.kernel == "fp32":
+            api.stepq_decode_step_fp32(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], st["S"], st["S"], o)
+        else:
+            api.stepq_decode_step_int8(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], st["codes"], st["s"],
+                                       st["codes"], st["s"], o)
+
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for i in range(R):          # first launches outside capture (kernel attributes, occupancy)
+            launch(i)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(R):
+            launch(i)
+    rounds_warm = max(1, -(-args.warmup // R))
+    rounds = max(1, -(-args.steps // R))
+    K = rounds * R
+    with torch.cuda.stream(stream):
+        for _ in range(rounds_warm):
+            graph.replay()
+    stream.synchronize()
+    flags = api.stepq_read_device_flags()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local_rank) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(rounds):
+                graph.replay()
+            ev1.record(stream)
+        stream.synchronize()
+        barrier()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / K
+    value = world * tiles * K / (elapsed_ms * 1e-3)
+    achieved_gbs = bytes_launch / (ms_per_step * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+
+    # ---- end to end through the public API with host buffers (H2D inputs, D2H output) ----
+    host_tok = [synth.tokens(wl, t % wl.T) for t in range(8)]
+    pinned = []
+    for tk in host_tok:
+        pinned.append({k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16) if v.dtype == np.uint16 else
+                                           np.ascontiguousarray(v)).pin_memory() for k, v in tk.items()})
+    o_host = torch.empty((wl.B, wl.H, wl.d), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned[0].values())
+    d2h = o_host.numel() * o_host.element_size()
+    n_e2e = max(R, (args.e2e_steps // R) * R)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for s in range(n_e2e):
+            i = s % R
+            src = pinned[s % len(pinned)]
+            for name in ("q", "k", "v"):
+                toks[i][name].view(torch.int16).copy_(src[name], non_blocking=True)
+            toks[i]["beta"].copy_(src["beta"], non_blocking=True)
+            toks[i]["gate"].copy_(src["gate"], non_blocking=True)
+            launch(i)
+            o_host.copy_(outs[i], non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * tiles * n_e2e / (e2e_ms * 1e-3)
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": rounds_warm * R,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "kernel": args.kernel, "B": wl.B, "H": wl.H, "d_k": wl.d, "d_v": wl.d,
+                       "bits_mean": float(bits.astype(np.float64).mean()),
+                       "allocation": wl.alloc, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": f"inputs larger than L2: {R} state replicas stepped round-robin, "
+                             f"{R * per_rep / 2**20:.0f} MiB touched per round",
+                       "timing": "CUDA graph of one round of launches, CUDA events on the launching stream"},
+            "elements_per_s": value * wl.d * wl.d,
+            "achieved_gbs": achieved_gbs,
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": achieved_gbs / peak, "peak_kind": peak_kind, "traffic": None,
+                         "bytes_per_launch": bytes_launch,
+                         "bytes_per_launch_formula": "2*B*bytes_per_seq + B*H*(2*(2d+2d) + 6d + 4 + gate + 4d)"},
+            "gpu_launches": K,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": n_e2e},
+            "device_flags": flags,
+            "clocks": clk.summary(),
+        }
+    if world > 1:
+        graph = None
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1 and args.kernel == "quant":
+            line["cpu_baseline"] = cpu_baseline(wl, bits, args.cpu_seconds)
+        else:
+            line["cpu_baseline"] = None
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

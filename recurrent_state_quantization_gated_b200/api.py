@@ -1,0 +1,186 @@
+"""Python binding of libstepq: the entry points of include/stepq.h under the same names,
+taking PyTorch CUDA tensors. Argument marshalling only; every step runs in the CUDA library.
+
+Tensor conventions (all C-contiguous; device tensors on the current CUDA device):
+  S float32 [B,H,d,d] (row = key channel, column = value channel)
+  q, k, v bfloat16 [B,H,d]; beta float32 [B,H]; gate float32 [B,H] or [B,H,d]
+  bits uint8 [H,d]; w float32 [H,d]; head_off int64 [H]
+  r, c float16 [B,H,d]; packed uint8 [B*bytes_per_seq]; o float32 [B,H,d]
+  INT8 state: codes int8 [B,H,d,d], s float16 [B,H,d]
+All calls are queued on torch's current CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from ._lib import Dims, call, lib
+
+__all__ = [
+    "stepq_packed_layout", "stepq_fit_scales", "stepq_pack_state", "stepq_unpack_state",
+    "stepq_decode_step", "stepq_decode_step_fp32", "stepq_int8_quantize_state",
+    "stepq_decode_step_int8", "stepq_row_impact", "stepq_calib_distortion", "stepq_allocate_bits",
+    "stepq_read_device_flags", "stepq_build_info",
+]
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t: torch.Tensor, dtype: torch.dtype, name: str):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dims(B, H, d, gate_per_channel=0):
+    return Dims(int(B), int(H), int(d), int(d), int(gate_per_channel))
+
+
+def stepq_build_info() -> str:
+    return lib().stepq_build_info().decode()
+
+
+def stepq_packed_layout(bits_host, dv: int, B: int = 1):
+    """(head_off int64 numpy [H], bytes_per_seq, total_bytes) for a host bit map [H][dk]."""
+    bits_host = np.ascontiguousarray(np.asarray(bits_host, dtype=np.uint8))
+    H, dk = bits_host.shape
+    head_off = np.zeros(H, dtype=np.int64)
+    bps = ctypes.c_int64(0)
+    total = ctypes.c_int64(0)
+    call("stepq_packed_layout", Dims(B, H, dk, dv, 0), bits_host.ctypes.data_as(ctypes.c_void_p),
+         head_off.ctypes.data_as(ctypes.c_void_p), ctypes.byref(bps), ctypes.byref(total))
+    return head_off, bps.value, total.value
+
+
+def stepq_fit_scales(S, w, bits, r=None, c=None):
+    B, H, d, _ = S.shape
+    r = torch.empty((B, H, d), dtype=torch.float16, device=S.device) if r is None else r
+    c = torch.empty((B, H, d), dtype=torch.float16, device=S.device) if c is None else c
+    call("stepq_fit_scales", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
+         _ptr(bits, torch.uint8, "bits"), _ptr(r, torch.float16, "r"), _ptr(c, torch.float16, "c"), _stream())
+    return r, c
+
+
+def stepq_pack_state(S, bits, head_off, bytes_per_seq, r, c, packed=None):
+    B, H, d, _ = S.shape
+    packed = torch.empty(B * bytes_per_seq, dtype=torch.uint8, device=S.device) if packed is None else packed
+    call("stepq_pack_state", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(bits, torch.uint8, "bits"),
+         _ptr(head_off, torch.int64, "head_off"), ctypes.c_int64(int(bytes_per_seq)),
+         _ptr(r, torch.float16, "r"), _ptr(c, torch.float16, "c"), _ptr(packed, torch.uint8, "packed"), _stream())
+    return packed
+
+
+def stepq_unpack_state(packed, bits, head_off, bytes_per_seq, r, c, S_out=None):
+    B, H, d = r.shape
+    S_out = torch.empty((B, H, d, d), dtype=torch.float32, device=r.device) if S_out is None else S_out
+    call("stepq_unpack_state", _dims(B, H, d), _ptr(packed, torch.uint8, "packed"), _ptr(bits, torch.uint8, "bits"),
+         _ptr(head_off, torch.int64, "head_off"), ctypes.c_int64(int(bytes_per_seq)),
+         _ptr(r, torch.float16, "r"), _ptr(c, torch.float16, "c"), _ptr(S_out, torch.float32, "S_out"), _stream())
+    return S_out
+
+
+def stepq_decode_step(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
+                      packed_out=None, r_out=None, c_out=None, o=None):
+    """One fused quantized decode step; outputs may alias the inputs (in-place update).
+    Returns (packed_out, r_out, c_out, o)."""
+    B, H, d = q.shape
+    gpc = 1 if gate.dim() == 3 else 0
+    packed_out = torch.empty_like(packed_in) if packed_out is None else packed_out
+    r_out = torch.empty_like(r_in) if r_out is None else r_out
+    c_out = torch.empty_like(c_in) if c_out is None else c_out
+    o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
+    call("stepq_decode_step", _dims(B, H, d, gpc), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+         _ptr(v, torch.bfloat16, "v"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
+         _ptr(bits, torch.uint8, "bits"), _ptr(w, torch.float32, "w"), _ptr(head_off, torch.int64, "head_off"),
+         ctypes.c_int64(int(bytes_per_seq)), _ptr(packed_in, torch.uint8, "packed_in"),
+         _ptr(r_in, torch.float16, "r_in"), _ptr(c_in, torch.float16, "c_in"),
+         _ptr(packed_out, torch.uint8, "packed_out"), _ptr(r_out, torch.float16, "r_out"),
+         _ptr(c_out, torch.float16, "c_out"), _ptr(o, torch.float32, "o"), _stream())
+    return packed_out, r_out, c_out, o
+
+
+def stepq_decode_step_fp32(q, k, v, beta, gate, S_in, S_out=None, o=None):
+    B, H, d = q.shape
+    gpc = 1 if gate.dim() == 3 else 0
+    S_out = torch.empty_like(S_in) if S_out is None else S_out
+    o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
+    call("stepq_decode_step_fp32", _dims(B, H, d, gpc), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+         _ptr(v, torch.bfloat16, "v"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
+         _ptr(S_in, torch.float32, "S_in"), _ptr(S_out, torch.float32, "S_out"), _ptr(o, torch.float32, "o"),
+         _stream())
+    return S_out, o
+
+
+def stepq_int8_quantize_state(S, codes=None, s=None):
+    B, H, d, _ = S.shape
+    codes = torch.empty((B, H, d, d), dtype=torch.int8, device=S.device) if codes is None else codes
+    s = torch.empty((B, H, d), dtype=torch.float16, device=S.device) if s is None else s
+    call("stepq_int8_quantize_state", _dims(B, H, d), _ptr(S, torch.float32, "S"),
+         _ptr(codes, torch.int8, "codes"), _ptr(s, torch.float16, "s"), _stream())
+    return codes, s
+
+
+def stepq_decode_step_int8(q, k, v, beta, gate, codes_in, s_in, codes_out=None, s_out=None, o=None):
+    B, H, d = q.shape
+    gpc = 1 if gate.dim() == 3 else 0
+    codes_out = torch.empty_like(codes_in) if codes_out is None else codes_out
+    s_out = torch.empty_like(s_in) if s_out is None else s_out
+    o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
+    call("stepq_decode_step_int8", _dims(B, H, d, gpc), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+         _ptr(v, torch.bfloat16, "v"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
+         _ptr(codes_in, torch.int8, "codes_in"), _ptr(s_in, torch.float16, "s_in"),
+         _ptr(codes_out, torch.int8, "codes_out"), _ptr(s_out, torch.float16, "s_out"), _ptr(o, torch.float32, "o"),
+         _stream())
+    return codes_out, s_out, o
+
+
+def stepq_row_impact(q, k, beta, gate, w_out=None):
+    """Row impact w [H,d] from a calibration stream with a leading step axis: q, k [T,B,H,d]."""
+    T, B, H, d = q.shape
+    gpc = 1 if gate.dim() == 4 else 0
+    w_out = torch.empty((H, d), dtype=torch.float32, device=q.device) if w_out is None else w_out
+    call("stepq_row_impact", _dims(B, H, d, gpc), ctypes.c_int(T), _ptr(q, torch.bfloat16, "q"),
+         _ptr(k, torch.bfloat16, "k"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
+         _ptr(w_out, torch.float32, "w_out"), _stream())
+    return w_out
+
+
+def stepq_calib_distortion(S, w, b, d_row=None, d_head=None, scratch=None):
+    """(d_row float64 [H,d], d_head float64 [H]) at the uniform width b over the states S."""
+    B, H, d, _ = S.shape
+    dev = S.device
+    d_row = torch.empty((H, d), dtype=torch.float64, device=dev) if d_row is None else d_row
+    d_head = torch.empty((H,), dtype=torch.float64, device=dev) if d_head is None else d_head
+    scratch = torch.empty((B, H, d), dtype=torch.float64, device=dev) if scratch is None else scratch
+    call("stepq_calib_distortion", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
+         ctypes.c_int(int(b)), _ptr(d_row, torch.float64, "d_row"), _ptr(d_head, torch.float64, "d_head"),
+         _ptr(scratch, torch.float64, "scratch"), _stream())
+    return d_row, d_head
+
+
+def stepq_allocate_bits(J, cand, budget_bits: int, mode: int):
+    """Host bit allocation: uint8 numpy [n_units] with exactly budget_bits bits in total."""
+    J = np.ascontiguousarray(np.asarray(J, dtype=np.float64))
+    cand = np.ascontiguousarray(np.asarray(cand, dtype=np.int32))
+    n, nc = J.shape
+    out = np.zeros(n, dtype=np.uint8)
+    call("stepq_allocate_bits", ctypes.c_int(n), ctypes.c_int(nc), cand.ctypes.data_as(ctypes.c_void_p),
+         J.ctypes.data_as(ctypes.c_void_p), ctypes.c_int64(int(budget_bits)), ctypes.c_int(int(mode)),
+         out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def stepq_read_device_flags() -> int:
+    flags = ctypes.c_uint32(0)
+    call("stepq_read_device_flags", ctypes.byref(flags))
+    return flags.value

@@ -1,0 +1,289 @@
+// stepq_baseline.cu -- the two comparison state formats of STEPQuant §5.1 on sm_100a: the FP32
+// state (the serving default) and the uniform symmetric rowwise-absmax INT8 state. Both run the
+// same gated Delta-rule decode step (§2.1) with the readout taken before any requantisation.
+//
+// One CTA per (sequence, head) tile with the register mapping of stepq_device.cuh; the tile is
+// loaded with 16-byte vector loads straight from HBM (each warp instruction reads one full row)
+// and written back the same way.
+#include <cuda_runtime.h>
+
+#include "stepq_device.cuh"
+#include "stepq_internal.h"
+
+namespace stepq {
+
+struct BaselineArgs {
+    int H, gate_per_channel;
+    const uint16_t* q;
+    const uint16_t* k;
+    const uint16_t* v;
+    const float* beta;
+    const float* gate;
+    const float* S_in;
+    float* S_out;
+    const int8_t* codes_in;
+    const uint16_t* s_in;
+    int8_t* codes_out;
+    uint16_t* s_out;
+    float* o;
+};
+
+template <int D>
+struct BaselineSmem {
+    using M = Map<D>;
+    alignas(16) float4 rowc[D];     // alpha_i (gate x row scale), alpha k_i, alpha q_i, k_i
+    alignas(16) float colu[D];
+    alignas(16) float red[M::kWarps][2][D];
+    alignas(16) float rowbuf[M::kWarps][32 * (M::RPT + 1)];
+    alignas(16) float rows[D];      // int8: 1/s~_i
+    float qk;
+};
+
+// Per-row constants (alpha_i = gate_i * row_scale_i) and q.k; one __syncthreads inside.
+template <int D>
+__device__ __forceinline__ void baseline_prologue(BaselineSmem<D>& sm, const BaselineArgs& a, int tile,
+                                                  const uint16_t* row_scale) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid < D) {
+        const float g = a.gate_per_channel ? a.gate[static_cast<int64_t>(tile) * D + tid] : __ldg(a.gate + tile);
+        const float sc = row_scale ? half_bits_to_float(row_scale[static_cast<int64_t>(tile) * D + tid]) : 1.0f;
+        const float alpha = g * sc;
+        const float kk = bf16_bits_to_float(a.k[static_cast<int64_t>(tile) * D + tid]);
+        const float qq = bf16_bits_to_float(a.q[static_cast<int64_t>(tile) * D + tid]);
+        sm.rowc[tid] = make_float4(alpha, alpha * kk, alpha * qq, kk);
+    } else if (warp == D / 32) {
+        constexpr int RL = D / 32;
+        float acc = 0.f;
+#pragma unroll
+        for (int r = 0; r < RL; ++r) {
+            const int i = lane * RL + r;
+            acc = fmaf(bf16_bits_to_float(a.q[static_cast<int64_t>(tile) * D + i]),
+                       bf16_bits_to_float(a.k[static_cast<int64_t>(tile) * D + i]), acc);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) sm.qk = acc;
+    }
+    __syncthreads();
+}
+
+// Shared middle of both kernels: Z holds the state divided by nothing (fp32) or the codes
+// (int8) so that X_ij = alpha_i Z_ij before the update. Computes u and o, then overwrites Z
+// with the updated state X = alpha Z + k u^T.
+template <int D>
+__device__ __forceinline__ void baseline_update(BaselineSmem<D>& sm, const BaselineArgs& a, int tile,
+                                                float Z[Map<D>::RPT][4]) {
+    using M = Map<D>;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cl = M::col_lane(lane);
+    float pacc[4] = {0.f, 0.f, 0.f, 0.f}, oacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r) {
+        const float4 rc = sm.rowc[M::row(warp, lane, r)];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            pacc[k] = fmaf(rc.y, Z[r][k], pacc[k]);
+            oacc[k] = fmaf(rc.z, Z[r][k], oacc[k]);
+        }
+    }
+    combine_subrows<D, float>(pacc, OpAdd());
+    combine_subrows<D, float>(oacc, OpAdd());
+    if (lane < M::LPR) {
+        *reinterpret_cast<float4*>(&sm.red[warp][0][4 * cl]) = make_float4(pacc[0], pacc[1], pacc[2], pacc[3]);
+        *reinterpret_cast<float4*>(&sm.red[warp][1][4 * cl]) = make_float4(oacc[0], oacc[1], oacc[2], oacc[3]);
+    }
+    __syncthreads();
+    if (tid < D) {
+        float ps = 0.f, os = 0.f;
+#pragma unroll
+        for (int w = 0; w < M::kWarps; ++w) {
+            ps += sm.red[w][0][tid];
+            os += sm.red[w][1][tid];
+        }
+        const float u = __ldg(a.beta + tile) * (bf16_bits_to_float(a.v[static_cast<int64_t>(tile) * D + tid]) - ps);
+        a.o[static_cast<int64_t>(tile) * D + tid] = fmaf(sm.qk, u, os);
+        sm.colu[tid] = u;
+    }
+    __syncthreads();
+    const float4 u4 = *reinterpret_cast<const float4*>(&sm.colu[4 * cl]);
+    const float u[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r) {
+        const float4 rc = sm.rowc[M::row(warp, lane, r)];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) Z[r][k] = fmaf(rc.x, Z[r][k], rc.w * u[k]);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) decode_fp32_kernel(const BaselineArgs a) {
+    using M = Map<D>;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    BaselineSmem<D>& sm = *reinterpret_cast<BaselineSmem<D>*>(smem_raw);
+    const int tile = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cl = M::col_lane(lane);
+    const float* S = a.S_in + static_cast<int64_t>(tile) * D * D;
+    float Z[M::RPT][4];
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r) {
+        const float4 x = __ldg(reinterpret_cast<const float4*>(S + M::row(warp, lane, r) * D + 4 * cl));
+        Z[r][0] = x.x; Z[r][1] = x.y; Z[r][2] = x.z; Z[r][3] = x.w;
+    }
+    baseline_prologue<D>(sm, a, tile, nullptr);
+    baseline_update<D>(sm, a, tile, Z);
+    float* So = a.S_out + static_cast<int64_t>(tile) * D * D;
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r)
+        *reinterpret_cast<float4*>(So + M::row(warp, lane, r) * D + 4 * cl) = make_float4(Z[r][0], Z[r][1], Z[r][2], Z[r][3]);
+}
+
+// Rowwise absmax requantisation of a register tile; writes codes and scales.
+template <int D>
+__device__ __forceinline__ void int8_requantise(BaselineSmem<D>& sm, const float X[Map<D>::RPT][4], int tile,
+                                                int8_t* codes_out, uint16_t* s_out) {
+    using M = Map<D>;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cl = M::col_lane(lane);
+    float part[M::RPT];
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r)
+        part[r] = fmaxf(fmaxf(fabsf(X[r][0]), fabsf(X[r][1])), fmaxf(fabsf(X[r][2]), fabsf(X[r][3])));
+    int slot;
+    bool owner;
+    const float mx = row_reduce<D, float>(sm.rowbuf[warp], lane, part, slot, OpMax());
+    const int i = reduced_row<D>(warp, lane, slot, owner);
+    if (owner) {
+        const __half sh = scale_to_half(mx / 127.0f);
+        s_out[static_cast<int64_t>(tile) * D + i] = __half_as_ushort(sh);
+        sm.rows[i] = 1.0f / __half2float(sh);
+    }
+    __syncwarp();
+    int8_t* out = codes_out + static_cast<int64_t>(tile) * D * D;
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r) {
+        const int row = M::row(warp, lane, r);
+        const float is = sm.rows[row];
+        int q[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q[k] = min(max(static_cast<int>(rintf(__fmul_rn(X[r][k], is))), -127), 127);
+        const uint32_t t01 = __byte_perm(q[0], q[1], 0x0040);
+        const uint32_t t23 = __byte_perm(q[2], q[3], 0x0040);
+        *reinterpret_cast<uint32_t*>(out + row * D + 4 * cl) = __byte_perm(t01, t23, 0x5410);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) decode_int8_kernel(const BaselineArgs a) {
+    using M = Map<D>;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    BaselineSmem<D>& sm = *reinterpret_cast<BaselineSmem<D>*>(smem_raw);
+    const int tile = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cl = M::col_lane(lane);
+    const int8_t* C = a.codes_in + static_cast<int64_t>(tile) * D * D;
+    float Z[M::RPT][4];
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r) {
+        const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(C + M::row(warp, lane, r) * D + 4 * cl)) ^ 0x80808080u;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) Z[r][k] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650 | k)) - (kTwo23 + 128.0f);
+    }
+    baseline_prologue<D>(sm, a, tile, a.s_in);
+    baseline_update<D>(sm, a, tile, Z);
+    int8_requantise<D>(sm, Z, tile, a.codes_out, a.s_out);
+}
+
+template <int D>
+__global__ void __launch_bounds__(Map<D>::kThreads) int8_quantize_kernel(const BaselineArgs a) {
+    using M = Map<D>;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    BaselineSmem<D>& sm = *reinterpret_cast<BaselineSmem<D>*>(smem_raw);
+    const int tile = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cl = M::col_lane(lane);
+    const float* S = a.S_in + static_cast<int64_t>(tile) * D * D;
+    float X[M::RPT][4];
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r) {
+        const float4 x = __ldg(reinterpret_cast<const float4*>(S + M::row(warp, lane, r) * D + 4 * cl));
+        X[r][0] = x.x; X[r][1] = x.y; X[r][2] = x.z; X[r][3] = x.w;
+    }
+    int8_requantise<D>(sm, X, tile, a.codes_out, a.s_out);
+}
+
+template <int D>
+static int launch_baseline(const char* fn, void (*kern)(BaselineArgs), int tiles, const BaselineArgs& a,
+                           cudaStream_t st) {
+    if (tiles == 0) return STEPQ_OK;
+    const size_t smem = sizeof(BaselineSmem<D>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "%s: %s", fn, cudaGetErrorString(e));
+    kern<<<tiles, Map<D>::kThreads, smem, st>>>(a);
+    return check_launch(fn);
+}
+
+static int tiles_of(const stepq_dims& d, const char* fn, long long& tiles) {
+    int rc = check_dims(d, fn);
+    if (rc) return rc;
+    tiles = static_cast<long long>(d.B) * d.H;
+    if (tiles > 0x7fffffffLL) return set_error(STEPQ_EINVAL, "%s: too many tiles", fn);
+    return STEPQ_OK;
+}
+
+}  // namespace stepq
+
+using namespace stepq;
+
+extern "C" int stepq_decode_step_fp32(stepq_dims dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                      const float* beta, const float* gate, const float* S_in, float* S_out,
+                                      float* o, void* stream) {
+    clear_error();
+    long long tiles;
+    int rc = tiles_of(dims, "stepq_decode_step_fp32", tiles);
+    if (rc || tiles == 0) return rc;
+    rc = check_ptrs("stepq_decode_step_fp32", {{"q", q}, {"k", k}, {"v", v}, {"beta", beta}, {"gate", gate},
+                                               {"S_in", S_in}, {"S_out", S_out}, {"o", o}});
+    if (rc) return rc;
+    BaselineArgs a{};
+    a.H = dims.H; a.gate_per_channel = dims.gate_per_channel; a.q = q; a.k = k; a.v = v; a.beta = beta;
+    a.gate = gate; a.S_in = S_in; a.S_out = S_out; a.o = o;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return dims.dk == 128 ? launch_baseline<128>("stepq_decode_step_fp32", decode_fp32_kernel<128>, (int)tiles, a, st)
+                          : launch_baseline<64>("stepq_decode_step_fp32", decode_fp32_kernel<64>, (int)tiles, a, st);
+}
+
+extern "C" int stepq_int8_quantize_state(stepq_dims dims, const float* S, int8_t* codes, uint16_t* s, void* stream) {
+    clear_error();
+    long long tiles;
+    int rc = tiles_of(dims, "stepq_int8_quantize_state", tiles);
+    if (rc || tiles == 0) return rc;
+    rc = check_ptrs("stepq_int8_quantize_state", {{"S", S}, {"codes", codes}, {"s", s}});
+    if (rc) return rc;
+    BaselineArgs a{};
+    a.H = dims.H; a.S_in = S; a.codes_out = codes; a.s_out = s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return dims.dk == 128
+               ? launch_baseline<128>("stepq_int8_quantize_state", int8_quantize_kernel<128>, (int)tiles, a, st)
+               : launch_baseline<64>("stepq_int8_quantize_state", int8_quantize_kernel<64>, (int)tiles, a, st);
+}
+
+extern "C" int stepq_decode_step_int8(stepq_dims dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                      const float* beta, const float* gate, const int8_t* codes_in,
+                                      const uint16_t* s_in, int8_t* codes_out, uint16_t* s_out, float* o,
+                                      void* stream) {
+    clear_error();
+    long long tiles;
+    int rc = tiles_of(dims, "stepq_decode_step_int8", tiles);
+    if (rc || tiles == 0) return rc;
+    rc = check_ptrs("stepq_decode_step_int8", {{"q", q}, {"k", k}, {"v", v}, {"beta", beta}, {"gate", gate},
+                                               {"codes_in", codes_in}, {"s_in", s_in}, {"codes_out", codes_out},
+                                               {"s_out", s_out}, {"o", o}});
+    if (rc) return rc;
+    BaselineArgs a{};
+    a.H = dims.H; a.gate_per_channel = dims.gate_per_channel; a.q = q; a.k = k; a.v = v; a.beta = beta;
+    a.gate = gate; a.codes_in = codes_in; a.s_in = s_in; a.codes_out = codes_out; a.s_out = s_out; a.o = o;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return dims.dk == 128 ? launch_baseline<128>("stepq_decode_step_int8", decode_int8_kernel<128>, (int)tiles, a, st)
+                          : launch_baseline<64>("stepq_decode_step_int8", decode_int8_kernel<64>, (int)tiles, a, st);
+}

@@ -1,0 +1,268 @@
+// stepq_device.cuh -- device building blocks shared by the libstepq kernels (sm_100a).
+//
+// Tile mapping (one (sequence, head) state tile of D x D, D = 64 or 128, row = key channel i,
+// column = value channel j): a thread owns 4 adjacent columns (lane % LPR) of RPT rows.
+// LPR = D/4 lanes span one row; a warp covers RPW = 32/LPR rows per instruction; warp w owns
+// the contiguous rows [w*RPT*RPW, (w+1)*RPT*RPW). With D = 128 that is 8 warps x 16 rows and
+// a whole warp on one row at a time, so the bit width (a property of the row) is warp-uniform.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace stepq {
+
+constexpr float kHalfMinNormal = 6.103515625e-05f;   // 2^-14
+constexpr float kHalfMax = 65504.0f;
+constexpr float kRoundMagic = 12582912.0f;            // 1.5 * 2^23: x + M rounds x to an integer
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+constexpr float kTwo23 = 8388608.0f;                  // 2^23
+
+template <int D>
+struct Map {
+    static constexpr int kThreads = (D == 128) ? 256 : 128;
+    static constexpr int kMinBlocks = (D == 128) ? 2 : 4;          // keeps registers <= 128
+    static constexpr int kWarps = kThreads / 32;
+    static constexpr int LPR = D / 4;                  // lanes per row
+    static constexpr int RPW = 32 / LPR;               // rows per warp instruction
+    static constexpr int RPT = D / (kWarps * RPW);     // rows per thread
+    static constexpr int kRowsPerWarp = RPT * RPW;
+    __device__ static int col_lane(int lane) { return lane % LPR; }
+    __device__ static int sub_row(int lane) { return lane / LPR; }
+    __device__ static int row(int warp, int lane, int r) {
+        return warp * kRowsPerWarp + r * RPW + sub_row(lane);
+    }
+};
+
+// ------------------------------------------------------------------------------------------
+// small numeric helpers
+// ------------------------------------------------------------------------------------------
+
+__device__ __forceinline__ int qmax_of(int b) { return (1 << (b - 1)) - 1; }
+__device__ __forceinline__ float znorm_of(int b) { return __int_as_float((127 + 8 - b) << 23); }  // 2^(8-b)
+
+// A positive scale to binary16: clamp into [2^-14, 65504] (NaN -> floor), round to nearest even.
+__device__ __forceinline__ __half scale_to_half(float x) {
+    x = fminf(fmaxf(x, kHalfMinNormal), kHalfMax);   // fmaxf(NaN, a) = a
+    return __float2half_rn(x);
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) {
+    return __half2float(__ushort_as_half(h));
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// ------------------------------------------------------------------------------------------
+// packed codes: 4 adjacent columns (cl*4 .. cl*4+3) of one row at width b.
+// Codes are stored as b-bit two's complement; XOR with the sign bit gives q + 2^(b-1) as an
+// unsigned field, which OR-ed into the mantissa of 2^23 is an exact float.
+// ------------------------------------------------------------------------------------------
+
+template <int D>
+__device__ __forceinline__ void unpack4(const uint8_t* row, int cl, int b, float z[4]) {
+    switch (b) {
+        case 8: {
+            uint32_t u = *reinterpret_cast<const uint32_t*>(row + 4 * cl) ^ 0x80808080u;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                z[k] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650 | k)) - (kTwo23 + 128.0f);
+            break;
+        }
+        case 4: {
+            uint32_t u = *reinterpret_cast<const uint16_t*>(row + 2 * cl) ^ 0x8888u;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                z[k] = __uint_as_float(0x4B000000u | ((u >> (4 * k)) & 0xFu)) - (kTwo23 + 8.0f);
+            break;
+        }
+        case 2: {
+            uint32_t u = row[cl] ^ 0xAAu;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                z[k] = __uint_as_float(0x4B000000u | ((u >> (2 * k)) & 0x3u)) - (kTwo23 + 2.0f);
+            break;
+        }
+        default: {  // 6: low-nibble plane then high-crumb plane
+            uint32_t lo = *reinterpret_cast<const uint16_t*>(row + 2 * cl);
+            uint32_t hi = row[D / 2 + cl] ^ 0xAAu;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                z[k] = __uint_as_float(0x4B000000u | ((lo >> (4 * k)) & 0xFu) |
+                                       (((hi >> (2 * k)) & 0x3u) << 4)) - (kTwo23 + 32.0f);
+            break;
+        }
+    }
+}
+
+// Store 4 signed codes (already clamped to [-q_b, q_b]) of one row at width b.
+template <int D>
+__device__ __forceinline__ void pack4_store(uint8_t* row, int cl, int b, const int q[4]) {
+    switch (b) {
+        case 8: {
+            uint32_t t01 = __byte_perm(q[0], q[1], 0x0040);
+            uint32_t t23 = __byte_perm(q[2], q[3], 0x0040);
+            *reinterpret_cast<uint32_t*>(row + 4 * cl) = __byte_perm(t01, t23, 0x5410);
+            break;
+        }
+        case 4: {
+            uint32_t v = (q[0] & 0xF) | ((q[1] & 0xF) << 4) | ((q[2] & 0xF) << 8) | ((q[3] & 0xF) << 12);
+            *reinterpret_cast<uint16_t*>(row + 2 * cl) = static_cast<uint16_t>(v);
+            break;
+        }
+        case 2: {
+            uint32_t v = (q[0] & 0x3) | ((q[1] & 0x3) << 2) | ((q[2] & 0x3) << 4) | ((q[3] & 0x3) << 6);
+            row[cl] = static_cast<uint8_t>(v);
+            break;
+        }
+        default: {
+            uint32_t lo = (q[0] & 0xF) | ((q[1] & 0xF) << 4) | ((q[2] & 0xF) << 8) | ((q[3] & 0xF) << 12);
+            uint32_t hi = ((q[0] >> 4) & 0x3) | (((q[1] >> 4) & 0x3) << 2) | (((q[2] >> 4) & 0x3) << 4) |
+                          (((q[3] >> 4) & 0x3) << 6);
+            *reinterpret_cast<uint16_t*>(row + 2 * cl) = static_cast<uint16_t>(lo);
+            row[D / 2 + cl] = static_cast<uint8_t>(hi);
+            break;
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// row reduction: every thread holds one partial per owned row (RPT values); the LPR lanes of
+// a sub-row hold the partials of the same rows. Result: the full sum of row r lands in the
+// lanes (s*LPR + hh*RPT + r) for hh in {0, 1}; returns it together with the row slot r.
+// buf: per-warp scratch of 32 * (RPT + 1) floats (padded so both passes are conflict-free).
+// ------------------------------------------------------------------------------------------
+
+template <int D, typename T, typename Op>
+__device__ __forceinline__ T row_reduce(T* buf, int lane, const T part[Map<D>::RPT], int& slot, Op op) {
+    using M = Map<D>;
+    constexpr int RPT = M::RPT;
+    constexpr int LPR = M::LPR;
+    static_assert(LPR == 2 * RPT, "two lanes per row in the reduction");
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) buf[lane * (RPT + 1) + r] = part[r];
+    __syncwarp();
+    const int s = lane / LPR, ll = lane % LPR;
+    const int rr = ll % RPT, hh = ll / RPT;
+    T acc = buf[(s * LPR + hh * RPT) * (RPT + 1) + rr];
+#pragma unroll
+    for (int m = 1; m < RPT; ++m) acc = op(acc, buf[(s * LPR + hh * RPT + m) * (RPT + 1) + rr]);
+    acc = op(acc, __shfl_xor_sync(0xffffffffu, acc, RPT));
+    __syncwarp();
+    slot = rr;
+    return acc;
+}
+
+struct OpAdd {
+    template <typename T>
+    __device__ T operator()(T x, T y) const { return x + y; }
+};
+struct OpMax {
+    __device__ float operator()(float x, float y) const { return fmaxf(x, y); }
+};
+
+// Row of the value returned by row_reduce to this lane, and whether this lane is the one of
+// the two holders that should act on it.
+template <int D>
+__device__ __forceinline__ int reduced_row(int warp, int lane, int slot, bool& owner) {
+    using M = Map<D>;
+    owner = (lane % M::LPR) < M::RPT;
+    return warp * M::kRowsPerWarp + slot * M::RPW + M::sub_row(lane);
+}
+
+// Exclusive prefix of the row byte sizes (D/8 * b_i) of a tile: done by one warp.
+template <int D>
+__device__ __forceinline__ void row_offsets_warp(const uint8_t* bits, uint16_t* roff, int lane) {
+    constexpr int RL = D / 32;
+    int loc[RL], sum = 0;
+#pragma unroll
+    for (int r = 0; r < RL; ++r) {
+        loc[r] = sum;
+        sum += bits[lane * RL + r] * (D / 8);
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+#pragma unroll
+    for (int r = 0; r < RL; ++r) roff[lane * RL + r] = static_cast<uint16_t>(incl - sum + loc[r]);
+}
+
+// Combine the per-thread column partials of the RPW sub-rows of a warp (D = 64 has two).
+template <int D, typename T, typename Op>
+__device__ __forceinline__ void combine_subrows(T v[4], Op op) {
+#pragma unroll
+    for (int m = Map<D>::LPR; m < 32; m <<= 1)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[k] = op(v[k], __shfl_xor_sync(0xffffffffu, v[k], m));
+}
+
+// ------------------------------------------------------------------------------------------
+// bulk async copies (TMA engine, 1-D, no multicast) and mbarriers
+// ------------------------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Global -> shared bulk copy completing on `bar`. bytes: multiple of 16; both addresses
+// 16-byte aligned.
+__device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst_smem)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `parity` of `bar` for at most `limit_ns` nanoseconds of wall time. Returns
+// false (and raises bit 0 of *flags, the caller's device error word) if the limit was reached.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                                  uint32_t* flags) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (global_timer_ns() - t0 > limit_ns) break;
+    }
+    atomicOr(flags, 1u);
+    return false;
+}
+
+}  // namespace stepq

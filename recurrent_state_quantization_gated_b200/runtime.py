@@ -1,0 +1,118 @@
+"""State container and offline calibration built on the libstepq entry points.
+
+``QuantizedState`` keeps one layer's packed recurrent states (codes, fp16 row/column scales,
+the frozen bit map, row-impact vector and packed layout) resident on the GPU and advances them
+with the fused decode kernel. ``calibrate`` runs the offline part of STEPQuant (App. C.2): row
+impact (App. B.3) and candidate distortions (App. A.3) on the GPU, lifetime weighting (§3.2)
+and the discrete allocation (multiple-choice DP or Lagrangian) in the host library.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import api
+
+
+@dataclass
+class Layout:
+    bits: np.ndarray          # uint8 [H][d] (host copy)
+    head_off: np.ndarray      # int64 [H]
+    bytes_per_seq: int
+    d: int
+    bits_dev: torch.Tensor
+    head_off_dev: torch.Tensor
+
+    @classmethod
+    def build(cls, bits: np.ndarray, d: int, device="cuda") -> "Layout":
+        bits = np.ascontiguousarray(np.asarray(bits, dtype=np.uint8))
+        head_off, bps, _ = api.stepq_packed_layout(bits, d, B=1)
+        return cls(bits, head_off, bps, d, torch.from_numpy(bits).to(device),
+                   torch.from_numpy(head_off).to(device))
+
+    @property
+    def H(self) -> int:
+        return self.bits.shape[0]
+
+
+class QuantizedState:
+    """Packed states of B sequences x H heads (one layer)."""
+
+    def __init__(self, layout: Layout, w: torch.Tensor, packed: torch.Tensor, r: torch.Tensor, c: torch.Tensor):
+        self.layout, self.w, self.packed, self.r, self.c = layout, w, packed, r, c
+
+    @classmethod
+    def from_fp32(cls, S: torch.Tensor, layout: Layout, w: torch.Tensor) -> "QuantizedState":
+        """Post-training quantisation of initial states S [B,H,d,d] (fit, then pack)."""
+        r, c = api.stepq_fit_scales(S, w, layout.bits_dev)
+        packed = api.stepq_pack_state(S, layout.bits_dev, layout.head_off_dev, layout.bytes_per_seq, r, c)
+        return cls(layout, w, packed, r, c)
+
+    @property
+    def B(self) -> int:
+        return self.r.shape[0]
+
+    def unpack(self) -> torch.Tensor:
+        L = self.layout
+        return api.stepq_unpack_state(self.packed, L.bits_dev, L.head_off_dev, L.bytes_per_seq, self.r, self.c)
+
+    def step(self, q, k, v, beta, gate, o=None) -> torch.Tensor:
+        """One decode token for every sequence, updating the state in place; returns o [B,H,d]."""
+        L = self.layout
+        _, _, _, o = api.stepq_decode_step(q, k, v, beta, gate, L.bits_dev, self.w, L.head_off_dev,
+                                           L.bytes_per_seq, self.packed, self.r, self.c,
+                                           self.packed, self.r, self.c, o)
+        return o
+
+    def nbytes(self) -> int:
+        return self.packed.numel() + 2 * (self.r.numel() + self.c.numel())
+
+
+def lifetime(unit_gates) -> np.ndarray:
+    """L_u = 1/(1 - g_u): the sum over j >= 0 of g_u^j, the retention of a unit's error (§3.2)."""
+    g = np.asarray(unit_gates, dtype=np.float64)
+    return 1.0 / (1.0 - g)
+
+
+def calibrate(alloc: str, candidates, nominal_bits: int, unit_gates, S0: torch.Tensor, calib: dict):
+    """Offline calibration of one layer. Returns (bits uint8 numpy [H][d], w float32 [H][d] on GPU).
+
+    alloc: "dp_head" (head units, Eq. 17 distortion, multiple-choice DP) or "lagrange_row"
+    (key-row units, Eq. 18 distortion, Lagrangian allocation with repair).
+    unit_gates: [H] (head gates) or [H][d] (key-channel gates); S0: the sample states
+    [B,H,d,d] on the GPU; calib: the calibration stream as GPU tensors with a leading step axis.
+    """
+    w = api.stepq_row_impact(calib["q"], calib["k"], calib["beta"], calib["gate"])
+    H, d = w.shape
+    cand = [int(b) for b in candidates]
+    gates = np.asarray(unit_gates, dtype=np.float64)
+    rows, heads = [], []
+    for b in cand:
+        d_row, d_head = api.stepq_calib_distortion(S0, w, b)
+        rows.append(d_row.cpu().numpy())
+        heads.append(d_head.cpu().numpy())
+    if alloc == "dp_head":
+        dist = np.stack(heads, axis=1)
+        g = gates if gates.ndim == 1 else gates.mean(axis=1)
+        J = lifetime(g)[:, None] * dist
+        bh = api.stepq_allocate_bits(J, cand, nominal_bits * H, mode=1)
+        return np.repeat(bh[:, None], d, axis=1).astype(np.uint8), w
+    if alloc == "lagrange_row":
+        dist = np.stack([x.reshape(-1) for x in rows], axis=1)
+        g = gates.reshape(-1) if gates.ndim == 2 else np.repeat(gates, d)
+        J = lifetime(g)[:, None] * dist
+        br = api.stepq_allocate_bits(J, cand, nominal_bits * H * d, mode=0)
+        return br.reshape(H, d).astype(np.uint8), w
+    raise ValueError(f"unknown allocation {alloc!r}")
+
+
+def to_device_tokens(tok: dict, device="cuda") -> dict:
+    """Host token arrays (bf16 bit patterns as uint16) to GPU tensors of the right dtypes."""
+    out = {}
+    for name in ("q", "k", "v"):
+        out[name] = torch.from_numpy(np.ascontiguousarray(tok[name]).view(np.int16)).to(device).view(torch.bfloat16)
+    out["beta"] = torch.from_numpy(np.ascontiguousarray(tok["beta"], dtype=np.float32)).to(device)
+    out["gate"] = torch.from_numpy(np.ascontiguousarray(tok["gate"], dtype=np.float32)).to(device)
+    return out

@@ -1,0 +1,63 @@
+"""Shared helpers of the GPU parity tests: moving seeded host inputs to the device and comparing
+the CUDA library's results with the oracle's under the stated tolerances."""
+import numpy as np
+
+import oracle
+
+
+def dev(a, dtype=None):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:                    # bf16 / fp16 bit patterns
+        t = torch.from_numpy(a.view(np.int16)).cuda()
+        return t.view(dtype) if dtype is not None else t
+    return torch.from_numpy(a).cuda()
+
+
+def host_half(t):
+    """fp16 torch tensor -> uint16 bit patterns (numpy)."""
+    import torch
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def tokens_dev(tok):
+    import torch
+    return dict(q=dev(tok["q"], torch.bfloat16), k=dev(tok["k"], torch.bfloat16), v=dev(tok["v"], torch.bfloat16),
+                beta=dev(tok["beta"]), gate=dev(tok["gate"]))
+
+
+def tile_codes(packed, bits, d, B):
+    """All codes [B][H][d][d] of a packed state (oracle's unpacker)."""
+    head_off, bps = oracle.layout(bits, d)
+    H = bits.shape[0]
+    out = np.zeros((B, H, d, d), dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            n = oracle.tile_bytes(bits[h], d)
+            off = b * bps + head_off[h]
+            out[b, h] = oracle.unpack_codes(packed[off:off + n], bits[h], d)
+    return out
+
+
+def half_ulps(a, b):
+    """Distance in binary16 units in the last place between two arrays of positive fp16 bits."""
+    return np.abs(a.astype(np.int32) - b.astype(np.int32))
+
+
+def assert_outputs_close(o_gpu, o_ref, rtol=1e-3):
+    """Per-tile relative L2 error and max-normalised elementwise error, both <= rtol."""
+    og = o_gpu.reshape(-1, o_gpu.shape[-1]).astype(np.float64)
+    orf = o_ref.reshape(-1, o_ref.shape[-1]).astype(np.float64)
+    num = np.linalg.norm(og - orf, axis=1)
+    den = np.maximum(np.linalg.norm(orf, axis=1), 1e-30)
+    assert np.max(num / den) <= rtol, f"per-tile L2 rel err {np.max(num / den):.3e}"
+    scale = np.maximum(np.abs(orf).max(axis=1, keepdims=True), 1e-30)
+    assert np.max(np.abs(og - orf) / scale) <= rtol
+
+
+def assert_codes_close(c_gpu, c_ref, max_frac=1e-3):
+    diff = np.abs(c_gpu.astype(np.int64) - c_ref.astype(np.int64))
+    assert diff.max() <= 1, f"codes differ by {diff.max()}"
+    frac = (diff > 0).mean()
+    assert frac <= max_frac, f"{frac:.2e} of codes differ by one step"
+    return frac
