@@ -40,9 +40,12 @@
  *      q = clamp(rint(t), -q_b, q_b), rint = nearest with ties to even.
  *   R4 dequantise: x_hat = (r_i * c_j) * (float)(q 2^(8-b_i)), fp32.
  *   R5 packed layout: tile (b,h) at b*bytes_per_seq + head_off[h]; row i at
- *      (d_v/8) sum_{i'<i} b_i'; a b in {2,4,8} row stores field j at bit j*b of a
- *      little-endian bit stream (two's complement); a 6-bit row stores the low-4-bit plane
- *      (as a 4-bit row) followed by the high-2-bit plane (as a 2-bit row).
+ *      (d_v/8) sum_{i'<i} b_i'; codes are b-bit two's complement. A 2- or 8-bit row stores
+ *      the code of column j at bit j*b of a little-endian bit stream. A 4-bit row stores each
+ *      group of four columns 4g..4g+3 in the 16-bit little-endian halfword g with the
+ *      columns in nibble order (0, 2, 1, 3): column 4g+m sits at bit 4*pos(m),
+ *      pos = {0, 2, 1, 3}. A 6-bit row stores the low 4 bits of every code (laid out as a
+ *      4-bit row) followed by the high 2 bits (laid out as a 2-bit row).
  *   R6 KDA code normalisation (z = 2^(8-b) q) for every workload.
  *   R7 omega floor 1e-12 max_i omega_i; w normalised to mean 1 per head.
  */
@@ -160,6 +163,16 @@ static unsigned get_bits(const uint8_t* base, int64_t bitpos, int width) {
     return v;
 }
 
+/* Bit position of column j inside a row of width b (reading R5). In a 4-bit row the four
+   columns of each 16-bit group are kept in nibble order (0, 2, 1, 3). */
+static int64_t field_bit(int j, int b) {
+    if (b == 4) {
+        static const int pos[4] = {0, 2, 1, 3};
+        return (int64_t)(j / 4) * 16 + 4 * pos[j % 4];
+    }
+    return (int64_t)j * b;
+}
+
 /* Write the signed codes of one row (dv columns) at width b. */
 static void pack_row(uint8_t* row, int dv, int b, const int* q) {
     if (b == 6) {
@@ -167,20 +180,20 @@ static void pack_row(uint8_t* row, int dv, int b, const int* q) {
         uint8_t* hi_plane = row + dv / 2;
         for (int j = 0; j < dv; ++j) {
             unsigned v = (unsigned)q[j] & 63u;             /* 6-bit two's complement */
-            put_bits(lo_plane, (int64_t)j * 4, 4, v & 15u);
-            put_bits(hi_plane, (int64_t)j * 2, 2, v >> 4);
+            put_bits(lo_plane, field_bit(j, 4), 4, v & 15u);
+            put_bits(hi_plane, field_bit(j, 2), 2, v >> 4);
         }
     } else {
         for (int j = 0; j < dv; ++j)
-            put_bits(row, (int64_t)j * b, b, (unsigned)q[j] & ((1u << b) - 1u));
+            put_bits(row, field_bit(j, b), b, (unsigned)q[j] & ((1u << b) - 1u));
     }
 }
 
 static void unpack_row(const uint8_t* row, int dv, int b, int* q) {
     for (int j = 0; j < dv; ++j) {
         unsigned v;
-        if (b == 6) v = get_bits(row, (int64_t)j * 4, 4) | (get_bits(row + dv / 2, (int64_t)j * 2, 2) << 4);
-        else v = get_bits(row, (int64_t)j * b, b);
+        if (b == 6) v = get_bits(row, field_bit(j, 4), 4) | (get_bits(row + dv / 2, field_bit(j, 2), 2) << 4);
+        else v = get_bits(row, field_bit(j, b), b);
         int s = (int)v;
         if (s >= (1 << (b - 1))) s -= (1 << b);            /* sign-extend from b bits */
         q[j] = s;

@@ -43,12 +43,20 @@ def test_every_code_round_trips(b, dv):
 
 
 def _expected_row_bytes(q, b):
-    """Independent construction: 32-bit little-endian words, field j of a b in {2,4,8} row at
-    bit (j*b) mod 32 of word floor(j*b/32); a 6-bit row = 4-bit low plane + 2-bit high plane."""
+    """Independent construction from 32-bit little-endian words: a 2- or 8-bit row holds field
+    j at bit (j*b) mod 32 of word floor(j*b/32); a 4-bit row holds columns 4g..4g+3 in the
+    16-bit halfword g in nibble order 0, 2, 1, 3; a 6-bit row = 4-bit low plane + 2-bit high
+    plane."""
     q = np.asarray(q, dtype=np.int64)
     if b == 6:
         u = q & 63
         return np.concatenate([_expected_row_bytes(u & 15, 4), _expected_row_bytes(u >> 4, 2)])
+    if b == 4:
+        halves = []
+        for g in range(0, len(q), 4):
+            c = [int(x) & 15 for x in q[g:g + 4]]
+            halves.append(c[0] | (c[2] << 4) | (c[1] << 8) | (c[3] << 12))
+        return np.array(halves, dtype="<u2").view(np.uint8)
     per_word = 32 // b
     words = []
     for w0 in range(0, len(q), per_word):
@@ -70,15 +78,16 @@ def test_bytes_match_word_construction_mixed_rows():
 
 
 def test_hand_written_row():
-    """A 4-bit row of codes 1, -1, 7, -7, 0, ... : nibbles 0x1, 0xF, 0x7, 0x9 -> bytes F1 97."""
+    """A 4-bit row of codes 1, -1, 7, -7, 0, ...: nibbles 0x1, 0xF, 0x7, 0x9 stored in the
+    order of columns 0, 2, 1, 3 -> halfword 0x9F71 -> bytes 71 9F."""
     codes = np.zeros((1, 64), dtype=np.int32)
     codes[0, :4] = [1, -1, 7, -7]
     packed = oracle.pack_codes(codes, np.array([4], dtype=np.uint8))
-    assert packed[0] == 0xF1 and packed[1] == 0x97 and not packed[2:].any()
+    assert packed[0] == 0x71 and packed[1] == 0x9F and not packed[2:].any()
     codes6 = np.zeros((1, 64), dtype=np.int32)
     codes6[0, :2] = [-31, 17]   # 6-bit two's complement 0b100001, 0b010001
     p6 = oracle.pack_codes(codes6, np.array([6], dtype=np.uint8))
-    assert p6[0] == 0x11          # low nibbles 1, 1
+    assert p6[0] == 0x01 and p6[1] == 0x01   # low nibbles 1 (col 0, bits 0-3) and 1 (col 1, bits 8-11)
     assert p6[32] == 0x06         # high crumbs 0b10 (bits 0-1), 0b01 (bits 2-3)
 
 
