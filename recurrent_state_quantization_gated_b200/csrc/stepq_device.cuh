@@ -57,75 +57,114 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
 }
 
 // ------------------------------------------------------------------------------------------
-// packed codes: 4 adjacent columns (cl*4 .. cl*4+3) of one row at width b.
-// Codes are stored as b-bit two's complement; XOR with the sign bit gives q + 2^(b-1) as an
-// unsigned field, which OR-ed into the mantissa of 2^23 is an exact float.
+// packed codes: the 4 adjacent columns (4cl .. 4cl+3) of one row at width b.
+// Codes are b-bit two's complement. 2- and 8-bit rows keep column j at bit j*b; a 4-bit row
+// (and the low plane of a 6-bit row) keeps the four columns of each 16-bit group in nibble
+// order 0, 2, 1, 3, i.e. column 4cl+m at bit 4*{0,2,1,3}[m] of halfword cl; a 6-bit row is
+// the low-nibble plane (D/2 bytes) followed by the high-crumb plane (D/4 bytes).
+//
+// Unpacking ORs (sign-flipped) fields into the mantissa of 2^23 so that each field becomes an
+// exact float 2^23 + (q + 2^(b-1)) 2^p, p its bit position; one fused multiply-add by 2^-p
+// then yields q exactly. Packing reads q from the low bits of the float M + q (M = 1.5 2^23).
 // ------------------------------------------------------------------------------------------
 
-template <int D>
-__device__ __forceinline__ void unpack4(const uint8_t* row, int cl, int b, float z[4]) {
-    switch (b) {
-        case 8: {
-            uint32_t u = *reinterpret_cast<const uint32_t*>(row + 4 * cl) ^ 0x80808080u;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                z[k] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650 | k)) - (kTwo23 + 128.0f);
-            break;
-        }
-        case 4: {
-            uint32_t u = *reinterpret_cast<const uint16_t*>(row + 2 * cl) ^ 0x8888u;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                z[k] = __uint_as_float(0x4B000000u | ((u >> (4 * k)) & 0xFu)) - (kTwo23 + 8.0f);
-            break;
-        }
-        case 2: {
-            uint32_t u = row[cl] ^ 0xAAu;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                z[k] = __uint_as_float(0x4B000000u | ((u >> (2 * k)) & 0x3u)) - (kTwo23 + 2.0f);
-            break;
-        }
-        default: {  // 6: low-nibble plane then high-crumb plane
-            uint32_t lo = *reinterpret_cast<const uint16_t*>(row + 2 * cl);
-            uint32_t hi = row[D / 2 + cl] ^ 0xAAu;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                z[k] = __uint_as_float(0x4B000000u | ((lo >> (4 * k)) & 0xFu) |
-                                       (((hi >> (2 * k)) & 0x3u) << 4)) - (kTwo23 + 32.0f);
-            break;
-        }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 bits2(uint32_t a, uint32_t b) { return make_float2(__uint_as_float(a), __uint_as_float(b)); }
+
+template <int D, int BW>
+__device__ __forceinline__ void unpack4(const uint8_t* row, int cl, float2& z01, float2& z23) {
+    constexpr uint32_t F = 0x4B000000u;   // bits of 2^23
+    if constexpr (BW == 8) {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(row + 4 * cl) ^ 0x80808080u;
+        const float2 c = make_float2(-(kTwo23 + 128.0f), -(kTwo23 + 128.0f));
+        z01 = add2(bits2(__byte_perm(u, F, 0x7650), __byte_perm(u, F, 0x7651)), c);
+        z23 = add2(bits2(__byte_perm(u, F, 0x7652), __byte_perm(u, F, 0x7653)), c);
+    } else if constexpr (BW == 4) {
+        const uint32_t u = *reinterpret_cast<const uint16_t*>(row + 2 * cl);
+        z01 = fma2(bits2((u & 0x000Fu) ^ (F | 0x0008u), (u & 0x0F00u) ^ (F | 0x0800u)),
+                   make_float2(1.0f, 0x1p-8f), make_float2(-(kTwo23 + 8.0f), -(0x1p15f + 8.0f)));
+        z23 = fma2(bits2((u & 0x00F0u) ^ (F | 0x0080u), (u & 0xF000u) ^ (F | 0x8000u)),
+                   make_float2(0x1p-4f, 0x1p-12f), make_float2(-(0x1p19f + 8.0f), -(0x1p11f + 8.0f)));
+    } else if constexpr (BW == 2) {
+        const uint32_t u = row[cl];
+        z01 = fma2(bits2((u & 0x03u) ^ (F | 0x02u), (u & 0x0Cu) ^ (F | 0x08u)),
+                   make_float2(1.0f, 0x1p-2f), make_float2(-(kTwo23 + 2.0f), -(0x1p21f + 2.0f)));
+        z23 = fma2(bits2((u & 0x30u) ^ (F | 0x20u), (u & 0xC0u) ^ (F | 0x80u)),
+                   make_float2(0x1p-4f, 0x1p-6f), make_float2(-(0x1p19f + 2.0f), -(0x1p17f + 2.0f)));
+    } else {  // 6: z = lo + 16 (hi - 2), hi = sign-flipped high crumb, both taken exactly
+        const uint32_t lo = *reinterpret_cast<const uint16_t*>(row + 2 * cl);
+        const uint32_t hi = row[D / 2 + cl];
+        const float2 h01 = fma2(bits2((hi & 0x03u) ^ (F | 0x02u), (hi & 0x0Cu) ^ (F | 0x08u)),
+                                make_float2(16.0f, 4.0f), make_float2(-142606368.0f, -33587232.0f));
+        const float2 h23 = fma2(bits2((hi & 0x30u) ^ (F | 0x20u), (hi & 0xC0u) ^ (F | 0x80u)),
+                                make_float2(1.0f, 0.25f), make_float2(-8912928.0f, -2099232.0f));
+        z01 = fma2(bits2((lo & 0x000Fu) | F, (lo & 0x0F00u) | F), make_float2(1.0f, 0x1p-8f), h01);
+        z23 = fma2(bits2((lo & 0x00F0u) | F, (lo & 0xF000u) | F), make_float2(0x1p-4f, 0x1p-12f), h23);
     }
 }
 
-// Store 4 signed codes (already clamped to [-q_b, q_b]) of one row at width b.
+__device__ __forceinline__ uint32_t vmax_s16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t vmin_s16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Store 4 codes of one row at width BW. zq are the bit patterns of M + q (|q| < 2^15); with
+// CLAMP the codes are first limited to [-q_b, q_b] (two at a time, as 16-bit pairs).
+template <int D, int BW, bool CLAMP>
+__device__ __forceinline__ void pack4(uint8_t* row, int cl, uint32_t zq0, uint32_t zq1, uint32_t zq2, uint32_t zq3) {
+    uint32_t p01 = __byte_perm(zq0, zq1, 0x5410);
+    uint32_t p23 = __byte_perm(zq2, zq3, 0x5410);
+    if constexpr (CLAMP) {
+        constexpr uint32_t qb = (1u << (BW - 1)) - 1u;
+        constexpr uint32_t hi = qb | (qb << 16);
+        constexpr uint32_t lo = ((0x10000u - qb) & 0xFFFFu) | ((0x10000u - qb) << 16);
+        p01 = vmin_s16x2(vmax_s16x2(p01, lo), hi);
+        p23 = vmin_s16x2(vmax_s16x2(p23, lo), hi);
+    }
+    const uint32_t t = __byte_perm(p01, p23, 0x6420);   // bytes q0, q1, q2, q3
+    if constexpr (BW == 8) {
+        *reinterpret_cast<uint32_t*>(row + 4 * cl) = t;
+    } else if constexpr (BW == 4) {
+        *reinterpret_cast<uint16_t*>(row + 2 * cl) = static_cast<uint16_t>((t & 0x0F0Fu) | ((t >> 12) & 0xF0F0u));
+    } else if constexpr (BW == 2) {
+        row[cl] = static_cast<uint8_t>(__umulhi((t << 4) & 0x30303030u, 0x10410400u));
+    } else {
+        *reinterpret_cast<uint16_t*>(row + 2 * cl) = static_cast<uint16_t>((t & 0x0F0Fu) | ((t >> 12) & 0xF0F0u));
+        row[D / 2 + cl] = static_cast<uint8_t>(__umulhi(t & 0x30303030u, 0x10410400u));
+    }
+}
+
+// Runtime-width forms (the state conversion kernels; one warp-uniform branch per row).
+template <int D>
+__device__ __forceinline__ void unpack4(const uint8_t* row, int cl, int b, float z[4]) {
+    float2 a, c;
+    switch (b) {
+        case 8: unpack4<D, 8>(row, cl, a, c); break;
+        case 4: unpack4<D, 4>(row, cl, a, c); break;
+        case 2: unpack4<D, 2>(row, cl, a, c); break;
+        default: unpack4<D, 6>(row, cl, a, c); break;
+    }
+    z[0] = a.x; z[1] = a.y; z[2] = c.x; z[3] = c.y;
+}
+
+// Store 4 codes already limited to [-q_b, q_b].
 template <int D>
 __device__ __forceinline__ void pack4_store(uint8_t* row, int cl, int b, const int q[4]) {
+    const uint32_t a = static_cast<uint32_t>(q[0]), bb = static_cast<uint32_t>(q[1]);
+    const uint32_t c = static_cast<uint32_t>(q[2]), d = static_cast<uint32_t>(q[3]);
     switch (b) {
-        case 8: {
-            uint32_t t01 = __byte_perm(q[0], q[1], 0x0040);
-            uint32_t t23 = __byte_perm(q[2], q[3], 0x0040);
-            *reinterpret_cast<uint32_t*>(row + 4 * cl) = __byte_perm(t01, t23, 0x5410);
-            break;
-        }
-        case 4: {
-            uint32_t v = (q[0] & 0xF) | ((q[1] & 0xF) << 4) | ((q[2] & 0xF) << 8) | ((q[3] & 0xF) << 12);
-            *reinterpret_cast<uint16_t*>(row + 2 * cl) = static_cast<uint16_t>(v);
-            break;
-        }
-        case 2: {
-            uint32_t v = (q[0] & 0x3) | ((q[1] & 0x3) << 2) | ((q[2] & 0x3) << 4) | ((q[3] & 0x3) << 6);
-            row[cl] = static_cast<uint8_t>(v);
-            break;
-        }
-        default: {
-            uint32_t lo = (q[0] & 0xF) | ((q[1] & 0xF) << 4) | ((q[2] & 0xF) << 8) | ((q[3] & 0xF) << 12);
-            uint32_t hi = ((q[0] >> 4) & 0x3) | (((q[1] >> 4) & 0x3) << 2) | (((q[2] >> 4) & 0x3) << 4) |
-                          (((q[3] >> 4) & 0x3) << 6);
-            *reinterpret_cast<uint16_t*>(row + 2 * cl) = static_cast<uint16_t>(lo);
-            row[D / 2 + cl] = static_cast<uint8_t>(hi);
-            break;
-        }
+        case 8: pack4<D, 8, false>(row, cl, a, bb, c, d); break;
+        case 4: pack4<D, 4, false>(row, cl, a, bb, c, d); break;
+        case 2: pack4<D, 2, false>(row, cl, a, bb, c, d); break;
+        default: pack4<D, 6, false>(row, cl, a, bb, c, d); break;
     }
 }
 
