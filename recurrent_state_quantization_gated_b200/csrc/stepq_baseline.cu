@@ -86,8 +86,8 @@ __device__ __forceinline__ void baseline_update(BaselineSmem<D>& sm, const Basel
             oacc[k] = fmaf(rc.z, Z[r][k], oacc[k]);
         }
     }
-    combine_subrows<D, float>(pacc, OpAdd());
-    combine_subrows<D, float>(oacc, OpAdd());
+    combine_subrows<Map<D>, float>(pacc, OpAdd());
+    combine_subrows<Map<D>, float>(oacc, OpAdd());
     if (lane < M::LPR) {
         *reinterpret_cast<float4*>(&sm.red[warp][0][4 * cl]) = make_float4(pacc[0], pacc[1], pacc[2], pacc[3]);
         *reinterpret_cast<float4*>(&sm.red[warp][1][4 * cl]) = make_float4(oacc[0], oacc[1], oacc[2], oacc[3]);
@@ -151,8 +151,8 @@ __device__ __forceinline__ void int8_requantise(BaselineSmem<D>& sm, const float
         part[r] = fmaxf(fmaxf(fabsf(X[r][0]), fabsf(X[r][1])), fmaxf(fabsf(X[r][2]), fabsf(X[r][3])));
     int slot;
     bool owner;
-    const float mx = row_reduce<D, float>(sm.rowbuf[warp], lane, part, slot, OpMax());
-    const int i = reduced_row<D>(warp, lane, slot, owner);
+    const float mx = row_reduce<Map<D>, float>(sm.rowbuf[warp], lane, part, slot, OpMax());
+    const int i = reduced_row<Map<D>>(warp, lane, slot, owner);
     if (owner) {
         const __half sh = scale_to_half(mx / 127.0f);
         s_out[static_cast<int64_t>(tile) * D + i] = __half_as_ushort(sh);

@@ -1,10 +1,11 @@
 // stepq_decode.cu -- the fused quantized decode step (STEPQuant, Table C2) for sm_100a.
 //
-// One persistent CTA per SM slot walks over (sequence, head) tiles. For each tile the bulk-copy
-// (TMA) engine stages the packed codes, the old scales, q/k/v, the gate and the head's bit map
-// and row-impact vector into shared memory, double buffered so that the next tile's copy runs
-// while this one is computed. The tile then lives in registers (a thread owns 4 columns of 16
-// rows) through every phase:
+// One persistent CTA per SM slot walks over (sequence, head) tiles. The frozen bit map is
+// turned once per launch into per-head tables (rows sorted by width, byte offsets, row-impact
+// factors) kept in shared memory. For each tile the bulk-copy (TMA) engine stages the packed
+// codes, the old scales, q/k/v and the gate into shared memory, double buffered so that the
+// next tile's copy runs while this one is computed. The tile then lives in registers (a thread
+// owns 8 columns of D/16 rows) through every phase:
 //   1 unpack + dequantise (the column scale is factored out: Xi_ij = X_ij / c_j), and the two
 //     column dot products k^T D S and q^T D S of the Delta rule;
 //   2 u = beta (v - k^T D S), o = q^T X = q^T D S + (q.k) u          (§2.1, Table C2 step 3);
@@ -14,8 +15,9 @@
 //   6 final codes at (r, c), packed and stored straight to HBM.
 // Rows are visited sorted by bit width, so almost every warp runs a width-specialised unpack
 // and pack; floating-point work runs on packed f32x2 instructions. Column reductions cross
-// warps through shared memory, row reductions stay inside a warp. The state is read once and
-// written once; no tensor cores (a rank-1 update per token is not a dense contraction).
+// warps through shared memory, row reductions stay inside a warp. The state is read from HBM
+// once and written once; no tensor cores (a rank-1 update per token is not a dense
+// contraction).
 #include <cuda_runtime.h>
 
 #include "stepq_device.cuh"
@@ -46,9 +48,38 @@ struct DecodeArgs {
     float* o;
 };
 
+// Mapping of a tile onto one CTA: a thread owns 8 adjacent columns of RPT rows; LPR lanes span
+// a row; a warp covers RPW rows per instruction and owns 16 consecutive slots (rows sorted by
+// width).
+template <int D>
+struct DMap {
+    static constexpr int kCols = 8;
+    static constexpr int kThreads = (D == 128) ? 256 : 128;
+    static constexpr int kMinBlocks = (D == 128) ? 2 : 4;
+    static constexpr int kWarps = kThreads / 32;
+    static constexpr int LPR = D / kCols;               // lanes per row
+    static constexpr int RPW = 32 / LPR;                // rows per warp instruction
+    static constexpr int RPT = D / (kWarps * RPW);      // rows per thread
+    static constexpr int kRowsPerWarp = RPT * RPW;
+    __device__ static int col_lane(int lane) { return lane % LPR; }
+    __device__ static int sub_row(int lane) { return lane / LPR; }
+    __device__ static int row(int warp, int lane, int r) { return warp * kRowsPerWarp + r * RPW + sub_row(lane); }
+};
+
+constexpr int kStages = 3;   // tile copies in flight: the current tile and the next two
+
+// Sorted-row tables of heads kept in shared memory: a direct-mapped cache (head h lives in
+// entry h % kHeads), filled when a tile of a head not held is decoded. With at most kHeads
+// heads every table is built once per CTA and launch.
+template <int D>
+struct HeadCache {
+    static constexpr int kHeads = (D == 128) ? 32 : 64;
+};
+
 template <int D>
 struct DecodeSmem {
-    using M = Map<D>;
+    using M = DMap<D>;
+    static constexpr int CH = HeadCache<D>::kHeads;
     struct Stage {
         alignas(16) uint8_t codes[D * D];   // room for an all-8-bit tile
         alignas(16) uint16_t r[D];
@@ -57,37 +88,44 @@ struct DecodeSmem {
         alignas(16) uint16_t k[D];
         alignas(16) uint16_t v[D];
         alignas(16) float gate[D];
-        alignas(16) uint8_t bits[D];
         alignas(16) float w[D];
+        float beta;                          // scalars of this tile, prefetched with it
+        float gate1;
     };
-    Stage stage[2];
-    alignas(16) float4 rc0[D];      // by key row i: alpha, alpha, alpha k, alpha k  (alpha = g r 2^(8-b))
-    alignas(16) float4 rc1[D];      // by key row i: alpha q, alpha q, k, k
-    alignas(16) float4 rq[D];       // by slot: e, e, G, G  (e = 1/(r~ 2^(8-b)), G = (w r~ 2^(8-b))^2)
-    alignas(16) float riq[D];       // by slot: 1/q_b
-    alignas(16) uint32_t meta[D];   // by slot: row | width << 8 | byte offset << 16
+    Stage stage[kStages];
+    // Per head (cached): per slot (rows sorted by width, stable) the row's metadata
+    // row | width << 8 | byte offset << 16.
+    alignas(16) uint32_t hmeta[CH][D];
+    int htag[CH];                   // head held by each cache entry (-1: none)
+    // Per slot of the tile being decoded.
+    alignas(16) float4 kq[D];       // alpha k, alpha k, alpha q, alpha q   (alpha = g r 2^(8-b))
+    alignas(16) float4 ak[D];       // alpha, alpha, k, k
+    alignas(16) float4 rq[D];       // e, e, G, G  (e = 1/(r~ 2^(8-b)), G = (w r~ 2^(8-b))^2)
+    alignas(16) float riq[D];       // 1/q_b
+    // Per column.
     alignas(16) float colc[D];      // c_j (old column scale)
     alignas(16) float colb[D];      // per-phase column broadcast
     alignas(16) float col0[D];      // c0_j
     alignas(16) float colm[D];      // max_i |xi_ij| / q_b
     alignas(16) float red[M::kWarps][2][D];
     alignas(16) float rowbuf[M::kWarps][32 * (M::RPT + 1)];
-    alignas(8) uint64_t full[2];
+    alignas(8) uint64_t full[kStages];
     float qk;
 };
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a tile copy takes microseconds
 
+// Queue the bulk copies of `tile` into stage s (one thread). The tile's two scalars are
+// returned in registers for the caller to store later, so their load latency stays hidden.
 template <int D>
-__device__ __forceinline__ void issue_tile(const DecodeArgs& a, DecodeSmem<D>& sm, int n, int s) {
-    const int tile = blockIdx.x + n * gridDim.x;
-    if (tile >= a.num_tiles) return;
+__device__ __forceinline__ bool issue_tile(const DecodeArgs& a, DecodeSmem<D>& sm, int tile, int s, float& beta,
+                                           float& gate1) {
+    if (tile >= a.num_tiles) return false;
     const int b = tile / a.H, h = tile % a.H;
-    const int64_t hoff = a.head_off[h];
-    const int64_t hend = (h + 1 < a.H) ? a.head_off[h + 1] : a.bytes_per_seq;
+    const int64_t hoff = a.head_off[h], hend = (h + 1 < a.H) ? a.head_off[h + 1] : a.bytes_per_seq;
     const uint32_t pbytes = static_cast<uint32_t>(hend - hoff);
     auto& st = sm.stage[s];
-    const uint32_t total = pbytes + 5u * 2u * D + D + 4u * D + (a.gate_per_channel ? 4u * D : 0u);
+    const uint32_t total = pbytes + 5u * 2u * D + 4u * D + (a.gate_per_channel ? 4u * D : 0u);
     mbar_arrive_expect_tx(&sm.full[s], total);
     bulk_load(st.codes, a.packed_in + b * a.bytes_per_seq + hoff, pbytes, &sm.full[s]);
     bulk_load(st.r, a.r_in + static_cast<int64_t>(tile) * D, 2 * D, &sm.full[s]);
@@ -95,21 +133,22 @@ __device__ __forceinline__ void issue_tile(const DecodeArgs& a, DecodeSmem<D>& s
     bulk_load(st.q, a.q + static_cast<int64_t>(tile) * D, 2 * D, &sm.full[s]);
     bulk_load(st.k, a.k + static_cast<int64_t>(tile) * D, 2 * D, &sm.full[s]);
     bulk_load(st.v, a.v + static_cast<int64_t>(tile) * D, 2 * D, &sm.full[s]);
-    bulk_load(st.bits, a.bits + static_cast<int64_t>(h) * D, D, &sm.full[s]);
     bulk_load(st.w, a.w + static_cast<int64_t>(h) * D, 4 * D, &sm.full[s]);
     if (a.gate_per_channel) bulk_load(st.gate, a.gate + static_cast<int64_t>(tile) * D, 4 * D, &sm.full[s]);
+    beta = __ldg(a.beta + tile);
+    gate1 = a.gate_per_channel ? 0.f : __ldg(a.gate + tile);
+    return true;
 }
 
-// Sort the rows of a tile by bit width (stable) and record, per slot, the row, its width and
-// the byte offset of the row in the packed tile. One warp.
+// One warp sorts the rows of head h by bit width (stable) into cache entry e.
 template <int D>
-__device__ __forceinline__ void sort_rows_warp(const uint8_t* bits, uint32_t* meta, int lane) {
+__device__ __forceinline__ void sort_head_warp(const DecodeArgs& a, DecodeSmem<D>& sm, int h, int e, int lane) {
     constexpr int RL = D / 32;
     int bw[RL], loc[RL], rank[RL], sum = 0;
     int cnt[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int r = 0; r < RL; ++r) {
-        bw[r] = bits[lane * RL + r];
+        bw[r] = a.bits[static_cast<int64_t>(h) * D + lane * RL + r];
         loc[r] = sum;
         sum += bw[r] * (D / 8);
         const int cls = (bw[r] >> 1) - 1;
@@ -141,113 +180,143 @@ __device__ __forceinline__ void sort_rows_warp(const uint8_t* bits, uint32_t* me
     }
 #pragma unroll
     for (int r = 0; r < RL; ++r) {
+        const int i = lane * RL + r;
         const int cls = (bw[r] >> 1) - 1;
         int slot = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
             if (c == cls) slot = base_c[c] + excl_c[c] + rank[r];
         const int off = incl - sum + loc[r];
-        meta[slot] = static_cast<uint32_t>(lane * RL + r) | (static_cast<uint32_t>(bw[r]) << 8) |
-                     (static_cast<uint32_t>(off) << 16);
+        sm.hmeta[e][slot] = static_cast<uint32_t>(i) | (static_cast<uint32_t>(bw[r]) << 8) | (static_cast<uint32_t>(off) << 16);
     }
 }
 
 // ---- phase 1: unpack the thread's rows and accumulate the k^T and q^T products -------------
 template <int D, int BW>
-__device__ __forceinline__ void phase1_row(const DecodeSmem<D>& sm, const uint8_t* codes, uint32_t mt, int cl,
-                                           float2& z01, float2& z23, float2 pacc[2], float2 oacc[2]) {
-    const int i = mt & 0xFF;
-    unpack4<D, BW>(codes + (mt >> 16), cl, z01, z23);
-    const float4 c0 = sm.rc0[i], c1 = sm.rc1[i];
-    const float2 kap = make_float2(c0.z, c0.w), lam = make_float2(c1.x, c1.y);
-    pacc[0] = fma2(kap, z01, pacc[0]);
-    pacc[1] = fma2(kap, z23, pacc[1]);
-    oacc[0] = fma2(lam, z01, oacc[0]);
-    oacc[1] = fma2(lam, z23, oacc[1]);
+__device__ __forceinline__ void phase1_row(const DecodeSmem<D>& sm, const uint8_t* codes, int s, uint32_t mt,
+                                           int cl, float2 z[4], float2 pacc[4], float2 oacc[4]) {
+    unpack8<D, BW>(codes + (mt >> 16), cl, z);
+    const float4 c = sm.kq[s];
+    const float2 kap = make_float2(c.x, c.y), lam = make_float2(c.z, c.w);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        pacc[p] = fma2(kap, z[p], pacc[p]);
+        oacc[p] = fma2(lam, z[p], oacc[p]);
+    }
 }
 
 template <int D, int BW>
-__device__ __forceinline__ void phase1_uniform(const DecodeSmem<D>& sm, const uint8_t* codes, int warp, int lane,
-                                               float2 Z[][2], float2 pacc[2], float2 oacc[2]) {
-    using M = Map<D>;
-    const int cl = M::col_lane(lane);
-#pragma unroll
-    for (int r = 0; r < M::RPT; ++r)
-        phase1_row<D, BW>(sm, codes, sm.meta[M::row(warp, lane, r)], cl, Z[r][0], Z[r][1], pacc, oacc);
-}
-
-template <int D>
-__device__ __forceinline__ void phase1_mixed(const DecodeSmem<D>& sm, const uint8_t* codes, int warp, int lane,
-                                             float2 Z[][2], float2 pacc[2], float2 oacc[2]) {
-    using M = Map<D>;
+__device__ __forceinline__ void phase1_uniform(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* codes,
+                                               int warp, int lane, float2 Z[][4], float2 pacc[4], float2 oacc[4]) {
+    using M = DMap<D>;
     const int cl = M::col_lane(lane);
 #pragma unroll
     for (int r = 0; r < M::RPT; ++r) {
-        const uint32_t mt = sm.meta[M::row(warp, lane, r)];
+        const int s = M::row(warp, lane, r);
+        phase1_row<D, BW>(sm, codes, s, meta[s], cl, Z[r], pacc, oacc);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void phase1_mixed(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* codes,
+                                             int warp, int lane, float2 Z[][4], float2 pacc[4], float2 oacc[4]) {
+    using M = DMap<D>;
+    const int cl = M::col_lane(lane);
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r) {
+        const int s = M::row(warp, lane, r);
+        const uint32_t mt = meta[s];
         switch ((mt >> 8) & 0xFF) {
-            case 8: phase1_row<D, 8>(sm, codes, mt, cl, Z[r][0], Z[r][1], pacc, oacc); break;
-            case 6: phase1_row<D, 6>(sm, codes, mt, cl, Z[r][0], Z[r][1], pacc, oacc); break;
-            case 4: phase1_row<D, 4>(sm, codes, mt, cl, Z[r][0], Z[r][1], pacc, oacc); break;
-            default: phase1_row<D, 2>(sm, codes, mt, cl, Z[r][0], Z[r][1], pacc, oacc); break;
+            case 8: phase1_row<D, 8>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
+            case 6: phase1_row<D, 6>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
+            case 4: phase1_row<D, 4>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
+            default: phase1_row<D, 2>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
         }
     }
 }
 
 // ---- phase 6: final codes, packed and stored ------------------------------------------------
 template <int D, int BW, bool CLAMP>
-__device__ __forceinline__ void phase6_row(uint8_t* out, uint32_t mt, int cl, float2 x01, float2 x23, float2 f01,
-                                           float2 f23) {
+__device__ __forceinline__ void phase6_row(uint8_t* out, uint32_t mt, int cl, const float2 x[4], const float2 f[4]) {
     const float2 M2 = make_float2(kRoundMagic, kRoundMagic);
-    const float2 a = fma2(x01, f01, M2), b = fma2(x23, f23, M2);
-    pack4<D, BW, CLAMP>(out + (mt >> 16), cl, __float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x),
-                        __float_as_uint(b.y));
+    uint32_t zq[8];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float2 t = fma2(x[p], f[p], M2);
+        zq[2 * p] = __float_as_uint(t.x);
+        zq[2 * p + 1] = __float_as_uint(t.y);
+    }
+    pack8<D, BW, CLAMP>(out + (mt >> 16), cl, zq);
 }
 
 template <int D, int BW, bool CLAMP>
-__device__ __forceinline__ void phase6_uniform(const DecodeSmem<D>& sm, uint8_t* out, int warp, int lane,
-                                               const float2 Z[][2], float2 f01, float2 f23) {
-    using M = Map<D>;
+__device__ __forceinline__ void phase6_uniform(const uint32_t* meta, uint8_t* out, int warp, int lane,
+                                               const float2 Z[][4], const float2 f[4]) {
+    using M = DMap<D>;
     const int cl = M::col_lane(lane);
 #pragma unroll
-    for (int r = 0; r < M::RPT; ++r)
-        phase6_row<D, BW, CLAMP>(out, sm.meta[M::row(warp, lane, r)], cl, Z[r][0], Z[r][1], f01, f23);
+    for (int r = 0; r < M::RPT; ++r) phase6_row<D, BW, CLAMP>(out, meta[M::row(warp, lane, r)], cl, Z[r], f);
 }
 
 template <int D, bool CLAMP>
-__device__ __forceinline__ void phase6_mixed(const DecodeSmem<D>& sm, uint8_t* out, int warp, int lane,
-                                             const float2 Z[][2], float2 f01, float2 f23) {
-    using M = Map<D>;
+__device__ __forceinline__ void phase6_mixed(const uint32_t* meta, uint8_t* out, int warp, int lane,
+                                             const float2 Z[][4], const float2 f[4]) {
+    using M = DMap<D>;
     const int cl = M::col_lane(lane);
 #pragma unroll
     for (int r = 0; r < M::RPT; ++r) {
-        const uint32_t mt = sm.meta[M::row(warp, lane, r)];
+        const uint32_t mt = meta[M::row(warp, lane, r)];
         switch ((mt >> 8) & 0xFF) {
-            case 8: phase6_row<D, 8, CLAMP>(out, mt, cl, Z[r][0], Z[r][1], f01, f23); break;
-            case 6: phase6_row<D, 6, CLAMP>(out, mt, cl, Z[r][0], Z[r][1], f01, f23); break;
-            case 4: phase6_row<D, 4, CLAMP>(out, mt, cl, Z[r][0], Z[r][1], f01, f23); break;
-            default: phase6_row<D, 2, CLAMP>(out, mt, cl, Z[r][0], Z[r][1], f01, f23); break;
+            case 8: phase6_row<D, 8, CLAMP>(out, mt, cl, Z[r], f); break;
+            case 6: phase6_row<D, 6, CLAMP>(out, mt, cl, Z[r], f); break;
+            case 4: phase6_row<D, 4, CLAMP>(out, mt, cl, Z[r], f); break;
+            default: phase6_row<D, 2, CLAMP>(out, mt, cl, Z[r], f); break;
         }
     }
 }
 
 template <int D, bool CLAMP>
-__device__ __forceinline__ void phase6(const DecodeSmem<D>& sm, uint8_t* out, int warp, int lane, int ww,
-                                       const float2 Z[][2], float2 f01, float2 f23) {
+__device__ __forceinline__ void phase6(const uint32_t* meta, uint8_t* out, int warp, int lane, int ww,
+                                       const float2 Z[][4], const float2 f[4]) {
     switch (ww) {
-        case 8: phase6_uniform<D, 8, CLAMP>(sm, out, warp, lane, Z, f01, f23); break;
-        case 6: phase6_uniform<D, 6, CLAMP>(sm, out, warp, lane, Z, f01, f23); break;
-        case 4: phase6_uniform<D, 4, CLAMP>(sm, out, warp, lane, Z, f01, f23); break;
-        case 2: phase6_uniform<D, 2, CLAMP>(sm, out, warp, lane, Z, f01, f23); break;
-        default: phase6_mixed<D, CLAMP>(sm, out, warp, lane, Z, f01, f23); break;
+        case 8: phase6_uniform<D, 8, CLAMP>(meta, out, warp, lane, Z, f); break;
+        case 6: phase6_uniform<D, 6, CLAMP>(meta, out, warp, lane, Z, f); break;
+        case 4: phase6_uniform<D, 4, CLAMP>(meta, out, warp, lane, Z, f); break;
+        case 2: phase6_uniform<D, 2, CLAMP>(meta, out, warp, lane, Z, f); break;
+        default: phase6_mixed<D, CLAMP>(meta, out, warp, lane, Z, f); break;
     }
 }
 
+// Sum (over the warp's sub-rows) the per-thread partials of eight columns and store them.
 template <int D>
-__global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks)
+__device__ __forceinline__ void store_col_partials(float* dst, int lane, float2 v[4]) {
+    using M = DMap<D>;
+#pragma unroll
+    for (int m = M::LPR; m < 32; m <<= 1)
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+            v[p] = add2(v[p], make_float2(__shfl_xor_sync(0xffffffffu, v[p].x, m), __shfl_xor_sync(0xffffffffu, v[p].y, m)));
+    if (lane < M::LPR) {
+        const int cl = M::col_lane(lane);
+        *reinterpret_cast<float4*>(dst + 8 * cl) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+        *reinterpret_cast<float4*>(dst + 8 * cl + 4) = make_float4(v[2].x, v[2].y, v[3].x, v[3].y);
+    }
+}
+
+__device__ __forceinline__ void load_cols8(const float* src, int cl, float2 out[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(src + 8 * cl);
+    const float4 b = *reinterpret_cast<const float4*>(src + 8 * cl + 4);
+    out[0] = make_float2(a.x, a.y);
+    out[1] = make_float2(a.z, a.w);
+    out[2] = make_float2(b.x, b.y);
+    out[3] = make_float2(b.z, b.w);
+}
+
+template <int D>
+__global__ void __launch_bounds__(DMap<D>::kThreads, DMap<D>::kMinBlocks)
 decode_kernel(const DecodeArgs a) {
-    using M = Map<D>;
+    using M = DMap<D>;
     constexpr int RPT = M::RPT;
-    constexpr int LPR = M::LPR;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     DecodeSmem<D>& sm = *reinterpret_cast<DecodeSmem<D>*>(smem_raw);
 
@@ -255,88 +324,124 @@ decode_kernel(const DecodeArgs a) {
     const int warp = tid >> 5, lane = tid & 31;
     const int cl = M::col_lane(lane);
     const float2 M2 = make_float2(kRoundMagic, kRoundMagic);
+    // The last thread queues the copies (no prologue work waits on it).
+    const bool issuer = (tid == M::kThreads - 1);
 
-    if (tid == 0) {
-        mbar_init(&sm.full[0], 1);
-        mbar_init(&sm.full[1], 1);
+    // Per-head tables (the bit map is frozen and shared by all sequences): the heads of the
+    // CTA's first tiles are sorted up front, one warp per head; the rest on first use.
+    constexpr int CH = HeadCache<D>::kHeads;
+    for (int e = tid; e < CH; e += M::kThreads) sm.htag[e] = -1;
+    __syncthreads();
+    for (int n = warp; n < CH; n += M::kWarps) {
+        const int tile = blockIdx.x + n * gridDim.x;
+        if (tile >= a.num_tiles) break;
+        const int h = tile % a.H;
+        // Sort here only if no earlier tile of this CTA uses the same head or the same entry.
+        bool take = true;
+        for (int m = 0; m < n; ++m)
+            if (((blockIdx.x + m * gridDim.x) % a.H) % CH == h % CH) take = false;
+        if (take) {
+            sort_head_warp<D>(a, sm, h, h % CH, lane);
+            if (lane == 0) sm.htag[h % CH] = h;
+        }
+    }
+    if (issuer) {
+        for (int i = 0; i < kStages; ++i) mbar_init(&sm.full[i], 1);
         fence_barrier_init();
-        issue_tile<D>(a, sm, 0, 0);
+    }
+    __syncthreads();
+    if (issuer) {
+        for (int i = 0; i + 1 < kStages; ++i) {
+            float b0, g0;
+            if (issue_tile<D>(a, sm, blockIdx.x + i * gridDim.x, i, b0, g0)) {
+                sm.stage[i].beta = b0;
+                sm.stage[i].gate1 = g0;
+            }
+        }
     }
     __syncthreads();
 
     for (int n = 0;; ++n) {
         const int tile = blockIdx.x + n * gridDim.x;
         if (tile >= a.num_tiles) break;
-        const int s = n & 1;
-        const bool ok = mbar_wait_bounded(&sm.full[s], (n >> 1) & 1, kWaitLimitNs, &g_stepq_flags);
+        const int s = n % kStages;
+        const uint32_t parity = (n / kStages) & 1;
+        const auto& st = sm.stage[s];
+        const int h = tile % a.H, he = h % CH;
+        const uint32_t* meta = sm.hmeta[he];
+        const int64_t tile_base = static_cast<int64_t>(tile / a.H) * a.bytes_per_seq + a.head_off[h];
+        if (sm.htag[he] != h) {                     // every warp sees the same tag: uniform branch
+            __syncthreads();                        // nobody still reads the entry
+            if (warp == 0) {
+                sort_head_warp<D>(a, sm, h, he, lane);
+                if (lane == 0) sm.htag[he] = h;
+            }
+            __syncthreads();
+        }
+        const bool ok = mbar_wait_bounded(&sm.full[s], parity, kWaitLimitNs, &g_stepq_flags);
+
+        // ---- prologue: per-slot constants of this tile, q.k ------------------------------
+        if (ok) {
+            if (tid < D) {
+                const int sl = tid;
+                const uint32_t mt = meta[sl];
+                const int i = mt & 0xFF, bw = (mt >> 8) & 0xFF;
+                const float g = a.gate_per_channel ? st.gate[i] : st.gate1;
+                const float alpha = g * half_bits_to_float(st.r[i]) * znorm_of(bw);
+                const float kk = bf16_bits_to_float(st.k[i]);
+                const float qq = bf16_bits_to_float(st.q[i]);
+                sm.kq[sl] = make_float4(alpha * kk, alpha * kk, alpha * qq, alpha * qq);
+                sm.ak[sl] = make_float4(alpha, alpha, kk, kk);
+            } else if (warp == D / 32) {
+                constexpr int RL = D / 32;
+                float acc = 0.f;
+#pragma unroll
+                for (int r = 0; r < RL; ++r)
+                    acc = fmaf(bf16_bits_to_float(st.q[lane * RL + r]), bf16_bits_to_float(st.k[lane * RL + r]), acc);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                if (lane == 0) sm.qk = acc;
+            }
+        }
         if (__syncthreads_or(!ok)) {
             // A tile copy never arrived: give up (the host reads the error word), after one
-            // more bounded wait for that copy, the only one in flight.
-            if (tid == 0) mbar_wait_bounded(&sm.full[s], (n >> 1) & 1, kWaitLimitNs, &g_stepq_flags);
+            // more bounded wait for each copy still in flight.
+            if (issuer)
+                for (int i = 0; i + 1 < kStages; ++i)
+                    if (tile + i * gridDim.x < a.num_tiles)
+                        mbar_wait_bounded(&sm.full[(n + i) % kStages], ((n + i) / kStages) & 1, kWaitLimitNs,
+                                          &g_stepq_flags);
             return;
         }
-        // Every thread is past the previous tile: its buffers may be refilled.
-        if (tid == 0) issue_tile<D>(a, sm, n + 1, s ^ 1);
-
-        auto& st = sm.stage[s];
-        const int h = tile % a.H;
-        const int64_t tile_base = static_cast<int64_t>(tile / a.H) * a.bytes_per_seq + a.head_off[h];
-
-        // ---- prologue: per-row constants, width-sorted slots, q.k -----------------------
-        if (tid < D) {
-            const int i = tid;
-            const int bw = st.bits[i];
-            const float g = a.gate_per_channel ? st.gate[i] : __ldg(a.gate + tile);
-            const float alpha = g * half_bits_to_float(st.r[i]) * znorm_of(bw);
-            const float kk = bf16_bits_to_float(st.k[i]);
-            const float qq = bf16_bits_to_float(st.q[i]);
-            sm.rc0[i] = make_float4(alpha, alpha, alpha * kk, alpha * kk);
-            sm.rc1[i] = make_float4(alpha * qq, alpha * qq, kk, kk);
-        } else if (warp == D / 32) {
-            sort_rows_warp<D>(st.bits, sm.meta, lane);
-        } else if (warp == D / 32 + 1) {
-            constexpr int RL = D / 32;
-            float acc = 0.f;
-#pragma unroll
-            for (int r = 0; r < RL; ++r)
-                acc = fmaf(bf16_bits_to_float(st.q[lane * RL + r]), bf16_bits_to_float(st.k[lane * RL + r]), acc);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) sm.qk = acc;
-        }
-        __syncthreads();
+        // Every thread is past the previous tile: its stage may be refilled, kStages-1 ahead.
+        const int ahead = n + kStages - 1, sa = ahead % kStages;
+        bool issued = false;
+        float next_beta = 0.f, next_gate = 0.f;
+        if (issuer) issued = issue_tile<D>(a, sm, blockIdx.x + ahead * gridDim.x, sa, next_beta, next_gate);
 
         // The warp's 16 slots share one width unless the warp straddles a width boundary.
         int ww;
         {
-            const int w0 = (sm.meta[warp * M::kRowsPerWarp] >> 8) & 0xFF;
-            const int w1 = (sm.meta[warp * M::kRowsPerWarp + M::kRowsPerWarp - 1] >> 8) & 0xFF;
+            const int w0 = (meta[warp * M::kRowsPerWarp] >> 8) & 0xFF;
+            const int w1 = (meta[warp * M::kRowsPerWarp + M::kRowsPerWarp - 1] >> 8) & 0xFF;
             ww = (w0 == w1) ? w0 : 0;
         }
 
         // ---- phase 1: unpack, k^T D S and q^T D S (column scale factored out) ----------
-        float2 Z[RPT][2];
-        float2 pacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        float2 oacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        switch (ww) {
-            case 8: phase1_uniform<D, 8>(sm, st.codes, warp, lane, Z, pacc, oacc); break;
-            case 6: phase1_uniform<D, 6>(sm, st.codes, warp, lane, Z, pacc, oacc); break;
-            case 4: phase1_uniform<D, 4>(sm, st.codes, warp, lane, Z, pacc, oacc); break;
-            case 2: phase1_uniform<D, 2>(sm, st.codes, warp, lane, Z, pacc, oacc); break;
-            default: phase1_mixed<D>(sm, st.codes, warp, lane, Z, pacc, oacc); break;
-        }
+        float2 Z[RPT][4];
+        {
+            float2 pacc[4], oacc[4];
 #pragma unroll
-        for (int m = LPR; m < 32; m <<= 1)
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                pacc[q2].x += __shfl_xor_sync(0xffffffffu, pacc[q2].x, m);
-                pacc[q2].y += __shfl_xor_sync(0xffffffffu, pacc[q2].y, m);
-                oacc[q2].x += __shfl_xor_sync(0xffffffffu, oacc[q2].x, m);
-                oacc[q2].y += __shfl_xor_sync(0xffffffffu, oacc[q2].y, m);
+            for (int p = 0; p < 4; ++p) pacc[p] = oacc[p] = make_float2(0.f, 0.f);
+            switch (ww) {
+                case 8: phase1_uniform<D, 8>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
+                case 6: phase1_uniform<D, 6>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
+                case 4: phase1_uniform<D, 4>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
+                case 2: phase1_uniform<D, 2>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
+                default: phase1_mixed<D>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
             }
-        if (lane < LPR) {
-            *reinterpret_cast<float4*>(&sm.red[warp][0][4 * cl]) = make_float4(pacc[0].x, pacc[0].y, pacc[1].x, pacc[1].y);
-            *reinterpret_cast<float4*>(&sm.red[warp][1][4 * cl]) = make_float4(oacc[0].x, oacc[0].y, oacc[1].x, oacc[1].y);
+            store_col_partials<D>(sm.red[warp][0], lane, pacc);
+            store_col_partials<D>(sm.red[warp][1], lane, oacc);
         }
         __syncthreads();
 
@@ -350,8 +455,7 @@ decode_kernel(const DecodeArgs a) {
                 os += sm.red[w][1][j];
             }
             const float cj = half_bits_to_float(st.c[j]);
-            const float beta = __ldg(a.beta + tile);
-            const float u = beta * (bf16_bits_to_float(st.v[j]) - cj * ps);
+            const float u = st.beta * (bf16_bits_to_float(st.v[j]) - cj * ps);
             a.o[static_cast<int64_t>(tile) * D + j] = fmaf(cj, os, sm.qk * u);
             sm.colc[j] = cj;
             sm.colb[j] = u / cj;
@@ -359,29 +463,30 @@ decode_kernel(const DecodeArgs a) {
         __syncthreads();
 
         // ---- phase 3: X = D S + k u^T (divided by c_j), row |.| sums --------------------
-        const float4 c4 = *reinterpret_cast<const float4*>(&sm.colc[4 * cl]);
         {
-            const float4 u4 = *reinterpret_cast<const float4*>(&sm.colb[4 * cl]);
-            const float2 ut01 = make_float2(u4.x, u4.y), ut23 = make_float2(u4.z, u4.w);
+            float2 cf[4], ut[4];
+            load_cols8(sm.colc, cl, cf);
+            load_cols8(sm.colb, cl, ut);
             float part[RPT];
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
-                const int i = sm.meta[M::row(warp, lane, r)] & 0xFF;
-                const float4 c0 = sm.rc0[i], c1 = sm.rc1[i];
-                const float2 al = make_float2(c0.x, c0.y), kk = make_float2(c1.z, c1.w);
-                Z[r][0] = fma2(al, Z[r][0], mul2(kk, ut01));
-                Z[r][1] = fma2(al, Z[r][1], mul2(kk, ut23));
-                float acc = fabsf(Z[r][0].x) * c4.x;
-                acc = fmaf(fabsf(Z[r][0].y), c4.y, acc);
-                acc = fmaf(fabsf(Z[r][1].x), c4.z, acc);
-                part[r] = fmaf(fabsf(Z[r][1].y), c4.w, acc);
+                const float4 c = sm.ak[M::row(warp, lane, r)];
+                const float2 al = make_float2(c.x, c.y), kk = make_float2(c.z, c.w);
+                float acc = 0.f;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    Z[r][p] = fma2(al, Z[r][p], mul2(kk, ut[p]));
+                    acc = fmaf(fabsf(Z[r][p].x), cf[p].x, acc);
+                    acc = fmaf(fabsf(Z[r][p].y), cf[p].y, acc);
+                }
+                part[r] = acc;
             }
             int slot;
             bool owner;
-            const float rsum = row_reduce<D, float>(sm.rowbuf[warp], lane, part, slot, OpAdd());
-            const int sl = reduced_row<D>(warp, lane, slot, owner);   // a slot index here
+            const float rsum = row_reduce<M, float>(sm.rowbuf[warp], lane, part, slot, OpAdd());
+            const int sl = reduced_row<M>(warp, lane, slot, owner);   // a slot index
             if (owner) {
-                const uint32_t mt = sm.meta[sl];
+                const uint32_t mt = meta[sl];
                 const int i = mt & 0xFF, bw = (mt >> 8) & 0xFF;
                 const float wi = st.w[i];
                 const __half rh = scale_to_half(fmaxf(rsum * (1.0f / D), kHalfMinNormal) / wi);
@@ -397,22 +502,24 @@ decode_kernel(const DecodeArgs a) {
 
         // ---- phase 4: xi = X / (c_j r~_i 2^(8-b_i)); column no-clip scale c0 -----------
         {
-            float cmax[4] = {0.f, 0.f, 0.f, 0.f};
+            float2 cmax[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) cmax[p] = make_float2(0.f, 0.f);
             if (ww != 0) {
 #pragma unroll
                 for (int r = 0; r < RPT; ++r) {
                     const float4 q4 = sm.rq[M::row(warp, lane, r)];
                     const float2 e2 = make_float2(q4.x, q4.y);
-                    Z[r][0] = mul2(Z[r][0], e2);
-                    Z[r][1] = mul2(Z[r][1], e2);
-                    cmax[0] = fmaxf(cmax[0], fabsf(Z[r][0].x));
-                    cmax[1] = fmaxf(cmax[1], fabsf(Z[r][0].y));
-                    cmax[2] = fmaxf(cmax[2], fabsf(Z[r][1].x));
-                    cmax[3] = fmaxf(cmax[3], fabsf(Z[r][1].y));
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        Z[r][p] = mul2(Z[r][p], e2);
+                        cmax[p].x = fmaxf(cmax[p].x, fabsf(Z[r][p].x));
+                        cmax[p].y = fmaxf(cmax[p].y, fabsf(Z[r][p].y));
+                    }
                 }
                 const float iq = sm.riq[warp * M::kRowsPerWarp];
 #pragma unroll
-                for (int kx = 0; kx < 4; ++kx) cmax[kx] *= iq;
+                for (int p = 0; p < 4; ++p) cmax[p] = mul2(cmax[p], make_float2(iq, iq));
             } else {
 #pragma unroll
                 for (int r = 0; r < RPT; ++r) {
@@ -420,17 +527,25 @@ decode_kernel(const DecodeArgs a) {
                     const float4 q4 = sm.rq[sl];
                     const float2 e2 = make_float2(q4.x, q4.y);
                     const float iq = sm.riq[sl];
-                    Z[r][0] = mul2(Z[r][0], e2);
-                    Z[r][1] = mul2(Z[r][1], e2);
-                    cmax[0] = fmaxf(cmax[0], fabsf(Z[r][0].x) * iq);
-                    cmax[1] = fmaxf(cmax[1], fabsf(Z[r][0].y) * iq);
-                    cmax[2] = fmaxf(cmax[2], fabsf(Z[r][1].x) * iq);
-                    cmax[3] = fmaxf(cmax[3], fabsf(Z[r][1].y) * iq);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        Z[r][p] = mul2(Z[r][p], e2);
+                        cmax[p].x = fmaxf(cmax[p].x, fabsf(Z[r][p].x) * iq);
+                        cmax[p].y = fmaxf(cmax[p].y, fabsf(Z[r][p].y) * iq);
+                    }
                 }
             }
-            combine_subrows<D, float>(cmax, OpMax());
-            if (lane < LPR)
-                *reinterpret_cast<float4*>(&sm.red[warp][0][4 * cl]) = make_float4(cmax[0], cmax[1], cmax[2], cmax[3]);
+#pragma unroll
+            for (int m = M::LPR; m < 32; m <<= 1)
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    cmax[p].x = fmaxf(cmax[p].x, __shfl_xor_sync(0xffffffffu, cmax[p].x, m));
+                    cmax[p].y = fmaxf(cmax[p].y, __shfl_xor_sync(0xffffffffu, cmax[p].y, m));
+                }
+            if (lane < M::LPR) {
+                *reinterpret_cast<float4*>(&sm.red[warp][0][8 * cl]) = make_float4(cmax[0].x, cmax[0].y, cmax[1].x, cmax[1].y);
+                *reinterpret_cast<float4*>(&sm.red[warp][0][8 * cl + 4]) = make_float4(cmax[2].x, cmax[2].y, cmax[3].x, cmax[3].y);
+            }
         }
         __syncthreads();
         if (tid < D) {
@@ -448,36 +563,26 @@ decode_kernel(const DecodeArgs a) {
 
         // ---- phase 5: codes at (r~, c0); weighted least-squares column update ----------
         {
-            const float4 f4 = *reinterpret_cast<const float4*>(&sm.colb[4 * cl]);
-            const float2 f01 = make_float2(f4.x, f4.y), f23 = make_float2(f4.z, f4.w);
+            float2 f[4];
+            load_cols8(sm.colb, cl, f);
             const float2 mM2 = make_float2(-kRoundMagic, -kRoundMagic);
-            float2 num[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            float2 den[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            float2 num[4], den[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) num[p] = den[p] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
                 const float4 q4 = sm.rq[M::row(warp, lane, r)];
                 const float2 G2 = make_float2(q4.z, q4.w);
-                const float2 z01 = add2(fma2(Z[r][0], f01, M2), mM2);
-                const float2 z23 = add2(fma2(Z[r][1], f23, M2), mM2);
-                const float2 g01 = mul2(G2, z01), g23 = mul2(G2, z23);
-                num[0] = fma2(g01, Z[r][0], num[0]);
-                num[1] = fma2(g23, Z[r][1], num[1]);
-                den[0] = fma2(g01, z01, den[0]);
-                den[1] = fma2(g23, z23, den[1]);
-            }
 #pragma unroll
-            for (int m = LPR; m < 32; m <<= 1)
-#pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2) {
-                    num[q2].x += __shfl_xor_sync(0xffffffffu, num[q2].x, m);
-                    num[q2].y += __shfl_xor_sync(0xffffffffu, num[q2].y, m);
-                    den[q2].x += __shfl_xor_sync(0xffffffffu, den[q2].x, m);
-                    den[q2].y += __shfl_xor_sync(0xffffffffu, den[q2].y, m);
+                for (int p = 0; p < 4; ++p) {
+                    const float2 z0 = add2(fma2(Z[r][p], f[p], M2), mM2);
+                    const float2 gz = mul2(G2, z0);
+                    num[p] = fma2(gz, Z[r][p], num[p]);
+                    den[p] = fma2(gz, z0, den[p]);
                 }
-            if (lane < LPR) {
-                *reinterpret_cast<float4*>(&sm.red[warp][0][4 * cl]) = make_float4(num[0].x, num[0].y, num[1].x, num[1].y);
-                *reinterpret_cast<float4*>(&sm.red[warp][1][4 * cl]) = make_float4(den[0].x, den[0].y, den[1].x, den[1].y);
             }
+            store_col_partials<D>(sm.red[warp][0], lane, num);
+            store_col_partials<D>(sm.red[warp][1], lane, den);
         }
         __syncthreads();
         bool clip = false;
@@ -502,11 +607,15 @@ decode_kernel(const DecodeArgs a) {
 
         // ---- phase 6: final codes at (r~, c~), packed and stored -----------------------
         {
-            const float4 f4 = *reinterpret_cast<const float4*>(&sm.colb[4 * cl]);
-            const float2 f01 = make_float2(f4.x, f4.y), f23 = make_float2(f4.z, f4.w);
+            float2 f[4];
+            load_cols8(sm.colb, cl, f);
             uint8_t* out = a.packed_out + tile_base;
-            if (any_clip) phase6<D, true>(sm, out, warp, lane, ww, Z, f01, f23);
-            else phase6<D, false>(sm, out, warp, lane, ww, Z, f01, f23);
+            if (any_clip) phase6<D, true>(meta, out, warp, lane, ww, Z, f);
+            else phase6<D, false>(meta, out, warp, lane, ww, Z, f);
+        }
+        if (issued) {   // ordered before their use by the barriers of the next tiles
+            sm.stage[sa].beta = next_beta;
+            sm.stage[sa].gate1 = next_gate;
         }
     }
 }
@@ -519,15 +628,17 @@ static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "stepq_decode_step: %s", cudaGetErrorString(e));
         int occ = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D>, Map<D>::kThreads, smem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D>, DMap<D>::kThreads, smem);
         ctas_per_sm = occ > 0 ? occ : 1;
     }
     if (a.num_tiles == 0) return STEPQ_OK;
     int grid = num_sms * ctas_per_sm;
     if (grid > a.num_tiles) grid = a.num_tiles;
-    decode_kernel<D><<<grid, Map<D>::kThreads, smem, stream>>>(a);
+    decode_kernel<D><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
     return check_launch("stepq_decode_step");
 }
 

@@ -1,10 +1,11 @@
 // stepq_device.cuh -- device building blocks shared by the libstepq kernels (sm_100a).
 //
 // Tile mapping (one (sequence, head) state tile of D x D, D = 64 or 128, row = key channel i,
-// column = value channel j): a thread owns 4 adjacent columns (lane % LPR) of RPT rows.
-// LPR = D/4 lanes span one row; a warp covers RPW = 32/LPR rows per instruction; warp w owns
-// the contiguous rows [w*RPT*RPW, (w+1)*RPT*RPW). With D = 128 that is 8 warps x 16 rows and
-// a whole warp on one row at a time, so the bit width (a property of the row) is warp-uniform.
+// column = value channel j): a thread owns CPL adjacent columns (lane % LPR) of RPT rows.
+// LPR = D/CPL lanes span one row; a warp covers RPW = 32/LPR rows per instruction; warp w owns
+// the rows (slots) [w*RPT*RPW, (w+1)*RPT*RPW). The fused decode kernel uses CPL = 8 so that
+// the per-row work (metadata, constants, addresses) is shared by eight elements; the state
+// conversion and comparison kernels use CPL = 4.
 #pragma once
 
 #include <cstdint>
@@ -19,12 +20,13 @@ constexpr float kRoundMagic = 12582912.0f;            // 1.5 * 2^23: x + M round
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;
 constexpr float kTwo23 = 8388608.0f;                  // 2^23
 
-template <int D>
+template <int D, int CPL = 4>
 struct Map {
+    static constexpr int kCols = CPL;
     static constexpr int kThreads = (D == 128) ? 256 : 128;
     static constexpr int kMinBlocks = (D == 128) ? 2 : 4;          // keeps registers <= 128
     static constexpr int kWarps = kThreads / 32;
-    static constexpr int LPR = D / 4;                  // lanes per row
+    static constexpr int LPR = D / CPL;                // lanes per row
     static constexpr int RPW = 32 / LPR;               // rows per warp instruction
     static constexpr int RPT = D / (kWarps * RPW);     // rows per thread
     static constexpr int kRowsPerWarp = RPT * RPW;
@@ -73,35 +75,67 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 bits2(uint32_t a, uint32_t b) { return make_float2(__uint_as_float(a), __uint_as_float(b)); }
 
-template <int D, int BW>
-__device__ __forceinline__ void unpack4(const uint8_t* row, int cl, float2& z01, float2& z23) {
+// Four codes held in registers -> exact floats. lo: the four fields at their canonical bit
+// positions (8-bit: bytes 0..3; 4-bit: nibbles at bits 0, 8, 4, 12; 2-bit: crumbs at 0, 2, 4,
+// 6; 6-bit: the low nibbles as for 4-bit); hi: the high crumbs of a 6-bit row (bits 0..7).
+// Bits outside those positions are ignored.
+template <int BW>
+__device__ __forceinline__ void unpack4r(uint32_t lo, uint32_t hi, float2& z01, float2& z23) {
     constexpr uint32_t F = 0x4B000000u;   // bits of 2^23
     if constexpr (BW == 8) {
-        const uint32_t u = *reinterpret_cast<const uint32_t*>(row + 4 * cl) ^ 0x80808080u;
+        const uint32_t u = lo ^ 0x80808080u;
         const float2 c = make_float2(-(kTwo23 + 128.0f), -(kTwo23 + 128.0f));
         z01 = add2(bits2(__byte_perm(u, F, 0x7650), __byte_perm(u, F, 0x7651)), c);
         z23 = add2(bits2(__byte_perm(u, F, 0x7652), __byte_perm(u, F, 0x7653)), c);
     } else if constexpr (BW == 4) {
-        const uint32_t u = *reinterpret_cast<const uint16_t*>(row + 2 * cl);
-        z01 = fma2(bits2((u & 0x000Fu) ^ (F | 0x0008u), (u & 0x0F00u) ^ (F | 0x0800u)),
+        z01 = fma2(bits2((lo & 0x000Fu) ^ (F | 0x0008u), (lo & 0x0F00u) ^ (F | 0x0800u)),
                    make_float2(1.0f, 0x1p-8f), make_float2(-(kTwo23 + 8.0f), -(0x1p15f + 8.0f)));
-        z23 = fma2(bits2((u & 0x00F0u) ^ (F | 0x0080u), (u & 0xF000u) ^ (F | 0x8000u)),
+        z23 = fma2(bits2((lo & 0x00F0u) ^ (F | 0x0080u), (lo & 0xF000u) ^ (F | 0x8000u)),
                    make_float2(0x1p-4f, 0x1p-12f), make_float2(-(0x1p19f + 8.0f), -(0x1p11f + 8.0f)));
     } else if constexpr (BW == 2) {
-        const uint32_t u = row[cl];
-        z01 = fma2(bits2((u & 0x03u) ^ (F | 0x02u), (u & 0x0Cu) ^ (F | 0x08u)),
+        z01 = fma2(bits2((lo & 0x03u) ^ (F | 0x02u), (lo & 0x0Cu) ^ (F | 0x08u)),
                    make_float2(1.0f, 0x1p-2f), make_float2(-(kTwo23 + 2.0f), -(0x1p21f + 2.0f)));
-        z23 = fma2(bits2((u & 0x30u) ^ (F | 0x20u), (u & 0xC0u) ^ (F | 0x80u)),
+        z23 = fma2(bits2((lo & 0x30u) ^ (F | 0x20u), (lo & 0xC0u) ^ (F | 0x80u)),
                    make_float2(0x1p-4f, 0x1p-6f), make_float2(-(0x1p19f + 2.0f), -(0x1p17f + 2.0f)));
     } else {  // 6: z = lo + 16 (hi - 2), hi = sign-flipped high crumb, both taken exactly
-        const uint32_t lo = *reinterpret_cast<const uint16_t*>(row + 2 * cl);
-        const uint32_t hi = row[D / 2 + cl];
         const float2 h01 = fma2(bits2((hi & 0x03u) ^ (F | 0x02u), (hi & 0x0Cu) ^ (F | 0x08u)),
                                 make_float2(16.0f, 4.0f), make_float2(-142606368.0f, -33587232.0f));
         const float2 h23 = fma2(bits2((hi & 0x30u) ^ (F | 0x20u), (hi & 0xC0u) ^ (F | 0x80u)),
                                 make_float2(1.0f, 0.25f), make_float2(-8912928.0f, -2099232.0f));
         z01 = fma2(bits2((lo & 0x000Fu) | F, (lo & 0x0F00u) | F), make_float2(1.0f, 0x1p-8f), h01);
         z23 = fma2(bits2((lo & 0x00F0u) | F, (lo & 0xF000u) | F), make_float2(0x1p-4f, 0x1p-12f), h23);
+    }
+}
+
+// The CPL = 4 chunk of one row (lane cl owns columns 4cl .. 4cl+3).
+template <int D, int BW>
+__device__ __forceinline__ void unpack4(const uint8_t* row, int cl, float2& z01, float2& z23) {
+    if constexpr (BW == 8) unpack4r<8>(*reinterpret_cast<const uint32_t*>(row + 4 * cl), 0u, z01, z23);
+    else if constexpr (BW == 4) unpack4r<4>(*reinterpret_cast<const uint16_t*>(row + 2 * cl), 0u, z01, z23);
+    else if constexpr (BW == 2) unpack4r<2>(row[cl], 0u, z01, z23);
+    else unpack4r<6>(*reinterpret_cast<const uint16_t*>(row + 2 * cl), row[D / 2 + cl], z01, z23);
+}
+
+// The CPL = 8 chunk of one row (lane cl owns columns 8cl .. 8cl+7): one load per plane.
+template <int D, int BW>
+__device__ __forceinline__ void unpack8(const uint8_t* row, int cl, float2 z[4]) {
+    if constexpr (BW == 8) {
+        const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * cl);
+        unpack4r<8>(w.x, 0u, z[0], z[1]);
+        unpack4r<8>(w.y, 0u, z[2], z[3]);
+    } else if constexpr (BW == 4) {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(row + 4 * cl);
+        unpack4r<4>(u, 0u, z[0], z[1]);
+        unpack4r<4>(u >> 16, 0u, z[2], z[3]);
+    } else if constexpr (BW == 2) {
+        const uint32_t u = *reinterpret_cast<const uint16_t*>(row + 2 * cl);
+        unpack4r<2>(u, 0u, z[0], z[1]);
+        unpack4r<2>(u >> 8, 0u, z[2], z[3]);
+    } else {
+        const uint32_t lo = *reinterpret_cast<const uint32_t*>(row + 4 * cl);
+        const uint32_t hi = *reinterpret_cast<const uint16_t*>(row + D / 2 + 2 * cl);
+        unpack4r<6>(lo, hi, z[0], z[1]);
+        unpack4r<6>(lo >> 16, hi >> 8, z[2], z[3]);
     }
 }
 
@@ -116,10 +150,10 @@ __device__ __forceinline__ uint32_t vmin_s16x2(uint32_t a, uint32_t b) {
     return d;
 }
 
-// Store 4 codes of one row at width BW. zq are the bit patterns of M + q (|q| < 2^15); with
-// CLAMP the codes are first limited to [-q_b, q_b] (two at a time, as 16-bit pairs).
-template <int D, int BW, bool CLAMP>
-__device__ __forceinline__ void pack4(uint8_t* row, int cl, uint32_t zq0, uint32_t zq1, uint32_t zq2, uint32_t zq3) {
+// Bytes q0..q3 from four words holding q in their low 16 bits (e.g. the bits of M + q,
+// |q| < 2^15); with CLAMP the codes are first limited to [-q_b, q_b], two at a time.
+template <int BW, bool CLAMP>
+__device__ __forceinline__ uint32_t gather4(uint32_t zq0, uint32_t zq1, uint32_t zq2, uint32_t zq3) {
     uint32_t p01 = __byte_perm(zq0, zq1, 0x5410);
     uint32_t p23 = __byte_perm(zq2, zq3, 0x5410);
     if constexpr (CLAMP) {
@@ -129,20 +163,49 @@ __device__ __forceinline__ void pack4(uint8_t* row, int cl, uint32_t zq0, uint32
         p01 = vmin_s16x2(vmax_s16x2(p01, lo), hi);
         p23 = vmin_s16x2(vmax_s16x2(p23, lo), hi);
     }
-    const uint32_t t = __byte_perm(p01, p23, 0x6420);   // bytes q0, q1, q2, q3
+    return __byte_perm(p01, p23, 0x6420);
+}
+
+// Packed fields of four codes given as bytes t = q0 | q1 << 8 | q2 << 16 | q3 << 24.
+__device__ __forceinline__ uint32_t nibbles4(uint32_t t) { return (t & 0x0F0Fu) | ((t >> 12) & 0xF0F0u); }   // 16 bits
+__device__ __forceinline__ uint32_t crumbs4(uint32_t t) { return __umulhi((t << 4) & 0x30303030u, 0x10410400u); }  // low byte
+__device__ __forceinline__ uint32_t high_crumbs4(uint32_t t) { return __umulhi(t & 0x30303030u, 0x10410400u); }  // low byte
+
+// Store 4 codes (CPL = 4 chunk) at width BW.
+template <int D, int BW, bool CLAMP>
+__device__ __forceinline__ void pack4(uint8_t* row, int cl, uint32_t zq0, uint32_t zq1, uint32_t zq2, uint32_t zq3) {
+    const uint32_t t = gather4<BW, CLAMP>(zq0, zq1, zq2, zq3);
     if constexpr (BW == 8) {
         *reinterpret_cast<uint32_t*>(row + 4 * cl) = t;
     } else if constexpr (BW == 4) {
-        *reinterpret_cast<uint16_t*>(row + 2 * cl) = static_cast<uint16_t>((t & 0x0F0Fu) | ((t >> 12) & 0xF0F0u));
+        *reinterpret_cast<uint16_t*>(row + 2 * cl) = static_cast<uint16_t>(nibbles4(t));
     } else if constexpr (BW == 2) {
-        row[cl] = static_cast<uint8_t>(__umulhi((t << 4) & 0x30303030u, 0x10410400u));
+        row[cl] = static_cast<uint8_t>(crumbs4(t));
     } else {
-        *reinterpret_cast<uint16_t*>(row + 2 * cl) = static_cast<uint16_t>((t & 0x0F0Fu) | ((t >> 12) & 0xF0F0u));
-        row[D / 2 + cl] = static_cast<uint8_t>(__umulhi(t & 0x30303030u, 0x10410400u));
+        *reinterpret_cast<uint16_t*>(row + 2 * cl) = static_cast<uint16_t>(nibbles4(t));
+        row[D / 2 + cl] = static_cast<uint8_t>(high_crumbs4(t));
     }
 }
 
-// Runtime-width forms (the state conversion kernels; one warp-uniform branch per row).
+// Store 8 codes (CPL = 8 chunk) at width BW: one store per plane.
+template <int D, int BW, bool CLAMP>
+__device__ __forceinline__ void pack8(uint8_t* row, int cl, const uint32_t zq[8]) {
+    const uint32_t t0 = gather4<BW, CLAMP>(zq[0], zq[1], zq[2], zq[3]);
+    const uint32_t t1 = gather4<BW, CLAMP>(zq[4], zq[5], zq[6], zq[7]);
+    if constexpr (BW == 8) {
+        *reinterpret_cast<uint2*>(row + 8 * cl) = make_uint2(t0, t1);
+    } else if constexpr (BW == 4) {
+        *reinterpret_cast<uint32_t*>(row + 4 * cl) = __byte_perm(nibbles4(t0), nibbles4(t1), 0x5410);
+    } else if constexpr (BW == 2) {
+        *reinterpret_cast<uint16_t*>(row + 2 * cl) = static_cast<uint16_t>(__byte_perm(crumbs4(t0), crumbs4(t1), 0x0040));
+    } else {
+        *reinterpret_cast<uint32_t*>(row + 4 * cl) = __byte_perm(nibbles4(t0), nibbles4(t1), 0x5410);
+        *reinterpret_cast<uint16_t*>(row + D / 2 + 2 * cl) =
+            static_cast<uint16_t>(__byte_perm(high_crumbs4(t0), high_crumbs4(t1), 0x0040));
+    }
+}
+
+// Runtime-width CPL = 4 forms (the state conversion kernels; one warp-uniform branch per row).
 template <int D>
 __device__ __forceinline__ void unpack4(const uint8_t* row, int cl, int b, float z[4]) {
     float2 a, c;
@@ -175,9 +238,8 @@ __device__ __forceinline__ void pack4_store(uint8_t* row, int cl, int b, const i
 // buf: per-warp scratch of 32 * (RPT + 1) floats (padded so both passes are conflict-free).
 // ------------------------------------------------------------------------------------------
 
-template <int D, typename T, typename Op>
-__device__ __forceinline__ T row_reduce(T* buf, int lane, const T part[Map<D>::RPT], int& slot, Op op) {
-    using M = Map<D>;
+template <class M, typename T, typename Op>
+__device__ __forceinline__ T row_reduce(T* buf, int lane, const T part[M::RPT], int& slot, Op op) {
     constexpr int RPT = M::RPT;
     constexpr int LPR = M::LPR;
     static_assert(LPR == 2 * RPT, "two lanes per row in the reduction");
@@ -203,11 +265,10 @@ struct OpMax {
     __device__ float operator()(float x, float y) const { return fmaxf(x, y); }
 };
 
-// Row of the value returned by row_reduce to this lane, and whether this lane is the one of
-// the two holders that should act on it.
-template <int D>
+// Row (slot) of the value returned by row_reduce to this lane, and whether this lane is the
+// one of the two holders that should act on it.
+template <class M>
 __device__ __forceinline__ int reduced_row(int warp, int lane, int slot, bool& owner) {
-    using M = Map<D>;
     owner = (lane % M::LPR) < M::RPT;
     return warp * M::kRowsPerWarp + slot * M::RPW + M::sub_row(lane);
 }
@@ -232,13 +293,13 @@ __device__ __forceinline__ void row_offsets_warp(const uint8_t* bits, uint16_t* 
     for (int r = 0; r < RL; ++r) roff[lane * RL + r] = static_cast<uint16_t>(incl - sum + loc[r]);
 }
 
-// Combine the per-thread column partials of the RPW sub-rows of a warp (D = 64 has two).
-template <int D, typename T, typename Op>
-__device__ __forceinline__ void combine_subrows(T v[4], Op op) {
+// Combine the per-thread column partials of the RPW sub-rows of a warp.
+template <class M, typename T, typename Op, int N = 4>
+__device__ __forceinline__ void combine_subrows(T v[N], Op op) {
 #pragma unroll
-    for (int m = Map<D>::LPR; m < 32; m <<= 1)
+    for (int m = M::LPR; m < 32; m <<= 1)
 #pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = op(v[k], __shfl_xor_sync(0xffffffffu, v[k], m));
+        for (int k = 0; k < N; ++k) v[k] = op(v[k], __shfl_xor_sync(0xffffffffu, v[k], m));
 }
 
 // ------------------------------------------------------------------------------------------

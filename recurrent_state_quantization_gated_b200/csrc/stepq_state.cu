@@ -66,8 +66,8 @@ __device__ void fit_tile_regs(TileSmem<D>& sm, const float X[Map<D>::RPT][4], in
         part[r] = (static_cast<double>(fabsf(X[r][0])) + fabsf(X[r][1])) + (static_cast<double>(fabsf(X[r][2])) + fabsf(X[r][3]));
     int slot;
     bool owner;
-    const double rsum = row_reduce<D, double>(sm.rowbuf[warp], lane, part, slot, OpAdd());
-    const int i_red = reduced_row<D>(warp, lane, slot, owner);
+    const double rsum = row_reduce<Map<D>, double>(sm.rowbuf[warp], lane, part, slot, OpAdd());
+    const int i_red = reduced_row<Map<D>>(warp, lane, slot, owner);
     if (owner) {
         const int bw = sm.bits[i_red];
         double m = rsum / D;
@@ -91,7 +91,7 @@ __device__ void fit_tile_regs(TileSmem<D>& sm, const float X[Map<D>::RPT][4], in
 #pragma unroll
         for (int k = 0; k < 4; ++k) cm[k] = fmaxf(cm[k], __fmul_rn(fabsf(X[r][k]), a));
     }
-    combine_subrows<D, float>(cm, OpMax());
+    combine_subrows<Map<D>, float>(cm, OpMax());
     float* redf = reinterpret_cast<float*>(&sm.red[0][0][0]);
     if (lane < M::LPR)
 #pragma unroll
@@ -127,8 +127,8 @@ __device__ void fit_tile_regs(TileSmem<D>& sm, const float X[Map<D>::RPT][4], in
             den[k] += ww * v * v;
         }
     }
-    combine_subrows<D, double>(num, OpAdd());
-    combine_subrows<D, double>(den, OpAdd());
+    combine_subrows<Map<D>, double>(num, OpAdd());
+    combine_subrows<Map<D>, double>(den, OpAdd());
     if (lane < M::LPR)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -300,8 +300,8 @@ __global__ void __launch_bounds__(Map<D>::kThreads) distortion_kernel(const Stat
     }
     int slot;
     bool owner;
-    const double rs = row_reduce<D, double>(sm.rowbuf[warp], lane, part, slot, OpAdd());
-    const int i = reduced_row<D>(warp, lane, slot, owner);
+    const double rs = row_reduce<Map<D>, double>(sm.rowbuf[warp], lane, part, slot, OpAdd());
+    const int i = reduced_row<Map<D>>(warp, lane, slot, owner);
     if (owner) a.scratch[static_cast<int64_t>(tile) * D + i] = rs;
 }
 

@@ -88,6 +88,8 @@ def _check_step(api, wl, bits, w, head_off, bps, st, t, in_place):
     (128, 2, 7, (4, 6, 8), True),       # channel gates
     (64, 3, 3, (2, 4, 6, 8), True),
     (128, 1, 1, (6,), False),           # a single tile
+    (128, 3, 40, (4, 6, 8), False),     # more heads than the kernel's per-head table cache
+    (64, 2, 70, (2, 4, 8), True),
 ])
 def test_decode_teacher_forced(d, B, H, widths, gpc):
     from recurrent_state_quantization_gated_b200 import api
