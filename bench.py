@@ -54,6 +54,34 @@ def parse():
     return ap.parse_args()
 
 
+def kernel_revision() -> str:
+    """First 16 hex digits of the sha256 of the fused kernel's sources."""
+    import hashlib
+    csrc = ROOT / "recurrent_state_quantization_gated_b200" / "csrc"
+    data = (csrc / "stepq_decode.cu").read_bytes() + (csrc / "stepq_device.cuh").read_bytes()
+    return hashlib.sha256(data).hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes (read + write) per launch from the committed ncu capture of the fused kernel,
+    or None when the kernel source has changed since that capture."""
+    p = ROOT / "profiles" / "decode_kernel_gdn_b64_h32_d128.md"
+    if not p.exists():
+        return None
+    text = p.read_text()
+    rev = read = write = None
+    for line in text.splitlines():
+        if "Kernel source revision" in line:
+            rev = line.rsplit(":", 1)[-1].strip()
+        if line.startswith("| dram__bytes_read.sum"):
+            read = float(line.split("|")[2].split()[0]) * 1e6
+        if line.startswith("| dram__bytes_write.sum"):
+            write = float(line.split("|")[2].split()[0]) * 1e6
+    if rev != kernel_revision() or read is None or write is None:
+        return None
+    return read + write
+
+
 def peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -133,17 +161,38 @@ def algorithmic_bytes(layout_bps: int, B: int, H: int, d: int, gate_per_channel:
     return tiles * 2 * (4 * d * d) + small
 
 
-def run_reference(args, wl):
-    """The oracle (plain C, host cores) on a bounded sample of the same workload."""
+def workload_config(wl, bits, kernel: str, world: int) -> dict:
+    return {"workload": wl.name, "kernel": kernel, "B": wl.B, "H": wl.H, "d_k": wl.d, "d_v": wl.d,
+            "bits_mean": float(np.asarray(bits, dtype=np.float64).mean()), "allocation": wl.alloc,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def run_reference(args, wl, budget_s: float = 90.0):
+    """The oracle (plain C, host cores) on a bounded sample of the same workload: every step
+    decodes B' sequences x H heads, B' chosen so the whole run stays within ``budget_s``."""
     import oracle
     from recurrent_state_quantization_gated_b200 import synth
     cores = len(os.sched_getaffinity(0))
-    seqs = list(range(min(wl.B, 8)))
-    S0 = synth.initial_state(wl, seqs)
-    bits = synth.half_bits(wl) if wl.alloc == "half48" else np.full((wl.H, wl.d), wl.nominal_bits, np.uint8)
-    w = np.ones((wl.H, wl.d), dtype=np.float32)
-    r, c = oracle.fit_scales(S0, w, bits, nthreads=cores)
-    packed = oracle.pack_state(S0, bits, r, c, nthreads=cores)
+    # The oracle's own offline calibration of the workload (row impact, distortions on the
+    # initial states, allocation), as the GPU arm does with the CUDA library.
+    bits, w = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl),
+                               synth.initial_state(wl), synth.calib_tokens(wl))
+    if bits is None:
+        bits = synth.half_bits(wl)
+
+    def state(seqs):
+        S0 = synth.initial_state(wl, seqs)
+        r, c = oracle.fit_scales(S0, w, bits, nthreads=cores)
+        return oracle.pack_state(S0, bits, r, c, nthreads=cores), r, c
+
+    probe = list(range(min(wl.B, 2)))
+    packed, r, c = state(probe)
+    t0 = time.perf_counter()
+    oracle.decode_step(synth.tokens(wl, 0, seqs=probe), bits, w, packed, r, c, nthreads=cores)
+    rate = len(probe) * wl.H / (time.perf_counter() - t0)            # tiles per second
+    nseq = int(budget_s * rate / ((args.steps + args.warmup) * wl.H))
+    seqs = list(range(max(1, min(wl.B, nseq))))
+    packed, r, c = state(seqs)
     tiles = len(seqs) * wl.H
     times = []
     for step in range(args.warmup + args.steps):
@@ -156,7 +205,7 @@ def run_reference(args, wl):
     total = sum(times)
     value = tiles * len(times) / total
     sample = f"{len(seqs)} of {wl.B} sequences x {wl.H} heads ({tiles} tiles) per step, {len(times)} timed steps"
-    return dict(value=value, ms_per_step=1e3 * total / len(times), cores=cores, sample=sample)
+    return dict(value=value, ms_per_step=1e3 * total / len(times), cores=cores, sample=sample, bits=bits)
 
 
 def cpu_baseline(wl, bits, seconds):
@@ -197,7 +246,7 @@ def main():
         line = {"metric": METRIC, "value": ref["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ref["ms_per_step"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-                "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "d": wl.d},
+                "config": workload_config(wl, ref["bits"], "quant", args.gpus),
                 "cpu_baseline": {"value": ref["value"], "unit": UNIT, "cores": ref["cores"], "kind": "oracle",
                                  "sample": ref["sample"]},
                 "e2e": {"value": ref["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -343,16 +392,15 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": rounds_warm * R,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.name, "kernel": args.kernel, "B": wl.B, "H": wl.H, "d_k": wl.d, "d_v": wl.d,
-                       "bits_mean": float(bits.astype(np.float64).mean()),
-                       "allocation": wl.alloc, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "config": {**workload_config(wl, bits, args.kernel, world),
                        "l2": f"inputs larger than L2: {R} state replicas stepped round-robin, "
                              f"{R * per_rep / 2**20:.0f} MiB touched per round",
                        "timing": "CUDA graph of one round of launches, CUDA events on the launching stream"},
             "elements_per_s": value * wl.d * wl.d,
             "achieved_gbs": achieved_gbs,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
-                         "frac": achieved_gbs / peak, "peak_kind": peak_kind, "traffic": None,
+                         "frac": achieved_gbs / peak, "peak_kind": peak_kind,
+                         "traffic": profiled_traffic() if (args.kernel == "quant" and args.workload == 1) else None,
                          "bytes_per_launch": bytes_launch,
                          "bytes_per_launch_formula": "2*B*bytes_per_seq + B*H*(2*(2d+2d) + 6d + 4 + gate + 4d)"},
             "gpu_launches": K,
