@@ -96,11 +96,13 @@ struct DecodeSmem {
     // Per head (cached): per slot (rows sorted by width, stable) the row's metadata
     // row | width << 8 | byte offset << 16.
     alignas(16) uint32_t hmeta[CH][D];
+    alignas(16) uint16_t hslot[CH][D];   // by key row: slot | width << 8
     int htag[CH];                   // head held by each cache entry (-1: none)
     // Per slot of the tile being decoded.
     alignas(16) float4 kq[D];       // alpha k, alpha k, alpha q, alpha q   (alpha = g r 2^(8-b))
     alignas(16) float4 ak[D];       // alpha, alpha, k, k
     alignas(16) float4 rq[D];       // e, e, G, G  (e = 1/(r~ 2^(8-b)), G = (w r~ 2^(8-b))^2)
+    alignas(16) float2 wsl[D];      // w, 1/w
     alignas(16) float riq[D];       // 1/q_b
     // Per column.
     alignas(16) float colc[D];      // c_j (old column scale)
@@ -188,6 +190,7 @@ __device__ __forceinline__ void sort_head_warp(const DecodeArgs& a, DecodeSmem<D
             if (c == cls) slot = base_c[c] + excl_c[c] + rank[r];
         const int off = incl - sum + loc[r];
         sm.hmeta[e][slot] = static_cast<uint32_t>(i) | (static_cast<uint32_t>(bw[r]) << 8) | (static_cast<uint32_t>(off) << 16);
+        sm.hslot[e][i] = static_cast<uint16_t>(slot | (bw[r] << 8));
     }
 }
 
@@ -205,15 +208,29 @@ __device__ __forceinline__ void phase1_row(const DecodeSmem<D>& sm, const uint8_
     }
 }
 
+// Width-uniform warp: every row's metadata and code words are loaded first, so the shared
+// memory latencies overlap, then the rows are unpacked and accumulated.
 template <int D, int BW>
 __device__ __forceinline__ void phase1_uniform(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* codes,
                                                int warp, int lane, float2 Z[][4], float2 pacc[4], float2 oacc[4]) {
     using M = DMap<D>;
     const int cl = M::col_lane(lane);
+    uint32_t mt[M::RPT];
+    uint2 raw[M::RPT];
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r) mt[r] = meta[M::row(warp, lane, r)];
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r) raw[r] = load8<D, BW>(codes + (mt[r] >> 16), cl);
 #pragma unroll
     for (int r = 0; r < M::RPT; ++r) {
-        const int s = M::row(warp, lane, r);
-        phase1_row<D, BW>(sm, codes, s, meta[s], cl, Z[r], pacc, oacc);
+        unpack8r<BW>(raw[r], Z[r]);
+        const float4 c = sm.kq[M::row(warp, lane, r)];
+        const float2 kap = make_float2(c.x, c.y), lam = make_float2(c.z, c.w);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            pacc[p] = fma2(kap, Z[r][p], pacc[p]);
+            oacc[p] = fma2(lam, Z[r][p], oacc[p]);
+        }
     }
 }
 
@@ -383,15 +400,17 @@ decode_kernel(const DecodeArgs a) {
         // ---- prologue: per-slot constants of this tile, q.k ------------------------------
         if (ok) {
             if (tid < D) {
-                const int sl = tid;
-                const uint32_t mt = meta[sl];
-                const int i = mt & 0xFF, bw = (mt >> 8) & 0xFF;
+                const int i = tid;
+                const uint32_t sw = sm.hslot[he][i];
+                const int sl = sw & 0xFF, bw = sw >> 8;
                 const float g = a.gate_per_channel ? st.gate[i] : st.gate1;
                 const float alpha = g * half_bits_to_float(st.r[i]) * znorm_of(bw);
                 const float kk = bf16_bits_to_float(st.k[i]);
                 const float qq = bf16_bits_to_float(st.q[i]);
+                const float wi = st.w[i];
                 sm.kq[sl] = make_float4(alpha * kk, alpha * kk, alpha * qq, alpha * qq);
                 sm.ak[sl] = make_float4(alpha, alpha, kk, kk);
+                sm.wsl[sl] = make_float2(wi, rcp_approx(wi));
             } else if (warp == D / 32) {
                 constexpr int RL = D / 32;
                 float acc = 0.f;
@@ -458,7 +477,7 @@ decode_kernel(const DecodeArgs a) {
             const float u = st.beta * (bf16_bits_to_float(st.v[j]) - cj * ps);
             a.o[static_cast<int64_t>(tile) * D + j] = fmaf(cj, os, sm.qk * u);
             sm.colc[j] = cj;
-            sm.colb[j] = u / cj;
+            sm.colb[j] = u * rcp_approx(cj);
         }
         __syncthreads();
 
@@ -488,14 +507,14 @@ decode_kernel(const DecodeArgs a) {
             if (owner) {
                 const uint32_t mt = meta[sl];
                 const int i = mt & 0xFF, bw = (mt >> 8) & 0xFF;
-                const float wi = st.w[i];
-                const __half rh = scale_to_half(fmaxf(rsum * (1.0f / D), kHalfMinNormal) / wi);
+                const float2 w2 = sm.wsl[sl];
+                const __half rh = scale_to_half(fmaxf(rsum * (1.0f / D), kHalfMinNormal) * w2.y);
                 a.r_out[static_cast<int64_t>(tile) * D + i] = __half_as_ushort(rh);
                 const float rs = __half2float(rh) * znorm_of(bw);
-                const float e = __frcp_rn(rs);
-                const float g = wi * rs;
+                const float e = rcp_approx(rs);
+                const float g = w2.x * rs;
                 sm.rq[sl] = make_float4(e, e, g * g, g * g);
-                sm.riq[sl] = __frcp_rn(static_cast<float>(qmax_of(bw)));
+                sm.riq[sl] = inv_qmax_of(bw);
             }
             __syncwarp();
         }
@@ -557,7 +576,7 @@ decode_kernel(const DecodeArgs a) {
             const float c0 = fmaxf(cj * cm, kHalfMinNormal);
             sm.col0[j] = c0;
             sm.colm[j] = cm;
-            sm.colb[j] = cj / c0;
+            sm.colb[j] = cj * rcp_approx(c0);
         }
         __syncthreads();
 
@@ -595,10 +614,10 @@ decode_kernel(const DecodeArgs a) {
                 ds += sm.red[w][1][j];
             }
             const float cj = sm.colc[j];
-            const float c1 = ds > 0.f ? (cj * ns) / ds : sm.col0[j];
+            const float c1 = ds > 0.f ? (cj * ns) * rcp_approx(ds) : sm.col0[j];
             const __half ch = scale_to_half(c1);
             a.c_out[static_cast<int64_t>(tile) * D + j] = __half_as_ushort(ch);
-            const float fq = cj / __half2float(ch);
+            const float fq = cj * rcp_approx(__half2float(ch));
             sm.colb[j] = fq;
             // |t_ij| <= q_b max_i(|xi_ij|/q_b) fq_j: past this margin a code may round beyond q_b.
             clip = sm.colm[j] * fq > 1.0f + 0.4f / 127.0f;

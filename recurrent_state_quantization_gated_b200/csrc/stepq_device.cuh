@@ -43,6 +43,10 @@ struct Map {
 
 __device__ __forceinline__ int qmax_of(int b) { return (1 << (b - 1)) - 1; }
 __device__ __forceinline__ float znorm_of(int b) { return __int_as_float((127 + 8 - b) << 23); }  // 2^(8-b)
+// 1/q_b for b in {2, 4, 6, 8}, correctly rounded.
+__device__ __forceinline__ float inv_qmax_of(int b) {
+    return b == 2 ? 1.0f : b == 4 ? 1.0f / 7.0f : b == 6 ? 1.0f / 31.0f : 1.0f / 127.0f;
+}
 
 // A positive scale to binary16: clamp into [2^-14, 65504] (NaN -> floor), round to nearest even.
 __device__ __forceinline__ __half scale_to_half(float x) {
@@ -137,6 +141,42 @@ __device__ __forceinline__ void unpack8(const uint8_t* row, int cl, float2 z[4])
         unpack4r<6>(lo, hi, z[0], z[1]);
         unpack4r<6>(lo >> 16, hi >> 8, z[2], z[3]);
     }
+}
+
+// The code words of one CPL = 8 row chunk, loaded ahead of unpacking: x / y hold the 8-bit
+// row's two words, the 6-bit row's low plane word and high plane halfword, or the 4- and 2-bit
+// rows' single word (y unused).
+template <int D, int BW>
+__device__ __forceinline__ uint2 load8(const uint8_t* row, int cl) {
+    if constexpr (BW == 8) return *reinterpret_cast<const uint2*>(row + 8 * cl);
+    else if constexpr (BW == 4) return make_uint2(*reinterpret_cast<const uint32_t*>(row + 4 * cl), 0u);
+    else if constexpr (BW == 2) return make_uint2(*reinterpret_cast<const uint16_t*>(row + 2 * cl), 0u);
+    else return make_uint2(*reinterpret_cast<const uint32_t*>(row + 4 * cl),
+                           *reinterpret_cast<const uint16_t*>(row + D / 2 + 2 * cl));
+}
+
+template <int BW>
+__device__ __forceinline__ void unpack8r(uint2 w, float2 z[4]) {
+    if constexpr (BW == 8) {
+        unpack4r<8>(w.x, 0u, z[0], z[1]);
+        unpack4r<8>(w.y, 0u, z[2], z[3]);
+    } else if constexpr (BW == 4) {
+        unpack4r<4>(w.x, 0u, z[0], z[1]);
+        unpack4r<4>(w.x >> 16, 0u, z[2], z[3]);
+    } else if constexpr (BW == 2) {
+        unpack4r<2>(w.x, 0u, z[0], z[1]);
+        unpack4r<2>(w.x >> 8, 0u, z[2], z[3]);
+    } else {
+        unpack4r<6>(w.x, w.y, z[0], z[1]);
+        unpack4r<6>(w.x >> 16, w.y >> 8, z[2], z[3]);
+    }
+}
+
+// Reciprocal by the special-function unit (about one ulp; inputs are normal and positive).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t vmax_s16x2(uint32_t a, uint32_t b) {
