@@ -150,6 +150,29 @@ STEPQ_API int stepq_row_impact(stepq_dims dims, int T, const uint16_t* q, const 
 STEPQ_API int stepq_calib_distortion(stepq_dims dims, const float* S, const float* w, int b, double* d_row,
                            double* d_head, double* scratch, void* stream);
 
+/* Capacity, in float64 entries, of the static work space of stepq_calib_distortion_static:
+   it takes B * H * dk <= STEPQ_STATIC_SCRATCH_ROWS (4 MiB of device memory per device, held
+   by the loaded library). */
+#define STEPQ_STATIC_SCRATCH_ROWS 524288
+
+/* stepq_calib_distortion without the caller's work space, allocating nothing. No counterpart
+   in the paper: it exists for callers that may not allocate device memory when they measure
+   distortion, such as a process whose device memory is already reserved in full (a serving
+   process that sized its pool for the packed states and caches) or one that runs under an
+   allocator which forbids new device allocations after start-up; they cannot hand over the
+   [B][H][dk] work space of stepq_calib_distortion.
+   The work space is a file-scope device array of STEPQ_STATIC_SCRATCH_ROWS float64 entries,
+   one per device. The first call on each device (with that device current) looks up its
+   address with cudaGetSymbolAddress; make that first call before any stream capture. Every
+   entry the call reads it has written itself, so nothing in the array needs clearing.
+   All calls on one device share the array: calls that overlap in time (on different streams,
+   or from different host threads without ordering) race and give wrong results; order them
+   on one stream. Arguments, layout and results are those of stepq_calib_distortion.
+   Returns STEPQ_EINVAL when B * H * dk exceeds STEPQ_STATIC_SCRATCH_ROWS (nothing is
+   launched), STEPQ_ECUDA when the address lookup or a launch fails. */
+STEPQ_API int stepq_calib_distortion_static(stepq_dims dims, const float* S, const float* w, int b,
+                                  double* d_row, double* d_head, void* stream);
+
 /* Host only. Lifetime-aware bit allocation (§3.2, App. C.2): widths bits_out_host[u] from the
    ascending candidates cand_host[0..n_cand) minimising sum_u J_host[u][k] with exactly
    budget_bits bits in total (J is the lifetime-weighted distortion L_u d_u(b)).

@@ -17,7 +17,8 @@ SYMBOLS = (
     "stepq_last_error", "stepq_packed_layout", "stepq_fit_scales", "stepq_pack_state",
     "stepq_unpack_state", "stepq_decode_step", "stepq_decode_step_fp32",
     "stepq_int8_quantize_state", "stepq_decode_step_int8", "stepq_row_impact",
-    "stepq_calib_distortion", "stepq_allocate_bits", "stepq_read_device_flags", "stepq_build_info",
+    "stepq_calib_distortion", "stepq_calib_distortion_static", "stepq_allocate_bits", "stepq_read_device_flags",
+    "stepq_build_info",
 )
 
 
@@ -51,6 +52,7 @@ _SIGNATURES = {
     "stepq_decode_step_int8": ([Dims, P, P, P, P, P, P, P, P, P, P, P], I),
     "stepq_row_impact": ([Dims, I, P, P, P, P, P, P], I),
     "stepq_calib_distortion": ([Dims, P, P, I, P, P, P, P], I),
+    "stepq_calib_distortion_static": ([Dims, P, P, I, P, P, P], I),
     "stepq_allocate_bits": ([I, I, P, P, I64, I, P], I),
     "stepq_read_device_flags": ([P], I),
 }

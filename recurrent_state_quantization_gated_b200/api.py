@@ -21,7 +21,8 @@ from ._lib import Dims, call, lib
 __all__ = [
     "stepq_packed_layout", "stepq_fit_scales", "stepq_pack_state", "stepq_unpack_state",
     "stepq_decode_step", "stepq_decode_step_fp32", "stepq_int8_quantize_state",
-    "stepq_decode_step_int8", "stepq_row_impact", "stepq_calib_distortion", "stepq_allocate_bits",
+    "stepq_decode_step_int8", "stepq_row_impact", "stepq_calib_distortion", "stepq_calib_distortion_static",
+    "stepq_allocate_bits",
     "stepq_read_device_flags", "stepq_build_info",
 ]
 
@@ -165,6 +166,18 @@ def stepq_calib_distortion(S, w, b, d_row=None, d_head=None, scratch=None):
     call("stepq_calib_distortion", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
          ctypes.c_int(int(b)), _ptr(d_row, torch.float64, "d_row"), _ptr(d_head, torch.float64, "d_head"),
          _ptr(scratch, torch.float64, "scratch"), _stream())
+    return d_row, d_head
+
+
+def stepq_calib_distortion_static(S, w, b, d_row=None, d_head=None):
+    """stepq_calib_distortion on the library's static device work space (B*H*d at most
+    STEPQ_STATIC_SCRATCH_ROWS; overlapping calls on one device race)."""
+    B, H, d, _ = S.shape
+    dev = S.device
+    d_row = torch.empty((H, d), dtype=torch.float64, device=dev) if d_row is None else d_row
+    d_head = torch.empty((H,), dtype=torch.float64, device=dev) if d_head is None else d_head
+    call("stepq_calib_distortion_static", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
+         ctypes.c_int(int(b)), _ptr(d_row, torch.float64, "d_row"), _ptr(d_head, torch.float64, "d_head"), _stream())
     return d_row, d_head
 
 

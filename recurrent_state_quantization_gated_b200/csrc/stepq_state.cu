@@ -9,6 +9,8 @@
 // up to the final binary16 rounding.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "stepq_device.cuh"
 #include "stepq_internal.h"
 
@@ -426,4 +428,67 @@ extern "C" int stepq_calib_distortion(stepq_dims dims, const float* S, const flo
         distortion_finish_kernel<64><<<dims.H, 64, 0, st>>>(dims.B, dims.H, scratch, w, d_row, d_head);
     }
     return check_launch("stepq_calib_distortion");
+}
+
+namespace stepq {
+
+// Work space of stepq_calib_distortion_static: the squared error of each (sample state, head,
+// key row), written by the distortion kernel and summed by its finishing kernel. Host code
+// reaches it only through the address cudaGetSymbolAddress returns.
+static __device__ __align__(256) double g_distortion_scratch[STEPQ_STATIC_SCRATCH_ROWS];
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_scratch_mutex;
+static double* g_scratch_addr[kMaxDevices];
+
+// The current device's copy of the work space, looked up on the first call for that device.
+static int static_scratch(const char* fn, double** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "%s: cudaGetDevice: %s", fn, cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return set_error(STEPQ_EUNSUPPORTED, "%s: device ordinal %d", fn, dev);
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_distortion_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return set_error(STEPQ_ECUDA, "%s: cudaGetSymbolAddress: %s", fn, cudaGetErrorString(e));
+        g_scratch_addr[dev] = static_cast<double*>(p);
+    }
+    *out = g_scratch_addr[dev];
+    return STEPQ_OK;
+}
+
+}  // namespace stepq
+
+extern "C" int stepq_calib_distortion_static(stepq_dims dims, const float* S, const float* w, int b, double* d_row,
+                                             double* d_head, void* stream) {
+    const char* fn = "stepq_calib_distortion_static";
+    clear_error();
+    long long tiles;
+    int rc = common_checks(dims, fn, tiles);
+    if (rc) return rc;
+    if (b != 2 && b != 4 && b != 6 && b != 8) return set_error(STEPQ_EUNSUPPORTED, "%s: width %d", fn, b);
+    if (tiles == 0) return set_error(STEPQ_EINVAL, "%s: no sample states (B=0)", fn);
+    if (tiles * dims.dk > STEPQ_STATIC_SCRATCH_ROWS)
+        return set_error(STEPQ_EINVAL, "%s: B*H*dk = %lld exceeds the static work space of %d entries", fn,
+                         tiles * dims.dk, STEPQ_STATIC_SCRATCH_ROWS);
+    rc = check_ptrs(fn, {{"S", S}, {"w", w}, {"d_row", d_row}, {"d_head", d_head}});
+    if (rc) return rc;
+    double* scratch = nullptr;
+    rc = static_scratch(fn, &scratch);
+    if (rc) return rc;
+    StateArgs a{};
+    a.H = dims.H; a.S = S; a.w = w; a.uniform_bits = b; a.scratch = scratch;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dims.dk == 128) {
+        rc = launch_state<128>(fn, distortion_kernel<128>, (int)tiles, a, st);
+        if (rc) return rc;
+        distortion_finish_kernel<128><<<dims.H, 128, 0, st>>>(dims.B, dims.H, scratch, w, d_row, d_head);
+    } else {
+        rc = launch_state<64>(fn, distortion_kernel<64>, (int)tiles, a, st);
+        if (rc) return rc;
+        distortion_finish_kernel<64><<<dims.H, 64, 0, st>>>(dims.B, dims.H, scratch, w, d_row, d_head);
+    }
+    return check_launch(fn);
 }
