@@ -1,19 +1,22 @@
-"""GPU parity of the fused quantized decode step against the oracle, teacher-forced (the oracle
-starts every step from the GPU's packed state): readouts within 1e-3 relative; row scales within
-one binary16 ulp; requantised codes within one step on at most 0.1% of entries; plus in-place
-updates, every bit width, both gate modes, ragged tile counts and degenerate inputs."""
+"""GPU parity of the fused quantized decode step against the oracle. The oracle runs its own
+rollout; at every step the GPU starts from the oracle's packed state and scales (teacher
+forcing), so differences never accumulate: readouts within 1e-3 relative; row scales within
+one binary16 ulp; requantised codes within one step, on at most 0.1% of entries where both
+sides chose the same scales; plus in-place updates, every bit width, both gate modes, ragged
+tile counts and degenerate inputs."""
 import numpy as np
 import pytest
 
 import oracle
 from recurrent_state_quantization_gated_b200 import synth
-from tests.helpers import (assert_codes_close, assert_outputs_close, dev, half_ulps, host_half, tile_codes,
-                           tokens_dev)
+from tests.helpers import compare_decode, dev, host_half, tokens_dev
 
 pytestmark = pytest.mark.gpu
 
 
-def _setup(d, B, H, widths, gate_per_channel, seed):
+def _setup(d, B, H, widths, gate_per_channel, seed, host=True):
+    """Workload, bits, w, layout and the oracle's initial packed state (host arrays, or
+    device tensors with host=False)."""
     import torch
     from recurrent_state_quantization_gated_b200 import api
     wl = synth.workload(2 if gate_per_channel else 1, B=B, H=H, d=d, seed=seed)
@@ -23,63 +26,31 @@ def _setup(d, B, H, widths, gate_per_channel, seed):
     r, c = oracle.fit_scales(S0, w, bits)
     packed = oracle.pack_state(S0, bits, r, c)
     head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
-    state = dict(packed=dev(packed), r=dev(r, torch.float16), c=dev(c, torch.float16))
+    state = dict(packed=packed, r=r, c=c)
+    if not host:
+        state = dict(packed=dev(packed), r=dev(r, torch.float16), c=dev(c, torch.float16))
     return wl, bits, w, head_off, bps, state
 
 
-def _oracle_state_after(tok, bits, w, packed_in, r_in, c_in, d):
-    """The oracle's updated fp32 state X (steps 1-2 of the decode workflow) per tile."""
-    S_hat = oracle.unpack_state(packed_in, bits, r_in, c_in)
-    B, H = S_hat.shape[:2]
-    X = np.zeros_like(S_hat)
-    for b in range(B):
-        for h in range(H):
-            g = tok["gate"][b, h]
-            Xd, _ = oracle.delta_update(S_hat[b, h], synth.bf16_bits_to_f32(tok["q"][b, h]),
-                                        synth.bf16_bits_to_f32(tok["k"][b, h]), synth.bf16_bits_to_f32(tok["v"][b, h]),
-                                        float(tok["beta"][b, h]), g)
-            X[b, h] = Xd.astype(np.float32)
-    return X
-
-
 def _check_step(api, wl, bits, w, head_off, bps, st, t, in_place):
-    """One decode step on the GPU, checked against the oracle started from the same state.
-
-    The readout must agree to 1e-3. The refitted scales agree exactly except where an entry of
-    the updated state sits on a rounding boundary of the intermediate codes (the oracle forms X
-    in float64, the kernel in fp32): the least-squares column update can then move by a few
-    ulps, so scale mismatches are bounded in frequency and size. The final codes are compared
-    where the decision is well defined: the oracle's X quantised with the kernel's scales must
-    give the kernel's codes to within one step on at most 0.1% of entries."""
+    """Step t on both sides from the oracle's state st (host arrays packed, r, c); returns the
+    oracle's next state and the mismatch rates."""
     import torch
     tok = synth.tokens(wl, t)
     td = tokens_dev(tok)
-    packed_in = st["packed"].cpu().numpy()
-    r_in, c_in = host_half(st["r"]), host_half(st["c"])
+    pk, r, c = dev(st["packed"]), dev(st["r"], torch.float16), dev(st["c"], torch.float16)
     if in_place:
         out = api.stepq_decode_step(td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w),
-                                    dev(head_off), bps, st["packed"], st["r"], st["c"], st["packed"], st["r"],
-                                    st["c"])
+                                    dev(head_off), bps, pk, r, c, pk, r, c)
     else:
         out = api.stepq_decode_step(td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w),
-                                    dev(head_off), bps, st["packed"], st["r"], st["c"])
+                                    dev(head_off), bps, pk, r, c)
     torch.cuda.synchronize()
-    p_gpu, r_gpu, c_gpu, o_gpu = out
-    p_ref, r_ref, c_ref, o_ref = oracle.decode_step(tok, bits, w, packed_in, r_in, c_in)
-    assert_outputs_close(o_gpu.cpu().numpy(), o_ref)
-    rg, cg = host_half(r_gpu), host_half(c_gpu)
-    assert half_ulps(rg, r_ref).max() <= 1, "row factors are continuous in X: one ulp at most"
-    rf_g = rg.view(np.float16).astype(np.float64); cf_g = cg.view(np.float16).astype(np.float64)
-    cf_r = c_ref.view(np.float16).astype(np.float64)
-    assert np.max(np.abs(cf_g / cf_r - 1)) < 0.1
-    B, H, d = wl.B, wl.H, wl.d
-    X = _oracle_state_after(tok, bits, w, packed_in, r_in, c_in, d)
-    codes_gpu = tile_codes(p_gpu.cpu().numpy(), bits, d, B)
-    codes_same_scales = np.stack([np.stack([oracle.quantise_tile(X[b, h], bits[h], rg[b, h], cg[b, h])
-                                            for h in range(H)]) for b in range(B)])
-    frac = assert_codes_close(codes_gpu, codes_same_scales)
-    raw = np.abs(codes_gpu - tile_codes(p_ref, bits, d, B))
-    return dict(packed=p_gpu, r=r_gpu, c=c_gpu), frac, (rg != r_ref).mean(), (cg != c_ref).mean(), (raw > 0).mean()
+    p_g, r_g, c_g, o_g = out
+    ref = oracle.decode_step(tok, bits, w, st["packed"], st["r"], st["c"])
+    rates = compare_decode((p_g.cpu().numpy(), host_half(r_g), host_half(c_g), o_g.cpu().numpy()), ref, bits,
+                           wl.d, wl.B)
+    return dict(packed=ref[0], r=ref[1], c=ref[2]), rates
 
 
 @pytest.mark.parametrize("d,B,H,widths,gpc", [
@@ -94,12 +65,13 @@ def _check_step(api, wl, bits, w, head_off, bps, st, t, in_place):
 def test_decode_teacher_forced(d, B, H, widths, gpc):
     from recurrent_state_quantization_gated_b200 import api
     wl, bits, w, head_off, bps, st = _setup(d, B, H, widths, gpc, seed=d + B + H)
-    fracs, rmis, cmis, raws = [], [], [], []
+    rates = []
     for t in range(6):
-        st, frac, rm, cm, raw = _check_step(api, wl, bits, w, head_off, bps, st, t, in_place=(t % 2 == 0))
-        fracs.append(frac); rmis.append(rm); cmis.append(cm); raws.append(raw)
-    assert np.mean(fracs) <= 1e-3 and np.mean(rmis) < 1e-2 and np.mean(cmis) < 1e-2
-    assert np.mean(raws) < 1e-2       # against the oracle's own codes and scales
+        st, r = _check_step(api, wl, bits, w, head_off, bps, st, t, in_place=(t % 2 == 0))
+        rates.append(r)
+    frac, rmis, cmis, raw = np.mean(rates, axis=0)
+    assert frac <= 1e-3 and rmis < 1e-2 and cmis < 1e-2
+    assert raw < 1e-2       # every code, including columns whose scales differ
 
 
 def test_decode_many_tiles_ragged():
@@ -112,7 +84,7 @@ def test_decode_many_tiles_ragged():
 def test_in_place_equals_out_of_place():
     import torch
     from recurrent_state_quantization_gated_b200 import api
-    wl, bits, w, head_off, bps, st = _setup(128, 4, 6, (2, 4, 6, 8), True, seed=21)
+    wl, bits, w, head_off, bps, st = _setup(128, 4, 6, (2, 4, 6, 8), True, seed=21, host=False)
     td = tokens_dev(synth.tokens(wl, 3))
     a = api.stepq_decode_step(td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w), dev(head_off),
                               bps, st["packed"], st["r"], st["c"])
@@ -130,7 +102,7 @@ def test_decode_degenerate_inputs():
     import torch
     from recurrent_state_quantization_gated_b200 import api
     d, B, H = 128, 2, 3
-    wl, bits, w, head_off, bps, st = _setup(d, B, H, (2, 4, 6, 8), False, seed=5)
+    wl, bits, w, head_off, bps, st = _setup(d, B, H, (2, 4, 6, 8), False, seed=5, host=False)
     tok = synth.tokens(wl, 0)
     tok["beta"][:] = 0.0
     tok["gate"][:] = 1.0
@@ -159,7 +131,7 @@ def test_decode_degenerate_inputs():
 
 def test_device_error_word_is_clear_after_decodes():
     from recurrent_state_quantization_gated_b200 import api
-    wl, bits, w, head_off, bps, st = _setup(128, 3, 4, (4, 8), False, seed=2)
+    wl, bits, w, head_off, bps, st = _setup(128, 3, 4, (4, 8), False, seed=2, host=False)
     td = tokens_dev(synth.tokens(wl, 0))
     api.stepq_decode_step(td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w), dev(head_off), bps,
                           st["packed"], st["r"], st["c"])
