@@ -100,8 +100,8 @@ struct DecodeSmem {
     int htag[CH];                   // head held by each cache entry (-1: none)
     // Per slot of the tile being decoded.
     alignas(16) float4 kq[D];       // alpha k, alpha k, alpha q, alpha q   (alpha = g r 2^(8-b))
-    alignas(16) float4 ak[D];       // alpha, alpha, k, k
-    alignas(16) float4 rq[D];       // e, e, G, G  (e = 1/(r~ 2^(8-b)), G = (w r~ 2^(8-b))^2)
+    alignas(16) float4 ak[D];       // k/alpha, k/alpha, alpha, alpha
+    alignas(16) float4 rq[D];       // alpha e, alpha e, G, G  (e = 1/(r~ 2^(8-b)), G = (w r~ 2^(8-b))^2)
     alignas(16) float2 wsl[D];      // w, 1/w
     alignas(16) float riq[D];       // 1/q_b
     // Per column.
@@ -344,9 +344,22 @@ decode_kernel(const DecodeArgs a) {
     // The last thread queues the copies (no prologue work waits on it).
     const bool issuer = (tid == M::kThreads - 1);
 
+    // The first tiles' copies go out before anything else, so the HBM latency overlaps the
+    // per-head table set-up.
+    constexpr int CH = HeadCache<D>::kHeads;
+    if (issuer) {
+        for (int i = 0; i < kStages; ++i) mbar_init(&sm.full[i], 1);
+        fence_barrier_init();
+        for (int i = 0; i + 1 < kStages; ++i) {
+            float b0, g0;
+            if (issue_tile<D>(a, sm, blockIdx.x + i * gridDim.x, i, b0, g0)) {
+                sm.stage[i].beta = b0;
+                sm.stage[i].gate1 = g0;
+            }
+        }
+    }
     // Per-head tables (the bit map is frozen and shared by all sequences): the heads of the
     // CTA's first tiles are sorted up front, one warp per head; the rest on first use.
-    constexpr int CH = HeadCache<D>::kHeads;
     for (int e = tid; e < CH; e += M::kThreads) sm.htag[e] = -1;
     __syncthreads();
     for (int n = warp; n < CH; n += M::kWarps) {
@@ -360,20 +373,6 @@ decode_kernel(const DecodeArgs a) {
         if (take) {
             sort_head_warp<D>(a, sm, h, h % CH, lane);
             if (lane == 0) sm.htag[h % CH] = h;
-        }
-    }
-    if (issuer) {
-        for (int i = 0; i < kStages; ++i) mbar_init(&sm.full[i], 1);
-        fence_barrier_init();
-    }
-    __syncthreads();
-    if (issuer) {
-        for (int i = 0; i + 1 < kStages; ++i) {
-            float b0, g0;
-            if (issue_tile<D>(a, sm, blockIdx.x + i * gridDim.x, i, b0, g0)) {
-                sm.stage[i].beta = b0;
-                sm.stage[i].gate1 = g0;
-            }
         }
     }
     __syncthreads();
@@ -404,12 +403,14 @@ decode_kernel(const DecodeArgs a) {
                 const uint32_t sw = sm.hslot[he][i];
                 const int sl = sw & 0xFF, bw = sw >> 8;
                 const float g = a.gate_per_channel ? st.gate[i] : st.gate1;
-                const float alpha = g * half_bits_to_float(st.r[i]) * znorm_of(bw);
+                // alpha > 0 always (a zero gate leaves 2^-64: far below any term that counts)
+                const float alpha = fmaxf(g * half_bits_to_float(st.r[i]) * znorm_of(bw), 0x1p-64f);
                 const float kk = bf16_bits_to_float(st.k[i]);
                 const float qq = bf16_bits_to_float(st.q[i]);
                 const float wi = st.w[i];
+                const float ka = kk * rcp_approx(alpha);
                 sm.kq[sl] = make_float4(alpha * kk, alpha * kk, alpha * qq, alpha * qq);
-                sm.ak[sl] = make_float4(alpha, alpha, kk, kk);
+                sm.ak[sl] = make_float4(ka, ka, alpha, alpha);
                 sm.wsl[sl] = make_float2(wi, rcp_approx(wi));
             } else if (warp == D / 32) {
                 constexpr int RL = D / 32;
@@ -481,7 +482,8 @@ decode_kernel(const DecodeArgs a) {
         }
         __syncthreads();
 
-        // ---- phase 3: X = D S + k u^T (divided by c_j), row |.| sums --------------------
+        // ---- phase 3: X = D S + k u^T as alpha_i c_j Y_ij, Y = z + (k_i/alpha_i) u_j/c_j;
+        //      row sums of |X| -------------------------------------------------------------
         {
             float2 cf[4], ut[4];
             load_cols8(sm.colc, cl, cf);
@@ -490,11 +492,11 @@ decode_kernel(const DecodeArgs a) {
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
                 const float4 c = sm.ak[M::row(warp, lane, r)];
-                const float2 al = make_float2(c.x, c.y), kk = make_float2(c.z, c.w);
+                const float2 ka = make_float2(c.x, c.y);
                 float acc = 0.f;
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    Z[r][p] = fma2(al, Z[r][p], mul2(kk, ut[p]));
+                    Z[r][p] = fma2(ka, ut[p], Z[r][p]);
                     acc = fmaf(fabsf(Z[r][p].x), cf[p].x, acc);
                     acc = fmaf(fabsf(Z[r][p].y), cf[p].y, acc);
                 }
@@ -508,10 +510,11 @@ decode_kernel(const DecodeArgs a) {
                 const uint32_t mt = meta[sl];
                 const int i = mt & 0xFF, bw = (mt >> 8) & 0xFF;
                 const float2 w2 = sm.wsl[sl];
-                const __half rh = scale_to_half(fmaxf(rsum * (1.0f / D), kHalfMinNormal) * w2.y);
+                const float alpha = sm.ak[sl].z;
+                const __half rh = scale_to_half(fmaxf(alpha * rsum * (1.0f / D), kHalfMinNormal) * w2.y);
                 a.r_out[static_cast<int64_t>(tile) * D + i] = __half_as_ushort(rh);
                 const float rs = __half2float(rh) * znorm_of(bw);
-                const float e = rcp_approx(rs);
+                const float e = alpha * rcp_approx(rs);
                 const float g = w2.x * rs;
                 sm.rq[sl] = make_float4(e, e, g * g, g * g);
                 sm.riq[sl] = inv_qmax_of(bw);
@@ -526,14 +529,16 @@ decode_kernel(const DecodeArgs a) {
             for (int p = 0; p < 4; ++p) cmax[p] = make_float2(0.f, 0.f);
             if (ww != 0) {
 #pragma unroll
-                for (int r = 0; r < RPT; ++r) {
+                for (int r = 0; r < RPT; r += 2) {
                     const float4 q4 = sm.rq[M::row(warp, lane, r)];
-                    const float2 e2 = make_float2(q4.x, q4.y);
+                    const float4 q5 = sm.rq[M::row(warp, lane, r + 1)];
+                    const float2 e2 = make_float2(q4.x, q4.y), e3 = make_float2(q5.x, q5.y);
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
                         Z[r][p] = mul2(Z[r][p], e2);
-                        cmax[p].x = fmaxf(cmax[p].x, fabsf(Z[r][p].x));
-                        cmax[p].y = fmaxf(cmax[p].y, fabsf(Z[r][p].y));
+                        Z[r + 1][p] = mul2(Z[r + 1][p], e3);
+                        cmax[p].x = max_abs3(cmax[p].x, Z[r][p].x, Z[r + 1][p].x);
+                        cmax[p].y = max_abs3(cmax[p].y, Z[r][p].y, Z[r + 1][p].y);
                     }
                 }
                 const float iq = sm.riq[warp * M::kRowsPerWarp];

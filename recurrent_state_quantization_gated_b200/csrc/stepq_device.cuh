@@ -83,32 +83,58 @@ __device__ __forceinline__ float2 bits2(uint32_t a, uint32_t b) { return make_fl
 // positions (8-bit: bytes 0..3; 4-bit: nibbles at bits 0, 8, 4, 12; 2-bit: crumbs at 0, 2, 4,
 // 6; 6-bit: the low nibbles as for 4-bit); hi: the high crumbs of a 6-bit row (bits 0..7).
 // Bits outside those positions are ignored.
+// (a & M) | c in one logic instruction (the compiler's own lowering of this pattern takes two).
+template <uint32_t M>
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(M), "r"(c));
+    return d;
+}
+
+// Sign-bit flips that turn the b-bit two's complement fields of a code word into offset binary
+// (field + 2^(b-1)): applied once per word before the per-field float construction below.
 template <int BW>
-__device__ __forceinline__ void unpack4r(uint32_t lo, uint32_t hi, float2& z01, float2& z23) {
+__device__ __forceinline__ uint32_t flip_signs(uint32_t w) {
+    if constexpr (BW == 8) return w ^ 0x80808080u;
+    else if constexpr (BW == 4) return w ^ 0x88888888u;
+    else return w ^ 0xAAAAAAAAu;   // 2-bit fields, and the high-crumb plane of 6-bit rows
+}
+
+// Four codes as floats (exact small integers): fields of lo (and for b = 6 the high crumbs in
+// hi), both already passed through flip_signs. Each field is masked into the mantissa of 2^23
+// (one logic instruction), then one paired FMA removes the offset and the field's place value.
+template <int BW>
+__device__ __forceinline__ void unpack4f(uint32_t lo, uint32_t hi, float2& z01, float2& z23) {
     constexpr uint32_t F = 0x4B000000u;   // bits of 2^23
     if constexpr (BW == 8) {
-        const uint32_t u = lo ^ 0x80808080u;
         const float2 c = make_float2(-(kTwo23 + 128.0f), -(kTwo23 + 128.0f));
-        z01 = add2(bits2(__byte_perm(u, F, 0x7650), __byte_perm(u, F, 0x7651)), c);
-        z23 = add2(bits2(__byte_perm(u, F, 0x7652), __byte_perm(u, F, 0x7653)), c);
+        z01 = add2(bits2(__byte_perm(lo, F, 0x7650), __byte_perm(lo, F, 0x7651)), c);
+        z23 = add2(bits2(__byte_perm(lo, F, 0x7652), __byte_perm(lo, F, 0x7653)), c);
     } else if constexpr (BW == 4) {
-        z01 = fma2(bits2((lo & 0x000Fu) ^ (F | 0x0008u), (lo & 0x0F00u) ^ (F | 0x0800u)),
+        z01 = fma2(bits2(and_or<0x000Fu>(lo, F), and_or<0x0F00u>(lo, F)),
                    make_float2(1.0f, 0x1p-8f), make_float2(-(kTwo23 + 8.0f), -(0x1p15f + 8.0f)));
-        z23 = fma2(bits2((lo & 0x00F0u) ^ (F | 0x0080u), (lo & 0xF000u) ^ (F | 0x8000u)),
+        z23 = fma2(bits2(and_or<0x00F0u>(lo, F), and_or<0xF000u>(lo, F)),
                    make_float2(0x1p-4f, 0x1p-12f), make_float2(-(0x1p19f + 8.0f), -(0x1p11f + 8.0f)));
     } else if constexpr (BW == 2) {
-        z01 = fma2(bits2((lo & 0x03u) ^ (F | 0x02u), (lo & 0x0Cu) ^ (F | 0x08u)),
+        z01 = fma2(bits2(and_or<0x03u>(lo, F), and_or<0x0Cu>(lo, F)),
                    make_float2(1.0f, 0x1p-2f), make_float2(-(kTwo23 + 2.0f), -(0x1p21f + 2.0f)));
-        z23 = fma2(bits2((lo & 0x30u) ^ (F | 0x20u), (lo & 0xC0u) ^ (F | 0x80u)),
+        z23 = fma2(bits2(and_or<0x30u>(lo, F), and_or<0xC0u>(lo, F)),
                    make_float2(0x1p-4f, 0x1p-6f), make_float2(-(0x1p19f + 2.0f), -(0x1p17f + 2.0f)));
     } else {  // 6: z = lo + 16 (hi - 2), hi = sign-flipped high crumb, both taken exactly
-        const float2 h01 = fma2(bits2((hi & 0x03u) ^ (F | 0x02u), (hi & 0x0Cu) ^ (F | 0x08u)),
+        const float2 h01 = fma2(bits2(and_or<0x03u>(hi, F), and_or<0x0Cu>(hi, F)),
                                 make_float2(16.0f, 4.0f), make_float2(-142606368.0f, -33587232.0f));
-        const float2 h23 = fma2(bits2((hi & 0x30u) ^ (F | 0x20u), (hi & 0xC0u) ^ (F | 0x80u)),
+        const float2 h23 = fma2(bits2(and_or<0x30u>(hi, F), and_or<0xC0u>(hi, F)),
                                 make_float2(1.0f, 0.25f), make_float2(-8912928.0f, -2099232.0f));
-        z01 = fma2(bits2((lo & 0x000Fu) | F, (lo & 0x0F00u) | F), make_float2(1.0f, 0x1p-8f), h01);
-        z23 = fma2(bits2((lo & 0x00F0u) | F, (lo & 0xF000u) | F), make_float2(0x1p-4f, 0x1p-12f), h23);
+        z01 = fma2(bits2(and_or<0x000Fu>(lo, F), and_or<0x0F00u>(lo, F)), make_float2(1.0f, 0x1p-8f), h01);
+        z23 = fma2(bits2(and_or<0x00F0u>(lo, F), and_or<0xF000u>(lo, F)), make_float2(0x1p-4f, 0x1p-12f), h23);
     }
+}
+
+// As unpack4f, from the stored (two's complement) code words.
+template <int BW>
+__device__ __forceinline__ void unpack4r(uint32_t lo, uint32_t hi, float2& z01, float2& z23) {
+    if constexpr (BW == 6) unpack4f<6>(lo, flip_signs<2>(hi), z01, z23);
+    else unpack4f<BW>(flip_signs<BW>(lo), 0u, z01, z23);
 }
 
 // The CPL = 4 chunk of one row (lane cl owns columns 4cl .. 4cl+3).
@@ -118,29 +144,6 @@ __device__ __forceinline__ void unpack4(const uint8_t* row, int cl, float2& z01,
     else if constexpr (BW == 4) unpack4r<4>(*reinterpret_cast<const uint16_t*>(row + 2 * cl), 0u, z01, z23);
     else if constexpr (BW == 2) unpack4r<2>(row[cl], 0u, z01, z23);
     else unpack4r<6>(*reinterpret_cast<const uint16_t*>(row + 2 * cl), row[D / 2 + cl], z01, z23);
-}
-
-// The CPL = 8 chunk of one row (lane cl owns columns 8cl .. 8cl+7): one load per plane.
-template <int D, int BW>
-__device__ __forceinline__ void unpack8(const uint8_t* row, int cl, float2 z[4]) {
-    if constexpr (BW == 8) {
-        const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * cl);
-        unpack4r<8>(w.x, 0u, z[0], z[1]);
-        unpack4r<8>(w.y, 0u, z[2], z[3]);
-    } else if constexpr (BW == 4) {
-        const uint32_t u = *reinterpret_cast<const uint32_t*>(row + 4 * cl);
-        unpack4r<4>(u, 0u, z[0], z[1]);
-        unpack4r<4>(u >> 16, 0u, z[2], z[3]);
-    } else if constexpr (BW == 2) {
-        const uint32_t u = *reinterpret_cast<const uint16_t*>(row + 2 * cl);
-        unpack4r<2>(u, 0u, z[0], z[1]);
-        unpack4r<2>(u >> 8, 0u, z[2], z[3]);
-    } else {
-        const uint32_t lo = *reinterpret_cast<const uint32_t*>(row + 4 * cl);
-        const uint32_t hi = *reinterpret_cast<const uint16_t*>(row + D / 2 + 2 * cl);
-        unpack4r<6>(lo, hi, z[0], z[1]);
-        unpack4r<6>(lo >> 16, hi >> 8, z[2], z[3]);
-    }
 }
 
 // The code words of one CPL = 8 row chunk, loaded ahead of unpacking: x / y hold the 8-bit
@@ -155,21 +158,38 @@ __device__ __forceinline__ uint2 load8(const uint8_t* row, int cl) {
                            *reinterpret_cast<const uint16_t*>(row + D / 2 + 2 * cl));
 }
 
+// The eight codes of a CPL = 8 chunk from its code words (one sign flip per word).
 template <int BW>
 __device__ __forceinline__ void unpack8r(uint2 w, float2 z[4]) {
     if constexpr (BW == 8) {
-        unpack4r<8>(w.x, 0u, z[0], z[1]);
-        unpack4r<8>(w.y, 0u, z[2], z[3]);
+        unpack4f<8>(flip_signs<8>(w.x), 0u, z[0], z[1]);
+        unpack4f<8>(flip_signs<8>(w.y), 0u, z[2], z[3]);
     } else if constexpr (BW == 4) {
-        unpack4r<4>(w.x, 0u, z[0], z[1]);
-        unpack4r<4>(w.x >> 16, 0u, z[2], z[3]);
+        const uint32_t u = flip_signs<4>(w.x);
+        unpack4f<4>(u, 0u, z[0], z[1]);
+        unpack4f<4>(u >> 16, 0u, z[2], z[3]);
     } else if constexpr (BW == 2) {
-        unpack4r<2>(w.x, 0u, z[0], z[1]);
-        unpack4r<2>(w.x >> 8, 0u, z[2], z[3]);
+        const uint32_t u = flip_signs<2>(w.x);
+        unpack4f<2>(u, 0u, z[0], z[1]);
+        unpack4f<2>(u >> 8, 0u, z[2], z[3]);
     } else {
-        unpack4r<6>(w.x, w.y, z[0], z[1]);
-        unpack4r<6>(w.x >> 16, w.y >> 8, z[2], z[3]);
+        const uint32_t h = flip_signs<2>(w.y);
+        unpack4f<6>(w.x, h, z[0], z[1]);
+        unpack4f<6>(w.x >> 16, h >> 8, z[2], z[3]);
     }
+}
+
+// The CPL = 8 chunk of one row (lane cl owns columns 8cl .. 8cl+7): one load per plane.
+template <int D, int BW>
+__device__ __forceinline__ void unpack8(const uint8_t* row, int cl, float2 z[4]) {
+    unpack8r<BW>(load8<D, BW>(row, cl), z);
+}
+
+// max(|a|, |b|, |c|) in one instruction.
+__device__ __forceinline__ float max_abs3(float a, float b, float c) {
+    float d;
+    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 // Reciprocal by the special-function unit (about one ulp; inputs are normal and positive).
@@ -207,7 +227,11 @@ __device__ __forceinline__ uint32_t gather4(uint32_t zq0, uint32_t zq1, uint32_t
 }
 
 // Packed fields of four codes given as bytes t = q0 | q1 << 8 | q2 << 16 | q3 << 24.
-__device__ __forceinline__ uint32_t nibbles4(uint32_t t) { return (t & 0x0F0Fu) | ((t >> 12) & 0xF0F0u); }   // 16 bits
+__device__ __forceinline__ uint32_t nibbles4(uint32_t t) {   // (t & 0x0F0F) | ((t >> 12) & 0xF0F0), 16 bits
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(d) : "r"(t), "r"(t >> 12), "n"(0x0F0F0F0Fu));
+    return d;
+}
 __device__ __forceinline__ uint32_t crumbs4(uint32_t t) { return __umulhi((t << 4) & 0x30303030u, 0x10410400u); }  // low byte
 __device__ __forceinline__ uint32_t high_crumbs4(uint32_t t) { return __umulhi(t & 0x30303030u, 0x10410400u); }  // low byte
 
@@ -375,6 +399,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended for up to hint_ns while the phase is
+// incomplete, so a waiting warp takes few issue slots from the warps that have work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Global -> shared bulk copy completing on `bar`. bytes: multiple of 16; both addresses
 // 16-byte aligned.
 __device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -398,7 +436,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 10000u)) return true;
         if (global_timer_ns() - t0 > limit_ns) break;
     }
     atomicOr(flags, 1u);
