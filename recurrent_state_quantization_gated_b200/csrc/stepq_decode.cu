@@ -108,7 +108,6 @@ struct DecodeSmem {
     alignas(16) float colc[D];      // c_j (old column scale)
     alignas(16) float colb[D];      // per-phase column broadcast
     alignas(16) float col0[D];      // c0_j
-    alignas(16) float colm[D];      // max_i |xi_ij| / q_b
     alignas(16) float red[M::kWarps][2][D];
     alignas(16) float rowbuf[M::kWarps][32 * (M::RPT + 1)];
     alignas(8) uint64_t full[kStages];
@@ -141,6 +140,9 @@ __device__ __forceinline__ bool issue_tile(const DecodeArgs& a, DecodeSmem<D>& s
     gate1 = a.gate_per_channel ? 0.f : __ldg(a.gate + tile);
     return true;
 }
+
+// The n-th tile of this CTA (tiles are dealt round-robin over the persistent CTAs).
+__device__ __forceinline__ int cta_tile(int n) { return blockIdx.x + n * gridDim.x; }
 
 // One warp sorts the rows of head h by bit width (stable) into cache entry e.
 template <int D>
@@ -253,7 +255,9 @@ __device__ __forceinline__ void phase1_mixed(const DecodeSmem<D>& sm, const uint
 }
 
 // ---- phase 6: final codes, packed and stored ------------------------------------------------
-template <int D, int BW, bool CLAMP>
+// Codes are always limited to [-q_b, q_b]: the least-squares column scale is below the no-clip
+// scale in most columns, so the limit is nearly always needed somewhere in a tile.
+template <int D, int BW>
 __device__ __forceinline__ void phase6_row(uint8_t* out, uint32_t mt, int cl, const float2 x[4], const float2 f[4]) {
     const float2 M2 = make_float2(kRoundMagic, kRoundMagic);
     uint32_t zq[8];
@@ -263,19 +267,19 @@ __device__ __forceinline__ void phase6_row(uint8_t* out, uint32_t mt, int cl, co
         zq[2 * p] = __float_as_uint(t.x);
         zq[2 * p + 1] = __float_as_uint(t.y);
     }
-    pack8<D, BW, CLAMP>(out + (mt >> 16), cl, zq);
+    pack8<D, BW, true>(out + (mt >> 16), cl, zq);
 }
 
-template <int D, int BW, bool CLAMP>
+template <int D, int BW>
 __device__ __forceinline__ void phase6_uniform(const uint32_t* meta, uint8_t* out, int warp, int lane,
                                                const float2 Z[][4], const float2 f[4]) {
     using M = DMap<D>;
     const int cl = M::col_lane(lane);
 #pragma unroll
-    for (int r = 0; r < M::RPT; ++r) phase6_row<D, BW, CLAMP>(out, meta[M::row(warp, lane, r)], cl, Z[r], f);
+    for (int r = 0; r < M::RPT; ++r) phase6_row<D, BW>(out, meta[M::row(warp, lane, r)], cl, Z[r], f);
 }
 
-template <int D, bool CLAMP>
+template <int D>
 __device__ __forceinline__ void phase6_mixed(const uint32_t* meta, uint8_t* out, int warp, int lane,
                                              const float2 Z[][4], const float2 f[4]) {
     using M = DMap<D>;
@@ -284,23 +288,23 @@ __device__ __forceinline__ void phase6_mixed(const uint32_t* meta, uint8_t* out,
     for (int r = 0; r < M::RPT; ++r) {
         const uint32_t mt = meta[M::row(warp, lane, r)];
         switch ((mt >> 8) & 0xFF) {
-            case 8: phase6_row<D, 8, CLAMP>(out, mt, cl, Z[r], f); break;
-            case 6: phase6_row<D, 6, CLAMP>(out, mt, cl, Z[r], f); break;
-            case 4: phase6_row<D, 4, CLAMP>(out, mt, cl, Z[r], f); break;
-            default: phase6_row<D, 2, CLAMP>(out, mt, cl, Z[r], f); break;
+            case 8: phase6_row<D, 8>(out, mt, cl, Z[r], f); break;
+            case 6: phase6_row<D, 6>(out, mt, cl, Z[r], f); break;
+            case 4: phase6_row<D, 4>(out, mt, cl, Z[r], f); break;
+            default: phase6_row<D, 2>(out, mt, cl, Z[r], f); break;
         }
     }
 }
 
-template <int D, bool CLAMP>
+template <int D>
 __device__ __forceinline__ void phase6(const uint32_t* meta, uint8_t* out, int warp, int lane, int ww,
                                        const float2 Z[][4], const float2 f[4]) {
     switch (ww) {
-        case 8: phase6_uniform<D, 8, CLAMP>(meta, out, warp, lane, Z, f); break;
-        case 6: phase6_uniform<D, 6, CLAMP>(meta, out, warp, lane, Z, f); break;
-        case 4: phase6_uniform<D, 4, CLAMP>(meta, out, warp, lane, Z, f); break;
-        case 2: phase6_uniform<D, 2, CLAMP>(meta, out, warp, lane, Z, f); break;
-        default: phase6_mixed<D, CLAMP>(meta, out, warp, lane, Z, f); break;
+        case 8: phase6_uniform<D, 8>(meta, out, warp, lane, Z, f); break;
+        case 6: phase6_uniform<D, 6>(meta, out, warp, lane, Z, f); break;
+        case 4: phase6_uniform<D, 4>(meta, out, warp, lane, Z, f); break;
+        case 2: phase6_uniform<D, 2>(meta, out, warp, lane, Z, f); break;
+        default: phase6_mixed<D>(meta, out, warp, lane, Z, f); break;
     }
 }
 
@@ -352,7 +356,7 @@ decode_kernel(const DecodeArgs a) {
         fence_barrier_init();
         for (int i = 0; i + 1 < kStages; ++i) {
             float b0, g0;
-            if (issue_tile<D>(a, sm, blockIdx.x + i * gridDim.x, i, b0, g0)) {
+            if (issue_tile<D>(a, sm, cta_tile(i), i, b0, g0)) {
                 sm.stage[i].beta = b0;
                 sm.stage[i].gate1 = g0;
             }
@@ -363,13 +367,13 @@ decode_kernel(const DecodeArgs a) {
     for (int e = tid; e < CH; e += M::kThreads) sm.htag[e] = -1;
     __syncthreads();
     for (int n = warp; n < CH; n += M::kWarps) {
-        const int tile = blockIdx.x + n * gridDim.x;
+        const int tile = cta_tile(n);
         if (tile >= a.num_tiles) break;
         const int h = tile % a.H;
         // Sort here only if no earlier tile of this CTA uses the same head or the same entry.
         bool take = true;
         for (int m = 0; m < n; ++m)
-            if (((blockIdx.x + m * gridDim.x) % a.H) % CH == h % CH) take = false;
+            if ((cta_tile(m) % a.H) % CH == h % CH) take = false;
         if (take) {
             sort_head_warp<D>(a, sm, h, h % CH, lane);
             if (lane == 0) sm.htag[h % CH] = h;
@@ -378,7 +382,7 @@ decode_kernel(const DecodeArgs a) {
     __syncthreads();
 
     for (int n = 0;; ++n) {
-        const int tile = blockIdx.x + n * gridDim.x;
+        const int tile = cta_tile(n);
         if (tile >= a.num_tiles) break;
         const int s = n % kStages;
         const uint32_t parity = (n / kStages) & 1;
@@ -428,16 +432,16 @@ decode_kernel(const DecodeArgs a) {
             // more bounded wait for each copy still in flight.
             if (issuer)
                 for (int i = 0; i + 1 < kStages; ++i)
-                    if (tile + i * gridDim.x < a.num_tiles)
+                    if (cta_tile(n + i) < a.num_tiles)
                         mbar_wait_bounded(&sm.full[(n + i) % kStages], ((n + i) / kStages) & 1, kWaitLimitNs,
                                           &g_stepq_flags);
             return;
         }
-        // Every thread is past the previous tile: its stage may be refilled, kStages-1 ahead.
+        // Every thread is past the previous tile, so its stage may be refilled kStages-1 ahead;
+        // the copies are queued below while half of the CTA finalises the first reductions.
         const int ahead = n + kStages - 1, sa = ahead % kStages;
         bool issued = false;
         float next_beta = 0.f, next_gate = 0.f;
-        if (issuer) issued = issue_tile<D>(a, sm, blockIdx.x + ahead * gridDim.x, sa, next_beta, next_gate);
 
         // The warp's 16 slots share one width unless the warp straddles a width boundary.
         int ww;
@@ -479,6 +483,8 @@ decode_kernel(const DecodeArgs a) {
             a.o[static_cast<int64_t>(tile) * D + j] = fmaf(cj, os, sm.qk * u);
             sm.colc[j] = cj;
             sm.colb[j] = u * rcp_approx(cj);
+        } else if (issuer) {
+            issued = issue_tile<D>(a, sm, cta_tile(ahead), sa, next_beta, next_gate);
         }
         __syncthreads();
 
@@ -580,7 +586,6 @@ decode_kernel(const DecodeArgs a) {
             const float cj = sm.colc[j];
             const float c0 = fmaxf(cj * cm, kHalfMinNormal);
             sm.col0[j] = c0;
-            sm.colm[j] = cm;
             sm.colb[j] = cj * rcp_approx(c0);
         }
         __syncthreads();
@@ -609,7 +614,6 @@ decode_kernel(const DecodeArgs a) {
             store_col_partials<D>(sm.red[warp][1], lane, den);
         }
         __syncthreads();
-        bool clip = false;
         if (tid < D) {
             const int j = tid;
             float ns = 0.f, ds = 0.f;
@@ -622,20 +626,15 @@ decode_kernel(const DecodeArgs a) {
             const float c1 = ds > 0.f ? (cj * ns) * rcp_approx(ds) : sm.col0[j];
             const __half ch = scale_to_half(c1);
             a.c_out[static_cast<int64_t>(tile) * D + j] = __half_as_ushort(ch);
-            const float fq = cj * rcp_approx(__half2float(ch));
-            sm.colb[j] = fq;
-            // |t_ij| <= q_b max_i(|xi_ij|/q_b) fq_j: past this margin a code may round beyond q_b.
-            clip = sm.colm[j] * fq > 1.0f + 0.4f / 127.0f;
+            sm.colb[j] = cj * rcp_approx(__half2float(ch));
         }
-        const bool any_clip = __syncthreads_or(clip);
+        __syncthreads();
 
         // ---- phase 6: final codes at (r~, c~), packed and stored -----------------------
         {
             float2 f[4];
             load_cols8(sm.colb, cl, f);
-            uint8_t* out = a.packed_out + tile_base;
-            if (any_clip) phase6<D, true>(meta, out, warp, lane, ww, Z, f);
-            else phase6<D, false>(meta, out, warp, lane, ww, Z, f);
+            phase6<D>(meta, a.packed_out + tile_base, warp, lane, ww, Z, f);
         }
         if (issued) {   // ordered before their use by the barriers of the next tiles
             sm.stage[sa].beta = next_beta;
