@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--replicas", type=int, default=0, help="state replicas cycled (0 = enough to exceed L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-threads", type=int, default=0, help="oracle threads for cpu_baseline (0 = all cores)")
     ap.add_argument("--kernel", choices=["quant", "fp32", "int8"], default="quant")
     ap.add_argument("--e2e-steps", type=int, default=400)
     return ap.parse_args()
@@ -82,12 +83,42 @@ def profiled_traffic():
     return read + write
 
 
+def profiled_instructions():
+    """Lane instructions per state element of the fused kernel, from the committed ncu capture
+    (warp instructions x 32 / elements), or None when the kernel has changed since."""
+    p = ROOT / "profiles" / "decode_kernel_gdn_b64_h32_d128.md"
+    if not p.exists():
+        return None
+    rev = per_elem = None
+    for line in p.read_text().splitlines():
+        if "Kernel source revision" in line:
+            rev = line.rsplit(":", 1)[-1].strip()
+        if line.startswith("| smsp__inst_executed.sum"):
+            cell = line.split("|")[2]
+            per_elem = float(cell.split("(")[1].split()[0])
+    return per_elem if rev == kernel_revision() else None
+
+
 def peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
         d = json.loads(p.read_text())
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def alu_roofline(elements_per_s, clocks):
+    """The issue-rate roofline beside the HBM one: lane instructions per second against
+    148 SMs x 4 schedulers x 32 lanes x the SM clock seen during the timed region."""
+    per_elem = profiled_instructions()
+    mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    peak = 148 * 4 * 32 * mhz * 1e6
+    if per_elem is None:
+        return {"bound": "alu", "achieved": None, "peak": peak, "unit": "lane-instr/s", "frac": None,
+                "instr_per_element": None}
+    achieved = per_elem * elements_per_s
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "lane-instr/s", "frac": achieved / peak,
+            "instr_per_element": per_elem}
 
 
 class ClockSampler:
@@ -121,6 +152,12 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        if getattr(self, "_summary", None) is not None:
+            return self._summary
+        self._summary = self._read()
+        return self._summary
+
+    def _read(self):
         if self.tmp is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         rows = []
@@ -208,27 +245,29 @@ def run_reference(args, wl, budget_s: float = 90.0):
     return dict(value=value, ms_per_step=1e3 * total / len(times), cores=cores, sample=sample, bits=bits)
 
 
-def cpu_baseline(wl, bits, seconds):
+def cpu_baseline(wl, bits, seconds, threads=0):
+    """The oracle as it stands, timed on the host cores over a bounded sample of the workload:
+    16 sequences x all heads per step, inputs drawn before the timed loop."""
     import oracle
     from recurrent_state_quantization_gated_b200 import synth
-    cores = len(os.sched_getaffinity(0))
+    cores = threads if threads > 0 else len(os.sched_getaffinity(0))
     seqs = list(range(min(wl.B, 16)))
     S0 = synth.initial_state(wl, seqs)
     w = np.ones((wl.H, wl.d), dtype=np.float32)
     r, c = oracle.fit_scales(S0, w, bits, nthreads=cores)
     packed = oracle.pack_state(S0, bits, r, c, nthreads=cores)
+    toks = [synth.tokens(wl, t, seqs=seqs) for t in range(8)]
     tiles = len(seqs) * wl.H
     steps, t0 = 0, time.perf_counter()
     while True:
-        tok = synth.tokens(wl, steps % wl.T, seqs=seqs)
-        packed, r, c, _ = oracle.decode_step(tok, bits, w, packed, r, c, nthreads=cores)
+        packed, r, c, _ = oracle.decode_step(toks[steps % len(toks)], bits, w, packed, r, c, nthreads=cores)
         steps += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             break
     return {"value": tiles * steps / el, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{steps} decode steps of {len(seqs)} sequences x {wl.H} heads ({tiles} tiles), "
-                      f"OpenMP over tiles, {el:.1f} s"}
+                      f"{'OpenMP over tiles' if cores > 1 else 'one thread'}, {el:.1f} s"}
 
 
 def main():
@@ -359,25 +398,43 @@ def main():
     for tk in host_tok:
         pinned.append({k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16) if v.dtype == np.uint16 else
                                            np.ascontiguousarray(v)).pin_memory() for k, v in tk.items()})
-    o_host = torch.empty((wl.B, wl.H, wl.d), dtype=torch.float32).pin_memory()
+    o_host = [torch.empty((wl.B, wl.H, wl.d), dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in pinned[0].values())
-    d2h = o_host.numel() * o_host.element_size()
+    d2h = o_host[0].numel() * o_host[0].element_size()
     n_e2e = max(R, (args.e2e_steps // R) * R)
+    # Three streams: inputs in, decode, readout out. Step s's copies overlap the decode of
+    # step s-1; buffers are reused R steps later, ordered by events.
+    cs, ds = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_h = [torch.cuda.Event() for _ in range(R)]
+    ev_k = [torch.cuda.Event() for _ in range(R)]
+    ev_d = [torch.cuda.Event() for _ in range(R)]
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for s in range(n_e2e):
-            i = s % R
-            src = pinned[s % len(pinned)]
+    e0.record(cs)
+    for s_ in range(n_e2e):
+        i = s_ % R
+        src = pinned[s_ % len(pinned)]
+        with torch.cuda.stream(cs):
+            if s_ >= R:
+                cs.wait_event(ev_k[i])          # the decode that last read toks[i] is done
             for name in ("q", "k", "v"):
                 toks[i][name].view(torch.int16).copy_(src[name], non_blocking=True)
             toks[i]["beta"].copy_(src["beta"], non_blocking=True)
             toks[i]["gate"].copy_(src["gate"], non_blocking=True)
+            ev_h[i].record(cs)
+        with torch.cuda.stream(stream):
+            stream.wait_event(ev_h[i])
+            if s_ >= R:
+                stream.wait_event(ev_d[i])      # outs[i] has been read back
             launch(i)
-            o_host.copy_(outs[i], non_blocking=True)
-        e1.record(stream)
-    stream.synchronize()
+            ev_k[i].record(stream)
+        with torch.cuda.stream(ds):
+            ds.wait_event(ev_k[i])
+            o_host[s_ % 2].copy_(outs[i], non_blocking=True)
+            ev_d[i].record(ds)
+    e1.record(ds)
+    ds.synchronize()
+    torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1)
     if world > 1:
@@ -388,13 +445,16 @@ def main():
 
     line = None
     if rank == 0:
+        clocks = clk.summary()
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": rounds_warm * R,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
             "config": {**workload_config(wl, bits, args.kernel, world),
-                       "l2": f"inputs larger than L2: {R} state replicas stepped round-robin, "
-                             f"{R * per_rep / 2**20:.0f} MiB touched per round",
+                       "l2": (f"inputs larger than L2: {R} state replicas stepped round-robin, "
+                              f"{R * per_rep / 2**20:.0f} MiB touched per round") if R * per_rep > L2_BYTES else
+                             (f"inputs in L2 (latency case): {R} state replicas, "
+                              f"{R * per_rep / 2**20:.1f} MiB touched per round"),
                        "timing": "CUDA graph of one round of launches, CUDA events on the launching stream"},
             "elements_per_s": value * wl.d * wl.d,
             "achieved_gbs": achieved_gbs,
@@ -403,11 +463,13 @@ def main():
                          "traffic": profiled_traffic() if (args.kernel == "quant" and args.workload == 1) else None,
                          "bytes_per_launch": bytes_launch,
                          "bytes_per_launch_formula": "2*B*bytes_per_seq + B*H*(2*(2d+2d) + 6d + 4 + gate + 4d)"},
+            "alu_roofline": alu_roofline(value * wl.d * wl.d, clocks)
+            if (args.kernel == "quant" and args.workload == 1) else None,
             "gpu_launches": K,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": n_e2e},
             "device_flags": flags,
-            "clocks": clk.summary(),
+            "clocks": clocks,
         }
     if world > 1:
         graph = None
@@ -415,7 +477,7 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         if not args.no_cpu_baseline and world == 1 and args.kernel == "quant":
-            line["cpu_baseline"] = cpu_baseline(wl, bits, args.cpu_seconds)
+            line["cpu_baseline"] = cpu_baseline(wl, bits, args.cpu_seconds, args.cpu_threads)
         else:
             line["cpu_baseline"] = None
         print(json.dumps(line), flush=True)
