@@ -198,6 +198,23 @@ def algorithmic_bytes(layout_bps: int, B: int, H: int, d: int, gate_per_channel:
     return tiles * 2 * (4 * d * d) + small
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank takes part (same collective in the same order)."""
+    if world == 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tiles_per_rank: int, steps: int, ms: float) -> float:
+    """Tile updates per second of the whole job: every rank steps its own replica of the
+    workload (no data-path exchange), timed by the slowest rank."""
+    return world * tiles_per_rank * steps / (ms * 1e-3)
+
+
 def workload_config(wl, bits, kernel: str, world: int) -> dict:
     return {"workload": wl.name, "kernel": kernel, "B": wl.B, "H": wl.H, "d_k": wl.d, "d_v": wl.d,
             "bits_mean": float(np.asarray(bits, dtype=np.float64).mean()), "allocation": wl.alloc,
@@ -382,13 +399,9 @@ def main():
             ev1.record(stream)
         stream.synchronize()
         barrier()
-    elapsed_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world, "cuda")
     ms_per_step = elapsed_ms / K
-    value = world * tiles * K / (elapsed_ms * 1e-3)
+    value = job_throughput(world, tiles, K, elapsed_ms)
     achieved_gbs = bytes_launch / (ms_per_step * 1e-3) / 1e9
     peak, peak_kind = peaks()
 
@@ -436,12 +449,8 @@ def main():
     ds.synchronize()
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * tiles * n_e2e / (e2e_ms * 1e-3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
+    e2e_value = job_throughput(world, tiles, n_e2e, e2e_ms)
 
     line = None
     if rank == 0:
