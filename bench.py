@@ -50,7 +50,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--cpu-threads", type=int, default=0, help="oracle threads for cpu_baseline (0 = all cores)")
-    ap.add_argument("--kernel", choices=["quant", "fp32", "int8"], default="quant")
+    ap.add_argument("--kernel", choices=["quant", "split", "fp32", "int8"], default="quant",
+                    help="quant: the fused step; split: the split-form ablation; fp32 / int8: comparison states")
     ap.add_argument("--e2e-steps", type=int, default=400)
     return ap.parse_args()
 
@@ -193,6 +194,8 @@ def algorithmic_bytes(layout_bps: int, B: int, H: int, d: int, gate_per_channel:
     small = tiles * (qkv + 4 + gate + 4 * d)
     if kernel == "quant":
         return 2 * B * layout_bps + tiles * 2 * (2 * d + 2 * d) + small
+    if kernel == "split":   # the fused step's bytes + X written, read by the fit, read by the pack + r, c re-read
+        return 2 * B * layout_bps + tiles * 2 * (2 * d + 2 * d) + small + tiles * (3 * 4 * d * d + 4 * d)
     if kernel == "int8":
         return tiles * 2 * (d * d + 2 * d) + small
     return tiles * 2 * (4 * d * d) + small
@@ -346,8 +349,10 @@ def main():
     R = args.replicas or max(2, int(np.ceil(2 * L2_BYTES / per_rep)))
     R = min(R, 64)
     reps, toks, outs = [], [], []
+    side = torch.cuda.Stream() if args.kernel == "split" else None
+    x_ws = torch.empty((wl.B, wl.H, wl.d, wl.d), dtype=torch.float32, device="cuda") if side is not None else None
     for i in range(R):
-        if args.kernel == "quant":
+        if args.kernel in ("quant", "split"):
             reps.append(dict(packed=base.packed.clone(), r=base.r.clone(), c=base.c.clone()))
         elif args.kernel == "fp32":
             reps.append(dict(S=S0.clone()))
@@ -359,9 +364,15 @@ def main():
     del S0
     torch.cuda.synchronize()
 
-    def launch(i):
+    def launch(i, refit=True):
         st, tk, o = reps[i], toks[i], outs[i]
-        if args.kernel == "quant":
+        if args.kernel == "split":
+            api.stepq_decode_step_split(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
+                                        layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
+                                        st["packed"], st["r"], st["c"], o, x_ws, side_stream=side, refit=refit)
+            if refit:
+                torch.cuda.current_stream().wait_stream(side)   # writeback done before the next step
+        elif args.kernel == "quant":
             api.stepq_decode_step(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
                                   layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
                                   st["packed"], st["r"], st["c"], o)
@@ -404,6 +415,26 @@ def main():
     value = job_throughput(world, tiles, K, elapsed_ms)
     achieved_gbs = bytes_launch / (ms_per_step * 1e-3) / 1e9
     peak, peak_kind = peaks()
+
+    split_info = None
+    if args.kernel == "split":
+        # The first kernel alone (o available, X written): the split form's critical path when
+        # the refit and pack are hidden behind other work.
+        n1 = 10 * R
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            f0.record(stream)
+            for s_ in range(n1):
+                launch(s_ % R, refit=False)
+            f1.record(stream)
+        stream.synchronize()
+        ms1 = f0.elapsed_time(f1) / n1
+        bytes1 = (wl.B * layout.bytes_per_seq + tiles * 4 * wl.d + tiles * 4 * wl.d * wl.d
+                  + tiles * (3 * 2 * wl.d + 4 + (4 * wl.d if wl.gate_per_channel else 4) + 4 * wl.d))
+        split_info = {"first_kernel_ms": ms1, "first_kernel_gbs": bytes1 / (ms1 * 1e-3) / 1e9,
+                      "first_kernel_bytes": bytes1,
+                      "fused_bytes_per_step": algorithmic_bytes(layout.bytes_per_seq, wl.B, wl.H, wl.d,
+                                                                wl.gate_per_channel, "quant")}
 
     # ---- end to end through the public API with host buffers (H2D inputs, D2H output) ----
     host_tok = [synth.tokens(wl, t % wl.T) for t in range(8)]
@@ -478,6 +509,7 @@ def main():
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": n_e2e},
             "device_flags": flags,
+            "split": split_info,
             "clocks": clocks,
         }
     if world > 1:

@@ -116,6 +116,26 @@ STEPQ_API int stepq_decode_step(stepq_dims dims, const uint16_t* q, const uint16
                       const uint16_t* r_in, const uint16_t* c_in, uint8_t* packed_out,
                       uint16_t* r_out, uint16_t* c_out, float* o, void* stream);
 
+/* The split form of the same step (STEPQuant §4.4 and App. F.1: reconstruction, the update and
+   the readout fused; scale fitting and packed writeback run afterwards on a separate stream),
+   kept as an ablation of the single fused kernel:
+     on `stream`: one kernel does steps 1-3 of stepq_decode_step and writes o and the updated
+       state X (float32 [B][H][dk][dv]) into the caller's work space x_ws (64 KiB per tile at
+       d = 128);
+     on `side_stream`, ordered after that kernel by an event the library records on `stream`:
+       stepq_fit_scales(x_ws) -> r_out, c_out and stepq_pack_state(x_ws) -> packed_out.
+   The results equal the fused step's within its stated tolerance (o identically). The side
+   stream's work must complete before anything reads packed_out, r_out, c_out or reuses x_ws:
+   the caller orders that (e.g. an event recorded on side_stream after this call). Passing
+   packed_out, r_out and c_out all NULL runs the first kernel only (o and X). In-place use as
+   for stepq_decode_step. The library keeps one event per device, created on the first call. */
+STEPQ_API int stepq_decode_step_split(stepq_dims dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                            const float* beta, const float* gate, const uint8_t* bits, const float* w,
+                            const int64_t* head_off, int64_t bytes_per_seq, const uint8_t* packed_in,
+                            const uint16_t* r_in, const uint16_t* c_in, uint8_t* packed_out,
+                            uint16_t* r_out, uint16_t* c_out, float* o, float* x_ws, void* stream,
+                            void* side_stream);
+
 /* FP32-state decode step (the unquantised state of §5.1): S_out = D S + beta k (v^T - k^T D S),
    o = S_out^T q. S_out may equal S_in. */
 STEPQ_API int stepq_decode_step_fp32(stepq_dims dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,

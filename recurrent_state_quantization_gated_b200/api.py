@@ -20,7 +20,7 @@ from ._lib import Dims, call, lib
 
 __all__ = [
     "stepq_packed_layout", "stepq_fit_scales", "stepq_pack_state", "stepq_unpack_state",
-    "stepq_decode_step", "stepq_decode_step_fp32", "stepq_int8_quantize_state",
+    "stepq_decode_step", "stepq_decode_step_split", "stepq_decode_step_fp32", "stepq_int8_quantize_state",
     "stepq_decode_step_int8", "stepq_row_impact", "stepq_calib_distortion", "stepq_calib_distortion_static",
     "stepq_allocate_bits",
     "stepq_read_device_flags", "stepq_build_info",
@@ -108,6 +108,37 @@ def stepq_decode_step(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, pac
          _ptr(packed_out, torch.uint8, "packed_out"), _ptr(r_out, torch.float16, "r_out"),
          _ptr(c_out, torch.float16, "c_out"), _ptr(o, torch.float32, "o"), _stream())
     return packed_out, r_out, c_out, o
+
+
+def stepq_decode_step_split(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
+                            packed_out=None, r_out=None, c_out=None, o=None, x_ws=None, side_stream=None,
+                            refit=True):
+    """The split form: the first kernel (o, X) on the current stream, refit and pack on
+    side_stream after it; the current stream then waits for the side stream unless the caller
+    passes its own side_stream (and orders it). refit=False runs the first kernel only.
+    Returns (packed_out, r_out, c_out, o, x_ws)."""
+    B, H, d = q.shape
+    gpc = 1 if gate.dim() == 3 else 0
+    o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
+    x_ws = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device) if x_ws is None else x_ws
+    if refit:
+        packed_out = torch.empty_like(packed_in) if packed_out is None else packed_out
+        r_out = torch.empty_like(r_in) if r_out is None else r_out
+        c_out = torch.empty_like(c_in) if c_out is None else c_out
+    own = side_stream is None and refit
+    side = torch.cuda.Stream() if own else side_stream
+    opt = lambda t, dt, n: _ptr(t, dt, n) if t is not None else None
+    call("stepq_decode_step_split", _dims(B, H, d, gpc), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+         _ptr(v, torch.bfloat16, "v"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
+         _ptr(bits, torch.uint8, "bits"), _ptr(w, torch.float32, "w"), _ptr(head_off, torch.int64, "head_off"),
+         ctypes.c_int64(int(bytes_per_seq)), _ptr(packed_in, torch.uint8, "packed_in"),
+         _ptr(r_in, torch.float16, "r_in"), _ptr(c_in, torch.float16, "c_in"),
+         opt(packed_out, torch.uint8, "packed_out"), opt(r_out, torch.float16, "r_out"),
+         opt(c_out, torch.float16, "c_out"), _ptr(o, torch.float32, "o"), _ptr(x_ws, torch.float32, "x_ws"),
+         _stream(), ctypes.c_void_p(side.cuda_stream if side is not None else 0))
+    if own:
+        torch.cuda.current_stream().wait_stream(side)
+    return packed_out, r_out, c_out, o, x_ws
 
 
 def stepq_decode_step_fp32(q, k, v, beta, gate, S_in, S_out=None, o=None):

@@ -20,6 +20,8 @@
 // contraction).
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "stepq_device.cuh"
 #include "stepq_internal.h"
 
@@ -46,6 +48,7 @@ struct DecodeArgs {
     uint16_t* r_out;
     uint16_t* c_out;
     float* o;
+    float* x_out;   // split form only: the updated state X [B][H][dk][dv] before requantisation
 };
 
 // Mapping of a tile onto one CTA: a thread owns 8 adjacent columns of RPT rows; LPR lanes span
@@ -333,7 +336,10 @@ __device__ __forceinline__ void load_cols8(const float* src, int cl, float2 out[
     out[3] = make_float2(b.z, b.w);
 }
 
-template <int D>
+// kSplit: the first kernel of the split form. It reconstructs, updates and reads out like the
+// fused step, then writes the updated state X in fp32 and stops; the refit and the pack run
+// as separate kernels (stepq_decode_step_split).
+template <int D, bool kSplit = false>
 __global__ void __launch_bounds__(DMap<D>::kThreads, DMap<D>::kMinBlocks)
 decode_kernel(const DecodeArgs a) {
     using M = DMap<D>;
@@ -494,6 +500,28 @@ decode_kernel(const DecodeArgs a) {
             float2 cf[4], ut[4];
             load_cols8(sm.colc, cl, cf);
             load_cols8(sm.colb, cl, ut);
+            if constexpr (kSplit) {
+                // X_ij = alpha_i c_j Y_ij, written row by row in natural key order.
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) {
+                    const int sl = M::row(warp, lane, r);
+                    const float4 c = sm.ak[sl];
+                    const float2 ka = make_float2(c.x, c.y), al = make_float2(c.z, c.z);
+                    float4* dst = reinterpret_cast<float4*>(
+                        a.x_out + (static_cast<int64_t>(tile) * D + (meta[sl] & 0xFF)) * D + 8 * cl);
+                    float2 x[4];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) x[p] = mul2(mul2(fma2(ka, ut[p], Z[r][p]), al), cf[p]);
+                    dst[0] = make_float4(x[0].x, x[0].y, x[1].x, x[1].y);
+                    dst[1] = make_float4(x[2].x, x[2].y, x[3].x, x[3].y);
+                }
+                if (issued) {
+                    sm.stage[sa].beta = next_beta;
+                    sm.stage[sa].gate1 = next_gate;
+                }
+                __syncthreads();   // the next tile's prologue rewrites the per-slot constants
+                continue;
+            }
             float part[RPT];
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
@@ -643,7 +671,7 @@ decode_kernel(const DecodeArgs a) {
     }
 }
 
-template <int D>
+template <int D, bool kSplit = false>
 static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     static int ctas_per_sm = -1, num_sms = 0;
     const size_t smem = sizeof(DecodeSmem<D>);
@@ -651,18 +679,35 @@ static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "stepq_decode_step: %s", cudaGetErrorString(e));
         int occ = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D>, DMap<D>::kThreads, smem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D, kSplit>, DMap<D>::kThreads, smem);
         ctas_per_sm = occ > 0 ? occ : 1;
     }
     if (a.num_tiles == 0) return STEPQ_OK;
     int grid = num_sms * ctas_per_sm;
     if (grid > a.num_tiles) grid = a.num_tiles;
-    decode_kernel<D><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
+    decode_kernel<D, kSplit><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
     return check_launch("stepq_decode_step");
+}
+
+// One event per device orders the refit and pack of the split form after its first kernel.
+static int split_event(cudaEvent_t* ev) {
+    static std::mutex mu;
+    static cudaEvent_t events[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64)
+        return set_error(STEPQ_ECUDA, "stepq_decode_step_split: device %d: %s", dev, cudaGetErrorString(e));
+    std::lock_guard<std::mutex> lock(mu);
+    if (events[dev] == nullptr) {
+        e = cudaEventCreateWithFlags(&events[dev], cudaEventDisableTiming);
+        if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "stepq_decode_step_split: %s", cudaGetErrorString(e));
+    }
+    *ev = events[dev];
+    return STEPQ_OK;
 }
 
 }  // namespace stepq
@@ -689,9 +734,52 @@ extern "C" int stepq_decode_step(stepq_dims dims, const uint16_t* q, const uint1
     const long long tiles = static_cast<long long>(dims.B) * dims.H;
     if (tiles > 0x7fffffffLL) return set_error(STEPQ_EINVAL, "stepq_decode_step: too many tiles");
     DecodeArgs a{dims.B, dims.H, dims.gate_per_channel, static_cast<int>(tiles), q, k, v, beta, gate, bits, w,
-                 head_off, bytes_per_seq, packed_in, r_in, c_in, packed_out, r_out, c_out, o};
+                 head_off, bytes_per_seq, packed_in, r_in, c_in, packed_out, r_out, c_out, o, nullptr};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return dims.dk == 128 ? launch_decode<128>(a, st) : launch_decode<64>(a, st);
+}
+
+extern "C" int stepq_decode_step_split(stepq_dims dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                       const float* beta, const float* gate, const uint8_t* bits, const float* w,
+                                       const int64_t* head_off, int64_t bytes_per_seq, const uint8_t* packed_in,
+                                       const uint16_t* r_in, const uint16_t* c_in, uint8_t* packed_out,
+                                       uint16_t* r_out, uint16_t* c_out, float* o, float* x_ws, void* stream,
+                                       void* side_stream) {
+    const char* fn = "stepq_decode_step_split";
+    clear_error();
+    int rc = check_dims(dims, fn);
+    if (rc) return rc;
+    if (dims.B == 0) return STEPQ_OK;
+    rc = check_ptrs(fn, {{"q", q}, {"k", k}, {"v", v}, {"beta", beta}, {"gate", gate}, {"bits", bits}, {"w", w},
+                         {"head_off", head_off}, {"packed_in", packed_in}, {"r_in", r_in}, {"c_in", c_in},
+                         {"o", o}, {"x_ws", x_ws}});
+    if (rc) return rc;
+    const bool refit = packed_out || r_out || c_out;
+    if (refit) {
+        rc = check_ptrs(fn, {{"packed_out", packed_out}, {"r_out", r_out}, {"c_out", c_out}});
+        if (rc) return rc;
+    }
+    if (bytes_per_seq <= 0 || (bytes_per_seq & 15))
+        return set_error(STEPQ_EINVAL, "%s: bytes_per_seq=%lld", fn, (long long)bytes_per_seq);
+    const long long tiles = static_cast<long long>(dims.B) * dims.H;
+    if (tiles > 0x7fffffffLL) return set_error(STEPQ_EINVAL, "%s: too many tiles", fn);
+    DecodeArgs a{dims.B, dims.H, dims.gate_per_channel, static_cast<int>(tiles), q, k, v, beta, gate, bits, w,
+                 head_off, bytes_per_seq, packed_in, r_in, c_in, nullptr, nullptr, nullptr, o, x_ws};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = dims.dk == 128 ? launch_decode<128, true>(a, st) : launch_decode<64, true>(a, st);
+    if (rc || !refit) return rc;
+    // Refit and pack on the side stream, after the first kernel.
+    cudaStream_t side = static_cast<cudaStream_t>(side_stream);
+    cudaEvent_t ev;
+    rc = split_event(&ev);
+    if (rc) return rc;
+    cudaError_t e = cudaEventRecord(ev, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev, 0);
+    if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "%s: %s", fn, cudaGetErrorString(e));
+    stepq_dims fd{dims.B, dims.H, dims.dk, dims.dv, 0};
+    rc = stepq_fit_scales(fd, x_ws, w, bits, r_out, c_out, side_stream);
+    if (rc) return rc;
+    return stepq_pack_state(fd, x_ws, bits, head_off, bytes_per_seq, r_out, c_out, packed_out, side_stream);
 }
 
 extern "C" int stepq_read_device_flags(uint32_t* flags_host) {
