@@ -52,6 +52,8 @@ def lib():
         _lib.orc_scale_to_half.argtypes = [ctypes.c_double]
         _lib.orc_half_to_float.restype = ctypes.c_float
         _lib.orc_half_to_float.argtypes = [ctypes.c_uint16]
+        _lib.orc_float_to_half.restype = ctypes.c_uint16
+        _lib.orc_float_to_half.argtypes = [ctypes.c_float]
         _lib.orc_layout.restype = ctypes.c_int64
         _lib.orc_tile_bytes.restype = ctypes.c_int64
     return _lib
@@ -276,6 +278,21 @@ def row_impact(calib):
     return w
 
 
+def float_to_half(x: float) -> int:
+    """The binary16 bits of an FP16 pivot value (nearest-even, saturating)."""
+    return int(lib().orc_float_to_half(float(x)))
+
+
+def calib_distortion_bits(S, w, bits, nthreads=0):
+    """(d_row [H][dk], d_head [H]) under the per-row bit map bits [H][dk] (16 = FP16 pivot)."""
+    S = _c(S, np.float32); w = _c(w, np.float32); bits = _c(bits, np.uint8)
+    B, H, dk, dv = S.shape
+    d_row = np.zeros((H, dk)); d_head = np.zeros(H)
+    _check(lib().orc_calib_distortion_bits(B, H, dk, dv, _p(S), _p(w), _p(bits), _p(d_row), _p(d_head), nthreads),
+           "calib_distortion_bits")
+    return d_row, d_head
+
+
 def calib_distortion(S, w, b, nthreads=0):
     """(d_row [H][dk], d_head [H]) at uniform width b over the sample states S [B][H][dk][dv]."""
     S = _c(S, np.float32); w = _c(w, np.float32)
@@ -310,14 +327,31 @@ def objective(d, gate):
     return lifetime(gate)[:, None] * np.asarray(d, dtype=np.float64)
 
 
-def calibrate(alloc, candidates, nominal_bits, gates, S0, calib):
+def pivot_order(score):
+    """Units by descending score, ties to the lower index."""
+    score = np.asarray(score, dtype=np.float64)
+    return np.lexsort((np.arange(score.size), -score))
+
+
+def calibrate(alloc, candidates, nominal_bits, gates, S0, calib, n_pivots=0):
     """The offline calibration done by the oracle (App. A.3, B.3, C.2): returns
     (bits uint8 [H][dk] or None, w float32 [H][dk]).
 
     alloc: "dp_head" (head units, multiple-choice DP, Eq. 17 distortion) or "lagrange_row"
     (key-row units, Lagrangian allocation with repair, Eq. 18 distortion); any other value
     returns bits=None (the caller supplies a fixed map). gates: unit gates [H] or [H][dk];
-    S0: the sample states [B][H][dk][dv]; calib: the calibration stream."""
+    S0: the sample states [B][H][dk][dv]; calib: the calibration stream.
+
+    n_pivots > 0 keeps that many units in FP16 (width 16, App. C.2, Table B1):
+      key rows: ranked by the lifetime-weighted reduction of error from the integer format at
+        the nominal width to FP16, L_u (d_u(b_nominal) - d_u(16)); with the pivots fixed the
+        candidate distortions of the other rows are measured again with the pivots left out
+        of the shared column fit, and those rows are allocated;
+      heads: allocated first; the heads with the largest residual risk L_u d_u(b_u) become
+        pivots and the other heads are allocated again.
+    Each pivot unit counts 8 bits toward the integer budget n_units * nominal_bits and its
+    other 8 bits come on top (the (16 - 8) accounting of App. D), so the remaining units share
+    n_units * nominal_bits - 8 n_pivots bits."""
     w = row_impact(calib)
     H, dk = w.shape
     if alloc not in ("dp_head", "lagrange_row"):
@@ -332,9 +366,35 @@ def calibrate(alloc, candidates, nominal_bits, gates, S0, calib):
     if alloc == "dp_head":
         dist = np.stack(dheads, axis=1)                          # [H][n_cand]
         g = gates if gates.ndim == 1 else gates.mean(axis=1)
-        bh = allocate_bits(objective(dist, g), cand, nominal_bits * H, mode=1)
+        J = objective(dist, g)
+        bh = allocate_bits(J, cand, nominal_bits * H, mode=1)
+        if n_pivots:
+            risk = J[np.arange(H), [cand.index(int(b)) for b in bh]]
+            piv = np.sort(pivot_order(risk)[:n_pivots])
+            rest = np.setdiff1d(np.arange(H), piv)
+            bh = bh.astype(np.uint8)
+            bh[rest] = allocate_bits(J[rest], cand, nominal_bits * H - 8 * n_pivots, mode=1)
+            bh[piv] = 16
         return np.repeat(bh[:, None], dk, axis=1).astype(np.uint8), w
-    dist = np.stack([dr.reshape(-1) for dr in drows], axis=1)   # [H*dk][n_cand]
     g = gates.reshape(-1) if gates.ndim == 2 else np.repeat(gates, dk)
-    br = allocate_bits(objective(dist, g), cand, nominal_bits * H * dk, mode=0)
-    return br.reshape(H, dk).astype(np.uint8), w
+    n = H * dk
+    if not n_pivots:
+        dist = np.stack([dr.reshape(-1) for dr in drows], axis=1)   # [H*dk][n_cand]
+        br = allocate_bits(objective(dist, g), cand, nominal_bits * n, mode=0)
+        return br.reshape(H, dk).astype(np.uint8), w
+    d16, _ = calib_distortion(S0, w, 16)
+    dnom = drows[cand.index(int(nominal_bits))] if int(nominal_bits) in cand else \
+        calib_distortion(S0, w, nominal_bits)[0]
+    score = lifetime(g) * (dnom.reshape(-1) - d16.reshape(-1))
+    piv = np.sort(pivot_order(score)[:n_pivots])
+    rest = np.setdiff1d(np.arange(n), piv)
+    dist = []
+    for b in cand:
+        m = np.full(n, b, dtype=np.uint8)
+        m[piv] = 16
+        dist.append(calib_distortion_bits(S0, w, m.reshape(H, dk))[0].reshape(-1))
+    dist = np.stack(dist, axis=1)
+    br = np.zeros(n, dtype=np.uint8)
+    br[rest] = allocate_bits(objective(dist[rest], g[rest]), cand, nominal_bits * n - 8 * n_pivots, mode=0)
+    br[piv] = 16
+    return br.reshape(H, dk), w

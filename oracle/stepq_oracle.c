@@ -48,6 +48,13 @@
  *      4-bit row) followed by the high 2 bits (laid out as a 2-bit row).
  *   R6 KDA code normalisation (z = 2^(8-b) q) for every workload.
  *   R7 omega floor 1e-12 max_i omega_i; w normalised to mean 1 per head.
+ *   R8 FP16 pivot rows (App. C.2; Table C2 steps 1 and 6), marked by width 16: the row keeps
+ *      its values as binary16 (2 d_v bytes, column j at byte 2j, little-endian), stored
+ *      after all integer rows of the tile; it takes no part in the shared column fit (c0 and
+ *      the least-squares sums run over the integer rows); its row factor is computed like
+ *      any other (R1) and is not used.
+ *   R9 a pivot value is the fp32 X rounded to binary16, nearest with ties to even,
+ *      saturating at +-65504.
  */
 #include <math.h>
 #include <stdint.h>
@@ -66,9 +73,11 @@ enum { ORC_OK = 0, ORC_EINVAL = 1, ORC_EUNSUPPORTED = 2, ORC_EBUDGET = 4, ORC_EN
 /* Bit widths and codebooks (§2.2, App. C.1).                                                 */
 /* ------------------------------------------------------------------------------------------ */
 
-static int width_ok(int b) { return b == 2 || b == 4 || b == 6 || b == 8; }
-static int qmax_of(int b) { return (1 << (b - 1)) - 1; }   /* q_b = 2^(b-1) - 1 */
-static int znorm_of(int b) { return 1 << (8 - b); }        /* z = 2^(8-b) q       */
+/* b = 16 marks an FP16 pivot row (App. C.2, Table C2 steps 1 and 6; reading R8). */
+static int is_pivot(int b) { return b == 16; }
+static int width_ok(int b) { return b == 2 || b == 4 || b == 6 || b == 8 || b == 16; }
+static int qmax_of(int b) { return (1 << (b - 1)) - 1; }   /* q_b = 2^(b-1) - 1 (integer rows) */
+static int znorm_of(int b) { return 1 << (8 - b); }        /* z = 2^(8-b) q       (integer rows) */
 
 int orc_dims_ok(int dk, int dv) { return (dk == 64 || dk == 128) && (dv == 64 || dv == 128); }
 
@@ -105,6 +114,27 @@ uint16_t orc_scale_to_half(double x) {
     return (uint16_t)((E << 10) | ((int)sig - 1024));
 }
 
+/* fp32 -> binary16, nearest with ties to even, saturating at +-65504 (reading R9): the value
+   stored for an FP16 pivot entry. Written from the binary16 format definition. */
+uint16_t orc_float_to_half(float xf) {
+    double x = (double)xf;
+    uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    x = fabs(x);
+    if (isnan(x)) return 0x7E00u;
+    if (x > HALF_MAX) return (uint16_t)(sign | 0x7BFFu);
+    if (x < HALF_MIN_NORMAL) {                       /* subnormal: steps of 2^-24      */
+        double q = nearbyint(ldexp(x, 24));          /* 1024 is 2^-14, the first normal */
+        return (uint16_t)(sign | (uint16_t)q);
+    }
+    int e;
+    double m = frexp(x, &e);
+    double sig = nearbyint(ldexp(m, 11));
+    if (sig == 2048.0) { sig = 1024.0; e += 1; }
+    int E = e - 1 + 15;
+    if (E >= 31) return (uint16_t)(sign | 0x7BFFu);
+    return (uint16_t)(sign | (E << 10) | ((int)sig - 1024));
+}
+
 /* ------------------------------------------------------------------------------------------ */
 /* Quantiser and dequantiser contract (readings R3, R4), fp32.                                */
 /* ------------------------------------------------------------------------------------------ */
@@ -133,6 +163,18 @@ int64_t orc_tile_bytes(int dk, int dv, const uint8_t* bits) {
     int64_t n = 0;
     for (int i = 0; i < dk; ++i) n += row_bytes(dv, bits[i]);
     return n;
+}
+
+/* Byte offset of every row inside its tile (readings R5, R8): the integer rows first, in key
+   order, then the FP16 pivot rows, in key order. */
+static void row_offsets(int dk, int dv, const uint8_t* bits, int64_t* off) {
+    int64_t o = 0;
+    for (int pass = 0; pass < 2; ++pass)
+        for (int i = 0; i < dk; ++i)
+            if (is_pivot(bits[i]) == pass) {
+                off[i] = o;
+                o += row_bytes(dv, bits[i]);
+            }
 }
 
 /* head_off[h] = bytes of heads 0..h-1 of one sequence; returns bytes per sequence. */
@@ -195,8 +237,8 @@ static void unpack_row(const uint8_t* row, int dv, int b, int* q) {
         if (b == 6) v = get_bits(row, field_bit(j, 4), 4) | (get_bits(row + dv / 2, field_bit(j, 2), 2) << 4);
         else v = get_bits(row, field_bit(j, b), b);
         int s = (int)v;
-        if (s >= (1 << (b - 1))) s -= (1 << b);            /* sign-extend from b bits */
-        q[j] = s;
+        if (!is_pivot(b) && s >= (1 << (b - 1))) s -= (1 << b);   /* sign-extend from b bits */
+        q[j] = s;                                   /* a pivot entry: its binary16 bit pattern */
     }
 }
 
@@ -209,6 +251,10 @@ void orc_quantise_tile(int dk, int dv, const float* X, const uint8_t* bits, cons
                        const uint16_t* c, int* codes) {
     for (int i = 0; i < dk; ++i) {
         int b = bits[i];
+        if (is_pivot(b)) {                           /* FP16 pivot row: the value itself */
+            for (int j = 0; j < dv; ++j) codes[i * dv + j] = orc_float_to_half(X[i * dv + j]);
+            continue;
+        }
         float ir = 1.0f / (orc_half_to_float(r[i]) * (float)znorm_of(b));
         for (int j = 0; j < dv; ++j) {
             float ic = 1.0f / orc_half_to_float(c[j]);
@@ -218,19 +264,17 @@ void orc_quantise_tile(int dk, int dv, const float* X, const uint8_t* bits, cons
 }
 
 void orc_pack_codes(int dk, int dv, const uint8_t* bits, const int* codes, uint8_t* packed) {
-    int64_t off = 0;
-    for (int i = 0; i < dk; ++i) {
-        pack_row(packed + off, dv, bits[i], codes + (int64_t)i * dv);
-        off += row_bytes(dv, bits[i]);
-    }
+    int64_t* off = (int64_t*)malloc(sizeof(int64_t) * dk);
+    row_offsets(dk, dv, bits, off);
+    for (int i = 0; i < dk; ++i) pack_row(packed + off[i], dv, bits[i], codes + (int64_t)i * dv);
+    free(off);
 }
 
 void orc_unpack_codes(int dk, int dv, const uint8_t* bits, const uint8_t* packed, int* codes) {
-    int64_t off = 0;
-    for (int i = 0; i < dk; ++i) {
-        unpack_row(packed + off, dv, bits[i], codes + (int64_t)i * dv);
-        off += row_bytes(dv, bits[i]);
-    }
+    int64_t* off = (int64_t*)malloc(sizeof(int64_t) * dk);
+    row_offsets(dk, dv, bits, off);
+    for (int i = 0; i < dk; ++i) unpack_row(packed + off[i], dv, bits[i], codes + (int64_t)i * dv);
+    free(off);
 }
 
 void orc_pack_tile(int dk, int dv, const float* X, const uint8_t* bits, const uint16_t* r,
@@ -248,7 +292,8 @@ void orc_unpack_tile(int dk, int dv, const uint8_t* packed, const uint8_t* bits,
     for (int i = 0; i < dk; ++i) {
         float ri = orc_half_to_float(r[i]);
         for (int j = 0; j < dv; ++j)
-            X[i * dv + j] = dequantise(ri, orc_half_to_float(c[j]), codes[i * dv + j], bits[i]);
+            X[i * dv + j] = is_pivot(bits[i]) ? orc_half_to_float((uint16_t)codes[i * dv + j])
+                                              : dequantise(ri, orc_half_to_float(c[j]), codes[i * dv + j], bits[i]);
     }
     free(codes);
 }
@@ -273,11 +318,14 @@ void orc_fit_tile_detail(int dk, int dv, const float* X, const float* w, const u
         rf[i] = orc_half_to_float(r_out[i]);
     }
 
-    /* Column initialisation: smallest scale at which no entry of the column clips. */
+    /* Column initialisation: smallest scale at which no entry of the column clips. The shared
+       column scales serve the integer rows only: FP16 pivot rows take no part (App. C.1, the
+       sums over the non-pivot rows I). */
     for (int j = 0; j < dv; ++j) {
         float mx = 0.0f;
         for (int i = 0; i < dk; ++i) {
             int b = bits[i];
+            if (is_pivot(b)) continue;
             float a = 1.0f / (rf[i] * (float)(znorm_of(b) * qmax_of(b)));
             float t = fabsf(X[i * dv + j]) * a;
             if (t > mx) mx = t;
@@ -288,6 +336,10 @@ void orc_fit_tile_detail(int dk, int dv, const float* X, const float* w, const u
     /* Codes at (r, c0), decided in fp32 by the quantiser contract. */
     for (int i = 0; i < dk; ++i) {
         int b = bits[i];
+        if (is_pivot(b)) {
+            for (int j = 0; j < dv; ++j) z0[i * dv + j] = 0;
+            continue;
+        }
         float ir = 1.0f / (rf[i] * (float)znorm_of(b));
         for (int j = 0; j < dv; ++j) z0[i * dv + j] = quantise(X[i * dv + j], ir, 1.0f / c0[j], b);
     }
@@ -297,6 +349,7 @@ void orc_fit_tile_detail(int dk, int dv, const float* X, const float* w, const u
     for (int j = 0; j < dv; ++j) {
         double num = 0.0, den = 0.0;
         for (int i = 0; i < dk; ++i) {
+            if (is_pivot(bits[i])) continue;
             double v = (double)rf[i] * znorm_of(bits[i]) * z0[i * dv + j];
             double ww = (double)w[i] * (double)w[i];
             num += ww * v * (double)X[i * dv + j];
@@ -611,23 +664,23 @@ int orc_row_impact(int T, int B, int H, int dk, int gate_per_channel, const uint
     return ORC_OK;
 }
 
-/* Candidate-format distortion at uniform width b over the B sample states (App. A.3):
-   d_row[h][i] = (1/(B d_v)) sum_b sum_j (x_hat - x)^2                 (Eq. 18, KDA rows)
-   d_head[h]   = (1/(B d_k d_v)) sum_b sum_ij w_i^2 (x_hat - x)^2       (Eq. 17, Qwen heads)
-   where x_hat is the state fitted, packed and unpacked at width b. */
-int orc_calib_distortion(int B, int H, int dk, int dv, const float* S, const float* w, int b,
-                         double* d_row, double* d_head, int nthreads) {
-    if (!orc_dims_ok(dk, dv) || !width_ok(b)) return ORC_EUNSUPPORTED;
-    uint8_t* bits = (uint8_t*)malloc(dk);
-    memset(bits, b, dk);
-    int64_t tb = orc_tile_bytes(dk, dv, bits);
+/* Candidate-format distortion of the B sample states under the bit map bits [H][dk]
+   (App. A.3): d_row[h][i] = (1/(B d_v)) sum_b sum_j (x_hat - x)^2                (Eq. 18)
+               d_head[h]   = (1/(B d_k d_v)) sum_b sum_ij w_i^2 (x_hat - x)^2      (Eq. 17)
+   where x_hat is the state fitted, packed and unpacked under that map. */
+int orc_calib_distortion_bits(int B, int H, int dk, int dv, const float* S, const float* w,
+                              const uint8_t* bits_map, double* d_row, double* d_head, int nthreads) {
+    if (!orc_dims_ok(dk, dv)) return ORC_EUNSUPPORTED;
+    for (int64_t u = 0; u < (int64_t)H * dk; ++u)
+        if (!width_ok(bits_map[u])) return ORC_EUNSUPPORTED;
     int nt = set_threads(nthreads);
     (void)nt;
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
     for (int h = 0; h < H; ++h) {
+        const uint8_t* bits = bits_map + (int64_t)h * dk;
         uint16_t* r = (uint16_t*)malloc(sizeof(uint16_t) * dk);
         uint16_t* c = (uint16_t*)malloc(sizeof(uint16_t) * dv);
-        uint8_t* pk = (uint8_t*)malloc(tb);
+        uint8_t* pk = (uint8_t*)malloc(orc_tile_bytes(dk, dv, bits));
         float* Xh = (float*)malloc(sizeof(float) * dk * dv);
         double dh = 0.0;
         for (int i = 0; i < dk; ++i) d_row[(int64_t)h * dk + i] = 0.0;
@@ -651,8 +704,18 @@ int orc_calib_distortion(int B, int H, int dk, int dv, const float* S, const flo
         d_head[h] = dh / ((double)B * dk * dv);
         free(r); free(c); free(pk); free(Xh);
     }
-    free(bits);
     return ORC_OK;
+}
+
+/* The same at the uniform width b (every row of every head). */
+int orc_calib_distortion(int B, int H, int dk, int dv, const float* S, const float* w, int b,
+                         double* d_row, double* d_head, int nthreads) {
+    if (!orc_dims_ok(dk, dv) || !width_ok(b)) return ORC_EUNSUPPORTED;
+    uint8_t* bits = (uint8_t*)malloc((size_t)H * dk);
+    memset(bits, b, (size_t)H * dk);
+    int rc = orc_calib_distortion_bits(B, H, dk, dv, S, w, bits, d_row, d_head, nthreads);
+    free(bits);
+    return rc;
 }
 
 /* ------------------------------------------------------------------------------------------ */
