@@ -14,22 +14,29 @@
  *     `stream` (a cudaStream_t passed as void*; NULL = the legacy default stream).
  *   - Device pointers must be 16-byte aligned (STEPQ_EALIGN otherwise); packed buffers must
  *     also have a 16-byte aligned base.
- *   - d_k = d_v = 64 or 128 (STEPQ_EUNSUPPORTED otherwise); bit widths are 2, 4, 6 or 8.
+ *   - d_k = d_v = 64 or 128 (STEPQ_EUNSUPPORTED otherwise); bit widths are 2, 4, 6 or 8, or
+ *     16 for an FP16 pivot row (App. C.2; Table C2 steps 1 and 6), which keeps its values in
+ *     binary16 and takes no part in the shared column fit.
  *   - Arrays are row-major: S float32 [B][H][dk][dv]; q, k bf16 bits (uint16) [B][H][dk];
  *     v bf16 bits [B][H][dv]; beta float32 [B][H]; gate float32 [B][H] (scalar gate per head,
  *     GDN) or [B][H][dk] (one gate per key channel, KDA; dims.gate_per_channel = 1);
  *     bits uint8 [H][dk]; w float32 [H][dk]; r binary16 bits [B][H][dk]; c binary16 bits
  *     [B][H][dv]; o float32 [B][H][dv].
- *   - Packed state: tile (b, h) starts at byte b * bytes_per_seq + head_off[h]; its row i
- *     starts at (dv/8) * sum_{i'<i} bits[h][i']; a row of width 2, 4 or 8 stores the code of
- *     column j at bit j*b of a little-endian bit stream as a b-bit two's complement integer;
- *     a 6-bit row stores the low 4 bits of every code (laid out as a 4-bit row) followed by
- *     the high 2 bits (laid out as a 2-bit row). Codes q lie in [-q_b, q_b], q_b = 2^(b-1)-1.
+ *   - Packed state: tile (b, h) starts at byte b * bytes_per_seq + head_off[h]; a row of
+ *     width b takes dv*b/8 bytes; the integer rows come first, in key order, then the FP16
+ *     pivot rows, in key order. Codes are b-bit two's complement integers q in [-q_b, q_b],
+ *     q_b = 2^(b-1)-1. A 2- or 8-bit row stores column j at bit j*b of a little-endian bit
+ *     stream; a 4-bit row stores columns 4g..4g+3 in the little-endian halfword g, column
+ *     4g+m at bit 4*pos(m), pos = (0, 2, 1, 3); a 6-bit row stores the low 4 bits of every
+ *     code (laid out as a 4-bit row) followed by the high 2 bits (laid out as a 2-bit row).
+ *     A pivot row stores column j as binary16 at byte 2j.
  *   - Reconstruction (dequantisation), fp32: x_hat_ij = (r_i * c_j) * (q_ij * 2^(8-b_i)),
  *     i.e. the code normalisation z = 2^(8-b) q of App. C.1 with scales X_hat = r_i c_j z_ij
  *     (§4.3).
  *   - Quantisation, fp32: t = (x * ir_i) * ic_j with ir_i = 1/(r_i 2^(8-b_i)), ic_j = 1/c_j;
- *     q = clamp(rint(t), -q_b, q_b), rint rounding to nearest, ties to even (§2.2).
+ *     q = clamp(rint(t), -q_b, q_b), rint rounding to nearest, ties to even (§2.2). A pivot
+ *     entry is x rounded to binary16 (nearest-even, saturating at +-65504); its row factor is
+ *     computed like any other and not used.
  *   - Return value: STEPQ_OK or an error code; stepq_last_error() then describes it (per
  *     thread). On an error nothing has been queued.
  */
@@ -51,7 +58,7 @@ extern "C" {
 enum {
     STEPQ_OK = 0,
     STEPQ_EINVAL = 1,        /* bad argument (null pointer, negative size, ...)            */
-    STEPQ_EUNSUPPORTED = 2,  /* d_k / d_v not in {64, 128}, or a bit width not in {2,4,6,8} */
+    STEPQ_EUNSUPPORTED = 2,  /* d_k / d_v not in {64, 128}, or a width not in {2,4,6,8,16} */
     STEPQ_EALIGN = 3,        /* a device pointer is not 16-byte aligned                     */
     STEPQ_EBUDGET = 4,       /* bit allocation: no assignment reaches the budget exactly    */
     STEPQ_ECUDA = 5          /* a CUDA launch failed; stepq_last_error() names the error    */
@@ -169,6 +176,12 @@ STEPQ_API int stepq_row_impact(stepq_dims dims, int T, const uint16_t* q, const 
    scratch: caller-provided float64 [B][H][dk] work space. */
 STEPQ_API int stepq_calib_distortion(stepq_dims dims, const float* S, const float* w, int b, double* d_row,
                            double* d_head, double* scratch, void* stream);
+
+/* The same under a per-row bit map bits [H][dk] (widths 2, 4, 6, 8 and 16 = FP16 pivot rows,
+   which take no part in the shared column fit): the candidate distortions recalibrated with
+   the pivots fixed (App. C.2, KDA calibration). */
+STEPQ_API int stepq_calib_distortion_bits(stepq_dims dims, const float* S, const float* w, const uint8_t* bits,
+                                double* d_row, double* d_head, double* scratch, void* stream);
 
 /* Capacity, in float64 entries, of the static work space of stepq_calib_distortion_static:
    it takes B * H * dk <= STEPQ_STATIC_SCRATCH_ROWS (4 MiB of device memory per device, held

@@ -48,12 +48,12 @@
  *      4-bit row) followed by the high 2 bits (laid out as a 2-bit row).
  *   R6 KDA code normalisation (z = 2^(8-b) q) for every workload.
  *   R7 omega floor 1e-12 max_i omega_i; w normalised to mean 1 per head.
- *   R8 FP16 pivot rows (App. C.2; Table C2 steps 1 and 6), marked by width 16: the row keeps
+ *   R14 FP16 pivot rows (App. C.2; Table C2 steps 1 and 6), marked by width 16: the row keeps
  *      its values as binary16 (2 d_v bytes, column j at byte 2j, little-endian), stored
  *      after all integer rows of the tile; it takes no part in the shared column fit (c0 and
  *      the least-squares sums run over the integer rows); its row factor is computed like
  *      any other (R1) and is not used.
- *   R9 a pivot value is the fp32 X rounded to binary16, nearest with ties to even,
+ *   R15 a pivot value is the fp32 X rounded to binary16, nearest with ties to even,
  *      saturating at +-65504.
  */
 #include <math.h>
@@ -73,7 +73,7 @@ enum { ORC_OK = 0, ORC_EINVAL = 1, ORC_EUNSUPPORTED = 2, ORC_EBUDGET = 4, ORC_EN
 /* Bit widths and codebooks (§2.2, App. C.1).                                                 */
 /* ------------------------------------------------------------------------------------------ */
 
-/* b = 16 marks an FP16 pivot row (App. C.2, Table C2 steps 1 and 6; reading R8). */
+/* b = 16 marks an FP16 pivot row (App. C.2, Table C2 steps 1 and 6; reading R14). */
 static int is_pivot(int b) { return b == 16; }
 static int width_ok(int b) { return b == 2 || b == 4 || b == 6 || b == 8 || b == 16; }
 static int qmax_of(int b) { return (1 << (b - 1)) - 1; }   /* q_b = 2^(b-1) - 1 (integer rows) */
@@ -114,7 +114,7 @@ uint16_t orc_scale_to_half(double x) {
     return (uint16_t)((E << 10) | ((int)sig - 1024));
 }
 
-/* fp32 -> binary16, nearest with ties to even, saturating at +-65504 (reading R9): the value
+/* fp32 -> binary16, nearest with ties to even, saturating at +-65504 (reading R15): the value
    stored for an FP16 pivot entry. Written from the binary16 format definition. */
 uint16_t orc_float_to_half(float xf) {
     double x = (double)xf;
@@ -165,7 +165,7 @@ int64_t orc_tile_bytes(int dk, int dv, const uint8_t* bits) {
     return n;
 }
 
-/* Byte offset of every row inside its tile (readings R5, R8): the integer rows first, in key
+/* Byte offset of every row inside its tile (readings R5, R14): the integer rows first, in key
    order, then the FP16 pivot rows, in key order. */
 static void row_offsets(int dk, int dv, const uint8_t* bits, int64_t* off) {
     int64_t o = 0;

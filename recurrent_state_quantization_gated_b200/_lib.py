@@ -17,7 +17,7 @@ SYMBOLS = (
     "stepq_last_error", "stepq_packed_layout", "stepq_fit_scales", "stepq_pack_state",
     "stepq_unpack_state", "stepq_decode_step", "stepq_decode_step_split", "stepq_decode_step_fp32",
     "stepq_int8_quantize_state", "stepq_decode_step_int8", "stepq_row_impact",
-    "stepq_calib_distortion", "stepq_calib_distortion_static", "stepq_allocate_bits", "stepq_read_device_flags",
+    "stepq_calib_distortion", "stepq_calib_distortion_bits", "stepq_calib_distortion_static", "stepq_allocate_bits", "stepq_read_device_flags",
     "stepq_build_info",
 )
 
@@ -54,6 +54,7 @@ _SIGNATURES = {
     "stepq_row_impact": ([Dims, I, P, P, P, P, P, P], I),
     "stepq_calib_distortion": ([Dims, P, P, I, P, P, P, P], I),
     "stepq_calib_distortion_static": ([Dims, P, P, I, P, P, P], I),
+    "stepq_calib_distortion_bits": ([Dims, P, P, P, P, P, P, P], I),
     "stepq_allocate_bits": ([I, I, P, P, I64, I, P], I),
     "stepq_read_device_flags": ([P], I),
 }

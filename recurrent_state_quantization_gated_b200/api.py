@@ -21,7 +21,7 @@ from ._lib import Dims, call, lib
 __all__ = [
     "stepq_packed_layout", "stepq_fit_scales", "stepq_pack_state", "stepq_unpack_state",
     "stepq_decode_step", "stepq_decode_step_split", "stepq_decode_step_fp32", "stepq_int8_quantize_state",
-    "stepq_decode_step_int8", "stepq_row_impact", "stepq_calib_distortion", "stepq_calib_distortion_static",
+    "stepq_decode_step_int8", "stepq_row_impact", "stepq_calib_distortion", "stepq_calib_distortion_bits", "stepq_calib_distortion_static",
     "stepq_allocate_bits",
     "stepq_read_device_flags", "stepq_build_info",
 ]
@@ -196,6 +196,20 @@ def stepq_calib_distortion(S, w, b, d_row=None, d_head=None, scratch=None):
     scratch = torch.empty((B, H, d), dtype=torch.float64, device=dev) if scratch is None else scratch
     call("stepq_calib_distortion", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
          ctypes.c_int(int(b)), _ptr(d_row, torch.float64, "d_row"), _ptr(d_head, torch.float64, "d_head"),
+         _ptr(scratch, torch.float64, "scratch"), _stream())
+    return d_row, d_head
+
+
+def stepq_calib_distortion_bits(S, w, bits, d_row=None, d_head=None, scratch=None):
+    """(d_row float64 [H,d], d_head float64 [H]) under the per-row bit map bits (uint8 [H,d],
+    16 = FP16 pivot row) over the states S."""
+    B, H, d, _ = S.shape
+    dev = S.device
+    d_row = torch.empty((H, d), dtype=torch.float64, device=dev) if d_row is None else d_row
+    d_head = torch.empty((H,), dtype=torch.float64, device=dev) if d_head is None else d_head
+    scratch = torch.empty((B, H, d), dtype=torch.float64, device=dev) if scratch is None else scratch
+    call("stepq_calib_distortion_bits", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
+         _ptr(bits, torch.uint8, "bits"), _ptr(d_row, torch.float64, "d_row"), _ptr(d_head, torch.float64, "d_head"),
          _ptr(scratch, torch.float64, "scratch"), _stream())
     return d_row, d_head
 

@@ -109,6 +109,7 @@ struct DecodeSmem {
     alignas(16) float riq[D];       // 1/q_b
     // Per column.
     alignas(16) float colc[D];      // c_j (old column scale)
+    alignas(16) float icol[D];      // 1/c_j (FP16 pivot rows enter the tile as x / c_j)
     alignas(16) float colb[D];      // per-phase column broadcast
     alignas(16) float col0[D];      // c0_j
     alignas(16) float red[M::kWarps][2][D];
@@ -127,7 +128,9 @@ __device__ __forceinline__ bool issue_tile(const DecodeArgs& a, DecodeSmem<D>& s
     if (tile >= a.num_tiles) return false;
     const int b = tile / a.H, h = tile % a.H;
     const int64_t hoff = a.head_off[h], hend = (h + 1 < a.H) ? a.head_off[h + 1] : a.bytes_per_seq;
-    const uint32_t pbytes = static_cast<uint32_t>(hend - hoff);
+    // The stage holds the integer rows (at most D*D bytes); FP16 pivot rows, stored after them,
+    // are read from global memory where they are used.
+    const uint32_t pbytes = static_cast<uint32_t>(min(hend - hoff, static_cast<int64_t>(D) * D));
     auto& st = sm.stage[s];
     const uint32_t total = pbytes + 5u * 2u * D + 4u * D + (a.gate_per_channel ? 4u * D : 0u);
     mbar_arrive_expect_tx(&sm.full[s], total);
@@ -150,31 +153,36 @@ __device__ __forceinline__ int cta_tile(int n) { return blockIdx.x + n * gridDim
 // One warp sorts the rows of head h by bit width (stable) into cache entry e.
 template <int D>
 __device__ __forceinline__ void sort_head_warp(const DecodeArgs& a, DecodeSmem<D>& sm, int h, int e, int lane) {
-    constexpr int RL = D / 32;
-    int bw[RL], loc[RL], rank[RL], sum = 0;
-    int cnt[4] = {0, 0, 0, 0};
+    // Width classes in slot order: 2, 4, 6, 8, then 16 (FP16 pivot rows). Byte offsets follow
+    // the packed layout: integer rows in key order, then pivot rows in key order.
+    constexpr int RL = D / 32, NC = 5;
+    int bw[RL], loc[RL], rank[RL], sum_i = 0, sum_p = 0;
+    int cnt[NC] = {0, 0, 0, 0, 0};
 #pragma unroll
     for (int r = 0; r < RL; ++r) {
         bw[r] = a.bits[static_cast<int64_t>(h) * D + lane * RL + r];
-        loc[r] = sum;
-        sum += bw[r] * (D / 8);
-        const int cls = (bw[r] >> 1) - 1;
+        const bool piv = bw[r] == 16;
+        loc[r] = piv ? sum_p : sum_i;
+        (piv ? sum_p : sum_i) += bw[r] * (D / 8);
+        const int cls = piv ? 4 : (bw[r] >> 1) - 1;
         rank[r] = 0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < NC; ++c) {
             if (c == cls) rank[r] = cnt[c];
             cnt[c] += (c == cls);
         }
     }
-    int incl = sum;
+    int inc_i = sum_i, inc_p = sum_p;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
+        const int ti = __shfl_up_sync(0xffffffffu, inc_i, o);
+        const int tp = __shfl_up_sync(0xffffffffu, inc_p, o);
+        if (lane >= o) { inc_i += ti; inc_p += tp; }
     }
-    int excl_c[4], base_c[4], base = 0;
+    const int total_i = __shfl_sync(0xffffffffu, inc_i, 31);
+    int excl_c[NC], base_c[NC], base = 0;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < NC; ++c) {
         int x = cnt[c];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -188,12 +196,13 @@ __device__ __forceinline__ void sort_head_warp(const DecodeArgs& a, DecodeSmem<D
 #pragma unroll
     for (int r = 0; r < RL; ++r) {
         const int i = lane * RL + r;
-        const int cls = (bw[r] >> 1) - 1;
+        const bool piv = bw[r] == 16;
+        const int cls = piv ? 4 : (bw[r] >> 1) - 1;
         int slot = 0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < NC; ++c)
             if (c == cls) slot = base_c[c] + excl_c[c] + rank[r];
-        const int off = incl - sum + loc[r];
+        const int off = (piv ? total_i + inc_p - sum_p : inc_i - sum_i) + loc[r];
         sm.hmeta[e][slot] = static_cast<uint32_t>(i) | (static_cast<uint32_t>(bw[r]) << 8) | (static_cast<uint32_t>(off) << 16);
         sm.hslot[e][i] = static_cast<uint16_t>(slot | (bw[r] << 8));
     }
@@ -210,6 +219,45 @@ __device__ __forceinline__ void phase1_row(const DecodeSmem<D>& sm, const uint8_
     for (int p = 0; p < 4; ++p) {
         pacc[p] = fma2(kap, z[p], pacc[p]);
         oacc[p] = fma2(lam, z[p], oacc[p]);
+    }
+}
+
+// An FP16 pivot row: eight values straight from global memory (pivot rows follow the integer
+// rows of a tile and are not staged), divided by their column scales so that the row joins
+// the tile's factored form X = alpha_i c_j Y_ij with alpha_i = g_i.
+template <int D>
+__device__ __forceinline__ void load_pivot8(const uint8_t* row_g, int cl, const float* icol, float2 z[4]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(row_g + 16 * cl);
+    const float4 i0 = *reinterpret_cast<const float4*>(icol + 8 * cl);
+    const float4 i1 = *reinterpret_cast<const float4*>(icol + 8 * cl + 4);
+    z[0] = mul2(__half22float2(*reinterpret_cast<const __half2*>(&u.x)), make_float2(i0.x, i0.y));
+    z[1] = mul2(__half22float2(*reinterpret_cast<const __half2*>(&u.y)), make_float2(i0.z, i0.w));
+    z[2] = mul2(__half22float2(*reinterpret_cast<const __half2*>(&u.z)), make_float2(i1.x, i1.y));
+    z[3] = mul2(__half22float2(*reinterpret_cast<const __half2*>(&u.w)), make_float2(i1.z, i1.w));
+}
+
+template <int D>
+__device__ __forceinline__ void phase1_pivot_row(const DecodeSmem<D>& sm, const uint8_t* gin, int s, uint32_t mt,
+                                                 int cl, float2 z[4], float2 pacc[4], float2 oacc[4]) {
+    load_pivot8<D>(gin + (mt >> 16), cl, sm.icol, z);
+    const float4 c = sm.kq[s];
+    const float2 kap = make_float2(c.x, c.y), lam = make_float2(c.z, c.w);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        pacc[p] = fma2(kap, z[p], pacc[p]);
+        oacc[p] = fma2(lam, z[p], oacc[p]);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void phase1_pivots(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* gin,
+                                              int warp, int lane, float2 Z[][4], float2 pacc[4], float2 oacc[4]) {
+    using M = DMap<D>;
+    const int cl = M::col_lane(lane);
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r) {
+        const int s = M::row(warp, lane, r);
+        phase1_pivot_row<D>(sm, gin, s, meta[s], cl, Z[r], pacc, oacc);
     }
 }
 
@@ -241,7 +289,8 @@ __device__ __forceinline__ void phase1_uniform(const DecodeSmem<D>& sm, const ui
 
 template <int D>
 __device__ __forceinline__ void phase1_mixed(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* codes,
-                                             int warp, int lane, float2 Z[][4], float2 pacc[4], float2 oacc[4]) {
+                                             const uint8_t* gin, int warp, int lane, float2 Z[][4], float2 pacc[4],
+                                             float2 oacc[4]) {
     using M = DMap<D>;
     const int cl = M::col_lane(lane);
 #pragma unroll
@@ -252,6 +301,7 @@ __device__ __forceinline__ void phase1_mixed(const DecodeSmem<D>& sm, const uint
             case 8: phase1_row<D, 8>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
             case 6: phase1_row<D, 6>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
             case 4: phase1_row<D, 4>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
+            case 16: phase1_pivot_row<D>(sm, gin, s, mt, cl, Z[r], pacc, oacc); break;
             default: phase1_row<D, 2>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
         }
     }
@@ -273,18 +323,35 @@ __device__ __forceinline__ void phase6_row(uint8_t* out, uint32_t mt, int cl, co
     pack8<D, BW, true>(out + (mt >> 16), cl, zq);
 }
 
+// An FP16 pivot row: X_ij = xi_ij c_j (xi = alpha_i Y_ij for pivot rows), rounded to binary16
+// (nearest-even, saturating) and stored straight to global memory.
+template <int D>
+__device__ __forceinline__ void phase6_pivot_row(uint8_t* out, uint32_t mt, int cl, const float2 x[4], const float2 cc[4]) {
+    uint32_t h[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float2 v = mul2(x[p], cc[p]);
+        __half2 hv = __halves2half2(pivot_half(v.x), pivot_half(v.y));
+        h[p] = *reinterpret_cast<uint32_t*>(&hv);
+    }
+    *reinterpret_cast<uint4*>(out + (mt >> 16) + 16 * cl) = make_uint4(h[0], h[1], h[2], h[3]);
+}
+
 template <int D, int BW>
 __device__ __forceinline__ void phase6_uniform(const uint32_t* meta, uint8_t* out, int warp, int lane,
-                                               const float2 Z[][4], const float2 f[4]) {
+                                               const float2 Z[][4], const float2 f[4], const float2 cc[4]) {
     using M = DMap<D>;
     const int cl = M::col_lane(lane);
 #pragma unroll
-    for (int r = 0; r < M::RPT; ++r) phase6_row<D, BW>(out, meta[M::row(warp, lane, r)], cl, Z[r], f);
+    for (int r = 0; r < M::RPT; ++r) {
+        if constexpr (BW == 16) phase6_pivot_row<D>(out, meta[M::row(warp, lane, r)], cl, Z[r], cc);
+        else phase6_row<D, BW>(out, meta[M::row(warp, lane, r)], cl, Z[r], f);
+    }
 }
 
 template <int D>
 __device__ __forceinline__ void phase6_mixed(const uint32_t* meta, uint8_t* out, int warp, int lane,
-                                             const float2 Z[][4], const float2 f[4]) {
+                                             const float2 Z[][4], const float2 f[4], const float2 cc[4]) {
     using M = DMap<D>;
     const int cl = M::col_lane(lane);
 #pragma unroll
@@ -294,6 +361,7 @@ __device__ __forceinline__ void phase6_mixed(const uint32_t* meta, uint8_t* out,
             case 8: phase6_row<D, 8>(out, mt, cl, Z[r], f); break;
             case 6: phase6_row<D, 6>(out, mt, cl, Z[r], f); break;
             case 4: phase6_row<D, 4>(out, mt, cl, Z[r], f); break;
+            case 16: phase6_pivot_row<D>(out, mt, cl, Z[r], cc); break;
             default: phase6_row<D, 2>(out, mt, cl, Z[r], f); break;
         }
     }
@@ -301,13 +369,14 @@ __device__ __forceinline__ void phase6_mixed(const uint32_t* meta, uint8_t* out,
 
 template <int D>
 __device__ __forceinline__ void phase6(const uint32_t* meta, uint8_t* out, int warp, int lane, int ww,
-                                       const float2 Z[][4], const float2 f[4]) {
+                                       const float2 Z[][4], const float2 f[4], const float2 cc[4]) {
     switch (ww) {
-        case 8: phase6_uniform<D, 8>(meta, out, warp, lane, Z, f); break;
-        case 6: phase6_uniform<D, 6>(meta, out, warp, lane, Z, f); break;
-        case 4: phase6_uniform<D, 4>(meta, out, warp, lane, Z, f); break;
-        case 2: phase6_uniform<D, 2>(meta, out, warp, lane, Z, f); break;
-        default: phase6_mixed<D>(meta, out, warp, lane, Z, f); break;
+        case 8: phase6_uniform<D, 8>(meta, out, warp, lane, Z, f, cc); break;
+        case 6: phase6_uniform<D, 6>(meta, out, warp, lane, Z, f, cc); break;
+        case 4: phase6_uniform<D, 4>(meta, out, warp, lane, Z, f, cc); break;
+        case 2: phase6_uniform<D, 2>(meta, out, warp, lane, Z, f, cc); break;
+        case 16: phase6_uniform<D, 16>(meta, out, warp, lane, Z, f, cc); break;
+        default: phase6_mixed<D>(meta, out, warp, lane, Z, f, cc); break;
     }
 }
 
@@ -413,8 +482,9 @@ decode_kernel(const DecodeArgs a) {
                 const uint32_t sw = sm.hslot[he][i];
                 const int sl = sw & 0xFF, bw = sw >> 8;
                 const float g = a.gate_per_channel ? st.gate[i] : st.gate1;
-                // alpha > 0 always (a zero gate leaves 2^-64: far below any term that counts)
-                const float alpha = fmaxf(g * half_bits_to_float(st.r[i]) * znorm_of(bw), 0x1p-64f);
+                // alpha > 0 always (a zero gate leaves 2^-64: far below any term that counts);
+                // an FP16 pivot row carries its values, so alpha is the gate alone.
+                const float alpha = fmaxf(bw == 16 ? g : g * half_bits_to_float(st.r[i]) * znorm_of(bw), 0x1p-64f);
                 const float kk = bf16_bits_to_float(st.k[i]);
                 const float qq = bf16_bits_to_float(st.q[i]);
                 const float wi = st.w[i];
@@ -422,6 +492,7 @@ decode_kernel(const DecodeArgs a) {
                 sm.kq[sl] = make_float4(alpha * kk, alpha * kk, alpha * qq, alpha * qq);
                 sm.ak[sl] = make_float4(ka, ka, alpha, alpha);
                 sm.wsl[sl] = make_float2(wi, rcp_approx(wi));
+                sm.icol[i] = rcp_approx(half_bits_to_float(st.c[i]));   // column i
             } else if (warp == D / 32) {
                 constexpr int RL = D / 32;
                 float acc = 0.f;
@@ -468,7 +539,9 @@ decode_kernel(const DecodeArgs a) {
                 case 6: phase1_uniform<D, 6>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
                 case 4: phase1_uniform<D, 4>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
                 case 2: phase1_uniform<D, 2>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
-                default: phase1_mixed<D>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
+                case 16: phase1_pivots<D>(sm, meta, a.packed_in + tile_base, warp, lane, Z, pacc, oacc); break;
+                default: phase1_mixed<D>(sm, meta, st.codes, a.packed_in + tile_base, warp, lane, Z, pacc, oacc);
+                         break;
             }
             store_col_partials<D>(sm.red[warp][0], lane, pacc);
             store_col_partials<D>(sm.red[warp][1], lane, oacc);
@@ -548,10 +621,15 @@ decode_kernel(const DecodeArgs a) {
                 const __half rh = scale_to_half(fmaxf(alpha * rsum * (1.0f / D), kHalfMinNormal) * w2.y);
                 a.r_out[static_cast<int64_t>(tile) * D + i] = __half_as_ushort(rh);
                 const float rs = __half2float(rh) * znorm_of(bw);
-                const float e = alpha * rcp_approx(rs);
-                const float g = w2.x * rs;
-                sm.rq[sl] = make_float4(e, e, g * g, g * g);
-                sm.riq[sl] = inv_qmax_of(bw);
+                if (bw == 16) {   // FP16 pivot row: xi = alpha Y, outside the shared column fit
+                    sm.rq[sl] = make_float4(alpha, alpha, 0.f, 0.f);
+                    sm.riq[sl] = 0.f;
+                } else {
+                    const float e = alpha * rcp_approx(rs);
+                    const float g = w2.x * rs;
+                    sm.rq[sl] = make_float4(e, e, g * g, g * g);
+                    sm.riq[sl] = inv_qmax_of(bw);
+                }
             }
             __syncwarp();
         }
@@ -662,7 +740,9 @@ decode_kernel(const DecodeArgs a) {
         {
             float2 f[4];
             load_cols8(sm.colb, cl, f);
-            phase6<D>(meta, a.packed_out + tile_base, warp, lane, ww, Z, f);
+            float2 cc[4];
+            load_cols8(sm.colc, cl, cc);
+            phase6<D>(meta, a.packed_out + tile_base, warp, lane, ww, Z, f, cc);
         }
         if (issued) {   // ordered before their use by the barriers of the next tiles
             sm.stage[sa].beta = next_beta;

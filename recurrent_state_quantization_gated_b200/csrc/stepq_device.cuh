@@ -277,9 +277,20 @@ __device__ __forceinline__ void unpack4(const uint8_t* row, int cl, int b, float
         case 8: unpack4<D, 8>(row, cl, a, c); break;
         case 4: unpack4<D, 4>(row, cl, a, c); break;
         case 2: unpack4<D, 2>(row, cl, a, c); break;
+        case 16: {   // FP16 pivot row: the values themselves
+            const uint2 u = *reinterpret_cast<const uint2*>(row + 8 * cl);
+            a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+            c = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+            break;
+        }
         default: unpack4<D, 6>(row, cl, a, c); break;
     }
     z[0] = a.x; z[1] = a.y; z[2] = c.x; z[3] = c.y;
+}
+
+// An FP16 pivot value: fp32 -> binary16, nearest-even, saturating at +-65504.
+__device__ __forceinline__ __half pivot_half(float x) {
+    return __float2half_rn(fminf(fmaxf(x, -kHalfMax), kHalfMax));
 }
 
 // Store 4 codes already limited to [-q_b, q_b].
@@ -337,24 +348,32 @@ __device__ __forceinline__ int reduced_row(int warp, int lane, int slot, bool& o
     return warp * M::kRowsPerWarp + slot * M::RPW + M::sub_row(lane);
 }
 
-// Exclusive prefix of the row byte sizes (D/8 * b_i) of a tile: done by one warp.
+// Byte offset of every row inside its tile (one warp): the integer rows first, in key order,
+// then the FP16 pivot rows (width 16), in key order. Row i has D/8 * b_i bytes.
 template <int D>
 __device__ __forceinline__ void row_offsets_warp(const uint8_t* bits, uint16_t* roff, int lane) {
     constexpr int RL = D / 32;
-    int loc[RL], sum = 0;
+    int loc[RL], sum_i = 0, sum_p = 0;
 #pragma unroll
     for (int r = 0; r < RL; ++r) {
-        loc[r] = sum;
-        sum += bits[lane * RL + r] * (D / 8);
+        const int b = bits[lane * RL + r];
+        loc[r] = b == 16 ? sum_p : sum_i;
+        (b == 16 ? sum_p : sum_i) += b * (D / 8);
     }
-    int incl = sum;
+    int inc_i = sum_i, inc_p = sum_p;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
+        const int ti = __shfl_up_sync(0xffffffffu, inc_i, o);
+        const int tp = __shfl_up_sync(0xffffffffu, inc_p, o);
+        if (lane >= o) { inc_i += ti; inc_p += tp; }
     }
+    const int total_i = __shfl_sync(0xffffffffu, inc_i, 31);
 #pragma unroll
-    for (int r = 0; r < RL; ++r) roff[lane * RL + r] = static_cast<uint16_t>(incl - sum + loc[r]);
+    for (int r = 0; r < RL; ++r) {
+        const int b = bits[lane * RL + r];
+        const int base = b == 16 ? total_i + inc_p - sum_p : inc_i - sum_i;
+        roff[lane * RL + r] = static_cast<uint16_t>(base + loc[r]);
+    }
 }
 
 // Combine the per-thread column partials of the RPW sub-rows of a warp.

@@ -217,7 +217,7 @@ using namespace stepq;
 extern "C" const char* stepq_last_error(void) { return g_last_error.c_str(); }
 
 extern "C" const char* stepq_build_info(void) {
-    return "libstepq: STEPQuant quantized gated Delta-rule decode; sm_100a; d in {64,128}; widths {2,4,6,8}";
+    return "libstepq: STEPQuant quantized gated Delta-rule decode; sm_100a; d in {64,128}; widths {2,4,6,8} and FP16 pivot rows (16)";
 }
 
 extern "C" int stepq_packed_layout(stepq_dims dims, const uint8_t* bits_host, int64_t* head_off_host,
@@ -232,7 +232,7 @@ extern "C" int stepq_packed_layout(stepq_dims dims, const uint8_t* bits_host, in
         int64_t sum = 0;
         for (int i = 0; i < dims.dk; ++i) {
             const int b = bits_host[static_cast<int64_t>(h) * dims.dk + i];
-            if (b != 2 && b != 4 && b != 6 && b != 8)
+            if (b != 2 && b != 4 && b != 6 && b != 8 && b != 16)
                 return set_error(STEPQ_EUNSUPPORTED, "stepq_packed_layout: bits[%d][%d] = %d", h, i, b);
             sum += b;
         }

@@ -79,9 +79,15 @@ __device__ void fit_tile_regs(TileSmem<D>& sm, const float X[Map<D>::RPT][4], in
         const __half rh = __double2half(rr);
         if (r_out) r_out[i_red] = __half_as_ushort(rh);
         const float rf = __half2float(rh);
-        const float a = 1.0f / (rf * static_cast<float>((1 << (8 - bw)) * qmax_of(bw)));
-        const float ir = 1.0f / (rf * znorm_of(bw));
-        sm.rowa[i_red] = make_float4(a, ir, sm.w[i_red], rf * znorm_of(bw));
+        if (bw == 16) {
+            // FP16 pivot row: no part in the shared column fit (a = 0 leaves the column max
+            // alone, weight 0 leaves the least-squares sums alone).
+            sm.rowa[i_red] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+            const float a = 1.0f / (rf * static_cast<float>((1 << (8 - bw)) * qmax_of(bw)));
+            const float ir = 1.0f / (rf * znorm_of(bw));
+            sm.rowa[i_red] = make_float4(a, ir, sm.w[i_red], rf * znorm_of(bw));
+        }
     }
     __syncwarp();
 
@@ -208,7 +214,7 @@ __global__ void __launch_bounds__(Map<D>::kThreads) pack_kernel(const StateArgs 
     if (tid < D) {
         const int bw = a.bits[h * D + tid];
         const float rf = half_bits_to_float(a.r_in[static_cast<int64_t>(tile) * D + tid]);
-        sm.rowa[tid] = make_float4(0.f, 1.0f / (rf * znorm_of(bw)), 0.f, 0.f);
+        sm.rowa[tid] = make_float4(0.f, bw == 16 ? 0.f : 1.0f / (rf * znorm_of(bw)), 0.f, 0.f);
         sm.colf[tid] = 1.0f / half_bits_to_float(a.c_in[static_cast<int64_t>(tile) * D + tid]);
     }
     float X[M::RPT][4];
@@ -224,6 +230,13 @@ __global__ void __launch_bounds__(Map<D>::kThreads) pack_kernel(const StateArgs 
     for (int r = 0; r < M::RPT; ++r) {
         const int i = M::row(warp, lane, r);
         const int bw = sm.bits[i];
+        if (bw == 16) {   // FP16 pivot row
+            __half2 h01 = __halves2half2(pivot_half(X[r][0]), pivot_half(X[r][1]));
+            __half2 h23 = __halves2half2(pivot_half(X[r][2]), pivot_half(X[r][3]));
+            *reinterpret_cast<uint2*>(out + sm.roff[i] + 8 * cl) =
+                make_uint2(*reinterpret_cast<uint32_t*>(&h01), *reinterpret_cast<uint32_t*>(&h23));
+            continue;
+        }
         const float ir = sm.rowa[i].y;
         int q[4];
 #pragma unroll
@@ -262,7 +275,8 @@ __global__ void __launch_bounds__(Map<D>::kThreads) unpack_kernel(const StateArg
         unpack4<D>(in + sm.roff[i], cl, bw, z);
         float x[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) x[k] = __fmul_rn(__fmul_rn(rf, cf[k]), __fmul_rn(z[k], znorm_of(bw)));
+        for (int k = 0; k < 4; ++k)
+            x[k] = bw == 16 ? z[k] : __fmul_rn(__fmul_rn(rf, cf[k]), __fmul_rn(z[k], znorm_of(bw)));
         *reinterpret_cast<float4*>(S + i * D + 4 * cl) = make_float4(x[0], x[1], x[2], x[3]);
     }
 }
@@ -282,21 +296,30 @@ __global__ void __launch_bounds__(Map<D>::kThreads) distortion_kernel(const Stat
     load_tile<D>(a.S + static_cast<int64_t>(tile) * D * D, warp, lane, X);
     __syncthreads();
     fit_tile_regs<D>(sm, X, warp, lane, nullptr, nullptr);
-    const int qb = qmax_of(a.uniform_bits);
-    const float zn = znorm_of(a.uniform_bits);
     double part[M::RPT];
 #pragma unroll
     for (int r = 0; r < M::RPT; ++r) {
         const int i = M::row(warp, lane, r);
+        const int bw = sm.bits[i];
         const float4 ra = sm.rowa[i];
-        const float rf = ra.w / zn;
         double acc = 0;
+        if (bw == 16) {   // FP16 pivot row: the binary16 rounding error
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int q = quantise(X[r][k], ra.y, sm.colf[4 * cl + k], qb);
-            const float xh = __fmul_rn(__fmul_rn(rf, sm.colc[4 * cl + k]), static_cast<float>(q) * zn);
-            const double e = static_cast<double>(xh) - static_cast<double>(X[r][k]);
-            acc += e * e;
+            for (int k = 0; k < 4; ++k) {
+                const double e = static_cast<double>(__half2float(pivot_half(X[r][k]))) - static_cast<double>(X[r][k]);
+                acc += e * e;
+            }
+        } else {
+            const int qb = qmax_of(bw);
+            const float zn = znorm_of(bw);
+            const float rf = ra.w / zn;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int q = quantise(X[r][k], ra.y, sm.colf[4 * cl + k], qb);
+                const float xh = __fmul_rn(__fmul_rn(rf, sm.colc[4 * cl + k]), static_cast<float>(q) * zn);
+                const double e = static_cast<double>(xh) - static_cast<double>(X[r][k]);
+                acc += e * e;
+            }
         }
         part[r] = acc;
     }
@@ -409,7 +432,7 @@ extern "C" int stepq_calib_distortion(stepq_dims dims, const float* S, const flo
     long long tiles;
     int rc = common_checks(dims, "stepq_calib_distortion", tiles);
     if (rc) return rc;
-    if (b != 2 && b != 4 && b != 6 && b != 8)
+    if (b != 2 && b != 4 && b != 6 && b != 8 && b != 16)
         return set_error(STEPQ_EUNSUPPORTED, "stepq_calib_distortion: width %d", b);
     if (tiles == 0) return set_error(STEPQ_EINVAL, "stepq_calib_distortion: no sample states (B=0)");
     rc = check_ptrs("stepq_calib_distortion",
@@ -428,6 +451,31 @@ extern "C" int stepq_calib_distortion(stepq_dims dims, const float* S, const flo
         distortion_finish_kernel<64><<<dims.H, 64, 0, st>>>(dims.B, dims.H, scratch, w, d_row, d_head);
     }
     return check_launch("stepq_calib_distortion");
+}
+
+extern "C" int stepq_calib_distortion_bits(stepq_dims dims, const float* S, const float* w, const uint8_t* bits,
+                                           double* d_row, double* d_head, double* scratch, void* stream) {
+    const char* fn = "stepq_calib_distortion_bits";
+    clear_error();
+    long long tiles;
+    int rc = common_checks(dims, fn, tiles);
+    if (rc) return rc;
+    if (tiles == 0) return set_error(STEPQ_EINVAL, "%s: no sample states (B=0)", fn);
+    rc = check_ptrs(fn, {{"S", S}, {"w", w}, {"bits", bits}, {"d_row", d_row}, {"d_head", d_head}, {"scratch", scratch}});
+    if (rc) return rc;
+    StateArgs a{};
+    a.H = dims.H; a.S = S; a.w = w; a.bits = bits; a.uniform_bits = 0; a.scratch = scratch;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dims.dk == 128) {
+        rc = launch_state<128>(fn, distortion_kernel<128>, (int)tiles, a, st);
+        if (rc) return rc;
+        distortion_finish_kernel<128><<<dims.H, 128, 0, st>>>(dims.B, dims.H, scratch, w, d_row, d_head);
+    } else {
+        rc = launch_state<64>(fn, distortion_kernel<64>, (int)tiles, a, st);
+        if (rc) return rc;
+        distortion_finish_kernel<64><<<dims.H, 64, 0, st>>>(dims.B, dims.H, scratch, w, d_row, d_head);
+    }
+    return check_launch(fn);
 }
 
 namespace stepq {
@@ -468,7 +516,7 @@ extern "C" int stepq_calib_distortion_static(stepq_dims dims, const float* S, co
     long long tiles;
     int rc = common_checks(dims, fn, tiles);
     if (rc) return rc;
-    if (b != 2 && b != 4 && b != 6 && b != 8) return set_error(STEPQ_EUNSUPPORTED, "%s: width %d", fn, b);
+    if (b != 2 && b != 4 && b != 6 && b != 8 && b != 16) return set_error(STEPQ_EUNSUPPORTED, "%s: width %d", fn, b);
     if (tiles == 0) return set_error(STEPQ_EINVAL, "%s: no sample states (B=0)", fn);
     if (tiles * dims.dk > STEPQ_STATIC_SCRATCH_ROWS)
         return set_error(STEPQ_EINVAL, "%s: B*H*dk = %lld exceeds the static work space of %d entries", fn,

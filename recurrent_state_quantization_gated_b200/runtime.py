@@ -76,13 +76,17 @@ def lifetime(unit_gates) -> np.ndarray:
     return 1.0 / (1.0 - g)
 
 
-def calibrate(alloc: str, candidates, nominal_bits: int, unit_gates, S0: torch.Tensor, calib: dict):
+def calibrate(alloc: str, candidates, nominal_bits: int, unit_gates, S0: torch.Tensor, calib: dict, n_pivots: int = 0):
     """Offline calibration of one layer. Returns (bits uint8 numpy [H][d], w float32 [H][d] on GPU).
 
     alloc: "dp_head" (head units, Eq. 17 distortion, multiple-choice DP) or "lagrange_row"
     (key-row units, Eq. 18 distortion, Lagrangian allocation with repair).
     unit_gates: [H] (head gates) or [H][d] (key-channel gates); S0: the sample states
     [B,H,d,d] on the GPU; calib: the calibration stream as GPU tensors with a leading step axis.
+    n_pivots: units kept in FP16 (width 16; App. C.2): key rows ranked by the lifetime-weighted
+    error reduction L_u (d_u(nominal) - d_u(16)), then the other rows' distortions measured
+    again without the pivots in the column fit; heads ranked by residual risk L_u d_u(b_u)
+    after a first allocation. A pivot counts 8 bits of the integer budget (App. D accounting).
     """
     w = api.stepq_row_impact(calib["q"], calib["k"], calib["beta"], calib["gate"])
     H, d = w.shape
@@ -98,13 +102,39 @@ def calibrate(alloc: str, candidates, nominal_bits: int, unit_gates, S0: torch.T
         g = gates if gates.ndim == 1 else gates.mean(axis=1)
         J = lifetime(g)[:, None] * dist
         bh = api.stepq_allocate_bits(J, cand, nominal_bits * H, mode=1)
+        if n_pivots:
+            risk = J[np.arange(H), [cand.index(int(b)) for b in bh]]
+            piv = np.sort(np.lexsort((np.arange(H), -risk))[:n_pivots])
+            rest = np.setdiff1d(np.arange(H), piv)
+            bh = bh.astype(np.uint8)
+            bh[rest] = api.stepq_allocate_bits(J[rest], cand, nominal_bits * H - 8 * n_pivots, mode=1)
+            bh[piv] = 16
         return np.repeat(bh[:, None], d, axis=1).astype(np.uint8), w
     if alloc == "lagrange_row":
-        dist = np.stack([x.reshape(-1) for x in rows], axis=1)
         g = gates.reshape(-1) if gates.ndim == 2 else np.repeat(gates, d)
-        J = lifetime(g)[:, None] * dist
-        br = api.stepq_allocate_bits(J, cand, nominal_bits * H * d, mode=0)
-        return br.reshape(H, d).astype(np.uint8), w
+        n = H * d
+        L = lifetime(g)
+        if not n_pivots:
+            dist = np.stack([x.reshape(-1) for x in rows], axis=1)
+            br = api.stepq_allocate_bits(L[:, None] * dist, cand, nominal_bits * n, mode=0)
+            return br.reshape(H, d).astype(np.uint8), w
+        d16 = api.stepq_calib_distortion(S0, w, 16)[0].cpu().numpy().reshape(-1)
+        dnom = (rows[cand.index(int(nominal_bits))] if int(nominal_bits) in cand else
+                api.stepq_calib_distortion(S0, w, nominal_bits)[0].cpu().numpy()).reshape(-1)
+        score = L * (dnom - d16)
+        piv = np.sort(np.lexsort((np.arange(n), -score))[:n_pivots])
+        rest = np.setdiff1d(np.arange(n), piv)
+        dist = []
+        for b in cand:
+            m = np.full(n, b, dtype=np.uint8)
+            m[piv] = 16
+            bits_dev = torch.from_numpy(m.reshape(H, d)).to(S0.device)
+            dist.append(api.stepq_calib_distortion_bits(S0, w, bits_dev)[0].cpu().numpy().reshape(-1))
+        dist = np.stack(dist, axis=1)
+        br = np.zeros(n, dtype=np.uint8)
+        br[rest] = api.stepq_allocate_bits(L[rest, None] * dist[rest], cand, nominal_bits * n - 8 * n_pivots, mode=0)
+        br[piv] = 16
+        return br.reshape(H, d), w
     raise ValueError(f"unknown allocation {alloc!r}")
 
 

@@ -52,12 +52,19 @@ class Workload:
     outliers: bool
     v_dist: str           # "normal" | "t3"
     gate_split: bool = False
+    pivot_frac: float = 0.0   # share of allocation units kept as FP16 pivots (App. C.2)
     seed: int = 0
     _cache: dict = field(default_factory=dict, compare=False, repr=False)
 
     @property
     def tiles(self) -> int:
         return self.B * self.H
+
+    @property
+    def n_pivots(self) -> int:
+        """FP16 pivot units of one layer: key rows (row allocation) or heads (head allocation)."""
+        units = self.H * self.d if self.alloc == "lagrange_row" else self.H
+        return int(round(self.pivot_frac * units))
 
 
 _SPECS = [
@@ -67,7 +74,7 @@ _SPECS = [
          nominal_bits=6, candidates=(4, 6, 8), alloc="dp_head", outliers=True, v_dist="normal"),
     dict(name="kda_b256_h32_d128_t128", B=256, H=32, d=128, T=128, gate_per_channel=True,
          nominal_bits=6, candidates=(4, 6, 8), alloc="lagrange_row", outliers=True,
-         v_dist="normal"),
+         v_dist="normal", pivot_frac=512 / 81920),
     dict(name="gdn4_b1024_h16_d128_t64", B=1024, H=16, d=128, T=64, gate_per_channel=False,
          nominal_bits=4, candidates=(2, 4, 8), alloc="lagrange_row", outliers=True,
          v_dist="normal"),

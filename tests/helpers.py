@@ -39,6 +39,15 @@ def tile_codes(packed, bits, d, B):
     return out
 
 
+def with_pivots(bits, n, seed):
+    """A copy of the bit map with n seeded key rows made FP16 pivots (width 16)."""
+    rng = np.random.default_rng(seed)
+    out = bits.copy()
+    flat = out.reshape(-1)
+    flat[rng.choice(flat.size, size=n, replace=False)] = 16
+    return out
+
+
 def half_ulps(a, b):
     """Distance in binary16 units in the last place between two arrays of positive fp16 bits."""
     return np.abs(a.astype(np.int32) - b.astype(np.int32))
@@ -84,9 +93,15 @@ def compare_decode(gpu, ref, bits, d, B, max_frac=1e-3):
     assert c_mis < 1e-2, f"{c_mis:.2e} of column scales differ"
     codes_g = tile_codes(p_g, bits, d, B)
     codes_r = tile_codes(p_r, bits, d, B)
-    diff = np.abs(codes_g.astype(np.int64) - codes_r)
+    piv = np.broadcast_to((bits == 16)[None, :, :, None], codes_g.shape)
+    if piv.any():   # FP16 pivot entries: binary16 values within one unit in the last place
+        vg = codes_g[piv].astype(np.uint16).view(np.float16).astype(np.float64)
+        vr = codes_r[piv].astype(np.uint16).view(np.float16).astype(np.float64)
+        ulp = np.spacing(np.maximum(np.abs(vg), np.abs(vr)).astype(np.float16)).astype(np.float64)
+        assert (np.abs(vg - vr) <= ulp).all(), "pivot values differ by more than one binary16 ulp"
+    diff = np.where(piv, 0, np.abs(codes_g.astype(np.int64) - codes_r))
     assert diff.max() <= 1, f"codes differ by {diff.max()}"
-    same = (r_g == r_r)[..., :, None] & (c_g == c_r)[..., None, :]
+    same = (r_g == r_r)[..., :, None] & (c_g == c_r)[..., None, :] & ~piv
     frac = (diff[same] > 0).mean() if same.any() else 0.0
     assert frac <= max_frac, f"{frac:.2e} of codes with equal scales differ by one step"
     return frac, (r_g != r_r).mean(), c_mis, (diff > 0).mean()

@@ -9,19 +9,19 @@ import pytest
 
 import oracle
 from recurrent_state_quantization_gated_b200 import synth
-from tests.helpers import compare_decode, dev, host_half, tokens_dev
+from tests.helpers import compare_decode, dev, host_half, tokens_dev, with_pivots
 
 pytestmark = pytest.mark.gpu
 
 
-def _setup(d, B, H, widths, gate_per_channel, seed, host=True):
+def _setup(d, B, H, widths, gate_per_channel, seed, host=True, pivots=0):
     """Workload, bits, w, layout and the oracle's initial packed state (host arrays, or
-    device tensors with host=False)."""
+    device tensors with host=False). pivots: key rows made FP16 pivots (width 16)."""
     import torch
     from recurrent_state_quantization_gated_b200 import api
     wl = synth.workload(2 if gate_per_channel else 1, B=B, H=H, d=d, seed=seed)
     S0 = synth.initial_state(wl)
-    bits = synth.random_bits(H, d, choices=widths, seed=seed + 3)
+    bits = with_pivots(synth.random_bits(H, d, choices=widths, seed=seed + 3), pivots, seed + 5)
     w = synth.random_weights(H, d, seed=seed + 4)
     r, c = oracle.fit_scales(S0, w, bits)
     packed = oracle.pack_state(S0, bits, r, c)
@@ -53,18 +53,22 @@ def _check_step(api, wl, bits, w, head_off, bps, st, t, in_place):
     return dict(packed=ref[0], r=ref[1], c=ref[2]), rates
 
 
-@pytest.mark.parametrize("d,B,H,widths,gpc", [
-    (64, 2, 2, (4, 8), False),          # the tiny workload's shape
-    (128, 3, 5, (2, 4, 6, 8), False),   # every width, 15 tiles
-    (128, 2, 7, (4, 6, 8), True),       # channel gates
-    (64, 3, 3, (2, 4, 6, 8), True),
-    (128, 1, 1, (6,), False),           # a single tile
-    (128, 3, 40, (4, 6, 8), False),     # more heads than the kernel's per-head table cache
-    (64, 2, 70, (2, 4, 8), True),
+@pytest.mark.parametrize("d,B,H,widths,gpc,pivots", [
+    (64, 2, 2, (4, 8), False, 0),          # the tiny workload's shape
+    (128, 3, 5, (2, 4, 6, 8), False, 0),   # every width, 15 tiles
+    (128, 2, 7, (4, 6, 8), True, 0),       # channel gates
+    (64, 3, 3, (2, 4, 6, 8), True, 0),
+    (128, 1, 1, (6,), False, 0),           # a single tile
+    (128, 3, 40, (4, 6, 8), False, 0),     # more heads than the kernel's per-head table cache
+    (64, 2, 70, (2, 4, 8), True, 0),
+    (128, 3, 6, (4, 6, 8), True, 13),      # FP16 pivot rows among the integer rows (KDA)
+    (64, 2, 5, (2, 4, 6, 8), False, 21),
+    (128, 2, 3, (16,), False, 0),          # whole pivot heads (every row FP16)
+    (128, 2, 4, (6, 16), False, 0),        # mixed, pivot rows in width-uniform and mixed warps
 ])
-def test_decode_teacher_forced(d, B, H, widths, gpc):
+def test_decode_teacher_forced(d, B, H, widths, gpc, pivots):
     from recurrent_state_quantization_gated_b200 import api
-    wl, bits, w, head_off, bps, st = _setup(d, B, H, widths, gpc, seed=d + B + H)
+    wl, bits, w, head_off, bps, st = _setup(d, B, H, widths, gpc, seed=d + B + H, pivots=pivots)
     rates = []
     for t in range(6):
         st, r = _check_step(api, wl, bits, w, head_off, bps, st, t, in_place=(t % 2 == 0))

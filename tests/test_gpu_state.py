@@ -5,7 +5,7 @@ import pytest
 
 import oracle
 from recurrent_state_quantization_gated_b200 import synth
-from tests.helpers import dev, half_ulps, host_half
+from tests.helpers import dev, half_ulps, host_half, with_pivots
 
 pytestmark = pytest.mark.gpu
 
@@ -15,16 +15,22 @@ def _api():
     return api
 
 
-CASES = [(64, 2, 3, (2, 4, 6, 8)), (128, 3, 5, (2, 4, 6, 8)), (128, 2, 4, (6,)), (64, 5, 1, (8,)),
-         (128, 1, 37, (4, 8))]
+# (d, B, H, widths, FP16 pivot rows added): width 16 in `widths` makes whole pivot heads too
+CASES = [(64, 2, 3, (2, 4, 6, 8), 0), (128, 3, 5, (2, 4, 6, 8), 0), (128, 2, 4, (6,), 0), (64, 5, 1, (8,), 0),
+         (128, 1, 37, (4, 8), 0), (64, 2, 3, (2, 4, 6, 8), 7), (128, 3, 5, (4, 6, 8), 11), (128, 2, 3, (16,), 0),
+         (64, 3, 2, (4, 16), 0)]
 
 
-@pytest.mark.parametrize("d,B,H,widths", CASES)
-def test_pack_unpack_bit_exact(d, B, H, widths):
+def _bits(H, d, widths, npiv, seed):
+    return with_pivots(synth.random_bits(H, d, choices=widths, seed=seed), npiv, seed + 100)
+
+
+@pytest.mark.parametrize("d,B,H,widths,npiv", CASES)
+def test_pack_unpack_bit_exact(d, B, H, widths, npiv):
     import torch
     api = _api()
     S = synth.random_tile_state(B, H, d, seed=d + B + H)
-    bits = synth.random_bits(H, d, choices=widths, seed=H)
+    bits = _bits(H, d, widths, npiv, seed=H)
     w = synth.random_weights(H, d, seed=B)
     r, c = oracle.fit_scales(S, w, bits)                    # scales from the oracle: inputs only
     packed_ref = oracle.pack_state(S, bits, r, c)
@@ -37,11 +43,11 @@ def test_pack_unpack_bit_exact(d, B, H, widths):
                                   oracle.unpack_state(packed_ref, bits, r, c).view(np.uint32))
 
 
-@pytest.mark.parametrize("d,B,H,widths", CASES)
-def test_fit_scales_within_one_ulp(d, B, H, widths):
+@pytest.mark.parametrize("d,B,H,widths,npiv", CASES)
+def test_fit_scales_within_one_ulp(d, B, H, widths, npiv):
     api = _api()
     S = synth.random_tile_state(B, H, d, seed=2 * d + B)
-    bits = synth.random_bits(H, d, choices=widths, seed=H + 1)
+    bits = _bits(H, d, widths, npiv, seed=H + 1)
     w = synth.random_weights(H, d, seed=B + 1)
     r_ref, c_ref = oracle.fit_scales(S, w, bits)
     r, c = api.stepq_fit_scales(dev(S), dev(w), dev(bits))
@@ -101,6 +107,20 @@ def test_calib_distortion_matches_oracle(d):
         np.testing.assert_allclose(dh.cpu().numpy(), dh_ref, rtol=1e-9, atol=0)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_calib_distortion_under_a_bit_map_with_pivots(d):
+    api = _api()
+    S = synth.random_tile_state(3, 4, d, seed=50 + d)
+    w = synth.random_weights(4, d, seed=51)
+    bits = _bits(4, d, (4, 6, 8), 9, seed=52)
+    dr_ref, dh_ref = oracle.calib_distortion_bits(S, w, bits)
+    dr, dh = api.stepq_calib_distortion_bits(dev(S), dev(w), dev(bits))
+    np.testing.assert_allclose(dr.cpu().numpy(), dr_ref, rtol=1e-9, atol=0)
+    np.testing.assert_allclose(dh.cpu().numpy(), dh_ref, rtol=1e-9, atol=0)
+    dr16, _ = api.stepq_calib_distortion(dev(S), dev(w), 16)
+    np.testing.assert_allclose(dr16.cpu().numpy(), oracle.calib_distortion(S, w, 16)[0], rtol=1e-9, atol=0)
+
+
 def test_calibration_allocation_matches_oracle():
     """The whole offline calibration of two synthetic workloads gives the oracle's bit maps."""
     import torch
@@ -109,10 +129,13 @@ def test_calibration_allocation_matches_oracle():
         wl = synth.workload(idx, **over)
         S0 = synth.initial_state(wl)
         cal = synth.calib_tokens(wl)
-        bits_ref, w_ref = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), S0, cal)
+        bits_ref, w_ref = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), S0, cal,
+                                           n_pivots=wl.n_pivots)
         cal_dev = dict(q=dev(cal["q"], torch.bfloat16), k=dev(cal["k"], torch.bfloat16), beta=dev(cal["beta"]),
                        gate=dev(cal["gate"]))
-        bits, w = runtime.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), dev(S0), cal_dev)
+        bits, w = runtime.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), dev(S0), cal_dev,
+                                    n_pivots=wl.n_pivots)
         np.testing.assert_allclose(w.cpu().numpy(), w_ref, rtol=1e-6)
         np.testing.assert_array_equal(bits, bits_ref)
-        assert bits.astype(np.int64).mean() == wl.nominal_bits
+        assert int((bits == 16).sum()) == wl.n_pivots * (1 if wl.alloc == "lagrange_row" else wl.d)
+        assert bits.astype(np.int64).sum() == wl.nominal_bits * bits.size + 8 * int((bits == 16).sum())
