@@ -370,13 +370,14 @@ def main():
         if args.kernel == "split":
             api.stepq_decode_step_split(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
                                         layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
-                                        st["packed"], st["r"], st["c"], o, x_ws, side_stream=side, refit=refit)
+                                        st["packed"], st["r"], st["c"], o, x_ws, side_stream=side, refit=refit,
+                                        pivots=layout.pivots)
             if refit:
                 torch.cuda.current_stream().wait_stream(side)   # writeback done before the next step
         elif args.kernel == "quant":
             api.stepq_decode_step(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
                                   layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
-                                  st["packed"], st["r"], st["c"], o)
+                                  st["packed"], st["r"], st["c"], o, pivots=layout.pivots)
         elif args.kernel == "fp32":
             api.stepq_decode_step_fp32(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], st["S"], st["S"], o)
         else:

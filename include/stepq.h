@@ -70,6 +70,10 @@ typedef struct {
     int dk;                  /* key width (rows of a state tile)             */
     int dv;                  /* value width (columns of a state tile)        */
     int gate_per_channel;    /* 0: gate [B][H]; 1: gate [B][H][dk]           */
+    int pivots;              /* 1: the bit map may hold width-16 (FP16 pivot) rows. Read by the
+                                decode steps, which then run their pivot-capable kernel; a
+                                pivot row met with pivots = 0 raises bit 1 of the device error
+                                word and its results are undefined. Other calls ignore it.  */
 } stepq_dims;
 
 /* Text of the last error raised on the calling thread ("" if none). */
@@ -223,7 +227,8 @@ STEPQ_API int stepq_allocate_bits(int n_units, int n_cand, const int* cand_host,
                         int64_t budget_bits, int mode, uint8_t* bits_out_host);
 
 /* Device error word of the fused decode kernel: bit 0 is set when a bounded wait for a tile
-   copy gave up. Reads (synchronously, on the current device) and clears it. */
+   copy gave up; bit 1 when a width-16 row was met in a launch with dims.pivots = 0. Reads
+   (synchronously, on the current device) and clears it. */
 STEPQ_API int stepq_read_device_flags(uint32_t* flags_host);
 
 /* Build description (compute capability compiled for, and version). */

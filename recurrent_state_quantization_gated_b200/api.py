@@ -43,8 +43,14 @@ def _ptr(t: torch.Tensor, dtype: torch.dtype, name: str):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _dims(B, H, d, gate_per_channel=0):
-    return Dims(int(B), int(H), int(d), int(d), int(gate_per_channel))
+def _dims(B, H, d, gate_per_channel=0, pivots=0):
+    return Dims(int(B), int(H), int(d), int(d), int(gate_per_channel), int(pivots))
+
+
+def _has_pivots(bits, pivots):
+    """The pivots flag of a decode call: as given, else read from the bit map (a device
+    reduction and a host read; pass it to avoid both)."""
+    return int(bool((bits == 16).any().item())) if pivots is None else int(bool(pivots))
 
 
 def stepq_build_info() -> str:
@@ -91,7 +97,7 @@ def stepq_unpack_state(packed, bits, head_off, bytes_per_seq, r, c, S_out=None):
 
 
 def stepq_decode_step(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
-                      packed_out=None, r_out=None, c_out=None, o=None):
+                      packed_out=None, r_out=None, c_out=None, o=None, pivots=None):
     """One fused quantized decode step; outputs may alias the inputs (in-place update).
     Returns (packed_out, r_out, c_out, o)."""
     B, H, d = q.shape
@@ -100,7 +106,8 @@ def stepq_decode_step(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, pac
     r_out = torch.empty_like(r_in) if r_out is None else r_out
     c_out = torch.empty_like(c_in) if c_out is None else c_out
     o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
-    call("stepq_decode_step", _dims(B, H, d, gpc), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+    call("stepq_decode_step", _dims(B, H, d, gpc, _has_pivots(bits, pivots)), _ptr(q, torch.bfloat16, "q"),
+         _ptr(k, torch.bfloat16, "k"),
          _ptr(v, torch.bfloat16, "v"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
          _ptr(bits, torch.uint8, "bits"), _ptr(w, torch.float32, "w"), _ptr(head_off, torch.int64, "head_off"),
          ctypes.c_int64(int(bytes_per_seq)), _ptr(packed_in, torch.uint8, "packed_in"),
@@ -112,7 +119,7 @@ def stepq_decode_step(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, pac
 
 def stepq_decode_step_split(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
                             packed_out=None, r_out=None, c_out=None, o=None, x_ws=None, side_stream=None,
-                            refit=True):
+                            refit=True, pivots=None):
     """The split form: the first kernel (o, X) on the current stream, refit and pack on
     side_stream after it; the current stream then waits for the side stream unless the caller
     passes its own side_stream (and orders it). refit=False runs the first kernel only.
@@ -128,7 +135,8 @@ def stepq_decode_step_split(q, k, v, beta, gate, bits, w, head_off, bytes_per_se
     own = side_stream is None and refit
     side = torch.cuda.Stream() if own else side_stream
     opt = lambda t, dt, n: _ptr(t, dt, n) if t is not None else None
-    call("stepq_decode_step_split", _dims(B, H, d, gpc), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+    call("stepq_decode_step_split", _dims(B, H, d, gpc, _has_pivots(bits, pivots)), _ptr(q, torch.bfloat16, "q"),
+         _ptr(k, torch.bfloat16, "k"),
          _ptr(v, torch.bfloat16, "v"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
          _ptr(bits, torch.uint8, "bits"), _ptr(w, torch.float32, "w"), _ptr(head_off, torch.int64, "head_off"),
          ctypes.c_int64(int(bytes_per_seq)), _ptr(packed_in, torch.uint8, "packed_in"),

@@ -151,7 +151,7 @@ __device__ __forceinline__ bool issue_tile(const DecodeArgs& a, DecodeSmem<D>& s
 __device__ __forceinline__ int cta_tile(int n) { return blockIdx.x + n * gridDim.x; }
 
 // One warp sorts the rows of head h by bit width (stable) into cache entry e.
-template <int D>
+template <int D, bool kPiv>
 __device__ __forceinline__ void sort_head_warp(const DecodeArgs& a, DecodeSmem<D>& sm, int h, int e, int lane) {
     // Width classes in slot order: 2, 4, 6, 8, then 16 (FP16 pivot rows). Byte offsets follow
     // the packed layout: integer rows in key order, then pivot rows in key order.
@@ -202,10 +202,29 @@ __device__ __forceinline__ void sort_head_warp(const DecodeArgs& a, DecodeSmem<D
 #pragma unroll
         for (int c = 0; c < NC; ++c)
             if (c == cls) slot = base_c[c] + excl_c[c] + rank[r];
-        const int off = (piv ? total_i + inc_p - sum_p : inc_i - sum_i) + loc[r];
-        sm.hmeta[e][slot] = static_cast<uint32_t>(i) | (static_cast<uint32_t>(bw[r]) << 8) | (static_cast<uint32_t>(off) << 16);
-        sm.hslot[e][i] = static_cast<uint16_t>(slot | (bw[r] << 8));
+        int off = (piv ? total_i + inc_p - sum_p : inc_i - sum_i) + loc[r];
+        int wb = bw[r];
+        if (!kPiv && piv) {
+            // A pivot row in a launch declared without pivots: flagged (bit 1); the row is
+            // handled as an in-bounds 8-bit row so that nothing is read or written outside
+            // the tile (its results are undefined).
+            atomicOr(&g_stepq_flags, 2u);
+            wb = 8;
+            off = min(off, D * D - D);
+        }
+        sm.hmeta[e][slot] = static_cast<uint32_t>(i) | (static_cast<uint32_t>(wb) << 8) | (static_cast<uint32_t>(off) << 16);
+        sm.hslot[e][i] = static_cast<uint16_t>(slot | (wb << 8));
     }
+}
+
+// Eight consecutive per-column values (columns 8cl .. 8cl+7) as four pairs.
+__device__ __forceinline__ void load_cols8(const float* src, int cl, float2 out[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(src + 8 * cl);
+    const float4 b = *reinterpret_cast<const float4*>(src + 8 * cl + 4);
+    out[0] = make_float2(a.x, a.y);
+    out[1] = make_float2(a.z, a.w);
+    out[2] = make_float2(b.x, b.y);
+    out[3] = make_float2(b.z, b.w);
 }
 
 // ---- phase 1: unpack the thread's rows and accumulate the k^T and q^T products -------------
@@ -222,12 +241,13 @@ __device__ __forceinline__ void phase1_row(const DecodeSmem<D>& sm, const uint8_
     }
 }
 
-// An FP16 pivot row: eight values straight from global memory (pivot rows follow the integer
-// rows of a tile and are not staged), divided by their column scales so that the row joins
-// the tile's factored form X = alpha_i c_j Y_ij with alpha_i = g_i.
+// An FP16 pivot row: eight values, divided by their column scales so that the row joins the
+// tile's factored form X = alpha_i c_j Y_ij with alpha_i = g_i. Pivot rows follow the integer
+// rows of a tile: those inside the staged first d*d bytes are read from shared memory, the
+// rest from global memory (a generic load serves both).
 template <int D>
-__device__ __forceinline__ void load_pivot8(const uint8_t* row_g, int cl, const float* icol, float2 z[4]) {
-    const uint4 u = *reinterpret_cast<const uint4*>(row_g + 16 * cl);
+__device__ __forceinline__ void load_pivot8(const uint8_t* row, int cl, const float* icol, float2 z[4]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(row + 16 * cl);
     const float4 i0 = *reinterpret_cast<const float4*>(icol + 8 * cl);
     const float4 i1 = *reinterpret_cast<const float4*>(icol + 8 * cl + 4);
     z[0] = mul2(__half22float2(*reinterpret_cast<const __half2*>(&u.x)), make_float2(i0.x, i0.y));
@@ -237,9 +257,11 @@ __device__ __forceinline__ void load_pivot8(const uint8_t* row_g, int cl, const 
 }
 
 template <int D>
-__device__ __forceinline__ void phase1_pivot_row(const DecodeSmem<D>& sm, const uint8_t* gin, int s, uint32_t mt,
-                                                 int cl, float2 z[4], float2 pacc[4], float2 oacc[4]) {
-    load_pivot8<D>(gin + (mt >> 16), cl, sm.icol, z);
+__device__ __forceinline__ void phase1_pivot_row(const DecodeSmem<D>& sm, const uint8_t* codes, const uint8_t* gin,
+                                                 int s, uint32_t mt, int cl, float2 z[4], float2 pacc[4],
+                                                 float2 oacc[4]) {
+    const uint32_t off = mt >> 16;
+    load_pivot8<D>((off + 2 * D <= D * D ? codes : gin) + off, cl, sm.icol, z);
     const float4 c = sm.kq[s];
     const float2 kap = make_float2(c.x, c.y), lam = make_float2(c.z, c.w);
 #pragma unroll
@@ -250,14 +272,15 @@ __device__ __forceinline__ void phase1_pivot_row(const DecodeSmem<D>& sm, const 
 }
 
 template <int D>
-__device__ __forceinline__ void phase1_pivots(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* gin,
-                                              int warp, int lane, float2 Z[][4], float2 pacc[4], float2 oacc[4]) {
+__device__ __forceinline__ void phase1_pivots(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* codes,
+                                              const uint8_t* gin, int warp, int lane, float2 Z[][4], float2 pacc[4],
+                                              float2 oacc[4]) {
     using M = DMap<D>;
     const int cl = M::col_lane(lane);
 #pragma unroll
     for (int r = 0; r < M::RPT; ++r) {
         const int s = M::row(warp, lane, r);
-        phase1_pivot_row<D>(sm, gin, s, meta[s], cl, Z[r], pacc, oacc);
+        phase1_pivot_row<D>(sm, codes, gin, s, meta[s], cl, Z[r], pacc, oacc);
     }
 }
 
@@ -287,7 +310,7 @@ __device__ __forceinline__ void phase1_uniform(const DecodeSmem<D>& sm, const ui
     }
 }
 
-template <int D>
+template <int D, bool kPiv>
 __device__ __forceinline__ void phase1_mixed(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* codes,
                                              const uint8_t* gin, int warp, int lane, float2 Z[][4], float2 pacc[4],
                                              float2 oacc[4]) {
@@ -301,8 +324,15 @@ __device__ __forceinline__ void phase1_mixed(const DecodeSmem<D>& sm, const uint
             case 8: phase1_row<D, 8>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
             case 6: phase1_row<D, 6>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
             case 4: phase1_row<D, 4>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
-            case 16: phase1_pivot_row<D>(sm, gin, s, mt, cl, Z[r], pacc, oacc); break;
-            default: phase1_row<D, 2>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
+            default:
+                if constexpr (kPiv) {
+                    if (((mt >> 8) & 0xFF) == 16) {
+                        phase1_pivot_row<D>(sm, codes, gin, s, mt, cl, Z[r], pacc, oacc);
+                        break;
+                    }
+                }
+                phase1_row<D, 2>(sm, codes, s, mt, cl, Z[r], pacc, oacc);
+                break;
         }
     }
 }
@@ -339,9 +369,11 @@ __device__ __forceinline__ void phase6_pivot_row(uint8_t* out, uint32_t mt, int 
 
 template <int D, int BW>
 __device__ __forceinline__ void phase6_uniform(const uint32_t* meta, uint8_t* out, int warp, int lane,
-                                               const float2 Z[][4], const float2 f[4], const float2 cc[4]) {
+                                               const float2 Z[][4], const float2 f[4], const float* colc) {
     using M = DMap<D>;
     const int cl = M::col_lane(lane);
+    float2 cc[4];
+    if constexpr (BW == 16) load_cols8(colc, cl, cc);
 #pragma unroll
     for (int r = 0; r < M::RPT; ++r) {
         if constexpr (BW == 16) phase6_pivot_row<D>(out, meta[M::row(warp, lane, r)], cl, Z[r], cc);
@@ -349,11 +381,13 @@ __device__ __forceinline__ void phase6_uniform(const uint32_t* meta, uint8_t* ou
     }
 }
 
-template <int D>
+template <int D, bool kPiv>
 __device__ __forceinline__ void phase6_mixed(const uint32_t* meta, uint8_t* out, int warp, int lane,
-                                             const float2 Z[][4], const float2 f[4], const float2 cc[4]) {
+                                             const float2 Z[][4], const float2 f[4], const float* colc) {
     using M = DMap<D>;
     const int cl = M::col_lane(lane);
+    float2 cc[4] = {};
+    if constexpr (kPiv) load_cols8(colc, cl, cc);
 #pragma unroll
     for (int r = 0; r < M::RPT; ++r) {
         const uint32_t mt = meta[M::row(warp, lane, r)];
@@ -361,22 +395,58 @@ __device__ __forceinline__ void phase6_mixed(const uint32_t* meta, uint8_t* out,
             case 8: phase6_row<D, 8>(out, mt, cl, Z[r], f); break;
             case 6: phase6_row<D, 6>(out, mt, cl, Z[r], f); break;
             case 4: phase6_row<D, 4>(out, mt, cl, Z[r], f); break;
-            case 16: phase6_pivot_row<D>(out, mt, cl, Z[r], cc); break;
-            default: phase6_row<D, 2>(out, mt, cl, Z[r], f); break;
+            default:
+                if constexpr (kPiv) {
+                    if (((mt >> 8) & 0xFF) == 16) {
+                        phase6_pivot_row<D>(out, mt, cl, Z[r], cc);
+                        break;
+                    }
+                }
+                phase6_row<D, 2>(out, mt, cl, Z[r], f);
+                break;
         }
     }
 }
 
-template <int D>
+// kPiv: the pivot-capable instantiation (width-16 rows handled); without it the code is leaner.
+template <int D, bool kPiv>
 __device__ __forceinline__ void phase6(const uint32_t* meta, uint8_t* out, int warp, int lane, int ww,
-                                       const float2 Z[][4], const float2 f[4], const float2 cc[4]) {
+                                       const float2 Z[][4], const float2 f[4], const float* colc) {
     switch (ww) {
-        case 8: phase6_uniform<D, 8>(meta, out, warp, lane, Z, f, cc); break;
-        case 6: phase6_uniform<D, 6>(meta, out, warp, lane, Z, f, cc); break;
-        case 4: phase6_uniform<D, 4>(meta, out, warp, lane, Z, f, cc); break;
-        case 2: phase6_uniform<D, 2>(meta, out, warp, lane, Z, f, cc); break;
-        case 16: phase6_uniform<D, 16>(meta, out, warp, lane, Z, f, cc); break;
-        default: phase6_mixed<D>(meta, out, warp, lane, Z, f, cc); break;
+        case 8: phase6_uniform<D, 8>(meta, out, warp, lane, Z, f, colc); break;
+        case 6: phase6_uniform<D, 6>(meta, out, warp, lane, Z, f, colc); break;
+        case 4: phase6_uniform<D, 4>(meta, out, warp, lane, Z, f, colc); break;
+        case 2: phase6_uniform<D, 2>(meta, out, warp, lane, Z, f, colc); break;
+        default:
+            if constexpr (kPiv) {
+                if (ww == 16) {
+                    phase6_uniform<D, 16>(meta, out, warp, lane, Z, f, colc);
+                    break;
+                }
+            }
+            phase6_mixed<D, kPiv>(meta, out, warp, lane, Z, f, colc);
+            break;
+    }
+}
+
+template <int D, bool kPiv>
+__device__ __forceinline__ void phase1(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* codes,
+                                       const uint8_t* gin, int warp, int lane, int ww, float2 Z[][4],
+                                       float2 pacc[4], float2 oacc[4]) {
+    switch (ww) {
+        case 8: phase1_uniform<D, 8>(sm, meta, codes, warp, lane, Z, pacc, oacc); break;
+        case 6: phase1_uniform<D, 6>(sm, meta, codes, warp, lane, Z, pacc, oacc); break;
+        case 4: phase1_uniform<D, 4>(sm, meta, codes, warp, lane, Z, pacc, oacc); break;
+        case 2: phase1_uniform<D, 2>(sm, meta, codes, warp, lane, Z, pacc, oacc); break;
+        default:
+            if constexpr (kPiv) {
+                if (ww == 16) {
+                    phase1_pivots<D>(sm, meta, codes, gin, warp, lane, Z, pacc, oacc);
+                    break;
+                }
+            }
+            phase1_mixed<D, kPiv>(sm, meta, codes, gin, warp, lane, Z, pacc, oacc);
+            break;
     }
 }
 
@@ -396,66 +466,19 @@ __device__ __forceinline__ void store_col_partials(float* dst, int lane, float2 
     }
 }
 
-__device__ __forceinline__ void load_cols8(const float* src, int cl, float2 out[4]) {
-    const float4 a = *reinterpret_cast<const float4*>(src + 8 * cl);
-    const float4 b = *reinterpret_cast<const float4*>(src + 8 * cl + 4);
-    out[0] = make_float2(a.x, a.y);
-    out[1] = make_float2(a.z, a.w);
-    out[2] = make_float2(b.x, b.y);
-    out[3] = make_float2(b.z, b.w);
-}
-
-// kSplit: the first kernel of the split form. It reconstructs, updates and reads out like the
-// fused step, then writes the updated state X in fp32 and stops; the refit and the pack run
-// as separate kernels (stepq_decode_step_split).
-template <int D, bool kSplit = false>
-__global__ void __launch_bounds__(DMap<D>::kThreads, DMap<D>::kMinBlocks)
-decode_kernel(const DecodeArgs a) {
+// The tile loop of the decode kernel. kPiv: the bit map may hold FP16 pivot rows (declared by
+// the caller in stepq_dims.pivots); launches without them run the leaner instantiation. A
+// width-16 row met in a launch declared without pivots raises bit 1 of the device error word.
+template <int D, bool kSplit, bool kPiv>
+__device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm) {
     using M = DMap<D>;
     constexpr int RPT = M::RPT;
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    DecodeSmem<D>& sm = *reinterpret_cast<DecodeSmem<D>*>(smem_raw);
-
+    constexpr int CH = HeadCache<D>::kHeads;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int cl = M::col_lane(lane);
     const float2 M2 = make_float2(kRoundMagic, kRoundMagic);
-    // The last thread queues the copies (no prologue work waits on it).
     const bool issuer = (tid == M::kThreads - 1);
-
-    // The first tiles' copies go out before anything else, so the HBM latency overlaps the
-    // per-head table set-up.
-    constexpr int CH = HeadCache<D>::kHeads;
-    if (issuer) {
-        for (int i = 0; i < kStages; ++i) mbar_init(&sm.full[i], 1);
-        fence_barrier_init();
-        for (int i = 0; i + 1 < kStages; ++i) {
-            float b0, g0;
-            if (issue_tile<D>(a, sm, cta_tile(i), i, b0, g0)) {
-                sm.stage[i].beta = b0;
-                sm.stage[i].gate1 = g0;
-            }
-        }
-    }
-    // Per-head tables (the bit map is frozen and shared by all sequences): the heads of the
-    // CTA's first tiles are sorted up front, one warp per head; the rest on first use.
-    for (int e = tid; e < CH; e += M::kThreads) sm.htag[e] = -1;
-    __syncthreads();
-    for (int n = warp; n < CH; n += M::kWarps) {
-        const int tile = cta_tile(n);
-        if (tile >= a.num_tiles) break;
-        const int h = tile % a.H;
-        // Sort here only if no earlier tile of this CTA uses the same head or the same entry.
-        bool take = true;
-        for (int m = 0; m < n; ++m)
-            if ((cta_tile(m) % a.H) % CH == h % CH) take = false;
-        if (take) {
-            sort_head_warp<D>(a, sm, h, h % CH, lane);
-            if (lane == 0) sm.htag[h % CH] = h;
-        }
-    }
-    __syncthreads();
-
     for (int n = 0;; ++n) {
         const int tile = cta_tile(n);
         if (tile >= a.num_tiles) break;
@@ -468,7 +491,7 @@ decode_kernel(const DecodeArgs a) {
         if (sm.htag[he] != h) {                     // every warp sees the same tag: uniform branch
             __syncthreads();                        // nobody still reads the entry
             if (warp == 0) {
-                sort_head_warp<D>(a, sm, h, he, lane);
+                sort_head_warp<D, kPiv>(a, sm, h, he, lane);
                 if (lane == 0) sm.htag[he] = h;
             }
             __syncthreads();
@@ -484,7 +507,7 @@ decode_kernel(const DecodeArgs a) {
                 const float g = a.gate_per_channel ? st.gate[i] : st.gate1;
                 // alpha > 0 always (a zero gate leaves 2^-64: far below any term that counts);
                 // an FP16 pivot row carries its values, so alpha is the gate alone.
-                const float alpha = fmaxf(bw == 16 ? g : g * half_bits_to_float(st.r[i]) * znorm_of(bw), 0x1p-64f);
+                const float alpha = fmaxf(kPiv && bw == 16 ? g : g * half_bits_to_float(st.r[i]) * znorm_of(bw), 0x1p-64f);
                 const float kk = bf16_bits_to_float(st.k[i]);
                 const float qq = bf16_bits_to_float(st.q[i]);
                 const float wi = st.w[i];
@@ -492,7 +515,7 @@ decode_kernel(const DecodeArgs a) {
                 sm.kq[sl] = make_float4(alpha * kk, alpha * kk, alpha * qq, alpha * qq);
                 sm.ak[sl] = make_float4(ka, ka, alpha, alpha);
                 sm.wsl[sl] = make_float2(wi, rcp_approx(wi));
-                sm.icol[i] = rcp_approx(half_bits_to_float(st.c[i]));   // column i
+                if constexpr (kPiv) sm.icol[i] = rcp_approx(half_bits_to_float(st.c[i]));   // column i
             } else if (warp == D / 32) {
                 constexpr int RL = D / 32;
                 float acc = 0.f;
@@ -534,15 +557,7 @@ decode_kernel(const DecodeArgs a) {
             float2 pacc[4], oacc[4];
 #pragma unroll
             for (int p = 0; p < 4; ++p) pacc[p] = oacc[p] = make_float2(0.f, 0.f);
-            switch (ww) {
-                case 8: phase1_uniform<D, 8>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
-                case 6: phase1_uniform<D, 6>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
-                case 4: phase1_uniform<D, 4>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
-                case 2: phase1_uniform<D, 2>(sm, meta, st.codes, warp, lane, Z, pacc, oacc); break;
-                case 16: phase1_pivots<D>(sm, meta, a.packed_in + tile_base, warp, lane, Z, pacc, oacc); break;
-                default: phase1_mixed<D>(sm, meta, st.codes, a.packed_in + tile_base, warp, lane, Z, pacc, oacc);
-                         break;
-            }
+            phase1<D, kPiv>(sm, meta, st.codes, a.packed_in + tile_base, warp, lane, ww, Z, pacc, oacc);
             store_col_partials<D>(sm.red[warp][0], lane, pacc);
             store_col_partials<D>(sm.red[warp][1], lane, oacc);
         }
@@ -621,7 +636,7 @@ decode_kernel(const DecodeArgs a) {
                 const __half rh = scale_to_half(fmaxf(alpha * rsum * (1.0f / D), kHalfMinNormal) * w2.y);
                 a.r_out[static_cast<int64_t>(tile) * D + i] = __half_as_ushort(rh);
                 const float rs = __half2float(rh) * znorm_of(bw);
-                if (bw == 16) {   // FP16 pivot row: xi = alpha Y, outside the shared column fit
+                if (kPiv && bw == 16) {   // FP16 pivot row: xi = alpha Y, outside the shared column fit
                     sm.rq[sl] = make_float4(alpha, alpha, 0.f, 0.f);
                     sm.riq[sl] = 0.f;
                 } else {
@@ -740,9 +755,7 @@ decode_kernel(const DecodeArgs a) {
         {
             float2 f[4];
             load_cols8(sm.colb, cl, f);
-            float2 cc[4];
-            load_cols8(sm.colc, cl, cc);
-            phase6<D>(meta, a.packed_out + tile_base, warp, lane, ww, Z, f, cc);
+            phase6<D, kPiv>(meta, a.packed_out + tile_base, warp, lane, ww, Z, f, sm.colc);
         }
         if (issued) {   // ordered before their use by the barriers of the next tiles
             sm.stage[sa].beta = next_beta;
@@ -751,7 +764,61 @@ decode_kernel(const DecodeArgs a) {
     }
 }
 
-template <int D, bool kSplit = false>
+// kSplit: the first kernel of the split form. It reconstructs, updates and reads out like the
+// fused step, then writes the updated state X in fp32 and stops; the refit and the pack run
+// as separate kernels (stepq_decode_step_split).
+template <int D, bool kSplit, bool kPiv>
+__global__ void __launch_bounds__(DMap<D>::kThreads, DMap<D>::kMinBlocks)
+decode_kernel(const DecodeArgs a) {
+    using M = DMap<D>;
+    constexpr int RPT = M::RPT;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    DecodeSmem<D>& sm = *reinterpret_cast<DecodeSmem<D>*>(smem_raw);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int cl = M::col_lane(lane);
+    const float2 M2 = make_float2(kRoundMagic, kRoundMagic);
+    // The last thread queues the copies (no prologue work waits on it).
+    const bool issuer = (tid == M::kThreads - 1);
+
+    // The first tiles' copies go out before anything else, so the HBM latency overlaps the
+    // per-head table set-up.
+    constexpr int CH = HeadCache<D>::kHeads;
+    if (issuer) {
+        for (int i = 0; i < kStages; ++i) mbar_init(&sm.full[i], 1);
+        fence_barrier_init();
+        for (int i = 0; i + 1 < kStages; ++i) {
+            float b0, g0;
+            if (issue_tile<D>(a, sm, cta_tile(i), i, b0, g0)) {
+                sm.stage[i].beta = b0;
+                sm.stage[i].gate1 = g0;
+            }
+        }
+    }
+    // Per-head tables (the bit map is frozen and shared by all sequences): the heads of the
+    // CTA's first tiles are sorted up front, one warp per head; the rest on first use.
+    for (int e = tid; e < CH; e += M::kThreads) sm.htag[e] = -1;
+    __syncthreads();
+    for (int n = warp; n < CH; n += M::kWarps) {
+        const int tile = cta_tile(n);
+        if (tile >= a.num_tiles) break;
+        const int h = tile % a.H;
+        // Sort here only if no earlier tile of this CTA uses the same head or the same entry.
+        bool take = true;
+        for (int m = 0; m < n; ++m)
+            if ((cta_tile(m) % a.H) % CH == h % CH) take = false;
+        if (take) {
+            sort_head_warp<D, kPiv>(a, sm, h, h % CH, lane);
+            if (lane == 0) sm.htag[h % CH] = h;
+        }
+    }
+    __syncthreads();
+
+    run_tiles<D, kSplit, kPiv>(a, sm);
+}
+
+template <int D, bool kSplit, bool kPiv>
 static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     static int ctas_per_sm = -1, num_sms = 0;
     const size_t smem = sizeof(DecodeSmem<D>);
@@ -759,17 +826,17 @@ static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, kSplit, kPiv>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "stepq_decode_step: %s", cudaGetErrorString(e));
         int occ = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D, kSplit>, DMap<D>::kThreads, smem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D, kSplit, kPiv>, DMap<D>::kThreads, smem);
         ctas_per_sm = occ > 0 ? occ : 1;
     }
     if (a.num_tiles == 0) return STEPQ_OK;
     int grid = num_sms * ctas_per_sm;
     if (grid > a.num_tiles) grid = a.num_tiles;
-    decode_kernel<D, kSplit><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
+    decode_kernel<D, kSplit, kPiv><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
     return check_launch("stepq_decode_step");
 }
 
@@ -816,7 +883,8 @@ extern "C" int stepq_decode_step(stepq_dims dims, const uint16_t* q, const uint1
     DecodeArgs a{dims.B, dims.H, dims.gate_per_channel, static_cast<int>(tiles), q, k, v, beta, gate, bits, w,
                  head_off, bytes_per_seq, packed_in, r_in, c_in, packed_out, r_out, c_out, o, nullptr};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return dims.dk == 128 ? launch_decode<128>(a, st) : launch_decode<64>(a, st);
+    if (dims.pivots) return dims.dk == 128 ? launch_decode<128, false, true>(a, st) : launch_decode<64, false, true>(a, st);
+    return dims.dk == 128 ? launch_decode<128, false, false>(a, st) : launch_decode<64, false, false>(a, st);
 }
 
 extern "C" int stepq_decode_step_split(stepq_dims dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -846,7 +914,8 @@ extern "C" int stepq_decode_step_split(stepq_dims dims, const uint16_t* q, const
     DecodeArgs a{dims.B, dims.H, dims.gate_per_channel, static_cast<int>(tiles), q, k, v, beta, gate, bits, w,
                  head_off, bytes_per_seq, packed_in, r_in, c_in, nullptr, nullptr, nullptr, o, x_ws};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = dims.dk == 128 ? launch_decode<128, true>(a, st) : launch_decode<64, true>(a, st);
+    if (dims.pivots) rc = dims.dk == 128 ? launch_decode<128, true, true>(a, st) : launch_decode<64, true, true>(a, st);
+    else rc = dims.dk == 128 ? launch_decode<128, true, false>(a, st) : launch_decode<64, true, false>(a, st);
     if (rc || !refit) return rc;
     // Refit and pack on the side stream, after the first kernel.
     cudaStream_t side = static_cast<cudaStream_t>(side_stream);
@@ -856,7 +925,7 @@ extern "C" int stepq_decode_step_split(stepq_dims dims, const uint16_t* q, const
     cudaError_t e = cudaEventRecord(ev, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev, 0);
     if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "%s: %s", fn, cudaGetErrorString(e));
-    stepq_dims fd{dims.B, dims.H, dims.dk, dims.dv, 0};
+    stepq_dims fd{dims.B, dims.H, dims.dk, dims.dv, 0, dims.pivots};
     rc = stepq_fit_scales(fd, x_ws, w, bits, r_out, c_out, side_stream);
     if (rc) return rc;
     return stepq_pack_state(fd, x_ws, bits, head_off, bytes_per_seq, r_out, c_out, packed_out, side_stream);

@@ -36,6 +36,11 @@ class Layout:
     def H(self) -> int:
         return self.bits.shape[0]
 
+    @property
+    def pivots(self) -> int:
+        """1 when the bit map holds FP16 pivot rows (width 16)."""
+        return int((self.bits == 16).any())
+
 
 class QuantizedState:
     """Packed states of B sequences x H heads (one layer)."""
@@ -63,7 +68,7 @@ class QuantizedState:
         L = self.layout
         _, _, _, o = api.stepq_decode_step(q, k, v, beta, gate, L.bits_dev, self.w, L.head_off_dev,
                                            L.bytes_per_seq, self.packed, self.r, self.c,
-                                           self.packed, self.r, self.c, o)
+                                           self.packed, self.r, self.c, o, pivots=L.pivots)
         return o
 
     def nbytes(self) -> int:

@@ -140,3 +140,22 @@ def test_device_error_word_is_clear_after_decodes():
     api.stepq_decode_step(td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w), dev(head_off), bps,
                           st["packed"], st["r"], st["c"])
     assert api.stepq_read_device_flags() == 0
+
+
+def test_undeclared_pivot_rows_raise_the_device_flag():
+    """A bit map with FP16 pivot rows decoded with dims.pivots = 0: the kernel keeps every
+    access inside the tile and raises bit 1 of the device error word."""
+    import torch
+    from recurrent_state_quantization_gated_b200 import api
+    wl, bits, w, head_off, bps, st = _setup(128, 2, 3, (4, 16), False, seed=12, host=False)
+    assert (bits == 16).any()
+    td = tokens_dev(synth.tokens(wl, 0))
+    assert api.stepq_read_device_flags() == 0
+    api.stepq_decode_step(td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w), dev(head_off), bps,
+                          st["packed"], st["r"], st["c"], pivots=0)
+    torch.cuda.synchronize()
+    assert api.stepq_read_device_flags() == 2
+    api.stepq_decode_step(td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w), dev(head_off), bps,
+                          st["packed"], st["r"], st["c"], pivots=1)
+    torch.cuda.synchronize()
+    assert api.stepq_read_device_flags() == 0
