@@ -232,6 +232,25 @@ def decode_step(tok, bits, w, packed, r, c, nthreads=0):
     return p_out, r_out, c_out, o
 
 
+def prefill_chunk(toks, bits, w, packed, r, c, nthreads=0):
+    """A prefill chunk: toks holds q, k, v, beta, gate with a leading token axis [C][B][H]...;
+    returns (packed_out, r_out, c_out, o [C][B][H][dv])."""
+    q = _c(toks["q"], np.uint16); k = _c(toks["k"], np.uint16); v = _c(toks["v"], np.uint16)
+    beta = _c(toks["beta"], np.float32); gate = _c(toks["gate"], np.float32)
+    bits = _c(bits, np.uint8); w = _c(w, np.float32)
+    packed = _c(packed, np.uint8); r = _c(r, np.uint16); c = _c(c, np.uint16)
+    C, B, H, dk = q.shape
+    dv = v.shape[3]
+    gpc = int(gate.ndim == 4)
+    head_off, bps = layout(bits, dv)
+    p_out = np.zeros_like(packed); r_out = np.zeros_like(r); c_out = np.zeros_like(c)
+    o = np.zeros((C, B, H, dv), dtype=np.float32)
+    _check(lib().orc_prefill_chunk(C, B, H, dk, dv, gpc, _p(q), _p(k), _p(v), _p(beta), _p(gate), _p(bits),
+                                   _p(w), _p(head_off), ctypes.c_int64(bps), _p(packed), _p(r), _p(c),
+                                   _p(p_out), _p(r_out), _p(c_out), _p(o), nthreads), "prefill_chunk")
+    return p_out, r_out, c_out, o
+
+
 def decode_step_fp32(tok, S, nthreads=0):
     q = _c(tok["q"], np.uint16); k = _c(tok["k"], np.uint16); v = _c(tok["v"], np.uint16)
     beta = _c(tok["beta"], np.float32); gate = _c(tok["gate"], np.float32)

@@ -584,6 +584,50 @@ int orc_decode_step(int B, int H, int dk, int dv, int gate_per_channel, const ui
     return ORC_OK;
 }
 
+/* A prefill chunk of C tokens on the packed state (App. F.1: the native chunk update runs on
+   the unpacked state and the boundary state is packed once; App. B.2): reconstruct S_hat,
+   apply the gated Delta rule C times in double (each readout o_t = X_t^T q_t), then fit and
+   pack the final state once. Inputs carry a leading token axis: q, k [C][B][H][dk], v
+   [C][B][H][dv], beta [C][B][H], gate [C][B][H] or [C][B][H][dk]; o [C][B][H][dv]. */
+int orc_prefill_chunk(int C, int B, int H, int dk, int dv, int gate_per_channel, const uint16_t* q,
+                      const uint16_t* k, const uint16_t* v, const float* beta, const float* gate,
+                      const uint8_t* bits, const float* w, const int64_t* head_off,
+                      int64_t bytes_per_seq, const uint8_t* packed_in, const uint16_t* r_in,
+                      const uint16_t* c_in, uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out,
+                      float* o, int nthreads) {
+    if (!orc_dims_ok(dk, dv)) return ORC_EUNSUPPORTED;
+    if (C < 1) return ORC_EINVAL;
+    int nt = set_threads(nthreads);
+    int64_t n = (int64_t)B * H;
+    int gstride = gate_per_channel ? dk : 1;
+    (void)nt;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (int64_t tl = 0; tl < n; ++tl) {
+        int64_t b = tl / H;
+        int h = (int)(tl % H);
+        int64_t off = b * bytes_per_seq + head_off[h];
+        const uint8_t* bh = bits + (int64_t)h * dk;
+        orc_tile_scratch t;
+        scratch_alloc(&t, dk, dv);
+        float* S32 = (float*)malloc(sizeof(float) * dk * dv);
+        orc_unpack_tile(dk, dv, packed_in + off, bh, r_in + tl * dk, c_in + tl * dv, S32);
+        for (int e = 0; e < dk * dv; ++e) t.S[e] = S32[e];
+        for (int c = 0; c < C; ++c) {
+            int64_t tc = (int64_t)c * n + tl;
+            tile_inputs(&t, q + tc * dk, k + tc * dk, v + tc * dv, gate + tc * gstride, gate_per_channel);
+            orc_delta_update(dk, dv, t.S, t.q, t.k, t.v, (double)beta[tc], t.g, t.X, t.o);
+            for (int j = 0; j < dv; ++j) o[tc * dv + j] = (float)t.o[j];
+            memcpy(t.S, t.X, sizeof(double) * dk * dv);            /* full precision in between */
+        }
+        for (int e = 0; e < dk * dv; ++e) S32[e] = (float)t.X[e];
+        orc_fit_tile(dk, dv, S32, w + (int64_t)h * dk, bh, r_out + tl * dk, c_out + tl * dv);
+        orc_pack_tile(dk, dv, S32, bh, r_out + tl * dk, c_out + tl * dv, packed_out + off);
+        free(S32);
+        scratch_free(&t);
+    }
+    return ORC_OK;
+}
+
 int orc_decode_step_fp32(int B, int H, int dk, int dv, int gate_per_channel, const uint16_t* q,
                          const uint16_t* k, const uint16_t* v, const float* beta, const float* gate,
                          const float* S_in, float* S_out, float* o, int nthreads) {
