@@ -50,8 +50,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--cpu-threads", type=int, default=0, help="oracle threads for cpu_baseline (0 = all cores)")
-    ap.add_argument("--kernel", choices=["quant", "split", "fp32", "int8"], default="quant",
-                    help="quant: the fused step; split: the split-form ablation; fp32 / int8: comparison states")
+    ap.add_argument("--kernel", choices=["quant", "split", "prefill", "fp32", "int8"], default="quant",
+                    help="quant: the fused step; split: the split-form ablation; prefill: a chunk of --chunk "
+                         "tokens per launch; fp32 / int8: comparison states")
+    ap.add_argument("--chunk", type=int, default=64, help="tokens per prefill chunk (--kernel prefill)")
     ap.add_argument("--e2e-steps", type=int, default=400)
     return ap.parse_args()
 
@@ -194,6 +196,9 @@ def algorithmic_bytes(layout_bps: int, B: int, H: int, d: int, gate_per_channel:
     small = tiles * (qkv + 4 + gate + 4 * d)
     if kernel == "quant":
         return 2 * B * layout_bps + tiles * 2 * (2 * d + 2 * d) + small
+    if kernel.startswith("prefill"):   # the state once per chunk; every token's inputs and readout
+        C = int(kernel.split(":")[1])
+        return 2 * B * layout_bps + tiles * 2 * (2 * d + 2 * d) + C * small
     if kernel == "split":   # the fused step's bytes + X written, read by the fit, read by the pack + r, c re-read
         return 2 * B * layout_bps + tiles * 2 * (2 * d + 2 * d) + small + tiles * (3 * 4 * d * d + 4 * d)
     if kernel == "int8":
@@ -218,8 +223,9 @@ def job_throughput(world: int, tiles_per_rank: int, steps: int, ms: float) -> fl
     return world * tiles_per_rank * steps / (ms * 1e-3)
 
 
-def workload_config(wl, bits, kernel: str, world: int) -> dict:
-    return {"workload": wl.name, "kernel": kernel, "B": wl.B, "H": wl.H, "d_k": wl.d, "d_v": wl.d,
+def workload_config(wl, bits, kernel: str, world: int, chunk: int = 1) -> dict:
+    extra = {"chunk": chunk} if kernel == "prefill" else {}
+    return {"workload": wl.name, "kernel": kernel, **extra, "B": wl.B, "H": wl.H, "d_k": wl.d, "d_v": wl.d,
             "bits_mean": float(np.asarray(bits, dtype=np.float64).mean()), "allocation": wl.alloc,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
@@ -343,7 +349,8 @@ def main():
     layout = runtime.Layout.build(bits, wl.d)
     base = runtime.QuantizedState.from_fp32(S0, layout, w)
     tiles = wl.B * wl.H
-    bytes_launch = algorithmic_bytes(layout.bytes_per_seq, wl.B, wl.H, wl.d, wl.gate_per_channel, args.kernel)
+    bytes_launch = algorithmic_bytes(layout.bytes_per_seq, wl.B, wl.H, wl.d, wl.gate_per_channel,
+                                     f"prefill:{args.chunk}" if args.kernel == "prefill" else args.kernel)
 
     # Replicas: enough independent states that > 2x L2 is touched between reuses.
     per_rep = bytes_launch
@@ -353,15 +360,21 @@ def main():
     side = torch.cuda.Stream() if args.kernel == "split" else None
     x_ws = torch.empty((wl.B, wl.H, wl.d, wl.d), dtype=torch.float32, device="cuda") if side is not None else None
     for i in range(R):
-        if args.kernel in ("quant", "split"):
+        if args.kernel in ("quant", "split", "prefill"):
             reps.append(dict(packed=base.packed.clone(), r=base.r.clone(), c=base.c.clone()))
         elif args.kernel == "fp32":
             reps.append(dict(S=S0.clone()))
         else:
             cds, s = api.stepq_int8_quantize_state(S0)
             reps.append(dict(codes=cds, s=s))
-        toks.append(runtime.to_device_tokens(synth.tokens(wl, i % wl.T)))
-        outs.append(torch.empty((wl.B, wl.H, wl.d), dtype=torch.float32, device="cuda"))
+        if args.kernel == "prefill":
+            steps = [synth.tokens(wl, (i * args.chunk + t) % wl.T) for t in range(args.chunk)]
+            toks.append(runtime.to_device_tokens({n: np.ascontiguousarray(np.stack([x[n] for x in steps]))
+                                                  for n in steps[0]}))
+        else:
+            toks.append(runtime.to_device_tokens(synth.tokens(wl, i % wl.T)))
+        oshape = (args.chunk, wl.B, wl.H, wl.d) if args.kernel == "prefill" else (wl.B, wl.H, wl.d)
+        outs.append(torch.empty(oshape, dtype=torch.float32, device="cuda"))
     del S0
     torch.cuda.synchronize()
 
@@ -374,6 +387,10 @@ def main():
                                         pivots=layout.pivots)
             if refit:
                 torch.cuda.current_stream().wait_stream(side)   # writeback done before the next step
+        elif args.kernel == "prefill":
+            api.stepq_prefill_chunk(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
+                                    layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
+                                    st["packed"], st["r"], st["c"], o, pivots=layout.pivots)
         elif args.kernel == "quant":
             api.stepq_decode_step(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
                                   layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
@@ -414,7 +431,8 @@ def main():
         barrier()
     elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world, "cuda")
     ms_per_step = elapsed_ms / K
-    value = job_throughput(world, tiles, K, elapsed_ms)
+    upd = tiles * (args.chunk if args.kernel == "prefill" else 1)   # tile updates per launch
+    value = job_throughput(world, upd, K, elapsed_ms)
     achieved_gbs = bytes_launch / (ms_per_step * 1e-3) / 1e9
     peak, peak_kind = peaks()
 
@@ -439,12 +457,18 @@ def main():
                                                                 wl.gate_per_channel, "quant")}
 
     # ---- end to end through the public API with host buffers (H2D inputs, D2H output) ----
-    host_tok = [synth.tokens(wl, t % wl.T) for t in range(8)]
+    if args.kernel == "prefill":
+        host_tok = []
+        for e in range(2):
+            steps = [synth.tokens(wl, (e * args.chunk + t) % wl.T) for t in range(args.chunk)]
+            host_tok.append({n: np.ascontiguousarray(np.stack([x[n] for x in steps])) for n in steps[0]})
+    else:
+        host_tok = [synth.tokens(wl, t % wl.T) for t in range(8)]
     pinned = []
     for tk in host_tok:
         pinned.append({k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16) if v.dtype == np.uint16 else
                                            np.ascontiguousarray(v)).pin_memory() for k, v in tk.items()})
-    o_host = [torch.empty((wl.B, wl.H, wl.d), dtype=torch.float32).pin_memory() for _ in range(2)]
+    o_host = [torch.empty(tuple(outs[0].shape), dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in pinned[0].values())
     d2h = o_host[0].numel() * o_host[0].element_size()
     n_e2e = max(R, (args.e2e_steps // R) * R)
@@ -483,7 +507,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
-    e2e_value = job_throughput(world, tiles, n_e2e, e2e_ms)
+    e2e_value = job_throughput(world, upd, n_e2e, e2e_ms)
 
     line = None
     if rank == 0:
@@ -492,7 +516,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": rounds_warm * R,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": {**workload_config(wl, bits, args.kernel, world),
+            "config": {**workload_config(wl, bits, args.kernel, world, args.chunk),
                        "l2": (f"inputs larger than L2: {R} state replicas stepped round-robin, "
                               f"{R * per_rep / 2**20:.0f} MiB touched per round") if R * per_rep > L2_BYTES else
                              (f"inputs in L2 (latency case): {R} state replicas, "

@@ -127,6 +127,20 @@ STEPQ_API int stepq_decode_step(stepq_dims dims, const uint16_t* q, const uint16
                       const uint16_t* r_in, const uint16_t* c_in, uint8_t* packed_out,
                       uint16_t* r_out, uint16_t* c_out, float* o, void* stream);
 
+/* A prefill chunk on the packed state (STEPQuant App. F.1 "prefill unpacks active states, runs
+   the native chunk kernel, and packs the resulting boundary states"; App. B.2): per tile,
+   reconstruct S_hat once, apply the gated Delta rule for `chunk` tokens in fp32 without
+   requantising in between (readout o_t = X_t^T q_t after each token), then refit and pack the
+   boundary state once, as steps 4-6 of stepq_decode_step. Token inputs and o carry a leading
+   token axis: q, k [chunk][B][H][dk], v [chunk][B][H][dv], beta [chunk][B][H], gate
+   [chunk][B][H] or [chunk][B][H][dk], o [chunk][B][H][dv]. chunk = 1 is one decode step
+   (identical results). In-place use and dims.pivots as for stepq_decode_step. */
+STEPQ_API int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
+                        const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,
+                        const float* w, const int64_t* head_off, int64_t bytes_per_seq,
+                        const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,
+                        uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream);
+
 /* The split form of the same step (STEPQuant §4.4 and App. F.1: reconstruction, the update and
    the readout fused; scale fitting and packed writeback run afterwards on a separate stream),
    kept as an ablation of the single fused kernel:

@@ -49,6 +49,8 @@ struct DecodeArgs {
     uint16_t* c_out;
     float* o;
     float* x_out;   // split form only: the updated state X [B][H][dk][dv] before requantisation
+    int chunk;      // tokens per launch (1: one decode step; > 1: a prefill chunk, inputs and o
+                    // with a leading token axis)
 };
 
 // Mapping of a tile onto one CTA: a thread owns 8 adjacent columns of RPT rows; LPR lanes span
@@ -103,7 +105,7 @@ struct DecodeSmem {
     int htag[CH];                   // head held by each cache entry (-1: none)
     // Per slot of the tile being decoded.
     alignas(16) float4 kq[D];       // alpha k, alpha k, alpha q, alpha q   (alpha = g r 2^(8-b))
-    alignas(16) float4 ak[D];       // k/alpha, k/alpha, alpha, alpha
+    alignas(16) float4 ak[2][D];    // k/alpha, k/alpha, alpha, alpha (two tokens of a chunk)
     alignas(16) float4 rq[D];       // alpha e, alpha e, G, G  (e = 1/(r~ 2^(8-b)), G = (w r~ 2^(8-b))^2)
     alignas(16) float2 wsl[D];      // w, 1/w
     alignas(16) float riq[D];       // 1/q_b
@@ -116,6 +118,7 @@ struct DecodeSmem {
     alignas(16) float rowbuf[M::kWarps][32 * (M::RPT + 1)];
     alignas(8) uint64_t full[kStages];
     float qk;
+    float qkp[D / 32];              // q.k of a chunk's token, one partial per 32 key rows
 };
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a tile copy takes microseconds
@@ -469,7 +472,7 @@ __device__ __forceinline__ void store_col_partials(float* dst, int lane, float2 
 // The tile loop of the decode kernel. kPiv: the bit map may hold FP16 pivot rows (declared by
 // the caller in stepq_dims.pivots); launches without them run the leaner instantiation. A
 // width-16 row met in a launch declared without pivots raises bit 1 of the device error word.
-template <int D, bool kSplit, bool kPiv>
+template <int D, bool kSplit, bool kPiv, bool kChunk>
 __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm) {
     using M = DMap<D>;
     constexpr int RPT = M::RPT;
@@ -513,7 +516,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
                 const float wi = st.w[i];
                 const float ka = kk * rcp_approx(alpha);
                 sm.kq[sl] = make_float4(alpha * kk, alpha * kk, alpha * qq, alpha * qq);
-                sm.ak[sl] = make_float4(ka, ka, alpha, alpha);
+                sm.ak[0][sl] = make_float4(ka, ka, alpha, alpha);
                 sm.wsl[sl] = make_float2(wi, rcp_approx(wi));
                 if constexpr (kPiv) sm.icol[i] = rcp_approx(half_bits_to_float(st.c[i]));   // column i
             } else if (warp == D / 32) {
@@ -582,6 +585,85 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
         }
         __syncthreads();
 
+        // ---- prefill chunk: tokens 1 .. C-1 in full precision on the register-resident tile
+        //      (no requantisation between them); the gate folds into alpha_i ---------------
+        int kb = 0;   // the buffer of ak holding the last token's k/alpha and alpha
+        if constexpr (kChunk) {
+            const int64_t T = a.num_tiles;
+            // Thread tid < D holds the inputs of the next token, loaded one token ahead: key row
+            // tid's k, q, gate, and column tid's v, with the token's beta.
+            float nk = 0.f, nq = 0.f, ng = 0.f, nv = 0.f, nb = 0.f;
+            auto prefetch = [&](int t) {
+                const int64_t ti = (t * T + tile) * D + tid;
+                nk = bf16_bits_to_float(__ldg(a.k + ti));
+                nq = bf16_bits_to_float(__ldg(a.q + ti));
+                ng = a.gate_per_channel ? __ldg(a.gate + ti) : __ldg(a.gate + t * T + tile);
+                nv = bf16_bits_to_float(__ldg(a.v + ti));
+                nb = __ldg(a.beta + t * T + tile);
+            };
+            if (tid < D && a.chunk > 1) prefetch(1);
+            for (int t = 1; t < a.chunk; ++t) {
+                const int cb = t & 1, pb = cb ^ 1;
+                const float vt = nv, bt = nb;   // column tid's v and beta of token t
+                if (tid < D) {   // per-slot constants of token t (thread i = key row i)
+                    const int i = tid;
+                    const uint32_t sw = sm.hslot[he][i];
+                    const int sl = sw & 0xFF;
+                    const float alpha = fmaxf(ng * sm.ak[pb][sl].z, 0x1p-64f);
+                    const float kk = nk, qq = nq;
+                    if (t + 1 < a.chunk) prefetch(t + 1);
+                    sm.kq[sl] = make_float4(alpha * kk, alpha * kk, alpha * qq, alpha * qq);
+                    const float ka = kk * rcp_approx(alpha);
+                    sm.ak[cb][sl] = make_float4(ka, ka, alpha, alpha);
+                    float qk = qq * kk;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
+                    if (lane == 0) sm.qkp[warp] = qk;
+                }
+                __syncthreads();
+                {   // token t-1's rank-1 update fused with token t's k^T X and q^T X
+                    float2 ut[4], pacc[4], oacc[4];
+                    load_cols8(sm.colb, cl, ut);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) pacc[p] = oacc[p] = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int r = 0; r < RPT; ++r) {
+                        const int sl = M::row(warp, lane, r);
+                        const float4 c = sm.ak[pb][sl];
+                        const float4 kq = sm.kq[sl];
+                        const float2 ka = make_float2(c.x, c.y);
+                        const float2 kap = make_float2(kq.x, kq.y), lam = make_float2(kq.z, kq.w);
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            Z[r][p] = fma2(ka, ut[p], Z[r][p]);
+                            pacc[p] = fma2(kap, Z[r][p], pacc[p]);
+                            oacc[p] = fma2(lam, Z[r][p], oacc[p]);
+                        }
+                    }
+                    store_col_partials<D>(sm.red[warp][0], lane, pacc);
+                    store_col_partials<D>(sm.red[warp][1], lane, oacc);
+                }
+                __syncthreads();
+                if (tid < D) {   // u_t and o_t, column j
+                    const int j = tid;
+                    float ps = 0.f, os = 0.f, qk = 0.f;
+#pragma unroll
+                    for (int w = 0; w < M::kWarps; ++w) {
+                        ps += sm.red[w][0][j];
+                        os += sm.red[w][1][j];
+                    }
+#pragma unroll
+                    for (int w = 0; w < D / 32; ++w) qk += sm.qkp[w];
+                    const float cj = sm.colc[j];
+                    const float u = bt * (vt - cj * ps);
+                    a.o[(t * T + tile) * D + j] = fmaf(cj, os, qk * u);
+                    sm.colb[j] = u * rcp_approx(cj);
+                }
+                __syncthreads();
+            }
+            kb = (a.chunk - 1) & 1;
+        }
+
         // ---- phase 3: X = D S + k u^T as alpha_i c_j Y_ij, Y = z + (k_i/alpha_i) u_j/c_j;
         //      row sums of |X| -------------------------------------------------------------
         {
@@ -593,7 +675,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
 #pragma unroll
                 for (int r = 0; r < RPT; ++r) {
                     const int sl = M::row(warp, lane, r);
-                    const float4 c = sm.ak[sl];
+                    const float4 c = sm.ak[0][sl];
                     const float2 ka = make_float2(c.x, c.y), al = make_float2(c.z, c.z);
                     float4* dst = reinterpret_cast<float4*>(
                         a.x_out + (static_cast<int64_t>(tile) * D + (meta[sl] & 0xFF)) * D + 8 * cl);
@@ -613,7 +695,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
             float part[RPT];
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
-                const float4 c = sm.ak[M::row(warp, lane, r)];
+                const float4 c = sm.ak[kb][M::row(warp, lane, r)];
                 const float2 ka = make_float2(c.x, c.y);
                 float acc = 0.f;
 #pragma unroll
@@ -632,7 +714,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
                 const uint32_t mt = meta[sl];
                 const int i = mt & 0xFF, bw = (mt >> 8) & 0xFF;
                 const float2 w2 = sm.wsl[sl];
-                const float alpha = sm.ak[sl].z;
+                const float alpha = sm.ak[kb][sl].z;
                 const __half rh = scale_to_half(fmaxf(alpha * rsum * (1.0f / D), kHalfMinNormal) * w2.y);
                 a.r_out[static_cast<int64_t>(tile) * D + i] = __half_as_ushort(rh);
                 const float rs = __half2float(rh) * znorm_of(bw);
@@ -767,7 +849,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
 // kSplit: the first kernel of the split form. It reconstructs, updates and reads out like the
 // fused step, then writes the updated state X in fp32 and stops; the refit and the pack run
 // as separate kernels (stepq_decode_step_split).
-template <int D, bool kSplit, bool kPiv>
+template <int D, bool kSplit, bool kPiv, bool kChunk = false>
 __global__ void __launch_bounds__(DMap<D>::kThreads, DMap<D>::kMinBlocks)
 decode_kernel(const DecodeArgs a) {
     using M = DMap<D>;
@@ -815,10 +897,10 @@ decode_kernel(const DecodeArgs a) {
     }
     __syncthreads();
 
-    run_tiles<D, kSplit, kPiv>(a, sm);
+    run_tiles<D, kSplit, kPiv, kChunk>(a, sm);
 }
 
-template <int D, bool kSplit, bool kPiv>
+template <int D, bool kSplit, bool kPiv, bool kChunk = false>
 static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     static int ctas_per_sm = -1, num_sms = 0;
     const size_t smem = sizeof(DecodeSmem<D>);
@@ -826,17 +908,17 @@ static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, kSplit, kPiv>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, kSplit, kPiv, kChunk>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "stepq_decode_step: %s", cudaGetErrorString(e));
         int occ = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D, kSplit, kPiv>, DMap<D>::kThreads, smem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D, kSplit, kPiv, kChunk>, DMap<D>::kThreads, smem);
         ctas_per_sm = occ > 0 ? occ : 1;
     }
     if (a.num_tiles == 0) return STEPQ_OK;
     int grid = num_sms * ctas_per_sm;
     if (grid > a.num_tiles) grid = a.num_tiles;
-    decode_kernel<D, kSplit, kPiv><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
+    decode_kernel<D, kSplit, kPiv, kChunk><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
     return check_launch("stepq_decode_step");
 }
 
@@ -881,10 +963,37 @@ extern "C" int stepq_decode_step(stepq_dims dims, const uint16_t* q, const uint1
     const long long tiles = static_cast<long long>(dims.B) * dims.H;
     if (tiles > 0x7fffffffLL) return set_error(STEPQ_EINVAL, "stepq_decode_step: too many tiles");
     DecodeArgs a{dims.B, dims.H, dims.gate_per_channel, static_cast<int>(tiles), q, k, v, beta, gate, bits, w,
-                 head_off, bytes_per_seq, packed_in, r_in, c_in, packed_out, r_out, c_out, o, nullptr};
+                 head_off, bytes_per_seq, packed_in, r_in, c_in, packed_out, r_out, c_out, o, nullptr, 1};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dims.pivots) return dims.dk == 128 ? launch_decode<128, false, true>(a, st) : launch_decode<64, false, true>(a, st);
     return dims.dk == 128 ? launch_decode<128, false, false>(a, st) : launch_decode<64, false, false>(a, st);
+}
+
+extern "C" int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
+                                   const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,
+                                   const float* w, const int64_t* head_off, int64_t bytes_per_seq,
+                                   const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,
+                                   uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream) {
+    const char* fn = "stepq_prefill_chunk";
+    clear_error();
+    int rc = check_dims(dims, fn);
+    if (rc) return rc;
+    if (chunk < 1) return set_error(STEPQ_EINVAL, "%s: chunk=%d", fn, chunk);
+    if (dims.B == 0) return STEPQ_OK;
+    rc = check_ptrs(fn, {{"q", q}, {"k", k}, {"v", v}, {"beta", beta}, {"gate", gate}, {"bits", bits}, {"w", w},
+                         {"head_off", head_off}, {"packed_in", packed_in}, {"r_in", r_in}, {"c_in", c_in},
+                         {"packed_out", packed_out}, {"r_out", r_out}, {"c_out", c_out}, {"o", o}});
+    if (rc) return rc;
+    if (bytes_per_seq <= 0 || (bytes_per_seq & 15))
+        return set_error(STEPQ_EINVAL, "%s: bytes_per_seq=%lld", fn, (long long)bytes_per_seq);
+    const long long tiles = static_cast<long long>(dims.B) * dims.H;
+    if (tiles > 0x7fffffffLL) return set_error(STEPQ_EINVAL, "%s: too many tiles", fn);
+    DecodeArgs a{dims.B, dims.H, dims.gate_per_channel, static_cast<int>(tiles), q, k, v, beta, gate, bits, w,
+                 head_off, bytes_per_seq, packed_in, r_in, c_in, packed_out, r_out, c_out, o, nullptr, chunk};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dims.pivots)
+        return dims.dk == 128 ? launch_decode<128, false, true, true>(a, st) : launch_decode<64, false, true, true>(a, st);
+    return dims.dk == 128 ? launch_decode<128, false, false, true>(a, st) : launch_decode<64, false, false, true>(a, st);
 }
 
 extern "C" int stepq_decode_step_split(stepq_dims dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -912,7 +1021,7 @@ extern "C" int stepq_decode_step_split(stepq_dims dims, const uint16_t* q, const
     const long long tiles = static_cast<long long>(dims.B) * dims.H;
     if (tiles > 0x7fffffffLL) return set_error(STEPQ_EINVAL, "%s: too many tiles", fn);
     DecodeArgs a{dims.B, dims.H, dims.gate_per_channel, static_cast<int>(tiles), q, k, v, beta, gate, bits, w,
-                 head_off, bytes_per_seq, packed_in, r_in, c_in, nullptr, nullptr, nullptr, o, x_ws};
+                 head_off, bytes_per_seq, packed_in, r_in, c_in, nullptr, nullptr, nullptr, o, x_ws, 1};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dims.pivots) rc = dims.dk == 128 ? launch_decode<128, true, true>(a, st) : launch_decode<64, true, true>(a, st);
     else rc = dims.dk == 128 ? launch_decode<128, true, false>(a, st) : launch_decode<64, true, false>(a, st);
