@@ -118,7 +118,7 @@ struct DecodeSmem {
     alignas(16) float rowbuf[M::kWarps][32 * (M::RPT + 1)];
     alignas(8) uint64_t full[kStages];
     float qk;
-    float qkp[D / 32];              // q.k of a chunk's token, one partial per 32 key rows
+    float qkp[2][D / 32];           // q.k of a chunk's token, one partial per 32 key rows
 };
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a tile copy takes microseconds
@@ -469,6 +469,44 @@ __device__ __forceinline__ void store_col_partials(float* dst, int lane, float2 
     }
 }
 
+// A prefill token's inputs as one thread needs them: key row i's k, q and gate (the thread
+// writing row i's constants) or column j's v and the token's beta (the thread finalising
+// column j). Inputs carry a leading token axis of T tiles each.
+template <int D>
+struct TokenRow {
+    float k = 0.f, q = 0.f, g = 0.f;
+    __device__ __forceinline__ void load(const DecodeArgs& a, int64_t T, int tile, int i, int t) {
+        const int64_t tt = t * T + tile, ti = tt * D + i;
+        k = bf16_bits_to_float(__ldg(a.k + ti));
+        q = bf16_bits_to_float(__ldg(a.q + ti));
+        g = a.gate_per_channel ? __ldg(a.gate + ti) : __ldg(a.gate + tt);
+    }
+};
+template <int D>
+struct TokenCol {
+    float v = 0.f, beta = 0.f;
+    __device__ __forceinline__ void load(const DecodeArgs& a, int64_t T, int tile, int j, int t) {
+        const int64_t tt = t * T + tile;
+        v = bf16_bits_to_float(__ldg(a.v + tt * D + j));
+        beta = __ldg(a.beta + tt);
+    }
+};
+
+// Per-slot constants of prefill token t for key row i (alpha_t = g_t alpha_{t-1}), written by
+// the D threads that are not finalising columns; their warps reduce q.k partials.
+template <int D>
+__device__ __forceinline__ void token_constants(DecodeSmem<D>& sm, int he, int i, int t, const TokenRow<D>& in) {
+    const int sl = sm.hslot[he][i] & 0xFF;
+    const float alpha = fmaxf(in.g * sm.ak[(t - 1) & 1][sl].z, 0x1p-64f);
+    sm.kq[sl] = make_float4(alpha * in.k, alpha * in.k, alpha * in.q, alpha * in.q);
+    const float ka = in.k * rcp_approx(alpha);
+    sm.ak[t & 1][sl] = make_float4(ka, ka, alpha, alpha);
+    float qk = in.q * in.k;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
+    if ((i & 31) == 0) sm.qkp[t & 1][i >> 5] = qk;
+}
+
 // The tile loop of the decode kernel. kPiv: the bit map may hold FP16 pivot rows (declared by
 // the caller in stepq_dims.pivots); launches without them run the leaner instantiation. A
 // width-16 row met in a launch declared without pivots raises bit 1 of the device error word.
@@ -500,6 +538,17 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
             __syncthreads();
         }
         const bool ok = mbar_wait_bounded(&sm.full[s], parity, kWaitLimitNs, &g_stepq_flags);
+
+        // A prefill chunk's token 1: its inputs are loaded now, behind the unpack (rows by the
+        // threads tid >= D, columns by the threads tid < D); later tokens one window ahead.
+        TokenRow<D> rowA;
+        TokenCol<D> colA;
+        if constexpr (kChunk) {
+            if (a.chunk > 1) {
+                if (tid >= D) rowA.load(a, a.num_tiles, tile, tid - D, 1);
+                else colA.load(a, a.num_tiles, tile, tid, 1);
+            }
+        }
 
         // ---- prologue: per-slot constants of this tile, q.k ------------------------------
         if (ok) {
@@ -580,8 +629,14 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
             a.o[static_cast<int64_t>(tile) * D + j] = fmaf(cj, os, sm.qk * u);
             sm.colc[j] = cj;
             sm.colb[j] = u * rcp_approx(cj);
-        } else if (issuer) {
-            issued = issue_tile<D>(a, sm, cta_tile(ahead), sa, next_beta, next_gate);
+        } else {
+            if (issuer) issued = issue_tile<D>(a, sm, cta_tile(ahead), sa, next_beta, next_gate);
+            if constexpr (kChunk) {
+                if (a.chunk > 1) {   // token 1's constants, while token 0 is finalised
+                    token_constants<D>(sm, he, tid - D, 1, rowA);
+                    if (a.chunk > 2) rowA.load(a, a.num_tiles, tile, tid - D, 2);
+                }
+            }
         }
         __syncthreads();
 
@@ -590,37 +645,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
         int kb = 0;   // the buffer of ak holding the last token's k/alpha and alpha
         if constexpr (kChunk) {
             const int64_t T = a.num_tiles;
-            // Thread tid < D holds the inputs of the next token, loaded one token ahead: key row
-            // tid's k, q, gate, and column tid's v, with the token's beta.
-            float nk = 0.f, nq = 0.f, ng = 0.f, nv = 0.f, nb = 0.f;
-            auto prefetch = [&](int t) {
-                const int64_t ti = (t * T + tile) * D + tid;
-                nk = bf16_bits_to_float(__ldg(a.k + ti));
-                nq = bf16_bits_to_float(__ldg(a.q + ti));
-                ng = a.gate_per_channel ? __ldg(a.gate + ti) : __ldg(a.gate + t * T + tile);
-                nv = bf16_bits_to_float(__ldg(a.v + ti));
-                nb = __ldg(a.beta + t * T + tile);
-            };
-            if (tid < D && a.chunk > 1) prefetch(1);
             for (int t = 1; t < a.chunk; ++t) {
-                const int cb = t & 1, pb = cb ^ 1;
-                const float vt = nv, bt = nb;   // column tid's v and beta of token t
-                if (tid < D) {   // per-slot constants of token t (thread i = key row i)
-                    const int i = tid;
-                    const uint32_t sw = sm.hslot[he][i];
-                    const int sl = sw & 0xFF;
-                    const float alpha = fmaxf(ng * sm.ak[pb][sl].z, 0x1p-64f);
-                    const float kk = nk, qq = nq;
-                    if (t + 1 < a.chunk) prefetch(t + 1);
-                    sm.kq[sl] = make_float4(alpha * kk, alpha * kk, alpha * qq, alpha * qq);
-                    const float ka = kk * rcp_approx(alpha);
-                    sm.ak[cb][sl] = make_float4(ka, ka, alpha, alpha);
-                    float qk = qq * kk;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
-                    if (lane == 0) sm.qkp[warp] = qk;
-                }
-                __syncthreads();
                 {   // token t-1's rank-1 update fused with token t's k^T X and q^T X
                     float2 ut[4], pacc[4], oacc[4];
                     load_cols8(sm.colb, cl, ut);
@@ -629,7 +654,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
 #pragma unroll
                     for (int r = 0; r < RPT; ++r) {
                         const int sl = M::row(warp, lane, r);
-                        const float4 c = sm.ak[pb][sl];
+                        const float4 c = sm.ak[(t - 1) & 1][sl];
                         const float4 kq = sm.kq[sl];
                         const float2 ka = make_float2(c.x, c.y);
                         const float2 kap = make_float2(kq.x, kq.y), lam = make_float2(kq.z, kq.w);
@@ -653,11 +678,15 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
                         os += sm.red[w][1][j];
                     }
 #pragma unroll
-                    for (int w = 0; w < D / 32; ++w) qk += sm.qkp[w];
+                    for (int w = 0; w < D / 32; ++w) qk += sm.qkp[t & 1][w];
                     const float cj = sm.colc[j];
-                    const float u = bt * (vt - cj * ps);
+                    const float u = colA.beta * (colA.v - cj * ps);
                     a.o[(t * T + tile) * D + j] = fmaf(cj, os, qk * u);
                     sm.colb[j] = u * rcp_approx(cj);
+                    if (t + 1 < a.chunk) colA.load(a, T, tile, j, t + 1);
+                } else if (t + 1 < a.chunk) {   // meanwhile token t+1's constants
+                    token_constants<D>(sm, he, tid - D, t + 1, rowA);
+                    if (t + 2 < a.chunk) rowA.load(a, T, tile, tid - D, t + 2);
                 }
                 __syncthreads();
             }
