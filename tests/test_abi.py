@@ -122,3 +122,30 @@ def test_device_calls_validate_before_touching_cuda():
     with pytest.raises(_lib.StepqError) as e:
         api.stepq_packed_layout(bits, 64)
     assert e.value.code == _lib.STEPQ_EUNSUPPORTED
+
+
+def test_new_entry_points_validate_before_touching_cuda():
+    lib = _lib.lib()
+    P = _fake
+    # prefill: chunk must be positive; an empty batch is a no-op
+    rc = lib.stepq_prefill_chunk(_dims(), 0, *([P()] * 8), 4096, *([P()] * 7), None)
+    assert rc == _lib.STEPQ_EINVAL and b"chunk" in lib.stepq_last_error()
+    assert lib.stepq_prefill_chunk(_dims(B=0), 4, *([P()] * 8), 4096, *([P()] * 7), None) == _lib.STEPQ_OK
+    rc = lib.stepq_prefill_chunk(_dims(), 4, *([P()] * 8), 4097, *([P()] * 7), None)
+    assert rc == _lib.STEPQ_EINVAL
+    # split form: the work space is required
+    rc = lib.stepq_decode_step_split(_dims(), *([P()] * 8), 4096, *([P()] * 7), ctypes.c_void_p(0), None, None)
+    assert rc == _lib.STEPQ_EINVAL and b"x_ws is NULL" in lib.stepq_last_error()
+    # distortion under a bit map: pointers checked; width 16 accepted by the uniform form
+    rc = lib.stepq_calib_distortion_bits(_dims(), P(), P(), ctypes.c_void_p(0), P(), P(), P(), None)
+    assert rc == _lib.STEPQ_EINVAL and b"bits is NULL" in lib.stepq_last_error()
+    rc = lib.stepq_calib_distortion(_dims(), P(), P(), 12, P(), P(), P(), None)
+    assert rc == _lib.STEPQ_EUNSUPPORTED
+    # the static work space refuses sizes beyond its capacity before any CUDA call
+    rc = lib.stepq_calib_distortion_static(_dims(B=8193, H=1, d=64), P(), P(), 4, P(), P(), None)
+    assert rc == _lib.STEPQ_EINVAL and b"static work space" in lib.stepq_last_error()
+    # FP16 pivot rows are a valid width in a layout
+    bits = np.full((2, 64), 6, dtype=np.uint8)
+    bits[1, :3] = 16
+    head_off, bps, _ = api.stepq_packed_layout(bits, 64)
+    assert bps == oracle.layout(bits, 64)[1] == 64 * 6 // 8 * 125 + 64 * 2 * 3
