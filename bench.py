@@ -54,15 +54,18 @@ def parse():
                     help="quant: the fused step; split: the split-form ablation; prefill: a chunk of --chunk "
                          "tokens per launch; fp32 / int8: comparison states")
     ap.add_argument("--chunk", type=int, default=64, help="tokens per prefill chunk (--kernel prefill)")
+    ap.add_argument("--prefill-form", choices=["auto", "seq", "wy"], default="auto",
+                    help="prefill chunk form: the library's choice, the sequential register-tile form, "
+                         "or the chunked WY form on the tensor cores")
     ap.add_argument("--e2e-steps", type=int, default=400)
     return ap.parse_args()
 
 
 def kernel_revision() -> str:
-    """First 16 hex digits of the sha256 of the fused kernel's sources."""
+    """First 16 hex digits of the sha256 of the fused decode kernel's sources."""
     import hashlib
     csrc = ROOT / "recurrent_state_quantization_gated_b200" / "csrc"
-    data = (csrc / "stepq_decode.cu").read_bytes() + (csrc / "stepq_device.cuh").read_bytes()
+    data = b"".join((csrc / f).read_bytes() for f in ("stepq_decode.cu", "stepq_device.cuh", "stepq_tile.cuh"))
     return hashlib.sha256(data).hexdigest()[:16]
 
 
@@ -223,8 +226,8 @@ def job_throughput(world: int, tiles_per_rank: int, steps: int, ms: float) -> fl
     return world * tiles_per_rank * steps / (ms * 1e-3)
 
 
-def workload_config(wl, bits, kernel: str, world: int, chunk: int = 1) -> dict:
-    extra = {"chunk": chunk} if kernel == "prefill" else {}
+def workload_config(wl, bits, kernel: str, world: int, chunk: int = 1, prefill_form: str = "auto") -> dict:
+    extra = {"chunk": chunk, "prefill_form": prefill_form} if kernel == "prefill" else {}
     return {"workload": wl.name, "kernel": kernel, **extra, "B": wl.B, "H": wl.H, "d_k": wl.d, "d_v": wl.d,
             "bits_mean": float(np.asarray(bits, dtype=np.float64).mean()), "allocation": wl.alloc,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
@@ -390,7 +393,8 @@ def main():
         elif args.kernel == "prefill":
             api.stepq_prefill_chunk(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
                                     layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
-                                    st["packed"], st["r"], st["c"], o, pivots=layout.pivots)
+                                    st["packed"], st["r"], st["c"], o, pivots=layout.pivots,
+                                    form=None if args.prefill_form == "auto" else args.prefill_form)
         elif args.kernel == "quant":
             api.stepq_decode_step(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
                                   layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
@@ -516,7 +520,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": rounds_warm * R,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": {**workload_config(wl, bits, args.kernel, world, args.chunk),
+            "config": {**workload_config(wl, bits, args.kernel, world, args.chunk, args.prefill_form),
                        "l2": (f"inputs larger than L2: {R} state replicas stepped round-robin, "
                               f"{R * per_rep / 2**20:.0f} MiB touched per round") if R * per_rep > L2_BYTES else
                              (f"inputs in L2 (latency case): {R} state replicas, "

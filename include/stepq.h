@@ -127,15 +127,37 @@ STEPQ_API int stepq_decode_step(stepq_dims dims, const uint16_t* q, const uint16
                       const uint16_t* r_in, const uint16_t* c_in, uint8_t* packed_out,
                       uint16_t* r_out, uint16_t* c_out, float* o, void* stream);
 
-/* A prefill chunk on the packed state (STEPQuant App. F.1 "prefill unpacks active states, runs
-   the native chunk kernel, and packs the resulting boundary states"; App. B.2): per tile,
+/* A prefill chunk on the packed state (STEPQuant App. F.1 "prefill unpacks active states,
+   runs the native chunk kernel, and packs the resulting boundary states"; App. B.2): per tile,
    reconstruct S_hat once, apply the gated Delta rule for `chunk` tokens in fp32 without
    requantising in between (readout o_t = X_t^T q_t after each token), then refit and pack the
    boundary state once, as steps 4-6 of stepq_decode_step. Token inputs and o carry a leading
    token axis: q, k [chunk][B][H][dk], v [chunk][B][H][dv], beta [chunk][B][H], gate
-   [chunk][B][H] or [chunk][B][H][dk], o [chunk][B][H][dv]. chunk = 1 is one decode step
-   (identical results). In-place use and dims.pivots as for stepq_decode_step. */
+   [chunk][B][H] or [chunk][B][H][dk], o [chunk][B][H][dv]. In-place use and dims.pivots as for
+   stepq_decode_step.
+   Two forms compute it:
+     stepq_prefill_chunk_seq: the tokens one after another on the register-resident tile (any
+       supported shape and chunk length; chunk = 1 is bit-identical to stepq_decode_step);
+     stepq_prefill_chunk_wy: the chunked WY/UT form on the tensor cores (§2.1's affine form
+       unrolled over the chunk: one unit lower triangular solve and dense products per tile).
+       Requires dk = dv = 128, scalar gates, no FP16 pivot rows and
+       1 <= chunk <= STEPQ_WY_MAX_CHUNK; otherwise STEPQ_EUNSUPPORTED. Products run on bf16
+       operands (q, k, v and the integer codes exactly; computed operands split into two or
+       three bf16 parts) with fp32 accumulation: the boundary state carries fp32 precision, the
+       readouts about 1e-6 relative.
+   stepq_prefill_chunk takes the WY form where it applies and the sequential form elsewhere. */
+#define STEPQ_WY_MAX_CHUNK 64
 STEPQ_API int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
+                        const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,
+                        const float* w, const int64_t* head_off, int64_t bytes_per_seq,
+                        const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,
+                        uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream);
+STEPQ_API int stepq_prefill_chunk_seq(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
+                        const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,
+                        const float* w, const int64_t* head_off, int64_t bytes_per_seq,
+                        const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,
+                        uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream);
+STEPQ_API int stepq_prefill_chunk_wy(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
                         const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,
                         const float* w, const int64_t* head_off, int64_t bytes_per_seq,
                         const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,

@@ -16,6 +16,7 @@ _NAMES = {0: "OK", 1: "EINVAL", 2: "EUNSUPPORTED", 3: "EALIGN", 4: "EBUDGET", 5:
 SYMBOLS = (
     "stepq_last_error", "stepq_packed_layout", "stepq_fit_scales", "stepq_pack_state",
     "stepq_unpack_state", "stepq_decode_step", "stepq_decode_step_split", "stepq_prefill_chunk",
+    "stepq_prefill_chunk_seq", "stepq_prefill_chunk_wy",
     "stepq_decode_step_fp32",
     "stepq_int8_quantize_state", "stepq_decode_step_int8", "stepq_row_impact",
     "stepq_calib_distortion", "stepq_calib_distortion_bits", "stepq_calib_distortion_static", "stepq_allocate_bits", "stepq_read_device_flags",
@@ -50,6 +51,8 @@ _SIGNATURES = {
     "stepq_decode_step": ([Dims, P, P, P, P, P, P, P, P, I64, P, P, P, P, P, P, P, P], I),
     "stepq_decode_step_split": ([Dims, P, P, P, P, P, P, P, P, I64, P, P, P, P, P, P, P, P, P, P], I),
     "stepq_prefill_chunk": ([Dims, I, P, P, P, P, P, P, P, P, I64, P, P, P, P, P, P, P, P], I),
+    "stepq_prefill_chunk_seq": ([Dims, I, P, P, P, P, P, P, P, P, I64, P, P, P, P, P, P, P, P], I),
+    "stepq_prefill_chunk_wy": ([Dims, I, P, P, P, P, P, P, P, P, I64, P, P, P, P, P, P, P, P], I),
     "stepq_decode_step_fp32": ([Dims, P, P, P, P, P, P, P, P, P], I),
     "stepq_int8_quantize_state": ([Dims, P, P, P, P], I),
     "stepq_decode_step_int8": ([Dims, P, P, P, P, P, P, P, P, P, P, P], I),

@@ -20,7 +20,8 @@ from ._lib import Dims, call, lib
 
 __all__ = [
     "stepq_packed_layout", "stepq_fit_scales", "stepq_pack_state", "stepq_unpack_state",
-    "stepq_decode_step", "stepq_decode_step_split", "stepq_prefill_chunk", "stepq_decode_step_fp32", "stepq_int8_quantize_state",
+    "stepq_decode_step", "stepq_decode_step_split", "stepq_prefill_chunk",
+    "stepq_prefill_chunk_seq", "stepq_prefill_chunk_wy", "stepq_decode_step_fp32", "stepq_int8_quantize_state",
     "stepq_decode_step_int8", "stepq_row_impact", "stepq_calib_distortion", "stepq_calib_distortion_bits", "stepq_calib_distortion_static",
     "stepq_allocate_bits",
     "stepq_read_device_flags", "stepq_build_info",
@@ -150,9 +151,11 @@ def stepq_decode_step_split(q, k, v, beta, gate, bits, w, head_off, bytes_per_se
 
 
 def stepq_prefill_chunk(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
-                        packed_out=None, r_out=None, c_out=None, o=None, pivots=None):
+                        packed_out=None, r_out=None, c_out=None, o=None, pivots=None, form=None):
     """A prefill chunk: q, k, v [C,B,H,d], beta [C,B,H], gate [C,B,H] or [C,B,H,d]; the state is
-    reconstructed once, updated C times in fp32 and packed once. Returns (packed_out, r_out,
+    reconstructed once, updated C times in fp32 and packed once. form: None (the library picks),
+    "seq" (tokens one after another on the register tile) or "wy" (the chunked WY form on the
+    tensor cores; d = 128, scalar gates, no pivot rows, C <= 64). Returns (packed_out, r_out,
     c_out, o [C,B,H,d])."""
     C, B, H, d = q.shape
     gpc = 1 if gate.dim() == 4 else 0
@@ -160,7 +163,8 @@ def stepq_prefill_chunk(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, p
     r_out = torch.empty_like(r_in) if r_out is None else r_out
     c_out = torch.empty_like(c_in) if c_out is None else c_out
     o = torch.empty((C, B, H, d), dtype=torch.float32, device=q.device) if o is None else o
-    call("stepq_prefill_chunk", _dims(B, H, d, gpc, _has_pivots(bits, pivots)), ctypes.c_int(int(C)),
+    name = {None: "stepq_prefill_chunk", "seq": "stepq_prefill_chunk_seq", "wy": "stepq_prefill_chunk_wy"}[form]
+    call(name, _dims(B, H, d, gpc, _has_pivots(bits, pivots)), ctypes.c_int(int(C)),
          _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
          _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"), _ptr(bits, torch.uint8, "bits"),
          _ptr(w, torch.float32, "w"), _ptr(head_off, torch.int64, "head_off"), ctypes.c_int64(int(bytes_per_seq)),

@@ -23,6 +23,7 @@
 #include <mutex>
 
 #include "stepq_device.cuh"
+#include "stepq_tile.cuh"
 #include "stepq_internal.h"
 
 namespace stepq {
@@ -51,24 +52,6 @@ struct DecodeArgs {
     float* x_out;   // split form only: the updated state X [B][H][dk][dv] before requantisation
     int chunk;      // tokens per launch (1: one decode step; > 1: a prefill chunk, inputs and o
                     // with a leading token axis)
-};
-
-// Mapping of a tile onto one CTA: a thread owns 8 adjacent columns of RPT rows; LPR lanes span
-// a row; a warp covers RPW rows per instruction and owns 16 consecutive slots (rows sorted by
-// width).
-template <int D>
-struct DMap {
-    static constexpr int kCols = 8;
-    static constexpr int kThreads = (D == 128) ? 256 : 128;
-    static constexpr int kMinBlocks = (D == 128) ? 2 : 4;
-    static constexpr int kWarps = kThreads / 32;
-    static constexpr int LPR = D / kCols;               // lanes per row
-    static constexpr int RPW = 32 / LPR;                // rows per warp instruction
-    static constexpr int RPT = D / (kWarps * RPW);      // rows per thread
-    static constexpr int kRowsPerWarp = RPT * RPW;
-    __device__ static int col_lane(int lane) { return lane % LPR; }
-    __device__ static int sub_row(int lane) { return lane / LPR; }
-    __device__ static int row(int warp, int lane, int r) { return warp * kRowsPerWarp + r * RPW + sub_row(lane); }
 };
 
 constexpr int kStages = 3;   // tile copies in flight: the current tile and the next two
@@ -152,83 +135,6 @@ __device__ __forceinline__ bool issue_tile(const DecodeArgs& a, DecodeSmem<D>& s
 
 // The n-th tile of this CTA (tiles are dealt round-robin over the persistent CTAs).
 __device__ __forceinline__ int cta_tile(int n) { return blockIdx.x + n * gridDim.x; }
-
-// One warp sorts the rows of head h by bit width (stable) into cache entry e.
-template <int D, bool kPiv>
-__device__ __forceinline__ void sort_head_warp(const DecodeArgs& a, DecodeSmem<D>& sm, int h, int e, int lane) {
-    // Width classes in slot order: 2, 4, 6, 8, then 16 (FP16 pivot rows). Byte offsets follow
-    // the packed layout: integer rows in key order, then pivot rows in key order.
-    constexpr int RL = D / 32, NC = 5;
-    int bw[RL], loc[RL], rank[RL], sum_i = 0, sum_p = 0;
-    int cnt[NC] = {0, 0, 0, 0, 0};
-#pragma unroll
-    for (int r = 0; r < RL; ++r) {
-        bw[r] = a.bits[static_cast<int64_t>(h) * D + lane * RL + r];
-        const bool piv = bw[r] == 16;
-        loc[r] = piv ? sum_p : sum_i;
-        (piv ? sum_p : sum_i) += bw[r] * (D / 8);
-        const int cls = piv ? 4 : (bw[r] >> 1) - 1;
-        rank[r] = 0;
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            if (c == cls) rank[r] = cnt[c];
-            cnt[c] += (c == cls);
-        }
-    }
-    int inc_i = sum_i, inc_p = sum_p;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int ti = __shfl_up_sync(0xffffffffu, inc_i, o);
-        const int tp = __shfl_up_sync(0xffffffffu, inc_p, o);
-        if (lane >= o) { inc_i += ti; inc_p += tp; }
-    }
-    const int total_i = __shfl_sync(0xffffffffu, inc_i, 31);
-    int excl_c[NC], base_c[NC], base = 0;
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-        int x = cnt[c];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += t;
-        }
-        excl_c[c] = x - cnt[c];
-        base_c[c] = base;
-        base += __shfl_sync(0xffffffffu, x, 31);
-    }
-#pragma unroll
-    for (int r = 0; r < RL; ++r) {
-        const int i = lane * RL + r;
-        const bool piv = bw[r] == 16;
-        const int cls = piv ? 4 : (bw[r] >> 1) - 1;
-        int slot = 0;
-#pragma unroll
-        for (int c = 0; c < NC; ++c)
-            if (c == cls) slot = base_c[c] + excl_c[c] + rank[r];
-        int off = (piv ? total_i + inc_p - sum_p : inc_i - sum_i) + loc[r];
-        int wb = bw[r];
-        if (!kPiv && piv) {
-            // A pivot row in a launch declared without pivots: flagged (bit 1); the row is
-            // handled as an in-bounds 8-bit row so that nothing is read or written outside
-            // the tile (its results are undefined).
-            atomicOr(&g_stepq_flags, 2u);
-            wb = 8;
-            off = min(off, D * D - D);
-        }
-        sm.hmeta[e][slot] = static_cast<uint32_t>(i) | (static_cast<uint32_t>(wb) << 8) | (static_cast<uint32_t>(off) << 16);
-        sm.hslot[e][i] = static_cast<uint16_t>(slot | (wb << 8));
-    }
-}
-
-// Eight consecutive per-column values (columns 8cl .. 8cl+7) as four pairs.
-__device__ __forceinline__ void load_cols8(const float* src, int cl, float2 out[4]) {
-    const float4 a = *reinterpret_cast<const float4*>(src + 8 * cl);
-    const float4 b = *reinterpret_cast<const float4*>(src + 8 * cl + 4);
-    out[0] = make_float2(a.x, a.y);
-    out[1] = make_float2(a.z, a.w);
-    out[2] = make_float2(b.x, b.y);
-    out[3] = make_float2(b.z, b.w);
-}
 
 // ---- phase 1: unpack the thread's rows and accumulate the k^T and q^T products -------------
 template <int D, int BW>
@@ -340,98 +246,6 @@ __device__ __forceinline__ void phase1_mixed(const DecodeSmem<D>& sm, const uint
     }
 }
 
-// ---- phase 6: final codes, packed and stored ------------------------------------------------
-// Codes are always limited to [-q_b, q_b]: the least-squares column scale is below the no-clip
-// scale in most columns, so the limit is nearly always needed somewhere in a tile.
-template <int D, int BW>
-__device__ __forceinline__ void phase6_row(uint8_t* out, uint32_t mt, int cl, const float2 x[4], const float2 f[4]) {
-    const float2 M2 = make_float2(kRoundMagic, kRoundMagic);
-    uint32_t zq[8];
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const float2 t = fma2(x[p], f[p], M2);
-        zq[2 * p] = __float_as_uint(t.x);
-        zq[2 * p + 1] = __float_as_uint(t.y);
-    }
-    pack8<D, BW, true>(out + (mt >> 16), cl, zq);
-}
-
-// An FP16 pivot row: X_ij = xi_ij c_j (xi = alpha_i Y_ij for pivot rows), rounded to binary16
-// (nearest-even, saturating) and stored straight to global memory.
-template <int D>
-__device__ __forceinline__ void phase6_pivot_row(uint8_t* out, uint32_t mt, int cl, const float2 x[4], const float2 cc[4]) {
-    uint32_t h[4];
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const float2 v = mul2(x[p], cc[p]);
-        __half2 hv = __halves2half2(pivot_half(v.x), pivot_half(v.y));
-        h[p] = *reinterpret_cast<uint32_t*>(&hv);
-    }
-    *reinterpret_cast<uint4*>(out + (mt >> 16) + 16 * cl) = make_uint4(h[0], h[1], h[2], h[3]);
-}
-
-template <int D, int BW>
-__device__ __forceinline__ void phase6_uniform(const uint32_t* meta, uint8_t* out, int warp, int lane,
-                                               const float2 Z[][4], const float2 f[4], const float* colc) {
-    using M = DMap<D>;
-    const int cl = M::col_lane(lane);
-    float2 cc[4];
-    if constexpr (BW == 16) load_cols8(colc, cl, cc);
-#pragma unroll
-    for (int r = 0; r < M::RPT; ++r) {
-        if constexpr (BW == 16) phase6_pivot_row<D>(out, meta[M::row(warp, lane, r)], cl, Z[r], cc);
-        else phase6_row<D, BW>(out, meta[M::row(warp, lane, r)], cl, Z[r], f);
-    }
-}
-
-template <int D, bool kPiv>
-__device__ __forceinline__ void phase6_mixed(const uint32_t* meta, uint8_t* out, int warp, int lane,
-                                             const float2 Z[][4], const float2 f[4], const float* colc) {
-    using M = DMap<D>;
-    const int cl = M::col_lane(lane);
-    float2 cc[4] = {};
-    if constexpr (kPiv) load_cols8(colc, cl, cc);
-#pragma unroll
-    for (int r = 0; r < M::RPT; ++r) {
-        const uint32_t mt = meta[M::row(warp, lane, r)];
-        switch ((mt >> 8) & 0xFF) {
-            case 8: phase6_row<D, 8>(out, mt, cl, Z[r], f); break;
-            case 6: phase6_row<D, 6>(out, mt, cl, Z[r], f); break;
-            case 4: phase6_row<D, 4>(out, mt, cl, Z[r], f); break;
-            default:
-                if constexpr (kPiv) {
-                    if (((mt >> 8) & 0xFF) == 16) {
-                        phase6_pivot_row<D>(out, mt, cl, Z[r], cc);
-                        break;
-                    }
-                }
-                phase6_row<D, 2>(out, mt, cl, Z[r], f);
-                break;
-        }
-    }
-}
-
-// kPiv: the pivot-capable instantiation (width-16 rows handled); without it the code is leaner.
-template <int D, bool kPiv>
-__device__ __forceinline__ void phase6(const uint32_t* meta, uint8_t* out, int warp, int lane, int ww,
-                                       const float2 Z[][4], const float2 f[4], const float* colc) {
-    switch (ww) {
-        case 8: phase6_uniform<D, 8>(meta, out, warp, lane, Z, f, colc); break;
-        case 6: phase6_uniform<D, 6>(meta, out, warp, lane, Z, f, colc); break;
-        case 4: phase6_uniform<D, 4>(meta, out, warp, lane, Z, f, colc); break;
-        case 2: phase6_uniform<D, 2>(meta, out, warp, lane, Z, f, colc); break;
-        default:
-            if constexpr (kPiv) {
-                if (ww == 16) {
-                    phase6_uniform<D, 16>(meta, out, warp, lane, Z, f, colc);
-                    break;
-                }
-            }
-            phase6_mixed<D, kPiv>(meta, out, warp, lane, Z, f, colc);
-            break;
-    }
-}
-
 template <int D, bool kPiv>
 __device__ __forceinline__ void phase1(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* codes,
                                        const uint8_t* gin, int warp, int lane, int ww, float2 Z[][4],
@@ -450,22 +264,6 @@ __device__ __forceinline__ void phase1(const DecodeSmem<D>& sm, const uint32_t* 
             }
             phase1_mixed<D, kPiv>(sm, meta, codes, gin, warp, lane, Z, pacc, oacc);
             break;
-    }
-}
-
-// Sum (over the warp's sub-rows) the per-thread partials of eight columns and store them.
-template <int D>
-__device__ __forceinline__ void store_col_partials(float* dst, int lane, float2 v[4]) {
-    using M = DMap<D>;
-#pragma unroll
-    for (int m = M::LPR; m < 32; m <<= 1)
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-            v[p] = add2(v[p], make_float2(__shfl_xor_sync(0xffffffffu, v[p].x, m), __shfl_xor_sync(0xffffffffu, v[p].y, m)));
-    if (lane < M::LPR) {
-        const int cl = M::col_lane(lane);
-        *reinterpret_cast<float4*>(dst + 8 * cl) = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
-        *reinterpret_cast<float4*>(dst + 8 * cl + 4) = make_float4(v[2].x, v[2].y, v[3].x, v[3].y);
     }
 }
 
@@ -532,7 +330,8 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
         if (sm.htag[he] != h) {                     // every warp sees the same tag: uniform branch
             __syncthreads();                        // nobody still reads the entry
             if (warp == 0) {
-                sort_head_warp<D, kPiv>(a, sm, h, he, lane);
+                sort_head_rows<D, kPiv>(a.bits + static_cast<int64_t>(h) * D, sm.hmeta[he], sm.hslot[he], lane,
+                                           &g_stepq_flags);
                 if (lane == 0) sm.htag[he] = h;
             }
             __syncthreads();
@@ -695,11 +494,11 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
 
         // ---- phase 3: X = D S + k u^T as alpha_i c_j Y_ij, Y = z + (k_i/alpha_i) u_j/c_j;
         //      row sums of |X| -------------------------------------------------------------
-        {
+        if constexpr (kSplit) {
             float2 cf[4], ut[4];
             load_cols8(sm.colc, cl, cf);
             load_cols8(sm.colb, cl, ut);
-            if constexpr (kSplit) {
+            {
                 // X_ij = alpha_i c_j Y_ij, written row by row in natural key order.
 #pragma unroll
                 for (int r = 0; r < RPT; ++r) {
@@ -721,153 +520,8 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
                 __syncthreads();   // the next tile's prologue rewrites the per-slot constants
                 continue;
             }
-            float part[RPT];
-#pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const float4 c = sm.ak[kb][M::row(warp, lane, r)];
-                const float2 ka = make_float2(c.x, c.y);
-                float acc = 0.f;
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    Z[r][p] = fma2(ka, ut[p], Z[r][p]);
-                    acc = fmaf(fabsf(Z[r][p].x), cf[p].x, acc);
-                    acc = fmaf(fabsf(Z[r][p].y), cf[p].y, acc);
-                }
-                part[r] = acc;
-            }
-            int slot;
-            bool owner;
-            const float rsum = row_reduce<M, float>(sm.rowbuf[warp], lane, part, slot, OpAdd());
-            const int sl = reduced_row<M>(warp, lane, slot, owner);   // a slot index
-            if (owner) {
-                const uint32_t mt = meta[sl];
-                const int i = mt & 0xFF, bw = (mt >> 8) & 0xFF;
-                const float2 w2 = sm.wsl[sl];
-                const float alpha = sm.ak[kb][sl].z;
-                const __half rh = scale_to_half(fmaxf(alpha * rsum * (1.0f / D), kHalfMinNormal) * w2.y);
-                a.r_out[static_cast<int64_t>(tile) * D + i] = __half_as_ushort(rh);
-                const float rs = __half2float(rh) * znorm_of(bw);
-                if (kPiv && bw == 16) {   // FP16 pivot row: xi = alpha Y, outside the shared column fit
-                    sm.rq[sl] = make_float4(alpha, alpha, 0.f, 0.f);
-                    sm.riq[sl] = 0.f;
-                } else {
-                    const float e = alpha * rcp_approx(rs);
-                    const float g = w2.x * rs;
-                    sm.rq[sl] = make_float4(e, e, g * g, g * g);
-                    sm.riq[sl] = inv_qmax_of(bw);
-                }
-            }
-            __syncwarp();
         }
-
-        // ---- phase 4: xi = X / (c_j r~_i 2^(8-b_i)); column no-clip scale c0 -----------
-        {
-            float2 cmax[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) cmax[p] = make_float2(0.f, 0.f);
-            if (ww != 0) {
-#pragma unroll
-                for (int r = 0; r < RPT; r += 2) {
-                    const float4 q4 = sm.rq[M::row(warp, lane, r)];
-                    const float4 q5 = sm.rq[M::row(warp, lane, r + 1)];
-                    const float2 e2 = make_float2(q4.x, q4.y), e3 = make_float2(q5.x, q5.y);
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        Z[r][p] = mul2(Z[r][p], e2);
-                        Z[r + 1][p] = mul2(Z[r + 1][p], e3);
-                        cmax[p].x = max_abs3(cmax[p].x, Z[r][p].x, Z[r + 1][p].x);
-                        cmax[p].y = max_abs3(cmax[p].y, Z[r][p].y, Z[r + 1][p].y);
-                    }
-                }
-                const float iq = sm.riq[warp * M::kRowsPerWarp];
-#pragma unroll
-                for (int p = 0; p < 4; ++p) cmax[p] = mul2(cmax[p], make_float2(iq, iq));
-            } else {
-#pragma unroll
-                for (int r = 0; r < RPT; ++r) {
-                    const int sl = M::row(warp, lane, r);
-                    const float4 q4 = sm.rq[sl];
-                    const float2 e2 = make_float2(q4.x, q4.y);
-                    const float iq = sm.riq[sl];
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        Z[r][p] = mul2(Z[r][p], e2);
-                        cmax[p].x = fmaxf(cmax[p].x, fabsf(Z[r][p].x) * iq);
-                        cmax[p].y = fmaxf(cmax[p].y, fabsf(Z[r][p].y) * iq);
-                    }
-                }
-            }
-#pragma unroll
-            for (int m = M::LPR; m < 32; m <<= 1)
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    cmax[p].x = fmaxf(cmax[p].x, __shfl_xor_sync(0xffffffffu, cmax[p].x, m));
-                    cmax[p].y = fmaxf(cmax[p].y, __shfl_xor_sync(0xffffffffu, cmax[p].y, m));
-                }
-            if (lane < M::LPR) {
-                *reinterpret_cast<float4*>(&sm.red[warp][0][8 * cl]) = make_float4(cmax[0].x, cmax[0].y, cmax[1].x, cmax[1].y);
-                *reinterpret_cast<float4*>(&sm.red[warp][0][8 * cl + 4]) = make_float4(cmax[2].x, cmax[2].y, cmax[3].x, cmax[3].y);
-            }
-        }
-        __syncthreads();
-        if (tid < D) {
-            const int j = tid;
-            float cm = 0.f;
-#pragma unroll
-            for (int w = 0; w < M::kWarps; ++w) cm = fmaxf(cm, sm.red[w][0][j]);
-            const float cj = sm.colc[j];
-            const float c0 = fmaxf(cj * cm, kHalfMinNormal);
-            sm.col0[j] = c0;
-            sm.colb[j] = cj * rcp_approx(c0);
-        }
-        __syncthreads();
-
-        // ---- phase 5: codes at (r~, c0); weighted least-squares column update ----------
-        {
-            float2 f[4];
-            load_cols8(sm.colb, cl, f);
-            const float2 mM2 = make_float2(-kRoundMagic, -kRoundMagic);
-            float2 num[4], den[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) num[p] = den[p] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const float4 q4 = sm.rq[M::row(warp, lane, r)];
-                const float2 G2 = make_float2(q4.z, q4.w);
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const float2 z0 = add2(fma2(Z[r][p], f[p], M2), mM2);
-                    const float2 gz = mul2(G2, z0);
-                    num[p] = fma2(gz, Z[r][p], num[p]);
-                    den[p] = fma2(gz, z0, den[p]);
-                }
-            }
-            store_col_partials<D>(sm.red[warp][0], lane, num);
-            store_col_partials<D>(sm.red[warp][1], lane, den);
-        }
-        __syncthreads();
-        if (tid < D) {
-            const int j = tid;
-            float ns = 0.f, ds = 0.f;
-#pragma unroll
-            for (int w = 0; w < M::kWarps; ++w) {
-                ns += sm.red[w][0][j];
-                ds += sm.red[w][1][j];
-            }
-            const float cj = sm.colc[j];
-            const float c1 = ds > 0.f ? (cj * ns) * rcp_approx(ds) : sm.col0[j];
-            const __half ch = scale_to_half(c1);
-            a.c_out[static_cast<int64_t>(tile) * D + j] = __half_as_ushort(ch);
-            sm.colb[j] = cj * rcp_approx(__half2float(ch));
-        }
-        __syncthreads();
-
-        // ---- phase 6: final codes at (r~, c~), packed and stored -----------------------
-        {
-            float2 f[4];
-            load_cols8(sm.colb, cl, f);
-            phase6<D, kPiv>(meta, a.packed_out + tile_base, warp, lane, ww, Z, f, sm.colc);
-        }
+        refit_pack<D, kPiv, true>(sm, meta, Z, ww, kb, tile, a.r_out, a.c_out, a.packed_out + tile_base);
         if (issued) {   // ordered before their use by the barriers of the next tiles
             sm.stage[sa].beta = next_beta;
             sm.stage[sa].gate1 = next_gate;
@@ -920,7 +574,8 @@ decode_kernel(const DecodeArgs a) {
         for (int m = 0; m < n; ++m)
             if ((cta_tile(m) % a.H) % CH == h % CH) take = false;
         if (take) {
-            sort_head_warp<D, kPiv>(a, sm, h, h % CH, lane);
+            sort_head_rows<D, kPiv>(a.bits + static_cast<int64_t>(h) * D, sm.hmeta[h % CH], sm.hslot[h % CH], lane,
+                                       &g_stepq_flags);
             if (lane == 0) sm.htag[h % CH] = h;
         }
     }
@@ -949,6 +604,22 @@ static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     if (grid > a.num_tiles) grid = a.num_tiles;
     decode_kernel<D, kSplit, kPiv, kChunk><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
     return check_launch("stepq_decode_step");
+}
+
+int device_flags_ptr(uint32_t** p) {
+    static std::mutex mu;
+    static uint32_t* ptrs[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64)
+        return set_error(STEPQ_ECUDA, "device error word: device %d: %s", dev, cudaGetErrorString(e));
+    std::lock_guard<std::mutex> lock(mu);
+    if (ptrs[dev] == nullptr) {
+        e = cudaGetSymbolAddress(reinterpret_cast<void**>(&ptrs[dev]), g_stepq_flags);
+        if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "device error word: %s", cudaGetErrorString(e));
+    }
+    *p = ptrs[dev];
+    return STEPQ_OK;
 }
 
 // One event per device orders the refit and pack of the split form after its first kernel.
@@ -998,12 +669,12 @@ extern "C" int stepq_decode_step(stepq_dims dims, const uint16_t* q, const uint1
     return dims.dk == 128 ? launch_decode<128, false, false>(a, st) : launch_decode<64, false, false>(a, st);
 }
 
-extern "C" int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
-                                   const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,
-                                   const float* w, const int64_t* head_off, int64_t bytes_per_seq,
-                                   const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,
-                                   uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream) {
-    const char* fn = "stepq_prefill_chunk";
+extern "C" int stepq_prefill_chunk_seq(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
+                                       const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,
+                                       const float* w, const int64_t* head_off, int64_t bytes_per_seq,
+                                       const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,
+                                       uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream) {
+    const char* fn = "stepq_prefill_chunk_seq";
     clear_error();
     int rc = check_dims(dims, fn);
     if (rc) return rc;
@@ -1023,6 +694,18 @@ extern "C" int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q
     if (dims.pivots)
         return dims.dk == 128 ? launch_decode<128, false, true, true>(a, st) : launch_decode<64, false, true, true>(a, st);
     return dims.dk == 128 ? launch_decode<128, false, false, true>(a, st) : launch_decode<64, false, false, true>(a, st);
+}
+
+extern "C" int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
+                                   const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,
+                                   const float* w, const int64_t* head_off, int64_t bytes_per_seq,
+                                   const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,
+                                   uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream) {
+    const bool wy = dims.dk == 128 && dims.dv == 128 && dims.gate_per_channel == 0 && dims.pivots == 0 && chunk >= 1 &&
+                    chunk <= STEPQ_WY_MAX_CHUNK;
+    return (wy ? stepq_prefill_chunk_wy : stepq_prefill_chunk_seq)(dims, chunk, q, k, v, beta, gate, bits, w, head_off,
+                                                                   bytes_per_seq, packed_in, r_in, c_in, packed_out,
+                                                                   r_out, c_out, o, stream);
 }
 
 extern "C" int stepq_decode_step_split(stepq_dims dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,

@@ -36,4 +36,7 @@ int check_ptrs(const char* fn, std::initializer_list<std::pair<const char*, cons
 // Maps a CUDA launch status to STEPQ_OK / STEPQ_ECUDA (with the message recorded).
 int check_launch(const char* fn);
 
+// Device address of the current device's error word (the one stepq_read_device_flags reads).
+int device_flags_ptr(uint32_t** p);
+
 }  // namespace stepq

@@ -1,0 +1,764 @@
+// stepq_prefill_wy.cu -- the prefill chunk (STEPQuant App. F.1 and App. B.2: reconstruct the
+// packed state once, run the native chunk update over the chunk's tokens, refit and pack the
+// boundary state once) in the chunked WY/UT form of the gated Delta rule, on the fifth-generation
+// tensor cores of sm_100a.
+//
+// Per (sequence, head) tile with state S0 (d_k x d_v, d = 128) and C <= 64 tokens, gates g_t,
+// gamma_t = g_1 ... g_t and R_ts = gamma_t / gamma_s, the recurrence of §2.1
+//   S_t = g_t S_{t-1} + k_t u_t^T,   u_t = beta_t (v_t - g_t S_{t-1}^T k_t),   o_t = S_t^T q_t
+// unrolls to S_t = gamma_t S0 + sum_{s<=t} R_ts k_s u_s^T, so that the rows u_t solve the unit
+// lower triangular system (I + L) U = diag(beta) (V - diag(gamma) K S0) with
+// L_ts = beta_t R_ts k_t.k_s (s < t). With T = (I + L)^-1:
+//   U   = T diag(beta) V - T diag(beta gamma) K S0
+//   O   = diag(gamma) Q S0 + (R o tril(Q K^T)) U
+//   S_C = gamma_C S0 + (diag(gamma_C / gamma) K)^T U.
+// Every product is an M = 128 tcgen05.mma (bf16 operands, fp32 accumulation in tensor memory).
+// One operand of each product is exact in bf16: q, k and v are bf16 inputs and S0 enters as its
+// integer codes Z (S0 = diag(r 2^(8-b)) Z diag(c), |Z| <= 127). The other operand, computed in
+// fp32, is split into bf16 parts whose products are accumulated: three parts (high, middle, low:
+// 24 significant bits, as fp32) for every product that reaches the boundary state, whose codes
+// must agree with a float64 evaluation; two parts (about 2^-17) for the readout's P U, which takes
+// the three largest of its four part products. T comes from a blocked inversion (16 x 16
+// diagonal blocks by substitution, then block rows) on the CUDA cores. The boundary state then
+// runs through the same refit and pack as the fused decode step (steps 4-6 of Table C2).
+//
+// One CTA per SM (the operands of a tile take 224 KB of shared memory), 256 threads, 512 TMEM
+// columns; tiles are dealt round-robin. The next tile's packed codes are copied by the bulk-copy
+// engine while the current tile is computed; q, k and v arrive through 16-byte asynchronous
+// copies straight into the tensor cores' operand layout.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "stepq_device.cuh"
+#include "stepq_internal.h"
+#include "stepq_tile.cuh"
+#include "stepq_umma.cuh"
+
+namespace stepq {
+namespace {
+
+constexpr int D = 128;        // d_k = d_v
+constexpr int C = 64;         // tokens per tile pass (a shorter chunk is padded: k = q = v = 0,
+                              // beta = 0, g = 1 leave every result unchanged)
+constexpr int NT = 256;       // threads per CTA
+using M = DMap<D>;
+static_assert(M::kThreads == NT, "the refit runs on the decode kernel's thread mapping");
+
+struct WyArgs {
+    int B, H, num_tiles, chunk;
+    const uint16_t* q;        // [chunk][B][H][D] bf16
+    const uint16_t* k;
+    const uint16_t* v;
+    const float* beta;        // [chunk][B][H]
+    const float* gate;        // [chunk][B][H]
+    const uint8_t* bits;
+    const float* w;
+    const int64_t* head_off;
+    int64_t bytes_per_seq;
+    const uint8_t* packed_in;
+    const uint16_t* r_in;
+    const uint16_t* c_in;
+    uint8_t* packed_out;
+    uint16_t* r_out;
+    uint16_t* c_out;
+    float* o;                 // [chunk][B][H][D]
+    uint32_t* flags;          // device error word (bit 0: a bounded wait gave up)
+};
+
+// Per-slot and per-column work space of the refit (same fields as the decode kernel's).
+struct FitScratch {
+    alignas(16) float4 ak[1][D];
+    alignas(16) float4 rq[D];
+    alignas(16) float2 wsl[D];
+    alignas(16) float riq[D];
+    alignas(16) float colc[D];
+    alignas(16) float colb[D];
+    alignas(16) float col0[D];
+    alignas(16) float icol[D];
+    alignas(16) float red[M::kWarps][2][D];
+    alignas(16) float rowbuf[M::kWarps][32 * (M::RPT + 1)];
+};
+
+struct Small {
+    alignas(16) uint32_t hmeta[D];   // per slot: row | width << 8 | byte offset << 16
+    alignas(16) uint16_t hslot[D];   // per row: slot | width << 8
+    alignas(16) float rho[D];        // r_i 2^(8 - b_i)
+    alignas(16) float cs[D];         // c_j
+    alignas(16) float icol[D];       // 1 / c_j
+    alignas(16) float beta[C];
+    alignas(16) float l2g[C];        // log2 gamma_t (a zero gate counts as 2^-64)
+    alignas(8) uint64_t bar_mma;
+    alignas(8) uint64_t bar_codes;
+    uint32_t tmem;
+};
+
+// Shared-memory map (bytes). The work region is reused phase by phase.
+constexpr uint32_t OFF_KQ = 0;            // bf16 [K; Q]: rows t (k) and 64 + t (q), K-major over d
+constexpr uint32_t OFF_V = 32768;         // bf16 V: rows t, K-major over d
+constexpr uint32_t OFF_Z = 49152;         // bf16 codes Z: rows i, K-major over j
+constexpr uint32_t OFF_CODES = 81920;     // the tile's packed codes (bulk copy)
+constexpr uint32_t OFF_W = 98304;         // 128 KB work region, laid out per phase (see the kernel)
+constexpr uint32_t OFF_SMALL = 229376;
+constexpr uint32_t SMEM_BYTES = OFF_SMALL + sizeof(Small);
+static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
+static_assert(65536 + sizeof(FitScratch) <= OFF_SMALL - OFF_W, "refit work space");
+
+// TMEM columns (512 allocated): G = [K;Q] K^T | W, later S_C | U_v | [W S0; gamma Q S0 + P U/c]
+constexpr uint32_t TM_G = 0, TM_W = 64, TM_U = 192, TM_S = 320;
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+// Eight fp32 values -> high bf16 parts and low bf16 parts (x - hi), each as one 16-byte chunk.
+__device__ __forceinline__ void split8(const float x[8], uint4& hi, uint4& lo) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(x[2 * p], x[2 * p + 1]);
+        const float2 hf = __bfloat1622float2(hb);
+        h[p] = *reinterpret_cast<const uint32_t*>(&hb);
+        l[p] = bf16x2_bits(x[2 * p] - hf.x, x[2 * p + 1] - hf.y);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Eight fp32 values -> three bf16 parts (x = hi + mid + lo to 24 significant bits).
+__device__ __forceinline__ void split8x3(const float x[8], uint4& hi, uint4& mid, uint4& lo) {
+    uint32_t h[4], m[4], l[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(x[2 * p], x[2 * p + 1]);
+        const float2 hf = __bfloat1622float2(hb);
+        const float r0 = x[2 * p] - hf.x, r1 = x[2 * p + 1] - hf.y;
+        const __nv_bfloat162 mb = __floats2bfloat162_rn(r0, r1);
+        const float2 mf = __bfloat1622float2(mb);
+        h[p] = *reinterpret_cast<const uint32_t*>(&hb);
+        m[p] = *reinterpret_cast<const uint32_t*>(&mb);
+        l[p] = bf16x2_bits(r0 - mf.x, r1 - mf.y);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    mid = make_uint4(m[0], m[1], m[2], m[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// fp32 64 x 64 matrices (L, T) with the 16-byte chunks of a row rotated by the row index.
+__device__ __forceinline__ int sw64(int row, int col) {
+    return row * 64 + ((((col >> 2) ^ row) & 15) << 2) + (col & 3);
+}
+// fp32 128 x 128 boundary state X, chunks rotated by row % 8.
+__device__ __forceinline__ int swx(int row, int col) {
+    return row * D + ((((col >> 2) ^ row) & 7) | ((col >> 2) & ~7)) * 4 + (col & 3);
+}
+
+// 2^x with the special function unit (relative error about 2^-22). The running log2 of the gate
+// product is formed with the accurate log2f: its error would accumulate over the chunk.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float4 ld4(const float* m, int row, int col) {
+    return *reinterpret_cast<const float4*>(m + sw64(row, col));
+}
+__device__ __forceinline__ float4 fma4(float a, float4 b, float4 c) {
+    return make_float4(fmaf(a, b.x, c.x), fmaf(a, b.y, c.y), fmaf(a, b.z, c.z), fmaf(a, b.w, c.w));
+}
+
+// TMEM columns of this warp's lanes.
+__device__ __forceinline__ uint32_t tm_at(uint32_t tm, int warp, uint32_t col) {
+    return umma::tmem_at(tm, 32 * (warp & 3), static_cast<int>(col));
+}
+
+// The small inputs of a tile, loaded into registers one tile ahead: warp 0 the gates and betas
+// of tokens 2 lane and 2 lane + 1, warp 1 the head's row widths, threads < 128 r_i and c_i.
+struct Ahead {
+    float g0, g1, b0, b1;
+    uint32_t widths;
+    uint32_t rc;   // r_i | c_i << 16 (binary16 bits)
+};
+
+__device__ __forceinline__ Ahead load_ahead(const WyArgs& a, int tile, int tid, int warp, int lane) {
+    Ahead n{1.0f, 1.0f, 0.0f, 0.0f, 0u, 0u};
+    const int64_t T = a.num_tiles;
+    if (warp == 0) {
+        const int t0 = 2 * lane, t1 = t0 + 1;
+        if (t0 < a.chunk) { n.g0 = __ldg(a.gate + t0 * T + tile); n.b0 = __ldg(a.beta + t0 * T + tile); }
+        if (t1 < a.chunk) { n.g1 = __ldg(a.gate + t1 * T + tile); n.b1 = __ldg(a.beta + t1 * T + tile); }
+    } else if (warp == 1) {
+        n.widths = head_widths<D>(a.bits + static_cast<int64_t>(tile % a.H) * D, lane);
+    }
+    if (tid < D)
+        n.rc = static_cast<uint32_t>(__ldg(a.r_in + static_cast<int64_t>(tile) * D + tid)) |
+               static_cast<uint32_t>(__ldg(a.c_in + static_cast<int64_t>(tile) * D + tid)) << 16;
+    return n;
+}
+
+// q, k, v rows t < chunk (zero rows past it) of a tile into the K-major operand layout.
+__device__ __forceinline__ void load_tokens(const WyArgs& a, int tile, int tid, uint16_t* KQ, uint16_t* Vs) {
+    const int64_t T = a.num_tiles;
+#pragma unroll 4
+    for (int m = 0; m < 12; ++m) {
+        const int e = tid + NT * m;              // 3 matrices x 64 rows x 16 chunks
+        const int mat = e >> 10, row = (e & 7) | ((e >> 7) & 7) << 3, ch = (e >> 3) & 15;
+        const uint16_t* src = mat == 0 ? a.k : (mat == 1 ? a.q : a.v);
+        const bool valid = row < a.chunk;
+        src += (static_cast<int64_t>(valid ? row : 0) * T + tile) * D + 8 * ch;
+        uint16_t* dst = mat == 2 ? Vs + umma::kmajor_off(row, 8 * ch, D) : KQ + umma::kmajor_off(row + 64 * mat, 8 * ch, D);
+        cp_async16(dst, src, valid ? 16u : 0u);
+    }
+    cp_async_commit();
+}
+
+__device__ __forceinline__ void issue_codes(const WyArgs& a, int tile, uint8_t* dst, uint64_t* bar) {
+    const int b = tile / a.H, h = tile % a.H;
+    const int64_t hoff = a.head_off[h], hend = (h + 1 < a.H) ? a.head_off[h + 1] : a.bytes_per_seq;
+    const uint32_t bytes = static_cast<uint32_t>(min(hend - hoff, static_cast<int64_t>(D) * D));
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(dst, a.packed_in + static_cast<int64_t>(b) * a.bytes_per_seq + hoff, bytes, bar);
+}
+
+__global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    Small& sm = *reinterpret_cast<Small*>(smem + OFF_SMALL);
+    uint16_t* KQ = reinterpret_cast<uint16_t*>(smem + OFF_KQ);
+    uint16_t* Vs = reinterpret_cast<uint16_t*>(smem + OFF_V);
+    uint16_t* Zs = reinterpret_cast<uint16_t*>(smem + OFF_Z);
+    uint8_t* codes = smem + OFF_CODES;
+    // The work region, phase by phase (KB offsets):
+    //   B: [T''; T'] planes 0, 16, 32 | L 64 | T 80 | block products 96
+    //   C: [W rho; gamma Q rho] planes 0, 32, 64
+    //   D: U/c planes 0, 16 | U~ planes 32, 48, 64 | P planes 88, 96 (their MMA operand starts
+    //      8 KB earlier: rows 0-63 there only reach TMEM lanes already consumed)
+    //   E: X 0 | refit work space 64
+    uint8_t* W = smem + OFF_W;
+    auto h16 = [&](uint32_t kb) { return reinterpret_cast<uint16_t*>(W + 1024 * kb); };
+    uint16_t* AT[3] = {h16(0), h16(16), h16(32)};
+    float* Lf = reinterpret_cast<float*>(W + 64 * 1024);
+    float* Tf = reinterpret_cast<float*>(W + 80 * 1024);
+    float* Mt = reinterpret_cast<float*>(W + 96 * 1024);
+    uint16_t* WQ[3] = {h16(0), h16(32), h16(64)};
+    uint16_t* BUC[2] = {h16(0), h16(16)};
+    uint16_t* BUT[3] = {h16(32), h16(48), h16(64)};
+    uint16_t* Pp[2] = {h16(88), h16(96)};
+    float* X = reinterpret_cast<float*>(W);
+    FitScratch& fit = *reinterpret_cast<FitScratch*>(W + 64 * 1024);
+
+    if (tid == 0) {
+        mbar_init(&sm.bar_mma, 1);
+        mbar_init(&sm.bar_codes, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) umma::tmem_alloc(&sm.tmem, 512);
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    const uint32_t tm = sm.tmem;
+    uint32_t mma_phase = 0, codes_phase = 0;
+    bool codes_pending = false;
+    const int64_t T = a.num_tiles;
+
+    // Waits for the tensor core's last commit; false (uniformly over the CTA) if it never came.
+    auto wait_mma = [&]() -> bool {
+        const bool ok = mbar_wait_bounded(&sm.bar_mma, mma_phase, kWaitLimitNs, a.flags);
+        mma_phase ^= 1u;
+        const bool all = !__syncthreads_or(!ok);
+        umma::fence_after_sync();
+        return all;
+    };
+    // Orders this thread's shared-memory writes and TMEM reads before an MMA that the
+    // issuing thread starts after the barrier.
+    auto to_tensor_core = [&]() {
+        umma::fence_async_smem();
+        umma::fence_before_sync();
+        __syncthreads();
+    };
+
+    // The first tile's inputs; later tiles' arrive during the previous tile's refit.
+    Ahead nx{};
+    if (static_cast<int>(blockIdx.x) < a.num_tiles) {
+        if (tid == 0) {
+            issue_codes(a, blockIdx.x, codes, &sm.bar_codes);
+            codes_pending = true;
+        }
+        load_tokens(a, blockIdx.x, tid, KQ, Vs);
+        nx = load_ahead(a, blockIdx.x, tid, warp, lane);
+    }
+
+    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
+        const int b = tile / a.H, h = tile % a.H;
+        const int64_t tile_base = static_cast<int64_t>(b) * a.bytes_per_seq + a.head_off[h];
+        const int next = tile + gridDim.x;
+
+        // ---- A: tables, gates, scales, codes -----------------------------------------------
+        if (warp == 1) sort_head_rows_w<D, false>(nx.widths, sm.hmeta, sm.hslot, lane, a.flags);
+        if (warp == 0) {   // beta and the running log2 of the gate product (a zero gate counts 2^-64)
+            const float l0 = log2f(fmaxf(nx.g0, 0x1p-64f));
+            const float l1 = l0 + log2f(fmaxf(nx.g1, 0x1p-64f));
+            float inc = l1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += y;
+            }
+            const float excl = inc - l1;
+            sm.l2g[2 * lane] = excl + l0;
+            sm.l2g[2 * lane + 1] = excl + l1;
+            sm.beta[2 * lane] = nx.b0;
+            sm.beta[2 * lane + 1] = nx.b1;
+        }
+        __syncthreads();
+        float w_slot = 1.0f;   // row-impact factor of slot tid (used by the refit)
+        if (tid < D) {
+            const int bw = sm.hslot[tid] >> 8;
+            const float cj = half_bits_to_float(static_cast<uint16_t>(nx.rc >> 16));
+            sm.rho[tid] = half_bits_to_float(static_cast<uint16_t>(nx.rc & 0xFFFFu)) * znorm_of(bw);
+            sm.cs[tid] = cj;
+            sm.icol[tid] = 1.0f / cj;
+            w_slot = __ldg(a.w + static_cast<int64_t>(h) * D + (sm.hmeta[tid] & 0xFF));
+        }
+        const bool ok = mbar_wait_bounded(&sm.bar_codes, codes_phase, kWaitLimitNs, a.flags);
+        codes_phase ^= 1u;
+        if (__syncthreads_or(!ok)) break;
+        codes_pending = false;
+#pragma unroll 2
+        for (int m = 0; m < 8; ++m) {
+            const int e = tid + NT * m;              // 128 rows x 16 chunks, 8 rows per 8 lanes
+            const int i = (e & 7) | ((e >> 7) << 3), cc = (e >> 3) & 15;
+            const uint32_t hs = sm.hslot[i];
+            const uint8_t* row = codes + (sm.hmeta[hs & 0xFF] >> 16);
+            float2 z[4];
+            switch (hs >> 8) {
+                case 8: unpack8<D, 8>(row, cc, z); break;
+                case 6: unpack8<D, 6>(row, cc, z); break;
+                case 4: unpack8<D, 4>(row, cc, z); break;
+                default: unpack8<D, 2>(row, cc, z); break;
+            }
+            *reinterpret_cast<uint4*>(Zs + umma::kmajor_off(i, 8 * cc, D)) =
+                make_uint4(bf16x2_bits(z[0].x, z[0].y), bf16x2_bits(z[1].x, z[1].y), bf16x2_bits(z[2].x, z[2].y),
+                           bf16x2_bits(z[3].x, z[3].y));
+        }
+        cp_async_wait_all();
+        to_tensor_core();
+        if (tid == 0) {
+            umma::fence_after_sync();
+            const uint32_t id = umma::idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+                umma::mma_bf16(tm + TM_G, umma::desc_kmajor(KQ, ks, D), umma::desc_kmajor(KQ, ks, D), id, ks > 0);
+            umma::commit(&sm.bar_mma);
+            if (next < a.num_tiles) {   // the codes buffer is free: fetch the next tile's
+                issue_codes(a, next, codes, &sm.bar_codes);
+                codes_pending = true;
+            }
+        }
+        if (!wait_mma()) break;
+
+        // ---- B: L, T = (I + L)^-1, and the [T diag(beta); T diag(beta gamma)] planes ---------
+        if (warp < 2) {   // lanes 0-63: row t of K K^T
+            const int t = tid;
+            const float lt = sm.l2g[t], bt = sm.beta[t];
+#pragma unroll
+            for (int c32 = 0; c32 < 2; ++c32) {
+                float g[32];
+                umma::tmem_ld32(tm_at(tm, warp, TM_G + 32 * c32), g);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const int s0 = 32 * c32 + 4 * q4;
+                    const float4 l2 = *reinterpret_cast<const float4*>(sm.l2g + s0);
+                    const float ls[4] = {l2.x, l2.y, l2.z, l2.w};
+                    float l[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) l[e] = s0 + e < t ? bt * ex2(lt - ls[e]) * g[4 * q4 + e] : 0.0f;
+                    *reinterpret_cast<float4*>(Lf + sw64(t, s0)) = make_float4(l[0], l[1], l[2], l[3]);
+                }
+            }
+        } else {   // T above the diagonal blocks is zero
+            for (int e = tid - 64; e < 6 * 64; e += NT - 64) {
+                const int blk = e >> 6, rr = (e >> 2) & 15, cq = e & 3;
+                const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                *reinterpret_cast<float4*>(Tf + sw64(16 * bi + rr, 16 * bj + 4 * cq)) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        umma::fence_before_sync();
+        __syncthreads();
+        if (tid < 64) {   // diagonal 16 x 16 blocks by substitution, one column per thread
+            const int o = 16 * (tid >> 4), c = tid & 15;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) x[r] = r == c ? 1.0f : 0.0f;
+#pragma unroll
+            for (int r = 1; r < 16; ++r) {
+                float acc0 = 0.0f, acc1 = 0.0f;   // L_rr' = 0 for r' >= r
+#pragma unroll
+                for (int u4 = 0; u4 < (r + 3) / 4; ++u4) {
+                    const float4 l = ld4(Lf, o + r, o + 4 * u4);
+                    acc0 = fmaf(l.x, x[4 * u4], acc0);
+                    acc1 = fmaf(l.y, x[4 * u4 + 1], acc1);
+                    acc0 = fmaf(l.z, x[4 * u4 + 2], acc0);
+                    acc1 = fmaf(l.w, x[4 * u4 + 3], acc1);
+                }
+                if (r > c) x[r] = -(acc0 + acc1);
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tf[sw64(o + r, o + c)] = x[r];
+        }
+        __syncthreads();
+        // Block rows: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj, by distance lv = i - j; a thread
+        // computes four adjacent entries of one block.
+#pragma unroll
+        for (int lv = 1; lv <= 3; ++lv) {
+            const bool act = tid < 64 * (4 - lv);
+            const int j = tid >> 6, i = j + lv, ra = (tid >> 2) & 15, c4 = 4 * (tid & 3);
+            if (act) {
+                float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int u0 = 0; u0 < 16 * lv; u0 += 4) {
+                    const int u = 16 * j + u0;
+                    const float4 l = ld4(Lf, 16 * i + ra, u);
+                    m = fma4(l.x, ld4(Tf, u, 16 * j + c4), m);
+                    m = fma4(l.y, ld4(Tf, u + 1, 16 * j + c4), m);
+                    m = fma4(l.z, ld4(Tf, u + 2, 16 * j + c4), m);
+                    m = fma4(l.w, ld4(Tf, u + 3, 16 * j + c4), m);
+                }
+                *reinterpret_cast<float4*>(Mt + (j * 16 + ra) * 16 + c4) = m;
+            }
+            __syncthreads();
+            if (act) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int u0 = 0; u0 < 16; u0 += 4) {
+                    const float4 l = ld4(Tf, 16 * i + ra, 16 * i + u0);
+                    const float* mr = Mt + (j * 16 + u0) * 16 + c4;
+                    acc = fma4(l.x, *reinterpret_cast<const float4*>(mr), acc);
+                    acc = fma4(l.y, *reinterpret_cast<const float4*>(mr + 16), acc);
+                    acc = fma4(l.z, *reinterpret_cast<const float4*>(mr + 32), acc);
+                    acc = fma4(l.w, *reinterpret_cast<const float4*>(mr + 48), acc);
+                }
+                *reinterpret_cast<float4*>(Tf + sw64(16 * i + ra, 16 * j + c4)) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+            }
+            __syncthreads();
+        }
+        // [T''; T'] with T''_ts = T_ts beta_s (rows 0-63), T'_ts = T_ts beta_s gamma_s (rows 64-127).
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int e = tid + NT * m;              // 128 rows x 8 chunks
+            const int row = (e & 7) | ((e >> 6) << 3), cc = (e >> 3) & 7;
+            const int t = row & 63, s0 = 8 * cc;
+            const float4 t0 = ld4(Tf, t, s0), t1 = ld4(Tf, t, s0 + 4);
+            const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+            float x[8];
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                const float f = row < 64 ? sm.beta[s0 + p] : sm.beta[s0 + p] * ex2(sm.l2g[s0 + p]);
+                x[p] = tv[p] * f;
+            }
+            uint4 hi, mid, lo;
+            split8x3(x, hi, mid, lo);
+            *reinterpret_cast<uint4*>(AT[0] + umma::kmajor_off(row, s0, C)) = hi;
+            *reinterpret_cast<uint4*>(AT[1] + umma::kmajor_off(row, s0, C)) = mid;
+            *reinterpret_cast<uint4*>(AT[2] + umma::kmajor_off(row, s0, C)) = lo;
+        }
+        to_tensor_core();
+        if (tid == 0) {   // [T''; T'] K (W = T' K in lanes 64-127) and [T''; T'] V (U_v in lanes 0-63)
+            umma::fence_after_sync();
+            const uint32_t id = umma::idesc_bf16(128, 128, false, true);
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks) {
+                    const uint64_t da = umma::desc_kmajor(AT[p], ks, C);
+                    umma::mma_bf16(tm + TM_W, da, umma::desc_mnmajor(KQ, ks, D), id, p > 0 || ks > 0);
+                    umma::mma_bf16(tm + TM_U, da, umma::desc_mnmajor(Vs, ks, D), id, p > 0 || ks > 0);
+                }
+            umma::commit(&sm.bar_mma);
+        }
+        if (!wait_mma()) break;
+
+        // ---- C: the [W diag(rho); diag(gamma) Q diag(rho)] planes ---------------------------
+        {
+            const int t = 32 * (warp & 1) + lane, hf = warp >> 2;
+            if (warp & 2) {   // W rows from TMEM lanes 64 + t
+#pragma unroll
+                for (int c32 = 0; c32 < 2; ++c32) {
+                    float wv[32];
+                    umma::tmem_ld32(tm_at(tm, warp, TM_W + 64 * hf + 32 * c32), wv);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int i0 = 64 * hf + 32 * c32 + 8 * q;
+                        const float4 r0 = *reinterpret_cast<const float4*>(sm.rho + i0);
+                        const float4 r1 = *reinterpret_cast<const float4*>(sm.rho + i0 + 4);
+                        const float x[8] = {wv[8 * q] * r0.x, wv[8 * q + 1] * r0.y, wv[8 * q + 2] * r0.z,
+                                            wv[8 * q + 3] * r0.w, wv[8 * q + 4] * r1.x, wv[8 * q + 5] * r1.y,
+                                            wv[8 * q + 6] * r1.z, wv[8 * q + 7] * r1.w};
+                        uint4 hi, mid, lo;
+                        split8x3(x, hi, mid, lo);
+                        *reinterpret_cast<uint4*>(WQ[0] + umma::kmajor_off(t, i0, D)) = hi;
+                        *reinterpret_cast<uint4*>(WQ[1] + umma::kmajor_off(t, i0, D)) = mid;
+                        *reinterpret_cast<uint4*>(WQ[2] + umma::kmajor_off(t, i0, D)) = lo;
+                    }
+                }
+            } else {          // gamma_t q_t rho
+                const float gt = ex2(sm.l2g[t]);
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const int i0 = 64 * hf + 8 * cc;
+                    const uint4 qb = *reinterpret_cast<const uint4*>(KQ + umma::kmajor_off(64 + t, i0, D));
+                    const uint32_t qw[4] = {qb.x, qb.y, qb.z, qb.w};
+                    const float4 r0 = *reinterpret_cast<const float4*>(sm.rho + i0);
+                    const float4 r1 = *reinterpret_cast<const float4*>(sm.rho + i0 + 4);
+                    const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+                    float x[8];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        x[2 * p] = __uint_as_float(qw[p] << 16) * gt * rr[2 * p];
+                        x[2 * p + 1] = __uint_as_float(qw[p] & 0xFFFF0000u) * gt * rr[2 * p + 1];
+                    }
+                    uint4 hi, mid, lo;
+                    split8x3(x, hi, mid, lo);
+                    *reinterpret_cast<uint4*>(WQ[0] + umma::kmajor_off(64 + t, i0, D)) = hi;
+                    *reinterpret_cast<uint4*>(WQ[1] + umma::kmajor_off(64 + t, i0, D)) = mid;
+                    *reinterpret_cast<uint4*>(WQ[2] + umma::kmajor_off(64 + t, i0, D)) = lo;
+                }
+            }
+        }
+        to_tensor_core();
+        if (tid == 0) {   // [W rho; gamma Q rho] Z: lanes 0-63 W S0, lanes 64-127 gamma Q S0 (without c)
+            umma::fence_after_sync();
+            const uint32_t id = umma::idesc_bf16(128, 128, false, true);
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                    umma::mma_bf16(tm + TM_S, umma::desc_kmajor(WQ[p], ks, D), umma::desc_mnmajor(Zs, ks, D), id,
+                                   p > 0 || ks > 0);
+            umma::commit(&sm.bar_mma);
+        }
+        if (!wait_mma()) break;
+
+        // ---- D: U = U_v - (W S0) diag(c); the U/c and U~ planes; the P planes ---------------
+        {
+            const int t = 32 * (warp & 1) + lane, hf = warp >> 2;
+            if (!(warp & 2)) {   // TMEM lanes t: U_v and W S0
+                const float ratio = ex2(sm.l2g[C - 1] - sm.l2g[t]);
+#pragma unroll
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    float uv[16], ws[16];
+                    umma::tmem_ld16x2(tm_at(tm, warp, TM_U + 64 * hf + 16 * c16), tm_at(tm, warp, TM_S + 64 * hf + 16 * c16),
+                                      uv, ws);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int j0 = 64 * hf + 16 * c16 + 8 * half;
+                        float xc[8], xt[8];
+#pragma unroll
+                        for (int p = 0; p < 8; ++p) {
+                            const float u = fmaf(-sm.cs[j0 + p], ws[8 * half + p], uv[8 * half + p]);
+                            xc[p] = u * sm.icol[j0 + p];
+                            xt[p] = u * ratio;
+                        }
+                        uint4 hi, lo;
+                        split8(xc, hi, lo);
+                        *reinterpret_cast<uint4*>(BUC[0] + umma::kmajor_off(t, j0, D)) = hi;
+                        *reinterpret_cast<uint4*>(BUC[1] + umma::kmajor_off(t, j0, D)) = lo;
+                        uint4 mid;
+                        split8x3(xt, hi, mid, lo);
+                        *reinterpret_cast<uint4*>(BUT[0] + umma::kmajor_off(t, j0, D)) = hi;
+                        *reinterpret_cast<uint4*>(BUT[1] + umma::kmajor_off(t, j0, D)) = mid;
+                        *reinterpret_cast<uint4*>(BUT[2] + umma::kmajor_off(t, j0, D)) = lo;
+                    }
+                }
+            } else {             // TMEM lanes 64 + t: Q K^T row t -> P row t, s in [32 hf, 32 hf + 32)
+                const float lt = sm.l2g[t];
+                float g[32];
+                umma::tmem_ld32(tm_at(tm, warp, TM_G + 32 * hf), g);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int s0 = 32 * hf + 8 * q;
+                    float x[8];
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) x[p] = s0 + p <= t ? ex2(lt - sm.l2g[s0 + p]) * g[8 * q + p] : 0.0f;
+                    uint4 hi, lo;
+                    split8(x, hi, lo);
+                    *reinterpret_cast<uint4*>(Pp[0] + umma::kmajor_off(t, s0, C)) = hi;
+                    *reinterpret_cast<uint4*>(Pp[1] + umma::kmajor_off(t, s0, C)) = lo;
+                }
+            }
+        }
+        to_tensor_core();
+        if (tid == 0) {
+            umma::fence_after_sync();
+            // O: lanes 64-127 of TM_S += P (U/c), three part products. The A operand's rows 0-63
+            // are the 8 KB before each P plane; they only add to lanes 0-63, already consumed.
+            const uint32_t id_o = umma::idesc_bf16(128, 128, false, true);
+#pragma unroll
+            for (int pq = 0; pq < 3; ++pq) {
+                const int p = pq == 2 ? 1 : 0, q = pq == 1 ? 1 : 0;
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    umma::mma_bf16(tm + TM_S, umma::desc_kmajor(Pp[p] - 64 * C, ks, C), umma::desc_mnmajor(BUC[q], ks, D),
+                                   id_o, 1u);
+            }
+            // S_C - gamma_C S0 = K^T U~ into the W columns (W was consumed in C).
+            const uint32_t id_s = umma::idesc_bf16(128, 128, true, true);
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    umma::mma_bf16(tm + TM_W, umma::desc_mnmajor(KQ, ks, D), umma::desc_mnmajor(BUT[p], ks, D), id_s,
+                                   p > 0 || ks > 0);
+            umma::commit(&sm.bar_mma);
+        }
+        if (!wait_mma()) break;
+
+        // ---- E: readouts, the boundary state X, its refit and pack --------------------------
+        {
+            const int hf = warp >> 2;
+            if (warp & 2) {   // o_t = c (gamma Q S0 + P U/c), TMEM lanes 64 + t
+                const int t = 32 * (warp & 1) + lane;
+                float* orow = a.o + (static_cast<int64_t>(t) * T + tile) * D;
+#pragma unroll
+                for (int c32 = 0; c32 < 2; ++c32) {
+                    float ov[32];
+                    umma::tmem_ld32(tm_at(tm, warp, TM_S + 64 * hf + 32 * c32), ov);
+                    if (t < a.chunk) {
+                        const int j0 = 64 * hf + 32 * c32;
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 cj = *reinterpret_cast<const float4*>(sm.cs + j0 + 4 * q4);
+                            *reinterpret_cast<float4*>(orow + j0 + 4 * q4) =
+                                make_float4(cj.x * ov[4 * q4], cj.y * ov[4 * q4 + 1], cj.z * ov[4 * q4 + 2], cj.w * ov[4 * q4 + 3]);
+                        }
+                    }
+                }
+            }
+            // X_ij = (K^T U~)_ij + gamma_C rho_i c_j Z_ij, TMEM lane i, columns j in [64 hf, 64 hf + 64).
+            const int i = 32 * (warp & 3) + lane;
+            const float fi = ex2(sm.l2g[C - 1]) * sm.rho[i];
+#pragma unroll
+            for (int c32 = 0; c32 < 2; ++c32) {
+                float sv[32];
+                umma::tmem_ld32(tm_at(tm, warp, TM_W + 64 * hf + 32 * c32), sv);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int j0 = 64 * hf + 32 * c32 + 8 * q;
+                    const uint4 zb = *reinterpret_cast<const uint4*>(Zs + umma::kmajor_off(i, j0, D));
+                    const uint32_t zw[4] = {zb.x, zb.y, zb.z, zb.w};
+                    const float4 c0 = *reinterpret_cast<const float4*>(sm.cs + j0);
+                    const float4 c1 = *reinterpret_cast<const float4*>(sm.cs + j0 + 4);
+                    const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                    float x[8];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        x[2 * p] = fmaf(fi * cc[2 * p], __uint_as_float(zw[p] << 16), sv[8 * q + 2 * p]);
+                        x[2 * p + 1] = fmaf(fi * cc[2 * p + 1], __uint_as_float(zw[p] & 0xFFFF0000u), sv[8 * q + 2 * p + 1]);
+                    }
+                    *reinterpret_cast<float4*>(X + swx(i, j0)) = make_float4(x[0], x[1], x[2], x[3]);
+                    *reinterpret_cast<float4*>(X + swx(i, j0 + 4)) = make_float4(x[4], x[5], x[6], x[7]);
+                }
+            }
+            if (tid < D) {   // the refit's constants: alpha = 1 and c = 1 (X is explicit)
+                fit.wsl[tid] = make_float2(w_slot, rcp_approx(w_slot));
+                fit.ak[0][tid] = make_float4(0.0f, 0.0f, 1.0f, 1.0f);
+                fit.colc[tid] = 1.0f;
+            }
+        }
+        umma::fence_before_sync();
+        __syncthreads();
+        if (next < a.num_tiles) {   // the next tile's q, k, v and small inputs arrive during the refit
+            load_tokens(a, next, tid, KQ, Vs);
+            nx = load_ahead(a, next, tid, warp, lane);
+        }
+        {
+            float2 Zr[M::RPT][4];
+            const int cl = M::col_lane(lane);
+#pragma unroll
+            for (int r = 0; r < M::RPT; ++r) {
+                const int row = sm.hmeta[M::row(warp, lane, r)] & 0xFF;
+                const float4 x0 = *reinterpret_cast<const float4*>(X + swx(row, 8 * cl));
+                const float4 x1 = *reinterpret_cast<const float4*>(X + swx(row, 8 * cl + 4));
+                Zr[r][0] = make_float2(x0.x, x0.y);
+                Zr[r][1] = make_float2(x0.z, x0.w);
+                Zr[r][2] = make_float2(x1.x, x1.y);
+                Zr[r][3] = make_float2(x1.z, x1.w);
+            }
+            const int w0 = (sm.hmeta[warp * M::kRowsPerWarp] >> 8) & 0xFF;
+            const int w1 = (sm.hmeta[warp * M::kRowsPerWarp + M::kRowsPerWarp - 1] >> 8) & 0xFF;
+            const int ww = (w0 == w1) ? w0 : 0;
+            refit_pack<D, false, false>(fit, sm.hmeta, Zr, ww, 0, tile, a.r_out, a.c_out, a.packed_out + tile_base);
+        }
+        __syncthreads();   // the next tile rewrites the tables and the regions
+    }
+
+    // Copies still in flight (a wait above gave up) are waited for, boundedly, before exit.
+    cp_async_wait_all();
+    if (tid == 0 && codes_pending) mbar_wait_bounded(&sm.bar_codes, codes_phase, kWaitLimitNs, a.flags);
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) umma::tmem_free(tm, 512);
+}
+
+}  // namespace
+}  // namespace stepq
+
+using namespace stepq;
+
+extern "C" int stepq_prefill_chunk_wy(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
+                                      const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,
+                                      const float* w, const int64_t* head_off, int64_t bytes_per_seq,
+                                      const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,
+                                      uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream) {
+    const char* fn = "stepq_prefill_chunk_wy";
+    clear_error();
+    int rc = check_dims(dims, fn);
+    if (rc) return rc;
+    if (chunk < 1) return set_error(STEPQ_EINVAL, "%s: chunk=%d", fn, chunk);
+    if (dims.dk != D || dims.gate_per_channel || dims.pivots || chunk > C)
+        return set_error(STEPQ_EUNSUPPORTED,
+                         "%s: the tensor-core chunk form needs d = 128, scalar gates, no FP16 pivot rows and at most "
+                         "%d tokens (d=%d gate_per_channel=%d pivots=%d chunk=%d)",
+                         fn, C, dims.dk, dims.gate_per_channel, dims.pivots, chunk);
+    if (dims.B == 0) return STEPQ_OK;
+    rc = check_ptrs(fn, {{"q", q}, {"k", k}, {"v", v}, {"beta", beta}, {"gate", gate}, {"bits", bits}, {"w", w},
+                         {"head_off", head_off}, {"packed_in", packed_in}, {"r_in", r_in}, {"c_in", c_in},
+                         {"packed_out", packed_out}, {"r_out", r_out}, {"c_out", c_out}, {"o", o}});
+    if (rc) return rc;
+    if (bytes_per_seq <= 0 || (bytes_per_seq & 15))
+        return set_error(STEPQ_EINVAL, "%s: bytes_per_seq=%lld", fn, (long long)bytes_per_seq);
+    const long long tiles = static_cast<long long>(dims.B) * dims.H;
+    if (tiles > 0x7fffffffLL) return set_error(STEPQ_EINVAL, "%s: too many tiles", fn);
+    uint32_t* flags = nullptr;
+    rc = device_flags_ptr(&flags);
+    if (rc) return rc;
+    static int num_sms = 0;
+    static std::once_flag once;
+    static cudaError_t init_err = cudaSuccess;
+    std::call_once(once, [] {
+        int dev = 0;
+        init_err = cudaGetDevice(&dev);
+        if (init_err == cudaSuccess) init_err = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (init_err == cudaSuccess)
+            init_err = cudaFuncSetAttribute(prefill_wy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(SMEM_BYTES));
+    });
+    if (init_err != cudaSuccess) return set_error(STEPQ_ECUDA, "%s: %s", fn, cudaGetErrorString(init_err));
+    WyArgs a{dims.B, dims.H, static_cast<int>(tiles), chunk, q, k, v, beta, gate, bits, w, head_off, bytes_per_seq,
+             packed_in, r_in, c_in, packed_out, r_out, c_out, o, flags};
+    const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+    prefill_wy_kernel<<<grid, NT, SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(a);
+    return check_launch(fn);
+}

@@ -86,8 +86,8 @@ def test_allocation_rejects_infeasible_and_bad_arguments():
         api.stepq_allocate_bits(np.full((2, 3), np.nan), [4, 6, 8], 12, 0)
 
 
-def _dims(B=2, H=2, d=128, gpc=0):
-    return _lib.Dims(B, H, d, d, gpc)
+def _dims(B=2, H=2, d=128, gpc=0, pivots=0):
+    return _lib.Dims(B, H, d, d, gpc, pivots)
 
 
 def _fake(addr=0x10000):
@@ -149,3 +149,18 @@ def test_new_entry_points_validate_before_touching_cuda():
     bits[1, :3] = 16
     head_off, bps, _ = api.stepq_packed_layout(bits, 64)
     assert bps == oracle.layout(bits, 64)[1] == 64 * 6 // 8 * 125 + 64 * 2 * 3
+
+
+def test_tensor_core_prefill_refuses_shapes_it_does_not_cover():
+    """stepq_prefill_chunk_wy: d = 128, scalar gates, no pivot rows, 1 <= chunk <= 64; anything
+    else is STEPQ_EUNSUPPORTED (the sequential form covers it), checked before any CUDA call."""
+    lib = _lib.lib()
+    P = _fake
+    args = (*([P()] * 8), 4096, *([P()] * 7), None)
+    for dims, chunk in ((_dims(d=64), 8), (_dims(gpc=1), 8), (_dims(pivots=1), 8), (_dims(), 65)):
+        rc = lib.stepq_prefill_chunk_wy(dims, chunk, *args)
+        assert rc == _lib.STEPQ_EUNSUPPORTED and b"tensor-core chunk form" in lib.stepq_last_error()
+    assert lib.stepq_prefill_chunk_wy(_dims(), 0, *args) == _lib.STEPQ_EINVAL
+    assert lib.stepq_prefill_chunk_wy(_dims(B=0), 64, *args) == _lib.STEPQ_OK
+    rc = lib.stepq_prefill_chunk_wy(_dims(), 64, *([P()] * 8), 4097, *([P()] * 7), None)
+    assert rc == _lib.STEPQ_EINVAL

@@ -1,7 +1,8 @@
-"""GPU parity of the prefill chunk (reconstruct once, C full-precision gated Delta updates on
-the register-resident tile, fit and pack the boundary state once) against the oracle: every
-token's readout within 1e-3 relative, the boundary state under the decode step's criteria;
-one token identical to the fused decode step."""
+"""GPU parity of the prefill chunk (reconstruct once, C full-precision gated Delta updates, fit
+and pack the boundary state once) against the oracle, in both forms: the sequential form on the
+register-resident tile and the chunked WY form on the tensor cores. Every token's readout within
+1e-3 relative, the boundary state under the decode step's criteria; one token of the sequential
+form identical to the fused decode step; the two forms agree with each other to a few 1e-6."""
 import numpy as np
 import pytest
 
@@ -67,9 +68,100 @@ def test_one_token_chunk_is_the_decode_step():
     toks = _chunk(wl, 1, t0=3)
     td = _dev_tokens(toks)
     args = (dev(bits), dev(w), dev(head_off), bps, dev(packed), dev(r, torch.float16), dev(c, torch.float16))
-    a = api.stepq_prefill_chunk(td["q"], td["k"], td["v"], td["beta"], td["gate"], *args)
+    a = api.stepq_prefill_chunk(td["q"], td["k"], td["v"], td["beta"], td["gate"], *args, form="seq")
     b = api.stepq_decode_step(td["q"][0], td["k"][0], td["v"][0], td["beta"][0], td["gate"][0], *args)
     torch.cuda.synchronize()
     for x, y in zip(a[:3], b[:3]):
         assert torch.equal(x, y)
     assert torch.equal(a[3][0], b[3])
+
+
+def _run(api, td, bits, w, head_off, bps, packed, r, c, form, in_place=True):
+    import torch
+    pk, rr, cc = dev(packed), dev(r, torch.float16), dev(c, torch.float16)
+    outs = (pk, rr, cc) if in_place else (None, None, None)
+    res = api.stepq_prefill_chunk(td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w),
+                                  dev(head_off), bps, pk, rr, cc, *outs, form=form)
+    torch.cuda.synchronize()
+    return tuple(x.cpu().numpy() if x.dtype != torch.float16 else host_half(x) for x in res)
+
+
+def _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C):
+    p_r, r_r, c_r, o_r = oracle.prefill_chunk(toks, bits, w, packed, r, c)
+    p_g, r_g, c_g, og = res
+    for t in range(C):
+        err = np.abs(og[t] - o_r[t]).max(axis=-1) / np.maximum(np.abs(o_r[t]).max(axis=-1), 1e-30)
+        assert err.max() <= 1e-3, (t, err.max())
+    return compare_decode((p_g, r_g, c_g, og[-1]), (p_r, r_r, c_r, o_r[-1]), bits, d, B)
+
+
+@pytest.mark.parametrize("B,H,widths,C,in_place", [
+    (3, 5, (2, 4, 6, 8), 64, True),
+    (2, 7, (4, 6, 8), 17, False),     # a ragged chunk (padded to 64 inside)
+    (2, 3, (2, 4, 6, 8), 1, True),
+    (2, 2, (8,), 64, True),           # every row 8-bit
+    (2, 2, (2,), 40, True),           # every row 2-bit
+    (8, 40, (4, 6, 8), 33, True),     # 320 tiles: more tiles than SMs, the next codes prefetched
+    (4, 16, (8,), 64, True),          # 8-bit rows, 8192 columns: the column-scale rate is tight here
+])
+def test_tensor_core_prefill_matches_oracle(B, H, widths, C, in_place):
+    from recurrent_state_quantization_gated_b200 import api
+    d = 128
+    wl, bits, w, packed, r, c = _setup(d, B, H, widths, False, seed=7 * B + H + C)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    toks = _chunk(wl, C)
+    res = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, "wy", in_place)
+    _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C)
+    assert api.stepq_read_device_flags() == 0
+
+
+def test_tensor_core_prefill_with_fast_decaying_gates():
+    """Gates drawn in [0.2, 1] per token (and one exact zero): the gate products fall below
+    fp32's range inside the chunk; ratios of them stay exact (log domain)."""
+    from recurrent_state_quantization_gated_b200 import api
+    d, B, H, C = 128, 2, 3, 64
+    wl, bits, w, packed, r, c = _setup(d, B, H, (4, 6, 8), False, seed=77)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    toks = _chunk(wl, C)
+    rng = np.random.default_rng(5)
+    toks["gate"] = rng.uniform(0.2, 1.0, toks["gate"].shape).astype(np.float32)
+    toks["gate"][10, 0, 1] = 0.0
+    res = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, "wy")
+    _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C)
+
+
+def test_tensor_core_and_sequential_forms_agree():
+    """Same inputs through both forms: readouts within 2e-5 (max-normalised per tile) of each
+    other; scales within one binary16 ulp; codes equal up to one step on at most 0.1 %."""
+    from recurrent_state_quantization_gated_b200 import api
+    d, B, H, C = 128, 4, 8, 64
+    wl, bits, w, packed, r, c = _setup(d, B, H, (2, 4, 6, 8), False, seed=91)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    td = _dev_tokens(_chunk(wl, C))
+    pw, rw, cw, ow = _run(api, td, bits, w, head_off, bps, packed, r, c, "wy")
+    ps, rs, cs, os_ = _run(api, td, bits, w, head_off, bps, packed, r, c, "seq")
+    err = np.abs(ow - os_).max(axis=-1) / np.maximum(np.abs(os_).max(axis=-1), 1e-30)
+    assert err.max() <= 2e-5, err.max()
+    compare_decode((pw, rw, cw, ow[-1]), (ps, rs, cs, os_[-1]), bits, d, B)
+
+
+def test_tensor_core_prefill_full_size_sampled():
+    """The benchmark's prefill workload (GDN shape: 64 sequences x 32 heads, d = 128, 64-token
+    chunk) in one launch; the oracle checks four sampled sequences (every head of each)."""
+    import torch
+    from recurrent_state_quantization_gated_b200 import api
+    wl = synth.workload(1)
+    d, B, H, C = wl.d, wl.B, wl.H, 64
+    S0 = synth.initial_state(wl)
+    bits = synth.random_bits(H, d, choices=(4, 6, 8), seed=3)
+    w = synth.random_weights(H, d, seed=4)
+    seqs = [0, 21, 42, B - 1]
+    r, c = oracle.fit_scales(S0, w, bits)
+    packed = oracle.pack_state(S0, bits, r, c)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    toks = _chunk(wl, C)
+    p_g, r_g, c_g, o_g = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, "wy")
+    sub = {n: np.ascontiguousarray(a[:, seqs]) for n, a in toks.items()}
+    p_s = np.concatenate([packed[b * bps:(b + 1) * bps] for b in seqs])
+    res = (np.concatenate([p_g[b * bps:(b + 1) * bps] for b in seqs]), r_g[seqs], c_g[seqs], o_g[:, seqs])
+    _check_against_oracle(res, sub, bits, w, p_s, r[seqs], c[seqs], d, len(seqs), C)
