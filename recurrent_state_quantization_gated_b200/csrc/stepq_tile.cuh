@@ -239,7 +239,7 @@ __device__ __forceinline__ void phase6(const uint32_t* meta, uint8_t* out, int w
 // r_out and c_out point at the scales of tile `tile`, out at the tile's packed bytes.
 template <int D, bool kPiv, bool kUpdate, class Sm>
 __device__ __forceinline__ void refit_pack(Sm& sm, const uint32_t* meta, float2 (&Z)[DMap<D>::RPT][4], int ww, int kb,
-                                           int64_t tile, uint16_t* r_out, uint16_t* c_out, uint8_t* out) {
+                                           int tile, uint16_t* r_out, uint16_t* c_out, uint8_t* out) {
     using M = DMap<D>;
     constexpr int RPT = M::RPT;
     const int tid = threadIdx.x;
@@ -253,15 +253,15 @@ __device__ __forceinline__ void refit_pack(Sm& sm, const uint32_t* meta, float2 
         float part[RPT];
 #pragma unroll
         for (int r = 0; r < RPT; ++r) {
-            float acc = 0.f;
+            float2 ka = make_float2(0.f, 0.f);
             if constexpr (kUpdate) {
                 const float4 c = sm.ak[kb][M::row(warp, lane, r)];
-                const float2 ka = make_float2(c.x, c.y);
-#pragma unroll
-                for (int p = 0; p < 4; ++p) Z[r][p] = fma2(ka, ut[p], Z[r][p]);
+                ka = make_float2(c.x, c.y);
             }
+            float acc = 0.f;
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
+                if constexpr (kUpdate) Z[r][p] = fma2(ka, ut[p], Z[r][p]);
                 acc = fmaf(fabsf(Z[r][p].x), cf[p].x, acc);
                 acc = fmaf(fabsf(Z[r][p].y), cf[p].y, acc);
             }
@@ -277,7 +277,7 @@ __device__ __forceinline__ void refit_pack(Sm& sm, const uint32_t* meta, float2 
             const float2 w2 = sm.wsl[sl];
             const float alpha = sm.ak[kb][sl].z;
             const __half rh = scale_to_half(fmaxf(alpha * rsum * (1.0f / D), kHalfMinNormal) * w2.y);
-            r_out[tile * D + i] = __half_as_ushort(rh);
+            r_out[static_cast<int64_t>(tile) * D + i] = __half_as_ushort(rh);
             const float rs = __half2float(rh) * znorm_of(bw);
             if (kPiv && bw == 16) {   // FP16 pivot row: xi = alpha Y, outside the shared column fit
                 sm.rq[sl] = make_float4(alpha, alpha, 0.f, 0.f);
@@ -389,7 +389,7 @@ __device__ __forceinline__ void refit_pack(Sm& sm, const uint32_t* meta, float2 
         const float cj = sm.colc[j];
         const float c1 = ds > 0.f ? (cj * ns) * rcp_approx(ds) : sm.col0[j];
         const __half ch = scale_to_half(c1);
-        c_out[tile * D + j] = __half_as_ushort(ch);
+        c_out[static_cast<int64_t>(tile) * D + j] = __half_as_ushort(ch);
         sm.colb[j] = cj * rcp_approx(__half2float(ch));
     }
     __syncthreads();
