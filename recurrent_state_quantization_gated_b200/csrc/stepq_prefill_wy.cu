@@ -23,7 +23,9 @@
 // runs through the same refit and pack as the fused decode step (steps 4-6 of Table C2).
 //
 // One CTA per SM (the operands of a tile take 224 KB of shared memory), 256 threads, 512 TMEM
-// columns; tiles are dealt round-robin. The next tile's packed codes are copied by the bulk-copy
+// columns; tiles are dealt round-robin. With one CTA of 8 warps per SM the phases' code must
+// stay small: loops whose bodies are large are kept rolled (instruction-cache misses were the
+// first stall reason when they were unrolled). The next tile's packed codes are copied by the bulk-copy
 // engine while the current tile is computed; q, k and v arrive through 16-byte asynchronous
 // copies straight into the tensor cores' operand layout.
 #include <cuda_runtime.h>
@@ -188,12 +190,20 @@ __device__ __forceinline__ uint32_t tm_at(uint32_t tm, int warp, uint32_t col) {
 struct Ahead {
     float g0, g1, b0, b1;
     uint32_t widths;
-    uint32_t rc;   // r_i | c_i << 16 (binary16 bits)
+    uint32_t rc;          // r_i | c_i << 16 (binary16 bits)
+    int64_t codes_src;    // thread 0: the packed codes of the tile after this one (their copy is
+    uint32_t codes_bytes; // queued while this one is computed), or 0 bytes if there is none
 };
 
 __device__ __forceinline__ Ahead load_ahead(const WyArgs& a, int tile, int tid, int warp, int lane) {
-    Ahead n{1.0f, 1.0f, 0.0f, 0.0f, 0u, 0u};
+    Ahead n{1.0f, 1.0f, 0.0f, 0.0f, 0u, 0u, 0, 0u};
     const int64_t T = a.num_tiles;
+    if (tid == 0 && tile + static_cast<int>(gridDim.x) < a.num_tiles) {
+        const int t2 = tile + gridDim.x, b2 = t2 / a.H, h2 = t2 % a.H;
+        const int64_t hoff = a.head_off[h2], hend = (h2 + 1 < a.H) ? a.head_off[h2 + 1] : a.bytes_per_seq;
+        n.codes_src = static_cast<int64_t>(b2) * a.bytes_per_seq + hoff;
+        n.codes_bytes = static_cast<uint32_t>(min(hend - hoff, static_cast<int64_t>(D) * D));
+    }
     if (warp == 0) {
         const int t0 = 2 * lane, t1 = t0 + 1;
         if (t0 < a.chunk) { n.g0 = __ldg(a.gate + t0 * T + tile); n.b0 = __ldg(a.beta + t0 * T + tile); }
@@ -210,7 +220,7 @@ __device__ __forceinline__ Ahead load_ahead(const WyArgs& a, int tile, int tid, 
 // q, k, v rows t < chunk (zero rows past it) of a tile into the K-major operand layout.
 __device__ __forceinline__ void load_tokens(const WyArgs& a, int tile, int tid, uint16_t* KQ, uint16_t* Vs) {
     const int64_t T = a.num_tiles;
-#pragma unroll 4
+#pragma unroll 1
     for (int m = 0; m < 12; ++m) {
         const int e = tid + NT * m;              // 3 matrices x 64 rows x 16 chunks
         const int mat = e >> 10, row = (e & 7) | ((e >> 7) & 7) << 3, ch = (e >> 3) & 15;
@@ -240,7 +250,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
     uint16_t* Zs = reinterpret_cast<uint16_t*>(smem + OFF_Z);
     uint8_t* codes = smem + OFF_CODES;
     // The work region, phase by phase (KB offsets):
-    //   B: [T''; T'] planes 0, 16, 32 | L 64 | T 80 | block products 96
+    //   B: [T''; T'] planes 0, 16, 32 | L 64 | T 80 | G blocks 96
     //   C: [W rho; gamma Q rho] planes 0, 32, 64
     //   D: U/c planes 0, 16 | U~ planes 32, 48, 64 | P planes 88, 96 (their MMA operand starts
     //      8 KB earlier: rows 0-63 there only reach TMEM lanes already consumed)
@@ -250,7 +260,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
     uint16_t* AT[3] = {h16(0), h16(16), h16(32)};
     float* Lf = reinterpret_cast<float*>(W + 64 * 1024);
     float* Tf = reinterpret_cast<float*>(W + 80 * 1024);
-    float* Mt = reinterpret_cast<float*>(W + 96 * 1024);
+    float* Gt = reinterpret_cast<float*>(W + 96 * 1024);
     uint16_t* WQ[3] = {h16(0), h16(32), h16(64)};
     uint16_t* BUC[2] = {h16(0), h16(16)};
     uint16_t* BUT[3] = {h16(32), h16(48), h16(64)};
@@ -335,7 +345,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
         codes_phase ^= 1u;
         if (__syncthreads_or(!ok)) break;
         codes_pending = false;
-#pragma unroll 2
+#pragma unroll 1
         for (int m = 0; m < 8; ++m) {
             const int e = tid + NT * m;              // 128 rows x 16 chunks, 8 rows per 8 lanes
             const int i = (e & 7) | ((e >> 7) << 3), cc = (e >> 3) & 15;
@@ -361,8 +371,9 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             for (int ks = 0; ks < D / 16; ++ks)
                 umma::mma_bf16(tm + TM_G, umma::desc_kmajor(KQ, ks, D), umma::desc_kmajor(KQ, ks, D), id, ks > 0);
             umma::commit(&sm.bar_mma);
-            if (next < a.num_tiles) {   // the codes buffer is free: fetch the next tile's
-                issue_codes(a, next, codes, &sm.bar_codes);
+            if (nx.codes_bytes) {   // the codes buffer is free: fetch the next tile's
+                mbar_arrive_expect_tx(&sm.bar_codes, nx.codes_bytes);
+                bulk_load(codes, a.packed_in + nx.codes_src, nx.codes_bytes, &sm.bar_codes);
                 codes_pending = true;
             }
         }
@@ -372,7 +383,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
         if (warp < 2) {   // lanes 0-63: row t of K K^T
             const int t = tid;
             const float lt = sm.l2g[t], bt = sm.beta[t];
-#pragma unroll
+#pragma unroll 1
             for (int c32 = 0; c32 < 2; ++c32) {
                 float g[32];
                 umma::tmem_ld32(tm_at(tm, warp, TM_G + 32 * c32), g);
@@ -419,43 +430,48 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             for (int r = 0; r < 16; ++r) Tf[sw64(o + r, o + c)] = x[r];
         }
         __syncthreads();
-        // Block rows: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj, by distance lv = i - j; a thread
-        // computes four adjacent entries of one block.
+        // Block rows: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj = -sum_k G_ik T_kj with G_ik = T_ii L_ik,
+        // formed once; then one level per distance lv = i - j. A thread computes four adjacent
+        // entries of one 16 x 16 block.
+#pragma unroll 1
+        for (int e = tid; e < 6 * 64; e += NT) {
+            const int pr = e >> 6, ra = (e >> 2) & 15, c4 = 4 * (e & 3);
+            const int i = pr < 1 ? 1 : (pr < 3 ? 2 : 3), k = pr - i * (i - 1) / 2;
+            float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int lv = 1; lv <= 3; ++lv) {
-            const bool act = tid < 64 * (4 - lv);
-            const int j = tid >> 6, i = j + lv, ra = (tid >> 2) & 15, c4 = 4 * (tid & 3);
-            if (act) {
-                float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int u0 = 0; u0 < 16 * lv; u0 += 4) {
-                    const int u = 16 * j + u0;
-                    const float4 l = ld4(Lf, 16 * i + ra, u);
-                    m = fma4(l.x, ld4(Tf, u, 16 * j + c4), m);
-                    m = fma4(l.y, ld4(Tf, u + 1, 16 * j + c4), m);
-                    m = fma4(l.z, ld4(Tf, u + 2, 16 * j + c4), m);
-                    m = fma4(l.w, ld4(Tf, u + 3, 16 * j + c4), m);
-                }
-                *reinterpret_cast<float4*>(Mt + (j * 16 + ra) * 16 + c4) = m;
+            for (int u0 = 0; u0 < 16; u0 += 4) {
+                const float4 t = ld4(Tf, 16 * i + ra, 16 * i + u0);
+                g = fma4(t.x, ld4(Lf, 16 * i + u0, 16 * k + c4), g);
+                g = fma4(t.y, ld4(Lf, 16 * i + u0 + 1, 16 * k + c4), g);
+                g = fma4(t.z, ld4(Lf, 16 * i + u0 + 2, 16 * k + c4), g);
+                g = fma4(t.w, ld4(Lf, 16 * i + u0 + 3, 16 * k + c4), g);
             }
-            __syncthreads();
-            if (act) {
+            *reinterpret_cast<float4*>(Gt + (pr * 16 + ra) * 16 + c4) = g;
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int lv = 1; lv <= 3; ++lv) {
+            if (tid < 64 * (4 - lv)) {
+                const int j = tid >> 6, i = j + lv, ra = (tid >> 2) & 15, c4 = 4 * (tid & 3);
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+                for (int k = j; k < i; ++k) {
+                    const float* gr = Gt + ((i * (i - 1) / 2 + k) * 16 + ra) * 16;
 #pragma unroll
-                for (int u0 = 0; u0 < 16; u0 += 4) {
-                    const float4 l = ld4(Tf, 16 * i + ra, 16 * i + u0);
-                    const float* mr = Mt + (j * 16 + u0) * 16 + c4;
-                    acc = fma4(l.x, *reinterpret_cast<const float4*>(mr), acc);
-                    acc = fma4(l.y, *reinterpret_cast<const float4*>(mr + 16), acc);
-                    acc = fma4(l.z, *reinterpret_cast<const float4*>(mr + 32), acc);
-                    acc = fma4(l.w, *reinterpret_cast<const float4*>(mr + 48), acc);
+                    for (int u0 = 0; u0 < 16; u0 += 4) {
+                        const float4 g = *reinterpret_cast<const float4*>(gr + u0);
+                        acc = fma4(g.x, ld4(Tf, 16 * k + u0, 16 * j + c4), acc);
+                        acc = fma4(g.y, ld4(Tf, 16 * k + u0 + 1, 16 * j + c4), acc);
+                        acc = fma4(g.z, ld4(Tf, 16 * k + u0 + 2, 16 * j + c4), acc);
+                        acc = fma4(g.w, ld4(Tf, 16 * k + u0 + 3, 16 * j + c4), acc);
+                    }
                 }
                 *reinterpret_cast<float4*>(Tf + sw64(16 * i + ra, 16 * j + c4)) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
             }
             __syncthreads();
         }
         // [T''; T'] with T''_ts = T_ts beta_s (rows 0-63), T'_ts = T_ts beta_s gamma_s (rows 64-127).
-#pragma unroll
+#pragma unroll 1
         for (int m = 0; m < 4; ++m) {
             const int e = tid + NT * m;              // 128 rows x 8 chunks
             const int row = (e & 7) | ((e >> 6) << 3), cc = (e >> 3) & 7;
@@ -494,7 +510,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
         {
             const int t = 32 * (warp & 1) + lane, hf = warp >> 2;
             if (warp & 2) {   // W rows from TMEM lanes 64 + t
-#pragma unroll
+#pragma unroll 1
                 for (int c32 = 0; c32 < 2; ++c32) {
                     float wv[32];
                     umma::tmem_ld32(tm_at(tm, warp, TM_W + 64 * hf + 32 * c32), wv);
@@ -515,7 +531,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                 }
             } else {          // gamma_t q_t rho
                 const float gt = ex2(sm.l2g[t]);
-#pragma unroll
+#pragma unroll 1
                 for (int cc = 0; cc < 8; ++cc) {
                     const int i0 = 64 * hf + 8 * cc;
                     const uint4 qb = *reinterpret_cast<const uint4*>(KQ + umma::kmajor_off(64 + t, i0, D));
@@ -556,7 +572,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             const int t = 32 * (warp & 1) + lane, hf = warp >> 2;
             if (!(warp & 2)) {   // TMEM lanes t: U_v and W S0
                 const float ratio = ex2(sm.l2g[C - 1] - sm.l2g[t]);
-#pragma unroll
+#pragma unroll 1
                 for (int c16 = 0; c16 < 4; ++c16) {
                     float uv[16], ws[16];
                     umma::tmem_ld16x2(tm_at(tm, warp, TM_U + 64 * hf + 16 * c16), tm_at(tm, warp, TM_S + 64 * hf + 16 * c16),
@@ -631,7 +647,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             if (warp & 2) {   // o_t = c (gamma Q S0 + P U/c), TMEM lanes 64 + t
                 const int t = 32 * (warp & 1) + lane;
                 float* orow = a.o + (static_cast<int64_t>(t) * T + tile) * D;
-#pragma unroll
+#pragma unroll 1
                 for (int c32 = 0; c32 < 2; ++c32) {
                     float ov[32];
                     umma::tmem_ld32(tm_at(tm, warp, TM_S + 64 * hf + 32 * c32), ov);
@@ -649,7 +665,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             // X_ij = (K^T U~)_ij + gamma_C rho_i c_j Z_ij, TMEM lane i, columns j in [64 hf, 64 hf + 64).
             const int i = 32 * (warp & 3) + lane;
             const float fi = ex2(sm.l2g[C - 1]) * sm.rho[i];
-#pragma unroll
+#pragma unroll 1
             for (int c32 = 0; c32 < 2; ++c32) {
                 float sv[32];
                 umma::tmem_ld32(tm_at(tm, warp, TM_W + 64 * hf + 32 * c32), sv);

@@ -143,6 +143,44 @@ def calibrate(alloc: str, candidates, nominal_bits: int, unit_gates, S0: torch.T
     raise ValueError(f"unknown allocation {alloc!r}")
 
 
+TOKEN_FIELDS = ("q", "k", "v", "beta", "gate")
+
+
+def _token_parts(tok: dict):
+    """(name, uint8 view, dtype, shape, offset) of each token input in the packed order; every
+    part starts on a 16-byte boundary (the library's alignment rule)."""
+    parts, off = [], 0
+    for name in TOKEN_FIELDS:
+        a = np.ascontiguousarray(tok[name])
+        raw = a.view(np.uint8).reshape(-1)
+        parts.append((name, raw, a.dtype, a.shape, off))
+        off += (raw.size + 15) // 16 * 16
+    return parts, off
+
+
+def pack_tokens(tok: dict) -> np.ndarray:
+    """The token inputs of one step (or one chunk) as one contiguous byte buffer:
+    q | k | v | beta | gate, so that moving them to the GPU is a single copy."""
+    parts, size = _token_parts(tok)
+    buf = np.zeros(size, dtype=np.uint8)
+    for _, raw, _, _, off in parts:
+        buf[off:off + raw.size] = raw
+    return buf
+
+
+def token_views(buf: torch.Tensor, like: dict) -> dict:
+    """Typed views (q, k, v bf16; beta, gate fp32) into a packed token buffer `buf` (uint8, on
+    any device) laid out by pack_tokens for host tokens shaped like `like`."""
+    parts, size = _token_parts(like)
+    if buf.numel() != size:
+        raise ValueError(f"packed token buffer holds {buf.numel()} bytes, expected {size}")
+    out = {}
+    for name, raw, dtype, shape, off in parts:
+        seg = buf[off:off + raw.size]
+        out[name] = seg.view(torch.bfloat16 if dtype == np.uint16 else torch.float32).view(shape)
+    return out
+
+
 def to_device_tokens(tok: dict, device="cuda") -> dict:
     """Host token arrays (bf16 bit patterns as uint16) to GPU tensors of the right dtypes."""
     out = {}
