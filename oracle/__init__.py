@@ -251,6 +251,25 @@ def prefill_chunk(toks, bits, w, packed, r, c, nthreads=0):
     return p_out, r_out, c_out, o
 
 
+def leap_window(toks, codes, s, nthreads=0):
+    """A window of W tokens on the per-window 8-bit state (LeapQuant's per-window quantisation
+    as read from its abstract): toks holds q, k, v, beta, gate with a leading token axis
+    [W][B][H]...; the state is the rowwise-absmax INT8 codes [B][H][dk][dv] with scales s
+    (binary16 bits) [B][H][dk]. Every token's readout comes from the exact (float64) running
+    state; the window's final state is quantised once. Returns (codes_out, s_out, o [W][B][H][dv])."""
+    q = _c(toks["q"], np.uint16); k = _c(toks["k"], np.uint16); v = _c(toks["v"], np.uint16)
+    beta = _c(toks["beta"], np.float32); gate = _c(toks["gate"], np.float32)
+    codes = _c(codes, np.int8); s = _c(s, np.uint16)
+    W, B, H, dk = q.shape
+    dv = v.shape[3]
+    gpc = int(gate.ndim == 4)
+    c_out = np.zeros_like(codes); s_out = np.zeros_like(s)
+    o = np.zeros((W, B, H, dv), dtype=np.float32)
+    _check(lib().orc_leap_window(W, B, H, dk, dv, gpc, _p(q), _p(k), _p(v), _p(beta), _p(gate), _p(codes),
+                                 _p(s), _p(c_out), _p(s_out), _p(o), nthreads), "leap_window")
+    return c_out, s_out, o
+
+
 def decode_step_fp32(tok, S, nthreads=0):
     q = _c(tok["q"], np.uint16); k = _c(tok["k"], np.uint16); v = _c(tok["v"], np.uint16)
     beta = _c(tok["beta"], np.float32); gate = _c(tok["gate"], np.float32)

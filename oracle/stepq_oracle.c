@@ -628,6 +628,48 @@ int orc_prefill_chunk(int C, int B, int H, int dk, int dv, int gate_per_channel,
     return ORC_OK;
 }
 
+/* Per-window 8-bit state (LeapQuant, "Compensator Tokens and per-window quantization", abstract:
+   the state is quantised once at the end of a window of tokens; inside the window, readouts come
+   from the fixed low-bit state together with high-precision buffered updates). Reading: the
+   state between windows is the rowwise-absmax INT8 format of §5.1 (orc_int8_quantise_tile); a
+   window of W tokens applies the gated Delta rule exactly (float64) to the reconstructed state
+   S_hat = diag(s) codes, every token's readout taken from that running state (which is what the
+   fixed state plus the buffered updates equal), and the window's final state is quantised once.
+   Token inputs carry a leading token axis of B*H tiles each, like orc_prefill_chunk. */
+int orc_leap_window(int W, int B, int H, int dk, int dv, int gate_per_channel, const uint16_t* q,
+                    const uint16_t* k, const uint16_t* v, const float* beta, const float* gate,
+                    const int8_t* codes_in, const uint16_t* s_in, int8_t* codes_out, uint16_t* s_out,
+                    float* o, int nthreads) {
+    if (!orc_dims_ok(dk, dv)) return ORC_EUNSUPPORTED;
+    if (W < 1) return ORC_EINVAL;
+    int nt = set_threads(nthreads);
+    int64_t n = (int64_t)B * H;
+    int gstride = gate_per_channel ? dk : 1;
+    (void)nt;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt)
+    for (int64_t tl = 0; tl < n; ++tl) {
+        orc_tile_scratch t;
+        scratch_alloc(&t, dk, dv);
+        float* S32 = (float*)malloc(sizeof(float) * dk * dv);
+        for (int i = 0; i < dk; ++i) {
+            float si = orc_half_to_float(s_in[tl * dk + i]);
+            for (int j = 0; j < dv; ++j) t.S[i * dv + j] = (double)(si * (float)codes_in[(tl * dk + i) * dv + j]);
+        }
+        for (int c = 0; c < W; ++c) {
+            int64_t tc = (int64_t)c * n + tl;
+            tile_inputs(&t, q + tc * dk, k + tc * dk, v + tc * dv, gate + tc * gstride, gate_per_channel);
+            orc_delta_update(dk, dv, t.S, t.q, t.k, t.v, (double)beta[tc], t.g, t.X, t.o);
+            for (int j = 0; j < dv; ++j) o[tc * dv + j] = (float)t.o[j];
+            memcpy(t.S, t.X, sizeof(double) * dk * dv);            /* no quantisation inside the window */
+        }
+        for (int e = 0; e < dk * dv; ++e) S32[e] = (float)t.X[e];
+        orc_int8_quantise_tile(dk, dv, S32, codes_out + tl * dk * dv, s_out + tl * dk);
+        free(S32);
+        scratch_free(&t);
+    }
+    return ORC_OK;
+}
+
 int orc_decode_step_fp32(int B, int H, int dk, int dv, int gate_per_channel, const uint16_t* q,
                          const uint16_t* k, const uint16_t* v, const float* beta, const float* gate,
                          const float* S_in, float* S_out, float* o, int nthreads) {
