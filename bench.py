@@ -50,10 +50,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--cpu-threads", type=int, default=0, help="oracle threads for cpu_baseline (0 = all cores)")
-    ap.add_argument("--kernel", choices=["quant", "split", "prefill", "fp32", "int8"], default="quant",
+    ap.add_argument("--kernel", choices=["quant", "split", "prefill", "fp32", "int8", "leap"], default="quant",
                     help="quant: the fused step; split: the split-form ablation; prefill: a chunk of --chunk "
                          "tokens per launch; fp32 / int8: comparison states")
     ap.add_argument("--chunk", type=int, default=64, help="tokens per prefill chunk (--kernel prefill)")
+    ap.add_argument("--window", type=int, default=16, help="tokens per window of the per-window 8-bit state "
+                                                            "(--kernel leap)")
     ap.add_argument("--prefill-form", choices=["auto", "seq", "wy"], default="auto",
                     help="prefill chunk form: the library's choice, the sequential register-tile form, "
                          "or the chunked WY form on the tensor cores")
@@ -206,6 +208,11 @@ def algorithmic_bytes(layout_bps: int, B: int, H: int, d: int, gate_per_channel:
         return 2 * B * layout_bps + tiles * 2 * (2 * d + 2 * d) + small + tiles * (3 * 4 * d * d + 4 * d)
     if kernel == "int8":
         return tiles * 2 * (d * d + 2 * d) + small
+    if kernel.startswith("leap"):   # one token on the per-window 8-bit state, averaged over a window
+        W = int(kernel.split(":")[1])
+        entry = 2 * d + 4 * d + 4                       # a buffered key (bf16), u (fp32) and log gate
+        per_tile = (d * d + 2 * d) + entry + (W - 1) / 2 * entry + (d * d + 2 * d + W * entry) / W
+        return int(tiles * per_tile) + small
     return tiles * 2 * (4 * d * d) + small
 
 
@@ -228,6 +235,8 @@ def job_throughput(world: int, tiles_per_rank: int, steps: int, ms: float) -> fl
 
 def workload_config(wl, bits, kernel: str, world: int, chunk: int = 1, prefill_form: str = "auto") -> dict:
     extra = {"chunk": chunk, "prefill_form": prefill_form} if kernel == "prefill" else {}
+    if kernel == "leap":
+        extra = {"window": chunk, "format": "rowwise-absmax INT8 between windows"}
     return {"workload": wl.name, "kernel": kernel, **extra, "B": wl.B, "H": wl.H, "d_k": wl.d, "d_v": wl.d,
             "bits_mean": float(np.asarray(bits, dtype=np.float64).mean()), "allocation": wl.alloc,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
@@ -352,8 +361,11 @@ def main():
     layout = runtime.Layout.build(bits, wl.d)
     base = runtime.QuantizedState.from_fp32(S0, layout, w)
     tiles = wl.B * wl.H
-    bytes_launch = algorithmic_bytes(layout.bytes_per_seq, wl.B, wl.H, wl.d, wl.gate_per_channel,
-                                     f"prefill:{args.chunk}" if args.kernel == "prefill" else args.kernel)
+    kname = {"prefill": f"prefill:{args.chunk}", "leap": f"leap:{args.window}"}.get(args.kernel, args.kernel)
+    bytes_launch = algorithmic_bytes(layout.bytes_per_seq, wl.B, wl.H, wl.d, wl.gate_per_channel, kname)
+    LW = args.window if args.kernel == "leap" else 1   # launches per replica per round (one window)
+    if args.kernel == "leap" and wl.gate_per_channel:
+        raise SystemExit("--kernel leap takes scalar gates (workloads 0, 1, 3, 4)")
 
     # Replicas: enough independent states that > 2x L2 is touched between reuses.
     per_rep = bytes_launch
@@ -367,18 +379,25 @@ def main():
             reps.append(dict(packed=base.packed.clone(), r=base.r.clone(), c=base.c.clone()))
         elif args.kernel == "fp32":
             reps.append(dict(S=S0.clone()))
+        elif args.kernel == "leap":
+            reps.append(dict(win=runtime.WindowState.from_fp32(S0, args.window)))
         else:
             cds, s = api.stepq_int8_quantize_state(S0)
             reps.append(dict(codes=cds, s=s))
         # Each replica's token inputs live in one packed device buffer (q | k | v | beta | gate),
-        # filled end to end by one host-to-device copy per step.
+        # filled end to end by one host-to-device copy per step (per window position for leap).
         if args.kernel == "prefill":
             steps = [synth.tokens(wl, (i * args.chunk + t) % wl.T) for t in range(args.chunk)]
             host = {n: np.ascontiguousarray(np.stack([x[n] for x in steps])) for n in steps[0]}
         else:
             host = synth.tokens(wl, i % wl.T)
-        tok_bufs.append(torch.from_numpy(runtime.pack_tokens(host)).cuda())
-        toks.append(runtime.token_views(tok_bufs[-1], host))
+        if args.kernel == "leap":
+            hosts = [synth.tokens(wl, (i * LW + t) % wl.T) for t in range(LW)]
+            tok_bufs.append([torch.from_numpy(runtime.pack_tokens(hh)).cuda() for hh in hosts])
+            toks.append([runtime.token_views(b_, hh) for b_, hh in zip(tok_bufs[-1], hosts)])
+        else:
+            tok_bufs.append(torch.from_numpy(runtime.pack_tokens(host)).cuda())
+            toks.append(runtime.token_views(tok_bufs[-1], host))
         oshape = (args.chunk, wl.B, wl.H, wl.d) if args.kernel == "prefill" else (wl.B, wl.H, wl.d)
         outs.append(torch.empty(oshape, dtype=torch.float32, device="cuda"))
     del S0
@@ -404,22 +423,28 @@ def main():
                                   st["packed"], st["r"], st["c"], o, pivots=layout.pivots)
         elif args.kernel == "fp32":
             api.stepq_decode_step_fp32(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], st["S"], st["S"], o)
+        elif args.kernel == "leap":
+            win = st["win"]
+            t_ = tk[win.t]
+            win.step(t_["q"], t_["k"], t_["v"], t_["beta"], t_["gate"], o)
         else:
             api.stepq_decode_step_int8(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], st["codes"], st["s"],
                                        st["codes"], st["s"], o)
 
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
-        for i in range(R):          # first launches outside capture (kernel attributes, occupancy)
-            launch(i)
+        for _ in range(LW):
+            for i in range(R):      # first launches outside capture (kernel attributes, occupancy)
+                launch(i)
     stream.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        for i in range(R):
-            launch(i)
-    rounds_warm = max(1, -(-args.warmup // R))
-    rounds = max(1, -(-args.steps // R))
-    K = rounds * R
+        for _ in range(LW):
+            for i in range(R):
+                launch(i)
+    rounds_warm = max(1, -(-args.warmup // (R * LW)))
+    rounds = max(1, -(-args.steps // (R * LW)))
+    K = rounds * R * LW
     with torch.cuda.stream(stream):
         for _ in range(rounds_warm):
             graph.replay()
@@ -475,7 +500,7 @@ def main():
     o_host = [torch.empty(tuple(outs[0].shape), dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = pinned[0].numel()
     d2h = o_host[0].numel() * o_host[0].element_size()
-    n_e2e = max(R, (args.e2e_steps // R) * R)
+    n_e2e = max(R * LW, (args.e2e_steps // (R * LW)) * R * LW)
     # Three streams: inputs in, decode, readout out. Step s's copies overlap the decode of
     # step s-1; buffers are reused R steps later, ordered by events.
     cs, ds = torch.cuda.Stream(), torch.cuda.Stream()
@@ -491,7 +516,8 @@ def main():
         with torch.cuda.stream(cs):
             if s_ >= R:
                 cs.wait_event(ev_k[i])          # the decode that last read toks[i] is done
-            tok_bufs[i].copy_(src, non_blocking=True)   # q, k, v, beta, gate in one copy
+            dst = tok_bufs[i][reps[i]["win"].t] if args.kernel == "leap" else tok_bufs[i]
+            dst.copy_(src, non_blocking=True)   # q, k, v, beta, gate in one copy
             ev_h[i].record(cs)
         with torch.cuda.stream(stream):
             stream.wait_event(ev_h[i])
@@ -514,10 +540,11 @@ def main():
     if rank == 0:
         clocks = clk.summary()
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": rounds_warm * R,
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": rounds_warm * R * LW,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": {**workload_config(wl, bits, args.kernel, world, args.chunk, args.prefill_form),
+            "config": {**workload_config(wl, bits, args.kernel, world,
+                                         args.window if args.kernel == "leap" else args.chunk, args.prefill_form),
                        "l2": (f"inputs larger than L2: {R} state replicas stepped round-robin, "
                               f"{R * per_rep / 2**20:.0f} MiB touched per round") if R * per_rep > L2_BYTES else
                              (f"inputs in L2 (latency case): {R} state replicas, "

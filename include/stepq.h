@@ -201,6 +201,24 @@ STEPQ_API int stepq_decode_step_int8(stepq_dims dims, const uint16_t* q, const u
                            const uint16_t* s_in, int8_t* codes_out, uint16_t* s_out, float* o,
                            void* stream);
 
+/* One token of the per-window 8-bit state (LeapQuant, "Compensator Tokens and per-window
+   quantization": quantise the state once at the end of a window of tokens; inside the window the
+   readouts come from the fixed low-bit state plus high-precision buffered updates). The state
+   between windows is the rowwise-absmax INT8 format above (codes, s). Token t of the window
+   (0 <= t < window <= STEPQ_LEAP_MAX_WINDOW) reads codes and s and the window's buffers entries
+   0 .. t-1, and writes entry t:
+     kbuf  bf16 [window][B][H][dk]  the window's keys,
+     ubuf  fp32 [window][B][H][dv]  the pseudo-values u_r = beta_r (v_r - g_r S_{r-1}^T k_r),
+     lbuf  fp32 [window][B][H]      the running log2 of the gate product (a zero gate counts 2^-64).
+   With gamma_r = 2^lbuf_r: o_t = S_t^T q_t with S_t = gamma_t S_hat + sum_{r<=t} (gamma_t/gamma_r)
+   k_r u_r^T, all in fp32; the last token (t = window - 1) also writes that state, requantised,
+   over codes and s. Scalar gates only (dims.gate_per_channel = 1 is STEPQ_EUNSUPPORTED); the
+   buffers belong to the caller and must not be changed while a window is open. */
+#define STEPQ_LEAP_MAX_WINDOW 256
+STEPQ_API int stepq_leap_step(stepq_dims dims, int window, int t, const uint16_t* q, const uint16_t* k,
+                    const uint16_t* v, const float* beta, const float* gate, int8_t* codes, uint16_t* s,
+                    uint16_t* kbuf, float* ubuf, float* lbuf, float* o, void* stream);
+
 /* Offline calibration (not on the decode path).
    Row impact (App. B.3, C.1) over a calibration stream of T steps, arrays with a leading
    step axis ([T][B][H]...): omega_{h,i} = mean_{t,b} (d_{t,i} (q_{t,i} - beta_t k_{t,i}

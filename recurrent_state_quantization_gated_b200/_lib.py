@@ -18,7 +18,7 @@ SYMBOLS = (
     "stepq_unpack_state", "stepq_decode_step", "stepq_decode_step_split", "stepq_prefill_chunk",
     "stepq_prefill_chunk_seq", "stepq_prefill_chunk_wy",
     "stepq_decode_step_fp32",
-    "stepq_int8_quantize_state", "stepq_decode_step_int8", "stepq_row_impact",
+    "stepq_int8_quantize_state", "stepq_decode_step_int8", "stepq_leap_step", "stepq_row_impact",
     "stepq_calib_distortion", "stepq_calib_distortion_bits", "stepq_calib_distortion_static", "stepq_allocate_bits", "stepq_read_device_flags",
     "stepq_build_info",
 )
@@ -56,6 +56,7 @@ _SIGNATURES = {
     "stepq_decode_step_fp32": ([Dims, P, P, P, P, P, P, P, P, P], I),
     "stepq_int8_quantize_state": ([Dims, P, P, P, P], I),
     "stepq_decode_step_int8": ([Dims, P, P, P, P, P, P, P, P, P, P, P], I),
+    "stepq_leap_step": ([Dims, I, I, P, P, P, P, P, P, P, P, P, P, P, P], I),
     "stepq_row_impact": ([Dims, I, P, P, P, P, P, P], I),
     "stepq_calib_distortion": ([Dims, P, P, I, P, P, P, P], I),
     "stepq_calib_distortion_static": ([Dims, P, P, I, P, P, P], I),

@@ -22,7 +22,7 @@ __all__ = [
     "stepq_packed_layout", "stepq_fit_scales", "stepq_pack_state", "stepq_unpack_state",
     "stepq_decode_step", "stepq_decode_step_split", "stepq_prefill_chunk",
     "stepq_prefill_chunk_seq", "stepq_prefill_chunk_wy", "stepq_decode_step_fp32", "stepq_int8_quantize_state",
-    "stepq_decode_step_int8", "stepq_row_impact", "stepq_calib_distortion", "stepq_calib_distortion_bits", "stepq_calib_distortion_static",
+    "stepq_decode_step_int8", "stepq_leap_step", "stepq_row_impact", "stepq_calib_distortion", "stepq_calib_distortion_bits", "stepq_calib_distortion_static",
     "stepq_allocate_bits",
     "stepq_read_device_flags", "stepq_build_info",
 ]
@@ -208,6 +208,20 @@ def stepq_decode_step_int8(q, k, v, beta, gate, codes_in, s_in, codes_out=None, 
          _ptr(codes_out, torch.int8, "codes_out"), _ptr(s_out, torch.float16, "s_out"), _ptr(o, torch.float32, "o"),
          _stream())
     return codes_out, s_out, o
+
+
+def stepq_leap_step(window, t, q, k, v, beta, gate, codes, s, kbuf, ubuf, lbuf, o=None):
+    """Token t of a window on the per-window 8-bit state: q, k, v [B,H,d], beta, gate [B,H];
+    codes int8 [B,H,d,d] and s fp16 [B,H,d] (rewritten at the window's last token); buffers
+    kbuf bf16 [window,B,H,d], ubuf fp32 [window,B,H,d], lbuf fp32 [window,B,H]. Returns o."""
+    B, H, d = q.shape
+    o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
+    call("stepq_leap_step", _dims(B, H, d, 0), ctypes.c_int(int(window)), ctypes.c_int(int(t)),
+         _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
+         _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"), _ptr(codes, torch.int8, "codes"),
+         _ptr(s, torch.float16, "s"), _ptr(kbuf, torch.bfloat16, "kbuf"), _ptr(ubuf, torch.float32, "ubuf"),
+         _ptr(lbuf, torch.float32, "lbuf"), _ptr(o, torch.float32, "o"), _stream())
+    return o
 
 
 def stepq_row_impact(q, k, beta, gate, w_out=None):

@@ -139,8 +139,8 @@ __global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) decode_f
 }
 
 // Rowwise absmax requantisation of a register tile; writes codes and scales.
-template <int D>
-__device__ __forceinline__ void int8_requantise(BaselineSmem<D>& sm, const float X[Map<D>::RPT][4], int tile,
+template <int D, class Sm>
+__device__ __forceinline__ void int8_requantise(Sm& sm, const float X[Map<D>::RPT][4], int tile,
                                                 int8_t* codes_out, uint16_t* s_out) {
     using M = Map<D>;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -210,6 +210,198 @@ __global__ void __launch_bounds__(Map<D>::kThreads) int8_quantize_kernel(const B
         X[r][0] = x.x; X[r][1] = x.y; X[r][2] = x.z; X[r][3] = x.w;
     }
     int8_requantise<D>(sm, X, tile, a.codes_out, a.s_out);
+}
+
+// ---- the per-window 8-bit state (LeapQuant: quantise once per window, buffered updates) ------
+// Per tile, with the window's running log2 gate product l_s and gamma_s = 2^l_s, the state after
+// token s of the window is S_s = gamma_s S_hat + sum_{r<=s} (gamma_s / gamma_r) k_r u_r^T, so
+// token t needs only the fixed INT8 state and the buffered k_r, u_r (r < t):
+//   p_t = S_{t-1}^T k_t = gamma_{t-1} S_hat^T k_t + sum_{r<t} (gamma_{t-1}/gamma_r) (k_r.k_t) u_r
+//   u_t = beta_t (v_t - g_t p_t)
+//   o_t = S_t^T q_t = gamma_t S_hat^T q_t + sum_{r<t} (gamma_t/gamma_r) (k_r.q_t) u_r + (k_t.q_t) u_t.
+// The window's last token forms S_W in registers and requantises it (rowwise absmax INT8).
+constexpr int kLeapMaxWindow = 256;
+constexpr int kLeapBatch = 16;   // buffered tokens staged per pass of the window-end update
+
+struct LeapArgs {
+    int H, window, t, num_tiles;
+    const uint16_t* q;
+    const uint16_t* k;
+    const uint16_t* v;
+    const float* beta;
+    const float* gate;
+    int8_t* codes;
+    uint16_t* s;
+    uint16_t* kbuf;
+    float* ubuf;
+    float* lbuf;
+    float* o;
+};
+
+template <int D>
+struct LeapSmem {
+    using M = Map<D>;
+    alignas(16) float2 rowc[D];                    // s_i k_i, s_i q_i
+    alignas(16) float red[M::kWarps][2][D];
+    alignas(16) float dots[2][kLeapMaxWindow];     // (gamma_{t-1}/gamma_r) k_r.k_t, (gamma_t/gamma_r) k_r.q_t
+    alignas(16) float colu[D];                     // u_t
+    alignas(16) float rowbuf[M::kWarps][32 * (M::RPT + 1)];
+    alignas(16) float rows[D];
+    alignas(16) float kb[kLeapBatch][D];           // window end: buffered keys
+    alignas(16) float ub[kLeapBatch][D];           // window end: (gamma_W/gamma_r) u_r
+    float qk, lprev, lt;
+};
+
+template <int D>
+__global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) leap_step_kernel(const LeapArgs a) {
+    using M = Map<D>;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    LeapSmem<D>& sm = *reinterpret_cast<LeapSmem<D>*>(smem_raw);
+    const int tile = blockIdx.x, t = a.t;
+    const int64_t T = a.num_tiles;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cl = M::col_lane(lane);
+    const int8_t* Cd = a.codes + static_cast<int64_t>(tile) * D * D;
+    float Z[M::RPT][4];
+#pragma unroll
+    for (int r = 0; r < M::RPT; ++r) {
+        const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(Cd + M::row(warp, lane, r) * D + 4 * cl)) ^ 0x80808080u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) Z[r][c] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650 | c)) - (kTwo23 + 128.0f);
+    }
+    const uint16_t* kt_g = a.k + static_cast<int64_t>(tile) * D;
+    const uint16_t* qt_g = a.q + static_cast<int64_t>(tile) * D;
+    if (tid < D) {
+        const float si = half_bits_to_float(a.s[static_cast<int64_t>(tile) * D + tid]);
+        const uint16_t kb = kt_g[tid];
+        sm.rowc[tid] = make_float2(si * bf16_bits_to_float(kb), si * bf16_bits_to_float(qt_g[tid]));
+        a.kbuf[(static_cast<int64_t>(t) * T + tile) * D + tid] = kb;   // this token joins the window's buffer
+    }
+    if (tid == 0) {
+        const float lp = t > 0 ? a.lbuf[static_cast<int64_t>(t - 1) * T + tile] : 0.0f;
+        const float lt = lp + log2f(fmaxf(__ldg(a.gate + tile), 0x1p-64f));   // a zero gate counts 2^-64
+        sm.lprev = lp;
+        sm.lt = lt;
+        a.lbuf[static_cast<int64_t>(t) * T + tile] = lt;
+    }
+    __syncthreads();
+    // k_t and q_t of this lane's D/32 key rows, for the dot products with the buffered keys.
+    constexpr int RL = D / 32;
+    float kl[RL], ql[RL];
+#pragma unroll
+    for (int e = 0; e < RL; ++e) {
+        kl[e] = bf16_bits_to_float(kt_g[lane * RL + e]);
+        ql[e] = bf16_bits_to_float(qt_g[lane * RL + e]);
+    }
+    if (warp == 0) {
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < RL; ++e) acc = fmaf(kl[e], ql[e], acc);
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+        if (lane == 0) sm.qk = acc;
+    }
+    for (int r = warp; r < t; r += M::kWarps) {   // one buffered token per warp
+        const uint16_t* kr = a.kbuf + (static_cast<int64_t>(r) * T + tile) * D + lane * RL;
+        float ck = 0.f, cq = 0.f;
+#pragma unroll
+        for (int e = 0; e < RL; ++e) {
+            const float x = bf16_bits_to_float(kr[e]);
+            ck = fmaf(x, kl[e], ck);
+            cq = fmaf(x, ql[e], cq);
+        }
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) {
+            ck += __shfl_xor_sync(0xffffffffu, ck, m);
+            cq += __shfl_xor_sync(0xffffffffu, cq, m);
+        }
+        if (lane == 0) {
+            const float lr = a.lbuf[static_cast<int64_t>(r) * T + tile];
+            sm.dots[0][r] = ck * exp2f(sm.lprev - lr);
+            sm.dots[1][r] = cq * exp2f(sm.lt - lr);
+        }
+    }
+    // S_hat^T k_t and S_hat^T q_t, column partial sums.
+    {
+        float pacc[4] = {0.f, 0.f, 0.f, 0.f}, oacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < M::RPT; ++r) {
+            const float2 rc = sm.rowc[M::row(warp, lane, r)];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                pacc[c] = fmaf(rc.x, Z[r][c], pacc[c]);
+                oacc[c] = fmaf(rc.y, Z[r][c], oacc[c]);
+            }
+        }
+        combine_subrows<Map<D>, float>(pacc, OpAdd());
+        combine_subrows<Map<D>, float>(oacc, OpAdd());
+        if (lane < M::LPR) {
+            *reinterpret_cast<float4*>(&sm.red[warp][0][4 * cl]) = make_float4(pacc[0], pacc[1], pacc[2], pacc[3]);
+            *reinterpret_cast<float4*>(&sm.red[warp][1][4 * cl]) = make_float4(oacc[0], oacc[1], oacc[2], oacc[3]);
+        }
+    }
+    __syncthreads();
+    if (tid < D) {   // column j: u_t and o_t
+        const int j = tid;
+        float a0 = 0.f, b0 = 0.f;
+#pragma unroll
+        for (int w = 0; w < M::kWarps; ++w) {
+            a0 += sm.red[w][0][j];
+            b0 += sm.red[w][1][j];
+        }
+        float bp = 0.f, bo = 0.f;
+        const float* ur = a.ubuf + static_cast<int64_t>(tile) * D + j;
+#pragma unroll 4
+        for (int r = 0; r < t; ++r) {
+            const float u = ur[static_cast<int64_t>(r) * T * D];
+            bp = fmaf(sm.dots[0][r], u, bp);
+            bo = fmaf(sm.dots[1][r], u, bo);
+        }
+        const float p = fmaf(exp2f(sm.lprev), a0, bp);
+        const float g = __ldg(a.gate + tile);
+        const float u = __ldg(a.beta + tile) * (bf16_bits_to_float(a.v[static_cast<int64_t>(tile) * D + j]) - g * p);
+        a.o[static_cast<int64_t>(tile) * D + j] = fmaf(sm.qk, u, fmaf(exp2f(sm.lt), b0, bo));
+        a.ubuf[(static_cast<int64_t>(t) * T + tile) * D + j] = u;
+        sm.colu[j] = u;
+    }
+    if (t + 1 < a.window) return;
+
+    // ---- the window's last token: S_W = gamma_W S_hat + sum_r (gamma_W/gamma_r) k_r u_r^T ----
+    __syncthreads();
+    {
+        const float gw = exp2f(sm.lt);
+#pragma unroll
+        for (int r = 0; r < M::RPT; ++r) {
+            const float f = gw * half_bits_to_float(a.s[static_cast<int64_t>(tile) * D + M::row(warp, lane, r)]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) Z[r][c] *= f;
+        }
+    }
+    for (int r0 = 0; r0 <= t; r0 += kLeapBatch) {
+        const int nb = min(kLeapBatch, t + 1 - r0);
+        __syncthreads();   // the previous batch has been used
+        for (int e = tid; e < nb * D; e += M::kThreads) {
+            const int rb = e / D, i = e % D, r = r0 + rb;
+            sm.kb[rb][i] = bf16_bits_to_float(r == t ? kt_g[i] : a.kbuf[(static_cast<int64_t>(r) * T + tile) * D + i]);
+            const float u = r == t ? sm.colu[i] : a.ubuf[(static_cast<int64_t>(r) * T + tile) * D + i];
+            const float lr = r == t ? sm.lt : a.lbuf[static_cast<int64_t>(r) * T + tile];
+            sm.ub[rb][i] = u * exp2f(sm.lt - lr);
+        }
+        __syncthreads();
+        for (int rb = 0; rb < nb; ++rb) {
+            const float4 u4 = *reinterpret_cast<const float4*>(&sm.ub[rb][4 * cl]);
+#pragma unroll
+            for (int r = 0; r < M::RPT; ++r) {
+                const float kk = sm.kb[rb][M::row(warp, lane, r)];
+                Z[r][0] = fmaf(kk, u4.x, Z[r][0]);
+                Z[r][1] = fmaf(kk, u4.y, Z[r][1]);
+                Z[r][2] = fmaf(kk, u4.z, Z[r][2]);
+                Z[r][3] = fmaf(kk, u4.w, Z[r][3]);
+            }
+        }
+    }
+    __syncthreads();   // every thread has read its codes and the scales before they are rewritten
+    int8_requantise<D>(sm, Z, tile, a.codes, a.s);
 }
 
 template <int D>
@@ -286,4 +478,31 @@ extern "C" int stepq_decode_step_int8(stepq_dims dims, const uint16_t* q, const 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return dims.dk == 128 ? launch_baseline<128>("stepq_decode_step_int8", decode_int8_kernel<128>, (int)tiles, a, st)
                           : launch_baseline<64>("stepq_decode_step_int8", decode_int8_kernel<64>, (int)tiles, a, st);
+}
+
+extern "C" int stepq_leap_step(stepq_dims dims, int window, int t, const uint16_t* q, const uint16_t* k,
+                               const uint16_t* v, const float* beta, const float* gate, int8_t* codes, uint16_t* s,
+                               uint16_t* kbuf, float* ubuf, float* lbuf, float* o, void* stream) {
+    const char* fn = "stepq_leap_step";
+    clear_error();
+    long long tiles;
+    int rc = tiles_of(dims, fn, tiles);
+    if (rc) return rc;
+    if (dims.gate_per_channel)
+        return set_error(STEPQ_EUNSUPPORTED, "%s: channel gates are not supported by the per-window form", fn);
+    if (window < 1 || window > kLeapMaxWindow || t < 0 || t >= window)
+        return set_error(STEPQ_EINVAL, "%s: window=%d t=%d (need 0 <= t < window <= %d)", fn, window, t, kLeapMaxWindow);
+    if (tiles == 0) return STEPQ_OK;
+    rc = check_ptrs(fn, {{"q", q}, {"k", k}, {"v", v}, {"beta", beta}, {"gate", gate}, {"codes", codes}, {"s", s},
+                         {"kbuf", kbuf}, {"ubuf", ubuf}, {"lbuf", lbuf}, {"o", o}});
+    if (rc) return rc;
+    LeapArgs a{dims.H, window, t, static_cast<int>(tiles), q, k, v, beta, gate, codes, s, kbuf, ubuf, lbuf, o};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    auto go = [&](auto kern, size_t smem) -> int {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "%s: %s", fn, cudaGetErrorString(e));
+        kern<<<static_cast<int>(tiles), dims.dk == 128 ? Map<128>::kThreads : Map<64>::kThreads, smem, st>>>(a);
+        return check_launch(fn);
+    };
+    return dims.dk == 128 ? go(leap_step_kernel<128>, sizeof(LeapSmem<128>)) : go(leap_step_kernel<64>, sizeof(LeapSmem<64>));
 }

@@ -75,6 +75,35 @@ class QuantizedState:
         return self.packed.numel() + 2 * (self.r.numel() + self.c.numel())
 
 
+class WindowState:
+    """States of B sequences x H heads on the per-window 8-bit format (LeapQuant's per-window
+    quantisation): rowwise-absmax INT8 between windows, the open window's buffered updates in
+    fp32. step() decodes one token; every `window` tokens the state is requantised once."""
+
+    def __init__(self, codes: torch.Tensor, s: torch.Tensor, window: int):
+        B, H, d, _ = codes.shape
+        self.codes, self.s, self.window, self.t = codes, s, int(window), 0
+        dev = codes.device
+        self.kbuf = torch.empty((window, B, H, d), dtype=torch.bfloat16, device=dev)
+        self.ubuf = torch.empty((window, B, H, d), dtype=torch.float32, device=dev)
+        self.lbuf = torch.empty((window, B, H), dtype=torch.float32, device=dev)
+
+    @classmethod
+    def from_fp32(cls, S: torch.Tensor, window: int) -> "WindowState":
+        codes, s = api.stepq_int8_quantize_state(S)
+        return cls(codes, s, window)
+
+    def step(self, q, k, v, beta, gate, o=None) -> torch.Tensor:
+        """One decode token for every sequence; returns o [B,H,d]."""
+        o = api.stepq_leap_step(self.window, self.t, q, k, v, beta, gate, self.codes, self.s, self.kbuf, self.ubuf,
+                                self.lbuf, o)
+        self.t = (self.t + 1) % self.window
+        return o
+
+    def nbytes(self) -> int:
+        return self.codes.numel() + 2 * self.s.numel()
+
+
 def lifetime(unit_gates) -> np.ndarray:
     """L_u = 1/(1 - g_u): the sum over j >= 0 of g_u^j, the retention of a unit's error (§3.2)."""
     g = np.asarray(unit_gates, dtype=np.float64)

@@ -164,3 +164,18 @@ def test_tensor_core_prefill_refuses_shapes_it_does_not_cover():
     assert lib.stepq_prefill_chunk_wy(_dims(B=0), 64, *args) == _lib.STEPQ_OK
     rc = lib.stepq_prefill_chunk_wy(_dims(), 64, *([P()] * 8), 4097, *([P()] * 7), None)
     assert rc == _lib.STEPQ_EINVAL
+
+
+def test_per_window_step_validates_before_touching_cuda():
+    """stepq_leap_step: scalar gates only; 0 <= t < window <= 256; pointers checked; an empty
+    batch is a no-op."""
+    lib = _lib.lib()
+    P = _fake
+    args = (*([P()] * 5), P(), P(), P(), P(), P(), P(), None)
+    rc = lib.stepq_leap_step(_dims(gpc=1), 16, 0, *args)
+    assert rc == _lib.STEPQ_EUNSUPPORTED and b"channel gates" in lib.stepq_last_error()
+    for window, t in ((0, 0), (257, 0), (16, 16), (16, -1)):
+        assert lib.stepq_leap_step(_dims(), window, t, *args) == _lib.STEPQ_EINVAL
+    assert lib.stepq_leap_step(_dims(B=0), 16, 3, *args) == _lib.STEPQ_OK
+    rc = lib.stepq_leap_step(_dims(), 16, 3, *([P()] * 5), P(), P(), ctypes.c_void_p(0), P(), P(), P(), None)
+    assert rc == _lib.STEPQ_EINVAL and b"kbuf is NULL" in lib.stepq_last_error()
