@@ -201,9 +201,10 @@ STEPQ_API int stepq_decode_step_int8(stepq_dims dims, const uint16_t* q, const u
                            const uint16_t* s_in, int8_t* codes_out, uint16_t* s_out, float* o,
                            void* stream);
 
-/* One token of the per-window 8-bit state (LeapQuant, "Compensator Tokens and per-window
-   quantization": quantise the state once at the end of a window of tokens; inside the window the
-   readouts come from the fixed low-bit state plus high-precision buffered updates). The state
+/* One token of the per-window 8-bit state (LeapQuant's abstract on the page "When Dynamic Scaling
+   Fails: A Scale-State Feedback Governs Recurrent-State Quantization in Linear-Attention and SSM
+   LLMs": quantise the state once at the end of a window of tokens; inside the window the readouts
+   come from the fixed low-bit state plus high-precision buffered updates). The state
    between windows is the rowwise-absmax INT8 format above (codes, s). Token t of the window
    (0 <= t < window <= STEPQ_LEAP_MAX_WINDOW) reads codes and s and the window's buffers entries
    0 .. t-1, and writes entry t:

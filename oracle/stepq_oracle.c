@@ -628,9 +628,10 @@ int orc_prefill_chunk(int C, int B, int H, int dk, int dv, int gate_per_channel,
     return ORC_OK;
 }
 
-/* Per-window 8-bit state (LeapQuant, "Compensator Tokens and per-window quantization", abstract:
-   the state is quantised once at the end of a window of tokens; inside the window, readouts come
-   from the fixed low-bit state together with high-precision buffered updates). Reading: the
+/* Per-window 8-bit state (LeapQuant, as its abstract on the page "When Dynamic Scaling Fails: A
+   Scale-State Feedback Governs Recurrent-State Quantization in Linear-Attention and SSM LLMs"
+   describes it: the state is quantised once at the end of a window of tokens; inside the window,
+   readouts come from the fixed low-bit state together with high-precision buffered updates). Reading: the
    state between windows is the rowwise-absmax INT8 format of §5.1 (orc_int8_quantise_tile); a
    window of W tokens applies the gated Delta rule exactly (float64) to the reconstructed state
    S_hat = diag(s) codes, every token's readout taken from that running state (which is what the

@@ -1,6 +1,7 @@
-"""Pins of the oracle's per-window 8-bit state (LeapQuant, "Compensator Tokens and per-window
-quantization", abstract: quantise the state once at the end of a window; inside it, readouts
-come from the fixed low-bit state plus the window's high-precision updates). A one-token window
+"""Pins of the oracle's per-window 8-bit state (LeapQuant's abstract on the page "When Dynamic
+Scaling Fails: A Scale-State Feedback Governs Recurrent-State Quantization in Linear-Attention
+and SSM LLMs": quantise the state once at the end of a window; inside it, readouts come from
+the fixed low-bit state plus the window's high-precision updates). A one-token window
 is the per-step INT8 decode of §5.1; inside a window the readouts follow the affine form
 S_t = A_t S_{t-1} + B_t of §2.1 started from the reconstructed state; the window's end state is
 the textbook rowwise-absmax INT8 quantisation of that recurrence's final state."""
