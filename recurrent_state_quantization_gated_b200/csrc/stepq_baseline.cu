@@ -222,6 +222,7 @@ __global__ void __launch_bounds__(Map<D>::kThreads) int8_quantize_kernel(const B
 // The window's last token forms S_W in registers and requantises it (rowwise absmax INT8).
 constexpr int kLeapMaxWindow = 256;
 constexpr int kLeapBatch = 16;   // buffered tokens staged per pass of the window-end update
+constexpr int kLeapStage = 64;   // buffered tokens staged in shared memory per pass of a token
 
 struct LeapArgs {
     int H, window, t, num_tiles;
@@ -249,6 +250,8 @@ struct LeapSmem {
     alignas(16) float rows[D];
     alignas(16) float kb[kLeapBatch][D];           // window end: buffered keys
     alignas(16) float ub[kLeapBatch][D];           // window end: (gamma_W/gamma_r) u_r
+    alignas(16) float us[kLeapStage][D];           // buffered u_r, staged for the column sums
+    alignas(16) uint16_t ks[kLeapStage][D];        // buffered k_r, staged for the dot products
     float qk, lprev, lt;
 };
 
@@ -301,25 +304,36 @@ __global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) leap_ste
         for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
         if (lane == 0) sm.qk = acc;
     }
-    for (int r = warp; r < t; r += M::kWarps) {   // one buffered token per warp
-        const uint16_t* kr = a.kbuf + (static_cast<int64_t>(r) * T + tile) * D + lane * RL;
-        float ck = 0.f, cq = 0.f;
+    // The buffered tokens' dot products with k_t and q_t, kLeapStage tokens at a time: the keys
+    // are staged with independent 16-byte loads, then one warp per buffered token.
+    for (int r0 = 0; r0 < t; r0 += kLeapStage) {
+        const int nb = min(kLeapStage, t - r0);
+        for (int e = tid; e < nb * (D / 8); e += M::kThreads) {
+            const int rb = e / (D / 8), c8 = e % (D / 8);
+            *reinterpret_cast<uint4*>(&sm.ks[rb][8 * c8]) = __ldg(reinterpret_cast<const uint4*>(
+                a.kbuf + (static_cast<int64_t>(r0 + rb) * T + tile) * D + 8 * c8));
+        }
+        __syncthreads();
+        for (int rb = warp; rb < nb; rb += M::kWarps) {
+            float ck = 0.f, cq = 0.f;
 #pragma unroll
-        for (int e = 0; e < RL; ++e) {
-            const float x = bf16_bits_to_float(kr[e]);
-            ck = fmaf(x, kl[e], ck);
-            cq = fmaf(x, ql[e], cq);
-        }
+            for (int e = 0; e < RL; ++e) {
+                const float x = bf16_bits_to_float(sm.ks[rb][lane * RL + e]);
+                ck = fmaf(x, kl[e], ck);
+                cq = fmaf(x, ql[e], cq);
+            }
 #pragma unroll
-        for (int m = 16; m > 0; m >>= 1) {
-            ck += __shfl_xor_sync(0xffffffffu, ck, m);
-            cq += __shfl_xor_sync(0xffffffffu, cq, m);
+            for (int m = 16; m > 0; m >>= 1) {
+                ck += __shfl_xor_sync(0xffffffffu, ck, m);
+                cq += __shfl_xor_sync(0xffffffffu, cq, m);
+            }
+            if (lane == 0) {
+                const float lr = a.lbuf[static_cast<int64_t>(r0 + rb) * T + tile];
+                sm.dots[0][r0 + rb] = ck * exp2f(sm.lprev - lr);
+                sm.dots[1][r0 + rb] = cq * exp2f(sm.lt - lr);
+            }
         }
-        if (lane == 0) {
-            const float lr = a.lbuf[static_cast<int64_t>(r) * T + tile];
-            sm.dots[0][r] = ck * exp2f(sm.lprev - lr);
-            sm.dots[1][r] = cq * exp2f(sm.lt - lr);
-        }
+        __syncthreads();
     }
     // S_hat^T k_t and S_hat^T q_t, column partial sums.
     {
@@ -341,6 +355,27 @@ __global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) leap_ste
         }
     }
     __syncthreads();
+    // The buffered u_r weighted by those dot products, kLeapStage tokens at a time (staged with
+    // independent 16-byte loads); threads j < D own column j.
+    float bp = 0.f, bo = 0.f;
+    for (int r0 = 0; r0 < t; r0 += kLeapStage) {
+        const int nb = min(kLeapStage, t - r0);
+        if (r0 > 0) __syncthreads();   // the previous stage has been read
+        for (int e = tid; e < nb * (D / 4); e += M::kThreads) {
+            const int rb = e / (D / 4), c4 = e % (D / 4);
+            *reinterpret_cast<float4*>(&sm.us[rb][4 * c4]) = __ldg(reinterpret_cast<const float4*>(
+                a.ubuf + (static_cast<int64_t>(r0 + rb) * T + tile) * D + 4 * c4));
+        }
+        __syncthreads();
+        if (tid < D) {
+#pragma unroll 4
+            for (int rb = 0; rb < nb; ++rb) {
+                const float u = sm.us[rb][tid];
+                bp = fmaf(sm.dots[0][r0 + rb], u, bp);
+                bo = fmaf(sm.dots[1][r0 + rb], u, bo);
+            }
+        }
+    }
     if (tid < D) {   // column j: u_t and o_t
         const int j = tid;
         float a0 = 0.f, b0 = 0.f;
@@ -348,14 +383,6 @@ __global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) leap_ste
         for (int w = 0; w < M::kWarps; ++w) {
             a0 += sm.red[w][0][j];
             b0 += sm.red[w][1][j];
-        }
-        float bp = 0.f, bo = 0.f;
-        const float* ur = a.ubuf + static_cast<int64_t>(tile) * D + j;
-#pragma unroll 4
-        for (int r = 0; r < t; ++r) {
-            const float u = ur[static_cast<int64_t>(r) * T * D];
-            bp = fmaf(sm.dots[0][r], u, bp);
-            bo = fmaf(sm.dots[1][r], u, bo);
         }
         const float p = fmaf(exp2f(sm.lprev), a0, bp);
         const float g = __ldg(a.gate + tile);
