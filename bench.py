@@ -420,7 +420,7 @@ def main():
         elif args.kernel == "quant":
             api.stepq_decode_step(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
                                   layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
-                                  st["packed"], st["r"], st["c"], o, pivots=layout.pivots)
+                                  st["packed"], st["r"], st["c"], o, pivots=layout.pivots, mixed=layout.mixed)
         elif args.kernel == "fp32":
             api.stepq_decode_step_fp32(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], st["S"], st["S"], o)
         elif args.kernel == "leap":

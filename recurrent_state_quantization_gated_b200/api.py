@@ -44,14 +44,22 @@ def _ptr(t: torch.Tensor, dtype: torch.dtype, name: str):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _dims(B, H, d, gate_per_channel=0, pivots=0):
-    return Dims(int(B), int(H), int(d), int(d), int(gate_per_channel), int(pivots))
+def _dims(B, H, d, gate_per_channel=0, pivots=0, mixed=0):
+    return Dims(int(B), int(H), int(d), int(d), int(gate_per_channel), int(pivots), int(mixed))
 
 
 def _has_pivots(bits, pivots):
     """The pivots flag of a decode call: as given, else read from the bit map (a device
     reduction and a host read; pass it to avoid both)."""
     return int(bool((bits == 16).any().item())) if pivots is None else int(bool(pivots))
+
+
+def _has_mixed(bits, mixed):
+    """The mixed flag of a decode call (some head's key rows have different widths): as given,
+    else read from the bit map (a device reduction and a host read; pass it to avoid both)."""
+    if mixed is not None:
+        return int(bool(mixed))
+    return int(bool((bits != bits[:, :1]).any().item()))
 
 
 def stepq_build_info() -> str:
@@ -98,16 +106,18 @@ def stepq_unpack_state(packed, bits, head_off, bytes_per_seq, r, c, S_out=None):
 
 
 def stepq_decode_step(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
-                      packed_out=None, r_out=None, c_out=None, o=None, pivots=None):
+                      packed_out=None, r_out=None, c_out=None, o=None, pivots=None, mixed=None):
     """One fused quantized decode step; outputs may alias the inputs (in-place update).
-    Returns (packed_out, r_out, c_out, o)."""
+    pivots / mixed: the bit map's FP16 pivot rows / rows of different widths within a head
+    (None: read from the bit map). Returns (packed_out, r_out, c_out, o)."""
     B, H, d = q.shape
     gpc = 1 if gate.dim() == 3 else 0
     packed_out = torch.empty_like(packed_in) if packed_out is None else packed_out
     r_out = torch.empty_like(r_in) if r_out is None else r_out
     c_out = torch.empty_like(c_in) if c_out is None else c_out
     o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
-    call("stepq_decode_step", _dims(B, H, d, gpc, _has_pivots(bits, pivots)), _ptr(q, torch.bfloat16, "q"),
+    call("stepq_decode_step", _dims(B, H, d, gpc, _has_pivots(bits, pivots), _has_mixed(bits, mixed)),
+         _ptr(q, torch.bfloat16, "q"),
          _ptr(k, torch.bfloat16, "k"),
          _ptr(v, torch.bfloat16, "v"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
          _ptr(bits, torch.uint8, "bits"), _ptr(w, torch.float32, "w"), _ptr(head_off, torch.int64, "head_off"),

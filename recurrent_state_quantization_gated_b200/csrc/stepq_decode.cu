@@ -308,7 +308,7 @@ __device__ __forceinline__ void token_constants(DecodeSmem<D>& sm, int he, int i
 // The tile loop of the decode kernel. kPiv: the bit map may hold FP16 pivot rows (declared by
 // the caller in stepq_dims.pivots); launches without them run the leaner instantiation. A
 // width-16 row met in a launch declared without pivots raises bit 1 of the device error word.
-template <int D, bool kSplit, bool kPiv, bool kChunk>
+template <int D, bool kSplit, bool kPiv, bool kChunk, bool kMixed>
 __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm) {
     using M = DMap<D>;
     constexpr int RPT = M::RPT;
@@ -399,7 +399,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
         {
             const int w0 = (meta[warp * M::kRowsPerWarp] >> 8) & 0xFF;
             const int w1 = (meta[warp * M::kRowsPerWarp + M::kRowsPerWarp - 1] >> 8) & 0xFF;
-            ww = (w0 == w1) ? w0 : 0;
+            ww = (!kMixed && w0 == w1) ? w0 : 0;   // kMixed: one code path for every width
         }
 
         // ---- phase 1: unpack, k^T D S and q^T D S (column scale factored out) ----------
@@ -532,7 +532,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
 // kSplit: the first kernel of the split form. It reconstructs, updates and reads out like the
 // fused step, then writes the updated state X in fp32 and stops; the refit and the pack run
 // as separate kernels (stepq_decode_step_split).
-template <int D, bool kSplit, bool kPiv, bool kChunk = false>
+template <int D, bool kSplit, bool kPiv, bool kChunk = false, bool kMixed = false>
 __global__ void __launch_bounds__(DMap<D>::kThreads, DMap<D>::kMinBlocks)
 decode_kernel(const DecodeArgs a) {
     using M = DMap<D>;
@@ -581,10 +581,10 @@ decode_kernel(const DecodeArgs a) {
     }
     __syncthreads();
 
-    run_tiles<D, kSplit, kPiv, kChunk>(a, sm);
+    run_tiles<D, kSplit, kPiv, kChunk, kMixed>(a, sm);
 }
 
-template <int D, bool kSplit, bool kPiv, bool kChunk = false>
+template <int D, bool kSplit, bool kPiv, bool kChunk = false, bool kMixed = false>
 static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     static int ctas_per_sm = -1, num_sms = 0;
     const size_t smem = sizeof(DecodeSmem<D>);
@@ -592,17 +592,17 @@ static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, kSplit, kPiv, kChunk>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, kSplit, kPiv, kChunk, kMixed>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "stepq_decode_step: %s", cudaGetErrorString(e));
         int occ = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D, kSplit, kPiv, kChunk>, DMap<D>::kThreads, smem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D, kSplit, kPiv, kChunk, kMixed>, DMap<D>::kThreads, smem);
         ctas_per_sm = occ > 0 ? occ : 1;
     }
     if (a.num_tiles == 0) return STEPQ_OK;
     int grid = num_sms * ctas_per_sm;
     if (grid > a.num_tiles) grid = a.num_tiles;
-    decode_kernel<D, kSplit, kPiv, kChunk><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
+    decode_kernel<D, kSplit, kPiv, kChunk, kMixed><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
     return check_launch("stepq_decode_step");
 }
 
@@ -665,6 +665,13 @@ extern "C" int stepq_decode_step(stepq_dims dims, const uint16_t* q, const uint1
     DecodeArgs a{dims.B, dims.H, dims.gate_per_channel, static_cast<int>(tiles), q, k, v, beta, gate, bits, w,
                  head_off, bytes_per_seq, packed_in, r_in, c_in, packed_out, r_out, c_out, o, nullptr, 1};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dims.mixed) {   // heads whose key rows have different widths: one code path for every width
+        if (dims.pivots)
+            return dims.dk == 128 ? launch_decode<128, false, true, false, true>(a, st)
+                                  : launch_decode<64, false, true, false, true>(a, st);
+        return dims.dk == 128 ? launch_decode<128, false, false, false, true>(a, st)
+                              : launch_decode<64, false, false, false, true>(a, st);
+    }
     if (dims.pivots) return dims.dk == 128 ? launch_decode<128, false, true>(a, st) : launch_decode<64, false, true>(a, st);
     return dims.dk == 128 ? launch_decode<128, false, false>(a, st) : launch_decode<64, false, false>(a, st);
 }
@@ -746,7 +753,7 @@ extern "C" int stepq_decode_step_split(stepq_dims dims, const uint16_t* q, const
     cudaError_t e = cudaEventRecord(ev, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev, 0);
     if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "%s: %s", fn, cudaGetErrorString(e));
-    stepq_dims fd{dims.B, dims.H, dims.dk, dims.dv, 0, dims.pivots};
+    stepq_dims fd{dims.B, dims.H, dims.dk, dims.dv, 0, dims.pivots, 0};
     rc = stepq_fit_scales(fd, x_ws, w, bits, r_out, c_out, side_stream);
     if (rc) return rc;
     return stepq_pack_state(fd, x_ws, bits, head_off, bytes_per_seq, r_out, c_out, packed_out, side_stream);

@@ -41,6 +41,11 @@ class Layout:
         """1 when the bit map holds FP16 pivot rows (width 16)."""
         return int((self.bits == 16).any())
 
+    @property
+    def mixed(self) -> int:
+        """1 when some head's key rows have different widths (a row-level allocation)."""
+        return int((self.bits != self.bits[:, :1]).any())
+
 
 class QuantizedState:
     """Packed states of B sequences x H heads (one layer)."""
@@ -68,7 +73,7 @@ class QuantizedState:
         L = self.layout
         _, _, _, o = api.stepq_decode_step(q, k, v, beta, gate, L.bits_dev, self.w, L.head_off_dev,
                                            L.bytes_per_seq, self.packed, self.r, self.c,
-                                           self.packed, self.r, self.c, o, pivots=L.pivots)
+                                           self.packed, self.r, self.c, o, pivots=L.pivots, mixed=L.mixed)
         return o
 
     def nbytes(self) -> int:

@@ -159,3 +159,30 @@ def test_undeclared_pivot_rows_raise_the_device_flag():
                           st["packed"], st["r"], st["c"], pivots=1)
     torch.cuda.synchronize()
     assert api.stepq_read_device_flags() == 0
+
+
+@pytest.mark.parametrize("pivots", [0, 6])
+def test_mixed_and_width_specialised_paths_agree(pivots):
+    """The decode step's two code organisations (stepq_dims.mixed: one path for every row width,
+    or width-specialised paths per warp) give the same bits on the same inputs; half the heads
+    here have one width per head, half mix widths across rows."""
+    import torch
+    from recurrent_state_quantization_gated_b200 import api
+    d, B, H = 128, 3, 6
+    wl = synth.workload(1, B=B, H=H, d=d, seed=17)
+    S0 = synth.initial_state(wl)
+    bits = synth.random_bits(H, d, choices=(2, 4, 6, 8), seed=5)
+    bits[: H // 2] = bits[: H // 2, :1]                      # heads 0-2: one width each
+    bits = with_pivots(bits, pivots, 7)
+    w = synth.random_weights(H, d, seed=6)
+    r, c = oracle.fit_scales(S0, w, bits)
+    packed = oracle.pack_state(S0, bits, r, c)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    td = tokens_dev(synth.tokens(wl, 2))
+    args = (td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w), dev(head_off), bps,
+            dev(packed), dev(r, torch.float16), dev(c, torch.float16))
+    a = api.stepq_decode_step(*args, mixed=0)
+    b = api.stepq_decode_step(*args, mixed=1)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
