@@ -415,7 +415,7 @@ def main():
         elif args.kernel == "prefill":
             api.stepq_prefill_chunk(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
                                     layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
-                                    st["packed"], st["r"], st["c"], o, pivots=layout.pivots,
+                                    st["packed"], st["r"], st["c"], o, pivots=layout.pivots, mixed=layout.mixed,
                                     form=None if args.prefill_form == "auto" else args.prefill_form)
         elif args.kernel == "quant":
             api.stepq_decode_step(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,

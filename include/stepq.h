@@ -75,8 +75,8 @@ typedef struct {
                                 pivot row met with pivots = 0 raises bit 1 of the device error
                                 word and its results are undefined. Other calls ignore it.  */
     int mixed;               /* 1: some head's key rows have different widths (a row-level bit
-                                allocation). Read by stepq_decode_step, which then runs one code
-                                path for every row width instead of width-specialised paths per
+                                allocation). Read by stepq_decode_step and the sequential prefill
+                                chunk, which then run one code path for every row width instead of width-specialised paths per
                                 warp (smaller code: faster for such maps, slower for maps whose
                                 heads each use one width). Results are identical either way.  */
 } stepq_dims;

@@ -161,7 +161,7 @@ def stepq_decode_step_split(q, k, v, beta, gate, bits, w, head_off, bytes_per_se
 
 
 def stepq_prefill_chunk(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
-                        packed_out=None, r_out=None, c_out=None, o=None, pivots=None, form=None):
+                        packed_out=None, r_out=None, c_out=None, o=None, pivots=None, form=None, mixed=None):
     """A prefill chunk: q, k, v [C,B,H,d], beta [C,B,H], gate [C,B,H] or [C,B,H,d]; the state is
     reconstructed once, updated C times in fp32 and packed once. form: None (the library picks),
     "seq" (tokens one after another on the register tile) or "wy" (the chunked WY form on the
@@ -174,7 +174,7 @@ def stepq_prefill_chunk(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, p
     c_out = torch.empty_like(c_in) if c_out is None else c_out
     o = torch.empty((C, B, H, d), dtype=torch.float32, device=q.device) if o is None else o
     name = {None: "stepq_prefill_chunk", "seq": "stepq_prefill_chunk_seq", "wy": "stepq_prefill_chunk_wy"}[form]
-    call(name, _dims(B, H, d, gpc, _has_pivots(bits, pivots)), ctypes.c_int(int(C)),
+    call(name, _dims(B, H, d, gpc, _has_pivots(bits, pivots), _has_mixed(bits, mixed)), ctypes.c_int(int(C)),
          _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
          _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"), _ptr(bits, torch.uint8, "bits"),
          _ptr(w, torch.float32, "w"), _ptr(head_off, torch.int64, "head_off"), ctypes.c_int64(int(bytes_per_seq)),

@@ -698,6 +698,13 @@ extern "C" int stepq_prefill_chunk_seq(stepq_dims dims, int chunk, const uint16_
     DecodeArgs a{dims.B, dims.H, dims.gate_per_channel, static_cast<int>(tiles), q, k, v, beta, gate, bits, w,
                  head_off, bytes_per_seq, packed_in, r_in, c_in, packed_out, r_out, c_out, o, nullptr, chunk};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dims.mixed) {   // heads whose key rows have different widths: one code path for every width
+        if (dims.pivots)
+            return dims.dk == 128 ? launch_decode<128, false, true, true, true>(a, st)
+                                  : launch_decode<64, false, true, true, true>(a, st);
+        return dims.dk == 128 ? launch_decode<128, false, false, true, true>(a, st)
+                              : launch_decode<64, false, false, true, true>(a, st);
+    }
     if (dims.pivots)
         return dims.dk == 128 ? launch_decode<128, false, true, true>(a, st) : launch_decode<64, false, true, true>(a, st);
     return dims.dk == 128 ? launch_decode<128, false, false, true>(a, st) : launch_decode<64, false, false, true>(a, st);

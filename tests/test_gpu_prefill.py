@@ -165,3 +165,21 @@ def test_tensor_core_prefill_full_size_sampled():
     p_s = np.concatenate([packed[b * bps:(b + 1) * bps] for b in seqs])
     res = (np.concatenate([p_g[b * bps:(b + 1) * bps] for b in seqs]), r_g[seqs], c_g[seqs], o_g[:, seqs])
     _check_against_oracle(res, sub, bits, w, p_s, r[seqs], c[seqs], d, len(seqs), C)
+
+
+def test_sequential_prefill_code_paths_agree():
+    """The sequential prefill form's two code organisations (stepq_dims.mixed) give the same bits
+    on a map with channel gates, pivot rows and rows of mixed widths."""
+    import torch
+    from recurrent_state_quantization_gated_b200 import api
+    d, B, H, C = 128, 2, 5, 9
+    wl, bits, w, packed, r, c = _setup(d, B, H, (4, 6, 8), True, seed=61, pivots=7)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    td = _dev_tokens(_chunk(wl, C))
+    args = (td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w), dev(head_off), bps, dev(packed),
+            dev(r, torch.float16), dev(c, torch.float16))
+    a = api.stepq_prefill_chunk(*args, form="seq", mixed=0)
+    b = api.stepq_prefill_chunk(*args, form="seq", mixed=1)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
