@@ -500,41 +500,63 @@ def main():
     o_host = [torch.empty(tuple(outs[0].shape), dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = pinned[0].numel()
     d2h = o_host[0].numel() * o_host[0].element_size()
-    n_e2e = max(R * LW, (args.e2e_steps // (R * LW)) * R * LW)
-    # Three streams: inputs in, decode, readout out. Step s's copies overlap the decode of
-    # step s-1; buffers are reused R steps later, ordered by events.
+    # Three streams: inputs in, step, readout out; step s's copies overlap step s-1's work, and
+    # buffers are reused R steps later, ordered by events. n_g such steps (each: one H2D copy of
+    # the step's inputs, the library call, one D2H copy of its readout) are captured in a CUDA
+    # graph, replayed back to back, so that the host's per-call overhead does not pace the loop.
+    n_g = R * LW * max(1, -(-16 // (R * LW)))
+    reps_e2e = max(1, -(-args.e2e_steps // n_g))
+    n_e2e = reps_e2e * n_g
     cs, ds = torch.cuda.Stream(), torch.cuda.Stream()
-    ev_h = [torch.cuda.Event() for _ in range(R)]
-    ev_k = [torch.cuda.Event() for _ in range(R)]
-    ev_d = [torch.cuda.Event() for _ in range(R)]
+
+    def e2e_steps(n):
+        ev_h = [torch.cuda.Event() for _ in range(R)]
+        ev_k = [torch.cuda.Event() for _ in range(R)]
+        ev_d = [torch.cuda.Event() for _ in range(R)]
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        cs.wait_event(fork)
+        ds.wait_event(fork)
+        for s_ in range(n):
+            i = s_ % R
+            src = pinned[s_ % len(pinned)]
+            with torch.cuda.stream(cs):
+                if s_ >= R:
+                    cs.wait_event(ev_k[i])          # the step that last read toks[i] is done
+                dst = tok_bufs[i][reps[i]["win"].t] if args.kernel == "leap" else tok_bufs[i]
+                dst.copy_(src, non_blocking=True)   # q, k, v, beta, gate in one copy
+                ev_h[i].record(cs)
+            with torch.cuda.stream(stream):
+                stream.wait_event(ev_h[i])
+                if s_ >= R:
+                    stream.wait_event(ev_d[i])      # outs[i] has been read back
+                launch(i)
+                ev_k[i].record(stream)
+            with torch.cuda.stream(ds):
+                ds.wait_event(ev_k[i])
+                o_host[s_ % 2].copy_(outs[i], non_blocking=True)
+                ev_d[i].record(ds)
+        stream.wait_stream(cs)
+        stream.wait_stream(ds)
+
+    with torch.cuda.stream(stream):
+        e2e_steps(n_g)                              # once outside capture
+    stream.synchronize()
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e, stream=stream):
+        e2e_steps(n_g)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(cs)
-    for s_ in range(n_e2e):
-        i = s_ % R
-        src = pinned[s_ % len(pinned)]
-        with torch.cuda.stream(cs):
-            if s_ >= R:
-                cs.wait_event(ev_k[i])          # the decode that last read toks[i] is done
-            dst = tok_bufs[i][reps[i]["win"].t] if args.kernel == "leap" else tok_bufs[i]
-            dst.copy_(src, non_blocking=True)   # q, k, v, beta, gate in one copy
-            ev_h[i].record(cs)
-        with torch.cuda.stream(stream):
-            stream.wait_event(ev_h[i])
-            if s_ >= R:
-                stream.wait_event(ev_d[i])      # outs[i] has been read back
-            launch(i)
-            ev_k[i].record(stream)
-        with torch.cuda.stream(ds):
-            ds.wait_event(ev_k[i])
-            o_host[s_ % 2].copy_(outs[i], non_blocking=True)
-            ev_d[i].record(ds)
-    e1.record(ds)
-    ds.synchronize()
-    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps_e2e):
+            g_e2e.replay()
+        e1.record(stream)
+    stream.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
     e2e_value = job_throughput(world, upd, n_e2e, e2e_ms)
+    del g_e2e
 
     line = None
     if rank == 0:
@@ -561,7 +583,9 @@ def main():
             if (args.kernel == "quant" and args.workload == 1) else None,
             "gpu_launches": K,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": n_e2e},
+                    "steps": n_e2e,
+                    "method": f"CUDA graphs of {n_g} steps (each: one H2D copy of the step's inputs from pinned "
+                              f"host memory, the library call, one D2H copy of its readout), replayed back to back"},
             "device_flags": flags,
             "split": split_info,
             "clocks": clocks,
