@@ -91,6 +91,7 @@ struct Small {
     alignas(16) float beta[C];
     alignas(16) float l2g[C];        // log2 gamma_t (a zero gate counts as 2^-64)
     alignas(8) uint64_t bar_mma;
+    alignas(8) uint64_t bar_sc;      // the last round's boundary-state product, committed apart
     alignas(8) uint64_t bar_codes;
     uint32_t tmem;
 };
@@ -270,6 +271,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
 
     if (tid == 0) {
         mbar_init(&sm.bar_mma, 1);
+        mbar_init(&sm.bar_sc, 1);
         mbar_init(&sm.bar_codes, 1);
         fence_barrier_init();
     }
@@ -278,18 +280,19 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tm = sm.tmem;
-    uint32_t mma_phase = 0, codes_phase = 0;
+    uint32_t mma_phase = 0, sc_phase = 0, codes_phase = 0;
     bool codes_pending = false;
     const int64_t T = a.num_tiles;
 
     // Waits for the tensor core's last commit; false (uniformly over the CTA) if it never came.
-    auto wait_mma = [&]() -> bool {
-        const bool ok = mbar_wait_bounded(&sm.bar_mma, mma_phase, kWaitLimitNs, a.flags);
-        mma_phase ^= 1u;
+    auto wait_bar = [&](uint64_t* bar, uint32_t& phase) -> bool {
+        const bool ok = mbar_wait_bounded(bar, phase, kWaitLimitNs, a.flags);
+        phase ^= 1u;
         const bool all = !__syncthreads_or(!ok);
         umma::fence_after_sync();
         return all;
     };
+    auto wait_mma = [&]() -> bool { return wait_bar(&sm.bar_mma, mma_phase); };
     // Orders this thread's shared-memory writes and TMEM reads before an MMA that the
     // issuing thread starts after the barrier.
     auto to_tensor_core = [&]() {
@@ -629,6 +632,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                     umma::mma_bf16(tm + TM_S, umma::desc_kmajor(Pp[p] - 64 * C, ks, C), umma::desc_mnmajor(BUC[q], ks, D),
                                    id_o, 1u);
             }
+            umma::commit(&sm.bar_mma);   // the readouts can be written while S_C is computed
             // S_C - gamma_C S0 = K^T U~ into the W columns (W was consumed in C).
             const uint32_t id_s = umma::idesc_bf16(128, 128, true, true);
 #pragma unroll
@@ -637,7 +641,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                 for (int ks = 0; ks < C / 16; ++ks)
                     umma::mma_bf16(tm + TM_W, umma::desc_mnmajor(KQ, ks, D), umma::desc_mnmajor(BUT[p], ks, D), id_s,
                                    p > 0 || ks > 0);
-            umma::commit(&sm.bar_mma);
+            umma::commit(&sm.bar_sc);
         }
         if (!wait_mma()) break;
 
@@ -663,6 +667,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                 }
             }
             // X_ij = (K^T U~)_ij + gamma_C rho_i c_j Z_ij, TMEM lane i, columns j in [64 hf, 64 hf + 64).
+            if (!wait_bar(&sm.bar_sc, sc_phase)) break;
             const int i = 32 * (warp & 3) + lane;
             const float fi = ex2(sm.l2g[C - 1]) * sm.rho[i];
 #pragma unroll 1
