@@ -581,7 +581,7 @@ def main():
                          "bytes_per_launch_formula": "2*B*bytes_per_seq + B*H*(2*(2d+2d) + 6d + 4 + gate + 4d)"},
             "alu_roofline": alu_roofline(value * wl.d * wl.d, clocks)
             if (args.kernel == "quant" and args.workload == 1) else None,
-            "gpu_launches": K,
+            "gpu_launches": K * (3 if args.kernel == "split" else 1),   # split: first kernel, fit, pack
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": n_e2e,
                     "method": f"CUDA graphs of {n_g} steps (each: one H2D copy of the step's inputs from pinned "
