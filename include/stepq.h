@@ -286,10 +286,17 @@ STEPQ_API int stepq_calib_distortion_static(stepq_dims dims, const float* S, con
 STEPQ_API int stepq_allocate_bits(int n_units, int n_cand, const int* cand_host, const double* J_host,
                         int64_t budget_bits, int mode, uint8_t* bits_out_host);
 
-/* Device error word of the fused decode kernel: bit 0 is set when a bounded wait for a tile
-   copy gave up; bit 1 when a width-16 row was met in a launch with dims.pivots = 0. Reads
-   (synchronously, on the current device) and clears it. */
+/* Device error word of the library's kernels: bit 0 is set when a bounded wait (for a tile
+   copy, or a tensor-core round of the prefill chunk) gave up after its limit (2 s); the kernel
+   then waits, bounded, for its own copies in flight, frees its tensor memory and returns, so the
+   context stays usable. Bit 1 is set when a width-16 row was met in a launch with
+   dims.pivots = 0. Reads (synchronously, on the current device) and clears it. */
 STEPQ_API int stepq_read_device_flags(uint32_t* flags_host);
+
+/* Self-test of that wait limit: one bounded wait that nothing completes (an mbarrier phase no
+   thread arrives on), giving up after limit_ns (1e3 to 1e9 ns, else STEPQ_EINVAL before any
+   CUDA call) and raising bit 0 of the device error word. Queued on `stream`. */
+STEPQ_API int stepq_selftest_wait(uint64_t limit_ns, void* stream);
 
 /* Build description (compute capability compiled for, and version). */
 STEPQ_API const char* stepq_build_info(void);

@@ -19,7 +19,7 @@ SYMBOLS = (
     "stepq_prefill_chunk_seq", "stepq_prefill_chunk_wy",
     "stepq_decode_step_fp32",
     "stepq_int8_quantize_state", "stepq_decode_step_int8", "stepq_leap_step", "stepq_row_impact",
-    "stepq_calib_distortion", "stepq_calib_distortion_bits", "stepq_calib_distortion_static", "stepq_allocate_bits", "stepq_read_device_flags",
+    "stepq_calib_distortion", "stepq_calib_distortion_bits", "stepq_calib_distortion_static", "stepq_allocate_bits", "stepq_read_device_flags", "stepq_selftest_wait",
     "stepq_build_info",
 )
 
@@ -63,6 +63,7 @@ _SIGNATURES = {
     "stepq_calib_distortion_bits": ([Dims, P, P, P, P, P, P, P], I),
     "stepq_allocate_bits": ([I, I, P, P, I64, I, P], I),
     "stepq_read_device_flags": ([P], I),
+    "stepq_selftest_wait": ([ctypes.c_uint64, P], I),
 }
 
 

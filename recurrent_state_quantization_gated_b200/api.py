@@ -24,7 +24,7 @@ __all__ = [
     "stepq_prefill_chunk_seq", "stepq_prefill_chunk_wy", "stepq_decode_step_fp32", "stepq_int8_quantize_state",
     "stepq_decode_step_int8", "stepq_leap_step", "stepq_row_impact", "stepq_calib_distortion", "stepq_calib_distortion_bits", "stepq_calib_distortion_static",
     "stepq_allocate_bits",
-    "stepq_read_device_flags", "stepq_build_info",
+    "stepq_read_device_flags", "stepq_selftest_wait", "stepq_build_info",
 ]
 
 
@@ -300,3 +300,9 @@ def stepq_read_device_flags() -> int:
     flags = ctypes.c_uint32(0)
     call("stepq_read_device_flags", ctypes.byref(flags))
     return flags.value
+
+
+def stepq_selftest_wait(limit_ns: int) -> None:
+    """One bounded wait that nothing completes, on the current stream: after limit_ns it gives
+    up and raises bit 0 of the device error word (read it with stepq_read_device_flags)."""
+    call("stepq_selftest_wait", ctypes.c_uint64(int(limit_ns)), _stream())

@@ -533,3 +533,29 @@ extern "C" int stepq_leap_step(stepq_dims dims, int window, int t, const uint16_
     };
     return dims.dk == 128 ? go(leap_step_kernel<128>, sizeof(LeapSmem<128>)) : go(leap_step_kernel<64>, sizeof(LeapSmem<64>));
 }
+
+namespace stepq {
+// One bounded wait that nothing completes: a fresh mbarrier's phase 0 never sees an arrival, so
+// the wait gives up after limit_ns and raises bit 0 of the device error word, as a stalled tile
+// copy or tensor-core round would in the library's kernels.
+__global__ void wait_selftest_kernel(uint64_t limit_ns, uint32_t* flags) {
+    __shared__ alignas(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, limit_ns, flags);
+}
+}  // namespace stepq
+
+extern "C" int stepq_selftest_wait(uint64_t limit_ns, void* stream) {
+    clear_error();
+    if (limit_ns < 1000 || limit_ns > 1000000000ull)
+        return set_error(STEPQ_EINVAL, "stepq_selftest_wait: limit_ns=%llu (need 1e3 to 1e9)", (unsigned long long)limit_ns);
+    uint32_t* flags = nullptr;
+    int rc = device_flags_ptr(&flags);
+    if (rc) return rc;
+    wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, flags);
+    return check_launch("stepq_selftest_wait");
+}

@@ -179,3 +179,10 @@ def test_per_window_step_validates_before_touching_cuda():
     assert lib.stepq_leap_step(_dims(B=0), 16, 3, *args) == _lib.STEPQ_OK
     rc = lib.stepq_leap_step(_dims(), 16, 3, *([P()] * 5), P(), P(), ctypes.c_void_p(0), P(), P(), P(), None)
     assert rc == _lib.STEPQ_EINVAL and b"kbuf is NULL" in lib.stepq_last_error()
+
+
+def test_wait_selftest_validates_its_limit_before_touching_cuda():
+    lib = _lib.lib()
+    for bad in (0, 999, 10**9 + 1):
+        assert lib.stepq_selftest_wait(ctypes.c_uint64(bad), None) == _lib.STEPQ_EINVAL
+    assert b"limit_ns" in lib.stepq_last_error()

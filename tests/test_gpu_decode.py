@@ -186,3 +186,35 @@ def test_mixed_and_width_specialised_paths_agree(pivots):
     torch.cuda.synchronize()
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def test_a_wait_that_runs_out_is_reported_and_the_context_stays_usable():
+    """The kernels' bounded waits (tile copies, tensor-core rounds) give up after their limit,
+    raise bit 0 of the device error word and return: a wait that nothing completes reports bit 0
+    after its limit, and the next decode step runs normally with the error word clear."""
+    import time
+
+    import torch
+    from recurrent_state_quantization_gated_b200 import api
+    assert api.stepq_read_device_flags() == 0
+    t0 = time.perf_counter()
+    api.stepq_selftest_wait(50_000_000)                     # 50 ms
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 >= 0.04
+    assert api.stepq_read_device_flags() == 1
+    wl = synth.workload(1, B=2, H=3, d=128, seed=23)
+    S0 = synth.initial_state(wl)
+    bits = synth.random_bits(wl.H, wl.d, choices=(4, 6, 8), seed=2)
+    w = synth.random_weights(wl.H, wl.d, seed=3)
+    r, c = oracle.fit_scales(S0, w, bits)
+    packed = oracle.pack_state(S0, bits, r, c)
+    head_off, bps, _ = api.stepq_packed_layout(bits, wl.d, wl.B)
+    tok = synth.tokens(wl, 0)
+    td = tokens_dev(tok)
+    p_g, r_g, c_g, o_g = api.stepq_decode_step(td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w),
+                                               dev(head_off), bps, dev(packed), dev(r, torch.float16),
+                                               dev(c, torch.float16))
+    torch.cuda.synchronize()
+    ref = oracle.decode_step(tok, bits, w, packed, r, c)
+    compare_decode((p_g.cpu().numpy(), host_half(r_g), host_half(c_g), o_g.cpu().numpy()), ref, bits, wl.d, wl.B)
+    assert api.stepq_read_device_flags() == 0
