@@ -250,8 +250,8 @@ def run_reference(args, wl, budget_s: float = 90.0):
     cores = len(os.sched_getaffinity(0))
     # The oracle's own offline calibration of the workload (row impact, distortions on the
     # initial states, allocation), as the GPU arm does with the CUDA library.
-    bits, w = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl),
-                               synth.initial_state(wl), synth.calib_tokens(wl), n_pivots=wl.n_pivots)
+    bits, w = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.initial_state(wl),
+                               synth.calib_tokens(wl), n_pivots=wl.n_pivots)
     if bits is None:
         bits = synth.half_bits(wl)
 
@@ -356,7 +356,7 @@ def main():
         bits = synth.half_bits(wl)
         w = api.stepq_row_impact(cal_dev["q"], cal_dev["k"], cal_dev["beta"], cal_dev["gate"])
     else:
-        bits, w = runtime.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), S0, cal_dev,
+        bits, w = runtime.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, S0, cal_dev,
                                     n_pivots=wl.n_pivots)
     layout = runtime.Layout.build(bits, wl.d)
     base = runtime.QuantizedState.from_fp32(S0, layout, w)

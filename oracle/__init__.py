@@ -354,15 +354,29 @@ def allocate_bits(J, cand, budget, mode):
     return out
 
 
-def lifetime(gate):
-    """Unit lifetime L_u = 1 / (1 - g_u): the sum over j >= 0 of the retention product g_u^j."""
+LIFETIME_HORIZON = 2048
+
+
+def mean_log_retention(gate):
+    """ell_u = E_cal[log r_{t,u}] (App. A.3, "Mean log retention"): the mean over the steps and
+    sequences of a calibration gate stream, gate [T][B][H] (head units, result [H]) or
+    [T][B][H][dk] (key-channel units, result [H][dk])."""
     g = np.asarray(gate, dtype=np.float64)
-    return 1.0 / (1.0 - g)
+    return np.log(g).mean(axis=(0, 1))
 
 
-def objective(d, gate):
-    """J_u(b) = L_u d_u(b): lifetime-weighted distortion, d [n_units][n_cand]."""
-    return lifetime(gate)[:, None] * np.asarray(d, dtype=np.float64)
+def lifetime(ell, horizon=LIFETIME_HORIZON):
+    """L_u = sum_{j=0}^{horizon-1} exp(2 j ell_u) (App. A.3), summed term by term: the squared
+    error a unit keeps over the horizon, per unit of squared error injected once, when each step
+    retains exp(ell_u) of it."""
+    ell = np.asarray(ell, dtype=np.float64)
+    j = np.arange(int(horizon), dtype=np.float64)
+    return np.exp(2.0 * ell[..., None] * j).sum(axis=-1)
+
+
+def objective(d, ell, horizon=LIFETIME_HORIZON):
+    """J_u(b) = L_u d_u(b): lifetime-weighted distortion, d [n_units][n_cand], ell [n_units]."""
+    return lifetime(ell, horizon)[:, None] * np.asarray(d, dtype=np.float64)
 
 
 def pivot_order(score):
@@ -371,14 +385,16 @@ def pivot_order(score):
     return np.lexsort((np.arange(score.size), -score))
 
 
-def calibrate(alloc, candidates, nominal_bits, gates, S0, calib, n_pivots=0):
+def calibrate(alloc, candidates, nominal_bits, S0, calib, n_pivots=0, horizon=LIFETIME_HORIZON):
     """The offline calibration done by the oracle (App. A.3, B.3, C.2): returns
     (bits uint8 [H][dk] or None, w float32 [H][dk]).
 
     alloc: "dp_head" (head units, multiple-choice DP, Eq. 17 distortion) or "lagrange_row"
     (key-row units, Lagrangian allocation with repair, Eq. 18 distortion); any other value
-    returns bits=None (the caller supplies a fixed map). gates: unit gates [H] or [H][dk];
-    S0: the sample states [B][H][dk][dv]; calib: the calibration stream.
+    returns bits=None (the caller supplies a fixed map). S0: the sample states [B][H][dk][dv];
+    calib: the calibration stream. Each unit's lifetime L_u comes from the mean log retention of
+    the stream's gates (App. A.3): a head unit averages the log gate over its key channels, a
+    key-row unit under a head gate takes its head's value; ``horizon`` is the H of that sum.
 
     n_pivots > 0 keeps that many units in FP16 (width 16, App. C.2, Table B1):
       key rows: ranked by the lifetime-weighted reduction of error from the integer format at
@@ -395,7 +411,7 @@ def calibrate(alloc, candidates, nominal_bits, gates, S0, calib, n_pivots=0):
     if alloc not in ("dp_head", "lagrange_row"):
         return None, w
     cand = [int(b) for b in candidates]
-    gates = np.asarray(gates, dtype=np.float32)
+    ell = mean_log_retention(calib["gate"])                    # [H] or [H][dk]
     drows, dheads = [], []
     for b in cand:
         dr, dh = calib_distortion(S0, w, b)
@@ -403,8 +419,8 @@ def calibrate(alloc, candidates, nominal_bits, gates, S0, calib, n_pivots=0):
         dheads.append(dh)
     if alloc == "dp_head":
         dist = np.stack(dheads, axis=1)                          # [H][n_cand]
-        g = gates if gates.ndim == 1 else gates.mean(axis=1)
-        J = objective(dist, g)
+        ell_h = ell if ell.ndim == 1 else ell.mean(axis=1)
+        J = objective(dist, ell_h, horizon)
         bh = allocate_bits(J, cand, nominal_bits * H, mode=1)
         if n_pivots:
             risk = J[np.arange(H), [cand.index(int(b)) for b in bh]]
@@ -414,16 +430,16 @@ def calibrate(alloc, candidates, nominal_bits, gates, S0, calib, n_pivots=0):
             bh[rest] = allocate_bits(J[rest], cand, nominal_bits * H - 8 * n_pivots, mode=1)
             bh[piv] = 16
         return np.repeat(bh[:, None], dk, axis=1).astype(np.uint8), w
-    g = gates.reshape(-1) if gates.ndim == 2 else np.repeat(gates, dk)
+    ell_r = ell.reshape(-1) if ell.ndim == 2 else np.repeat(ell, dk)
     n = H * dk
     if not n_pivots:
         dist = np.stack([dr.reshape(-1) for dr in drows], axis=1)   # [H*dk][n_cand]
-        br = allocate_bits(objective(dist, g), cand, nominal_bits * n, mode=0)
+        br = allocate_bits(objective(dist, ell_r, horizon), cand, nominal_bits * n, mode=0)
         return br.reshape(H, dk).astype(np.uint8), w
     d16, _ = calib_distortion(S0, w, 16)
     dnom = drows[cand.index(int(nominal_bits))] if int(nominal_bits) in cand else \
         calib_distortion(S0, w, nominal_bits)[0]
-    score = lifetime(g) * (dnom.reshape(-1) - d16.reshape(-1))
+    score = lifetime(ell_r, horizon) * (dnom.reshape(-1) - d16.reshape(-1))
     piv = np.sort(pivot_order(score)[:n_pivots])
     rest = np.setdiff1d(np.arange(n), piv)
     dist = []
@@ -433,6 +449,7 @@ def calibrate(alloc, candidates, nominal_bits, gates, S0, calib, n_pivots=0):
         dist.append(calib_distortion_bits(S0, w, m.reshape(H, dk))[0].reshape(-1))
     dist = np.stack(dist, axis=1)
     br = np.zeros(n, dtype=np.uint8)
-    br[rest] = allocate_bits(objective(dist[rest], g[rest]), cand, nominal_bits * n - 8 * n_pivots, mode=0)
+    br[rest] = allocate_bits(objective(dist[rest], ell_r[rest], horizon), cand, nominal_bits * n - 8 * n_pivots,
+                             mode=0)
     br[piv] = 16
     return br.reshape(H, dk), w

@@ -3,8 +3,8 @@
 ``QuantizedState`` keeps one layer's packed recurrent states (codes, fp16 row/column scales,
 the frozen bit map, row-impact vector and packed layout) resident on the GPU and advances them
 with the fused decode kernel. ``calibrate`` runs the offline part of STEPQuant (App. C.2): row
-impact (App. B.3) and candidate distortions (App. A.3) on the GPU, lifetime weighting (§3.2)
-and the discrete allocation (multiple-choice DP or Lagrangian) in the host library.
+impact (App. B.3) and candidate distortions (App. A.3) on the GPU, lifetime weighting (§3.2,
+App. A.3) and the discrete allocation (multiple-choice DP or Lagrangian) in the host library.
 """
 from __future__ import annotations
 
@@ -109,19 +109,36 @@ class WindowState:
         return self.codes.numel() + 2 * self.s.numel()
 
 
-def lifetime(unit_gates) -> np.ndarray:
-    """L_u = 1/(1 - g_u): the sum over j >= 0 of g_u^j, the retention of a unit's error (§3.2)."""
-    g = np.asarray(unit_gates, dtype=np.float64)
-    return 1.0 / (1.0 - g)
+LIFETIME_HORIZON = 2048
 
 
-def calibrate(alloc: str, candidates, nominal_bits: int, unit_gates, S0: torch.Tensor, calib: dict, n_pivots: int = 0):
+def mean_log_retention(gate) -> np.ndarray:
+    """ell_u = E[log r_{t,u}] over a calibration gate stream (App. A.3, mean log retention):
+    gate [T][B][H] gives one value per head [H], gate [T][B][H][d] one per key channel [H][d]."""
+    g = gate.detach().cpu().numpy() if isinstance(gate, torch.Tensor) else np.asarray(gate)
+    return np.log(g.astype(np.float64)).mean(axis=(0, 1))
+
+
+def lifetime(ell, horizon: int = LIFETIME_HORIZON) -> np.ndarray:
+    """L_u = sum over 0 <= j < horizon of exp(2 j ell_u) (App. A.3): the squared error a unit
+    keeps over the horizon per unit injected once. Geometric series in closed form,
+    expm1(2 horizon ell) / expm1(2 ell), which is horizon at ell = 0."""
+    x = 2.0 * np.asarray(ell, dtype=np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        L = np.expm1(horizon * x) / np.expm1(x)
+    return np.where(x == 0.0, float(horizon), L)
+
+
+def calibrate(alloc: str, candidates, nominal_bits: int, S0: torch.Tensor, calib: dict, n_pivots: int = 0,
+              horizon: int = LIFETIME_HORIZON):
     """Offline calibration of one layer. Returns (bits uint8 numpy [H][d], w float32 [H][d] on GPU).
 
     alloc: "dp_head" (head units, Eq. 17 distortion, multiple-choice DP) or "lagrange_row"
     (key-row units, Eq. 18 distortion, Lagrangian allocation with repair).
-    unit_gates: [H] (head gates) or [H][d] (key-channel gates); S0: the sample states
-    [B,H,d,d] on the GPU; calib: the calibration stream as GPU tensors with a leading step axis.
+    S0: the sample states [B,H,d,d] on the GPU; calib: the calibration stream as GPU tensors
+    with a leading step axis. Unit lifetimes come from the stream's mean log retention (App.
+    A.3): a head unit averages the log gate over its key channels, a key row under a head gate
+    takes its head's; ``horizon`` is the number of steps the lifetime sums over.
     n_pivots: units kept in FP16 (width 16; App. C.2): key rows ranked by the lifetime-weighted
     error reduction L_u (d_u(nominal) - d_u(16)), then the other rows' distortions measured
     again without the pivots in the column fit; heads ranked by residual risk L_u d_u(b_u)
@@ -130,7 +147,7 @@ def calibrate(alloc: str, candidates, nominal_bits: int, unit_gates, S0: torch.T
     w = api.stepq_row_impact(calib["q"], calib["k"], calib["beta"], calib["gate"])
     H, d = w.shape
     cand = [int(b) for b in candidates]
-    gates = np.asarray(unit_gates, dtype=np.float64)
+    ell = mean_log_retention(calib["gate"])
     rows, heads = [], []
     for b in cand:
         d_row, d_head = api.stepq_calib_distortion(S0, w, b)
@@ -138,8 +155,8 @@ def calibrate(alloc: str, candidates, nominal_bits: int, unit_gates, S0: torch.T
         heads.append(d_head.cpu().numpy())
     if alloc == "dp_head":
         dist = np.stack(heads, axis=1)
-        g = gates if gates.ndim == 1 else gates.mean(axis=1)
-        J = lifetime(g)[:, None] * dist
+        ell_h = ell if ell.ndim == 1 else ell.mean(axis=1)
+        J = lifetime(ell_h, horizon)[:, None] * dist
         bh = api.stepq_allocate_bits(J, cand, nominal_bits * H, mode=1)
         if n_pivots:
             risk = J[np.arange(H), [cand.index(int(b)) for b in bh]]
@@ -150,9 +167,9 @@ def calibrate(alloc: str, candidates, nominal_bits: int, unit_gates, S0: torch.T
             bh[piv] = 16
         return np.repeat(bh[:, None], d, axis=1).astype(np.uint8), w
     if alloc == "lagrange_row":
-        g = gates.reshape(-1) if gates.ndim == 2 else np.repeat(gates, d)
+        ell_r = ell.reshape(-1) if ell.ndim == 2 else np.repeat(ell, d)
         n = H * d
-        L = lifetime(g)
+        L = lifetime(ell_r, horizon)
         if not n_pivots:
             dist = np.stack([x.reshape(-1) for x in rows], axis=1)
             br = api.stepq_allocate_bits(L[:, None] * dist, cand, nominal_bits * n, mode=0)

@@ -21,7 +21,7 @@ def _calibrated(wl, n_samples=8):
     seqs = range(min(n_samples, wl.B))
     S0 = synth.initial_state(wl, seqs)
     cal = synth.calib_tokens(wl, seqs)
-    bits, w = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), S0, cal,
+    bits, w = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, S0, cal,
                                n_pivots=wl.n_pivots)
     # each FP16 pivot row counts 8 bits of the integer budget and 8 on top (App. D)
     assert bits.astype(np.int64).sum() == wl.nominal_bits * bits.size + 8 * int((bits == 16).sum())

@@ -129,11 +129,11 @@ def test_calibration_allocation_matches_oracle():
         wl = synth.workload(idx, **over)
         S0 = synth.initial_state(wl)
         cal = synth.calib_tokens(wl)
-        bits_ref, w_ref = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), S0, cal,
+        bits_ref, w_ref = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, S0, cal,
                                            n_pivots=wl.n_pivots)
         cal_dev = dict(q=dev(cal["q"], torch.bfloat16), k=dev(cal["k"], torch.bfloat16), beta=dev(cal["beta"]),
                        gate=dev(cal["gate"]))
-        bits, w = runtime.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), dev(S0), cal_dev,
+        bits, w = runtime.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, dev(S0), cal_dev,
                                     n_pivots=wl.n_pivots)
         np.testing.assert_allclose(w.cpu().numpy(), w_ref, rtol=1e-6)
         np.testing.assert_array_equal(bits, bits_ref)

@@ -106,14 +106,14 @@ def test_row_pivots_take_the_largest_lifetime_weighted_gain_and_the_budget_adds_
     S0 = synth.initial_state(wl)
     cal = synth.calib_tokens(wl)
     P = 5
-    bits, w = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), S0, cal, n_pivots=P)
+    bits, w = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, S0, cal, n_pivots=P)
     piv = np.flatnonzero(bits.reshape(-1) == 16)
     assert piv.size == P
     assert bits.astype(np.int64).sum() == wl.nominal_bits * bits.size + 8 * P
     assert set(np.unique(bits[bits != 16])) <= set(wl.candidates)
     d16, _ = oracle.calib_distortion(S0, w, 16)
     dnom, _ = oracle.calib_distortion(S0, w, wl.nominal_bits)
-    gain = oracle.lifetime(synth.unit_gates(wl)).reshape(-1) * (dnom - d16).reshape(-1)
+    gain = oracle.lifetime(np.log(synth.unit_gates(wl).astype(np.float64))).reshape(-1) * (dnom - d16).reshape(-1)
     assert gain[piv].min() >= np.delete(gain, piv).max()
 
 
@@ -121,13 +121,13 @@ def test_head_pivots_take_the_largest_residual_risk():
     wl = synth.workload(1, B=3, H=6, d=64)
     S0 = synth.initial_state(wl)
     cal = synth.calib_tokens(wl)
-    b0, w = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), S0, cal)
-    b1, _ = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, synth.unit_gates(wl), S0, cal, n_pivots=1)
+    b0, w = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, S0, cal)
+    b1, _ = oracle.calibrate(wl.alloc, wl.candidates, wl.nominal_bits, S0, cal, n_pivots=1)
     heads0, heads1 = b0[:, 0], b1[:, 0]
     assert (b1 == b1[:, :1]).all() and (heads1 == 16).sum() == 1
     assert heads1.astype(np.int64).sum() == wl.nominal_bits * wl.H + 8
     risk = []
     for h, b in enumerate(heads0):
         _, dh = oracle.calib_distortion(S0, w, int(b))
-        risk.append(oracle.lifetime(synth.unit_gates(wl))[h] * dh[h])
+        risk.append(oracle.lifetime(np.log(synth.unit_gates(wl).astype(np.float64)))[h] * dh[h])
     assert heads1[int(np.argmax(risk))] == 16
