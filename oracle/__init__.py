@@ -370,8 +370,10 @@ def lifetime(ell, horizon=LIFETIME_HORIZON):
     error a unit keeps over the horizon, per unit of squared error injected once, when each step
     retains exp(ell_u) of it."""
     ell = np.asarray(ell, dtype=np.float64)
-    j = np.arange(int(horizon), dtype=np.float64)
-    return np.exp(2.0 * ell[..., None] * j).sum(axis=-1)
+    total = np.zeros_like(ell)
+    for j in range(int(horizon)):
+        total += np.exp(2.0 * j * ell)
+    return total
 
 
 def objective(d, ell, horizon=LIFETIME_HORIZON):

@@ -166,9 +166,9 @@ MUTANTS = [
        ("if (!found || dj < bdj) { found = 1; bdj = dj; bu = u; bku = kk; bv = -1; }",
         "if (!found) { found = 1; bdj = dj; bu = u; bku = kk; bv = -1; }")),
     _m("lifetime sums the retention, not the squared error", PY_SRC,
-       ("return np.exp(2.0 * ell[..., None] * j).sum(axis=-1)", "return np.exp(ell[..., None] * j).sum(axis=-1)")),
+       ("total += np.exp(2.0 * j * ell)", "total += np.exp(j * ell)")),
     _m("lifetime sum starts one step late", PY_SRC,
-       ("j = np.arange(int(horizon), dtype=np.float64)", "j = np.arange(1, int(horizon), dtype=np.float64)")),
+       ("for j in range(int(horizon)):", "for j in range(1, int(horizon)):")),
     _m("mean log retention taken as the log of the mean gate", PY_SRC,
        ("return np.log(g).mean(axis=(0, 1))", "return np.log(g.mean(axis=(0, 1)))")),
     _m("objective without the lifetime", PY_SRC,
