@@ -44,6 +44,18 @@ def _ptr(t: torch.Tensor, dtype: torch.dtype, name: str):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _sizes(**tensors):
+    """Each tensor (name=(tensor, elements)) must hold at least that many elements, so that no
+    kernel reads or writes past a buffer given through the C ABI (which sees only pointers)."""
+    for name, (t, n) in tensors.items():
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.numel() < n:
+            raise ValueError(f"{name}: {t.numel()} elements, the call needs {n}")
+
+
 def _dims(B, H, d, gate_per_channel=0, pivots=0, mixed=0):
     return Dims(int(B), int(H), int(d), int(d), int(gate_per_channel), int(pivots), int(mixed))
 
@@ -82,6 +94,7 @@ def stepq_fit_scales(S, w, bits, r=None, c=None):
     B, H, d, _ = S.shape
     r = torch.empty((B, H, d), dtype=torch.float16, device=S.device) if r is None else r
     c = torch.empty((B, H, d), dtype=torch.float16, device=S.device) if c is None else c
+    _sizes(w=(w, H * d), bits=(bits, H * d), r=(r, B * H * d), c=(c, B * H * d))
     call("stepq_fit_scales", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
          _ptr(bits, torch.uint8, "bits"), _ptr(r, torch.float16, "r"), _ptr(c, torch.float16, "c"), _stream())
     return r, c
@@ -90,6 +103,8 @@ def stepq_fit_scales(S, w, bits, r=None, c=None):
 def stepq_pack_state(S, bits, head_off, bytes_per_seq, r, c, packed=None):
     B, H, d, _ = S.shape
     packed = torch.empty(B * bytes_per_seq, dtype=torch.uint8, device=S.device) if packed is None else packed
+    _sizes(bits=(bits, H * d), head_off=(head_off, H), r=(r, B * H * d), c=(c, B * H * d),
+           packed=(packed, B * int(bytes_per_seq)))
     call("stepq_pack_state", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(bits, torch.uint8, "bits"),
          _ptr(head_off, torch.int64, "head_off"), ctypes.c_int64(int(bytes_per_seq)),
          _ptr(r, torch.float16, "r"), _ptr(c, torch.float16, "c"), _ptr(packed, torch.uint8, "packed"), _stream())
@@ -99,10 +114,22 @@ def stepq_pack_state(S, bits, head_off, bytes_per_seq, r, c, packed=None):
 def stepq_unpack_state(packed, bits, head_off, bytes_per_seq, r, c, S_out=None):
     B, H, d = r.shape
     S_out = torch.empty((B, H, d, d), dtype=torch.float32, device=r.device) if S_out is None else S_out
+    _sizes(packed=(packed, B * int(bytes_per_seq)), bits=(bits, H * d), head_off=(head_off, H), c=(c, B * H * d),
+           S_out=(S_out, B * H * d * d))
     call("stepq_unpack_state", _dims(B, H, d), _ptr(packed, torch.uint8, "packed"), _ptr(bits, torch.uint8, "bits"),
          _ptr(head_off, torch.int64, "head_off"), ctypes.c_int64(int(bytes_per_seq)),
          _ptr(r, torch.float16, "r"), _ptr(c, torch.float16, "c"), _ptr(S_out, torch.float32, "S_out"), _stream())
     return S_out
+
+
+def _step_sizes(B, H, d, gpc, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
+                packed_out, r_out, c_out, o, C=1):
+    """Element counts of a decode step's (C = 1) or a prefill chunk's buffers."""
+    n = B * H * d
+    return dict(k=(k, C * n), v=(v, C * n), beta=(beta, C * B * H), gate=(gate, C * B * H * (d if gpc else 1)),
+                bits=(bits, H * d), w=(w, H * d), head_off=(head_off, H),
+                packed_in=(packed_in, B * int(bytes_per_seq)), r_in=(r_in, n), c_in=(c_in, n),
+                packed_out=(packed_out, B * int(bytes_per_seq)), r_out=(r_out, n), c_out=(c_out, n), o=(o, C * n))
 
 
 def stepq_decode_step(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
@@ -116,6 +143,8 @@ def stepq_decode_step(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, pac
     r_out = torch.empty_like(r_in) if r_out is None else r_out
     c_out = torch.empty_like(c_in) if c_out is None else c_out
     o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
+    _sizes(**_step_sizes(B, H, d, gpc, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
+                         packed_out, r_out, c_out, o))
     call("stepq_decode_step", _dims(B, H, d, gpc, _has_pivots(bits, pivots), _has_mixed(bits, mixed)),
          _ptr(q, torch.bfloat16, "q"),
          _ptr(k, torch.bfloat16, "k"),
@@ -145,6 +174,9 @@ def stepq_decode_step_split(q, k, v, beta, gate, bits, w, head_off, bytes_per_se
         c_out = torch.empty_like(c_in) if c_out is None else c_out
     own = side_stream is None and refit
     side = torch.cuda.Stream() if own else side_stream
+    _sizes(x_ws=(x_ws, B * H * d * d),
+           **_step_sizes(B, H, d, gpc, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
+                         packed_out, r_out, c_out, o))
     opt = lambda t, dt, n: _ptr(t, dt, n) if t is not None else None
     call("stepq_decode_step_split", _dims(B, H, d, gpc, _has_pivots(bits, pivots)), _ptr(q, torch.bfloat16, "q"),
          _ptr(k, torch.bfloat16, "k"),
@@ -174,6 +206,8 @@ def stepq_prefill_chunk(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, p
     c_out = torch.empty_like(c_in) if c_out is None else c_out
     o = torch.empty((C, B, H, d), dtype=torch.float32, device=q.device) if o is None else o
     name = {None: "stepq_prefill_chunk", "seq": "stepq_prefill_chunk_seq", "wy": "stepq_prefill_chunk_wy"}[form]
+    _sizes(**_step_sizes(B, H, d, gpc, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
+                         packed_out, r_out, c_out, o, C=C))
     call(name, _dims(B, H, d, gpc, _has_pivots(bits, pivots), _has_mixed(bits, mixed)), ctypes.c_int(int(C)),
          _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
          _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"), _ptr(bits, torch.uint8, "bits"),
@@ -190,6 +224,9 @@ def stepq_decode_step_fp32(q, k, v, beta, gate, S_in, S_out=None, o=None):
     gpc = 1 if gate.dim() == 3 else 0
     S_out = torch.empty_like(S_in) if S_out is None else S_out
     o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
+    n = B * H * d
+    _sizes(k=(k, n), v=(v, n), beta=(beta, B * H), gate=(gate, B * H * (d if gpc else 1)), S_in=(S_in, n * d),
+           S_out=(S_out, n * d), o=(o, n))
     call("stepq_decode_step_fp32", _dims(B, H, d, gpc), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
          _ptr(v, torch.bfloat16, "v"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
          _ptr(S_in, torch.float32, "S_in"), _ptr(S_out, torch.float32, "S_out"), _ptr(o, torch.float32, "o"),
@@ -201,6 +238,7 @@ def stepq_int8_quantize_state(S, codes=None, s=None):
     B, H, d, _ = S.shape
     codes = torch.empty((B, H, d, d), dtype=torch.int8, device=S.device) if codes is None else codes
     s = torch.empty((B, H, d), dtype=torch.float16, device=S.device) if s is None else s
+    _sizes(codes=(codes, B * H * d * d), s=(s, B * H * d))
     call("stepq_int8_quantize_state", _dims(B, H, d), _ptr(S, torch.float32, "S"),
          _ptr(codes, torch.int8, "codes"), _ptr(s, torch.float16, "s"), _stream())
     return codes, s
@@ -212,6 +250,9 @@ def stepq_decode_step_int8(q, k, v, beta, gate, codes_in, s_in, codes_out=None, 
     codes_out = torch.empty_like(codes_in) if codes_out is None else codes_out
     s_out = torch.empty_like(s_in) if s_out is None else s_out
     o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
+    n = B * H * d
+    _sizes(k=(k, n), v=(v, n), beta=(beta, B * H), gate=(gate, B * H * (d if gpc else 1)),
+           codes_in=(codes_in, n * d), s_in=(s_in, n), codes_out=(codes_out, n * d), s_out=(s_out, n), o=(o, n))
     call("stepq_decode_step_int8", _dims(B, H, d, gpc), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
          _ptr(v, torch.bfloat16, "v"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
          _ptr(codes_in, torch.int8, "codes_in"), _ptr(s_in, torch.float16, "s_in"),
@@ -226,6 +267,9 @@ def stepq_leap_step(window, t, q, k, v, beta, gate, codes, s, kbuf, ubuf, lbuf, 
     kbuf bf16 [window,B,H,d], ubuf fp32 [window,B,H,d], lbuf fp32 [window,B,H]. Returns o."""
     B, H, d = q.shape
     o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
+    n, W = B * H * d, int(window)
+    _sizes(k=(k, n), v=(v, n), beta=(beta, B * H), gate=(gate, B * H), codes=(codes, n * d), s=(s, n),
+           kbuf=(kbuf, W * n), ubuf=(ubuf, W * n), lbuf=(lbuf, W * B * H), o=(o, n))
     call("stepq_leap_step", _dims(B, H, d, 0), ctypes.c_int(int(window)), ctypes.c_int(int(t)),
          _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
          _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"), _ptr(codes, torch.int8, "codes"),
@@ -239,6 +283,8 @@ def stepq_row_impact(q, k, beta, gate, w_out=None):
     T, B, H, d = q.shape
     gpc = 1 if gate.dim() == 4 else 0
     w_out = torch.empty((H, d), dtype=torch.float32, device=q.device) if w_out is None else w_out
+    _sizes(k=(k, T * B * H * d), beta=(beta, T * B * H), gate=(gate, T * B * H * (d if gpc else 1)),
+           w_out=(w_out, H * d))
     call("stepq_row_impact", _dims(B, H, d, gpc), ctypes.c_int(T), _ptr(q, torch.bfloat16, "q"),
          _ptr(k, torch.bfloat16, "k"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),
          _ptr(w_out, torch.float32, "w_out"), _stream())
@@ -252,6 +298,7 @@ def stepq_calib_distortion(S, w, b, d_row=None, d_head=None, scratch=None):
     d_row = torch.empty((H, d), dtype=torch.float64, device=dev) if d_row is None else d_row
     d_head = torch.empty((H,), dtype=torch.float64, device=dev) if d_head is None else d_head
     scratch = torch.empty((B, H, d), dtype=torch.float64, device=dev) if scratch is None else scratch
+    _sizes(w=(w, H * d), d_row=(d_row, H * d), d_head=(d_head, H), scratch=(scratch, B * H * d))
     call("stepq_calib_distortion", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
          ctypes.c_int(int(b)), _ptr(d_row, torch.float64, "d_row"), _ptr(d_head, torch.float64, "d_head"),
          _ptr(scratch, torch.float64, "scratch"), _stream())
@@ -266,6 +313,7 @@ def stepq_calib_distortion_bits(S, w, bits, d_row=None, d_head=None, scratch=Non
     d_row = torch.empty((H, d), dtype=torch.float64, device=dev) if d_row is None else d_row
     d_head = torch.empty((H,), dtype=torch.float64, device=dev) if d_head is None else d_head
     scratch = torch.empty((B, H, d), dtype=torch.float64, device=dev) if scratch is None else scratch
+    _sizes(w=(w, H * d), bits=(bits, H * d), d_row=(d_row, H * d), d_head=(d_head, H), scratch=(scratch, B * H * d))
     call("stepq_calib_distortion_bits", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
          _ptr(bits, torch.uint8, "bits"), _ptr(d_row, torch.float64, "d_row"), _ptr(d_head, torch.float64, "d_head"),
          _ptr(scratch, torch.float64, "scratch"), _stream())
@@ -279,6 +327,7 @@ def stepq_calib_distortion_static(S, w, b, d_row=None, d_head=None):
     dev = S.device
     d_row = torch.empty((H, d), dtype=torch.float64, device=dev) if d_row is None else d_row
     d_head = torch.empty((H,), dtype=torch.float64, device=dev) if d_head is None else d_head
+    _sizes(w=(w, H * d), d_row=(d_row, H * d), d_head=(d_head, H))
     call("stepq_calib_distortion_static", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
          ctypes.c_int(int(b)), _ptr(d_row, torch.float64, "d_row"), _ptr(d_head, torch.float64, "d_head"), _stream())
     return d_row, d_head
