@@ -39,6 +39,9 @@ def _ptr(t: torch.Tensor, dtype: torch.dtype, name: str):
         raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}; the calls run on the current device, "
+                         f"cuda:{torch.cuda.current_device()}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
