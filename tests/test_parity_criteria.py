@@ -1,0 +1,135 @@
+"""The GPU parity comparator (tests/helpers.py) enforces the stated criteria, checked on the CPU.
+
+One oracle decode step gives a reference result (packed codes, row and column scales,
+readouts). A "device" result is then made from it with planted deviations, and the comparator
+must accept exactly what the criteria allow: readouts within 1e-3 relative, row scales within
+one binary16 ulp, codes within one step on at most 0.1% of the entries whose scales agree, and
+FP16 pivot values within one ulp. Anything beyond that must fail. So a GPU result that broke a
+criterion cannot pass the GPU tests through a slack comparison."""
+import numpy as np
+import pytest
+
+import oracle
+from recurrent_state_quantization_gated_b200 import synth
+from tests.helpers import compare_decode, tile_codes, with_pivots
+
+D, B, H = 64, 2, 3
+
+
+@pytest.fixture(scope="module")
+def case():
+    wl = synth.workload(1, B=B, H=H, d=D, seed=21)
+    S0 = synth.initial_state(wl)
+    bits = with_pivots(synth.random_bits(H, D, choices=(2, 4, 6, 8), seed=22), 3, 23)
+    w = synth.random_weights(H, D, seed=24)
+    r, c = oracle.fit_scales(S0, w, bits)
+    packed = oracle.pack_state(S0, bits, r, c)
+    ref = oracle.decode_step(synth.tokens(wl, 0), bits, w, packed, r, c)
+    return bits, ref
+
+
+def _repack(codes, bits):
+    """Packed bytes of a full set of codes [B][H][d][d] (the oracle's packer, tile by tile)."""
+    head_off, bps = oracle.layout(bits, D)
+    out = np.zeros(B * bps, dtype=np.uint8)
+    for b in range(B):
+        for h in range(H):
+            t = oracle.pack_codes(codes[b, h], bits[h])
+            out[b * bps + head_off[h]: b * bps + head_off[h] + t.size] = t
+    return out
+
+
+def _movable(codes, bits):
+    """Entries of integer rows whose code can move one step up and stay in range."""
+    qmax = np.where(bits == 16, 0, (1 << (bits.astype(np.int64) - 1)) - 1)[None, :, :, None]
+    return (bits != 16)[None, :, :, None] & (codes < qmax)
+
+
+def _with_codes_moved(ref, bits, n, seed=0):
+    """The reference result with n seeded integer codes one step up (scales unchanged)."""
+    p, r, c, o = ref
+    codes = tile_codes(p, bits, D, B).astype(np.int64)
+    idx = np.flatnonzero(_movable(codes, bits))
+    pick = np.random.default_rng(seed).choice(idx, size=n, replace=False)
+    codes.reshape(-1)[pick] += 1
+    return (_repack(codes, bits), r, c, o)
+
+
+def test_identical_results_pass(case):
+    bits, ref = case
+    assert compare_decode(ref, ref, bits, D, B)[0] == 0.0
+
+
+def test_readouts_at_and_beyond_the_tolerance(case):
+    bits, ref = case
+    p, r, c, o = ref
+    for scale, ok in ((5e-4, True), (2e-3, False)):
+        o2 = o.copy()
+        o2[1, 2, 7] += scale * np.abs(o[1, 2]).max()       # one entry of one tile
+        if ok:
+            compare_decode((p, r, c, o2), ref, bits, D, B)
+        else:
+            with pytest.raises(AssertionError):
+                compare_decode((p, r, c, o2), ref, bits, D, B)
+
+
+def test_row_scales_one_ulp_pass_two_fail(case):
+    bits, ref = case
+    p, r, c, o = ref
+    for delta, ok in ((1, True), (2, False)):
+        r2 = r.copy()
+        r2[0, 1, 5] += delta
+        if ok:
+            compare_decode((p, r2, c, o), ref, bits, D, B)
+        else:
+            with pytest.raises(AssertionError):
+                compare_decode((p, r2, c, o), ref, bits, D, B)
+
+
+def test_a_column_scale_far_off_fails(case):
+    bits, ref = case
+    p, r, c, o = ref
+    c2 = c.copy()
+    c2[1, 0, 3] = (c2[1, 0, 3].view(np.float16) * np.float16(1.25)).view(np.uint16)
+    with pytest.raises(AssertionError):
+        compare_decode((p, r, c2, o), ref, bits, D, B)
+
+
+def test_one_step_on_few_codes_passes_on_many_fails(case):
+    bits, ref = case
+    n_int = int((bits != 16).sum()) * D * B
+    few = max(1, int(0.0008 * n_int))
+    many = int(0.003 * n_int)
+    frac = compare_decode(_with_codes_moved(ref, bits, few, seed=1), ref, bits, D, B)[0]
+    assert 0 < frac <= 1e-3
+    with pytest.raises(AssertionError):
+        compare_decode(_with_codes_moved(ref, bits, many, seed=2), ref, bits, D, B)
+
+
+def test_one_code_two_steps_apart_fails(case):
+    bits, ref = case
+    p, r, c, o = ref
+    codes = tile_codes(p, bits, D, B).astype(np.int64)
+    qmax = np.where(bits == 16, 0, (1 << (bits.astype(np.int64) - 1)) - 1)[None, :, :, None]
+    ok = (bits != 16)[None, :, :, None] & (codes + 2 <= qmax)
+    i = np.flatnonzero(ok)[7]
+    codes.reshape(-1)[i] += 2
+    with pytest.raises(AssertionError, match="codes differ by 2"):
+        compare_decode((_repack(codes, bits), r, c, o), ref, bits, D, B)
+
+
+def test_pivot_values_one_ulp_pass_two_fail(case):
+    bits, ref = case
+    p, r, c, o = ref
+    codes = tile_codes(p, bits, D, B).astype(np.int64)
+    piv = np.broadcast_to((bits == 16)[None, :, :, None], codes.shape)
+    i = np.flatnonzero(piv & (np.abs(codes.astype(np.uint16).view(np.int16).astype(np.int64)) > 4))[0]
+    for delta, ok in ((1, True), (2, False)):
+        cc = codes.copy()
+        cc.reshape(-1)[i] += delta                         # the next binary16 value(s) of the same sign
+        got = (_repack(cc, bits), r, c, o)
+        if ok:
+            compare_decode(got, ref, bits, D, B)
+        else:
+            with pytest.raises(AssertionError, match="pivot values"):
+                compare_decode(got, ref, bits, D, B)
