@@ -354,6 +354,8 @@ def allocate_bits(J, cand, budget, mode):
     return out
 
 
+# The horizon H of the lifetime sum (App. A.3) is not stated; 2048, the length of the calibration
+# segments (App. C.2), is taken for it.
 LIFETIME_HORIZON = 2048
 
 

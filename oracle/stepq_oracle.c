@@ -15,7 +15,7 @@
  * What each part follows (sections, equations and tables of the STEPQuant paper):
  *   recurrence        §2.1, the gated Delta rule and its affine form S_t = A_t S_{t-1} + B_t;
  *                     readout y_t = S_t^T q_t taken before requantisation (Table C2, step 3).
- *   gate D_t          scalar per head (GDN) or diagonal over key rows (KDA), §6.1 / App. C.1.
+ *   gate D_t          scalar per head (GDN) or diagonal over key rows (KDA), §2.1 / App. C.1.
  *   quantiser         §2.2, Q_{b,s}(x) = s clip(round(x/s), -q_b, q_b), q_b = 2^(b-1) - 1.
  *   code normalisation App. C.1: stored integer q, reconstruction z = 2^(8-b) q.
  *   dual-axis scales  §4.3, X_hat_ij = r_i c_j z_ij; row factor m_i = mean_j |X_ij| (§4.3
@@ -55,6 +55,12 @@
  *      any other (R1) and is not used.
  *   R15 a pivot value is the fp32 X rounded to binary16, nearest with ties to even,
  *      saturating at +-65504.
+ *
+ * Parity unpinned: R1's division of the row factor by w_i and R7's use of the 1/8 exponent for
+ * KDA rows are readings the paper does not state (it omits the formula, and gives the exponent
+ * for Qwen only). The tests pin the definitions around them, such as m_i, omega_i from explicit
+ * transition matrices, and the no-clip and least-squares properties of the fit, but not the
+ * readings themselves.
  */
 #include <math.h>
 #include <stdint.h>

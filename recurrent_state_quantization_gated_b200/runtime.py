@@ -109,6 +109,8 @@ class WindowState:
         return self.codes.numel() + 2 * self.s.numel()
 
 
+# The horizon H of the lifetime sum (App. A.3) is not stated; 2048, the length of the calibration
+# segments (App. C.2), is taken for it.
 LIFETIME_HORIZON = 2048
 
 
