@@ -15,7 +15,7 @@
  * What each part follows (sections, equations and tables of the STEPQuant paper):
  *   recurrence        §2.1, the gated Delta rule and its affine form S_t = A_t S_{t-1} + B_t;
  *                     readout y_t = S_t^T q_t taken before requantisation (Table C2, step 3).
- *   gate D_t          scalar per head (GDN) or diagonal over key rows (KDA), §2.1 / App. C.1.
+ *   gate D_t          scalar per head (GDN) or diagonal over key rows (KDA), §2.1, §6.1 / App. C.1.
  *   quantiser         §2.2, Q_{b,s}(x) = s clip(round(x/s), -q_b, q_b), q_b = 2^(b-1) - 1.
  *   code normalisation App. C.1: stored integer q, reconstruction z = 2^(8-b) q.
  *   dual-axis scales  §4.3, X_hat_ij = r_i c_j z_ij; row factor m_i = mean_j |X_ij| (§4.3
