@@ -400,7 +400,7 @@ def calibrate(alloc, candidates, nominal_bits, S0, calib, n_pivots=0, horizon=LI
     the stream's gates (App. A.3): a head unit averages the log gate over its key channels, a
     key-row unit under a head gate takes its head's value; ``horizon`` is the H of that sum.
 
-    n_pivots > 0 keeps that many units in FP16 (width 16, App. C.2, Table B1):
+    n_pivots > 0 keeps that many units in FP16 (width 16, App. C.2, Table C1):
       key rows: ranked by the lifetime-weighted reduction of error from the integer format at
         the nominal width to FP16, L_u (d_u(b_nominal) - d_u(16)); with the pivots fixed the
         candidate distortions of the other rows are measured again with the pivots left out
