@@ -192,6 +192,32 @@ def test_rowwise_absmax_int8_is_the_8bit_contract_with_unit_columns():
     assert np.abs(textbook - codes8).max() <= 1 and (textbook != codes8).mean() < 1e-3
 
 
+@pytest.mark.parametrize("b", [2, 4, 6, 8])
+def test_quantiser_rounds_exact_half_steps_to_even(b):
+    """With unit steps (r = 2^-(8-b), so that r 2^(8-b) = 1, and c = 1) the quantiser reduces to
+    clip(rint(x), -q_b, q_b) with NumPy's rint (nearest, ties to even, R3), exact half steps
+    included, and clips beyond the end points."""
+    qb = _qmax(b)
+    vals = np.concatenate([np.arange(-qb, qb) + 0.5, [0.25, -0.75, qb + 0.5, -qb - 3.0]])
+    X = np.resize(vals, 2 * 64).reshape(2, 64).astype(np.float32)
+    bits = np.full(2, b, dtype=np.uint8)
+    r = np.full(2, np.float16(2.0 ** -(8 - b)).view(np.uint16), dtype=np.uint16)
+    c = np.full(64, np.float16(1.0).view(np.uint16), dtype=np.uint16)
+    codes = oracle.quantise_tile(X, bits, r, c)
+    np.testing.assert_array_equal(codes, np.clip(np.rint(X.astype(np.float64)), -qb, qb))
+
+
+def test_int8_baseline_rounds_exact_half_steps_to_even():
+    """Rows whose absolute maximum is 127 get the scale s = 1 exactly, so the rowwise-absmax INT8
+    baseline reduces to clip(rint(x), -127, 127): exact half steps go to the even neighbour."""
+    vals = np.arange(-126, 126) + 0.5
+    X = np.resize(vals, 4 * 64).reshape(4, 64).astype(np.float32)
+    X[:, 0] = 127.0
+    codes, s = oracle.int8_quantise_tile(X)
+    assert (s == np.float16(1.0).view(np.uint16)).all()
+    np.testing.assert_array_equal(codes, np.clip(np.rint(X.astype(np.float64)), -127, 127))
+
+
 def test_scale_rounding_matches_numpy_binary16():
     rng = np.random.default_rng(2)
     xs = np.concatenate([np.exp(rng.uniform(np.log(2.0 ** -14), np.log(65504.0), 20000)),

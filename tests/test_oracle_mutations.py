@@ -74,6 +74,10 @@ MUTANTS = [
        ("float n = rintf(t);", "float n = truncf(t);")),
     _m("negative codes clamped at -2^(b-1)", C_SRC,
        ("if (n < -qb) n = -qb;", "if (n < -qb - 1.0f) n = -qb - 1.0f;")),
+    _m("quantiser rounds ties away from zero", C_SRC,
+       ("float n = rintf(t);", "float n = roundf(t);")),
+    _m("INT8 baseline rounds ties away from zero", C_SRC,
+       ("float n = rintf(X[i * dv + j] * is);", "float n = roundf(X[i * dv + j] * is);")),
     _m("codebook step z dropped in the dequantiser", C_SRC,
        ("return rc * (float)(q * znorm_of(b));", "return rc * (float)q;")),
     # packed layout
@@ -98,6 +102,11 @@ MUTANTS = [
     # key-row-aware dual-axis fit (§4.3, App. C.1)
     _m("row factor is a sum, not a mean", C_SRC,
        ("        m /= dv;\n", "")),
+    _m("row factor takes the row maximum", C_SRC,
+       ("for (int j = 0; j < dv; ++j) m += fabs((double)X[i * dv + j]);",
+        "for (int j = 0; j < dv; ++j) m = fmax(m, fabs((double)X[i * dv + j]));")),
+    _m("pivot rows join the shared column init as 8-bit rows", C_SRC,
+       ("if (is_pivot(b)) continue;\n            float a = 1.0f", "if (is_pivot(b)) b = 8;\n            float a = 1.0f")),
     _m("row impact multiplies the row factor", C_SRC,
        ("r_out[i] = orc_scale_to_half(m / (double)w[i]);", "r_out[i] = orc_scale_to_half(m * (double)w[i]);")),
     _m("no-clip column init ignores the codebook step", C_SRC,
@@ -120,6 +129,9 @@ MUTANTS = [
         "orc_pack_tile(dk, dv, S32, bits, r_in, c_in, packed_out);")),
     _m("prefill chunk never advances its state", C_SRC,
        ("memcpy(t.S, t.X, sizeof(double) * dk * dv);            /* full precision in between */", "")),
+    _m("prefill readouts all written to the first token's slot", C_SRC,
+       ("o[tc * dv + j] = (float)t.o[j];\n            memcpy(t.S, t.X, sizeof(double) * dk * dv);            /* full precision in between */",
+        "o[tl * dv + j] = (float)t.o[j];\n            memcpy(t.S, t.X, sizeof(double) * dk * dv);            /* full precision in between */")),
     _m("prefill boundary fit with the first head's impact", C_SRC,
        ("orc_fit_tile(dk, dv, S32, w + (int64_t)h * dk, bh,", "orc_fit_tile(dk, dv, S32, w, bh,")),
     # per-window 8-bit state and the INT8 baseline (§5.1)
@@ -138,6 +150,9 @@ MUTANTS = [
     # calibration statistics (App. A.3, B.3)
     _m("row impact with the Delta feedback sign flipped", C_SRC,
        ("(orc_bf16_to_float(qq[i]) - (double)beta[tile]", "(orc_bf16_to_float(qq[i]) + (double)beta[tile]")),
+    _m("row impact feedback with q.q in place of k.q", C_SRC,
+       ("kq += (double)orc_bf16_to_float(kk[i]) * orc_bf16_to_float(qq[i]);",
+        "kq += (double)orc_bf16_to_float(qq[i]) * orc_bf16_to_float(qq[i]);")),
     _m("row impact without the gate", C_SRC,
        ("double g = d * (orc_bf16_to_float(qq[i])", "double g = (orc_bf16_to_float(qq[i])")),
     _m("row impact fourth root instead of eighth", C_SRC,

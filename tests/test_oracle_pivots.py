@@ -2,6 +2,7 @@
 16 keeps a key row's values in binary16, stored after the integer rows of the tile, outside the
 shared column fit; pivot selection and the (16 - 8) budget accounting of App. D."""
 import numpy as np
+import pytest
 
 import oracle
 from recurrent_state_quantization_gated_b200 import synth
@@ -34,10 +35,15 @@ def _tile(d=64, seed=0, pivots=(0, 5, 17)):
     return X, bits, w
 
 
-def test_fit_ignores_pivot_rows():
+@pytest.mark.parametrize("spike", [False, True])
+def test_fit_ignores_pivot_rows(spike):
     """The column scales of a tile with pivot rows are those of the tile without them; the row
-    factors of the other rows are unchanged; a pivot row's factor is the usual R1 value."""
+    factors of the other rows are unchanged; a pivot row's factor is the usual R1 value. With
+    `spike`, a pivot row holds one entry 50 times its row's largest (the kind of outlier a pivot
+    keeps); were that row in the shared column fit, it would set its column's scale."""
     X, bits, w = _tile()
+    if spike:
+        X[0, 7] = 50.0 * np.abs(X[0]).max()
     keep = bits != 16
     r, c = oracle.fit_tile(X, w, bits)
     r2, c2 = oracle.fit_tile(np.ascontiguousarray(X[keep]), np.ascontiguousarray(w[keep]), bits[keep])
