@@ -24,6 +24,18 @@ def test_row_factor_is_mean_abs_over_impact(d):
     np.testing.assert_array_equal(r, expect.view(np.uint16))
 
 
+def test_zero_row_factor_is_the_floor_over_its_impact():
+    """R1 floors the row mean at 2^-14 before dividing by the impact factor: an all-zero row with
+    w_i = 1/2 gets r_i = 2^-13, and one with w_i = 2 gets 2^-15, clamped back up to 2^-14."""
+    S, bits, w = _tile(64, 4)
+    S[3] = 0.0
+    S[4] = 0.0
+    w[3], w[4] = 0.5, 2.0
+    r, _ = oracle.fit_tile(S, w, bits)
+    assert r[3] == np.float16(2.0 ** -13).view(np.uint16)
+    assert r[4] == np.float16(2.0 ** -14).view(np.uint16)
+
+
 def test_column_init_clips_nothing_and_is_tight():
     S, bits, w = _tile(128, 5)
     r, c, det = oracle.fit_tile(S, w, bits, detail=True)

@@ -67,6 +67,10 @@ MUTANTS = [
        ("acc += q[i] * X[i * dv + j];", "acc += k[i] * X[i * dv + j];")),
     _m("readout through a transposed state", C_SRC,
        ("acc += q[i] * X[i * dv + j];", "acc += q[i] * X[j * dk + i];")),
+    _m("gate applied after the update instead of before it", C_SRC,
+       ("X[i * dv + j] = gate[i] * S[i * dv + j];", "X[i * dv + j] = S[i * dv + j];"),
+       ("X[i * dv + j] += k[i] * (beta * (v[j] - p[j]));",
+        "X[i * dv + j] = gate[i] * (X[i * dv + j] + k[i] * (beta * (v[j] - p[j])));")),
     _m("channel gate replaced by its first entry", C_SRC,
        ("t->g[i] = gate_per_channel ? (double)gate[i] : (double)gate[0];", "t->g[i] = (double)gate[0];")),
     # quantiser and dequantiser (§2.2)
@@ -88,6 +92,13 @@ MUTANTS = [
         "uint8_t* lo_plane = row + dv / 4;\n        uint8_t* hi_plane = row;"),
        ("get_bits(row, field_bit(j, 4), 4) | (get_bits(row + dv / 2, field_bit(j, 2), 2) << 4)",
         "get_bits(row + dv / 4, field_bit(j, 4), 4) | (get_bits(row, field_bit(j, 2), 2) << 4)")),
+    _m("packed codes lose their sign bit", C_SRC,
+       ("(unsigned)q[j] & ((1u << b) - 1u)", "(unsigned)q[j] & ((1u << (b - 1)) - 1u)")),
+    _m("6-bit high plane joined one bit low", C_SRC,
+       ("field_bit(j, 2), 2) << 4)", "field_bit(j, 2), 2) << 3)")),
+    _m("rows laid out in reverse key order", C_SRC,
+       ("        for (int i = 0; i < dk; ++i)\n            if (is_pivot(bits[i]) == pass) {",
+        "        for (int i = dk - 1; i >= 0; --i)\n            if (is_pivot(bits[i]) == pass) {")),
     _m("pivot rows stored before the integer rows", C_SRC,
        ("if (is_pivot(bits[i]) == pass) {", "if (is_pivot(bits[i]) != pass) {")),
     # binary16 conversions
@@ -107,6 +118,10 @@ MUTANTS = [
         "for (int j = 0; j < dv; ++j) m = fmax(m, fabs((double)X[i * dv + j]));")),
     _m("pivot rows join the shared column init as 8-bit rows", C_SRC,
        ("if (is_pivot(b)) continue;\n            float a = 1.0f", "if (is_pivot(b)) b = 8;\n            float a = 1.0f")),
+    _m("row factor floor dropped", C_SRC,
+       ("        if (m < HALF_MIN_NORMAL) m = HALF_MIN_NORMAL;\n", "")),
+    _m("column init floor dropped", C_SRC,
+       ("c0[j] = mx < (float)HALF_MIN_NORMAL ? (float)HALF_MIN_NORMAL : mx;", "c0[j] = mx;")),
     _m("row impact multiplies the row factor", C_SRC,
        ("r_out[i] = orc_scale_to_half(m / (double)w[i]);", "r_out[i] = orc_scale_to_half(m * (double)w[i]);")),
     _m("no-clip column init ignores the codebook step", C_SRC,
