@@ -101,6 +101,9 @@ MUTANTS = [
         "        for (int i = dk - 1; i >= 0; --i)\n            if (is_pivot(bits[i]) == pass) {")),
     _m("pivot rows stored before the integer rows", C_SRC,
        ("if (is_pivot(bits[i]) == pass) {", "if (is_pivot(bits[i]) != pass) {")),
+    _m("state unpack ignores the head offset", C_SRC,
+       ("orc_unpack_tile(dk, dv, packed + b * bytes_per_seq + head_off[h], bits",
+        "orc_unpack_tile(dk, dv, packed + b * bytes_per_seq, bits")),
     # binary16 conversions
     _m("scales truncated instead of rounded to nearest even", C_SRC,
        ("double sig = nearbyint(ldexp(m, 11)); /* 11 significant bits, ties to even    */",
@@ -139,6 +142,8 @@ MUTANTS = [
        ("    for (int e = 0; e < dk * dv; ++e) S32[e] = (float)t.X[e];\n"
         "    orc_fit_tile(dk, dv, S32, w, bits, r_out, c_out);",
         "    orc_fit_tile(dk, dv, S32, w, bits, r_out, c_out);")),
+    _m("decode batch fits every head with the first head's impact", C_SRC,
+       ("gate_per_channel, bits + (int64_t)h * dk, w + (int64_t)h * dk,", "gate_per_channel, bits + (int64_t)h * dk, w,")),
     _m("decode packs with the previous scales", C_SRC,
        ("orc_pack_tile(dk, dv, S32, bits, r_out, c_out, packed_out);",
         "orc_pack_tile(dk, dv, S32, bits, r_in, c_in, packed_out);")),
@@ -160,6 +165,8 @@ MUTANTS = [
         "                for (int j = 0; j < dv; ++j)\n"
         "                    t.S[i * dv + j] = (double)(orc_half_to_float(s_out[tl * dk + i]) *\n"
         "                                               (float)codes_out[(tl * dk + i) * dv + j]);")),
+    _m("window reads the first tile's scales for every tile", C_SRC,
+       ("float si = orc_half_to_float(s_in[tl * dk + i]);", "float si = orc_half_to_float(s_in[i]);")),
     _m("INT8 scale divides by 128", C_SRC,
        ("s[i] = orc_scale_to_half((double)mx / 127.0);", "s[i] = orc_scale_to_half((double)mx / 128.0);")),
     # calibration statistics (App. A.3, B.3)
@@ -176,6 +183,8 @@ MUTANTS = [
        ("(float)(mean > 0.0 ? oh[i] / mean : 1.0);", "(float)oh[i];")),
     _m("row impact floor dropped", C_SRC,
        ("if (oh[i] < 1e-12 * mx) oh[i] = 1e-12 * mx;", "")),
+    _m("distortion fits every head with the first head's impact", C_SRC,
+       ("const float* wh = w + (int64_t)h * dk;", "const float* wh = w;")),
     _m("head distortion weights not squared", C_SRC,
        ("dh += (double)wh[i] * (double)wh[i] * row;", "dh += (double)wh[i] * row;")),
     _m("row distortion not divided by the row length", C_SRC,
