@@ -204,6 +204,12 @@ MUTANTS = [
     _m("repair takes the first single move, not the cheapest", C_SRC,
        ("if (!found || dj < bdj) { found = 1; bdj = dj; bu = u; bku = kk; bv = -1; }",
         "if (!found) { found = 1; bdj = dj; bu = u; bku = kk; bv = -1; }")),
+    _m("decode wrapper passes channel gates as head gates", PY_SRC,
+       ("gpc = int(gate.ndim == 3)", "gpc = 0")),
+    _m("prefill wrapper passes channel gates as head gates", PY_SRC,
+       ("gpc = int(gate.ndim == 4)\n    head_off, bps = layout(bits, dv)", "gpc = 0\n    head_off, bps = layout(bits, dv)")),
+    _m("row impact wrapper passes channel gates as head gates", PY_SRC,
+       ("int(gate.ndim == 4), _p(q)", "0, _p(q)")),
     _m("lifetime sums the retention, not the squared error", PY_SRC,
        ("total += np.exp(2.0 * j * ell)", "total += np.exp(j * ell)")),
     _m("lifetime sum starts one step late", PY_SRC,
