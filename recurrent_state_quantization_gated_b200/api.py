@@ -97,7 +97,7 @@ def stepq_fit_scales(S, w, bits, r=None, c=None):
     B, H, d, _ = S.shape
     r = torch.empty((B, H, d), dtype=torch.float16, device=S.device) if r is None else r
     c = torch.empty((B, H, d), dtype=torch.float16, device=S.device) if c is None else c
-    _sizes(w=(w, H * d), bits=(bits, H * d), r=(r, B * H * d), c=(c, B * H * d))
+    _sizes(S=(S, B * H * d * d), w=(w, H * d), bits=(bits, H * d), r=(r, B * H * d), c=(c, B * H * d))
     call("stepq_fit_scales", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
          _ptr(bits, torch.uint8, "bits"), _ptr(r, torch.float16, "r"), _ptr(c, torch.float16, "c"), _stream())
     return r, c
@@ -106,7 +106,7 @@ def stepq_fit_scales(S, w, bits, r=None, c=None):
 def stepq_pack_state(S, bits, head_off, bytes_per_seq, r, c, packed=None):
     B, H, d, _ = S.shape
     packed = torch.empty(B * bytes_per_seq, dtype=torch.uint8, device=S.device) if packed is None else packed
-    _sizes(bits=(bits, H * d), head_off=(head_off, H), r=(r, B * H * d), c=(c, B * H * d),
+    _sizes(S=(S, B * H * d * d), bits=(bits, H * d), head_off=(head_off, H), r=(r, B * H * d), c=(c, B * H * d),
            packed=(packed, B * int(bytes_per_seq)))
     call("stepq_pack_state", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(bits, torch.uint8, "bits"),
          _ptr(head_off, torch.int64, "head_off"), ctypes.c_int64(int(bytes_per_seq)),
@@ -241,7 +241,7 @@ def stepq_int8_quantize_state(S, codes=None, s=None):
     B, H, d, _ = S.shape
     codes = torch.empty((B, H, d, d), dtype=torch.int8, device=S.device) if codes is None else codes
     s = torch.empty((B, H, d), dtype=torch.float16, device=S.device) if s is None else s
-    _sizes(codes=(codes, B * H * d * d), s=(s, B * H * d))
+    _sizes(S=(S, B * H * d * d), codes=(codes, B * H * d * d), s=(s, B * H * d))
     call("stepq_int8_quantize_state", _dims(B, H, d), _ptr(S, torch.float32, "S"),
          _ptr(codes, torch.int8, "codes"), _ptr(s, torch.float16, "s"), _stream())
     return codes, s
@@ -301,7 +301,7 @@ def stepq_calib_distortion(S, w, b, d_row=None, d_head=None, scratch=None):
     d_row = torch.empty((H, d), dtype=torch.float64, device=dev) if d_row is None else d_row
     d_head = torch.empty((H,), dtype=torch.float64, device=dev) if d_head is None else d_head
     scratch = torch.empty((B, H, d), dtype=torch.float64, device=dev) if scratch is None else scratch
-    _sizes(w=(w, H * d), d_row=(d_row, H * d), d_head=(d_head, H), scratch=(scratch, B * H * d))
+    _sizes(S=(S, B * H * d * d), w=(w, H * d), d_row=(d_row, H * d), d_head=(d_head, H), scratch=(scratch, B * H * d))
     call("stepq_calib_distortion", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
          ctypes.c_int(int(b)), _ptr(d_row, torch.float64, "d_row"), _ptr(d_head, torch.float64, "d_head"),
          _ptr(scratch, torch.float64, "scratch"), _stream())
@@ -316,7 +316,8 @@ def stepq_calib_distortion_bits(S, w, bits, d_row=None, d_head=None, scratch=Non
     d_row = torch.empty((H, d), dtype=torch.float64, device=dev) if d_row is None else d_row
     d_head = torch.empty((H,), dtype=torch.float64, device=dev) if d_head is None else d_head
     scratch = torch.empty((B, H, d), dtype=torch.float64, device=dev) if scratch is None else scratch
-    _sizes(w=(w, H * d), bits=(bits, H * d), d_row=(d_row, H * d), d_head=(d_head, H), scratch=(scratch, B * H * d))
+    _sizes(S=(S, B * H * d * d), w=(w, H * d), bits=(bits, H * d), d_row=(d_row, H * d), d_head=(d_head, H),
+           scratch=(scratch, B * H * d))
     call("stepq_calib_distortion_bits", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
          _ptr(bits, torch.uint8, "bits"), _ptr(d_row, torch.float64, "d_row"), _ptr(d_head, torch.float64, "d_head"),
          _ptr(scratch, torch.float64, "scratch"), _stream())
@@ -330,7 +331,7 @@ def stepq_calib_distortion_static(S, w, b, d_row=None, d_head=None):
     dev = S.device
     d_row = torch.empty((H, d), dtype=torch.float64, device=dev) if d_row is None else d_row
     d_head = torch.empty((H,), dtype=torch.float64, device=dev) if d_head is None else d_head
-    _sizes(w=(w, H * d), d_row=(d_row, H * d), d_head=(d_head, H))
+    _sizes(S=(S, B * H * d * d), w=(w, H * d), d_row=(d_row, H * d), d_head=(d_head, H))
     call("stepq_calib_distortion_static", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(w, torch.float32, "w"),
          ctypes.c_int(int(b)), _ptr(d_row, torch.float64, "d_row"), _ptr(d_head, torch.float64, "d_head"), _stream())
     return d_row, d_head

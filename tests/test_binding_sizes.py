@@ -73,8 +73,9 @@ CASES = {
                                              d_head=z(f64, H))),
 }
 
-# the tensor whose shape gives the call its dimensions is not checked against itself
-SHAPE_SOURCE = {"q", "S", "r"}
+# the tensor whose first axes give the call its dimensions is not checked against itself (a
+# state S [B][H][d][d] is: its last axis must match)
+SHAPE_SOURCE = {"q", "r"}
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
