@@ -3,16 +3,20 @@
 
 One step = one decode token for every (sequence, head) tile of the workload: unpack and
 dequantise the packed recurrent state, gated Delta update, readout, refit of the dual-axis
-scales and repack -- one launch of the fused kernel. The default workload is the Qwen-style
-Gated DeltaNet layer decode (B=64 sequences, H=32 heads, d_k=d_v=128, 6-bit nominal budget,
-head-level bits from the lifetime-aware DP allocation), on seeded synthetic data.
+scales and repack -- one launch of the fused kernel. The default workload is the largest
+single-GPU decode configuration: the high-concurrency 4-bit layer (B=1024 sequences, H=16 heads,
+d_k=d_v=128, per-key-row widths from {2, 4, 8} averaging 4 bits, lifetime-aware Lagrangian
+allocation), on seeded synthetic data. The FP32-state and uniform rowwise-INT8 comparison kernels
+are timed in the same run on identical inputs; the long-rollout workload also reports the output
+drift of the quantized state against the FP32 state over its T steps.
 
 Timing: R state replicas (independent layers of the same shape) are stepped round-robin so
 that more than the 126 MB L2 is touched between two uses of a replica; one round of R
 launches is captured in a CUDA graph and replayed; CUDA events on the launching stream bracket
-the K timed steps, after W untimed warm-up steps, with a barrier + synchronize on both sides.
-Under torchrun every rank runs its own replicas (weak scaling, no collective on the data path)
-and the time is the maximum over ranks.
+the K timed steps, after W untimed warm-up steps, with a barrier + synchronize on both sides;
+the K steps are timed five times and the median is reported. Under torchrun every rank runs its
+own replicas (weak scaling, no collective on the data path) and the time is the maximum over
+ranks; ``--gpus N`` without torchrun's environment starts N ranks itself.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -45,7 +49,14 @@ def parse():
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=1, help="synthetic workload index (1 = Qwen-style GDN)")
+    ap.add_argument("--workload", type=int, default=3,
+                    help="synthetic workload index (0 tiny, 1 GDN 64x32, 2 KDA 256x32, 3 GDN 4-bit 1024x16, "
+                         "4 long rollout 128x32)")
+    ap.add_argument("--repeats", type=int, default=5, help="timed repetitions of the K steps (median reported)")
+    ap.add_argument("--no-comparisons", action="store_true",
+                    help="leave out the FP32-state and INT8 comparison kernels")
+    ap.add_argument("--drift-steps", type=int, default=0,
+                    help="rollout steps of the drift figure (0: the workload's T; long-rollout workload only)")
     ap.add_argument("--replicas", type=int, default=0, help="state replicas cycled (0 = enough to exceed L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -71,40 +82,34 @@ def kernel_revision() -> str:
     return hashlib.sha256(data).hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes (read + write) per launch from the committed ncu capture of the fused kernel,
-    or None when the kernel source has changed since that capture."""
-    p = ROOT / "profiles" / "decode_kernel_gdn_b64_h32_d128.md"
+def _profile(workload_name: str):
+    """Figures of the committed ncu summary of the fused kernel on this workload
+    (profiles/decode_kernel_<workload>.md): {"traffic": DRAM bytes read + written per launch,
+    "instr_per_element": lane instructions per state element}, each None when absent or when
+    the kernel's source has changed since the capture (its revision line no longer matches)."""
+    out = {"traffic": None, "instr_per_element": None}
+    p = ROOT / "profiles" / f"decode_kernel_{workload_name}.md"
     if not p.exists():
-        return None
-    text = p.read_text()
-    rev = read = write = None
-    for line in text.splitlines():
-        if "Kernel source revision" in line:
-            rev = line.rsplit(":", 1)[-1].strip()
-        if line.startswith("| dram__bytes_read.sum"):
-            read = float(line.split("|")[2].split()[0]) * 1e6
-        if line.startswith("| dram__bytes_write.sum"):
-            write = float(line.split("|")[2].split()[0]) * 1e6
-    if rev != kernel_revision() or read is None or write is None:
-        return None
-    return read + write
-
-
-def profiled_instructions():
-    """Lane instructions per state element of the fused kernel, from the committed ncu capture
-    (warp instructions x 32 / elements), or None when the kernel has changed since."""
-    p = ROOT / "profiles" / "decode_kernel_gdn_b64_h32_d128.md"
-    if not p.exists():
-        return None
-    rev = per_elem = None
+        return out
+    rev = read = write = per_elem = None
     for line in p.read_text().splitlines():
         if "Kernel source revision" in line:
             rev = line.rsplit(":", 1)[-1].strip()
-        if line.startswith("| smsp__inst_executed.sum"):
-            cell = line.split("|")[2]
-            per_elem = float(cell.split("(")[1].split()[0])
-    return per_elem if rev == kernel_revision() else None
+        cells = [c.strip() for c in line.split("|")]
+        if len(cells) < 3:
+            continue
+        if cells[1].startswith("dram__bytes_read.sum per launch"):
+            read = float(cells[2].split()[0].replace(",", ""))
+        if cells[1].startswith("dram__bytes_write.sum per launch"):
+            write = float(cells[2].split()[0].replace(",", ""))
+        if cells[1].startswith("lane instructions per element"):
+            per_elem = float(cells[2].split()[0])
+    if rev != kernel_revision():
+        return out
+    if read is not None and write is not None:
+        out["traffic"] = read + write
+    out["instr_per_element"] = per_elem
+    return out
 
 
 def peaks():
@@ -115,10 +120,9 @@ def peaks():
     return 6650.0, "fallback"
 
 
-def alu_roofline(elements_per_s, clocks):
+def alu_roofline(elements_per_s, clocks, per_elem):
     """The issue-rate roofline beside the HBM one: lane instructions per second against
     148 SMs x 4 schedulers x 32 lanes x the SM clock seen during the timed region."""
-    per_elem = profiled_instructions()
     mhz = (clocks or {}).get("sm_mhz") or 1965.0
     peak = 148 * 4 * 32 * mhz * 1e6
     if per_elem is None:
@@ -283,15 +287,16 @@ def run_reference(args, wl, budget_s: float = 90.0):
     return dict(value=value, ms_per_step=1e3 * total / len(times), cores=cores, sample=sample, bits=bits)
 
 
-def cpu_baseline(wl, bits, seconds, threads=0):
+def cpu_baseline(wl, bits, w, seconds, threads=0):
     """The oracle as it stands, timed on the host cores over a bounded sample of the workload:
-    16 sequences x all heads per step, inputs drawn before the timed loop."""
+    16 sequences x all heads per step, the calibrated bit map and row weights, inputs drawn
+    before the timed loop."""
     import oracle
     from recurrent_state_quantization_gated_b200 import synth
     cores = threads if threads > 0 else len(os.sched_getaffinity(0))
     seqs = list(range(min(wl.B, 16)))
     S0 = synth.initial_state(wl, seqs)
-    w = np.ones((wl.H, wl.d), dtype=np.float32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
     r, c = oracle.fit_scales(S0, w, bits, nthreads=cores)
     packed = oracle.pack_state(S0, bits, r, c, nthreads=cores)
     toks = [synth.tokens(wl, t, seqs=seqs) for t in range(8)]
@@ -308,8 +313,69 @@ def cpu_baseline(wl, bits, seconds, threads=0):
                       f"{'OpenMP over tiles' if cores > 1 else 'one thread'}, {el:.1f} s"}
 
 
+def relaunch(args) -> int:
+    """``--gpus N`` (N > 1) outside torchrun: start N ranks of this script on this node (one
+    process per GPU), with the same arguments; rank 0 prints the line."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), str(Path(__file__).resolve()), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def _drift_tokens(index_t):
+    """Packed inputs of step t of workload `index` (process-pool worker of the drift rollout)."""
+    from recurrent_state_quantization_gated_b200 import runtime, synth
+    index, t = index_t
+    return runtime.pack_tokens(synth.tokens(synth.workload(index), t))
+
+
+def timed_rounds(launch_round, round_len, warmup, steps, repeats, stream, world, barrier, clock=None):
+    """Captures one round of launches (`launch_round()`, `round_len` steps) in a CUDA graph,
+    replays ceil(warmup / round_len) rounds untimed, then times ceil(steps / round_len) rounds
+    `repeats` times with CUDA events on the stream (barrier + synchronize around each), the
+    slowest rank's time each. Returns (K steps per repetition, warm-up steps, [ms per repetition])."""
+    import torch
+    with torch.cuda.stream(stream):
+        launch_round()                       # outside capture first (kernel attributes, occupancy)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        launch_round()
+    rounds_warm = max(1, -(-warmup // round_len))
+    rounds = max(1, -(-steps // round_len))
+    with torch.cuda.stream(stream):
+        for _ in range(rounds_warm):
+            graph.replay()
+    stream.synchronize()
+    times = []
+    if clock is not None:          # clocks sampled over every timed repetition
+        clock.__enter__()
+    try:
+        for _ in range(repeats):
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            with torch.cuda.stream(stream):
+                ev0.record(stream)
+                for _ in range(rounds):
+                    graph.replay()
+                ev1.record(stream)
+            stream.synchronize()
+            barrier()
+            times.append(max_over_ranks(ev0.elapsed_time(ev1), world, "cuda"))
+    finally:
+        if clock is not None:
+            clock.__exit__(None, None, None)
+    del graph
+    return rounds * round_len, rounds_warm * round_len, times
+
+
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch(args)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -320,10 +386,10 @@ def main():
         if rank != 0:
             return 0
         ref = run_reference(args, wl)
-        line = {"metric": METRIC, "value": ref["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        line = {"metric": METRIC, "value": ref["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ref["ms_per_step"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-                "config": workload_config(wl, ref["bits"], "quant", args.gpus),
+                "config": workload_config(wl, ref["bits"], "quant", world),
                 "cpu_baseline": {"value": ref["value"], "unit": UNIT, "cores": ref["cores"], "kind": "oracle",
                                  "sample": ref["sample"]},
                 "e2e": {"value": ref["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -368,9 +434,11 @@ def main():
         raise SystemExit("--kernel leap takes scalar gates (workloads 0, 1, 3, 4)")
 
     # Replicas: enough independent states that > 2x L2 is touched between reuses.
+    def replicas_for(per_launch):
+        return min(64, args.replicas or max(2, int(np.ceil(2 * L2_BYTES / per_launch))))
+
     per_rep = bytes_launch
-    R = args.replicas or max(2, int(np.ceil(2 * L2_BYTES / per_rep)))
-    R = min(R, 64)
+    R = replicas_for(per_rep)
     reps, toks, outs, tok_bufs = [], [], [], []
     side = torch.cuda.Stream() if args.kernel == "split" else None
     x_ws = torch.empty((wl.B, wl.H, wl.d, wl.d), dtype=torch.float32, device="cuda") if side is not None else None
@@ -400,7 +468,6 @@ def main():
             toks.append(runtime.token_views(tok_bufs[-1], host))
         oshape = (args.chunk, wl.B, wl.H, wl.d) if args.kernel == "prefill" else (wl.B, wl.H, wl.d)
         outs.append(torch.empty(oshape, dtype=torch.float32, device="cuda"))
-    del S0
     torch.cuda.synchronize()
 
     def launch(i, refit=True):
@@ -431,42 +498,62 @@ def main():
             api.stepq_decode_step_int8(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], st["codes"], st["s"],
                                        st["codes"], st["s"], o)
 
-    stream = torch.cuda.Stream()
-    with torch.cuda.stream(stream):
-        for _ in range(LW):
-            for i in range(R):      # first launches outside capture (kernel attributes, occupancy)
-                launch(i)
-    stream.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
+    def one_round():
         for _ in range(LW):
             for i in range(R):
                 launch(i)
-    rounds_warm = max(1, -(-args.warmup // (R * LW)))
-    rounds = max(1, -(-args.steps // (R * LW)))
-    K = rounds * R * LW
-    with torch.cuda.stream(stream):
-        for _ in range(rounds_warm):
-            graph.replay()
-    stream.synchronize()
-    flags = api.stepq_read_device_flags()
 
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    with ClockSampler(local_rank) as clk:
-        with torch.cuda.stream(stream):
-            ev0.record(stream)
-            for _ in range(rounds):
-                graph.replay()
-            ev1.record(stream)
-        stream.synchronize()
-        barrier()
-    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world, "cuda")
+    stream = torch.cuda.Stream()
+    clk = ClockSampler(local_rank)
+    K, warm, times = timed_rounds(one_round, R * LW, args.warmup, args.steps, args.repeats, stream, world, barrier,
+                                  clock=clk)
+    flags = api.stepq_read_device_flags()
+    elapsed_ms = statistics.median(times)
     ms_per_step = elapsed_ms / K
     upd = tiles * (args.chunk if args.kernel == "prefill" else 1)   # tile updates per launch
     value = job_throughput(world, upd, K, elapsed_ms)
     achieved_gbs = bytes_launch / (ms_per_step * 1e-3) / 1e9
     peak, peak_kind = peaks()
+
+    # ---- comparison state formats on identical inputs (same initial state, same tokens) ---
+    comparisons = None
+    if args.kernel == "quant" and not args.no_comparisons:
+        comparisons = {}
+        quant_bytes = bytes_launch
+        for kind in ("fp32", "int8"):
+            b_k = algorithmic_bytes(layout.bytes_per_seq, wl.B, wl.H, wl.d, wl.gate_per_channel, kind)
+            Rk = replicas_for(b_k)
+            sts = []
+            for i in range(Rk):
+                if kind == "fp32":
+                    sts.append(dict(S=S0.clone()))
+                else:
+                    cds, s_ = api.stepq_int8_quantize_state(S0)
+                    sts.append(dict(codes=cds, s=s_))
+            o_k = torch.empty((wl.B, wl.H, wl.d), dtype=torch.float32, device="cuda")
+
+            def round_k(kind=kind, sts=sts, o_k=o_k, Rk=Rk):
+                for i in range(Rk):
+                    tk = toks[i % R]
+                    if kind == "fp32":
+                        api.stepq_decode_step_fp32(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], sts[i]["S"],
+                                                   sts[i]["S"], o_k)
+                    else:
+                        api.stepq_decode_step_int8(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"],
+                                                   sts[i]["codes"], sts[i]["s"], sts[i]["codes"], sts[i]["s"], o_k)
+
+            Kk, _, tk_times = timed_rounds(round_k, Rk, args.warmup, max(Rk, args.steps // 4), args.repeats, stream,
+                                           world, barrier)
+            ms_k = statistics.median(tk_times) / Kk
+            gbs_k = b_k / (ms_k * 1e-3) / 1e9
+            comparisons[kind] = {
+                "value": job_throughput(world, tiles, Kk, statistics.median(tk_times)), "unit": UNIT,
+                "ms_per_step": ms_k, "achieved_gbs": gbs_k, "frac": gbs_k / peak, "bytes_per_launch": b_k,
+                "replicas": Rk, "steps": Kk,
+                "quant_speedup": ms_k / ms_per_step, "quant_bytes_ratio": b_k / quant_bytes,
+                "format": "FP32 state" if kind == "fp32" else "rowwise-absmax INT8 codes + FP16 row scales"}
+            del sts
+        torch.cuda.synchronize()
 
     split_info = None
     if args.kernel == "split":
@@ -488,6 +575,40 @@ def main():
                       "fused_bytes_per_step": algorithmic_bytes(layout.bytes_per_seq, wl.B, wl.H, wl.d,
                                                                 wl.gate_per_channel, "quant")}
 
+    # ---- output drift of the quantized state against the FP32 state (long rollout) ---------
+    drift = None
+    if args.kernel == "quant" and wl.name.startswith("drift"):
+        T = args.drift_steps or wl.T
+        import multiprocessing as mp
+        st_q = dict(packed=base.packed.clone(), r=base.r.clone(), c=base.c.clone())
+        S_f = S0.clone()
+        o_q = torch.empty((wl.B, wl.H, wl.d), dtype=torch.float32, device="cuda")
+        o_f = torch.empty_like(o_q)
+        num = torch.empty(T, dtype=torch.float64, device="cuda")
+        den = torch.empty(T, dtype=torch.float64, device="cuda")
+        tb = torch.empty_like(tok_bufs[0])
+        host0 = synth.tokens(wl, 0)
+        tv = runtime.token_views(tb, host0)
+        cores = len(os.sched_getaffinity(0))
+        with mp.get_context("spawn").Pool(max(1, min(16, cores))) as pool:
+            for t, packed_tok in enumerate(pool.imap(_drift_tokens, [(wl.index, t) for t in range(T)], chunksize=8)):
+                tb.copy_(torch.from_numpy(packed_tok))
+                api.stepq_decode_step(tv["q"], tv["k"], tv["v"], tv["beta"], tv["gate"], layout.bits_dev, w,
+                                      layout.head_off_dev, layout.bytes_per_seq, st_q["packed"], st_q["r"],
+                                      st_q["c"], st_q["packed"], st_q["r"], st_q["c"], o_q, pivots=layout.pivots,
+                                      mixed=layout.mixed)
+                api.stepq_decode_step_fp32(tv["q"], tv["k"], tv["v"], tv["beta"], tv["gate"], S_f, S_f, o_f)
+                num[t] = torch.linalg.vector_norm((o_q - o_f).double())
+                den[t] = torch.linalg.vector_norm(o_f.double())
+        d_t = (num / den).cpu().numpy()
+        drift = {"steps": T, "tiles": tiles, "mean": float(d_t.mean()), "final": float(d_t[-1]),
+                 "mean_first_256": float(d_t[:256].mean()),
+                 "definition": "||O_q(t) - O_fp32(t)||_F / ||O_fp32(t)||_F over every tile, averaged over "
+                               "t = 1..T; both states stepped on the GPU from the same initial state and tokens"}
+        del st_q, S_f
+        torch.cuda.synchronize()
+    del S0
+
     # ---- end to end through the public API with host buffers (H2D inputs, D2H output) ----
     if args.kernel == "prefill":
         host_tok = []
@@ -500,6 +621,21 @@ def main():
     o_host = [torch.empty(tuple(outs[0].shape), dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = pinned[0].numel()
     d2h = o_host[0].numel() * o_host[0].element_size()
+    # The host link alone: the step's input copy and readout copy, each timed by itself.
+    link = {}
+    for name, (dst, src) in (("h2d_gbs", (tok_bufs[0] if args.kernel != "leap" else tok_bufs[0][0], pinned[0])),
+                             ("d2h_gbs", (o_host[0], outs[0]))):
+        l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                dst.copy_(src, non_blocking=True)
+            l0.record(stream)
+            for _ in range(20):
+                dst.copy_(src, non_blocking=True)
+            l1.record(stream)
+        stream.synchronize()
+        link[name] = dst.numel() * dst.element_size() * 20 / (l0.elapsed_time(l1) * 1e-3) / 1e9
+    link["bound_ms_per_step"] = max(h2d / (link["h2d_gbs"] * 1e9), d2h / (link["d2h_gbs"] * 1e9)) * 1e3
     # Three streams: inputs in, step, readout out; step s's copies overlap step s-1's work, and
     # buffers are reused R steps later, ordered by events. n_g such steps (each: one H2D copy of
     # the step's inputs, the library call, one D2H copy of its readout) are captured in a CUDA
@@ -561,8 +697,9 @@ def main():
     line = None
     if rank == 0:
         clocks = clk.summary()
+        prof = _profile(wl.name) if args.kernel == "quant" else {"traffic": None, "instr_per_element": None}
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": rounds_warm * R * LW,
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": warm,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
             "config": {**workload_config(wl, bits, args.kernel, world,
@@ -571,19 +708,23 @@ def main():
                               f"{R * per_rep / 2**20:.0f} MiB touched per round") if R * per_rep > L2_BYTES else
                              (f"inputs in L2 (latency case): {R} state replicas, "
                               f"{R * per_rep / 2**20:.1f} MiB touched per round"),
-                       "timing": "CUDA graph of one round of launches, CUDA events on the launching stream"},
+                       "timing": f"CUDA graph of one round of launches, CUDA events on the launching stream; "
+                                 f"K steps timed {args.repeats} times, median"},
+            "timing_runs_ms_per_step": [t / K for t in times],
             "elements_per_s": value * wl.d * wl.d,
             "achieved_gbs": achieved_gbs,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
                          "frac": achieved_gbs / peak, "peak_kind": peak_kind,
-                         "traffic": profiled_traffic() if (args.kernel == "quant" and args.workload == 1) else None,
+                         "traffic": prof["traffic"],
                          "bytes_per_launch": bytes_launch,
                          "bytes_per_launch_formula": "2*B*bytes_per_seq + B*H*(2*(2d+2d) + 6d + 4 + gate + 4d)"},
-            "alu_roofline": alu_roofline(value * wl.d * wl.d, clocks)
-            if (args.kernel == "quant" and args.workload == 1) else None,
+            "alu_roofline": alu_roofline(value * wl.d * wl.d, clocks, prof["instr_per_element"])
+            if args.kernel == "quant" else None,
+            "comparisons": comparisons,
+            "drift": drift,
             "gpu_launches": K * (3 if args.kernel == "split" else 1),   # split: first kernel, fit, pack
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": n_e2e,
+                    "steps": n_e2e, "link": link,
                     "method": f"CUDA graphs of {n_g} steps (each: one H2D copy of the step's inputs from pinned "
                               f"host memory, the library call, one D2H copy of its readout), replayed back to back"},
             "device_flags": flags,
@@ -591,12 +732,15 @@ def main():
             "clocks": clocks,
         }
     if world > 1:
-        graph = None
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         if not args.no_cpu_baseline and world == 1 and args.kernel == "quant":
-            line["cpu_baseline"] = cpu_baseline(wl, bits, args.cpu_seconds, args.cpu_threads)
+            w_host = w.detach().cpu().numpy() if hasattr(w, "detach") else np.asarray(w)
+            half = max(1.0, args.cpu_seconds / 2)
+            cb = cpu_baseline(wl, bits, w_host, half, args.cpu_threads)
+            cb["single_thread"] = cpu_baseline(wl, bits, w_host, half, 1)
+            line["cpu_baseline"] = cb
         else:
             line["cpu_baseline"] = None
         print(json.dumps(line), flush=True)

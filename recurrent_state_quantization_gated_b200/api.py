@@ -12,6 +12,7 @@ All calls are queued on torch's current CUDA stream.
 from __future__ import annotations
 
 import ctypes
+import weakref
 
 import numpy as np
 import torch
@@ -57,6 +58,38 @@ def _sizes(**tensors):
             raise TypeError(f"{name} must be a torch.Tensor")
         if t.numel() < n:
             raise ValueError(f"{name}: {t.numel()} elements, the call needs {n}")
+
+
+_LAYOUTS_CHECKED = {}
+
+
+def _check_layout(bits, head_off, bytes_per_seq):
+    """head_off and bytes_per_seq must be the packed layout of the bit map (stepq_packed_layout:
+    each head's range holds its tile, and the sequence holds every head). Checked on the host
+    the first time a (bits, head_off) pair is seen -- one device-to-host read of each, then
+    remembered while neither tensor is modified in place -- so make the first call with a new
+    layout outside CUDA-graph capture; during capture an unchecked pair is left to the kernels,
+    which check every tile's range themselves, skip a tile that does not fit and raise bit 2 of
+    the device error word."""
+    if not (isinstance(bits, torch.Tensor) and isinstance(head_off, torch.Tensor)):
+        return
+    key = (id(bits), bits._version, id(head_off), head_off._version, int(bytes_per_seq))
+    if key in _LAYOUTS_CHECKED:
+        return
+    if bits.is_cuda and torch.cuda.is_current_stream_capturing():
+        return
+    if bits.dim() != 2 or head_off.numel() < bits.shape[0]:
+        raise ValueError(f"bits must be [H, d] and head_off [H]; got {tuple(bits.shape)} and {tuple(head_off.shape)}")
+    H, d = bits.shape
+    want_off, want_bps, _ = stepq_packed_layout(bits.detach().cpu().numpy(), d)
+    got = head_off.detach().reshape(-1)[:H].cpu().numpy()
+    if not np.array_equal(got, want_off) or int(bytes_per_seq) != want_bps:
+        raise ValueError("head_off / bytes_per_seq do not match the bit map's packed layout "
+                         f"(bytes_per_seq {int(bytes_per_seq)}, expected {want_bps}); "
+                         "take them from stepq_packed_layout(bits)")
+    _LAYOUTS_CHECKED[key] = True
+    for t in (bits, head_off):
+        weakref.finalize(t, _LAYOUTS_CHECKED.pop, key, None)
 
 
 def _dims(B, H, d, gate_per_channel=0, pivots=0, mixed=0):
@@ -108,6 +141,7 @@ def stepq_pack_state(S, bits, head_off, bytes_per_seq, r, c, packed=None):
     packed = torch.empty(B * bytes_per_seq, dtype=torch.uint8, device=S.device) if packed is None else packed
     _sizes(S=(S, B * H * d * d), bits=(bits, H * d), head_off=(head_off, H), r=(r, B * H * d), c=(c, B * H * d),
            packed=(packed, B * int(bytes_per_seq)))
+    _check_layout(bits, head_off, bytes_per_seq)
     call("stepq_pack_state", _dims(B, H, d), _ptr(S, torch.float32, "S"), _ptr(bits, torch.uint8, "bits"),
          _ptr(head_off, torch.int64, "head_off"), ctypes.c_int64(int(bytes_per_seq)),
          _ptr(r, torch.float16, "r"), _ptr(c, torch.float16, "c"), _ptr(packed, torch.uint8, "packed"), _stream())
@@ -119,6 +153,7 @@ def stepq_unpack_state(packed, bits, head_off, bytes_per_seq, r, c, S_out=None):
     S_out = torch.empty((B, H, d, d), dtype=torch.float32, device=r.device) if S_out is None else S_out
     _sizes(packed=(packed, B * int(bytes_per_seq)), bits=(bits, H * d), head_off=(head_off, H), c=(c, B * H * d),
            S_out=(S_out, B * H * d * d))
+    _check_layout(bits, head_off, bytes_per_seq)
     call("stepq_unpack_state", _dims(B, H, d), _ptr(packed, torch.uint8, "packed"), _ptr(bits, torch.uint8, "bits"),
          _ptr(head_off, torch.int64, "head_off"), ctypes.c_int64(int(bytes_per_seq)),
          _ptr(r, torch.float16, "r"), _ptr(c, torch.float16, "c"), _ptr(S_out, torch.float32, "S_out"), _stream())
@@ -148,6 +183,7 @@ def stepq_decode_step(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, pac
     o = torch.empty((B, H, d), dtype=torch.float32, device=q.device) if o is None else o
     _sizes(**_step_sizes(B, H, d, gpc, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
                          packed_out, r_out, c_out, o))
+    _check_layout(bits, head_off, bytes_per_seq)
     call("stepq_decode_step", _dims(B, H, d, gpc, _has_pivots(bits, pivots), _has_mixed(bits, mixed)),
          _ptr(q, torch.bfloat16, "q"),
          _ptr(k, torch.bfloat16, "k"),
@@ -180,6 +216,7 @@ def stepq_decode_step_split(q, k, v, beta, gate, bits, w, head_off, bytes_per_se
     _sizes(x_ws=(x_ws, B * H * d * d),
            **_step_sizes(B, H, d, gpc, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
                          packed_out, r_out, c_out, o))
+    _check_layout(bits, head_off, bytes_per_seq)
     opt = lambda t, dt, n: _ptr(t, dt, n) if t is not None else None
     call("stepq_decode_step_split", _dims(B, H, d, gpc, _has_pivots(bits, pivots)), _ptr(q, torch.bfloat16, "q"),
          _ptr(k, torch.bfloat16, "k"),
@@ -211,6 +248,7 @@ def stepq_prefill_chunk(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, p
     name = {None: "stepq_prefill_chunk", "seq": "stepq_prefill_chunk_seq", "wy": "stepq_prefill_chunk_wy"}[form]
     _sizes(**_step_sizes(B, H, d, gpc, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
                          packed_out, r_out, c_out, o, C=C))
+    _check_layout(bits, head_off, bytes_per_seq)
     call(name, _dims(B, H, d, gpc, _has_pivots(bits, pivots), _has_mixed(bits, mixed)), ctypes.c_int(int(C)),
          _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
          _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"), _ptr(bits, torch.uint8, "bits"),

@@ -28,7 +28,8 @@
 
 namespace stepq {
 
-// Device error word: bit 0 = a bounded wait for a tile copy gave up.
+// Device error word: bit 0 = a bounded wait for a tile copy gave up; bit 1 = an FP16 pivot row
+// in a launch declared without pivots; bit 2 = a head range that cannot hold its tile.
 __device__ uint32_t g_stepq_flags = 0;
 
 struct DecodeArgs {
@@ -86,6 +87,7 @@ struct DecodeSmem {
     alignas(16) uint32_t hmeta[CH][D];
     alignas(16) uint16_t hslot[CH][D];   // by key row: slot | width << 8
     int htag[CH];                   // head held by each cache entry (-1: none)
+    int htot[CH];                   // the tile's bytes under the head's bit map
     // Per slot of the tile being decoded.
     alignas(16) float4 kq[D];       // alpha k, alpha k, alpha q, alpha q   (alpha = g r 2^(8-b))
     alignas(16) float4 ak[2][D];    // k/alpha, k/alpha, alpha, alpha (two tokens of a chunk)
@@ -113,14 +115,16 @@ __device__ __forceinline__ bool issue_tile(const DecodeArgs& a, DecodeSmem<D>& s
                                            float& gate1) {
     if (tile >= a.num_tiles) return false;
     const int b = tile / a.H, h = tile % a.H;
-    const int64_t hoff = a.head_off[h], hend = (h + 1 < a.H) ? a.head_off[h + 1] : a.bytes_per_seq;
+    int64_t hoff, hend;
     // The stage holds the integer rows (at most D*D bytes); FP16 pivot rows, stored after them,
-    // are read from global memory where they are used.
-    const uint32_t pbytes = static_cast<uint32_t>(min(hend - hoff, static_cast<int64_t>(D) * D));
+    // are read from global memory where they are used. A head range that cannot hold a tile
+    // copies no codes (the tile is skipped where it is computed).
+    const bool range_ok = tile_range_ok(a.head_off, a.H, a.bytes_per_seq, h, -1, 2 * D * D, &g_stepq_flags, &hoff, &hend);
+    const uint32_t pbytes = range_ok ? static_cast<uint32_t>(min(hend - hoff, static_cast<int64_t>(D) * D)) : 0u;
     auto& st = sm.stage[s];
     const uint32_t total = pbytes + 5u * 2u * D + 4u * D + (a.gate_per_channel ? 4u * D : 0u);
     mbar_arrive_expect_tx(&sm.full[s], total);
-    bulk_load(st.codes, a.packed_in + b * a.bytes_per_seq + hoff, pbytes, &sm.full[s]);
+    if (pbytes) bulk_load(st.codes, a.packed_in + b * a.bytes_per_seq + hoff, pbytes, &sm.full[s]);
     bulk_load(st.r, a.r_in + static_cast<int64_t>(tile) * D, 2 * D, &sm.full[s]);
     bulk_load(st.c, a.c_in + static_cast<int64_t>(tile) * D, 2 * D, &sm.full[s]);
     bulk_load(st.q, a.q + static_cast<int64_t>(tile) * D, 2 * D, &sm.full[s]);
@@ -330,12 +334,18 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
         if (sm.htag[he] != h) {                     // every warp sees the same tag: uniform branch
             __syncthreads();                        // nobody still reads the entry
             if (warp == 0) {
-                sort_head_rows<D, kPiv>(a.bits + static_cast<int64_t>(h) * D, sm.hmeta[he], sm.hslot[he], lane,
-                                           &g_stepq_flags);
-                if (lane == 0) sm.htag[he] = h;
+                const int tot = sort_head_rows<D, kPiv>(a.bits + static_cast<int64_t>(h) * D, sm.hmeta[he],
+                                                        sm.hslot[he], lane, &g_stepq_flags);
+                if (lane == 0) {
+                    sm.htag[he] = h;
+                    sm.htot[he] = tot;
+                }
             }
             __syncthreads();
         }
+        // The head's byte range must hold the tile under the bit map (same answer in every thread).
+        const bool tile_ok = tile_range_ok(a.head_off, a.H, a.bytes_per_seq, h, sm.htot[he], 2 * D * D, nullptr);
+        if (!tile_ok && tid == 0) atomicOr(&g_stepq_flags, kFlagBadLayout);
         const bool ok = mbar_wait_bounded(&sm.full[s], parity, kWaitLimitNs, &g_stepq_flags);
 
         // A prefill chunk's token 1: its inputs are loaded now, behind the unpack (rows by the
@@ -350,7 +360,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
         }
 
         // ---- prologue: per-slot constants of this tile, q.k ------------------------------
-        if (ok) {
+        if (ok && tile_ok) {
             if (tid < D) {
                 const int i = tid;
                 const uint32_t sw = sm.hslot[he][i];
@@ -393,6 +403,14 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
         const int ahead = n + kStages - 1, sa = ahead % kStages;
         bool issued = false;
         float next_beta = 0.f, next_gate = 0.f;
+        if (!tile_ok) {   // uniform: nothing of this tile is read or written
+            if (issuer && issue_tile<D>(a, sm, cta_tile(ahead), sa, next_beta, next_gate)) {
+                sm.stage[sa].beta = next_beta;
+                sm.stage[sa].gate1 = next_gate;
+            }
+            __syncthreads();
+            continue;
+        }
 
         // The warp's 16 slots share one width unless the warp straddles a width boundary.
         int ww;
@@ -574,9 +592,12 @@ decode_kernel(const DecodeArgs a) {
         for (int m = 0; m < n; ++m)
             if ((cta_tile(m) % a.H) % CH == h % CH) take = false;
         if (take) {
-            sort_head_rows<D, kPiv>(a.bits + static_cast<int64_t>(h) * D, sm.hmeta[h % CH], sm.hslot[h % CH], lane,
-                                       &g_stepq_flags);
-            if (lane == 0) sm.htag[h % CH] = h;
+            const int tot = sort_head_rows<D, kPiv>(a.bits + static_cast<int64_t>(h) * D, sm.hmeta[h % CH],
+                                                    sm.hslot[h % CH], lane, &g_stepq_flags);
+            if (lane == 0) {
+                sm.htag[h % CH] = h;
+                sm.htot[h % CH] = tot;
+            }
         }
     }
     __syncthreads();

@@ -351,7 +351,7 @@ __device__ __forceinline__ int reduced_row(int warp, int lane, int slot, bool& o
 // Byte offset of every row inside its tile (one warp): the integer rows first, in key order,
 // then the FP16 pivot rows (width 16), in key order. Row i has D/8 * b_i bytes.
 template <int D>
-__device__ __forceinline__ void row_offsets_warp(const uint8_t* bits, uint16_t* roff, int lane) {
+__device__ __forceinline__ int row_offsets_warp(const uint8_t* bits, uint16_t* roff, int lane) {
     constexpr int RL = D / 32;
     int loc[RL], sum_i = 0, sum_p = 0;
 #pragma unroll
@@ -374,6 +374,30 @@ __device__ __forceinline__ void row_offsets_warp(const uint8_t* bits, uint16_t* 
         const int base = b == 16 ? total_i + inc_p - sum_p : inc_i - sum_i;
         roff[lane * RL + r] = static_cast<uint16_t>(base + loc[r]);
     }
+    return total_i + __shfl_sync(0xffffffffu, inc_p, 31);   // the tile's bytes
+}
+
+// Bit 2 of the device error word: a tile whose head-offset range cannot hold it (see below).
+constexpr uint32_t kFlagBadLayout = 4u;
+
+// Whether head h's byte range in a sequence, [head_off[h], end) with end = head_off[h+1] (or
+// bytes_per_seq for the last head), can hold a tile of `tile_bytes` bytes: both ends 16-byte
+// aligned, ascending, inside the sequence, and at least tile_bytes long. A kernel that gets false
+// skips the tile (reads and writes nothing of it) and raises bit 2 of *flags, so a head-offset
+// table that does not match the bit map, or a bytes_per_seq shorter than the table, never moves an
+// access outside the tile's own range. tile_bytes < 0 checks the range alone (at most max_bytes).
+__device__ __forceinline__ bool tile_range_ok(const int64_t* head_off, int H, int64_t bytes_per_seq, int h,
+                                              int64_t tile_bytes, int64_t max_bytes, uint32_t* flags,
+                                              int64_t* hoff_out = nullptr, int64_t* hend_out = nullptr) {
+    const int64_t hoff = head_off[h];
+    const int64_t hend = (h + 1 < H) ? head_off[h + 1] : bytes_per_seq;
+    const int64_t need = tile_bytes >= 0 ? tile_bytes : 0;
+    const bool ok = hoff >= 0 && ((hoff | hend) & 15) == 0 && hoff + need <= hend && hend <= bytes_per_seq &&
+                    hend - hoff <= max_bytes;
+    if (!ok && flags) atomicOr(flags, kFlagBadLayout);
+    if (hoff_out) *hoff_out = hoff;
+    if (hend_out) *hend_out = hend;
+    return ok;
 }
 
 // Combine the per-thread column partials of the RPW sub-rows of a warp.

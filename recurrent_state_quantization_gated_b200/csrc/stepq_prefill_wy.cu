@@ -94,6 +94,7 @@ struct Small {
     alignas(8) uint64_t bar_sc;      // the last round's boundary-state product, committed apart
     alignas(8) uint64_t bar_codes;
     uint32_t tmem;
+    int tile_ok;                     // the tile's head range holds it under the bit map
 };
 
 // Shared-memory map (bytes). The work region is reused phase by phase.
@@ -193,17 +194,21 @@ struct Ahead {
     uint32_t widths;
     uint32_t rc;          // r_i | c_i << 16 (binary16 bits)
     int64_t codes_src;    // thread 0: the packed codes of the tile after this one (their copy is
-    uint32_t codes_bytes; // queued while this one is computed), or 0 bytes if there is none
+    uint32_t codes_bytes; // queued while this one is computed); 0 bytes if its head range is bad
+    bool has_next;        // thread 0: there is a tile after this one
 };
 
 __device__ __forceinline__ Ahead load_ahead(const WyArgs& a, int tile, int tid, int warp, int lane) {
-    Ahead n{1.0f, 1.0f, 0.0f, 0.0f, 0u, 0u, 0, 0u};
+    Ahead n{1.0f, 1.0f, 0.0f, 0.0f, 0u, 0u, 0, 0u, false};
     const int64_t T = a.num_tiles;
     if (tid == 0 && tile + static_cast<int>(gridDim.x) < a.num_tiles) {
         const int t2 = tile + gridDim.x, b2 = t2 / a.H, h2 = t2 % a.H;
-        const int64_t hoff = a.head_off[h2], hend = (h2 + 1 < a.H) ? a.head_off[h2 + 1] : a.bytes_per_seq;
-        n.codes_src = static_cast<int64_t>(b2) * a.bytes_per_seq + hoff;
-        n.codes_bytes = static_cast<uint32_t>(min(hend - hoff, static_cast<int64_t>(D) * D));
+        int64_t hoff, hend;
+        n.has_next = true;
+        if (tile_range_ok(a.head_off, a.H, a.bytes_per_seq, h2, -1, 2 * D * D, a.flags, &hoff, &hend)) {
+            n.codes_src = static_cast<int64_t>(b2) * a.bytes_per_seq + hoff;
+            n.codes_bytes = static_cast<uint32_t>(min(hend - hoff, static_cast<int64_t>(D) * D));
+        }
     }
     if (warp == 0) {
         const int t0 = 2 * lane, t1 = t0 + 1;
@@ -234,12 +239,15 @@ __device__ __forceinline__ void load_tokens(const WyArgs& a, int tile, int tid, 
     cp_async_commit();
 }
 
+// Queues the copy of a tile's packed codes; a head range that cannot hold a tile copies nothing
+// (the arrival still completes the barrier phase, and the tile is skipped where it is computed).
 __device__ __forceinline__ void issue_codes(const WyArgs& a, int tile, uint8_t* dst, uint64_t* bar) {
     const int b = tile / a.H, h = tile % a.H;
-    const int64_t hoff = a.head_off[h], hend = (h + 1 < a.H) ? a.head_off[h + 1] : a.bytes_per_seq;
-    const uint32_t bytes = static_cast<uint32_t>(min(hend - hoff, static_cast<int64_t>(D) * D));
+    int64_t hoff, hend;
+    const bool ok = tile_range_ok(a.head_off, a.H, a.bytes_per_seq, h, -1, 2 * D * D, a.flags, &hoff, &hend);
+    const uint32_t bytes = ok ? static_cast<uint32_t>(min(hend - hoff, static_cast<int64_t>(D) * D)) : 0u;
     mbar_arrive_expect_tx(bar, bytes);
-    bulk_load(dst, a.packed_in + static_cast<int64_t>(b) * a.bytes_per_seq + hoff, bytes, bar);
+    if (bytes) bulk_load(dst, a.packed_in + static_cast<int64_t>(b) * a.bytes_per_seq + hoff, bytes, bar);
 }
 
 __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
@@ -318,7 +326,12 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
         const int next = tile + gridDim.x;
 
         // ---- A: tables, gates, scales, codes -----------------------------------------------
-        if (warp == 1) sort_head_rows_w<D, false>(nx.widths, sm.hmeta, sm.hslot, lane, a.flags);
+        if (warp == 1) {
+            const int total = sort_head_rows_w<D, false>(nx.widths, sm.hmeta, sm.hslot, lane, a.flags);
+            // A head range that cannot hold the tile under the bit map: the tile is computed on
+            // whatever the buffers hold and none of its results is written.
+            if (lane == 0) sm.tile_ok = tile_range_ok(a.head_off, a.H, a.bytes_per_seq, h, total, 2 * D * D, a.flags);
+        }
         if (warp == 0) {   // beta and the running log2 of the gate product (a zero gate counts 2^-64)
             const float l0 = log2f(fmaxf(nx.g0, 0x1p-64f));
             const float l1 = l0 + log2f(fmaxf(nx.g1, 0x1p-64f));
@@ -374,9 +387,9 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             for (int ks = 0; ks < D / 16; ++ks)
                 umma::mma_bf16(tm + TM_G, umma::desc_kmajor(KQ, ks, D), umma::desc_kmajor(KQ, ks, D), id, ks > 0);
             umma::commit(&sm.bar_mma);
-            if (nx.codes_bytes) {   // the codes buffer is free: fetch the next tile's
+            if (nx.has_next) {   // the codes buffer is free: fetch the next tile's
                 mbar_arrive_expect_tx(&sm.bar_codes, nx.codes_bytes);
-                bulk_load(codes, a.packed_in + nx.codes_src, nx.codes_bytes, &sm.bar_codes);
+                if (nx.codes_bytes) bulk_load(codes, a.packed_in + nx.codes_src, nx.codes_bytes, &sm.bar_codes);
                 codes_pending = true;
             }
         }
@@ -655,7 +668,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                 for (int c32 = 0; c32 < 2; ++c32) {
                     float ov[32];
                     umma::tmem_ld32(tm_at(tm, warp, TM_S + 64 * hf + 32 * c32), ov);
-                    if (t < a.chunk) {
+                    if (t < a.chunk && sm.tile_ok) {
                         const int j0 = 64 * hf + 32 * c32;
 #pragma unroll
                         for (int q4 = 0; q4 < 8; ++q4) {
@@ -720,7 +733,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             const int w0 = (sm.hmeta[warp * M::kRowsPerWarp] >> 8) & 0xFF;
             const int w1 = (sm.hmeta[warp * M::kRowsPerWarp + M::kRowsPerWarp - 1] >> 8) & 0xFF;
             const int ww = (w0 == w1) ? w0 : 0;
-            refit_pack<D, false, false>(fit, sm.hmeta, Zr, ww, 0, tile, a.r_out, a.c_out, a.packed_out + tile_base);
+            if (sm.tile_ok)   // uniform over the CTA
+                refit_pack<D, false, false>(fit, sm.hmeta, Zr, ww, 0, tile, a.r_out, a.c_out, a.packed_out + tile_base);
         }
         __syncthreads();   // the next tile rewrites the tables and the regions
     }

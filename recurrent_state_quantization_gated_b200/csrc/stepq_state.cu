@@ -28,6 +28,7 @@ struct TileSmem {
     alignas(16) double red[M::kWarps][2][D];
     alignas(16) double rowbuf[M::kWarps][32 * (M::RPT + 1)];
     alignas(16) uint16_t roff[D];
+    int ok;                          // pack / unpack: the head's byte range holds the tile
 };
 
 // The quantisation contract: t = (x * ir) * ic, nearest-even, clamped to [-q_b, q_b].
@@ -177,6 +178,7 @@ struct StateArgs {
     float* S_out;
     int uniform_bits;   // distortion: > 0 replaces the bit map by this width
     double* scratch;    // distortion: per-(tile, row) squared error
+    uint32_t* flags;    // pack / unpack: device error word (bit 2: head range cannot hold the tile)
 };
 
 template <int D>
@@ -220,8 +222,12 @@ __global__ void __launch_bounds__(Map<D>::kThreads) pack_kernel(const StateArgs 
     float X[M::RPT][4];
     load_tile<D>(a.S + static_cast<int64_t>(tile) * D * D, warp, lane, X);
     __syncthreads();
-    if (warp == 0) row_offsets_warp<D>(sm.bits, sm.roff, lane);
+    if (warp == 0) {
+        const int total = row_offsets_warp<D>(sm.bits, sm.roff, lane);
+        if (lane == 0) sm.ok = tile_range_ok(a.head_off, a.H, a.bytes_per_seq, h, total, 2 * D * D, a.flags);
+    }
     __syncthreads();
+    if (!sm.ok) return;   // offsets that do not match the bit map: nothing of the tile is written
     uint8_t* out = a.packed + static_cast<int64_t>(tile / a.H) * a.bytes_per_seq + a.head_off[h];
     float ic[4];
 #pragma unroll
@@ -259,8 +265,12 @@ __global__ void __launch_bounds__(Map<D>::kThreads) unpack_kernel(const StateArg
         sm.colc[tid] = half_bits_to_float(a.c_in[static_cast<int64_t>(tile) * D + tid]);
     }
     __syncthreads();
-    if (warp == 0) row_offsets_warp<D>(sm.bits, sm.roff, lane);
+    if (warp == 0) {
+        const int total = row_offsets_warp<D>(sm.bits, sm.roff, lane);
+        if (lane == 0) sm.ok = tile_range_ok(a.head_off, a.H, a.bytes_per_seq, h, total, 2 * D * D, a.flags);
+    }
     __syncthreads();
+    if (!sm.ok) return;   // offsets that do not match the bit map: nothing of the tile is read
     const uint8_t* in = a.packed_in + static_cast<int64_t>(tile / a.H) * a.bytes_per_seq + a.head_off[h];
     float* S = a.S_out + static_cast<int64_t>(tile) * D * D;
     float cf[4];
@@ -401,6 +411,8 @@ extern "C" int stepq_pack_state(stepq_dims dims, const float* S, const uint8_t* 
     StateArgs a{};
     a.H = dims.H; a.S = S; a.bits = bits; a.head_off = head_off; a.bytes_per_seq = bytes_per_seq;
     a.r_in = r; a.c_in = c; a.packed = packed;
+    rc = device_flags_ptr(&a.flags);
+    if (rc) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return dims.dk == 128 ? launch_state<128>("stepq_pack_state", pack_kernel<128>, (int)tiles, a, st)
                           : launch_state<64>("stepq_pack_state", pack_kernel<64>, (int)tiles, a, st);
@@ -421,6 +433,8 @@ extern "C" int stepq_unpack_state(stepq_dims dims, const uint8_t* packed, const 
     StateArgs a{};
     a.H = dims.H; a.bits = bits; a.head_off = head_off; a.bytes_per_seq = bytes_per_seq;
     a.r_in = r; a.c_in = c; a.packed_in = packed; a.S_out = S_out;
+    rc = device_flags_ptr(&a.flags);
+    if (rc) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return dims.dk == 128 ? launch_state<128>("stepq_unpack_state", unpack_kernel<128>, (int)tiles, a, st)
                           : launch_state<64>("stepq_unpack_state", unpack_kernel<64>, (int)tiles, a, st);

@@ -41,8 +41,8 @@ __device__ __forceinline__ uint32_t head_widths(const uint8_t* bits_h, int lane)
 // head's D widths. hmeta[slot] = row | width << 8 | byte offset << 16; hslot[row] = slot |
 // width << 8. A width-16 row with kPiv false raises bit 1 of *flags.
 template <int D, bool kPiv>
-__device__ __forceinline__ void sort_head_rows_w(uint32_t widths, uint32_t* hmeta, uint16_t* hslot, int lane,
-                                                 uint32_t* flags) {
+__device__ __forceinline__ int sort_head_rows_w(uint32_t widths, uint32_t* hmeta, uint16_t* hslot, int lane,
+                                                uint32_t* flags) {
     // Width classes in slot order: 2, 4, 6, 8, then 16 (FP16 pivot rows). Byte offsets follow
     // the packed layout: integer rows in key order, then pivot rows in key order.
     constexpr int RL = D / 32, NC = 5;
@@ -105,13 +105,14 @@ __device__ __forceinline__ void sort_head_rows_w(uint32_t widths, uint32_t* hmet
         hmeta[slot] = static_cast<uint32_t>(i) | (static_cast<uint32_t>(wb) << 8) | (static_cast<uint32_t>(off) << 16);
         hslot[i] = static_cast<uint16_t>(slot | (wb << 8));
     }
+    return total_i + __shfl_sync(0xffffffffu, inc_p, 31);   // the tile's bytes under this bit map
 }
 
 // As sort_head_rows_w, from the bit map row of the head (bits_h: D widths, 4-byte aligned).
 template <int D, bool kPiv>
-__device__ __forceinline__ void sort_head_rows(const uint8_t* bits_h, uint32_t* hmeta, uint16_t* hslot, int lane,
-                                               uint32_t* flags) {
-    sort_head_rows_w<D, kPiv>(head_widths<D>(bits_h, lane), hmeta, hslot, lane, flags);
+__device__ __forceinline__ int sort_head_rows(const uint8_t* bits_h, uint32_t* hmeta, uint16_t* hslot, int lane,
+                                              uint32_t* flags) {
+    return sort_head_rows_w<D, kPiv>(head_widths<D>(bits_h, lane), hmeta, hslot, lane, flags);
 }
 
 // Eight consecutive per-column values (columns 8cl .. 8cl+7) as four pairs.

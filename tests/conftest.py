@@ -1,6 +1,7 @@
 import os
 import sys
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -25,3 +26,27 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """The measured code-mismatch rates of the GPU decode comparisons in this run (one line per
+    test label): worst and mean over steps of the share of integer codes one step off."""
+    try:
+        from tests.helpers import RATES
+    except Exception:  # pragma: no cover
+        return
+    rows = [r for r in RATES if r.get("label")]
+    if not rows:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "decode code-mismatch rates (share of integer codes one step off)")
+    by = {}
+    for r in rows:
+        by.setdefault(r["label"], []).append(r)
+    for label, rs in by.items():
+        gs = [r["at_gpu_scales"] for r in rs if r["at_gpu_scales"] is not None]
+        tr.write_line(
+            f"{label}: steps {len(rs)}, codes {sum(r['n_codes'] for r in rs)}; at the GPU's scales max "
+            f"{max(gs) if gs else float('nan'):.2e}; vs the oracle's codes max {max(r['raw'] for r in rs):.2e} "
+            f"mean {np.mean([r['raw'] for r in rs]):.2e}; scales differing: r {np.mean([r['r_mismatch'] for r in rs]):.2e}, "
+            f"c {np.mean([r['c_mismatch'] for r in rs]):.2e}")

@@ -17,8 +17,13 @@ def z(dtype, *shape):
     return torch.zeros(shape, dtype=dtype)
 
 
+def HEAD_OFF():
+    """The packed layout's head offsets of a uniform 6-bit map: P_h = d/8 * 6 * d bytes per head."""
+    return torch.arange(H, dtype=i64) * (BPS // H)
+
+
 def _state_args():
-    return dict(bits=z(u8, H, d) + 6, w=z(f32, H, d), head_off=z(i64, H), bytes_per_seq=BPS,
+    return dict(bits=z(u8, H, d) + 6, w=z(f32, H, d), head_off=HEAD_OFF(), bytes_per_seq=BPS,
                 packed_in=z(u8, B * BPS), r_in=z(f16, B, H, d), c_in=z(f16, B, H, d),
                 packed_out=z(u8, B * BPS), r_out=z(f16, B, H, d), c_out=z(f16, B, H, d))
 
@@ -52,10 +57,10 @@ CASES = {
                    lambda: dict(S=z(f32, B, H, d, d), w=z(f32, H, d), bits=z(u8, H, d), r=z(f16, B, H, d),
                                 c=z(f16, B, H, d))),
     "pack_state": (api.stepq_pack_state,
-                   lambda: dict(S=z(f32, B, H, d, d), bits=z(u8, H, d), head_off=z(i64, H), bytes_per_seq=BPS,
+                   lambda: dict(S=z(f32, B, H, d, d), bits=z(u8, H, d) + 6, head_off=HEAD_OFF(), bytes_per_seq=BPS,
                                 r=z(f16, B, H, d), c=z(f16, B, H, d), packed=z(u8, B * BPS))),
     "unpack_state": (api.stepq_unpack_state,
-                     lambda: dict(packed=z(u8, B * BPS), bits=z(u8, H, d), head_off=z(i64, H), bytes_per_seq=BPS,
+                     lambda: dict(packed=z(u8, B * BPS), bits=z(u8, H, d) + 6, head_off=HEAD_OFF(), bytes_per_seq=BPS,
                                   r=z(f16, B, H, d), c=z(f16, B, H, d), S_out=z(f32, B, H, d, d))),
     "int8_quantize_state": (api.stepq_int8_quantize_state,
                             lambda: dict(S=z(f32, B, H, d, d), codes=z(i8, B, H, d, d), s=z(f16, B, H, d))),
@@ -96,3 +101,22 @@ def test_every_short_buffer_is_refused_by_name(name):
             fn(**args)
         checked += 1
     assert checked >= 2
+
+
+@pytest.mark.parametrize("name", ["decode_step", "decode_step_split", "prefill_chunk", "pack_state", "unpack_state"])
+def test_a_layout_that_does_not_match_the_bit_map_is_refused(name):
+    """head_off / bytes_per_seq are checked against the bit map's packed layout on the host before
+    the call reaches the C ABI (a wrong table would move the kernels' accesses; the kernels also
+    check every tile's range themselves)."""
+    fn, make = CASES[name]
+    args = make()
+    args["head_off"] = HEAD_OFF().flip(0)
+    with pytest.raises(ValueError, match="do not match the bit map's packed layout"):
+        fn(**args)
+    args = make()
+    args["bytes_per_seq"] = BPS - 16
+    for key in ("packed", "packed_in", "packed_out"):
+        if key in args:
+            args[key] = z(u8, B * BPS)
+    with pytest.raises(ValueError, match="do not match the bit map's packed layout"):
+        fn(**args)

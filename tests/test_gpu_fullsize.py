@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 from recurrent_state_quantization_gated_b200 import synth
-from tests.helpers import compare_decode, dev, half_ulps, host_half
+from tests.helpers import compare_decode, dev, half_ulps, host_half, oracle_updated_state
 
 pytestmark = pytest.mark.gpu
 
@@ -60,9 +60,11 @@ def _start_from_oracle(wl, bits, w, S0, seqs):
     return st, (p_ref, r_ref, c_ref)
 
 
-@pytest.mark.parametrize("index", [1, 2, 3])
+@pytest.mark.parametrize("index", [1, 2, 3, 4])
 def test_full_size_step_on_sampled_sequences(index):
-    """gdn 64x32, kda 256x32 (channel gates), gdn4 1024x16 ({2,4,8} bits), d = 128."""
+    """gdn 64x32, kda 256x32 (channel gates), gdn4 1024x16 ({2,4,8} bits), drift 128x32 (heads at
+    g = 0.999 / 0.9, Student-t values), d = 128; every integer code of the sampled sequences
+    checked at the GPU's scales."""
     import torch
     from recurrent_state_quantization_gated_b200 import runtime
     wl = synth.workload(index)
@@ -74,10 +76,12 @@ def test_full_size_step_on_sampled_sequences(index):
         tok = synth.tokens(wl, t)
         o = st.step(**runtime.to_device_tokens(tok))
         torch.cuda.synchronize()
-        ref = oracle.decode_step(_subset(tok, seqs), bits, w, p_ref, r_ref, c_ref)
+        ts = _subset(tok, seqs)
+        ref = oracle.decode_step(ts, bits, w, p_ref, r_ref, c_ref)
+        X_ref = oracle_updated_state(ts, bits, p_ref, r_ref, c_ref)
         gpu = (_seq_bytes(st.packed.cpu().numpy(), seqs, st.layout.bytes_per_seq), host_half(st.r)[seqs],
                host_half(st.c)[seqs], o.cpu().numpy()[seqs])
-        compare_decode(gpu, ref, bits, wl.d, len(seqs))
+        compare_decode(gpu, ref, bits, wl.d, len(seqs), X_ref=X_ref, label=f"full size {wl.name}, sampled sequences")
         # the next step starts both sides from the oracle's state again
         p_ref, r_ref, c_ref = ref[:3]
         bps = st.layout.bytes_per_seq

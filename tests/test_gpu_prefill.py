@@ -8,7 +8,7 @@ import pytest
 
 import oracle
 from recurrent_state_quantization_gated_b200 import synth
-from tests.helpers import compare_decode, dev, host_half, with_pivots
+from tests.helpers import compare_decode, dev, host_half, oracle_chunk_state, with_pivots
 
 pytestmark = pytest.mark.gpu
 
@@ -56,7 +56,8 @@ def test_prefill_chunk_matches_oracle(d, B, H, widths, gpc, C, pivots):
     for t in range(C):
         compare_o = np.abs(og[t] - orf[t]).max(axis=-1) / np.maximum(np.abs(orf[t]).max(axis=-1), 1e-30)
         assert compare_o.max() <= 1e-3, (t, compare_o.max())
-    compare_decode((p_g.cpu().numpy(), host_half(r_g), host_half(c_g), og[-1]), (p_r, r_r, c_r, o_r[-1]), bits, d, B)
+    compare_decode((p_g.cpu().numpy(), host_half(r_g), host_half(c_g), og[-1]), (p_r, r_r, c_r, o_r[-1]), bits, d, B,
+                   X_ref=oracle_chunk_state(toks, bits, packed, r, c), label=f"prefill chunk C={C} d={d} H={H}")
 
 
 def test_one_token_chunk_is_the_decode_step():
@@ -92,7 +93,8 @@ def _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C):
     for t in range(C):
         err = np.abs(og[t] - o_r[t]).max(axis=-1) / np.maximum(np.abs(o_r[t]).max(axis=-1), 1e-30)
         assert err.max() <= 1e-3, (t, err.max())
-    return compare_decode((p_g, r_g, c_g, og[-1]), (p_r, r_r, c_r, o_r[-1]), bits, d, B)
+    return compare_decode((p_g, r_g, c_g, og[-1]), (p_r, r_r, c_r, o_r[-1]), bits, d, B,
+                          X_ref=oracle_chunk_state(toks, bits, packed, r, c), label=f"prefill chunk C={C} (tensor-core form)")
 
 
 @pytest.mark.parametrize("B,H,widths,C,in_place", [

@@ -61,3 +61,21 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--gpus", "2"])
     assert bench.main() == 0
     assert capsys.readouterr().out == ""
+
+
+def test_gpus_two_outside_torchrun_starts_two_ranks():
+    """``bench.py --gpus 2`` run directly (no torchrun environment) starts two ranks itself
+    (torch.distributed.run, 127.0.0.1); rank 0 prints one line with n_gpus = 2 -- here through the
+    oracle arm, which needs no GPU; the other rank exits without output."""
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR",
+                                                            "MASTER_PORT")}
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                          "--workload", "0", "--steps", "2", "--warmup", "1"],
+                         env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["n_gpus"] == 2 and rec["impl"] == "reference"
