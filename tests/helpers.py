@@ -138,8 +138,9 @@ def compare_decode(gpu, ref, bits, d, B, X_ref=None, max_frac=1e-3, label=""):
       the oracle's quantiser at the GPU's own scales must give the GPU's codes within one step,
       with at most ``max_frac`` of them one step off -- the bound that isolates the kernel's
       quantisation from the choice of scales;
-    * against the oracle's own codes (its own scales): never more than one step apart, and at
-      most ``max_frac`` of the entries whose row and column scales agree on both sides differ.
+    * against the oracle's own codes (its own scales): never more than one step apart, at most
+      ``max_frac`` of every integer entry differ, and at most ``max_frac`` of the entries whose
+      row and column scales agree on both sides.
 
     Returns a dict of rates, also appended to ``RATES``."""
     p_g, r_g, c_g, o_g = gpu
@@ -176,5 +177,6 @@ def compare_decode(gpu, ref, bits, d, B, X_ref=None, max_frac=1e-3, label=""):
     rates["equal_scales"] = float(frac_same)
     rates["raw"] = float((diff[integer] > 0).mean() if integer.any() else 0.0)
     assert frac_same <= max_frac, f"{frac_same:.2e} of codes with equal scales differ by one step"
+    assert rates["raw"] <= max_frac, f"{rates['raw']:.2e} of all integer codes differ from the oracle's own codes"
     RATES.append(rates)
     return rates

@@ -79,7 +79,7 @@ def test_decode_teacher_forced(d, B, H, widths, gpc, pivots):
         rates.append(r)
     assert max(r["at_gpu_scales"] for r in rates) <= 1e-3   # every integer code, every step
     assert np.mean([r["r_mismatch"] for r in rates]) < 1e-2 and np.mean([r["c_mismatch"] for r in rates]) < 1e-2
-    assert np.mean([r["raw"] for r in rates]) < 1e-2         # against the oracle's own codes and scales
+    assert max(r["raw"] for r in rates) <= 1e-3              # against the oracle's own codes and scales
 
 
 def test_tiny_workload_as_specified():

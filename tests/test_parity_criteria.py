@@ -111,7 +111,7 @@ def test_one_step_on_few_codes_passes_on_many_fails(case):
 
 def test_codes_at_the_device_scales_few_pass_many_fail(case):
     """The bound over every integer code: the oracle's own X quantised at the device's scales.
-    0.08 % of the codes one step off passes, 0.3 % fails, even where the device's scales differ
+    0.05 % of the codes one step off passes, 0.3 % fails, even where the device's scales differ
     from the oracle's (a row scale one ulp off: its codes are compared at the device's scale)."""
     bits, ref, X = case
     n_int = int((bits != 16).sum()) * D * B
@@ -124,7 +124,7 @@ def test_codes_at_the_device_scales_few_pass_many_fail(case):
     codes[0, 1] = codes2
     got = (_repack(codes, bits), r2, c, o)
     assert compare_decode(got, ref, bits, D, B, X_ref=X)["at_gpu_scales"] == 0.0
-    few = max(1, int(0.0008 * n_int))
+    few = max(1, int(0.0005 * n_int))
     many = int(0.003 * n_int)
     moved = _with_codes_moved(got, bits, few, seed=3)
     frac = compare_decode(moved, ref, bits, D, B, X_ref=X)["at_gpu_scales"]
@@ -160,3 +160,12 @@ def test_pivot_values_one_ulp_pass_two_fail(case):
         else:
             with pytest.raises(AssertionError, match="pivot values"):
                 compare_decode(got, ref, bits, D, B)
+
+
+def test_codes_off_the_oracles_own_beyond_the_bound_fail(case):
+    """Against the oracle's own codes, over every integer entry: a device result whose scales
+    all agree but 0.3 % of whose codes are one step off fails even without the oracle's X."""
+    bits, ref, X = case
+    n_int = int((bits != 16).sum()) * D * B
+    with pytest.raises(AssertionError):
+        compare_decode(_with_codes_moved(ref, bits, int(0.003 * n_int), seed=5), ref, bits, D, B)
