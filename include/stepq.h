@@ -260,7 +260,10 @@ STEPQ_API int stepq_calib_distortion_bits(stepq_dims dims, const float* S, const
    [B][H][dk] work space of stepq_calib_distortion.
    The work space is a file-scope device array of STEPQ_STATIC_SCRATCH_ROWS float64 entries,
    one per device. The first call on each device (with that device current) looks up its
-   address with cudaGetSymbolAddress; make that first call before any stream capture. Every
+   address with cudaGetSymbolAddress; make that first call before any stream capture. The
+   address is kept for the life of the process: after cudaDeviceReset() of a device (which
+   unloads the library's device code there) this entry point must not be called on that device
+   again in the same process. Every
    entry the call reads it has written itself, so nothing in the array needs clearing.
    All calls on one device share the array: calls that overlap in time (on different streams,
    or from different host threads without ordering) race and give wrong results; order them
@@ -290,7 +293,11 @@ STEPQ_API int stepq_allocate_bits(int n_units, int n_cand, const int* cand_host,
    copy, or a tensor-core round of the prefill chunk) gave up after its limit (2 s); the kernel
    then waits, bounded, for its own copies in flight, frees its tensor memory and returns, so the
    context stays usable. Bit 1 is set when a width-16 row was met in a launch with
-   dims.pivots = 0. Reads (synchronously, on the current device) and clears it. */
+   dims.pivots = 0. Bit 2 is set when a head's byte range in the packed state, [head_off[h],
+   head_off[h+1]) (bytes_per_seq for the last head), is unaligned, out of order, outside the
+   sequence or shorter than the head's tile under the bit map; the kernels (decode step, prefill
+   chunk, split form, pack, unpack) then skip that tile and read or write nothing of it. Reads
+   (synchronously, on the current device) and clears it. */
 STEPQ_API int stepq_read_device_flags(uint32_t* flags_host);
 
 /* Self-test of that wait limit: one bounded wait that nothing completes (an mbarrier phase no

@@ -21,8 +21,8 @@ INCLUDE = ROOT / "include"
 LIB = PKG / "libstepq.so"
 BUILD_DIR = ROOT / "_build"
 
-SOURCES = ["stepq_decode.cu", "stepq_prefill_wy.cu", "stepq_state.cu", "stepq_baseline.cu", "stepq_calib.cu",
-           "stepq_host.cpp"]
+SOURCES = ["stepq_decode.cu", "stepq_prefill_wy.cu", "stepq_state.cu", "stepq_baseline.cu", "stepq_int8.cu",
+           "stepq_calib.cu", "stepq_host.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
               "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills"]

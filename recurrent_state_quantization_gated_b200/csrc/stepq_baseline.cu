@@ -1,6 +1,7 @@
 // stepq_baseline.cu -- the two comparison state formats of STEPQuant §5.1 on sm_100a: the FP32
-// state (the serving default) and the uniform symmetric rowwise-absmax INT8 state. Both run the
-// same gated Delta-rule decode step (§2.1) with the readout taken before any requantisation.
+// state (the serving default) and the quantisation of a state into the uniform symmetric
+// rowwise-absmax INT8 format (its decode step is the persistent kernel of stepq_int8.cu), and the
+// per-window 8-bit state. The decode steps take the readout before any requantisation.
 //
 // One CTA per (sequence, head) tile with the register mapping of stepq_device.cuh; the tile is
 // loaded with 16-byte vector loads straight from HBM (each warp instruction reads one full row)
@@ -171,27 +172,6 @@ __device__ __forceinline__ void int8_requantise(Sm& sm, const float X[Map<D>::RP
         const uint32_t t23 = __byte_perm(q[2], q[3], 0x0040);
         *reinterpret_cast<uint32_t*>(out + row * D + 4 * cl) = __byte_perm(t01, t23, 0x5410);
     }
-}
-
-template <int D>
-__global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) decode_int8_kernel(const BaselineArgs a) {
-    using M = Map<D>;
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    BaselineSmem<D>& sm = *reinterpret_cast<BaselineSmem<D>*>(smem_raw);
-    const int tile = blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int cl = M::col_lane(lane);
-    const int8_t* C = a.codes_in + static_cast<int64_t>(tile) * D * D;
-    float Z[M::RPT][4];
-#pragma unroll
-    for (int r = 0; r < M::RPT; ++r) {
-        const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(C + M::row(warp, lane, r) * D + 4 * cl)) ^ 0x80808080u;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) Z[r][k] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650 | k)) - (kTwo23 + 128.0f);
-    }
-    baseline_prologue<D>(sm, a, tile, a.s_in);
-    baseline_update<D>(sm, a, tile, Z);
-    int8_requantise<D>(sm, Z, tile, a.codes_out, a.s_out);
 }
 
 template <int D>
@@ -485,26 +465,6 @@ extern "C" int stepq_int8_quantize_state(stepq_dims dims, const float* S, int8_t
     return dims.dk == 128
                ? launch_baseline<128>("stepq_int8_quantize_state", int8_quantize_kernel<128>, (int)tiles, a, st)
                : launch_baseline<64>("stepq_int8_quantize_state", int8_quantize_kernel<64>, (int)tiles, a, st);
-}
-
-extern "C" int stepq_decode_step_int8(stepq_dims dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                      const float* beta, const float* gate, const int8_t* codes_in,
-                                      const uint16_t* s_in, int8_t* codes_out, uint16_t* s_out, float* o,
-                                      void* stream) {
-    clear_error();
-    long long tiles;
-    int rc = tiles_of(dims, "stepq_decode_step_int8", tiles);
-    if (rc || tiles == 0) return rc;
-    rc = check_ptrs("stepq_decode_step_int8", {{"q", q}, {"k", k}, {"v", v}, {"beta", beta}, {"gate", gate},
-                                               {"codes_in", codes_in}, {"s_in", s_in}, {"codes_out", codes_out},
-                                               {"s_out", s_out}, {"o", o}});
-    if (rc) return rc;
-    BaselineArgs a{};
-    a.H = dims.H; a.gate_per_channel = dims.gate_per_channel; a.q = q; a.k = k; a.v = v; a.beta = beta;
-    a.gate = gate; a.codes_in = codes_in; a.s_in = s_in; a.codes_out = codes_out; a.s_out = s_out; a.o = o;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return dims.dk == 128 ? launch_baseline<128>("stepq_decode_step_int8", decode_int8_kernel<128>, (int)tiles, a, st)
-                          : launch_baseline<64>("stepq_decode_step_int8", decode_int8_kernel<64>, (int)tiles, a, st);
 }
 
 extern "C" int stepq_leap_step(stepq_dims dims, int window, int t, const uint16_t* q, const uint16_t* k,

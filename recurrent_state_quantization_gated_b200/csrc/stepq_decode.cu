@@ -607,22 +607,12 @@ decode_kernel(const DecodeArgs a) {
 
 template <int D, bool kSplit, bool kPiv, bool kChunk = false, bool kMixed = false>
 static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-    static int ctas_per_sm = -1, num_sms = 0;
     const size_t smem = sizeof(DecodeSmem<D>);
-    if (ctas_per_sm < 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, kSplit, kPiv, kChunk, kMixed>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "stepq_decode_step: %s", cudaGetErrorString(e));
-        int occ = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<D, kSplit, kPiv, kChunk, kMixed>, DMap<D>::kThreads, smem);
-        ctas_per_sm = occ > 0 ? occ : 1;
-    }
     if (a.num_tiles == 0) return STEPQ_OK;
-    int grid = num_sms * ctas_per_sm;
-    if (grid > a.num_tiles) grid = a.num_tiles;
+    int grid = 0;
+    int rc = persistent_grid(reinterpret_cast<const void*>(decode_kernel<D, kSplit, kPiv, kChunk, kMixed>),
+                             DMap<D>::kThreads, smem, a.num_tiles, "stepq_decode_step", &grid);
+    if (rc) return rc;
     decode_kernel<D, kSplit, kPiv, kChunk, kMixed><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
     return check_launch("stepq_decode_step");
 }

@@ -6,6 +6,8 @@
 #include <cmath>
 #include <cstdarg>
 #include <limits>
+#include <map>
+#include <mutex>
 #include <queue>
 #include <utility>
 #include <vector>
@@ -39,6 +41,36 @@ int check_ptrs(const char* fn, std::initializer_list<std::pair<const char*, cons
 int check_launch(const char* fn) {
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "%s: %s", fn, cudaGetErrorString(e));
+    return STEPQ_OK;
+}
+
+int persistent_grid(const void* kernel, int threads, size_t smem, long long tiles, const char* fn, int* grid) {
+    struct Entry {
+        int sms = 0, per_sm = 0;
+    };
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, Entry> cache;   // (kernel, device)
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "%s: %s", fn, cudaGetErrorString(e));
+    Entry ent;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find({kernel, dev});
+        if (it != cache.end()) ent = it->second;
+    }
+    if (ent.per_sm == 0) {
+        e = cudaDeviceGetAttribute(&ent.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ent.per_sm, kernel, threads, smem);
+        if (e != cudaSuccess) return set_error(STEPQ_ECUDA, "%s: %s", fn, cudaGetErrorString(e));
+        if (ent.per_sm < 1) return set_error(STEPQ_ECUDA, "%s: the kernel does not fit on an SM", fn);
+        std::lock_guard<std::mutex> lock(mu);
+        cache[{kernel, dev}] = ent;
+    }
+    const long long g = static_cast<long long>(ent.sms) * ent.per_sm;
+    *grid = static_cast<int>(std::min<long long>(g, std::max<long long>(tiles, 1)));
     return STEPQ_OK;
 }
 

@@ -39,4 +39,9 @@ int check_launch(const char* fn);
 // Device address of the current device's error word (the one stepq_read_device_flags reads).
 int device_flags_ptr(uint32_t** p);
 
+// Grid of a persistent kernel on the current device: the SM count times the CTAs of `threads`
+// threads and `smem` bytes of dynamic shared memory that fit on one SM, capped at `tiles`. The
+// kernel's shared-memory attribute and the occupancy are set up once per (kernel, device).
+int persistent_grid(const void* kernel, int threads, size_t smem, long long tiles, const char* fn, int* grid);
+
 }  // namespace stepq

@@ -28,6 +28,14 @@ struct DMap {
     __device__ static int col_lane(int lane) { return lane % LPR; }
     __device__ static int sub_row(int lane) { return lane / LPR; }
     __device__ static int row(int warp, int lane, int r) { return warp * kRowsPerWarp + r * RPW + sub_row(lane); }
+    // Row length of the column-partial buffers red[kWarps][2][kRedRow] of a kernel that finalises
+    // columns with every thread: the two rows of a warp are 16 banks apart, so lanes 0-15 and
+    // 16-31 of a warp reading the two rows at the same 16 columns are free of bank conflicts.
+    static constexpr int kRedRow = D + 16;
+    // The column such a thread finalises (16 per warp; lanes l and l + 16 share it), and which
+    // of the two partial rows it sums.
+    __device__ static int fin_col(int warp, int lane) { return 16 * warp + (lane & 15); }
+    __device__ static int fin_row(int lane) { return lane >> 4; }
 };
 
 // The widths of a head's key rows lane*RL .. lane*RL + RL-1 (RL = D/32), one byte each.
