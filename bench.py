@@ -487,7 +487,8 @@ def main():
         elif args.kernel == "quant":
             api.stepq_decode_step(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], layout.bits_dev, w,
                                   layout.head_off_dev, layout.bytes_per_seq, st["packed"], st["r"], st["c"],
-                                  st["packed"], st["r"], st["c"], o, pivots=layout.pivots, mixed=layout.mixed)
+                                  st["packed"], st["r"], st["c"], o, pivots=layout.pivots, mixed=layout.mixed,
+                                  widths=layout.widths)
         elif args.kernel == "fp32":
             api.stepq_decode_step_fp32(tk["q"], tk["k"], tk["v"], tk["beta"], tk["gate"], st["S"], st["S"], o)
         elif args.kernel == "leap":
@@ -596,7 +597,7 @@ def main():
                 api.stepq_decode_step(tv["q"], tv["k"], tv["v"], tv["beta"], tv["gate"], layout.bits_dev, w,
                                       layout.head_off_dev, layout.bytes_per_seq, st_q["packed"], st_q["r"],
                                       st_q["c"], st_q["packed"], st_q["r"], st_q["c"], o_q, pivots=layout.pivots,
-                                      mixed=layout.mixed)
+                                      mixed=layout.mixed, widths=layout.widths)
                 api.stepq_decode_step_fp32(tv["q"], tv["k"], tv["v"], tv["beta"], tv["gate"], S_f, S_f, o_f)
                 num[t] = torch.linalg.vector_norm((o_q - o_f).double())
                 den[t] = torch.linalg.vector_norm(o_f.double())

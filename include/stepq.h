@@ -79,6 +79,14 @@ typedef struct {
                                 chunk, which then run one code path for every row width instead of width-specialised paths per
                                 warp (smaller code: faster for such maps, slower for maps whose
                                 heads each use one width). Results are identical either way.  */
+    int widths;              /* The row widths the bit map holds, as a bit mask (bit b set for
+                                width b: 2, 4, 6, 8, 16), or 0 when not declared. Read by
+                                stepq_decode_step with mixed = 1, whose per-row code then handles
+                                only the declared widths (less code: the {2, 4, 8} and {4, 6, 8}
+                                sets have their own kernels). A row of an undeclared width is
+                                decoded as one of the declared ones and its results are undefined;
+                                every access stays inside its tile. Other bits: STEPQ_EINVAL.
+                                Other calls ignore it.  */
 } stepq_dims;
 
 /* Text of the last error raised on the calling thread ("" if none). */

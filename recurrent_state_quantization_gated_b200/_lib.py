@@ -32,7 +32,8 @@ class StepqError(RuntimeError):
 
 class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("dk", ctypes.c_int), ("dv", ctypes.c_int),
-                ("gate_per_channel", ctypes.c_int), ("pivots", ctypes.c_int), ("mixed", ctypes.c_int)]
+                ("gate_per_channel", ctypes.c_int), ("pivots", ctypes.c_int), ("mixed", ctypes.c_int),
+                ("widths", ctypes.c_int)]
 
 
 _lib = None

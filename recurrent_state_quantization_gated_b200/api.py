@@ -92,8 +92,29 @@ def _check_layout(bits, head_off, bytes_per_seq):
         weakref.finalize(t, _LAYOUTS_CHECKED.pop, key, None)
 
 
-def _dims(B, H, d, gate_per_channel=0, pivots=0, mixed=0):
-    return Dims(int(B), int(H), int(d), int(d), int(gate_per_channel), int(pivots), int(mixed))
+def _dims(B, H, d, gate_per_channel=0, pivots=0, mixed=0, widths=0):
+    return Dims(int(B), int(H), int(d), int(d), int(gate_per_channel), int(pivots), int(mixed), int(widths))
+
+
+def width_mask(bits) -> int:
+    """The bit mask of the row widths a bit map holds (bit b for width b), from a host array or
+    a tensor (a device tensor is read back: one synchronisation)."""
+    if isinstance(bits, torch.Tensor):
+        vals = torch.unique(bits).cpu().tolist()
+    else:
+        vals = np.unique(np.asarray(bits)).tolist()
+    m = 0
+    for b in vals:
+        m |= 1 << int(b)
+    return m
+
+
+def _widths(bits, widths, mixed):
+    """The widths field of a decode call: as given, else read from the bit map when the launch
+    takes the per-row path (mixed), else 0 (not needed)."""
+    if widths is not None:
+        return int(widths)
+    return width_mask(bits) if mixed else 0
 
 
 def _has_pivots(bits, pivots):
@@ -171,10 +192,11 @@ def _step_sizes(B, H, d, gpc, k, v, beta, gate, bits, w, head_off, bytes_per_seq
 
 
 def stepq_decode_step(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
-                      packed_out=None, r_out=None, c_out=None, o=None, pivots=None, mixed=None):
+                      packed_out=None, r_out=None, c_out=None, o=None, pivots=None, mixed=None, widths=None):
     """One fused quantized decode step; outputs may alias the inputs (in-place update).
-    pivots / mixed: the bit map's FP16 pivot rows / rows of different widths within a head
-    (None: read from the bit map). Returns (packed_out, r_out, c_out, o)."""
+    pivots / mixed / widths: the bit map's FP16 pivot rows / rows of different widths within a
+    head / mask of the widths present (None: read from the bit map). Returns (packed_out, r_out,
+    c_out, o)."""
     B, H, d = q.shape
     gpc = 1 if gate.dim() == 3 else 0
     packed_out = torch.empty_like(packed_in) if packed_out is None else packed_out
@@ -184,7 +206,8 @@ def stepq_decode_step(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, pac
     _sizes(**_step_sizes(B, H, d, gpc, k, v, beta, gate, bits, w, head_off, bytes_per_seq, packed_in, r_in, c_in,
                          packed_out, r_out, c_out, o))
     _check_layout(bits, head_off, bytes_per_seq)
-    call("stepq_decode_step", _dims(B, H, d, gpc, _has_pivots(bits, pivots), _has_mixed(bits, mixed)),
+    mixed = _has_mixed(bits, mixed)
+    call("stepq_decode_step", _dims(B, H, d, gpc, _has_pivots(bits, pivots), mixed, _widths(bits, widths, mixed)),
          _ptr(q, torch.bfloat16, "q"),
          _ptr(k, torch.bfloat16, "k"),
          _ptr(v, torch.bfloat16, "v"), _ptr(beta, torch.float32, "beta"), _ptr(gate, torch.float32, "gate"),

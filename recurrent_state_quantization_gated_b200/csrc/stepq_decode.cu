@@ -223,34 +223,28 @@ __device__ __forceinline__ void phase1_uniform(const DecodeSmem<D>& sm, const ui
     }
 }
 
-template <int D, bool kPiv>
+template <int D, bool kPiv, int kW = 0>
 __device__ __forceinline__ void phase1_mixed(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* codes,
                                              const uint8_t* gin, int warp, int lane, float2 Z[][4], float2 pacc[4],
                                              float2 oacc[4]) {
     using M = DMap<D>;
+    using WS = WidthSet<kW>;
     const int cl = M::col_lane(lane);
 #pragma unroll
     for (int r = 0; r < M::RPT; ++r) {
         const int s = M::row(warp, lane, r);
         const uint32_t mt = meta[s];
-        switch ((mt >> 8) & 0xFF) {
-            case 8: phase1_row<D, 8>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
-            case 6: phase1_row<D, 6>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
-            case 4: phase1_row<D, 4>(sm, codes, s, mt, cl, Z[r], pacc, oacc); break;
-            default:
-                if constexpr (kPiv) {
-                    if (((mt >> 8) & 0xFF) == 16) {
-                        phase1_pivot_row<D>(sm, codes, gin, s, mt, cl, Z[r], pacc, oacc);
-                        break;
-                    }
-                }
-                phase1_row<D, 2>(sm, codes, s, mt, cl, Z[r], pacc, oacc);
-                break;
-        }
+        const int bw = (mt >> 8) & 0xFF;
+        if constexpr (WS::tested(8)) if (bw == 8) { phase1_row<D, 8>(sm, codes, s, mt, cl, Z[r], pacc, oacc); continue; }
+        if constexpr (WS::tested(6)) if (bw == 6) { phase1_row<D, 6>(sm, codes, s, mt, cl, Z[r], pacc, oacc); continue; }
+        if constexpr (WS::tested(4)) if (bw == 4) { phase1_row<D, 4>(sm, codes, s, mt, cl, Z[r], pacc, oacc); continue; }
+        if constexpr (WS::tested(2)) if (bw == 2) { phase1_row<D, 2>(sm, codes, s, mt, cl, Z[r], pacc, oacc); continue; }
+        if constexpr (kPiv) if (bw == 16) { phase1_pivot_row<D>(sm, codes, gin, s, mt, cl, Z[r], pacc, oacc); continue; }
+        phase1_row<D, WS::fallback>(sm, codes, s, mt, cl, Z[r], pacc, oacc);
     }
 }
 
-template <int D, bool kPiv>
+template <int D, bool kPiv, int kW = 0>
 __device__ __forceinline__ void phase1(const DecodeSmem<D>& sm, const uint32_t* meta, const uint8_t* codes,
                                        const uint8_t* gin, int warp, int lane, int ww, float2 Z[][4],
                                        float2 pacc[4], float2 oacc[4]) {
@@ -266,7 +260,7 @@ __device__ __forceinline__ void phase1(const DecodeSmem<D>& sm, const uint32_t* 
                     break;
                 }
             }
-            phase1_mixed<D, kPiv>(sm, meta, codes, gin, warp, lane, Z, pacc, oacc);
+            phase1_mixed<D, kPiv, kW>(sm, meta, codes, gin, warp, lane, Z, pacc, oacc);
             break;
     }
 }
@@ -312,7 +306,7 @@ __device__ __forceinline__ void token_constants(DecodeSmem<D>& sm, int he, int i
 // The tile loop of the decode kernel. kPiv: the bit map may hold FP16 pivot rows (declared by
 // the caller in stepq_dims.pivots); launches without them run the leaner instantiation. A
 // width-16 row met in a launch declared without pivots raises bit 1 of the device error word.
-template <int D, bool kSplit, bool kPiv, bool kChunk, bool kMixed>
+template <int D, bool kSplit, bool kPiv, bool kChunk, bool kMixed, int kW>
 __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm) {
     using M = DMap<D>;
     constexpr int RPT = M::RPT;
@@ -426,7 +420,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
             float2 pacc[4], oacc[4];
 #pragma unroll
             for (int p = 0; p < 4; ++p) pacc[p] = oacc[p] = make_float2(0.f, 0.f);
-            phase1<D, kPiv>(sm, meta, st.codes, a.packed_in + tile_base, warp, lane, ww, Z, pacc, oacc);
+            phase1<D, kPiv, kW>(sm, meta, st.codes, a.packed_in + tile_base, warp, lane, ww, Z, pacc, oacc);
             store_col_partials<D>(sm.red[warp][0], lane, pacc);
             store_col_partials<D>(sm.red[warp][1], lane, oacc);
         }
@@ -539,7 +533,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
                 continue;
             }
         }
-        refit_pack<D, kPiv, true>(sm, meta, Z, ww, kb, tile, a.r_out, a.c_out, a.packed_out + tile_base);
+        refit_pack<D, kPiv, true, kW>(sm, meta, Z, ww, kb, tile, a.r_out, a.c_out, a.packed_out + tile_base);
         if (issued) {   // ordered before their use by the barriers of the next tiles
             sm.stage[sa].beta = next_beta;
             sm.stage[sa].gate1 = next_gate;
@@ -549,8 +543,9 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
 
 // kSplit: the first kernel of the split form. It reconstructs, updates and reads out like the
 // fused step, then writes the updated state X in fp32 and stops; the refit and the pack run
-// as separate kernels (stepq_decode_step_split).
-template <int D, bool kSplit, bool kPiv, bool kChunk = false, bool kMixed = false>
+// as separate kernels (stepq_decode_step_split). kW: the row widths of a mixed launch's
+// per-row code (a bit mask; 0 = every width).
+template <int D, bool kSplit, bool kPiv, bool kChunk = false, bool kMixed = false, int kW = 0>
 __global__ void __launch_bounds__(DMap<D>::kThreads, DMap<D>::kMinBlocks)
 decode_kernel(const DecodeArgs a) {
     using M = DMap<D>;
@@ -602,18 +597,18 @@ decode_kernel(const DecodeArgs a) {
     }
     __syncthreads();
 
-    run_tiles<D, kSplit, kPiv, kChunk, kMixed>(a, sm);
+    run_tiles<D, kSplit, kPiv, kChunk, kMixed, kW>(a, sm);
 }
 
-template <int D, bool kSplit, bool kPiv, bool kChunk = false, bool kMixed = false>
+template <int D, bool kSplit, bool kPiv, bool kChunk = false, bool kMixed = false, int kW = 0>
 static int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     const size_t smem = sizeof(DecodeSmem<D>);
     if (a.num_tiles == 0) return STEPQ_OK;
     int grid = 0;
-    int rc = persistent_grid(reinterpret_cast<const void*>(decode_kernel<D, kSplit, kPiv, kChunk, kMixed>),
+    int rc = persistent_grid(reinterpret_cast<const void*>(decode_kernel<D, kSplit, kPiv, kChunk, kMixed, kW>),
                              DMap<D>::kThreads, smem, a.num_tiles, "stepq_decode_step", &grid);
     if (rc) return rc;
-    decode_kernel<D, kSplit, kPiv, kChunk, kMixed><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
+    decode_kernel<D, kSplit, kPiv, kChunk, kMixed, kW><<<grid, DMap<D>::kThreads, smem, stream>>>(a);
     return check_launch("stepq_decode_step");
 }
 
@@ -671,12 +666,22 @@ extern "C" int stepq_decode_step(stepq_dims dims, const uint16_t* q, const uint1
     if (rc) return rc;
     if (bytes_per_seq <= 0 || (bytes_per_seq & 15))
         return set_error(STEPQ_EINVAL, "stepq_decode_step: bytes_per_seq=%lld", (long long)bytes_per_seq);
+    if (dims.widths & ~((1 << 2) | (1 << 4) | (1 << 6) | (1 << 8) | (1 << 16)))
+        return set_error(STEPQ_EINVAL, "stepq_decode_step: widths=0x%x (bits 2, 4, 6, 8 and 16 only)", dims.widths);
     const long long tiles = static_cast<long long>(dims.B) * dims.H;
     if (tiles > 0x7fffffffLL) return set_error(STEPQ_EINVAL, "stepq_decode_step: too many tiles");
     DecodeArgs a{dims.B, dims.H, dims.gate_per_channel, static_cast<int>(tiles), q, k, v, beta, gate, bits, w,
                  head_off, bytes_per_seq, packed_in, r_in, c_in, packed_out, r_out, c_out, o, nullptr, 1};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dims.mixed) {   // heads whose key rows have different widths: one code path for every width
+        constexpr int W248 = (1 << 2) | (1 << 4) | (1 << 8), W468 = (1 << 4) | (1 << 6) | (1 << 8);
+        const int wi = dims.widths & ~(1 << 16);   // the integer widths declared
+        if (dims.dk == 128 && dims.widths != 0 && (wi & ~W248) == 0)
+            return dims.pivots ? launch_decode<128, false, true, false, true, W248>(a, st)
+                               : launch_decode<128, false, false, false, true, W248>(a, st);
+        if (dims.dk == 128 && dims.widths != 0 && (wi & ~W468) == 0)
+            return dims.pivots ? launch_decode<128, false, true, false, true, W468>(a, st)
+                               : launch_decode<128, false, false, false, true, W468>(a, st);
         if (dims.pivots)
             return dims.dk == 128 ? launch_decode<128, false, true, false, true>(a, st)
                                   : launch_decode<64, false, true, false, true>(a, st);

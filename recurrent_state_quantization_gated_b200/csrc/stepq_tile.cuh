@@ -123,6 +123,17 @@ __device__ __forceinline__ int sort_head_rows(const uint8_t* bits_h, uint32_t* h
     return sort_head_rows_w<D, kPiv>(head_widths<D>(bits_h, lane), hmeta, hslot, lane, flags);
 }
 
+// The row widths that a per-row (mixed) code path handles: every width (kW = 0), or the widths
+// of the bit mask kW (bit b for width b; width 16, the FP16 pivot rows, is governed by kPiv).
+// The lowest declared width, the fallback, also takes the rows of any undeclared width.
+template <int kW>
+struct WidthSet {
+    static constexpr bool has(int b) { return kW == 0 || ((kW >> b) & 1) != 0; }
+    static constexpr int fallback =
+        kW == 0 ? 2 : ((kW >> 2) & 1) ? 2 : ((kW >> 4) & 1) ? 4 : ((kW >> 6) & 1) ? 6 : 8;
+    static constexpr bool tested(int b) { return has(b) && b != fallback; }   // its own branch
+};
+
 // Eight consecutive per-column values (columns 8cl .. 8cl+7) as four pairs.
 __device__ __forceinline__ void load_cols8(const float* src, int cl, float2 out[4]) {
     const float4 a = *reinterpret_cast<const float4*>(src + 8 * cl);
@@ -193,35 +204,29 @@ __device__ __forceinline__ void phase6_uniform(const uint32_t* meta, uint8_t* ou
     }
 }
 
-template <int D, bool kPiv>
+template <int D, bool kPiv, int kW = 0>
 __device__ __forceinline__ void phase6_mixed(const uint32_t* meta, uint8_t* out, int warp, int lane,
                                              const float2 Z[][4], const float2 f[4], const float* colc) {
     using M = DMap<D>;
+    using WS = WidthSet<kW>;
     const int cl = M::col_lane(lane);
     float2 cc[4] = {};
     if constexpr (kPiv) load_cols8(colc, cl, cc);
 #pragma unroll
     for (int r = 0; r < M::RPT; ++r) {
         const uint32_t mt = meta[M::row(warp, lane, r)];
-        switch ((mt >> 8) & 0xFF) {
-            case 8: phase6_row<D, 8>(out, mt, cl, Z[r], f); break;
-            case 6: phase6_row<D, 6>(out, mt, cl, Z[r], f); break;
-            case 4: phase6_row<D, 4>(out, mt, cl, Z[r], f); break;
-            default:
-                if constexpr (kPiv) {
-                    if (((mt >> 8) & 0xFF) == 16) {
-                        phase6_pivot_row<D>(out, mt, cl, Z[r], cc);
-                        break;
-                    }
-                }
-                phase6_row<D, 2>(out, mt, cl, Z[r], f);
-                break;
-        }
+        const int bw = (mt >> 8) & 0xFF;
+        if constexpr (WS::tested(8)) if (bw == 8) { phase6_row<D, 8>(out, mt, cl, Z[r], f); continue; }
+        if constexpr (WS::tested(6)) if (bw == 6) { phase6_row<D, 6>(out, mt, cl, Z[r], f); continue; }
+        if constexpr (WS::tested(4)) if (bw == 4) { phase6_row<D, 4>(out, mt, cl, Z[r], f); continue; }
+        if constexpr (WS::tested(2)) if (bw == 2) { phase6_row<D, 2>(out, mt, cl, Z[r], f); continue; }
+        if constexpr (kPiv) if (bw == 16) { phase6_pivot_row<D>(out, mt, cl, Z[r], cc); continue; }
+        phase6_row<D, WS::fallback>(out, mt, cl, Z[r], f);
     }
 }
 
 // kPiv: the pivot-capable instantiation (width-16 rows handled); without it the code is leaner.
-template <int D, bool kPiv>
+template <int D, bool kPiv, int kW = 0>
 __device__ __forceinline__ void phase6(const uint32_t* meta, uint8_t* out, int warp, int lane, int ww,
                                        const float2 Z[][4], const float2 f[4], const float* colc) {
     switch (ww) {
@@ -236,7 +241,7 @@ __device__ __forceinline__ void phase6(const uint32_t* meta, uint8_t* out, int w
                     break;
                 }
             }
-            phase6_mixed<D, kPiv>(meta, out, warp, lane, Z, f, colc);
+            phase6_mixed<D, kPiv, kW>(meta, out, warp, lane, Z, f, colc);
             break;
     }
 }
@@ -246,7 +251,7 @@ __device__ __forceinline__ void phase6(const uint32_t* meta, uint8_t* out, int w
 // sm.ak[kb][slot].z, c_j in sm.colc); with kUpdate the last token's rank-1 update
 // Y += (k_i/alpha_i)(u_j/c_j) (k/alpha in sm.ak[kb][slot].xy, u/c in sm.colb) is applied first.
 // r_out and c_out point at the scales of tile `tile`, out at the tile's packed bytes.
-template <int D, bool kPiv, bool kUpdate, class Sm>
+template <int D, bool kPiv, bool kUpdate, int kW = 0, class Sm>
 __device__ __forceinline__ void refit_pack(Sm& sm, const uint32_t* meta, float2 (&Z)[DMap<D>::RPT][4], int ww, int kb,
                                            int tile, uint16_t* r_out, uint16_t* c_out, uint8_t* out) {
     using M = DMap<D>;
@@ -407,7 +412,7 @@ __device__ __forceinline__ void refit_pack(Sm& sm, const uint32_t* meta, float2 
     {
         float2 f[4];
         load_cols8(sm.colb, cl, f);
-        phase6<D, kPiv>(meta, out, warp, lane, ww, Z, f, sm.colc);
+        phase6<D, kPiv, kW>(meta, out, warp, lane, ww, Z, f, sm.colc);
     }
 }
 

@@ -46,6 +46,11 @@ class Layout:
         """1 when some head's key rows have different widths (a row-level allocation)."""
         return int((self.bits != self.bits[:, :1]).any())
 
+    @property
+    def widths(self) -> int:
+        """Bit mask of the row widths the bit map holds (bit b for width b)."""
+        return api.width_mask(self.bits)
+
 
 class QuantizedState:
     """Packed states of B sequences x H heads (one layer)."""
@@ -73,7 +78,8 @@ class QuantizedState:
         L = self.layout
         _, _, _, o = api.stepq_decode_step(q, k, v, beta, gate, L.bits_dev, self.w, L.head_off_dev,
                                            L.bytes_per_seq, self.packed, self.r, self.c,
-                                           self.packed, self.r, self.c, o, pivots=L.pivots, mixed=L.mixed)
+                                           self.packed, self.r, self.c, o, pivots=L.pivots, mixed=L.mixed,
+                                           widths=L.widths)
         return o
 
     def nbytes(self) -> int:

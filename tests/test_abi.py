@@ -117,6 +117,11 @@ def test_device_calls_validate_before_touching_cuda():
     assert rc == _lib.STEPQ_EUNSUPPORTED
     # empty batch is a no-op that never launches
     assert lib.stepq_decode_step(_dims(B=0), *([P()] * 8), 4096, *([P()] * 7), None) == _lib.STEPQ_OK
+    # a widths mask with a bit other than 2, 4, 6, 8, 16
+    d = _dims()
+    d.mixed, d.widths = 1, (1 << 4) | (1 << 5)
+    rc = lib.stepq_decode_step(d, *([P()] * 8), 4096, *([P()] * 7), None)
+    assert rc == _lib.STEPQ_EINVAL and b"widths" in lib.stepq_last_error()
     # unsupported width in a layout
     bits = np.full((1, 64), 3, dtype=np.uint8)
     with pytest.raises(_lib.StepqError) as e:

@@ -209,10 +209,37 @@ def test_mixed_and_width_specialised_paths_agree(pivots):
     args = (td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w), dev(head_off), bps,
             dev(packed), dev(r, torch.float16), dev(c, torch.float16))
     a = api.stepq_decode_step(*args, mixed=0)
-    b = api.stepq_decode_step(*args, mixed=1)
+    b = api.stepq_decode_step(*args, mixed=1, widths=0)
     torch.cuda.synchronize()
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("widths,pivots", [((2, 4, 8), 0), ((4, 6, 8), 0), ((4, 6, 8), 9), ((4, 8), 0)])
+def test_declared_width_sets_agree_with_the_generic_path(widths, pivots):
+    """A mixed launch whose bit map holds only {2, 4, 8} or only {4, 6, 8} (the 4-bit and
+    6-bit row allocations) runs per-row code for those widths alone; its results are the bits of
+    the generic per-row path (widths undeclared)."""
+    import torch
+    from recurrent_state_quantization_gated_b200 import api
+    d, B, H = 128, 3, 5
+    wl = synth.workload(1, B=B, H=H, d=d, seed=31)
+    S0 = synth.initial_state(wl)
+    bits = with_pivots(synth.random_bits(H, d, choices=widths, seed=8), pivots, 9)
+    w = synth.random_weights(H, d, seed=6)
+    r, c = oracle.fit_scales(S0, w, bits)
+    packed = oracle.pack_state(S0, bits, r, c)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    td = tokens_dev(synth.tokens(wl, 1))
+    args = (td["q"], td["k"], td["v"], td["beta"], td["gate"], dev(bits), dev(w), dev(head_off), bps,
+            dev(packed), dev(r, torch.float16), dev(c, torch.float16))
+    mask = api.width_mask(bits)
+    a = api.stepq_decode_step(*args, mixed=1, widths=0)
+    b = api.stepq_decode_step(*args, mixed=1, widths=mask)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    assert api.stepq_read_device_flags() == 0
 
 
 def test_a_wait_that_runs_out_is_reported_and_the_context_stays_usable():

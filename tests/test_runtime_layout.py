@@ -1,7 +1,8 @@
 """Host logic of runtime.Layout, on the CPU: the per-head byte offsets and bytes per sequence of
 a bit map equal the oracle's layout (rows of (d/8) b_i bytes, heads in order), and the two flags
 that select the decode step's kernel instantiation are read correctly from the map: `pivots`
-(some row has width 16) and `mixed` (some head's rows have different widths)."""
+(some row has width 16), `mixed` (some head's rows have different widths) and `widths` (the mask
+of the widths present, bit b for width b)."""
 import numpy as np
 import pytest
 
@@ -31,5 +32,6 @@ def test_layout_and_flags(d, kind):
     assert L.H == H and L.d == d
     assert L.pivots == int(kind in ("mixed_pivots", "head_pivot"))
     assert L.mixed == int(kind in ("mixed", "mixed_pivots"))
+    assert L.widths == sum(1 << int(b) for b in np.unique(bits))
     np.testing.assert_array_equal(L.bits_dev.numpy(), bits)
     np.testing.assert_array_equal(L.head_off_dev.numpy(), head_off)
