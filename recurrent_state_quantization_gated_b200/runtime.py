@@ -129,12 +129,15 @@ def mean_log_retention(gate) -> np.ndarray:
 
 def lifetime(ell, horizon: int = LIFETIME_HORIZON) -> np.ndarray:
     """L_u = sum over 0 <= j < horizon of exp(2 j ell_u) (App. A.3): the squared error a unit
-    keeps over the horizon per unit injected once. Geometric series in closed form,
-    expm1(2 horizon ell) / expm1(2 ell), which is horizon at ell = 0."""
+    keeps over the horizon per unit injected once. Summed term by term in increasing j, in
+    float64: the discrete allocation compares lifetime-weighted costs of nearly equal size, so
+    the series is evaluated in its plain order rather than through a closed form whose last bits
+    differ."""
     x = 2.0 * np.asarray(ell, dtype=np.float64)
-    with np.errstate(divide="ignore", invalid="ignore"):
-        L = np.expm1(horizon * x) / np.expm1(x)
-    return np.where(x == 0.0, float(horizon), L)
+    total = np.zeros_like(x)
+    for j in range(int(horizon)):
+        total += np.exp(j * x)
+    return total
 
 
 def calibrate(alloc: str, candidates, nominal_bits: int, S0: torch.Tensor, calib: dict, n_pivots: int = 0,

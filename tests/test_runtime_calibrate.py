@@ -62,3 +62,14 @@ def test_runtime_lifetime_closed_form_equals_the_oracle_sum(horizon):
     np.testing.assert_allclose(runtime.mean_log_retention(gate), oracle.mean_log_retention(gate), rtol=1e-15)
     np.testing.assert_allclose(runtime.mean_log_retention(torch.from_numpy(gate)),
                                oracle.mean_log_retention(gate), rtol=1e-15)
+
+
+def test_lifetime_weights_are_bit_identical_to_the_oracles():
+    """The runtime's lifetime weights L_u (App. A.3) equal the oracle's bit for bit over gates
+    from 0 to 1 (both sum the series term by term), so the lifetime-weighted costs J the two
+    allocators compare are the same numbers."""
+    import oracle
+    rng = np.random.default_rng(11)
+    g = np.concatenate([[1.0, 0.999, 0.9, 1e-30], rng.uniform(0.0, 1.0, 4000), 1.0 - rng.exponential(1e-3, 96)])
+    ell = np.log(np.clip(g, 1e-30, 1.0))
+    np.testing.assert_array_equal(runtime.lifetime(ell), oracle.lifetime(ell))
