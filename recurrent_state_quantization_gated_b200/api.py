@@ -111,10 +111,15 @@ def width_mask(bits) -> int:
 
 def _widths(bits, widths, mixed):
     """The widths field of a decode call: as given, else read from the bit map when the launch
-    takes the per-row path (mixed), else 0 (not needed)."""
+    takes the per-row path (mixed) -- except while a CUDA graph is being captured, where no
+    device read is possible and 0 (undeclared: the generic per-row code, same results) is used."""
     if widths is not None:
         return int(widths)
-    return width_mask(bits) if mixed else 0
+    if not mixed:
+        return 0
+    if isinstance(bits, torch.Tensor) and bits.is_cuda and torch.cuda.is_current_stream_capturing():
+        return 0
+    return width_mask(bits)
 
 
 def _has_pivots(bits, pivots):

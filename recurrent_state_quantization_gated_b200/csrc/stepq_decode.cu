@@ -87,7 +87,8 @@ struct DecodeSmem {
     alignas(16) uint32_t hmeta[CH][D];
     alignas(16) uint16_t hslot[CH][D];   // by key row: slot | width << 8
     int htag[CH];                   // head held by each cache entry (-1: none)
-    int htot[CH];                   // the tile's bytes under the head's bit map
+    int hok[CH];                    // the head's byte range holds its tile under the bit map
+    long long hoff[CH];             // head_off of the head
     // Per slot of the tile being decoded.
     alignas(16) float4 kq[D];       // alpha k, alpha k, alpha q, alpha q   (alpha = g r 2^(8-b))
     alignas(16) float4 ak[2][D];    // k/alpha, k/alpha, alpha, alpha (two tokens of a chunk)
@@ -324,22 +325,22 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
         const auto& st = sm.stage[s];
         const int h = tile % a.H, he = h % CH;
         const uint32_t* meta = sm.hmeta[he];
-        const int64_t tile_base = static_cast<int64_t>(tile / a.H) * a.bytes_per_seq + a.head_off[h];
         if (sm.htag[he] != h) {                     // every warp sees the same tag: uniform branch
             __syncthreads();                        // nobody still reads the entry
             if (warp == 0) {
                 const int tot = sort_head_rows<D, kPiv>(a.bits + static_cast<int64_t>(h) * D, sm.hmeta[he],
                                                         sm.hslot[he], lane, &g_stepq_flags);
                 if (lane == 0) {
+                    int64_t ho, hn;
+                    sm.hok[he] = tile_range_ok(a.head_off, a.H, a.bytes_per_seq, h, tot, 2 * D * D, &g_stepq_flags, &ho, &hn);
+                    sm.hoff[he] = ho;
                     sm.htag[he] = h;
-                    sm.htot[he] = tot;
                 }
             }
             __syncthreads();
         }
-        // The head's byte range must hold the tile under the bit map (same answer in every thread).
-        const bool tile_ok = tile_range_ok(a.head_off, a.H, a.bytes_per_seq, h, sm.htot[he], 2 * D * D, nullptr);
-        if (!tile_ok && tid == 0) atomicOr(&g_stepq_flags, kFlagBadLayout);
+        const bool tile_ok = sm.hok[he];
+        const int64_t tile_base = static_cast<int64_t>(tile / a.H) * a.bytes_per_seq + sm.hoff[he];
         const bool ok = mbar_wait_bounded(&sm.full[s], parity, kWaitLimitNs, &g_stepq_flags);
 
         // A prefill chunk's token 1: its inputs are loaded now, behind the unpack (rows by the
@@ -590,8 +591,10 @@ decode_kernel(const DecodeArgs a) {
             const int tot = sort_head_rows<D, kPiv>(a.bits + static_cast<int64_t>(h) * D, sm.hmeta[h % CH],
                                                     sm.hslot[h % CH], lane, &g_stepq_flags);
             if (lane == 0) {
+                int64_t ho, hn;
+                sm.hok[h % CH] = tile_range_ok(a.head_off, a.H, a.bytes_per_seq, h, tot, 2 * D * D, &g_stepq_flags, &ho, &hn);
+                sm.hoff[h % CH] = ho;
                 sm.htag[h % CH] = h;
-                sm.htot[h % CH] = tot;
             }
         }
     }

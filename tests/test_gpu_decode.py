@@ -272,3 +272,36 @@ def test_a_wait_that_runs_out_is_reported_and_the_context_stays_usable():
     ref = oracle.decode_step(tok, bits, w, packed, r, c)
     compare_decode((p_g.cpu().numpy(), host_half(r_g), host_half(c_g), o_g.cpu().numpy()), ref, bits, wl.d, wl.B)
     assert api.stepq_read_device_flags() == 0
+
+
+def test_a_mixed_launch_without_declared_widths_can_be_captured_in_a_graph():
+    """Inside CUDA-graph capture the binding cannot read the bit map back, so a mixed launch whose
+    widths are not declared runs the generic per-row code; its results equal the declared launch's."""
+    import torch
+    from recurrent_state_quantization_gated_b200 import api
+    d, B, H = 128, 2, 4
+    wl = synth.workload(1, B=B, H=H, d=d, seed=41)
+    S0 = synth.initial_state(wl)
+    bits = synth.random_bits(H, d, choices=(2, 4, 8), seed=12)
+    w = synth.random_weights(H, d, seed=13)
+    r, c = oracle.fit_scales(S0, w, bits)
+    packed = oracle.pack_state(S0, bits, r, c)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    td = tokens_dev(synth.tokens(wl, 0))
+    bits_d, w_d, ho_d = dev(bits), dev(w), dev(head_off)
+    ref = api.stepq_decode_step(td["q"], td["k"], td["v"], td["beta"], td["gate"], bits_d, w_d, ho_d, bps, dev(packed),
+                                dev(r, torch.float16), dev(c, torch.float16), pivots=0, mixed=1,
+                                widths=api.width_mask(bits))
+    pk, rr, cc = dev(packed), dev(r, torch.float16), dev(c, torch.float16)
+    out = (torch.empty_like(pk), torch.empty_like(rr), torch.empty_like(cc),
+           torch.empty((B, H, d), dtype=torch.float32, device="cuda"))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        api.stepq_decode_step(td["q"], td["k"], td["v"], td["beta"], td["gate"], bits_d, w_d, ho_d, bps, pk, rr, cc,
+                              *out, pivots=0, mixed=1)
+    g.replay()
+    torch.cuda.synchronize()
+    for x, y in zip(ref, out):
+        assert torch.equal(x, y)
