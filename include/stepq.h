@@ -153,11 +153,13 @@ STEPQ_API int stepq_decode_step(stepq_dims dims, const uint16_t* q, const uint16
        supported shape and chunk length; chunk = 1 is bit-identical to stepq_decode_step);
      stepq_prefill_chunk_wy: the chunked WY/UT form on the tensor cores (§2.1's affine form
        unrolled over the chunk: one unit lower triangular solve and dense products per tile).
-       Requires dk = dv = 128, scalar gates, no FP16 pivot rows and
-       1 <= chunk <= STEPQ_WY_MAX_CHUNK; otherwise STEPQ_EUNSUPPORTED. Products run on bf16
-       operands (q, k, v and the integer codes exactly; computed operands split into two or
-       three bf16 parts) with fp32 accumulation: the boundary state carries fp32 precision, the
-       readouts about 1e-6 relative.
+       Requires dk = dv = 128, no FP16 pivot rows and 1 <= chunk <= STEPQ_WY_MAX_CHUNK;
+       otherwise STEPQ_EUNSUPPORTED. Scalar and channel gates (gates in [0, 1]). Products run on
+       bf16 operands (q, k, v and the integer codes exactly; computed operands split into two or
+       three bf16 parts) with fp32 accumulation; under channel gates the gate-weighted token-pair
+       products (the triangular system's and the readouts' intra-chunk weights) are formed on
+       the CUDA cores in fp32. The boundary
+       state carries fp32 precision, the readouts about 1e-6 relative.
    stepq_prefill_chunk takes the WY form where it applies and the sequential form elsewhere. */
 #define STEPQ_WY_MAX_CHUNK 64
 STEPQ_API int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,

@@ -729,18 +729,6 @@ extern "C" int stepq_prefill_chunk_seq(stepq_dims dims, int chunk, const uint16_
     return dims.dk == 128 ? launch_decode<128, false, false, true>(a, st) : launch_decode<64, false, false, true>(a, st);
 }
 
-extern "C" int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
-                                   const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,
-                                   const float* w, const int64_t* head_off, int64_t bytes_per_seq,
-                                   const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,
-                                   uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream) {
-    const bool wy = dims.dk == 128 && dims.dv == 128 && dims.gate_per_channel == 0 && dims.pivots == 0 && chunk >= 1 &&
-                    chunk <= STEPQ_WY_MAX_CHUNK;
-    return (wy ? stepq_prefill_chunk_wy : stepq_prefill_chunk_seq)(dims, chunk, q, k, v, beta, gate, bits, w, head_off,
-                                                                   bytes_per_seq, packed_in, r_in, c_in, packed_out,
-                                                                   r_out, c_out, o, stream);
-}
-
 extern "C" int stepq_decode_step_split(stepq_dims dims, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                        const float* beta, const float* gate, const uint8_t* bits, const float* w,
                                        const int64_t* head_off, int64_t bytes_per_seq, const uint8_t* packed_in,

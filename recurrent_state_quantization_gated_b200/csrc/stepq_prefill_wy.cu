@@ -22,6 +22,24 @@
 // diagonal blocks by substitution, then block rows) on the CUDA cores. The boundary state then
 // runs through the same refit and pack as the fused decode step (steps 4-6 of Table C2).
 //
+// Channel gates (one gate per key channel, D_t = diag(g_t), as in Kimi Delta Attention): with
+// lambda_ti the running log2 of channel i's gate product and R_tsi = prod_{s < tau <= t} g_tau,i,
+// the same rearrangement holds with the gate factors inside the channel sums:
+//   L_ts = beta_t sum_i k_ti k_si R_tsi,   P_ts = sum_i q_ti k_si R_tsi (s <= t),
+//   U    = T diag(beta) V - T diag(beta) (K o 2^lambda) S0,
+//   O    = (Q o 2^lambda) S0 + P U,
+//   S_C  = diag(2^lambda_C) S0 + (K o 2^(lambda_C - lambda))^T U.
+// L and P are formed on the CUDA cores in fp32 through a hierarchy of reference tokens: the pairs
+// whose token indices first differ in bit l are the (upper half, lower half) pairs of the aligned
+// blocks of 2^(l+1) tokens, and with the last token of the lower half as reference R_tsi is the
+// product of a factor of t (the gates from the upper half's start to t) and a factor of s (the
+// gates after s to the lower half's end), both at most 1: no partial product can overflow,
+// whatever the gates. The gate-scaled operands (K o 2^lambda, Q o 2^lambda, K o 2^(lambda_C -
+// lambda)) are not exact in bf16, so both operands of W = T diag(beta) (K o 2^lambda) and of the
+// boundary-state product are split in three parts, of which the six largest part products are
+// accumulated (the three largest leave about 0.5 % of 8-bit column scales off those of a float64
+// evaluation; six leave none, in a NumPy emulation of this arithmetic).
+//
 // One CTA per SM (the operands of a tile take 224 KB of shared memory), 256 threads, 512 TMEM
 // columns; tiles are dealt round-robin. With one CTA of 8 warps per SM the phases' code must
 // stay small: loops whose bodies are large are kept rolled (instruction-cache misses were the
@@ -29,8 +47,6 @@
 // engine while the current tile is computed; q, k and v arrive through 16-byte asynchronous
 // copies straight into the tensor cores' operand layout.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "stepq_device.cuh"
 #include "stepq_internal.h"
@@ -90,6 +106,8 @@ struct Small {
     alignas(16) float icol[D];       // 1 / c_j
     alignas(16) float beta[C];
     alignas(16) float l2g[C];        // log2 gamma_t (a zero gate counts as 2^-64)
+    alignas(16) float lamC[D];       // channel gates: lambda_C,i, the chunk's log2 gate product
+    alignas(16) float lcarry[D];     // channel gates: lambda of the first 32 tokens (scan carry)
     alignas(8) uint64_t bar_mma;
     alignas(8) uint64_t bar_sc;      // the last round's boundary-state product, committed apart
     alignas(8) uint64_t bar_codes;
@@ -102,16 +120,26 @@ constexpr uint32_t OFF_KQ = 0;            // bf16 [K; Q]: rows t (k) and 64 + t 
 constexpr uint32_t OFF_V = 32768;         // bf16 V: rows t, K-major over d
 constexpr uint32_t OFF_Z = 49152;         // bf16 codes Z: rows i, K-major over j
 constexpr uint32_t OFF_CODES = 81920;     // the tile's packed codes (bulk copy)
-constexpr uint32_t OFF_W = 98304;         // 128 KB work region, laid out per phase (see the kernel)
-constexpr uint32_t OFF_SMALL = 229376;
+constexpr uint32_t OFF_W = 98304;         // 127 KB work region, laid out per phase (see the kernel)
+constexpr uint32_t OFF_SMALL = OFF_W + 127 * 1024;
+constexpr int GLD = D + 4;                // padded row (floats) of the [token][channel] fp32 arrays
+constexpr int PLD = C + 4;                // padded row (floats) of P
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + sizeof(Small);
 static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
 static_assert(65536 + sizeof(FitScratch) <= OFF_SMALL - OFF_W, "refit work space");
 
 // TMEM columns (512 allocated): G = [K;Q] K^T | W, later S_C | U_v | [W S0; gamma Q S0 + P U/c]
-constexpr uint32_t TM_G = 0, TM_W = 64, TM_U = 192, TM_S = 320;
+// | channel gates: lambda. Under channel gates G holds no product: lanes 0-63 keep lambda_ti
+// (lane t, column i for i < 64; columns TM_LAM + i - 64 for the others) and lanes 64-127 keep P
+// (lane 64 + t, column s).
+constexpr uint32_t TM_G = 0, TM_W = 64, TM_U = 192, TM_S = 320, TM_LAM = 448;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// The six largest products of two operands each split in three bf16 parts (high, middle, low):
+// part kPartA[n] of the first with part kPartB[n] of the second.
+__device__ constexpr int kPartA[6] = {0, 0, 1, 0, 2, 1};
+__device__ constexpr int kPartB[6] = {0, 1, 0, 2, 0, 1};
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes)
@@ -187,6 +215,146 @@ __device__ __forceinline__ uint32_t tm_at(uint32_t tm, int warp, uint32_t col) {
     return umma::tmem_at(tm, 32 * (warp & 3), static_cast<int>(col));
 }
 
+// ---- channel gates -------------------------------------------------------------------------
+
+// TMEM column of lambda_ti for the 32 channels from i0 (a multiple of 32), lanes 0-63.
+__host__ __device__ constexpr uint32_t lam_col(int i0) {
+    return i0 < 64 ? TM_G + static_cast<uint32_t>(i0) : TM_LAM + static_cast<uint32_t>(i0 - 64);
+}
+
+__host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x >> 1); }
+
+// One level of the reference hierarchy: the operands SK (every token) and SQ (upper halves only,
+// compacted) of the pairs whose token indices first differ in bit LV. Thread (i, hh) holds the
+// gates gv and the packed bf16 k | q << 16 of channel i, tokens 32 hh to 32 hh + 31.
+//   upper half token t: factor = gates from the half's first token to t
+//   lower half token s: factor = gates after s to the half's last token (1 for the last)
+template <int LV>
+__device__ __forceinline__ void level_operands(const float (&gv)[32], const uint32_t (&kq)[32], int hh, int i,
+                                               float* SK, float* SQ) {
+    constexpr int h = 1 << LV;
+    float f = 1.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const bool up = LV == 5 ? hh != 0 : (j & h) != 0;
+        const bool start = LV == 5 ? j == 0 : (j & (h - 1)) == 0;
+        f = start ? gv[j] : f * gv[j];
+        if (up) {
+            const int t = 32 * hh + j;
+            SK[t * GLD + i] = __uint_as_float(kq[j] << 16) * f;
+            SQ[(((t >> (LV + 1)) << LV) | (t & (h - 1))) * GLD + i] = __uint_as_float(kq[j] & 0xFFFF0000u) * f;
+        }
+    }
+    float b = 1.0f;
+#pragma unroll
+    for (int j = 31; j >= 0; --j) {
+        const bool up = LV == 5 ? hh != 0 : (j & h) != 0;
+        const bool end = LV == 5 ? j == 31 : (j & (h - 1)) == h - 1;
+        if (end) b = 1.0f;
+        if (!up) SK[(32 * hh + j) * GLD + i] = __uint_as_float(kq[j] << 16) * b;
+        b *= gv[j];
+    }
+}
+
+// Butterfly over the CS lanes of a tile (consecutive lanes, CS a power of two): each step halves
+// the N values a lane holds, keeping the half its lane bit selects and adding the partner's copy
+// of it; once one value is left the remaining steps add it up.
+template <int NO, int CS, int O = 1, int N = NO>
+__device__ __forceinline__ void reduce_tile(float (&v)[NO], int c) {
+    if constexpr (O < CS) {
+        if constexpr (N > 1) {
+            const bool up = (c & O) != 0;
+#pragma unroll
+            for (int j = 0; j < N / 2; ++j) {
+                const float send = up ? v[j] : v[j + N / 2];
+                const float keep = up ? v[j + N / 2] : v[j];
+                v[j] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+            }
+            reduce_tile<NO, CS, 2 * O, N / 2>(v, c);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+            reduce_tile<NO, CS, 2 * O, 1>(v, c);
+        }
+    }
+}
+
+// The pair products of level LV: for t in the upper and s in the lower half of each aligned block
+// of 2^(LV+1) tokens, L_ts = beta_t sum_i SK_ti SK_si (into the sw64 layout) and
+// P_ts = sum_i SQ_t'i SK_si (into Pf). Pairs are dealt in TT x TT tiles, the 128 channels of a tile
+// split over CS consecutive lanes (strided by 4 CS floats, so the lanes of a tile read adjacent
+// 16-byte chunks), and the CS partial sums folded by reduce_tile.
+template <int LV>
+__device__ __forceinline__ void level_pairs(const float* SK, const float* SQ, const float* beta, float* Lf, float* Pf,
+                                            int tid) {
+    constexpr int h = 1 << LV;
+    constexpr int TT = LV >= 2 ? 4 : (LV == 1 ? 2 : 1);
+    constexpr int NB = h / TT;                      // t- (and s-) tile rows per half
+    constexpr int NTILE = (32 / h) * NB * NB;
+    constexpr int CS = NT / NTILE;
+    constexpr int NG = D / (4 * CS);                // float4 channel groups per lane
+    constexpr int NO = 2 * TT * TT;                 // L then P outputs of a tile
+    static_assert(CS >= 1 && CS <= 32 && NG >= 1, "level tiling");
+    const int tile = tid / CS, c = tid % CS;
+    const int seg = tile / (NB * NB), rr = tile % (NB * NB);
+    const int tb = rr / NB, sb = rr % NB;
+    const int t0 = 2 * h * seg + h + TT * tb, s0 = 2 * h * seg + TT * sb, q0 = h * seg + TT * tb;
+    float v[NO];
+#pragma unroll
+    for (int e = 0; e < NO; ++e) v[e] = 0.0f;
+#pragma unroll 2
+    for (int g = 0; g < NG; ++g) {
+        const int i = 4 * c + 4 * CS * g;
+        float4 kt[TT], qt[TT], ks[TT];
+#pragma unroll
+        for (int a = 0; a < TT; ++a) {
+            kt[a] = *reinterpret_cast<const float4*>(SK + (t0 + a) * GLD + i);
+            qt[a] = *reinterpret_cast<const float4*>(SQ + (q0 + a) * GLD + i);
+            ks[a] = *reinterpret_cast<const float4*>(SK + (s0 + a) * GLD + i);
+        }
+#pragma unroll
+        for (int a = 0; a < TT; ++a)
+#pragma unroll
+            for (int b = 0; b < TT; ++b) {
+                float& l = v[a * TT + b];
+                float& p = v[TT * TT + a * TT + b];
+                l = fmaf(kt[a].x, ks[b].x, l); l = fmaf(kt[a].y, ks[b].y, l);
+                l = fmaf(kt[a].z, ks[b].z, l); l = fmaf(kt[a].w, ks[b].w, l);
+                p = fmaf(qt[a].x, ks[b].x, p); p = fmaf(qt[a].y, ks[b].y, p);
+                p = fmaf(qt[a].z, ks[b].z, p); p = fmaf(qt[a].w, ks[b].w, p);
+            }
+    }
+    reduce_tile<NO, CS>(v, c);
+    constexpr int HS = ilog2(CS) < ilog2(NO) ? ilog2(CS) : ilog2(NO);   // halving steps taken
+    constexpr int NF = NO >> HS;                                         // values left per lane
+    if ((c >> HS) == 0) {
+        int base = 0;
+#pragma unroll
+        for (int k = 0; k < HS; ++k) base += ((c >> k) & 1) * (NO >> (k + 1));
+#pragma unroll
+        for (int j = 0; j < NF; ++j) {
+            const int e = base + j, f = e % (TT * TT);
+            const int t = t0 + f / TT, s = s0 + f % TT;
+            if (e < TT * TT)
+                Lf[sw64(t, s)] = beta[t] * v[j];
+            else
+                Pf[t * PLD + s] = v[j];
+        }
+    }
+}
+
+// The gates of a tile's tokens t < chunk into Gs (fp32 [token][channel], rows of GLD floats);
+// rows past the chunk are left as they are (the scans take them as 1).
+__device__ __forceinline__ void load_gates(const WyArgs& a, int tile, int tid, float* Gs) {
+    const int64_t T = a.num_tiles;
+#pragma unroll 1
+    for (int m = 0; m < 8; ++m) {
+        const int e = tid + NT * m;                  // 64 rows x 32 chunks of 16 bytes
+        const int row = e >> 5, ch = e & 31;
+        if (row < a.chunk) cp_async16(Gs + row * GLD + 4 * ch, a.gate + (static_cast<int64_t>(row) * T + tile) * D + 4 * ch, 16u);
+    }
+    cp_async_commit();
+}
+
 // The small inputs of a tile, loaded into registers one tile ahead: warp 0 the gates and betas
 // of tokens 2 lane and 2 lane + 1, warp 1 the head's row widths, threads < 128 r_i and c_i.
 struct Ahead {
@@ -198,6 +366,7 @@ struct Ahead {
     bool has_next;        // thread 0: there is a tile after this one
 };
 
+template <bool kChan>
 __device__ __forceinline__ Ahead load_ahead(const WyArgs& a, int tile, int tid, int warp, int lane) {
     Ahead n{1.0f, 1.0f, 0.0f, 0.0f, 0u, 0u, 0, 0u, false};
     const int64_t T = a.num_tiles;
@@ -212,8 +381,14 @@ __device__ __forceinline__ Ahead load_ahead(const WyArgs& a, int tile, int tid, 
     }
     if (warp == 0) {
         const int t0 = 2 * lane, t1 = t0 + 1;
-        if (t0 < a.chunk) { n.g0 = __ldg(a.gate + t0 * T + tile); n.b0 = __ldg(a.beta + t0 * T + tile); }
-        if (t1 < a.chunk) { n.g1 = __ldg(a.gate + t1 * T + tile); n.b1 = __ldg(a.beta + t1 * T + tile); }
+        if (t0 < a.chunk) {
+            if (!kChan) n.g0 = __ldg(a.gate + t0 * T + tile);
+            n.b0 = __ldg(a.beta + t0 * T + tile);
+        }
+        if (t1 < a.chunk) {
+            if (!kChan) n.g1 = __ldg(a.gate + t1 * T + tile);
+            n.b1 = __ldg(a.beta + t1 * T + tile);
+        }
     } else if (warp == 1) {
         n.widths = head_widths<D>(a.bits + static_cast<int64_t>(tile % a.H) * D, lane);
     }
@@ -250,6 +425,7 @@ __device__ __forceinline__ void issue_codes(const WyArgs& a, int tile, uint8_t* 
     if (bytes) bulk_load(dst, a.packed_in + static_cast<int64_t>(b) * a.bytes_per_seq + hoff, bytes, bar);
 }
 
+template <bool kChan>
 __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -264,6 +440,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
     //   D: U/c planes 0, 16 | U~ planes 32, 48, 64 | P planes 88, 96 (their MMA operand starts
     //      8 KB earlier: rows 0-63 there only reach TMEM lanes already consumed)
     //   E: X 0 | refit work space 64
+    // Under channel gates, before B: gates, then lambda, then SK 0 | SQ 34 | L 64 | P 104; in B the
+    // (K o 2^lambda) planes at 48, 64 and 102 (L and the G blocks are consumed by then).
     uint8_t* W = smem + OFF_W;
     auto h16 = [&](uint32_t kb) { return reinterpret_cast<uint16_t*>(W + 1024 * kb); };
     uint16_t* AT[3] = {h16(0), h16(16), h16(32)};
@@ -276,6 +454,11 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
     uint16_t* Pp[2] = {h16(88), h16(96)};
     float* X = reinterpret_cast<float*>(W);
     FitScratch& fit = *reinterpret_cast<FitScratch*>(W + 64 * 1024);
+    float* Gs = reinterpret_cast<float*>(W);
+    float* SK = reinterpret_cast<float*>(W);
+    float* SQ = reinterpret_cast<float*>(W + 34 * 1024);
+    float* Pf = reinterpret_cast<float*>(W + 104 * 1024);
+    uint16_t* KT[3] = {h16(48), h16(64), h16(102)};
 
     if (tid == 0) {
         mbar_init(&sm.bar_mma, 1);
@@ -317,7 +500,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             codes_pending = true;
         }
         load_tokens(a, blockIdx.x, tid, KQ, Vs);
-        nx = load_ahead(a, blockIdx.x, tid, warp, lane);
+        nx = load_ahead<kChan>(a, blockIdx.x, tid, warp, lane);
     }
 
     for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
@@ -326,6 +509,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
         const int next = tile + gridDim.x;
 
         // ---- A: tables, gates, scales, codes -----------------------------------------------
+        if constexpr (kChan) load_gates(a, tile, tid, Gs);
         if (warp == 1) {
             const int total = sort_head_rows_w<D, false>(nx.widths, sm.hmeta, sm.hslot, lane, a.flags);
             // A head range that cannot hold the tile under the bit map: the tile is computed on
@@ -382,21 +566,126 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
         to_tensor_core();
         if (tid == 0) {
             umma::fence_after_sync();
-            const uint32_t id = umma::idesc_bf16(128, 64, false, false);
+            if (!kChan) {
+                const uint32_t id = umma::idesc_bf16(128, 64, false, false);
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks)
-                umma::mma_bf16(tm + TM_G, umma::desc_kmajor(KQ, ks, D), umma::desc_kmajor(KQ, ks, D), id, ks > 0);
-            umma::commit(&sm.bar_mma);
+                for (int ks = 0; ks < D / 16; ++ks)
+                    umma::mma_bf16(tm + TM_G, umma::desc_kmajor(KQ, ks, D), umma::desc_kmajor(KQ, ks, D), id, ks > 0);
+                umma::commit(&sm.bar_mma);
+            }
             if (nx.has_next) {   // the codes buffer is free: fetch the next tile's
                 mbar_arrive_expect_tx(&sm.bar_codes, nx.codes_bytes);
                 if (nx.codes_bytes) bulk_load(codes, a.packed_in + nx.codes_src, nx.codes_bytes, &sm.bar_codes);
                 codes_pending = true;
             }
         }
-        if (!wait_mma()) break;
+        if constexpr (!kChan) {
+            if (!wait_mma()) break;
+        } else {
+            // ---- A': lambda, and L and P through the reference hierarchy ---------------------
+            const int i = tid & (D - 1), hh = tid >> 7;   // channel i, tokens 32 hh to 32 hh + 31
+            float gv[32];
+            uint32_t kq[32];
+            float lam = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int t = 32 * hh + j;
+                gv[j] = t < a.chunk ? Gs[t * GLD + i] : 1.0f;
+                kq[j] = static_cast<uint32_t>(KQ[umma::kmajor_off(t, i, D)]) |
+                        static_cast<uint32_t>(KQ[umma::kmajor_off(64 + t, i, D)]) << 16;
+                lam += log2f(fmaxf(gv[j], 0x1p-64f));
+                Gs[t * GLD + i] = lam;
+            }
+            if (hh == 0) sm.lcarry[i] = lam;
+            __syncthreads();
+            if (hh == 1) {
+                const float carry = sm.lcarry[i];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) Gs[(32 + j) * GLD + i] += carry;
+                sm.lamC[i] = lam + carry;
+            }
+            __syncthreads();
+            if (!(warp & 2)) {   // lambda into TMEM lanes 0-63 (lane t)
+                const int t = 32 * (warp & 1) + lane, hf = warp >> 2;
+#pragma unroll 1
+                for (int c32 = 0; c32 < 2; ++c32) {
+                    const int i0 = 64 * hf + 32 * c32;
+                    float v[32];
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const float4 x = *reinterpret_cast<const float4*>(Gs + t * GLD + i0 + 4 * q4);
+                        v[4 * q4] = x.x; v[4 * q4 + 1] = x.y; v[4 * q4 + 2] = x.z; v[4 * q4 + 3] = x.w;
+                    }
+                    umma::tmem_st32(tm_at(tm, warp, lam_col(i0)), v);
+                }
+            }
+            umma::fence_before_sync();
+            __syncthreads();
+            level_operands<5>(gv, kq, hh, i, SK, SQ);
+            __syncthreads();
+            level_pairs<5>(SK, SQ, sm.beta, Lf, Pf, tid);
+            __syncthreads();
+            level_operands<4>(gv, kq, hh, i, SK, SQ);
+            __syncthreads();
+            level_pairs<4>(SK, SQ, sm.beta, Lf, Pf, tid);
+            __syncthreads();
+            level_operands<3>(gv, kq, hh, i, SK, SQ);
+            __syncthreads();
+            level_pairs<3>(SK, SQ, sm.beta, Lf, Pf, tid);
+            __syncthreads();
+            level_operands<2>(gv, kq, hh, i, SK, SQ);
+            __syncthreads();
+            level_pairs<2>(SK, SQ, sm.beta, Lf, Pf, tid);
+            __syncthreads();
+            level_operands<1>(gv, kq, hh, i, SK, SQ);
+            __syncthreads();
+            level_pairs<1>(SK, SQ, sm.beta, Lf, Pf, tid);
+            __syncthreads();
+            level_operands<0>(gv, kq, hh, i, SK, SQ);
+            __syncthreads();
+            level_pairs<0>(SK, SQ, sm.beta, Lf, Pf, tid);
+            {   // P_tt = q_t.k_t; zeros on and above the diagonal of L's 16 x 16 diagonal blocks
+                const int t = tid >> 2, cg = tid & 3;
+                float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const uint4 kb = *reinterpret_cast<const uint4*>(KQ + umma::kmajor_off(t, 32 * cg + 8 * m, D));
+                    const uint4 qb = *reinterpret_cast<const uint4*>(KQ + umma::kmajor_off(64 + t, 32 * cg + 8 * m, D));
+                    const uint32_t kw[4] = {kb.x, kb.y, kb.z, kb.w}, qw[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        acc0 = fmaf(__uint_as_float(qw[p] << 16), __uint_as_float(kw[p] << 16), acc0);
+                        acc1 = fmaf(__uint_as_float(qw[p] & 0xFFFF0000u), __uint_as_float(kw[p] & 0xFFFF0000u), acc1);
+                    }
+                }
+                float acc = acc0 + acc1;
+                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                if (cg == 0) Pf[t * PLD + t] = acc;
+                const int blk = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (c4 + e >= r) Lf[sw64(16 * blk + r, 16 * blk + c4 + e)] = 0.0f;
+            }
+            __syncthreads();
+            if (warp & 2) {   // P into TMEM lanes 64-127 (lane 64 + t, column s)
+                const int t = 32 * (warp & 1) + lane, hf = warp >> 2;
+                float v[32];
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 x = *reinterpret_cast<const float4*>(Pf + t * PLD + 32 * hf + 4 * q4);
+                    v[4 * q4] = x.x; v[4 * q4 + 1] = x.y; v[4 * q4 + 2] = x.z; v[4 * q4 + 3] = x.w;
+                }
+                umma::tmem_st32(tm_at(tm, warp, TM_G + 32 * hf), v);
+            }
+            umma::fence_before_sync();
+            __syncthreads();
+            umma::fence_after_sync();
+        }
 
         // ---- B: L, T = (I + L)^-1, and the [T diag(beta); T diag(beta gamma)] planes ---------
-        if (warp < 2) {   // lanes 0-63: row t of K K^T
+        if (warp < 2) {   // lanes 0-63: row t of K K^T (under channel gates L is already formed)
+          if constexpr (!kChan) {
             const int t = tid;
             const float lt = sm.l2g[t], bt = sm.beta[t];
 #pragma unroll 1
@@ -414,6 +703,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                     *reinterpret_cast<float4*>(Lf + sw64(t, s0)) = make_float4(l[0], l[1], l[2], l[3]);
                 }
             }
+          }
         } else {   // T above the diagonal blocks is zero
             for (int e = tid - 64; e < 6 * 64; e += NT - 64) {
                 const int blk = e >> 6, rr = (e >> 2) & 15, cq = e & 3;
@@ -497,7 +787,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             float x[8];
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
-                const float f = row < 64 ? sm.beta[s0 + p] : sm.beta[s0 + p] * ex2(sm.l2g[s0 + p]);
+                const float f = row < 64 || kChan ? sm.beta[s0 + p] : sm.beta[s0 + p] * ex2(sm.l2g[s0 + p]);
                 x[p] = tv[p] * f;
             }
             uint4 hi, mid, lo;
@@ -506,18 +796,60 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             *reinterpret_cast<uint4*>(AT[1] + umma::kmajor_off(row, s0, C)) = mid;
             *reinterpret_cast<uint4*>(AT[2] + umma::kmajor_off(row, s0, C)) = lo;
         }
+        if constexpr (kChan) {   // the planes of K o 2^lambda (rows t, channels i), lanes 0-63 of lambda
+            if (!(warp & 2)) {
+                const int t = 32 * (warp & 1) + lane, hf = warp >> 2;
+#pragma unroll 1
+                for (int c32 = 0; c32 < 2; ++c32) {
+                    const int i0 = 64 * hf + 32 * c32;
+                    float lv[32];
+                    umma::tmem_ld32(tm_at(tm, warp, lam_col(i0)), lv);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 kb = *reinterpret_cast<const uint4*>(KQ + umma::kmajor_off(t, i0 + 8 * q, D));
+                        const uint32_t kw[4] = {kb.x, kb.y, kb.z, kb.w};
+                        float x[8];
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            x[2 * p] = __uint_as_float(kw[p] << 16) * ex2(lv[8 * q + 2 * p]);
+                            x[2 * p + 1] = __uint_as_float(kw[p] & 0xFFFF0000u) * ex2(lv[8 * q + 2 * p + 1]);
+                        }
+                        uint4 hi, mid, lo;
+                        split8x3(x, hi, mid, lo);
+                        *reinterpret_cast<uint4*>(KT[0] + umma::kmajor_off(t, i0 + 8 * q, D)) = hi;
+                        *reinterpret_cast<uint4*>(KT[1] + umma::kmajor_off(t, i0 + 8 * q, D)) = mid;
+                        *reinterpret_cast<uint4*>(KT[2] + umma::kmajor_off(t, i0 + 8 * q, D)) = lo;
+                    }
+                }
+            }
+        }
         to_tensor_core();
         if (tid == 0) {   // [T''; T'] K (W = T' K in lanes 64-127) and [T''; T'] V (U_v in lanes 0-63)
             umma::fence_after_sync();
             const uint32_t id = umma::idesc_bf16(128, 128, false, true);
+            if constexpr (!kChan) {
 #pragma unroll
-            for (int p = 0; p < 3; ++p)
+                for (int p = 0; p < 3; ++p)
 #pragma unroll
-                for (int ks = 0; ks < C / 16; ++ks) {
-                    const uint64_t da = umma::desc_kmajor(AT[p], ks, C);
-                    umma::mma_bf16(tm + TM_W, da, umma::desc_mnmajor(KQ, ks, D), id, p > 0 || ks > 0);
-                    umma::mma_bf16(tm + TM_U, da, umma::desc_mnmajor(Vs, ks, D), id, p > 0 || ks > 0);
-                }
+                    for (int ks = 0; ks < C / 16; ++ks) {
+                        const uint64_t da = umma::desc_kmajor(AT[p], ks, C);
+                        umma::mma_bf16(tm + TM_W, da, umma::desc_mnmajor(KQ, ks, D), id, p > 0 || ks > 0);
+                        umma::mma_bf16(tm + TM_U, da, umma::desc_mnmajor(Vs, ks, D), id, p > 0 || ks > 0);
+                    }
+            } else {   // U_v from the three parts of T diag(beta); W from six part products with K o 2^lambda
+#pragma unroll
+                for (int p = 0; p < 3; ++p)
+#pragma unroll
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        umma::mma_bf16(tm + TM_U, umma::desc_kmajor(AT[p], ks, C), umma::desc_mnmajor(Vs, ks, D), id,
+                                       p > 0 || ks > 0);
+#pragma unroll
+                for (int pq = 0; pq < 6; ++pq)
+#pragma unroll
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        umma::mma_bf16(tm + TM_W, umma::desc_kmajor(AT[kPartA[pq]], ks, C),
+                                       umma::desc_mnmajor(KT[kPartB[pq]], ks, D), id, pq > 0 || ks > 0);
+            }
             umma::commit(&sm.bar_mma);
         }
         if (!wait_mma()) break;
@@ -545,7 +877,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                         *reinterpret_cast<uint4*>(WQ[2] + umma::kmajor_off(t, i0, D)) = lo;
                     }
                 }
-            } else {          // gamma_t q_t rho
+            } else if constexpr (!kChan) {   // gamma_t q_t rho
                 const float gt = ex2(sm.l2g[t]);
 #pragma unroll 1
                 for (int cc = 0; cc < 8; ++cc) {
@@ -567,6 +899,32 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                     *reinterpret_cast<uint4*>(WQ[1] + umma::kmajor_off(64 + t, i0, D)) = mid;
                     *reinterpret_cast<uint4*>(WQ[2] + umma::kmajor_off(64 + t, i0, D)) = lo;
                 }
+            } else {          // channel gates: 2^lambda_ti q_ti rho_i
+#pragma unroll 1
+                for (int c32 = 0; c32 < 2; ++c32) {
+                    float lv[32];
+                    umma::tmem_ld32(tm_at(tm, warp, lam_col(64 * hf + 32 * c32)), lv);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int i0 = 64 * hf + 32 * c32 + 8 * q;
+                        const uint4 qb = *reinterpret_cast<const uint4*>(KQ + umma::kmajor_off(64 + t, i0, D));
+                        const uint32_t qw[4] = {qb.x, qb.y, qb.z, qb.w};
+                        const float4 r0 = *reinterpret_cast<const float4*>(sm.rho + i0);
+                        const float4 r1 = *reinterpret_cast<const float4*>(sm.rho + i0 + 4);
+                        const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+                        float x[8];
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            x[2 * p] = __uint_as_float(qw[p] << 16) * ex2(lv[8 * q + 2 * p]) * rr[2 * p];
+                            x[2 * p + 1] = __uint_as_float(qw[p] & 0xFFFF0000u) * ex2(lv[8 * q + 2 * p + 1]) * rr[2 * p + 1];
+                        }
+                        uint4 hi, mid, lo;
+                        split8x3(x, hi, mid, lo);
+                        *reinterpret_cast<uint4*>(WQ[0] + umma::kmajor_off(64 + t, i0, D)) = hi;
+                        *reinterpret_cast<uint4*>(WQ[1] + umma::kmajor_off(64 + t, i0, D)) = mid;
+                        *reinterpret_cast<uint4*>(WQ[2] + umma::kmajor_off(64 + t, i0, D)) = lo;
+                    }
+                }
             }
         }
         to_tensor_core();
@@ -587,7 +945,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
         {
             const int t = 32 * (warp & 1) + lane, hf = warp >> 2;
             if (!(warp & 2)) {   // TMEM lanes t: U_v and W S0
-                const float ratio = ex2(sm.l2g[C - 1] - sm.l2g[t]);
+                const float ratio = kChan ? 1.0f : ex2(sm.l2g[C - 1] - sm.l2g[t]);
 #pragma unroll 1
                 for (int c16 = 0; c16 < 4; ++c16) {
                     float uv[16], ws[16];
@@ -623,11 +981,43 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                     const int s0 = 32 * hf + 8 * q;
                     float x[8];
 #pragma unroll
-                    for (int p = 0; p < 8; ++p) x[p] = s0 + p <= t ? ex2(lt - sm.l2g[s0 + p]) * g[8 * q + p] : 0.0f;
+                    for (int p = 0; p < 8; ++p)
+                        x[p] = s0 + p <= t ? (kChan ? g[8 * q + p] : ex2(lt - sm.l2g[s0 + p]) * g[8 * q + p]) : 0.0f;
                     uint4 hi, lo;
                     split8(x, hi, lo);
                     *reinterpret_cast<uint4*>(Pp[0] + umma::kmajor_off(t, s0, C)) = hi;
                     *reinterpret_cast<uint4*>(Pp[1] + umma::kmajor_off(t, s0, C)) = lo;
+                }
+            }
+            if constexpr (kChan) {   // the planes of K o 2^(lambda_C - lambda) over K, Q and V (consumed)
+                if (!(warp & 2)) {
+                    uint16_t* KH[3] = {KQ, KQ + 64 * D, Vs};
+#pragma unroll 1
+                    for (int c32 = 0; c32 < 2; ++c32) {
+                        const int i0 = 64 * hf + 32 * c32;
+                        float lv[32];
+                        umma::tmem_ld32(tm_at(tm, warp, lam_col(i0)), lv);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int off = umma::kmajor_off(t, i0 + 8 * q, D);
+                            const uint4 kb = *reinterpret_cast<const uint4*>(KQ + off);
+                            const uint32_t kw[4] = {kb.x, kb.y, kb.z, kb.w};
+                            const float4 c0 = *reinterpret_cast<const float4*>(sm.lamC + i0 + 8 * q);
+                            const float4 c1 = *reinterpret_cast<const float4*>(sm.lamC + i0 + 8 * q + 4);
+                            const float lc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                            float x[8];
+#pragma unroll
+                            for (int p = 0; p < 4; ++p) {
+                                x[2 * p] = __uint_as_float(kw[p] << 16) * ex2(lc[2 * p] - lv[8 * q + 2 * p]);
+                                x[2 * p + 1] = __uint_as_float(kw[p] & 0xFFFF0000u) * ex2(lc[2 * p + 1] - lv[8 * q + 2 * p + 1]);
+                            }
+                            uint4 hi, mid, lo;
+                            split8x3(x, hi, mid, lo);
+                            *reinterpret_cast<uint4*>(KH[0] + off) = hi;
+                            *reinterpret_cast<uint4*>(KH[1] + off) = mid;
+                            *reinterpret_cast<uint4*>(KH[2] + off) = lo;
+                        }
+                    }
                 }
             }
         }
@@ -648,12 +1038,22 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             umma::commit(&sm.bar_mma);   // the readouts can be written while S_C is computed
             // S_C - gamma_C S0 = K^T U~ into the W columns (W was consumed in C).
             const uint32_t id_s = umma::idesc_bf16(128, 128, true, true);
+            if constexpr (!kChan) {
 #pragma unroll
-            for (int p = 0; p < 3; ++p)
+                for (int p = 0; p < 3; ++p)
 #pragma unroll
-                for (int ks = 0; ks < C / 16; ++ks)
-                    umma::mma_bf16(tm + TM_W, umma::desc_mnmajor(KQ, ks, D), umma::desc_mnmajor(BUT[p], ks, D), id_s,
-                                   p > 0 || ks > 0);
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        umma::mma_bf16(tm + TM_W, umma::desc_mnmajor(KQ, ks, D), umma::desc_mnmajor(BUT[p], ks, D), id_s,
+                                       p > 0 || ks > 0);
+            } else {   // (K o 2^(lambda_C - lambda))^T U: six part products
+                const uint16_t* KH[3] = {KQ, KQ + 64 * D, Vs};
+#pragma unroll
+                for (int pq = 0; pq < 6; ++pq)
+#pragma unroll
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        umma::mma_bf16(tm + TM_W, umma::desc_mnmajor(KH[kPartA[pq]], ks, D),
+                                       umma::desc_mnmajor(BUT[kPartB[pq]], ks, D), id_s, pq > 0 || ks > 0);
+            }
             umma::commit(&sm.bar_sc);
         }
         if (!wait_mma()) break;
@@ -682,7 +1082,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             // X_ij = (K^T U~)_ij + gamma_C rho_i c_j Z_ij, TMEM lane i, columns j in [64 hf, 64 hf + 64).
             if (!wait_bar(&sm.bar_sc, sc_phase)) break;
             const int i = 32 * (warp & 3) + lane;
-            const float fi = ex2(sm.l2g[C - 1]) * sm.rho[i];
+            const float fi = (kChan ? ex2(sm.lamC[i]) : ex2(sm.l2g[C - 1])) * sm.rho[i];
 #pragma unroll 1
             for (int c32 = 0; c32 < 2; ++c32) {
                 float sv[32];
@@ -715,7 +1115,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
         __syncthreads();
         if (next < a.num_tiles) {   // the next tile's q, k, v and small inputs arrive during the refit
             load_tokens(a, next, tid, KQ, Vs);
-            nx = load_ahead(a, next, tid, warp, lane);
+            nx = load_ahead<kChan>(a, next, tid, warp, lane);
         }
         {
             float2 Zr[M::RPT][4];
@@ -762,11 +1162,11 @@ extern "C" int stepq_prefill_chunk_wy(stepq_dims dims, int chunk, const uint16_t
     int rc = check_dims(dims, fn);
     if (rc) return rc;
     if (chunk < 1) return set_error(STEPQ_EINVAL, "%s: chunk=%d", fn, chunk);
-    if (dims.dk != D || dims.gate_per_channel || dims.pivots || chunk > C)
+    if (dims.dk != D || dims.pivots || chunk > C)
         return set_error(STEPQ_EUNSUPPORTED,
-                         "%s: the tensor-core chunk form needs d = 128, scalar gates, no FP16 pivot rows and at most "
-                         "%d tokens (d=%d gate_per_channel=%d pivots=%d chunk=%d)",
-                         fn, C, dims.dk, dims.gate_per_channel, dims.pivots, chunk);
+                         "%s: the tensor-core chunk form needs d = 128, no FP16 pivot rows and at most %d tokens "
+                         "(d=%d pivots=%d chunk=%d)",
+                         fn, C, dims.dk, dims.pivots, chunk);
     if (dims.B == 0) return STEPQ_OK;
     rc = check_ptrs(fn, {{"q", q}, {"k", k}, {"v", v}, {"beta", beta}, {"gate", gate}, {"bits", bits}, {"w", w},
                          {"head_off", head_off}, {"packed_in", packed_in}, {"r_in", r_in}, {"c_in", c_in},
@@ -779,21 +1179,27 @@ extern "C" int stepq_prefill_chunk_wy(stepq_dims dims, int chunk, const uint16_t
     uint32_t* flags = nullptr;
     rc = device_flags_ptr(&flags);
     if (rc) return rc;
-    static int num_sms = 0;
-    static std::once_flag once;
-    static cudaError_t init_err = cudaSuccess;
-    std::call_once(once, [] {
-        int dev = 0;
-        init_err = cudaGetDevice(&dev);
-        if (init_err == cudaSuccess) init_err = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-        if (init_err == cudaSuccess)
-            init_err = cudaFuncSetAttribute(prefill_wy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            static_cast<int>(SMEM_BYTES));
-    });
-    if (init_err != cudaSuccess) return set_error(STEPQ_ECUDA, "%s: %s", fn, cudaGetErrorString(init_err));
     WyArgs a{dims.B, dims.H, static_cast<int>(tiles), chunk, q, k, v, beta, gate, bits, w, head_off, bytes_per_seq,
              packed_in, r_in, c_in, packed_out, r_out, c_out, o, flags};
-    const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-    prefill_wy_kernel<<<grid, NT, SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(a);
+    const void* kernel = dims.gate_per_channel ? reinterpret_cast<const void*>(&prefill_wy_kernel<true>)
+                                               : reinterpret_cast<const void*>(&prefill_wy_kernel<false>);
+    int grid = 0;
+    rc = persistent_grid(kernel, NT, SMEM_BYTES, tiles, fn, &grid);
+    if (rc) return rc;
+    if (dims.gate_per_channel)
+        prefill_wy_kernel<true><<<grid, NT, SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(a);
+    else
+        prefill_wy_kernel<false><<<grid, NT, SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(a);
     return check_launch(fn);
+}
+
+extern "C" int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
+                                   const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,
+                                   const float* w, const int64_t* head_off, int64_t bytes_per_seq,
+                                   const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,
+                                   uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream) {
+    const bool wy = dims.dk == 128 && dims.dv == 128 && dims.pivots == 0 && chunk >= 1 && chunk <= STEPQ_WY_MAX_CHUNK;
+    return (wy ? stepq_prefill_chunk_wy : stepq_prefill_chunk_seq)(dims, chunk, q, k, v, beta, gate, bits, w, head_off,
+                                                                   bytes_per_seq, packed_in, r_in, c_in, packed_out,
+                                                                   r_out, c_out, o, stream);
 }

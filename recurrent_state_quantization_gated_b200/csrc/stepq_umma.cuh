@@ -1,5 +1,5 @@
-// Fifth-generation tensor-core helpers for sm_100a: tensor-memory (TMEM) allocation, loads and
-// fences, shared-memory matrix descriptors, instruction descriptors and the single-thread
+// Fifth-generation tensor-core helpers for sm_100a: tensor-memory (TMEM) allocation, loads,
+// stores and fences, shared-memory matrix descriptors, instruction descriptors and the single-thread
 // tcgen05.mma issue of kind::f16 (bf16 operands, fp32 accumulate), cta_group::1.
 //
 // Operand layouts are the canonical no-swizzle "core matrix" layouts: a core matrix is 8 rows of
@@ -137,6 +137,24 @@ __device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, float (&va
     }
 }
 #undef STEPQ_R16
+
+// TMEM stores (warp-collective): 32 consecutive 32-bit columns of this thread's lane, followed by
+// the wait for their completion.
+#define STEPQ_S16(o) "r"(__float_as_uint(v[o + 0])), "r"(__float_as_uint(v[o + 1])), "r"(__float_as_uint(v[o + 2])), \
+    "r"(__float_as_uint(v[o + 3])), "r"(__float_as_uint(v[o + 4])), "r"(__float_as_uint(v[o + 5])),                 \
+    "r"(__float_as_uint(v[o + 6])), "r"(__float_as_uint(v[o + 7])), "r"(__float_as_uint(v[o + 8])),                 \
+    "r"(__float_as_uint(v[o + 9])), "r"(__float_as_uint(v[o + 10])), "r"(__float_as_uint(v[o + 11])),               \
+    "r"(__float_as_uint(v[o + 12])), "r"(__float_as_uint(v[o + 13])), "r"(__float_as_uint(v[o + 14])),              \
+    "r"(__float_as_uint(v[o + 15]))
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        STEPQ_S16(0), STEPQ_S16(16)
+        : "memory");
+}
+#undef STEPQ_S16
 
 // TMEM address of (lane, column) relative to an allocation base.
 __device__ __forceinline__ uint32_t tmem_at(uint32_t base, int lane, int col) {

@@ -1,8 +1,9 @@
 """GPU parity of the prefill chunk (reconstruct once, C full-precision gated Delta updates, fit
 and pack the boundary state once) against the oracle, in both forms: the sequential form on the
-register-resident tile and the chunked WY form on the tensor cores. Every token's readout within
-1e-3 relative, the boundary state under the decode step's criteria; one token of the sequential
-form identical to the fused decode step; the two forms agree with each other to a few 1e-6."""
+register-resident tile and the chunked WY form on the tensor cores (scalar and channel gates).
+Every token's readout within 1e-3 relative, the boundary state under the decode step's criteria;
+one token of the sequential form identical to the fused decode step; the two forms agree with
+each other to a few 1e-6."""
 import numpy as np
 import pytest
 
@@ -117,6 +118,60 @@ def test_tensor_core_prefill_matches_oracle(B, H, widths, C, in_place):
     assert api.stepq_read_device_flags() == 0
 
 
+@pytest.mark.parametrize("B,H,widths,C", [
+    (3, 5, (2, 4, 6, 8), 64),
+    (2, 7, (4, 6, 8), 17),            # a ragged chunk
+    (2, 3, (2, 4, 6, 8), 1),
+    (8, 40, (4, 6, 8), 33),           # 320 tiles: more tiles than SMs
+    (4, 16, (8,), 64),                # 8-bit rows: the column-scale rate is tight here
+])
+def test_tensor_core_prefill_with_channel_gates_matches_oracle(B, H, widths, C):
+    """Channel gates (one gate per key channel and token, the KDA workload's gates) through the
+    tensor-core form: the gate-weighted pair products through the reference hierarchy, the
+    gate-scaled operands in three bf16 parts."""
+    from recurrent_state_quantization_gated_b200 import api
+    d = 128
+    wl, bits, w, packed, r, c = _setup(d, B, H, widths, True, seed=5 * B + H + C)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    toks = _chunk(wl, C)
+    assert toks["gate"].shape == (C, B, H, d)
+    res = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, "wy")
+    _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C)
+    assert api.stepq_read_device_flags() == 0
+
+
+def test_tensor_core_prefill_with_steep_channel_gates():
+    """Channel gates down to 0.01, exact zeros (three in one channel within 16 tokens, a whole
+    channel of zeros, and ones): gate products of a channel run far below fp32's range inside the
+    chunk, where a factorisation through one reference per 16-token block would overflow."""
+    from recurrent_state_quantization_gated_b200 import api
+    d, B, H, C = 128, 2, 3, 64
+    wl, bits, w, packed, r, c = _setup(d, B, H, (4, 6, 8), True, seed=79)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    toks = _chunk(wl, C)
+    rng = np.random.default_rng(6)
+    g = rng.uniform(0.01, 1.0, toks["gate"].shape).astype(np.float32)
+    g[[3, 7, 12], 0, 1, 5] = 0.0
+    g[:, 1, 2, 9] = 0.0
+    g[:, 0, 0, 17] = 1.0
+    toks["gate"] = g
+    res = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, "wy")
+    _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C)
+
+
+def test_tensor_core_and_sequential_forms_agree_under_channel_gates():
+    from recurrent_state_quantization_gated_b200 import api
+    d, B, H, C = 128, 4, 8, 64
+    wl, bits, w, packed, r, c = _setup(d, B, H, (2, 4, 6, 8), True, seed=93)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    td = _dev_tokens(_chunk(wl, C))
+    pw, rw, cw, ow = _run(api, td, bits, w, head_off, bps, packed, r, c, "wy")
+    ps, rs, cs, os_ = _run(api, td, bits, w, head_off, bps, packed, r, c, "seq")
+    err = np.abs(ow - os_).max(axis=-1) / np.maximum(np.abs(os_).max(axis=-1), 1e-30)
+    assert err.max() <= 2e-5, err.max()
+    compare_decode((pw, rw, cw, ow[-1]), (ps, rs, cs, os_[-1]), bits, d, B)
+
+
 def test_tensor_core_prefill_with_fast_decaying_gates():
     """Gates drawn in [0.2, 1] per token (and one exact zero): the gate products fall below
     fp32's range inside the chunk; ratios of them stay exact (log domain)."""
@@ -163,6 +218,27 @@ def test_tensor_core_prefill_full_size_sampled():
     head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
     toks = _chunk(wl, C)
     p_g, r_g, c_g, o_g = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, "wy")
+    sub = {n: np.ascontiguousarray(a[:, seqs]) for n, a in toks.items()}
+    p_s = np.concatenate([packed[b * bps:(b + 1) * bps] for b in seqs])
+    res = (np.concatenate([p_g[b * bps:(b + 1) * bps] for b in seqs]), r_g[seqs], c_g[seqs], o_g[:, seqs])
+    _check_against_oracle(res, sub, bits, w, p_s, r[seqs], c[seqs], d, len(seqs), C)
+
+
+def test_tensor_core_prefill_full_size_kda_sampled():
+    """The KDA prefill workload (256 sequences x 32 heads, d = 128, channel gates, 64-token chunk)
+    in one launch; the oracle checks four sampled sequences (every head of each)."""
+    from recurrent_state_quantization_gated_b200 import api
+    wl = synth.workload(2)
+    d, B, H, C = wl.d, wl.B, wl.H, 64
+    S0 = synth.initial_state(wl)
+    bits = synth.random_bits(H, d, choices=(4, 6, 8), seed=8)
+    w = synth.random_weights(H, d, seed=9)
+    seqs = [0, 85, 170, B - 1]
+    r, c = oracle.fit_scales(S0, w, bits)
+    packed = oracle.pack_state(S0, bits, r, c)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    toks = _chunk(wl, C)
+    p_g, r_g, c_g, o_g = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, None)
     sub = {n: np.ascontiguousarray(a[:, seqs]) for n, a in toks.items()}
     p_s = np.concatenate([packed[b * bps:(b + 1) * bps] for b in seqs])
     res = (np.concatenate([p_g[b * bps:(b + 1) * bps] for b in seqs]), r_g[seqs], c_g[seqs], o_g[:, seqs])

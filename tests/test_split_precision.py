@@ -71,3 +71,116 @@ def test_three_bf16_parts_keep_the_column_scales_of_the_exact_state():
     two, three = _mismatch_rate(2), _mismatch_rate(3)
     assert three < 0.002
     assert two > 0.004
+
+
+# ---- channel gates ---------------------------------------------------------------------------
+# Under channel gates the operands K o 2^lambda (of W = T diag(beta) K~) and K o 2^(lambda_C -
+# lambda) (of the boundary-state product) are computed, so both operands of those two products
+# are split. The six largest part products (high x high, high x middle, middle x high, high x low,
+# low x high, middle x middle) keep the column scales of the float64 state; the three largest do
+# not. The pair weights L and P are formed in fp32 through the reference hierarchy (every factor
+# a product of gates, at most 1).
+
+_SIX = [(0, 0), (0, 1), (1, 0), (0, 2), (2, 0), (1, 1)]
+_THREE = [(0, 0), (0, 1), (1, 0)]
+
+
+def _mm_pairs(A_parts, B_parts, pairs):
+    acc = np.zeros((A_parts[0].shape[0], B_parts[0].shape[1]), np.float32)
+    for p, q in pairs:
+        acc = (acc + (A_parts[p].astype(np.float64) @ B_parts[q].astype(np.float64)).astype(np.float32)).astype(np.float32)
+    return acc
+
+
+def _hierarchy_pairs(K, Q, G):
+    """fp32 pair weights sum_i k_ti k_si R_tsi (L, s < t) and sum_i q_ti k_si R_tsi (P, s <= t),
+    R_tsi the gate product over s < tau <= t, through the reference of each level."""
+    n = K.shape[0]
+    L = np.zeros((n, n), np.float32)
+    P = np.zeros((n, n), np.float32)
+    for lv in range(5, -1, -1):
+        h = 1 << lv
+        F = np.ones_like(K)
+        for m in range(n // (2 * h)):
+            lo, up = 2 * h * m, 2 * h * m + h
+            acc = np.ones(K.shape[1], np.float32)
+            for t in range(up, up + h):                 # gates from the upper half's start to t
+                acc = (acc * G[t]).astype(np.float32)
+                F[t] = acc
+            acc = np.ones(K.shape[1], np.float32)
+            for s in range(up - 1, lo - 1, -1):         # gates after s to the lower half's end
+                F[s] = acc
+                acc = (acc * G[s]).astype(np.float32)
+        SK, SQ = (K * F).astype(np.float32), (Q * F).astype(np.float32)
+        for m in range(n // (2 * h)):
+            lo, up = 2 * h * m, 2 * h * m + h
+            L[up:up + h, lo:lo + h] = (SK[up:up + h].astype(np.float64) @ SK[lo:lo + h].T).astype(np.float32)
+            P[up:up + h, lo:lo + h] = (SQ[up:up + h].astype(np.float64) @ SK[lo:lo + h].T).astype(np.float32)
+    P[np.arange(n), np.arange(n)] = np.sum(Q.astype(np.float64) * K, axis=1).astype(np.float32)
+    return L, P
+
+
+def _channel_mismatch_rate(pairs, C=40, tiles=((0, 0), (0, 1), (1, 0), (1, 1))):
+    wl = synth.workload(2, B=2, H=2, d=128, seed=3)
+    S0 = synth.initial_state(wl)
+    bits = np.full((wl.H, wl.d), 8, np.uint8)
+    w = synth.random_weights(wl.H, wl.d, seed=4)
+    r, c = oracle.fit_scales(S0, w, bits)
+    S_hat = oracle.unpack_state(oracle.pack_state(S0, bits, r, c), bits, r, c)
+    steps = [synth.tokens(wl, t) for t in range(C)]
+    toks = {n: np.stack([s[n] for s in steps]) for n in steps[0]}
+    n = 64
+    pad = lambda A, fill=0.0: np.concatenate([A, np.full((n - C,) + A.shape[1:], fill, np.float32)])
+    mis = tot = 0
+    for b, h in tiles:
+        K = synth.bf16_bits_to_f32(toks["k"][:, b, h]); V = synth.bf16_bits_to_f32(toks["v"][:, b, h])
+        Q = synth.bf16_bits_to_f32(toks["q"][:, b, h])
+        beta = toks["beta"][:, b, h].astype(np.float32); g = toks["gate"][:, b, h].astype(np.float32)
+        S = S_hat[b, h].astype(np.float64)
+        for t in range(C):
+            S, _ = oracle.delta_update(S, Q[t], K[t], V[t], beta[t], g[t])
+        rf = r[b, h].view(np.float16).astype(np.float32); cf = c[b, h].view(np.float16).astype(np.float32)
+        Z = np.round(S_hat[b, h] / np.outer(rf, cf)).astype(np.float32)
+        Kp, Qp, Vp, bp, gp = pad(K), pad(Q), pad(V), pad(beta), pad(g, 1.0)
+        lam = np.cumsum(np.log2(np.maximum(gp, 2.0 ** -64)), axis=0).astype(np.float32)
+        Lh, _ = _hierarchy_pairs(Kp, Qp, gp)
+        L = np.tril(bp[:, None] * Lh, -1).astype(np.float32)
+        T = np.linalg.inv(np.eye(n) + L.astype(np.float64)).astype(np.float32)
+        AT = _parts((T * bp[None, :]).astype(np.float32), 3)
+        Uv = _mm_pairs(AT, [Vp], [(0, 0), (1, 0), (2, 0)])
+        W = _mm_pairs(AT, _parts((Kp * np.exp2(lam)).astype(np.float32), 3), pairs)
+        WS0 = _mm_pairs(_parts((W * rf[None, :]).astype(np.float32), 3), [Z], [(0, 0), (1, 0), (2, 0)])
+        U = (Uv - cf[None, :] * WS0).astype(np.float32)
+        Kh = (Kp * np.exp2(lam[-1][None, :] - lam)).astype(np.float32)
+        SC = _mm_pairs([p.T.copy() for p in _parts(Kh, 3)], _parts(U, 3), pairs)
+        X = (SC + (np.exp2(lam[-1]) * rf)[:, None] * cf[None, :] * Z).astype(np.float32)
+        _, c1 = oracle.fit_tile(X, w[h], bits[h])
+        _, c2 = oracle.fit_tile(S.astype(np.float32), w[h], bits[h])
+        mis += int((c1 != c2).sum())
+        tot += c1.size
+    return mis / tot
+
+
+def test_hierarchy_pair_weights_equal_their_definition():
+    rng = np.random.default_rng(11)
+    n, d = 64, 16
+    K = rng.standard_normal((n, d)).astype(np.float32)
+    Q = rng.standard_normal((n, d)).astype(np.float32)
+    G = rng.uniform(0.0, 1.0, (n, d)).astype(np.float32)
+    G[5:9, 3] = 0.0
+    L, P = _hierarchy_pairs(K, Q, G)
+    R = np.ones((n, n, d))
+    for t in range(n):
+        for s in range(t):
+            R[t, s] = np.prod(G[s + 1:t + 1].astype(np.float64), axis=0)
+    Ld = np.einsum("ti,si,tsi->ts", K.astype(np.float64), K, R)
+    Pd = np.einsum("ti,si,tsi->ts", Q.astype(np.float64), K, R)
+    low = np.tril(np.ones((n, n), bool), -1)
+    np.testing.assert_allclose(L[low], Ld[low], rtol=0, atol=1e-5 * np.abs(Ld).max())
+    np.testing.assert_allclose(np.tril(P), np.tril(Pd), rtol=0, atol=1e-5 * np.abs(Pd).max())
+
+
+def test_six_part_products_keep_the_column_scales_under_channel_gates():
+    six, three = _channel_mismatch_rate(_SIX), _channel_mismatch_rate(_THREE)
+    assert six < 0.002
+    assert three > 0.003
