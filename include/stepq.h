@@ -71,9 +71,10 @@ typedef struct {
     int dv;                  /* value width (columns of a state tile)        */
     int gate_per_channel;    /* 0: gate [B][H]; 1: gate [B][H][dk]           */
     int pivots;              /* 1: the bit map may hold width-16 (FP16 pivot) rows. Read by the
-                                decode steps, which then run their pivot-capable kernel; a
-                                pivot row met with pivots = 0 raises bit 1 of the device error
-                                word and its results are undefined. Other calls ignore it.  */
+                                decode steps and the prefill chunks, which then run their
+                                pivot-capable kernels; a pivot row met with pivots = 0 raises
+                                bit 1 of the device error word and its results are undefined.
+                                Other calls ignore it.  */
     int mixed;               /* 1: some head's key rows have different widths (a row-level bit
                                 allocation). Read by stepq_decode_step and the sequential prefill
                                 chunk, which then run one code path for every row width instead of width-specialised paths per
@@ -153,14 +154,17 @@ STEPQ_API int stepq_decode_step(stepq_dims dims, const uint16_t* q, const uint16
        supported shape and chunk length; chunk = 1 is bit-identical to stepq_decode_step);
      stepq_prefill_chunk_wy: the chunked WY/UT form on the tensor cores (§2.1's affine form
        unrolled over the chunk: one unit lower triangular solve and dense products per tile).
-       Requires dk = dv = 128, no FP16 pivot rows and 1 <= chunk <= STEPQ_WY_MAX_CHUNK;
-       otherwise STEPQ_EUNSUPPORTED. Scalar and channel gates (gates in [0, 1]). Products run on
+       Requires dk = dv = 128 and 1 <= chunk <= STEPQ_WY_MAX_CHUNK; otherwise
+       STEPQ_EUNSUPPORTED. Scalar and channel gates (gates in [0, 1]); FP16 pivot rows enter the
+       products as v_ij / c_j in two bf16 parts and the boundary state from their stored values. Products run on
        bf16 operands (q, k, v and the integer codes exactly; computed operands split into two or
        three bf16 parts) with fp32 accumulation; under channel gates the gate-weighted token-pair
        products (the triangular system's and the readouts' intra-chunk weights) are formed on
        the CUDA cores in fp32. The boundary
        state carries fp32 precision, the readouts about 1e-6 relative.
-   stepq_prefill_chunk takes the WY form where it applies and the sequential form elsewhere. */
+   stepq_prefill_chunk takes the WY form for dk = dv = 128, scalar gates and chunk <=
+   STEPQ_WY_MAX_CHUNK (FP16 pivot rows or not), and the sequential form elsewhere: under channel
+   gates the WY form's pair products on the CUDA cores make it the slower of the two. */
 #define STEPQ_WY_MAX_CHUNK 64
 STEPQ_API int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q, const uint16_t* k,
                         const uint16_t* v, const float* beta, const float* gate, const uint8_t* bits,

@@ -265,7 +265,7 @@ def stepq_prefill_chunk(q, k, v, beta, gate, bits, w, head_off, bytes_per_seq, p
     """A prefill chunk: q, k, v [C,B,H,d], beta [C,B,H], gate [C,B,H] or [C,B,H,d]; the state is
     reconstructed once, updated C times in fp32 and packed once. form: None (the library picks),
     "seq" (tokens one after another on the register tile) or "wy" (the chunked WY form on the
-    tensor cores; d = 128, scalar or channel gates, no pivot rows, C <= 64). Returns (packed_out, r_out,
+    tensor cores; d = 128, C <= 64). Returns (packed_out, r_out,
     c_out, o [C,B,H,d])."""
     C, B, H, d = q.shape
     gpc = 1 if gate.dim() == 4 else 0

@@ -113,6 +113,7 @@ struct Small {
     alignas(8) uint64_t bar_codes;
     uint32_t tmem;
     int tile_ok;                     // the tile's head range holds it under the bit map
+    uint32_t pmask;                  // FP16 pivot rows: bit n set if rows 16 n to 16 n + 15 hold one
 };
 
 // Shared-memory map (bytes). The work region is reused phase by phase.
@@ -213,6 +214,43 @@ __device__ __forceinline__ float4 fma4(float a, float4 b, float4 c) {
 // TMEM columns of this warp's lanes.
 __device__ __forceinline__ uint32_t tm_at(uint32_t tm, int warp, uint32_t col) {
     return umma::tmem_at(tm, 32 * (warp & 3), static_cast<int>(col));
+}
+
+// ---- FP16 pivot rows --------------------------------------------------------------------------
+
+// Eight stored binary16 values v_ij, j0 <= j < j0 + 8, of pivot row i (read from the packed input;
+// zeros when the tile's head range failed its check).
+__device__ __forceinline__ void pivot_values(const WyArgs& a, const Small& sm, int64_t tile_base, int i, int j0,
+                                             float (&v)[8]) {
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    if (sm.tile_ok) {
+        const uint8_t* row = a.packed_in + tile_base + (sm.hmeta[sm.hslot[i] & 0xFF] >> 16);
+        raw = *reinterpret_cast<const uint4*>(row + 2 * j0);
+    }
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        v[2 * p] = half_bits_to_float(static_cast<uint16_t>(w[p] & 0xFFFFu));
+        v[2 * p + 1] = half_bits_to_float(static_cast<uint16_t>(w[p] >> 16));
+    }
+}
+
+// v_ij / c_j (as v_ij times the reciprocal of c_j), the pivot row's entries of Z.
+__device__ __forceinline__ void pivot_over_c(const WyArgs& a, const Small& sm, int64_t tile_base, int i, int j0,
+                                             float (&x)[8]) {
+    pivot_values(a, sm, tile_base, i, j0, x);
+#pragma unroll
+    for (int p = 0; p < 8; ++p) x[p] *= sm.icol[j0 + p];
+}
+
+// 4 KB slot n (n < 16) for the middle or low parts of one 16-row group of pivot rows, over
+// regions free while the state product runs: Q (read by then), V (consumed by the second round),
+// the codes buffer (the next tile's codes are fetched after this round) and the work region's top.
+__device__ __forceinline__ uint16_t* zpart_slot(int n, uint16_t* KQ, uint16_t* Vs, uint8_t* codes, uint8_t* W) {
+    if (n < 4) return KQ + 64 * D + 2048 * n;
+    if (n < 8) return Vs + 2048 * (n - 4);
+    if (n < 12) return reinterpret_cast<uint16_t*>(codes) + 2048 * (n - 8);
+    return reinterpret_cast<uint16_t*>(W + 96 * 1024) + 2048 * (n - 12);
 }
 
 // ---- channel gates -------------------------------------------------------------------------
@@ -425,7 +463,7 @@ __device__ __forceinline__ void issue_codes(const WyArgs& a, int tile, uint8_t* 
     if (bytes) bulk_load(dst, a.packed_in + static_cast<int64_t>(b) * a.bytes_per_seq + hoff, bytes, bar);
 }
 
-template <bool kChan>
+template <bool kChan, bool kPiv>
 __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -511,10 +549,18 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
         // ---- A: tables, gates, scales, codes -----------------------------------------------
         if constexpr (kChan) load_gates(a, tile, tid, Gs);
         if (warp == 1) {
-            const int total = sort_head_rows_w<D, false>(nx.widths, sm.hmeta, sm.hslot, lane, a.flags);
+            const int total = sort_head_rows_w<D, kPiv>(nx.widths, sm.hmeta, sm.hslot, lane, a.flags);
             // A head range that cannot hold the tile under the bit map: the tile is computed on
             // whatever the buffers hold and none of its results is written.
             if (lane == 0) sm.tile_ok = tile_range_ok(a.head_off, a.H, a.bytes_per_seq, h, total, 2 * D * D, a.flags);
+            if constexpr (kPiv) {   // the 16-row groups (key order) that hold FP16 pivot rows
+                uint32_t m = 0;
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    if (((nx.widths >> (8 * r)) & 0xFFu) == 16u) m |= 1u << ((4 * lane + r) >> 4);
+                m = __reduce_or_sync(0xffffffffu, m);
+                if (lane == 0) sm.pmask = m;
+            }
         }
         if (warp == 0) {   // beta and the running log2 of the gate product (a zero gate counts 2^-64)
             const float l0 = log2f(fmaxf(nx.g0, 0x1p-64f));
@@ -536,7 +582,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
         if (tid < D) {
             const int bw = sm.hslot[tid] >> 8;
             const float cj = half_bits_to_float(static_cast<uint16_t>(nx.rc >> 16));
-            sm.rho[tid] = half_bits_to_float(static_cast<uint16_t>(nx.rc & 0xFFFFu)) * znorm_of(bw);
+            // an FP16 pivot row enters as Z_ij = v_ij / c_j with rho_i = 1
+            sm.rho[tid] = kPiv && bw == 16 ? 1.0f : half_bits_to_float(static_cast<uint16_t>(nx.rc & 0xFFFFu)) * znorm_of(bw);
             sm.cs[tid] = cj;
             sm.icol[tid] = 1.0f / cj;
             w_slot = __ldg(a.w + static_cast<int64_t>(h) * D + (sm.hmeta[tid] & 0xFF));
@@ -556,6 +603,15 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                 case 8: unpack8<D, 8>(row, cc, z); break;
                 case 6: unpack8<D, 6>(row, cc, z); break;
                 case 4: unpack8<D, 4>(row, cc, z); break;
+                case 16:
+                    if constexpr (kPiv) {   // the high bf16 part of v_ij / c_j (values from global memory)
+                        float x[8];
+                        pivot_over_c(a, sm, tile_base, i, 8 * cc, x);
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) z[p] = make_float2(x[2 * p], x[2 * p + 1]);
+                        break;
+                    }
+                    [[fallthrough]];
                 default: unpack8<D, 2>(row, cc, z); break;
             }
             *reinterpret_cast<uint4*>(Zs + umma::kmajor_off(i, 8 * cc, D)) =
@@ -573,7 +629,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                     umma::mma_bf16(tm + TM_G, umma::desc_kmajor(KQ, ks, D), umma::desc_kmajor(KQ, ks, D), id, ks > 0);
                 umma::commit(&sm.bar_mma);
             }
-            if (nx.has_next) {   // the codes buffer is free: fetch the next tile's
+            if (!kPiv && nx.has_next) {   // the codes buffer is free: fetch the next tile's
                 mbar_arrive_expect_tx(&sm.bar_codes, nx.codes_bytes);
                 if (nx.codes_bytes) bulk_load(codes, a.packed_in + nx.codes_src, nx.codes_bytes, &sm.bar_codes);
                 codes_pending = true;
@@ -927,6 +983,29 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                 }
             }
         }
+        if constexpr (kPiv) {
+            // The middle and low bf16 parts of v_ij / c_j (the high part is in Z) for every 16-row
+            // group holding pivot rows, zero in its integer rows: slots 2n and 2n + 1 for the n-th
+            // such group.
+            __syncthreads();
+            const uint32_t pm = sm.pmask;
+            int n = 0;
+#pragma unroll 1
+            for (int ks = 0; ks < D / 16; ++ks) {
+                if (!((pm >> ks) & 1u)) continue;
+                const int i = 16 * ks + (tid >> 4), cc = tid & 15;
+                uint4 hi, mid = make_uint4(0u, 0u, 0u, 0u), lo = make_uint4(0u, 0u, 0u, 0u);
+                if ((sm.hslot[i] >> 8) == 16) {
+                    float x[8];
+                    pivot_over_c(a, sm, tile_base, i, 8 * cc, x);
+                    split8x3(x, hi, mid, lo);
+                }
+                const int off = umma::kmajor_off(i, 8 * cc, D) - 2048 * ks;
+                *reinterpret_cast<uint4*>(zpart_slot(2 * n, KQ, Vs, codes, W) + off) = mid;
+                *reinterpret_cast<uint4*>(zpart_slot(2 * n + 1, KQ, Vs, codes, W) + off) = lo;
+                ++n;
+            }
+        }
         to_tensor_core();
         if (tid == 0) {   // [W rho; gamma Q rho] Z: lanes 0-63 W S0, lanes 64-127 gamma Q S0 (without c)
             umma::fence_after_sync();
@@ -937,9 +1016,30 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                 for (int ks = 0; ks < D / 16; ++ks)
                     umma::mma_bf16(tm + TM_S, umma::desc_kmajor(WQ[p], ks, D), umma::desc_mnmajor(Zs, ks, D), id,
                                    p > 0 || ks > 0);
+            if constexpr (kPiv) {   // the pivot rows' lower parts: A high x Z middle, A middle x Z middle, A high x Z low
+                const uint32_t pm = sm.pmask;
+                int n = 0;
+#pragma unroll 1
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    if (!((pm >> ks) & 1u)) continue;
+                    const uint64_t dm = umma::smem_desc(smem_addr(zpart_slot(2 * n, KQ, Vs, codes, W)), D * 16u, 128u);
+                    const uint64_t dl = umma::smem_desc(smem_addr(zpart_slot(2 * n + 1, KQ, Vs, codes, W)), D * 16u, 128u);
+                    umma::mma_bf16(tm + TM_S, umma::desc_kmajor(WQ[0], ks, D), dm, id, 1u);
+                    umma::mma_bf16(tm + TM_S, umma::desc_kmajor(WQ[1], ks, D), dm, id, 1u);
+                    umma::mma_bf16(tm + TM_S, umma::desc_kmajor(WQ[0], ks, D), dl, id, 1u);
+                    ++n;
+                }
+            }
             umma::commit(&sm.bar_mma);
         }
         if (!wait_mma()) break;
+        if constexpr (kPiv) {   // the pivot parts' slots are consumed: fetch the next tile's codes
+            if (tid == 0 && nx.has_next) {
+                mbar_arrive_expect_tx(&sm.bar_codes, nx.codes_bytes);
+                if (nx.codes_bytes) bulk_load(codes, a.packed_in + nx.codes_src, nx.codes_bytes, &sm.bar_codes);
+                codes_pending = true;
+            }
+        }
 
         // ---- D: U = U_v - (W S0) diag(c); the U/c and U~ planes; the P planes ---------------
         {
@@ -1101,6 +1201,14 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                         x[2 * p] = fmaf(fi * cc[2 * p], __uint_as_float(zw[p] << 16), sv[8 * q + 2 * p]);
                         x[2 * p + 1] = fmaf(fi * cc[2 * p + 1], __uint_as_float(zw[p] & 0xFFFF0000u), sv[8 * q + 2 * p + 1]);
                     }
+                    if constexpr (kPiv) {
+                        if ((sm.hslot[i] >> 8) == 16) {   // pivot row: gamma_C v_ij from the stored binary16 values
+                            float v[8];
+                            pivot_values(a, sm, tile_base, i, j0, v);
+#pragma unroll
+                            for (int p = 0; p < 8; ++p) x[p] = fmaf(fi, v[p], sv[8 * q + p]);
+                        }
+                    }
                     *reinterpret_cast<float4*>(X + swx(i, j0)) = make_float4(x[0], x[1], x[2], x[3]);
                     *reinterpret_cast<float4*>(X + swx(i, j0 + 4)) = make_float4(x[4], x[5], x[6], x[7]);
                 }
@@ -1134,7 +1242,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             const int w1 = (sm.hmeta[warp * M::kRowsPerWarp + M::kRowsPerWarp - 1] >> 8) & 0xFF;
             const int ww = (w0 == w1) ? w0 : 0;
             if (sm.tile_ok)   // uniform over the CTA
-                refit_pack<D, false, false>(fit, sm.hmeta, Zr, ww, 0, tile, a.r_out, a.c_out, a.packed_out + tile_base);
+                refit_pack<D, kPiv, false>(fit, sm.hmeta, Zr, ww, 0, tile, a.r_out, a.c_out, a.packed_out + tile_base);
         }
         __syncthreads();   // the next tile rewrites the tables and the regions
     }
@@ -1162,11 +1270,10 @@ extern "C" int stepq_prefill_chunk_wy(stepq_dims dims, int chunk, const uint16_t
     int rc = check_dims(dims, fn);
     if (rc) return rc;
     if (chunk < 1) return set_error(STEPQ_EINVAL, "%s: chunk=%d", fn, chunk);
-    if (dims.dk != D || dims.pivots || chunk > C)
+    if (dims.dk != D || chunk > C)
         return set_error(STEPQ_EUNSUPPORTED,
-                         "%s: the tensor-core chunk form needs d = 128, no FP16 pivot rows and at most %d tokens "
-                         "(d=%d pivots=%d chunk=%d)",
-                         fn, C, dims.dk, dims.pivots, chunk);
+                         "%s: the tensor-core chunk form needs d = 128 and at most %d tokens (d=%d chunk=%d)", fn, C,
+                         dims.dk, chunk);
     if (dims.B == 0) return STEPQ_OK;
     rc = check_ptrs(fn, {{"q", q}, {"k", k}, {"v", v}, {"beta", beta}, {"gate", gate}, {"bits", bits}, {"w", w},
                          {"head_off", head_off}, {"packed_in", packed_in}, {"r_in", r_in}, {"c_in", c_in},
@@ -1181,15 +1288,19 @@ extern "C" int stepq_prefill_chunk_wy(stepq_dims dims, int chunk, const uint16_t
     if (rc) return rc;
     WyArgs a{dims.B, dims.H, static_cast<int>(tiles), chunk, q, k, v, beta, gate, bits, w, head_off, bytes_per_seq,
              packed_in, r_in, c_in, packed_out, r_out, c_out, o, flags};
-    const void* kernel = dims.gate_per_channel ? reinterpret_cast<const void*>(&prefill_wy_kernel<true>)
-                                               : reinterpret_cast<const void*>(&prefill_wy_kernel<false>);
+    const bool chan = dims.gate_per_channel != 0, piv = dims.pivots != 0;
+    const void* kernel = chan ? (piv ? reinterpret_cast<const void*>(&prefill_wy_kernel<true, true>)
+                                     : reinterpret_cast<const void*>(&prefill_wy_kernel<true, false>))
+                              : (piv ? reinterpret_cast<const void*>(&prefill_wy_kernel<false, true>)
+                                     : reinterpret_cast<const void*>(&prefill_wy_kernel<false, false>));
     int grid = 0;
     rc = persistent_grid(kernel, NT, SMEM_BYTES, tiles, fn, &grid);
     if (rc) return rc;
-    if (dims.gate_per_channel)
-        prefill_wy_kernel<true><<<grid, NT, SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(a);
-    else
-        prefill_wy_kernel<false><<<grid, NT, SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(a);
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (chan && piv) prefill_wy_kernel<true, true><<<grid, NT, SMEM_BYTES, st>>>(a);
+    else if (chan) prefill_wy_kernel<true, false><<<grid, NT, SMEM_BYTES, st>>>(a);
+    else if (piv) prefill_wy_kernel<false, true><<<grid, NT, SMEM_BYTES, st>>>(a);
+    else prefill_wy_kernel<false, false><<<grid, NT, SMEM_BYTES, st>>>(a);
     return check_launch(fn);
 }
 
@@ -1198,7 +1309,11 @@ extern "C" int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q
                                    const float* w, const int64_t* head_off, int64_t bytes_per_seq,
                                    const uint8_t* packed_in, const uint16_t* r_in, const uint16_t* c_in,
                                    uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream) {
-    const bool wy = dims.dk == 128 && dims.dv == 128 && dims.pivots == 0 && chunk >= 1 && chunk <= STEPQ_WY_MAX_CHUNK;
+    // The tensor-core form under scalar gates; under channel gates its gate-weighted pair
+    // products on the CUDA cores make it slower than the sequential form (KDA workload, 64-token
+    // chunk: 3.72 against 2.93 ms), so the sequential form is taken there.
+    const bool wy = dims.dk == 128 && dims.dv == 128 && dims.gate_per_channel == 0 && chunk >= 1 &&
+                    chunk <= STEPQ_WY_MAX_CHUNK;
     return (wy ? stepq_prefill_chunk_wy : stepq_prefill_chunk_seq)(dims, chunk, q, k, v, beta, gate, bits, w, head_off,
                                                                    bytes_per_seq, packed_in, r_in, c_in, packed_out,
                                                                    r_out, c_out, o, stream);

@@ -157,13 +157,13 @@ def test_new_entry_points_validate_before_touching_cuda():
 
 
 def test_tensor_core_prefill_refuses_shapes_it_does_not_cover():
-    """stepq_prefill_chunk_wy: d = 128, no pivot rows, 1 <= chunk <= 64 (scalar or channel
-    gates); anything else is STEPQ_EUNSUPPORTED (the sequential form covers it), checked before
-    any CUDA call."""
+    """stepq_prefill_chunk_wy: d = 128 and 1 <= chunk <= 64 (scalar or channel gates, FP16 pivot
+    rows or not); anything else is STEPQ_EUNSUPPORTED (the sequential form covers it), checked
+    before any CUDA call."""
     lib = _lib.lib()
     P = _fake
     args = (*([P()] * 8), 4096, *([P()] * 7), None)
-    for dims, chunk in ((_dims(d=64), 8), (_dims(pivots=1), 8), (_dims(), 65)):
+    for dims, chunk in ((_dims(d=64), 8), (_dims(d=64, gpc=1, pivots=1), 8), (_dims(), 65)):
         rc = lib.stepq_prefill_chunk_wy(dims, chunk, *args)
         assert rc == _lib.STEPQ_EUNSUPPORTED and b"tensor-core chunk form" in lib.stepq_last_error()
     assert lib.stepq_prefill_chunk_wy(_dims(), 0, *args) == _lib.STEPQ_EINVAL

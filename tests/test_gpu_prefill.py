@@ -140,6 +140,40 @@ def test_tensor_core_prefill_with_channel_gates_matches_oracle(B, H, widths, C):
     assert api.stepq_read_device_flags() == 0
 
 
+@pytest.mark.parametrize("gpc,B,H,widths,C,n_piv", [
+    (True, 2, 5, (4, 6, 8), 9, 11),       # a few pivot rows among mixed widths, channel gates
+    (False, 3, 4, (2, 4, 6, 8), 64, 7),   # scalar gates
+    (True, 2, 3, (4, 8), 33, 40),         # pivot rows in every 16-row group of some heads
+])
+def test_tensor_core_prefill_with_pivot_rows_matches_oracle(gpc, B, H, widths, C, n_piv):
+    """FP16 pivot rows through the tensor-core form: Z_ij = v_ij / c_j in two bf16 parts for the
+    products, the boundary state's pivot rows from the stored binary16 values."""
+    from recurrent_state_quantization_gated_b200 import api
+    d = 128
+    wl, bits, w, packed, r, c = _setup(d, B, H, widths, gpc, seed=3 * B + H + C, pivots=n_piv)
+    assert (bits == 16).sum() == n_piv
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    toks = _chunk(wl, C)
+    res = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, "wy")
+    _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C)
+    assert api.stepq_read_device_flags() == 0
+
+
+def test_tensor_core_prefill_with_a_pivot_head():
+    """A head whose rows are all FP16 pivots (Qwen-style pivot head) beside integer heads."""
+    from recurrent_state_quantization_gated_b200 import api
+    d, B, H, C = 128, 2, 3, 64
+    wl, bits, w, packed, r, c = _setup(d, B, H, (4, 6, 8), False, seed=83)
+    bits = bits.copy()
+    bits[1] = 16
+    r, c = oracle.fit_scales(synth.initial_state(wl), w, bits)
+    packed = oracle.pack_state(synth.initial_state(wl), bits, r, c)
+    head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
+    toks = _chunk(wl, C)
+    res = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, "wy")
+    _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C)
+
+
 def test_tensor_core_prefill_with_steep_channel_gates():
     """Channel gates down to 0.01, exact zeros (three in one channel within 16 tokens, a whole
     channel of zeros, and ones): gate products of a channel run far below fp32's range inside the
@@ -225,20 +259,21 @@ def test_tensor_core_prefill_full_size_sampled():
 
 
 def test_tensor_core_prefill_full_size_kda_sampled():
-    """The KDA prefill workload (256 sequences x 32 heads, d = 128, channel gates, 64-token chunk)
-    in one launch; the oracle checks four sampled sequences (every head of each)."""
+    """The KDA prefill workload (256 sequences x 32 heads, d = 128, channel gates, FP16 pivot rows,
+    64-token chunk) in one launch of the tensor-core form; the oracle checks four sampled
+    sequences (every head of each)."""
     from recurrent_state_quantization_gated_b200 import api
     wl = synth.workload(2)
     d, B, H, C = wl.d, wl.B, wl.H, 64
     S0 = synth.initial_state(wl)
-    bits = synth.random_bits(H, d, choices=(4, 6, 8), seed=8)
+    bits = with_pivots(synth.random_bits(H, d, choices=(4, 6, 8), seed=8), wl.n_pivots, 10)
     w = synth.random_weights(H, d, seed=9)
     seqs = [0, 85, 170, B - 1]
     r, c = oracle.fit_scales(S0, w, bits)
     packed = oracle.pack_state(S0, bits, r, c)
     head_off, bps, _ = api.stepq_packed_layout(bits, d, B)
     toks = _chunk(wl, C)
-    p_g, r_g, c_g, o_g = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, None)
+    p_g, r_g, c_g, o_g = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, "wy")
     sub = {n: np.ascontiguousarray(a[:, seqs]) for n, a in toks.items()}
     p_s = np.concatenate([packed[b * bps:(b + 1) * bps] for b in seqs])
     res = (np.concatenate([p_g[b * bps:(b + 1) * bps] for b in seqs]), r_g[seqs], c_g[seqs], o_g[:, seqs])

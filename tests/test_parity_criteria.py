@@ -150,7 +150,8 @@ def test_pivot_values_one_ulp_pass_two_fail(case):
     p, r, c, o = ref
     codes = tile_codes(p, bits, D, B).astype(np.int64)
     piv = np.broadcast_to((bits == 16)[None, :, :, None], codes.shape)
-    i = np.flatnonzero(piv & (np.abs(codes.astype(np.uint16).view(np.int16).astype(np.int64)) > 4))[0]
+    vals = np.abs(codes.astype(np.uint16).view(np.float16).astype(np.float64))
+    i = int(np.argmax(np.where(piv, vals, -1.0)))              # the largest pivot value
     for delta, ok in ((1, True), (2, False)):
         cc = codes.copy()
         cc.reshape(-1)[i] += delta                         # the next binary16 value(s) of the same sign
@@ -169,3 +170,28 @@ def test_codes_off_the_oracles_own_beyond_the_bound_fail(case):
     n_int = int((bits != 16).sum()) * D * B
     with pytest.raises(AssertionError):
         compare_decode(_with_codes_moved(ref, bits, int(0.003 * n_int), seed=5), ref, bits, D, B)
+
+
+def test_a_pivot_value_far_below_its_row_may_differ_by_fp32_rounding(case):
+    """In a tile whose largest magnitude is 16 (a pivot entry set to 16), a pivot value of 1e-5
+    (binary16 subnormal, spacing 2^-24): three binary16 ulps off (1.8e-7, below 2^-20 x 16)
+    passes; 2^-16 x 16 off fails."""
+    bits, ref, X = case
+    p, r, c, o = ref
+    codes = tile_codes(p, bits, D, B).astype(np.int64)
+    b, h = 0, int(np.flatnonzero((bits == 16).any(axis=1))[0])
+    i = int(np.flatnonzero(bits[h] == 16)[0])
+    half = lambda x: int(np.array(np.float16(x)).view(np.uint16))
+    base = codes.copy()
+    base[b, h, i, 0] = half(16.0)
+    base[b, h, i, 1] = half(1e-5)
+    want = (_repack(base, bits), r, c, o)
+    for shift, ok in ((3 * 2.0 ** -24, True), (16 * 2.0 ** -16, False)):
+        cc = base.copy()
+        cc[b, h, i, 1] = half(1e-5 + shift)
+        got = (_repack(cc, bits), r, c, o)
+        if ok:
+            compare_decode(got, want, bits, D, B)
+        else:
+            with pytest.raises(AssertionError, match="pivot values"):
+                compare_decode(got, want, bits, D, B)
