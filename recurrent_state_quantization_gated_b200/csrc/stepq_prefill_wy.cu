@@ -130,9 +130,9 @@ static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
 static_assert(65536 + sizeof(FitScratch) <= OFF_SMALL - OFF_W, "refit work space");
 
 // TMEM columns (512 allocated): G = [K;Q] K^T | W, later S_C | U_v | [W S0; gamma Q S0 + P U/c]
-// | channel gates: lambda. Under channel gates G holds no product: lanes 0-63 keep lambda_ti
-// (lane t, column i for i < 64; columns TM_LAM + i - 64 for the others) and lanes 64-127 keep P
-// (lane 64 + t, column s).
+// | channel gates: lambda. Under channel gates G holds no product: its lanes 0-63 keep lambda_ti
+// of channels i < 64 (lane t, column i) and its lanes 64-127 keep P (lane 64 + t, column s); the
+// lambda columns' lanes 64-127 keep lambda_ti of channels i >= 64 (lane 64 + t, column i - 64).
 constexpr uint32_t TM_G = 0, TM_W = 64, TM_U = 192, TM_S = 320, TM_LAM = 448;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -255,10 +255,14 @@ __device__ __forceinline__ uint16_t* zpart_slot(int n, uint16_t* KQ, uint16_t* V
 
 // ---- channel gates -------------------------------------------------------------------------
 
-// TMEM column of lambda_ti for the 32 channels from i0 (a multiple of 32), lanes 0-63.
+// TMEM column of lambda_ti for the 32 channels from i0 (a multiple of 32): channels 0-63 in
+// lanes 0-63 (lane t) of the G columns, channels 64-127 in lanes 64-127 (lane 64 + t) of the
+// lambda columns, so that every warp reaches the channels of its lane quarter.
 __host__ __device__ constexpr uint32_t lam_col(int i0) {
     return i0 < 64 ? TM_G + static_cast<uint32_t>(i0) : TM_LAM + static_cast<uint32_t>(i0 - 64);
 }
+// The 32 channels whose lambda this warp's lane quarter holds (its token is 32 (warp & 1) + lane).
+__device__ __forceinline__ int lam_channels(int warp) { return (warp & 2 ? 64 : 0) + 32 * (warp >> 2); }
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x >> 1); }
 
@@ -661,19 +665,15 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                 sm.lamC[i] = lam + carry;
             }
             __syncthreads();
-            if (!(warp & 2)) {   // lambda into TMEM lanes 0-63 (lane t)
-                const int t = 32 * (warp & 1) + lane, hf = warp >> 2;
-#pragma unroll 1
-                for (int c32 = 0; c32 < 2; ++c32) {
-                    const int i0 = 64 * hf + 32 * c32;
-                    float v[32];
+            {   // lambda into TMEM, each warp the 32 channels of its lane quarter
+                const int t = 32 * (warp & 1) + lane, i0 = lam_channels(warp);
+                float v[32];
 #pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4) {
-                        const float4 x = *reinterpret_cast<const float4*>(Gs + t * GLD + i0 + 4 * q4);
-                        v[4 * q4] = x.x; v[4 * q4 + 1] = x.y; v[4 * q4 + 2] = x.z; v[4 * q4 + 3] = x.w;
-                    }
-                    umma::tmem_st32(tm_at(tm, warp, lam_col(i0)), v);
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 x = *reinterpret_cast<const float4*>(Gs + t * GLD + i0 + 4 * q4);
+                    v[4 * q4] = x.x; v[4 * q4 + 1] = x.y; v[4 * q4 + 2] = x.z; v[4 * q4 + 3] = x.w;
                 }
+                umma::tmem_st32(tm_at(tm, warp, lam_col(i0)), v);
             }
             umma::fence_before_sync();
             __syncthreads();
@@ -852,12 +852,11 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
             *reinterpret_cast<uint4*>(AT[1] + umma::kmajor_off(row, s0, C)) = mid;
             *reinterpret_cast<uint4*>(AT[2] + umma::kmajor_off(row, s0, C)) = lo;
         }
-        if constexpr (kChan) {   // the planes of K o 2^lambda (rows t, channels i), lanes 0-63 of lambda
-            if (!(warp & 2)) {
-                const int t = 32 * (warp & 1) + lane, hf = warp >> 2;
-#pragma unroll 1
-                for (int c32 = 0; c32 < 2; ++c32) {
-                    const int i0 = 64 * hf + 32 * c32;
+        if constexpr (kChan) {   // the planes of K o 2^lambda (rows t, channels i), every warp 32 channels
+            {
+                const int t = 32 * (warp & 1) + lane;
+                {
+                    const int i0 = lam_channels(warp);
                     float lv[32];
                     umma::tmem_ld32(tm_at(tm, warp, lam_col(i0)), lv);
 #pragma unroll
@@ -955,31 +954,30 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                     *reinterpret_cast<uint4*>(WQ[1] + umma::kmajor_off(64 + t, i0, D)) = mid;
                     *reinterpret_cast<uint4*>(WQ[2] + umma::kmajor_off(64 + t, i0, D)) = lo;
                 }
-            } else {          // channel gates: 2^lambda_ti q_ti rho_i
-#pragma unroll 1
-                for (int c32 = 0; c32 < 2; ++c32) {
-                    float lv[32];
-                    umma::tmem_ld32(tm_at(tm, warp, lam_col(64 * hf + 32 * c32)), lv);
+            }
+            if constexpr (kChan) {   // 2^lambda_ti q_ti rho_i, every warp the 32 channels of its lane quarter
+                const int ch0 = lam_channels(warp);
+                float lv[32];
+                umma::tmem_ld32(tm_at(tm, warp, lam_col(ch0)), lv);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int i0 = 64 * hf + 32 * c32 + 8 * q;
-                        const uint4 qb = *reinterpret_cast<const uint4*>(KQ + umma::kmajor_off(64 + t, i0, D));
-                        const uint32_t qw[4] = {qb.x, qb.y, qb.z, qb.w};
-                        const float4 r0 = *reinterpret_cast<const float4*>(sm.rho + i0);
-                        const float4 r1 = *reinterpret_cast<const float4*>(sm.rho + i0 + 4);
-                        const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-                        float x[8];
+                for (int q = 0; q < 4; ++q) {
+                    const int i0 = ch0 + 8 * q;
+                    const uint4 qb = *reinterpret_cast<const uint4*>(KQ + umma::kmajor_off(64 + t, i0, D));
+                    const uint32_t qw[4] = {qb.x, qb.y, qb.z, qb.w};
+                    const float4 r0 = *reinterpret_cast<const float4*>(sm.rho + i0);
+                    const float4 r1 = *reinterpret_cast<const float4*>(sm.rho + i0 + 4);
+                    const float rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+                    float x[8];
 #pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-                            x[2 * p] = __uint_as_float(qw[p] << 16) * ex2(lv[8 * q + 2 * p]) * rr[2 * p];
-                            x[2 * p + 1] = __uint_as_float(qw[p] & 0xFFFF0000u) * ex2(lv[8 * q + 2 * p + 1]) * rr[2 * p + 1];
-                        }
-                        uint4 hi, mid, lo;
-                        split8x3(x, hi, mid, lo);
-                        *reinterpret_cast<uint4*>(WQ[0] + umma::kmajor_off(64 + t, i0, D)) = hi;
-                        *reinterpret_cast<uint4*>(WQ[1] + umma::kmajor_off(64 + t, i0, D)) = mid;
-                        *reinterpret_cast<uint4*>(WQ[2] + umma::kmajor_off(64 + t, i0, D)) = lo;
+                    for (int p = 0; p < 4; ++p) {
+                        x[2 * p] = __uint_as_float(qw[p] << 16) * ex2(lv[8 * q + 2 * p]) * rr[2 * p];
+                        x[2 * p + 1] = __uint_as_float(qw[p] & 0xFFFF0000u) * ex2(lv[8 * q + 2 * p + 1]) * rr[2 * p + 1];
                     }
+                    uint4 hi, mid, lo;
+                    split8x3(x, hi, mid, lo);
+                    *reinterpret_cast<uint4*>(WQ[0] + umma::kmajor_off(64 + t, i0, D)) = hi;
+                    *reinterpret_cast<uint4*>(WQ[1] + umma::kmajor_off(64 + t, i0, D)) = mid;
+                    *reinterpret_cast<uint4*>(WQ[2] + umma::kmajor_off(64 + t, i0, D)) = lo;
                 }
             }
         }
@@ -1090,11 +1088,10 @@ __global__ void __launch_bounds__(NT, 1) prefill_wy_kernel(const WyArgs a) {
                 }
             }
             if constexpr (kChan) {   // the planes of K o 2^(lambda_C - lambda) over K, Q and V (consumed)
-                if (!(warp & 2)) {
+                {
                     uint16_t* KH[3] = {KQ, KQ + 64 * D, Vs};
-#pragma unroll 1
-                    for (int c32 = 0; c32 < 2; ++c32) {
-                        const int i0 = 64 * hf + 32 * c32;
+                    {
+                        const int i0 = lam_channels(warp);
                         float lv[32];
                         umma::tmem_ld32(tm_at(tm, warp, lam_col(i0)), lv);
 #pragma unroll
