@@ -201,6 +201,15 @@ __global__ void __launch_bounds__(Map<D>::kThreads) int8_quantize_kernel(const B
 //   o_t = S_t^T q_t = gamma_t S_hat^T q_t + sum_{r<t} (gamma_t/gamma_r) (k_r.q_t) u_r + (k_t.q_t) u_t.
 // The window's last token forms S_W in registers and requantises it (rowwise absmax INT8).
 constexpr int kLeapMaxWindow = 256;
+
+__device__ __forceinline__ void leap_cp16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void leap_cp4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void leap_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void leap_cp_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 constexpr int kLeapBatch = 16;   // buffered tokens staged per pass of the window-end update
 constexpr int kLeapStage = 64;   // buffered tokens staged in shared memory per pass of a token
 
@@ -232,6 +241,7 @@ struct LeapSmem {
     alignas(16) float ub[kLeapBatch][D];           // window end: (gamma_W/gamma_r) u_r
     alignas(16) float us[kLeapStage][D];           // buffered u_r, staged for the column sums
     alignas(16) uint16_t ks[kLeapStage][D];        // buffered k_r, staged for the dot products
+    alignas(16) float lr[kLeapStage];              // their running log2 gate products
     float qk, lprev, lt;
 };
 
@@ -244,6 +254,27 @@ __global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) leap_ste
     const int64_t T = a.num_tiles;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int cl = M::col_lane(lane);
+    // The first kLeapStage buffered tokens' keys, pseudo-values and log gates are fetched first,
+    // together with the tile's codes, so that their latencies overlap (independent 16-byte and
+    // 4-byte asynchronous copies into shared memory).
+    const int nb0 = min(kLeapStage, t);
+    for (int e = tid; e < nb0 * (D / 8); e += M::kThreads) {
+        const int rb = e / (D / 8), c8 = e % (D / 8);
+        leap_cp16(&sm.ks[rb][8 * c8], a.kbuf + (static_cast<int64_t>(rb) * T + tile) * D + 8 * c8);
+    }
+    for (int e = tid; e < nb0 * (D / 4); e += M::kThreads) {
+        const int rb = e / (D / 4), c4 = e % (D / 4);
+        leap_cp16(&sm.us[rb][4 * c4], a.ubuf + (static_cast<int64_t>(rb) * T + tile) * D + 4 * c4);
+    }
+    for (int e = tid; e < nb0; e += M::kThreads) leap_cp4(&sm.lr[e], a.lbuf + static_cast<int64_t>(e) * T + tile);
+    leap_cp_commit();
+    // This token's v_j, beta and gate for the final column step, fetched now as well.
+    float vj = 0.f, bt = 0.f, gt = 0.f;
+    if (tid < D) {
+        vj = bf16_bits_to_float(__ldg(a.v + static_cast<int64_t>(tile) * D + tid));
+        bt = __ldg(a.beta + tile);
+        gt = __ldg(a.gate + tile);
+    }
     const int8_t* Cd = a.codes + static_cast<int64_t>(tile) * D * D;
     float Z[M::RPT][4];
 #pragma unroll
@@ -284,16 +315,21 @@ __global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) leap_ste
         for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
         if (lane == 0) sm.qk = acc;
     }
-    // The buffered tokens' dot products with k_t and q_t, kLeapStage tokens at a time: the keys
-    // are staged with independent 16-byte loads, then one warp per buffered token.
+    leap_cp_wait();
+    __syncthreads();
+    // The buffered tokens' dot products with k_t and q_t, kLeapStage tokens at a time (the first
+    // stage is already in shared memory; later ones are staged with independent 16-byte loads),
+    // one warp per buffered token.
     for (int r0 = 0; r0 < t; r0 += kLeapStage) {
         const int nb = min(kLeapStage, t - r0);
-        for (int e = tid; e < nb * (D / 8); e += M::kThreads) {
-            const int rb = e / (D / 8), c8 = e % (D / 8);
-            *reinterpret_cast<uint4*>(&sm.ks[rb][8 * c8]) = __ldg(reinterpret_cast<const uint4*>(
-                a.kbuf + (static_cast<int64_t>(r0 + rb) * T + tile) * D + 8 * c8));
+        if (r0 > 0) {
+            for (int e = tid; e < nb * (D / 8); e += M::kThreads) {
+                const int rb = e / (D / 8), c8 = e % (D / 8);
+                *reinterpret_cast<uint4*>(&sm.ks[rb][8 * c8]) = __ldg(reinterpret_cast<const uint4*>(
+                    a.kbuf + (static_cast<int64_t>(r0 + rb) * T + tile) * D + 8 * c8));
+            }
+            __syncthreads();
         }
-        __syncthreads();
         for (int rb = warp; rb < nb; rb += M::kWarps) {
             float ck = 0.f, cq = 0.f;
 #pragma unroll
@@ -308,12 +344,12 @@ __global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) leap_ste
                 cq += __shfl_xor_sync(0xffffffffu, cq, m);
             }
             if (lane == 0) {
-                const float lr = a.lbuf[static_cast<int64_t>(r0 + rb) * T + tile];
+                const float lr = r0 == 0 ? sm.lr[rb] : a.lbuf[static_cast<int64_t>(r0 + rb) * T + tile];
                 sm.dots[0][r0 + rb] = ck * exp2f(sm.lprev - lr);
                 sm.dots[1][r0 + rb] = cq * exp2f(sm.lt - lr);
             }
         }
-        __syncthreads();
+        if (r0 + kLeapStage < t) __syncthreads();   // the next stage rewrites the keys
     }
     // S_hat^T k_t and S_hat^T q_t, column partial sums.
     {
@@ -340,13 +376,15 @@ __global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) leap_ste
     float bp = 0.f, bo = 0.f;
     for (int r0 = 0; r0 < t; r0 += kLeapStage) {
         const int nb = min(kLeapStage, t - r0);
-        if (r0 > 0) __syncthreads();   // the previous stage has been read
-        for (int e = tid; e < nb * (D / 4); e += M::kThreads) {
-            const int rb = e / (D / 4), c4 = e % (D / 4);
-            *reinterpret_cast<float4*>(&sm.us[rb][4 * c4]) = __ldg(reinterpret_cast<const float4*>(
-                a.ubuf + (static_cast<int64_t>(r0 + rb) * T + tile) * D + 4 * c4));
+        if (r0 > 0) {   // the first stage was fetched at the start
+            __syncthreads();   // the previous stage has been read
+            for (int e = tid; e < nb * (D / 4); e += M::kThreads) {
+                const int rb = e / (D / 4), c4 = e % (D / 4);
+                *reinterpret_cast<float4*>(&sm.us[rb][4 * c4]) = __ldg(reinterpret_cast<const float4*>(
+                    a.ubuf + (static_cast<int64_t>(r0 + rb) * T + tile) * D + 4 * c4));
+            }
+            __syncthreads();
         }
-        __syncthreads();
         if (tid < D) {
 #pragma unroll 4
             for (int rb = 0; rb < nb; ++rb) {
@@ -365,8 +403,7 @@ __global__ void __launch_bounds__(Map<D>::kThreads, Map<D>::kMinBlocks) leap_ste
             b0 += sm.red[w][1][j];
         }
         const float p = fmaf(exp2f(sm.lprev), a0, bp);
-        const float g = __ldg(a.gate + tile);
-        const float u = __ldg(a.beta + tile) * (bf16_bits_to_float(a.v[static_cast<int64_t>(tile) * D + j]) - g * p);
+        const float u = bt * (vj - gt * p);
         a.o[static_cast<int64_t>(tile) * D + j] = fmaf(sm.qk, u, fmaf(exp2f(sm.lt), b0, bo));
         a.ubuf[(static_cast<int64_t>(t) * T + tile) * D + j] = u;
         sm.colu[j] = u;
