@@ -132,7 +132,8 @@ def compare_decode(gpu, ref, bits, d, B, X_ref=None, max_frac=1e-3, label=""):
 
     o within 1e-3 relative; r within one binary16 ulp; c within 10 % (an entry of the updated
     state on a rounding boundary of the intermediate codes moves the least-squares column
-    update; such columns are under 1 %). Codes (every integer entry of every tile):
+    update; such columns are under 1 % of those of the tiles whose row scales agree). Codes
+    (every integer entry of every tile):
 
     * with ``X_ref`` (the oracle's updated state, ``oracle_updated_state``): X_ref quantised by
       the oracle's quantiser at the GPU's own scales must give the GPU's codes within one step,
@@ -151,7 +152,12 @@ def compare_decode(gpu, ref, bits, d, B, X_ref=None, max_frac=1e-3, label=""):
     cf_r = c_r.view(np.float16).astype(np.float64)
     assert np.max(np.abs(cf_g / cf_r - 1)) < 0.1
     c_mis = (c_g != c_r).mean()
-    assert c_mis < 1e-2, f"{c_mis:.2e} of column scales differ"
+    # A row scale one ulp apart changes that row's codes, which enter every column's
+    # least-squares sums of the tile, so all of that tile's column scales may move: the share of
+    # differing column scales is bounded over the tiles whose row scales agree.
+    r_same = (r_g == r_r).all(axis=-1)
+    c_mis_same = (c_g != c_r)[r_same].mean() if r_same.any() else 0.0
+    assert c_mis_same < 1e-2, f"{c_mis_same:.2e} of column scales differ in tiles whose row scales agree"
     codes_g = tile_codes(p_g, bits, d, B)
     codes_r = tile_codes(p_r, bits, d, B)
     piv = np.broadcast_to((bits == 16)[None, :, :, None], codes_g.shape)
