@@ -317,13 +317,22 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
     const int cl = M::col_lane(lane);
     const float2 M2 = make_float2(kRoundMagic, kRoundMagic);
     const bool issuer = (tid == M::kThreads - 1);
+    // The tile's (sequence, head) and stage, stepped per tile instead of divided out.
+    const int step_b = gridDim.x / a.H, step_h = gridDim.x % a.H;
+    int seq = blockIdx.x / a.H, h = blockIdx.x % a.H;
+    int s = 0;
+    uint32_t parity = 0;
     for (int n = 0;; ++n) {
+        if (n > 0) {
+            seq += step_b;
+            h += step_h;
+            if (h >= a.H) { h -= a.H; ++seq; }
+            if (++s == kStages) { s = 0; parity ^= 1u; }
+        }
         const int tile = cta_tile(n);
         if (tile >= a.num_tiles) break;
-        const int s = n % kStages;
-        const uint32_t parity = (n / kStages) & 1;
         const auto& st = sm.stage[s];
-        const int h = tile % a.H, he = h % CH;
+        const int he = h % CH;
         const uint32_t* meta = sm.hmeta[he];
         if (sm.htag[he] != h) {                     // every warp sees the same tag: uniform branch
             __syncthreads();                        // nobody still reads the entry
@@ -340,7 +349,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
             __syncthreads();
         }
         const bool tile_ok = sm.hok[he];
-        const int64_t tile_base = static_cast<int64_t>(tile / a.H) * a.bytes_per_seq + sm.hoff[he];
+        const int64_t tile_base = static_cast<int64_t>(seq) * a.bytes_per_seq + sm.hoff[he];
         const bool ok = mbar_wait_bounded(&sm.full[s], parity, kWaitLimitNs, &g_stepq_flags);
 
         // A prefill chunk's token 1: its inputs are loaded now, behind the unpack (rows by the
@@ -395,7 +404,7 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
         }
         // Every thread is past the previous tile, so its stage may be refilled kStages-1 ahead;
         // the copies are queued below while half of the CTA finalises the first reductions.
-        const int ahead = n + kStages - 1, sa = ahead % kStages;
+        const int ahead = n + kStages - 1, sa = s == 0 ? kStages - 1 : s - 1;   // ahead % kStages
         bool issued = false;
         float next_beta = 0.f, next_gate = 0.f;
         if (!tile_ok) {   // uniform: nothing of this tile is read or written
