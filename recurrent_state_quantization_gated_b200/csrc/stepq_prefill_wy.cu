@@ -1308,7 +1308,7 @@ extern "C" int stepq_prefill_chunk(stepq_dims dims, int chunk, const uint16_t* q
                                    uint8_t* packed_out, uint16_t* r_out, uint16_t* c_out, float* o, void* stream) {
     // The tensor-core form under scalar gates; under channel gates its gate-weighted pair
     // products on the CUDA cores make it slower than the sequential form (KDA workload, 64-token
-    // chunk: 3.72 against 2.93 ms), so the sequential form is taken there.
+    // chunk: 3.04 against 2.90 ms), so the sequential form is taken there.
     const bool wy = dims.dk == 128 && dims.dv == 128 && dims.gate_per_channel == 0 && chunk >= 1 &&
                     chunk <= STEPQ_WY_MAX_CHUNK;
     return (wy ? stepq_prefill_chunk_wy : stepq_prefill_chunk_seq)(dims, chunk, q, k, v, beta, gate, bits, w, head_off,
