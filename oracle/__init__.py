@@ -140,6 +140,19 @@ def fit_tile(X, w, bits, detail=False):
     return r, c, dict(c0=c0, z0=z0, c1=c1)
 
 
+def fit_columns(X, w, bits, r, detail=False):
+    """The column half of the fit at given binary16 row scales r (App. C.1): the no-clip start,
+    the codes at (r, c0) and one weighted least-squares update; returns c (binary16 bits), and
+    with ``detail`` also dict(c0, z0, c1) as fit_tile does."""
+    X = _c(X, np.float32); w = _c(w, np.float32); bits = _c(bits, np.uint8); r = _c(r, np.uint16)
+    dk, dv = X.shape
+    c = np.zeros(dv, dtype=np.uint16)
+    c0 = np.zeros(dv, dtype=np.float32); z0 = np.zeros((dk, dv), dtype=np.int32)
+    c1 = np.zeros(dv, dtype=np.float64)
+    lib().orc_fit_columns_detail(dk, dv, _p(X), _p(w), _p(bits), _p(r), _p(c), _p(c0), _p(z0), _p(c1))
+    return (c, dict(c0=c0, z0=z0, c1=c1)) if detail else c
+
+
 def pack_tile(X, bits, r, c):
     X = _c(X, np.float32); bits = _c(bits, np.uint8); r = _c(r, np.uint16); c = _c(c, np.uint16)
     dk, dv = X.shape

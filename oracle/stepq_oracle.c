@@ -304,25 +304,16 @@ void orc_unpack_tile(int dk, int dv, const uint8_t* packed, const uint8_t* bits,
     free(codes);
 }
 
-/* Key-row-aware dual-axis fit (§4.3, App. C.1; readings R1, R2). Returns r, c as binary16.
-   The optional detail outputs expose the intermediate column scales and codes:
-   c0 (fp32), z0 (codes at (r, c0)), c1 (double, the least-squares solution before rounding). */
-void orc_fit_tile_detail(int dk, int dv, const float* X, const float* w, const uint8_t* bits,
-                         uint16_t* r_out, uint16_t* c_out, float* c0_out, int* z0_out,
-                         double* c1_out) {
+/* The column half of the dual-axis fit (App. C.1; reading R2) at given binary16 row scales r:
+   the no-clip column start c0, the codes at (r, c0) and one weighted least-squares update.
+   Returns c as binary16; the optional detail outputs expose c0 (fp32), z0 (codes at (r, c0))
+   and c1 (double, the least-squares solution before rounding). */
+void orc_fit_columns_detail(int dk, int dv, const float* X, const float* w, const uint8_t* bits,
+                            const uint16_t* r, uint16_t* c_out, float* c0_out, int* z0_out, double* c1_out) {
     float* rf = (float*)malloc(sizeof(float) * dk);
     float* c0 = (float*)malloc(sizeof(float) * dv);
     int* z0 = (int*)malloc(sizeof(int) * dk * dv);
-
-    /* Row factors: m_i = (1/d_v) sum_j |X_ij|, impact folded in as r_i = m_i / w_i. */
-    for (int i = 0; i < dk; ++i) {
-        double m = 0.0;
-        for (int j = 0; j < dv; ++j) m += fabs((double)X[i * dv + j]);
-        m /= dv;
-        if (m < HALF_MIN_NORMAL) m = HALF_MIN_NORMAL;
-        r_out[i] = orc_scale_to_half(m / (double)w[i]);
-        rf[i] = orc_half_to_float(r_out[i]);
-    }
+    for (int i = 0; i < dk; ++i) rf[i] = orc_half_to_float(r[i]);
 
     /* Column initialisation: smallest scale at which no entry of the column clips. The shared
        column scales serve the integer rows only: FP16 pivot rows take no part (App. C.1, the
@@ -370,6 +361,22 @@ void orc_fit_tile_detail(int dk, int dv, const float* X, const float* w, const u
     free(rf);
     free(c0);
     free(z0);
+}
+
+/* Key-row-aware dual-axis fit (§4.3, App. C.1; readings R1, R2). Returns r, c as binary16.
+   The optional detail outputs are those of orc_fit_columns_detail. */
+void orc_fit_tile_detail(int dk, int dv, const float* X, const float* w, const uint8_t* bits,
+                         uint16_t* r_out, uint16_t* c_out, float* c0_out, int* z0_out,
+                         double* c1_out) {
+    /* Row factors: m_i = (1/d_v) sum_j |X_ij|, impact folded in as r_i = m_i / w_i. */
+    for (int i = 0; i < dk; ++i) {
+        double m = 0.0;
+        for (int j = 0; j < dv; ++j) m += fabs((double)X[i * dv + j]);
+        m /= dv;
+        if (m < HALF_MIN_NORMAL) m = HALF_MIN_NORMAL;
+        r_out[i] = orc_scale_to_half(m / (double)w[i]);
+    }
+    orc_fit_columns_detail(dk, dv, X, w, bits, r_out, c_out, c0_out, z0_out, c1_out);
 }
 
 void orc_fit_tile(int dk, int dv, const float* X, const float* w, const uint8_t* bits,

@@ -81,6 +81,45 @@ def test_zero_column_keeps_initial_scale():
     assert c[5] == np.float16(2.0 ** -14).view(np.uint16)
 
 
+def _representable_tile(d, seed):
+    """A tile X_ij = r_i 2^(8-b_i) c_j z_ij exactly, with binary16 scales r, c, integer codes
+    |z_ij| <= q_b and the code q_b in every column (so the no-clip start is c itself)."""
+    rng = np.random.default_rng(seed)
+    bits = rng.choice(np.array([2, 4, 6, 8], dtype=np.uint8), d)
+    qb = 2 ** (bits.astype(np.int64) - 1) - 1
+    z = np.stack([rng.integers(-q, q + 1, d) for q in qb])
+    rows = rng.integers(0, d, d)                             # one entry per column at its row's edge
+    z[rows, np.arange(d)] = qb[rows] * rng.choice([-1, 1], d)
+    r = (2.0 ** rng.integers(-6, 2, d)).astype(np.float16)
+    c = (2.0 ** rng.integers(-8, -2, d) * rng.choice([1.0, 1.25, 1.5, 1.75], d)).astype(np.float16)
+    X = (r.astype(np.float64)[:, None] * 2.0 ** (8 - bits.astype(np.float64))[:, None]
+         * c.astype(np.float64)[None, :] * z).astype(np.float32)
+    return X, bits, r.view(np.uint16), c.view(np.uint16), z
+
+
+@pytest.mark.parametrize("seed", [11, 12])
+def test_column_fit_at_given_row_scales_is_exact_on_representable_tiles(seed):
+    """At the row scales the tile was built with, the no-clip start is the column scale itself,
+    the codes at (r, c0) are the tile's codes, and the least-squares update returns the same
+    scale (App. C.1: the fit is exact where the state is exactly representable); at row scales
+    twice as large every column scale halves."""
+    d = 64
+    X, bits, r, c, z = _representable_tile(d, seed)
+    w = synth.random_weights(1, d, seed=seed)[0]
+    got, det = oracle.fit_columns(X, w, bits, r, detail=True)
+    np.testing.assert_array_equal(det["z0"], z)
+    np.testing.assert_array_equal(got, c)
+    r2 = (r.view(np.float16).astype(np.float64) * 2).astype(np.float16).view(np.uint16)
+    half = (c.view(np.float16).astype(np.float64) / 2).astype(np.float16).view(np.uint16)
+    np.testing.assert_array_equal(oracle.fit_columns(X, w, bits, r2), half)
+
+
+def test_column_fit_is_the_column_half_of_the_tile_fit():
+    S, bits, w = _tile(128, 13)
+    r, c = oracle.fit_tile(S, w, bits)
+    np.testing.assert_array_equal(oracle.fit_columns(S, w, bits, r), c)
+
+
 @pytest.mark.parametrize("gpc", [False, True])
 def test_decode_tile_is_unpack_update_fit_pack(gpc):
     """Table C2: reconstruct, update, emit the readout before requantisation, refit, repack."""
