@@ -47,6 +47,7 @@ def pytest_terminal_summary(terminalreporter):
         gs = [r["at_gpu_scales"] for r in rs if r["at_gpu_scales"] is not None]
         tr.write_line(
             f"{label}: steps {len(rs)}, codes {sum(r['n_codes'] for r in rs)}; at the GPU's scales max "
-            f"{max(gs) if gs else float('nan'):.2e}; vs the oracle's codes max {max(r['raw'] for r in rs):.2e} "
-            f"mean {np.mean([r['raw'] for r in rs]):.2e}; scales differing: r {np.mean([r['r_mismatch'] for r in rs]):.2e}, "
+            f"{max(gs) if gs else float('nan'):.2e}; vs the reference codes max {max(r['raw'] for r in rs):.2e} "
+            f"mean {np.mean([r['raw'] for r in rs]):.2e}; vs the oracle's own codes max "
+            f"{max(r['raw_own'] for r in rs):.2e}; scales differing: r {np.mean([r['r_mismatch'] for r in rs]):.2e}, "
             f"c {np.mean([r['c_mismatch'] for r in rs]):.2e}")

@@ -126,40 +126,60 @@ def quantise_with_scales(X, bits, r, c):
     return out
 
 
-def compare_decode(gpu, ref, bits, d, B, X_ref=None, max_frac=1e-3, label=""):
+def compare_decode(gpu, ref, bits, d, B, X_ref=None, max_frac=1e-3, label="", w=None):
     """Compares one decode step's results, (packed, r, c, o) as host arrays from both sides,
     started from the same packed state.
 
-    o within 1e-3 relative; r within one binary16 ulp; c within 10 % (an entry of the updated
-    state on a rounding boundary of the intermediate codes moves the least-squares column
-    update; such columns are under 1 % of those of the tiles whose row scales agree). Codes
-    (every integer entry of every tile):
+    o within 1e-3 relative; r within one binary16 ulp of the oracle's. A row scale one ulp apart
+    moves that row's intermediate codes, which enter every column's least-squares sums of the
+    tile (App. C.1), so the tile's column scales and codes may follow it. The reference for c and
+    the codes is therefore the oracle's own result where the row scales agree and, in a tile
+    where some row scale is one ulp apart (given ``X_ref`` and the row-impact factors ``w``
+    [H][dk]), the oracle's column fit of X_ref at the GPU's row scales with X_ref quantised at
+    (GPU's r, that c); without them the reference is the oracle's own result everywhere and
+    the column scales of such tiles are not compared. Against that reference: c within 10 %, with
+    at most 1 % of the column scales different, or one (an entry of X on a rounding boundary of the
+    intermediate codes moves the column update, by a few % in a column whose least-squares sums
+    a few entries dominate, and with it the final codes of that column); codes (every integer
+    entry of every tile):
 
     * with ``X_ref`` (the oracle's updated state, ``oracle_updated_state``): X_ref quantised by
       the oracle's quantiser at the GPU's own scales must give the GPU's codes within one step,
       with at most ``max_frac`` of them one step off -- the bound that isolates the kernel's
-      quantisation from the choice of scales;
-    * against the oracle's own codes (its own scales): never more than one step apart, at most
-      ``max_frac`` of every integer entry differ, and at most ``max_frac`` of the entries whose
-      row and column scales agree on both sides.
+      quantisation from the choice of scales -- and the entries whose row and column scales
+      agree with the reference's must match the reference codes within one step, at most
+      ``max_frac`` of them one step off;
+    * without ``X_ref``: every integer entry within one step of the reference codes, at most
+      ``max_frac`` of them and of the entries whose scales agree one step off.
 
-    Returns a dict of rates, also appended to ``RATES``."""
+    Returns a dict of rates (``raw_own``: the share of integer codes that differ from the
+    oracle's own codes, reported only), also appended to ``RATES``."""
     p_g, r_g, c_g, o_g = gpu
     p_r, r_r, c_r, o_r = ref
     assert_outputs_close(o_g, o_r)
     assert half_ulps(r_g, r_r).max() <= 1, "row factors are continuous in X: one ulp at most"
-    cf_g = c_g.view(np.float16).astype(np.float64)
-    cf_r = c_r.view(np.float16).astype(np.float64)
-    assert np.max(np.abs(cf_g / cf_r - 1)) < 0.1
-    c_mis = (c_g != c_r).mean()
-    # A row scale one ulp apart changes that row's codes, which enter every column's
-    # least-squares sums of the tile, so all of that tile's column scales may move: the share of
-    # differing column scales is bounded over the tiles whose row scales agree.
-    r_same = (r_g == r_r).all(axis=-1)
-    c_mis_same = (c_g != c_r)[r_same].mean() if r_same.any() else 0.0
-    assert c_mis_same < 1e-2, f"{c_mis_same:.2e} of column scales differ in tiles whose row scales agree"
     codes_g = tile_codes(p_g, bits, d, B)
     codes_r = tile_codes(p_r, bits, d, B)
+    # The reference scales and codes: the oracle's own, or at the GPU's row scales where they differ.
+    r_same = (r_g == r_r).all(axis=-1)
+    r_ref, c_ref, codes_ref, held = r_r.copy(), c_r.copy(), codes_r.copy(), r_same.copy()   # held: c compared
+    if X_ref is not None and w is not None:
+        for b, h in zip(*np.nonzero(~r_same)):
+            Xt = np.asarray(X_ref[b, h], dtype=np.float32)
+            r_ref[b, h] = r_g[b, h]
+            c_ref[b, h] = oracle.fit_columns(Xt, w[h], bits[h], r_g[b, h])
+            codes_ref[b, h] = oracle.quantise_tile(Xt, bits[h], r_ref[b, h], c_ref[b, h])
+        held[:] = True
+    cf_g = c_g.view(np.float16).astype(np.float64)[held]
+    cf_f = c_ref.view(np.float16).astype(np.float64)[held]
+    if cf_g.size:
+        gap = np.max(np.abs(cf_g / cf_f - 1))
+        assert gap < 0.1, f"a column scale {gap:.1%} away from the reference column fit"
+    moved = (c_g != c_ref)[held]
+    c_mis = float(moved.mean()) if moved.size else 0.0
+    # a flip is a per-column event: one column of a one-tile case is 1.6 % of its 64
+    assert moved.sum() <= max(1, int(1e-2 * moved.size)), \
+        f"{c_mis:.2e} of column scales differ from the reference column fit ({int(moved.sum())} columns)"
     piv = np.broadcast_to((bits == 16)[None, :, :, None], codes_g.shape)
     if piv.any():
         # FP16 pivot entries: binary16 values within one unit in the last place, or, for a value
@@ -176,10 +196,18 @@ def compare_decode(gpu, ref, bits, d, B, X_ref=None, max_frac=1e-3, label=""):
         ulp = np.spacing(np.maximum(np.abs(vg), np.abs(vr)).astype(np.float16)).astype(np.float64)
         assert (np.abs(vg - vr) <= np.maximum(ulp, floor)).all(), "pivot values differ by more than one binary16 ulp"
     integer = ~piv
-    diff = np.where(piv, 0, np.abs(codes_g.astype(np.int64) - codes_r))
-    assert diff.max() <= 1, f"codes differ by {diff.max()}"
+    diff = np.where(piv, 0, np.abs(codes_g.astype(np.int64) - codes_ref))
+    same = (r_g == r_ref)[..., :, None] & (c_g == c_ref)[..., None, :] & integer
+    if X_ref is None:
+        assert diff.max() <= 1, f"codes differ by {diff.max()}"
+    else:
+        # Where a column scale differs from the reference, the final codes of that column follow
+        # it: held to X_ref quantised at the GPU's own scales below.
+        assert diff[same].max(initial=0) <= 1, f"codes with equal scales differ by {diff[same].max(initial=0)}"
+    own = np.where(piv, 0, np.abs(codes_g.astype(np.int64) - codes_r))
     rates = dict(label=label, equal_scales=None, raw=None, r_mismatch=float((r_g != r_r).mean()),
-                 c_mismatch=float(c_mis), at_gpu_scales=None, n_codes=int(integer.sum()))
+                 c_mismatch=float((c_g != c_r).mean()), at_gpu_scales=None, n_codes=int(integer.sum()),
+                 raw_own=float((own[integer] > 0).mean() if integer.any() else 0.0))
     if X_ref is not None:
         codes_x = quantise_with_scales(X_ref, bits, r_g, c_g)
         dx = np.abs(codes_g.astype(np.int64) - codes_x)[integer]
@@ -187,11 +215,11 @@ def compare_decode(gpu, ref, bits, d, B, X_ref=None, max_frac=1e-3, label=""):
         fx = (dx > 0).mean() if dx.size else 0.0
         rates["at_gpu_scales"] = float(fx)
         assert fx <= max_frac, f"{fx:.2e} of all integer codes differ from the oracle's X at the GPU's scales"
-    same = (r_g == r_r)[..., :, None] & (c_g == c_r)[..., None, :] & integer
     frac_same = (diff[same] > 0).mean() if same.any() else 0.0
     rates["equal_scales"] = float(frac_same)
     rates["raw"] = float((diff[integer] > 0).mean() if integer.any() else 0.0)
     assert frac_same <= max_frac, f"{frac_same:.2e} of codes with equal scales differ by one step"
-    assert rates["raw"] <= max_frac, f"{rates['raw']:.2e} of all integer codes differ from the oracle's own codes"
+    if X_ref is None:   # with X_ref every code is bounded at the GPU's own scales instead
+        assert rates["raw"] <= max_frac, f"{rates['raw']:.2e} of the integer codes differ from the reference codes"
     RATES.append(rates)
     return rates

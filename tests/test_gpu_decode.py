@@ -52,7 +52,7 @@ def _check_step(api, wl, bits, w, head_off, bps, st, t, in_place, label=""):
     ref = oracle.decode_step(tok, bits, w, st["packed"], st["r"], st["c"])
     X_ref = oracle_updated_state(tok, bits, st["packed"], st["r"], st["c"])
     rates = compare_decode((p_g.cpu().numpy(), host_half(r_g), host_half(c_g), o_g.cpu().numpy()), ref, bits,
-                           wl.d, wl.B, X_ref=X_ref, label=label)
+                           wl.d, wl.B, X_ref=X_ref, label=label, w=w)
     return dict(packed=ref[0], r=ref[1], c=ref[2]), rates
 
 

@@ -81,7 +81,8 @@ def test_full_size_step_on_sampled_sequences(index):
         X_ref = oracle_updated_state(ts, bits, p_ref, r_ref, c_ref)
         gpu = (_seq_bytes(st.packed.cpu().numpy(), seqs, st.layout.bytes_per_seq), host_half(st.r)[seqs],
                host_half(st.c)[seqs], o.cpu().numpy()[seqs])
-        compare_decode(gpu, ref, bits, wl.d, len(seqs), X_ref=X_ref, label=f"full size {wl.name}, sampled sequences")
+        compare_decode(gpu, ref, bits, wl.d, len(seqs), X_ref=X_ref, label=f"full size {wl.name}, sampled sequences",
+                       w=w)
         # the next step starts both sides from the oracle's state again
         p_ref, r_ref, c_ref = ref[:3]
         bps = st.layout.bytes_per_seq

@@ -58,7 +58,7 @@ def test_prefill_chunk_matches_oracle(d, B, H, widths, gpc, C, pivots):
         compare_o = np.abs(og[t] - orf[t]).max(axis=-1) / np.maximum(np.abs(orf[t]).max(axis=-1), 1e-30)
         assert compare_o.max() <= 1e-3, (t, compare_o.max())
     compare_decode((p_g.cpu().numpy(), host_half(r_g), host_half(c_g), og[-1]), (p_r, r_r, c_r, o_r[-1]), bits, d, B,
-                   X_ref=oracle_chunk_state(toks, bits, packed, r, c), label=f"prefill chunk C={C} d={d} H={H}")
+                   X_ref=oracle_chunk_state(toks, bits, packed, r, c), label=f"prefill chunk C={C} d={d} H={H}", w=w)
 
 
 def test_one_token_chunk_is_the_decode_step():
@@ -95,7 +95,8 @@ def _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C):
         err = np.abs(og[t] - o_r[t]).max(axis=-1) / np.maximum(np.abs(o_r[t]).max(axis=-1), 1e-30)
         assert err.max() <= 1e-3, (t, err.max())
     return compare_decode((p_g, r_g, c_g, og[-1]), (p_r, r_r, c_r, o_r[-1]), bits, d, B,
-                          X_ref=oracle_chunk_state(toks, bits, packed, r, c), label=f"prefill chunk C={C} (tensor-core form)")
+                          X_ref=oracle_chunk_state(toks, bits, packed, r, c), label=f"prefill chunk C={C} (tensor-core form)",
+                          w=w)
 
 
 @pytest.mark.parametrize("B,H,widths,C,in_place", [

@@ -54,7 +54,7 @@ def test_randomized_decode_steps(seed):
         ref = oracle.decode_step(tok, bits, w, packed, r, c)
         X_ref = oracle_updated_state(tok, bits, packed, r, c)
         compare_decode((p_g.cpu().numpy(), host_half(r_g), host_half(c_g), o_g.cpu().numpy()), ref, bits, d, B,
-                       X_ref=X_ref, label=label)
+                       X_ref=X_ref, label=label, w=w)
         packed, r, c = ref[:3]
     assert api.stepq_read_device_flags() == 0
 
@@ -87,5 +87,5 @@ def test_randomized_prefill_chunks(seed):
         label = (f"randomized prefill C={C} form={form} d={d} B={B} H={H} widths={widths} "
                  f"gates={'channel' if gpc else 'head'} pivots={pivots}")
         compare_decode((p_g.cpu().numpy(), host_half(r_g), host_half(c_g), og[-1]), (ref[0], ref[1], ref[2], ref[3][-1]),
-                       bits, d, B, X_ref=X_ref, label=label)
+                       bits, d, B, X_ref=X_ref, label=label, w=w)
     assert api.stepq_read_device_flags() == 0

@@ -56,7 +56,7 @@ def test_split_form_matches_oracle(d, B, H, widths, gpc):
         ref = oracle.decode_step(tok, bits, w, st["packed"], st["r"], st["c"])
         rates.append(compare_decode((p_g.cpu().numpy(), host_half(r_g), host_half(c_g), o_g.cpu().numpy()), ref,
                                     bits, d, B, X_ref=oracle_updated_state(tok, bits, st["packed"], st["r"], st["c"]),
-                                    label=f"split form d={d} B={B} H={H}"))
+                                    label=f"split form d={d} B={B} H={H}", w=w))
         X_ref = _oracle_X(tok, bits, w, st, d)
         np.testing.assert_allclose(X_g.cpu().numpy(), X_ref, rtol=1e-5, atol=1e-6 * np.abs(X_ref).max())
         st = dict(packed=ref[0], r=ref[1], c=ref[2])

@@ -35,7 +35,7 @@ def _rank_main(rank, world, port, out):
 def test_two_gloo_ranks_agree_on_the_slowest_time():
     import torch.multiprocessing as mp
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:   # no fork of a process that may run OpenMP threads
         out = m.dict()
         mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
         res = dict(out)

@@ -3,11 +3,12 @@
 One oracle decode step gives a reference result (packed codes, row and column scales,
 readouts). A "device" result is then made from it with planted deviations, and the comparator
 must accept exactly what the criteria allow: readouts within 1e-3 relative, row scales within
-one binary16 ulp, column scales within 10 % and different on under 1 % of the columns of tiles
-whose row scales agree, codes within one step on at most 0.1% of the entries whose scales
-agree, the same bound over every integer code when the oracle's own updated state is quantised
-at the device's scales, and FP16 pivot values within one ulp (or, far below the tile's scale,
-within 2^-20 of it). Anything beyond that must fail. So a GPU result that broke a criterion
+one binary16 ulp, column scales within 10 % of the reference fit and different on under 1 % of
+the columns (the reference of a tile whose row scale is one ulp off is the oracle's column fit
+and codes at the device's row scales), codes within one step on at most 0.1% of the entries
+whose scales agree and of every integer entry, the same bound over every integer code when the
+oracle's own updated state is quantised at the device's scales, and FP16 pivot values within
+one ulp (or, far below the tile's scale, within 2^-20 of it). Anything beyond that must fail. So a GPU result that broke a criterion
 cannot pass the GPU tests through a slack comparison."""
 import numpy as np
 import pytest
@@ -113,6 +114,60 @@ def test_column_scales_of_a_tile_may_follow_its_row_scale(case):
     r2 = r.copy()
     r2[0, 0, int(np.flatnonzero(bits[0] != 16)[0])] += 1
     compare_decode((p, r2, c2, o), ref, bits, D, B)
+
+
+def test_a_tile_with_a_row_scale_off_is_held_to_the_refit_at_that_scale(case):
+    """Given X and the row-impact factors, a tile whose row scale is one ulp off is compared with
+    the oracle's column fit and codes at the device's row scales (App. C.1: the column update
+    starts from the codes at those row scales): that refit passes, even where its codes differ
+    from the oracle's own; a column of it 20 % off fails, and so do codes one step off on more
+    than 0.1 % of the entries."""
+    bits, ref, X = case
+    w = synth.random_weights(H, D, seed=24)
+    p, r, c, o = ref
+    codes = tile_codes(p, bits, D, B).astype(np.int64)
+    r2, c2 = r.copy(), c.copy()
+    for i in np.flatnonzero(bits[0] != 16)[:4]:                 # four row scales of tile (0, 0)
+        r2[0, 0, i] += 1
+    c2[0, 0] = oracle.fit_columns(X[0, 0], w[0], bits[0], r2[0, 0])
+    codes[0, 0] = oracle.quantise_tile(X[0, 0], bits[0], r2[0, 0], c2[0, 0])
+    got = (_repack(codes, bits), r2, c2, o)
+    rates = compare_decode(got, ref, bits, D, B, X_ref=X, w=w)
+    assert rates["raw"] == 0.0 and rates["at_gpu_scales"] == 0.0
+    c3 = c2.copy()
+    c3[0, 0, 7] = (c2[0, 0, 7:8].view(np.float16).astype(np.float64) * 1.2).astype(np.float16).view(np.uint16)[0]
+    with pytest.raises(AssertionError, match="reference column fit"):
+        compare_decode((got[0], r2, c3, o), ref, bits, D, B, X_ref=X, w=w)
+    n_int = int((bits != 16).sum()) * D * B
+    moved = _with_codes_moved(got, bits, int(0.003 * n_int), seed=6)
+    with pytest.raises(AssertionError):
+        compare_decode(moved, ref, bits, D, B, X_ref=X, w=w)
+
+
+def test_codes_of_a_column_whose_scale_moved_are_held_at_the_device_scales(case):
+    """A column scale 3 % off (an intermediate code on its rounding boundary flips the column
+    update, App. C.1), with its final codes at that scale -- several steps from the oracle's own
+    codes on the column's large entries -- passes when the oracle's X is given (the codes are
+    held at the device's own scales), fails without it, and fails with those codes one step
+    off on more than 0.1 % of the entries."""
+    bits, ref, X = case
+    w = synth.random_weights(H, D, seed=24)
+    p, r, c, o = ref
+    codes = tile_codes(p, bits, D, B).astype(np.int64)
+    big = np.abs(np.where((bits[0] == 8)[:, None], codes[0, 0], 0))
+    j = int(np.argmax(big.max(axis=0)))                     # the column with the largest 8-bit code
+    assert big[:, j].max() >= 70
+    c3 = c.copy()
+    c3[0, 0, j] = (c[0, 0, j:j + 1].view(np.float16).astype(np.float64) * 1.03).astype(np.float16).view(np.uint16)[0]
+    codes[0, 0] = oracle.quantise_tile(X[0, 0], bits[0], r[0, 0], c3[0, 0])
+    got = (_repack(codes, bits), r, c3, o)
+    rates = compare_decode(got, ref, bits, D, B, X_ref=X, w=w)
+    assert rates["at_gpu_scales"] == 0.0 and rates["raw"] > 0.0
+    with pytest.raises(AssertionError, match="codes differ by"):
+        compare_decode(got, ref, bits, D, B)
+    n_int = int((bits != 16).sum()) * D * B
+    with pytest.raises(AssertionError):
+        compare_decode(_with_codes_moved(got, bits, int(0.003 * n_int), seed=7), ref, bits, D, B, X_ref=X, w=w)
 
 
 def test_one_step_on_few_codes_passes_on_many_fails(case):
