@@ -36,7 +36,7 @@ def _state(d, B, H, widths, gpc, pivots, seed):
     return wl, bits, w, oracle.pack_state(S0, bits, r, c), r, c
 
 
-@pytest.mark.parametrize("seed", range(12))
+@pytest.mark.parametrize("seed", range(32))
 def test_randomized_decode_steps(seed):
     import torch
     from recurrent_state_quantization_gated_b200 import api
@@ -59,7 +59,7 @@ def test_randomized_decode_steps(seed):
     assert api.stepq_read_device_flags() == 0
 
 
-@pytest.mark.parametrize("seed", range(8))
+@pytest.mark.parametrize("seed", range(24))
 def test_randomized_prefill_chunks(seed):
     """Both forms where the tensor-core form applies (d = 128), the library's choice elsewhere."""
     import torch
