@@ -153,6 +153,18 @@ def fit_columns(X, w, bits, r, detail=False):
     return (c, dict(c0=c0, z0=z0, c1=c1)) if detail else c
 
 
+def ls_columns(X, w, bits, r, z, cfall):
+    """The fixed-code least-squares column update alone (App. C.1) at binary16 row scales r and
+    integer codes z [dk][dv]; a column with a zero denominator keeps cfall. Returns
+    (c binary16 bits, c1 float64 before rounding)."""
+    X = _c(X, np.float32); w = _c(w, np.float32); bits = _c(bits, np.uint8); r = _c(r, np.uint16)
+    z = _c(z, np.int32); cfall = _c(cfall, np.float32)
+    dk, dv = X.shape
+    c = np.zeros(dv, dtype=np.uint16); c1 = np.zeros(dv, dtype=np.float64)
+    lib().orc_ls_columns(dk, dv, _p(X), _p(w), _p(bits), _p(r), _p(z), _p(cfall), _p(c), _p(c1))
+    return c, c1
+
+
 def pack_tile(X, bits, r, c):
     X = _c(X, np.float32); bits = _c(bits, np.uint8); r = _c(r, np.uint16); c = _c(c, np.uint16)
     dk, dv = X.shape

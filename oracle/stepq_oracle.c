@@ -304,6 +304,27 @@ void orc_unpack_tile(int dk, int dv, const uint8_t* packed, const uint8_t* bits,
     free(codes);
 }
 
+/* One fixed-code least-squares update of every column scale (App. C.1) at binary16 row scales
+   r and integer codes z [dk][dv]: c_j = sum_i w_i^2 v_ij X_ij / sum_i w_i^2 v_ij^2 with
+   v_ij = r_i 2^(8-b_i) z_ij over the non-pivot rows; a column with a zero denominator keeps
+   cfall[j]. Returns c as binary16, c1 (double, before rounding) if given. */
+void orc_ls_columns(int dk, int dv, const float* X, const float* w, const uint8_t* bits, const uint16_t* r,
+                    const int* z, const float* cfall, uint16_t* c_out, double* c1_out) {
+    for (int j = 0; j < dv; ++j) {
+        double num = 0.0, den = 0.0;
+        for (int i = 0; i < dk; ++i) {
+            if (is_pivot(bits[i])) continue;
+            double v = (double)orc_half_to_float(r[i]) * znorm_of(bits[i]) * z[i * dv + j];
+            double ww = (double)w[i] * (double)w[i];
+            num += ww * v * (double)X[i * dv + j];
+            den += ww * v * v;
+        }
+        double c1 = den > 0.0 ? num / den : (double)cfall[j];
+        if (c1_out) c1_out[j] = c1;
+        c_out[j] = orc_scale_to_half(c1);
+    }
+}
+
 /* The column half of the dual-axis fit (App. C.1; reading R2) at given binary16 row scales r:
    the no-clip column start c0, the codes at (r, c0) and one weighted least-squares update.
    Returns c as binary16; the optional detail outputs expose c0 (fp32), z0 (codes at (r, c0))
@@ -341,21 +362,7 @@ void orc_fit_columns_detail(int dk, int dv, const float* X, const float* w, cons
         for (int j = 0; j < dv; ++j) z0[i * dv + j] = quantise(X[i * dv + j], ir, 1.0f / c0[j], b);
     }
 
-    /* One fixed-code least-squares update of every column scale (App. C.1):
-       c_j = sum_i w_i^2 v_ij X_ij / sum_i w_i^2 v_ij^2 with v_ij = r_i z_ij. */
-    for (int j = 0; j < dv; ++j) {
-        double num = 0.0, den = 0.0;
-        for (int i = 0; i < dk; ++i) {
-            if (is_pivot(bits[i])) continue;
-            double v = (double)rf[i] * znorm_of(bits[i]) * z0[i * dv + j];
-            double ww = (double)w[i] * (double)w[i];
-            num += ww * v * (double)X[i * dv + j];
-            den += ww * v * v;
-        }
-        double c1 = den > 0.0 ? num / den : (double)c0[j];
-        if (c1_out) c1_out[j] = c1;
-        c_out[j] = orc_scale_to_half(c1);
-    }
+    orc_ls_columns(dk, dv, X, w, bits, r, z0, c0, c_out, c1_out);
     if (c0_out) memcpy(c0_out, c0, sizeof(float) * dv);
     if (z0_out) memcpy(z0_out, z0, sizeof(int) * dk * dv);
     free(rf);

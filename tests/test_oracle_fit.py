@@ -114,6 +114,26 @@ def test_column_fit_at_given_row_scales_is_exact_on_representable_tiles(seed):
     np.testing.assert_array_equal(oracle.fit_columns(X, w, bits, r2), half)
 
 
+def test_least_squares_update_alone():
+    """The fixed-code least-squares update (App. C.1) on its own: the codes a representable tile
+    was built from give its column scales back; the weights' common scale cancels; an all-zero
+    column of codes keeps its fallback scale; at the tile fit's own codes it is the fit's c."""
+    d = 64
+    X, bits, r, c, z = _representable_tile(d, 14)
+    w = synth.random_weights(1, d, seed=14)[0]
+    fall = np.full(d, 0.5, dtype=np.float32)
+    got, c1 = oracle.ls_columns(X, w, bits, r, z, fall)
+    np.testing.assert_array_equal(got, c)
+    np.testing.assert_array_equal(oracle.ls_columns(X, 4.0 * w, bits, r, z, fall)[0], c)
+    z0 = z.copy()
+    z0[:, 3] = 0
+    got0, c10 = oracle.ls_columns(X, w, bits, r, z0, fall)
+    assert c10[3] == 0.5 and got0[3] == np.float16(0.5).view(np.uint16)
+    S, bits2, w2 = _tile(128, 15)
+    r2, c2, det = oracle.fit_tile(S, w2, bits2, detail=True)
+    np.testing.assert_array_equal(oracle.ls_columns(S, w2, bits2, r2, det["z0"], det["c0"])[0], c2)
+
+
 def test_column_fit_is_the_column_half_of_the_tile_fit():
     S, bits, w = _tile(128, 13)
     r, c = oracle.fit_tile(S, w, bits)

@@ -133,10 +133,10 @@ MUTANTS = [
     _m("least-squares weights not squared", C_SRC,
        ("double ww = (double)w[i] * (double)w[i];", "double ww = (double)w[i];")),
     _m("least-squares model drops the codebook step", C_SRC,
-       ("double v = (double)rf[i] * znorm_of(bits[i]) * z0[i * dv + j];",
-        "double v = (double)rf[i] * z0[i * dv + j];")),
+       ("double v = (double)orc_half_to_float(r[i]) * znorm_of(bits[i]) * z[i * dv + j];",
+        "double v = (double)orc_half_to_float(r[i]) * z[i * dv + j];")),
     _m("least-squares update skipped", C_SRC,
-       ("c_out[j] = orc_scale_to_half(c1);", "c_out[j] = orc_scale_to_half((double)c0[j]);")),
+       ("c_out[j] = orc_scale_to_half(c1);", "c_out[j] = orc_scale_to_half((double)cfall[j]);")),
     # the persistent decode step (Table C2) and the prefill boundary (App. F.1)
     _m("decode refits the previous state", C_SRC,
        ("    for (int e = 0; e < dk * dv; ++e) S32[e] = (float)t.X[e];\n"
