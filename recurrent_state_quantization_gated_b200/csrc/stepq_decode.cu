@@ -105,6 +105,7 @@ struct DecodeSmem {
     alignas(8) uint64_t full[kStages];
     float qk;
     float qkp[2][D / 32];           // q.k of a chunk's token, one partial per 32 key rows
+    int rn[2][D / 32];              // a chunk's token renormalises some key row's gate product
 };
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: a tile copy takes microseconds
@@ -290,18 +291,27 @@ struct TokenCol {
 };
 
 // Per-slot constants of prefill token t for key row i (alpha_t = g_t alpha_{t-1}), written by
-// the D threads that are not finalising columns; their warps reduce q.k partials.
+// the D threads that are not finalising columns; their warps reduce q.k partials. A row whose
+// gate product falls below 2^-32 is renormalised: its Y is scaled by that product and alpha
+// restarts at 1 (ak.w holds the scale, 1 otherwise), so that no product over a chunk, however
+// long or steep its gates, leaves fp32 range or is floored.
 template <int D>
 __device__ __forceinline__ void token_constants(DecodeSmem<D>& sm, int he, int i, int t, const TokenRow<D>& in) {
     const int sl = sm.hslot[he][i] & 0xFF;
-    const float alpha = fmaxf(in.g * sm.ak[(t - 1) & 1][sl].z, 0x1p-64f);
+    const float raw = in.g * sm.ak[(t - 1) & 1][sl].z;
+    const bool renorm = raw < 0x1p-32f;
+    const float alpha = renorm ? 1.0f : raw;
     sm.kq[sl] = make_float4(alpha * in.k, alpha * in.k, alpha * in.q, alpha * in.q);
     const float ka = in.k * rcp_approx(alpha);
-    sm.ak[t & 1][sl] = make_float4(ka, ka, alpha, alpha);
+    sm.ak[t & 1][sl] = make_float4(ka, ka, alpha, renorm ? raw : 1.0f);
+    const bool any = __any_sync(0xffffffffu, renorm);
     float qk = in.q * in.k;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
-    if ((i & 31) == 0) sm.qkp[t & 1][i >> 5] = qk;
+    if ((i & 31) == 0) {
+        sm.qkp[t & 1][i >> 5] = qk;
+        sm.rn[t & 1][i >> 5] = any;
+    }
 }
 
 // The tile loop of the decode kernel. kPiv: the bit map may hold FP16 pivot rows (declared by
@@ -467,23 +477,45 @@ __device__ __forceinline__ void run_tiles(const DecodeArgs& a, DecodeSmem<D>& sm
         if constexpr (kChunk) {
             const int64_t T = a.num_tiles;
             for (int t = 1; t < a.chunk; ++t) {
-                {   // token t-1's rank-1 update fused with token t's k^T X and q^T X
+                bool rn = false;   // some row's gate product renormalised at token t (uniform)
+#pragma unroll
+                for (int w = 0; w < D / 32; ++w) rn |= sm.rn[t & 1][w] != 0;
+                {   // token t-1's rank-1 update fused with token t's k^T X and q^T X (and, where
+                    // token t renormalises a row's gate product, its scaling in between)
                     float2 ut[4], pacc[4], oacc[4];
                     load_cols8(sm.colb, cl, ut);
 #pragma unroll
                     for (int p = 0; p < 4; ++p) pacc[p] = oacc[p] = make_float2(0.f, 0.f);
+                    if (!rn) {
 #pragma unroll
-                    for (int r = 0; r < RPT; ++r) {
-                        const int sl = M::row(warp, lane, r);
-                        const float4 c = sm.ak[(t - 1) & 1][sl];
-                        const float4 kq = sm.kq[sl];
-                        const float2 ka = make_float2(c.x, c.y);
-                        const float2 kap = make_float2(kq.x, kq.y), lam = make_float2(kq.z, kq.w);
+                        for (int r = 0; r < RPT; ++r) {
+                            const int sl = M::row(warp, lane, r);
+                            const float4 c = sm.ak[(t - 1) & 1][sl];
+                            const float4 kq = sm.kq[sl];
+                            const float2 ka = make_float2(c.x, c.y);
+                            const float2 kap = make_float2(kq.x, kq.y), lam = make_float2(kq.z, kq.w);
 #pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-                            Z[r][p] = fma2(ka, ut[p], Z[r][p]);
-                            pacc[p] = fma2(kap, Z[r][p], pacc[p]);
-                            oacc[p] = fma2(lam, Z[r][p], oacc[p]);
+                            for (int p = 0; p < 4; ++p) {
+                                Z[r][p] = fma2(ka, ut[p], Z[r][p]);
+                                pacc[p] = fma2(kap, Z[r][p], pacc[p]);
+                                oacc[p] = fma2(lam, Z[r][p], oacc[p]);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < RPT; ++r) {
+                            const int sl = M::row(warp, lane, r);
+                            const float4 c = sm.ak[(t - 1) & 1][sl];
+                            const float4 kq = sm.kq[sl];
+                            const float sr = sm.ak[t & 1][sl].w;
+                            const float2 ka = make_float2(c.x, c.y), s2 = make_float2(sr, sr);
+                            const float2 kap = make_float2(kq.x, kq.y), lam = make_float2(kq.z, kq.w);
+#pragma unroll
+                            for (int p = 0; p < 4; ++p) {
+                                Z[r][p] = mul2(fma2(ka, ut[p], Z[r][p]), s2);
+                                pacc[p] = fma2(kap, Z[r][p], pacc[p]);
+                                oacc[p] = fma2(lam, Z[r][p], oacc[p]);
+                            }
                         }
                     }
                     store_col_partials<D>(sm.red[warp][0], lane, pacc);

@@ -175,10 +175,13 @@ def test_tensor_core_prefill_with_a_pivot_head():
     _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C)
 
 
-def test_tensor_core_prefill_with_steep_channel_gates():
+@pytest.mark.parametrize("form", ["wy", "seq"])
+def test_prefill_with_steep_channel_gates(form):
     """Channel gates down to 0.01, exact zeros (three in one channel within 16 tokens, a whole
     channel of zeros, and ones): gate products of a channel run far below fp32's range inside the
-    chunk, where a factorisation through one reference per 16-token block would overflow."""
+    chunk, where a factorisation through one reference per 16-token block would overflow (the
+    tensor-core form) and one running product per key row would be floored (the sequential
+    form, which renormalises a row's product below 2^-32)."""
     from recurrent_state_quantization_gated_b200 import api
     d, B, H, C = 128, 2, 3, 64
     wl, bits, w, packed, r, c = _setup(d, B, H, (4, 6, 8), True, seed=79)
@@ -190,7 +193,7 @@ def test_tensor_core_prefill_with_steep_channel_gates():
     g[:, 1, 2, 9] = 0.0
     g[:, 0, 0, 17] = 1.0
     toks["gate"] = g
-    res = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, "wy")
+    res = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, form)
     _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C)
 
 
