@@ -88,14 +88,15 @@ def _run(api, td, bits, w, head_off, bps, packed, r, c, form, in_place=True):
     return tuple(x.cpu().numpy() if x.dtype != torch.float16 else host_half(x) for x in res)
 
 
-def _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C):
+def _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C, form="wy"):
     p_r, r_r, c_r, o_r = oracle.prefill_chunk(toks, bits, w, packed, r, c)
     p_g, r_g, c_g, og = res
     for t in range(C):
         err = np.abs(og[t] - o_r[t]).max(axis=-1) / np.maximum(np.abs(o_r[t]).max(axis=-1), 1e-30)
         assert err.max() <= 1e-3, (t, err.max())
     return compare_decode((p_g, r_g, c_g, og[-1]), (p_r, r_r, c_r, o_r[-1]), bits, d, B,
-                          X_ref=oracle_chunk_state(toks, bits, packed, r, c), label=f"prefill chunk C={C} (tensor-core form)",
+                          X_ref=oracle_chunk_state(toks, bits, packed, r, c),
+                          label=f"prefill chunk C={C} ({'tensor-core' if form == 'wy' else 'sequential'} form)",
                           w=w)
 
 
@@ -194,7 +195,7 @@ def test_prefill_with_steep_channel_gates(form):
     g[:, 0, 0, 17] = 1.0
     toks["gate"] = g
     res = _run(api, _dev_tokens(toks), bits, w, head_off, bps, packed, r, c, form)
-    _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C)
+    _check_against_oracle(res, toks, bits, w, packed, r, c, d, B, C, form)
 
 
 def test_tensor_core_and_sequential_forms_agree_under_channel_gates():
