@@ -137,6 +137,10 @@ MUTANTS = [
         "double v = (double)orc_half_to_float(r[i]) * z[i * dv + j];")),
     _m("least-squares update skipped", C_SRC,
        ("c_out[j] = orc_scale_to_half(c1);", "c_out[j] = orc_scale_to_half((double)cfall[j]);")),
+    _m("zero-denominator column loses its start scale", C_SRC,
+       ("double c1 = den > 0.0 ? num / den : (double)cfall[j];", "double c1 = den > 0.0 ? num / den : 0.0;")),
+    _m("column fit ignores the given row scales", C_SRC,
+       ("for (int i = 0; i < dk; ++i) rf[i] = orc_half_to_float(r[i]);", "for (int i = 0; i < dk; ++i) rf[i] = 1.0f;")),
     # the persistent decode step (Table C2) and the prefill boundary (App. F.1)
     _m("decode refits the previous state", C_SRC,
        ("    for (int e = 0; e < dk * dv; ++e) S32[e] = (float)t.X[e];\n"
